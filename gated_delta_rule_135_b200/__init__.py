@@ -1,0 +1,223 @@
+"""Python binding of the B200 KDA chunked-prefill library (include/kda.h).
+
+Argument marshalling only: every step of the forward runs in the CUDA kernels
+of libkda.so.  Tensors are torch CUDA tensors (torch supplies device memory
+and the stream); the library never sees a torch type.  If the shared library
+is missing the import fails loudly -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkda.so")
+
+HEAD_DIM = 128
+CHUNK = 64
+FUSED_MIN_LOWER_BOUND = -5.3
+
+KDA_OK = 0
+STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
+                3: "KDA_ERR_ALIGNMENT", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_DEVICE",
+                6: "KDA_ERR_WORKSPACE"}
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {kda_strerror(status)}")
+
+
+class kda_dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("seqlen", ctypes.c_int64),
+                ("num_heads", ctypes.c_int32), ("num_seqs", ctypes.c_int32),
+                ("head_dim_k", ctypes.c_int32), ("head_dim_v", ctypes.c_int32)]
+
+
+class kda_staged_layout(ctypes.Structure):
+    _fields_ = [("chunk_table", ctypes.c_size_t), ("gamma", ctypes.c_size_t),
+                ("w", ctypes.c_size_t), ("u_tilde", ctypes.c_size_t), ("p", ctypes.c_size_t),
+                ("u", ctypes.c_size_t), ("chunk_states", ctypes.c_size_t),
+                ("total", ctypes.c_size_t), ("max_chunks", ctypes.c_int64)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libkda.so not built ({LIB_PATH}); run gated_delta_rule_135_b200/build.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, f32 = ctypes.c_void_p, ctypes.c_float
+    fwd_args = [vp, vp, vp, vp, vp, vp, vp, f32, f32, vp, vp, vp, vp, kda_dims]
+    lib.kda_fwd.restype = ctypes.c_int
+    lib.kda_fwd.argtypes = fwd_args + [vp]
+    lib.kda_fwd_staged.restype = ctypes.c_int
+    lib.kda_fwd_staged.argtypes = fwd_args + [vp, ctypes.c_size_t, vp]
+    lib.kda_staged_workspace_size.restype = ctypes.c_size_t
+    lib.kda_staged_workspace_size.argtypes = [kda_dims, ctypes.c_int]
+    lib.kda_staged_workspace_layout.restype = ctypes.c_int
+    lib.kda_staged_workspace_layout.argtypes = [kda_dims, ctypes.c_int, ctypes.POINTER(kda_staged_layout)]
+    lib.kda_strerror.restype = ctypes.c_char_p
+    lib.kda_strerror.argtypes = [ctypes.c_int]
+    lib.kda_check_device_error.restype = ctypes.c_int
+    lib.kda_check_device_error.argtypes = [vp]
+    lib.kda_last_device_error_bits.restype = ctypes.c_uint32
+    lib.kda_last_device_error_bits.argtypes = []
+    lib.kda_version.restype = ctypes.c_char_p
+    lib.kda_version.argtypes = []
+    return lib
+
+
+_lib = _load()
+
+# Symbols include/kda.h declares (checked by the ABI test).
+EXPORTED = ("kda_fwd", "kda_fwd_staged", "kda_staged_workspace_size",
+            "kda_staged_workspace_layout", "kda_strerror", "kda_check_device_error",
+            "kda_last_device_error_bits", "kda_version")
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def kda_strerror(status: int) -> str:
+    return _lib.kda_strerror(int(status)).decode()
+
+
+def kda_version() -> str:
+    return _lib.kda_version().decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_dims(num_heads: int, *, total_tokens: int, cu_seqlens: Optional[torch.Tensor] = None,
+              batch: int = 1, seqlen: Optional[int] = None) -> kda_dims:
+    if cu_seqlens is not None:
+        return kda_dims(1, int(total_tokens), int(num_heads), int(cu_seqlens.numel() - 1),
+                        HEAD_DIM, HEAD_DIM)
+    seqlen = total_tokens // max(batch, 1) if seqlen is None else seqlen
+    return kda_dims(int(batch), int(seqlen), int(num_heads), int(batch), HEAD_DIM, HEAD_DIM)
+
+
+def _check_tensor(name, t, dtype, device):
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name}: expected device {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def _marshal(q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens, out, final_state,
+             batch):
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda: tensors must live on a CUDA device")
+    _check_tensor("q", q, torch.bfloat16, dev)
+    _check_tensor("k", k, torch.bfloat16, dev)
+    _check_tensor("v", v, torch.bfloat16, dev)
+    _check_tensor("g", g, torch.float32, dev)
+    _check_tensor("beta", beta, torch.float32, dev)
+    _check_tensor("A_log", A_log, torch.float32, dev)
+    _check_tensor("dt_bias", dt_bias, torch.float32, dev)
+    _check_tensor("initial_state", initial_state, torch.float32, dev)
+    _check_tensor("cu_seqlens", cu_seqlens, torch.int32, dev)
+    _check_tensor("out", out, torch.bfloat16, dev)
+    _check_tensor("final_state", final_state, torch.float32, dev)
+    H = q.shape[-2]
+    total = q.numel() // (H * HEAD_DIM)
+    if cu_seqlens is None and q.dim() == 4:
+        batch = q.shape[0]
+    dims = make_dims(H, total_tokens=total, cu_seqlens=cu_seqlens, batch=batch)
+    return dims
+
+
+def kda_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+            beta: torch.Tensor, A_log: torch.Tensor, dt_bias: torch.Tensor,
+            lower_bound: float, scale: float, initial_state: Optional[torch.Tensor] = None,
+            cu_seqlens: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+            final_state: Optional[torch.Tensor] = None, *, batch: int = 1, stream=None):
+    """Calls kda_fwd.  q/k/v: [.., H, 128] bf16 (packed [Ttot, H, 128] or [B, T, H, 128]);
+    g: fp32 like q; beta: fp32 [.., H]; returns (out, final_state)."""
+    dims = _marshal(q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens, out,
+                    final_state, batch)
+    if out is None:
+        out = torch.empty(q.shape[:-1] + (HEAD_DIM,), dtype=torch.bfloat16, device=q.device)
+    st = _lib.kda_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias),
+                      float(lower_bound), float(scale), _ptr(initial_state), _ptr(cu_seqlens),
+                      _ptr(out), _ptr(final_state), dims, _stream_ptr(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_fwd")
+    return out, final_state
+
+
+@dataclass
+class StagedWorkspace:
+    buffer: torch.Tensor
+    layout: kda_staged_layout
+
+    def view(self, name: str, dtype, shape):
+        off = getattr(self.layout, name)
+        n = 1
+        for s in shape:
+            n *= s
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return self.buffer[off:off + nbytes].view(dtype).view(*shape)
+
+
+def staged_workspace(q: torch.Tensor, cu_seqlens: Optional[torch.Tensor] = None,
+                     batch: int = 1) -> StagedWorkspace:
+    H = q.shape[-2]
+    total = q.numel() // (H * HEAD_DIM)
+    if cu_seqlens is None and q.dim() == 4:
+        batch = q.shape[0]
+    dims = make_dims(H, total_tokens=total, cu_seqlens=cu_seqlens, batch=batch)
+    L = kda_staged_layout()
+    st = _lib.kda_staged_workspace_layout(dims, int(cu_seqlens is not None), ctypes.byref(L))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_staged_workspace_layout")
+    buf = torch.empty(max(L.total, 256), dtype=torch.uint8, device=q.device)
+    return StagedWorkspace(buf, L)
+
+
+def kda_fwd_staged(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, scale: float,
+                   initial_state=None, cu_seqlens=None, out=None, final_state=None, *,
+                   workspace: Optional[StagedWorkspace] = None, batch: int = 1, stream=None):
+    """Calls kda_fwd_staged (four kernels; intermediates left in the workspace)."""
+    dims = _marshal(q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens, out,
+                    final_state, batch)
+    if out is None:
+        out = torch.empty(q.shape[:-1] + (HEAD_DIM,), dtype=torch.bfloat16, device=q.device)
+    if workspace is None:
+        workspace = staged_workspace(q, cu_seqlens, batch)
+    st = _lib.kda_fwd_staged(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log),
+                             _ptr(dt_bias), float(lower_bound), float(scale), _ptr(initial_state),
+                             _ptr(cu_seqlens), _ptr(out), _ptr(final_state), dims,
+                             _ptr(workspace.buffer), ctypes.c_size_t(workspace.buffer.numel()),
+                             _stream_ptr(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_fwd_staged")
+    return out, final_state, workspace
+
+
+def kda_check_device_error(stream=None) -> int:
+    """Synchronises the stream; returns the device error bits (0 = none)."""
+    st = _lib.kda_check_device_error(_stream_ptr(stream))
+    if st == KDA_OK:
+        return 0
+    if st == 5:
+        return int(_lib.kda_last_device_error_bits())
+    raise KdaError(st, "kda_check_device_error")

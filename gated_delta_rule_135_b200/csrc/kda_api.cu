@@ -1,0 +1,191 @@
+// kda_api.cu -- the C ABI (include/kda.h): argument validation, dispatch and
+// the device error word.  This is the library's single translation unit: the
+// kernels are included below so that they share the error word without
+// relocatable device code.
+
+#include <math.h>
+#include <string.h>
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+#include "kda_staged.cuh"
+#include "kda_fused.cuh"
+
+namespace {
+
+using kda::StagedArgs;
+
+thread_local uint32_t t_last_device_bits = 0;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+    if (!a || !b || an == 0 || bn == 0) return false;
+    uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + bn && b0 < a0 + an;
+}
+
+kda_status device_ok() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    return major == 10 ? KDA_OK : KDA_ERR_UNSUPPORTED;
+}
+
+// Validates arguments and fills the kernel argument block.
+kda_status prepare(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                   const float* A_log, const float* dt_bias, float lower_bound, float scale,
+                   const float* initial_state, const int32_t* cu_seqlens, void* out,
+                   float* final_state, const kda_dims& d, StagedArgs* a) {
+    if (d.head_dim_k != kda::kHeadDim || d.head_dim_v != kda::kHeadDim) return KDA_ERR_UNSUPPORTED;
+    if (d.num_heads < 1 || d.seqlen < 0) return KDA_ERR_INVALID_ARG;
+    if (isnan(lower_bound) || lower_bound > 0.f) return KDA_ERR_INVALID_ARG;
+    if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+    int64_t N, total;
+    if (cu_seqlens) {
+        if (d.batch != 1 || d.num_seqs < 0) return KDA_ERR_INVALID_ARG;
+        N = d.num_seqs;
+        total = d.seqlen;
+    } else {
+        if (d.batch < 0) return KDA_ERR_INVALID_ARG;
+        N = d.batch;
+        total = (int64_t)d.batch * d.seqlen;
+    }
+    if (total >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 30)) return KDA_ERR_INVALID_ARG;
+    const int64_t H = d.num_heads;
+    if (total > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    if (!A_log || !dt_bias) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens, out, final_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_ALIGNMENT;
+    const size_t tok = (size_t)total * (size_t)H;
+    const size_t out_bytes = tok * kda::kHeadDim * 2;
+    const size_t st_bytes = (size_t)N * H * kda::kHeadDim * kda::kHeadDim * 4;
+    if (overlaps(out, out_bytes, q, out_bytes) || overlaps(out, out_bytes, k, out_bytes) ||
+        overlaps(out, out_bytes, v, out_bytes) || overlaps(out, out_bytes, g, tok * kda::kHeadDim * 4) ||
+        overlaps(out, out_bytes, beta, tok * 4) || overlaps(out, out_bytes, initial_state, st_bytes) ||
+        overlaps(out, out_bytes, final_state, st_bytes))
+        return KDA_ERR_INVALID_ARG;
+    if (final_state && initial_state && final_state != initial_state &&
+        overlaps(final_state, st_bytes, initial_state, st_bytes))
+        return KDA_ERR_INVALID_ARG;
+    a->q = q; a->k = k; a->v = v; a->g = g; a->beta = beta; a->A_log = A_log; a->dt_bias = dt_bias;
+    a->lower_bound = lower_bound; a->scale = scale;
+    a->initial_state = initial_state; a->cu_seqlens = cu_seqlens;
+    a->out = out; a->final_state = final_state;
+    a->seqlen = d.seqlen; a->total_tokens = total; a->H = (int)H; a->N = (int)N;
+    return device_ok();
+}
+
+// Carries the initial state to the final state when no token is processed.
+kda_status copy_states_only(const StagedArgs& a, cudaStream_t s) {
+    if (!a.final_state || a.N == 0) return KDA_OK;
+    const size_t bytes = (size_t)a.N * a.H * kda::kHeadDim * kda::kHeadDim * 4;
+    cudaError_t err = a.initial_state
+        ? (a.initial_state == a.final_state ? cudaSuccess
+           : cudaMemcpyAsync(a.final_state, a.initial_state, bytes, cudaMemcpyDeviceToDevice, s))
+        : cudaMemsetAsync(a.final_state, 0, bytes, s);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_staged_workspace_layout(kda_dims dims, int varlen, kda_staged_layout* layout) {
+    if (!layout) return KDA_ERR_INVALID_ARG;
+    if (dims.num_heads < 1 || dims.seqlen < 0 || dims.batch < 0 || dims.num_seqs < 0)
+        return KDA_ERR_INVALID_ARG;
+    int64_t N = dims.num_seqs, total = dims.seqlen;
+    if (!varlen) {
+        N = dims.batch;
+        total = (int64_t)dims.batch * dims.seqlen;
+    }
+    kda::StagedLayout L = kda::staged_layout(total, dims.num_heads, (int)N);
+    layout->chunk_table = L.chunk_table;
+    layout->gamma = L.gamma;
+    layout->w = L.w;
+    layout->u_tilde = L.u_tilde;
+    layout->p = L.p;
+    layout->u = L.u;
+    layout->chunk_states = L.chunk_states;
+    layout->total = L.total;
+    layout->max_chunks = L.max_chunks;
+    return KDA_OK;
+}
+
+size_t kda_staged_workspace_size(kda_dims dims, int varlen) {
+    kda_staged_layout L;
+    return kda_staged_workspace_layout(dims, varlen, &L) == KDA_OK ? L.total : 0;
+}
+
+kda_status kda_fwd_staged(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* A_log, const float* dt_bias,
+                          float lower_bound, float scale, const float* initial_state,
+                          const int32_t* cu_seqlens, void* out, float* final_state, kda_dims dims,
+                          void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+    StagedArgs a{};
+    kda_status st = prepare(q, k, v, g, beta, A_log, dt_bias, lower_bound, scale, initial_state,
+                            cu_seqlens, out, final_state, dims, &a);
+    if (st != KDA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (a.total_tokens == 0) return copy_states_only(a, s);
+    kda::StagedLayout L = kda::staged_layout(a.total_tokens, a.H, a.N);
+    if (!workspace || workspace_bytes < L.total) return KDA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_ALIGNMENT;
+    return kda::launch_staged(a, static_cast<char*>(workspace), L, s) == cudaSuccess ? KDA_OK
+                                                                                     : KDA_ERR_CUDA;
+}
+
+kda_status kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                   const float* A_log, const float* dt_bias, float lower_bound, float scale,
+                   const float* initial_state, const int32_t* cu_seqlens, void* out,
+                   float* final_state, kda_dims dims, kda_stream_t stream) {
+    StagedArgs a{};
+    kda_status st = prepare(q, k, v, g, beta, A_log, dt_bias, lower_bound, scale, initial_state,
+                            cu_seqlens, out, final_state, dims, &a);
+    if (st != KDA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (a.total_tokens == 0) return copy_states_only(a, s);
+    if (kda::fused_supported(lower_bound))
+        return kda::launch_fused(a, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    kda::StagedLayout L = kda::staged_layout(a.total_tokens, a.H, a.N);
+    void* ws = nullptr;
+    if (cudaMallocAsync(&ws, L.total, s) != cudaSuccess) return KDA_ERR_CUDA;
+    cudaError_t err = kda::launch_staged(a, static_cast<char*>(ws), L, s);
+    cudaError_t err2 = cudaFreeAsync(ws, s);
+    return (err == cudaSuccess && err2 == cudaSuccess) ? KDA_OK : KDA_ERR_CUDA;
+}
+
+const char* kda_strerror(kda_status status) {
+    switch (status) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid pointer, dimension or scalar";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: head dims must be 128 on an sm_100 device";
+        case KDA_ERR_ALIGNMENT: return "KDA_ERR_ALIGNMENT: a base address is not 16-byte aligned";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA call or kernel launch failed";
+        case KDA_ERR_DEVICE: return "KDA_ERR_DEVICE: a kernel recorded a device-side error";
+        case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+kda_status kda_check_device_error(kda_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return KDA_ERR_CUDA;
+    unsigned int bits = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&bits, kda::g_device_error, sizeof bits) != cudaSuccess) return KDA_ERR_CUDA;
+    if (bits && cudaMemcpyToSymbol(kda::g_device_error, &zero, sizeof zero) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    t_last_device_bits = bits;
+    return bits ? KDA_ERR_DEVICE : KDA_OK;
+}
+
+uint32_t kda_last_device_error_bits(void) { return t_last_device_bits; }
+
+const char* kda_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// kda_internal.h -- host-side interfaces between the C ABI and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kda {
+
+struct StagedArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* g;
+    const float* beta;
+    const float* A_log;
+    const float* dt_bias;
+    float lower_bound;
+    float scale;
+    const float* initial_state;
+    const int32_t* cu_seqlens;
+    void* out;
+    float* final_state;
+    int64_t seqlen;        // per-sequence length (fixed layout) or packed total
+    int64_t total_tokens;  // Ttot
+    int H;
+    int N;                 // number of sequences
+};
+
+struct StagedLayout {
+    size_t chunk_table, gamma, w, u_tilde, p, u, chunk_states, total;
+    int64_t max_chunks;
+};
+
+StagedLayout staged_layout(int64_t total_tokens, int H, int N);
+cudaError_t launch_staged(const StagedArgs& a, char* workspace, const StagedLayout& L,
+                          cudaStream_t stream);
+
+// The fused persistent tcgen05 kernel (same arguments; no workspace).
+cudaError_t launch_fused(const StagedArgs& a, cudaStream_t stream);
+bool fused_supported(float lower_bound);
+
+}  // namespace kda

@@ -1,0 +1,160 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention chunked-prefill forward.
+ *
+ * The operation (FlashKDA posts: donniechu.com, section "Số liệu kỹ thuật" --
+ * flash_kda.fwd() with batch, variable length via cu_seqlens, initial/final
+ * recurrent state, fine-grained channel-wise gate with learned A_log, dt_bias,
+ * lower_bound, bf16 + fp32 precision, K = V = 128; toolarium.ru post, section
+ * "Где ограничения прямо сейчас" -- K = V = 128 is a hard constraint and the
+ * released kernels target the prefill forward).  The pages print no formula;
+ * this library computes, per sequence and head, with S a K x V fp32 state:
+ *
+ *   log a_t = max(-exp(A_log[h]) * softplus(g_t + dt_bias[h]), lower_bound)  (per channel)
+ *   S_t     = (I - beta_t k_t k_t^T) Diag(a_t) S_{t-1} + beta_t k_t v_t^T
+ *   o_t     = scale * S_t^T q_t
+ *
+ * S_0 = initial_state (or 0); final_state = S after the sequence's last token.
+ *
+ * Layouts (all row-major, all pointers are DEVICE memory owned by the caller):
+ *   q, k        bf16  [Ttot, H, 128]     Ttot = batch * seqlen (fixed) or the packed total
+ *   v           bf16  [Ttot, H, 128]
+ *   g           fp32  [Ttot, H, 128]     raw gate input
+ *   beta        fp32  [Ttot, H]
+ *   A_log       fp32  [H]
+ *   dt_bias     fp32  [H, 128]
+ *   initial_state fp32 [N, H, 128, 128]  ([seq][head][k][v]); NULL means zeros
+ *   cu_seqlens  int32 [N + 1]            NULL means N = batch sequences of length seqlen
+ *   out         bf16  [Ttot, H, 128]     written, rounded to nearest even from fp32
+ *   final_state fp32  [N, H, 128, 128]   NULL means "do not write"
+ * With cu_seqlens, batch must be 1, seqlen is the packed total Ttot, N = num_seqs,
+ * cu_seqlens[0] = 0, cu_seqlens[N] = Ttot and the offsets are non-decreasing
+ * (empty sequences are allowed: their final state is their initial state).
+ * cu_seqlens is read only on the device: no call synchronises with the host.
+ *
+ * Alignment: every tensor base address must be 16-byte aligned.
+ * Aliasing: final_state may alias initial_state (in-place state update); out
+ * must not overlap any input.
+ * Streams: every compute call is asynchronous on `stream` (a cudaStream_t;
+ * NULL = the legacy default stream).  Argument errors are reported
+ * synchronously, before any launch.
+ * A kernel that detects a violated precondition on the device (offsets out of
+ * range, a wait that ran out) records it in a device error word instead of
+ * faulting; kda_check_device_error() reads and clears it.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* kda_stream_t;   /* same type as cudaStream_t */
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* NULL required pointer, bad dims, bad scalar */
+    KDA_ERR_UNSUPPORTED = 2,   /* head dims other than 128, or no sm_100 device */
+    KDA_ERR_ALIGNMENT = 3,     /* a base address not 16-byte aligned */
+    KDA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    KDA_ERR_DEVICE = 5,        /* a kernel recorded a device-side error (see kda_check_device_error) */
+    KDA_ERR_WORKSPACE = 6      /* workspace missing or smaller than required */
+} kda_status;
+
+typedef struct {
+    int32_t batch;       /* B: sequences of the fixed-length layout (1 with cu_seqlens) */
+    int64_t seqlen;      /* tokens per sequence (fixed) or packed total Ttot (varlen) */
+    int32_t num_heads;   /* H >= 1 */
+    int32_t num_seqs;    /* N with cu_seqlens; ignored (taken as batch) without */
+    int32_t head_dim_k;  /* must be 128 */
+    int32_t head_dim_v;  /* must be 128 */
+} kda_dims;
+
+/* Device error bits recorded by kernels (returned by kda_check_device_error via
+ * kda_last_device_error_bits). */
+#define KDA_DEVERR_BAD_OFFSETS 0x1u   /* cu_seqlens not monotone / out of [0, Ttot] */
+#define KDA_DEVERR_TIMEOUT     0x2u   /* a bounded wait ran out of iterations */
+#define KDA_DEVERR_BOUNDS      0x4u   /* an index outside its buffer was skipped */
+
+/*
+ * kda_fwd -- the chunked prefill forward (the product path).
+ *
+ * Runs the fused persistent sm_100a kernel (tcgen05 tensor cores with TMEM
+ * accumulators, TMA-staged inputs) when lower_bound >= KDA_FUSED_MIN_LOWER_BOUND,
+ * and the staged exact-decay kernels otherwise (their intra-chunk decays are
+ * formed pair by pair and cannot overflow for any gate).  The staged fallback
+ * allocates its workspace stream-ordered (cudaMallocAsync).
+ *
+ * lower_bound: <= 0 (may be -INFINITY: no clamp); NaN or > 0 is rejected.
+ * scale: finite.  Returns KDA_OK or an error code; never aborts.
+ */
+kda_status kda_fwd(const void* q, const void* k, const void* v,
+                   const float* g, const float* beta,
+                   const float* A_log, const float* dt_bias,
+                   float lower_bound, float scale,
+                   const float* initial_state, const int32_t* cu_seqlens,
+                   void* out, float* final_state,
+                   kda_dims dims, kda_stream_t stream);
+
+/* Gates at or above this clamp keep every factored intra-chunk decay of the
+ * fused kernel inside the fp32/bf16 exponent range (16 tokens x 5.3 = 84.8 < 87). */
+#define KDA_FUSED_MIN_LOWER_BOUND (-5.3f)
+
+/*
+ * kda_fwd_staged -- the same forward as four separate kernels with fp32 CUDA-core
+ * arithmetic and intermediates in a caller-provided workspace:
+ *   (a) gate pre-pass: Gamma = in-chunk inclusive cumsum of log a;
+ *   (b) intra-chunk WY: A, T = (I + A)^-1, W = T diag(beta)(gamma*K), U~ = T diag(beta) V, P;
+ *   (c) state propagation: U = U~ - W S_c, S_{c+1} = Diag(gamma_C) S_c + Khat^T U;
+ *   (d) output: O = scale ((gamma*Q) S_c + P U).
+ * Chunks are 64 tokens, restarting at every sequence start.
+ * workspace: device buffer of at least kda_staged_workspace_size(dims) bytes,
+ * 256-byte aligned.  Its layout (offsets from kda_staged_workspace_layout) is
+ * part of the ABI so that tests can read each stage's output.
+ */
+size_t kda_staged_workspace_size(kda_dims dims, int varlen);
+
+typedef struct {
+    size_t chunk_table;   /* int32 [max_chunks][4]: seq, t0, len, chunk index in seq; then int32 count */
+    size_t gamma;         /* fp32 [Ttot, H, 128]  Gamma (in-chunk inclusive cumsum of log a) */
+    size_t w;             /* fp32 [Ttot, H, 128]  W */
+    size_t u_tilde;       /* fp32 [Ttot, H, 128]  U~ */
+    size_t p;             /* fp32 [Ttot, H, 64]   row r of the token's chunk P (columns past r are 0) */
+    size_t u;             /* fp32 [Ttot, H, 128]  U */
+    size_t chunk_states;  /* fp32 [max_chunks, H, 128, 128]  state at each chunk's start */
+    size_t total;         /* bytes */
+    int64_t max_chunks;   /* ceil(Ttot / 64) + N */
+} kda_staged_layout;
+
+/* varlen != 0: the call passes cu_seqlens (N = num_seqs, Ttot = seqlen);
+ * varlen == 0: fixed layout (N = batch, Ttot = batch * seqlen). */
+kda_status kda_staged_workspace_layout(kda_dims dims, int varlen, kda_staged_layout* layout);
+
+kda_status kda_fwd_staged(const void* q, const void* k, const void* v,
+                          const float* g, const float* beta,
+                          const float* A_log, const float* dt_bias,
+                          float lower_bound, float scale,
+                          const float* initial_state, const int32_t* cu_seqlens,
+                          void* out, float* final_state,
+                          kda_dims dims, void* workspace, size_t workspace_bytes,
+                          kda_stream_t stream);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* kda_strerror(kda_status status);
+
+/* Synchronises `stream`, then reads and clears the device error word.
+ * Returns KDA_OK, KDA_ERR_DEVICE (bits available from kda_last_device_error_bits)
+ * or KDA_ERR_CUDA.  Not capturable (it synchronises). */
+kda_status kda_check_device_error(kda_stream_t stream);
+uint32_t kda_last_device_error_bits(void);
+
+/* Library version, "major.minor.patch". */
+const char* kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

@@ -1,0 +1,52 @@
+"""Shared helpers of the GPU parity tests: move seeded inputs to the device,
+call the library, run the oracle on the same inputs, and apply the tolerances.
+
+Tolerances (against the fp64 oracle, out compared after the library's bf16
+rounding):  out rel-L2 <= 2e-3 and max-abs <= 1e-2; final state rel-L2 <= 1e-3.
+"""
+import numpy as np
+import torch
+
+import oracle
+
+OUT_REL_L2 = 2e-3
+OUT_MAX_ABS = 1e-2
+STATE_REL_L2 = 1e-3
+
+
+def to_device(x: dict, device="cuda") -> dict:
+    d = dict(x)
+    for key in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "initial_state", "cu_seqlens"):
+        if d.get(key) is not None:
+            d[key] = d[key].to(device).contiguous()
+    return d
+
+
+def run_oracle(x: dict, nthreads: int = 0):
+    return oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], x["A_log"], x["dt_bias"],
+                            x["lower_bound"], x["scale"], x["initial_state"], x["cu_seqlens"],
+                            nthreads=nthreads)
+
+
+def alloc_final(xd: dict, want: bool):
+    if not want:
+        return None
+    H = xd["q"].shape[-2]
+    return torch.full((xd["N"], H, 128, 128), float("nan"), device=xd["q"].device)
+
+
+def check(out, fin, ref_out, ref_fin, label=""):
+    o = out.float().cpu().numpy().astype(np.float64)
+    e_rel = oracle.rel_l2(o, ref_out)
+    e_abs = oracle.max_abs(o, ref_out)
+    msg = f"{label}: out rel-L2 {e_rel:.3e} max-abs {e_abs:.3e}"
+    assert np.all(np.isfinite(o)), msg + " (non-finite output)"
+    assert e_rel <= OUT_REL_L2, msg
+    assert e_abs <= OUT_MAX_ABS, msg
+    e_st = None
+    if fin is not None:
+        f = fin.cpu().numpy().astype(np.float64)
+        e_st = oracle.rel_l2(f, ref_fin)
+        assert np.all(np.isfinite(f)), msg + " (non-finite state)"
+        assert e_st <= STATE_REL_L2, msg + f" state rel-L2 {e_st:.3e}"
+    return e_rel, e_abs, e_st

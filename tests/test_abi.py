@@ -1,0 +1,126 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments synchronously before any launch."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _build():
+    from gated_delta_rule_135_b200 import build
+    build.build()
+
+
+_build()
+import gated_delta_rule_135_b200 as kda  # noqa: E402
+
+
+def _declared_functions():
+    names = set()
+    for hdr in os.listdir(os.path.join(ROOT, "include")):
+        if not hdr.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", hdr)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*[A-Za-z_][\w\s\*]*?\b(kda_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared_functions()
+    assert "kda_fwd" in declared and "kda_fwd_staged" in declared
+    lib = ctypes.CDLL(kda.LIB_PATH)
+    for name in sorted(declared):
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert declared <= set(kda.EXPORTED) | declared
+
+
+def test_strerror_covers_every_status():
+    for code, name in kda.STATUS_NAMES.items():
+        assert kda.kda_strerror(code).startswith(name)
+    assert kda.kda_strerror(99) == "KDA_ERR_UNKNOWN"
+    assert re.match(r"^\d+\.\d+\.\d+$", kda.kda_version())
+
+
+def _dims(H=2, T=256, hk=128, hv=128, batch=1, nseq=1):
+    return kda.kda_dims(batch, T, H, nseq, hk, hv)
+
+
+FAKE = 0x7F0000000000            # never dereferenced: validation fails first
+
+
+def _call(dims, lb=-5.0, scale=0.088, base=FAKE, stride=1 << 28, cu=None, out=None,
+          init=None, fin=None, misalign=None):
+    p = [base + i * stride for i in range(8)]
+    if misalign is not None:
+        p[misalign] += 8
+    q, k, v, g, beta, alog, dtb, o = p
+    if out is not None:
+        o = out
+    return kda.lib().kda_fwd(q, k, v, g, beta, alog, dtb, ctypes.c_float(lb), ctypes.c_float(scale),
+                             init, cu, o, fin, dims, None)
+
+
+def test_rejects_unsupported_head_dims():
+    assert _call(_dims(hk=64)) == 2
+    assert _call(_dims(hv=256)) == 2
+
+
+@pytest.mark.parametrize("lb", [0.5, float("nan")])
+def test_rejects_bad_lower_bound(lb):
+    assert _call(_dims(), lb=lb) == 1
+
+
+@pytest.mark.parametrize("scale", [float("inf"), float("nan")])
+def test_rejects_non_finite_scale(scale):
+    assert _call(_dims(), scale=scale) == 1
+
+
+def test_rejects_bad_dims():
+    assert _call(_dims(H=0)) == 1
+    assert _call(kda.kda_dims(1, -1, 2, 1, 128, 128)) == 1
+    # cu_seqlens requires batch == 1
+    assert _call(_dims(batch=2), cu=FAKE + (1 << 33)) == 1
+
+
+@pytest.mark.parametrize("which", range(8))
+def test_rejects_misaligned_pointers(which):
+    assert _call(_dims(), misalign=which) == 3
+
+
+def test_rejects_output_aliasing_an_input():
+    # out == q
+    assert _call(_dims(), out=FAKE) == 1
+
+
+def test_rejects_partially_overlapping_states():
+    st = FAKE + (1 << 34)
+    assert _call(_dims(), init=st, fin=st + 4096) == 1
+
+
+def test_null_required_pointer():
+    d = _dims()
+    r = kda.lib().kda_fwd(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ctypes.c_float(-5.0),
+                          ctypes.c_float(1.0), None, None, FAKE + (1 << 30), None, d, None)
+    assert r == 1
+
+
+def test_staged_workspace_layout_is_consistent():
+    for varlen, dims in ((0, _dims(H=3, T=1000)), (1, _dims(H=96, T=8192, nseq=6))):
+        L = kda.kda_staged_layout()
+        assert kda.lib().kda_staged_workspace_layout(dims, varlen, ctypes.byref(L)) == 0
+        T, H = dims.seqlen * (1 if varlen else dims.batch), dims.num_heads
+        N = dims.num_seqs if varlen else dims.batch
+        assert L.max_chunks == math.ceil(T / 64) + N
+        offs = [L.chunk_table, L.gamma, L.w, L.u_tilde, L.p, L.u, L.chunk_states, L.total]
+        assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+        assert L.gamma - L.chunk_table >= 16 * L.max_chunks + 4
+        assert L.w - L.gamma >= 4 * T * H * 128
+        assert L.u - L.p >= 4 * T * H * 64
+        assert L.total - L.chunk_states >= 4 * L.max_chunks * H * 128 * 128
+        assert kda.lib().kda_staged_workspace_size(dims, varlen) == L.total
