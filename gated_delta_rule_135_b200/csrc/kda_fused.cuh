@@ -1,11 +1,773 @@
-// kda_fused.cuh -- the fused persistent sm_100a kernel (placeholder until it lands).
+// kda_fused.cuh -- the fused persistent sm_100a KDA chunked-prefill kernel.
+//
+// One CTA per SM walks a static "snake" schedule of (sequence, head) units,
+// longest sequences first, and carries each unit's 128 x 128 fp32 state in
+// TMEM across its 64-token chunks.  Per chunk (all on chip; only q, k, v, g,
+// beta, the states and out touch HBM):
+//
+//  1  gate + operand formation (CUDA cores): log a, in-chunk cumsum Gamma per
+//     16-token block, and the decayed MMA operands written to swizzled smem;
+//     the next chunk's TMA loads are issued as soon as the inputs are read.
+//  2  one M=128 x N=160 x K=128 bf16 MMA gives every block of the decayed
+//     K K^T (rows 0-63) and Q K^T (rows 64-127): the column operand holds the
+//     diagonal blocks (reference point = start of the row's block, factor
+//     e^{Gamma_s - Gamma_i} >= 1, bounded by e^{16 |lower_bound|}) and the
+//     three "block distance" variants d = 1..3 (factors <= 1).
+//  3  TMEM -> A (x beta_r) in fp32 and P in fp16; P's main diagonal q_r . k_r
+//     (no decay, the dominant output term) is taken exactly in fp32.
+//  4  T = (I + A)^-1 by blocked forward substitution in fp32 -> fp16.
+//  5  W = T (beta gamma K) (M=64) and U~^T = (beta V)^T T^T (M=128), fp16 MMAs.
+//  6  W -> fp16 smem.
+//  7  S (TMEM, fp32) -> fp16 smem copy; S <- Diag(gamma_last) S in TMEM;
+//     U^T = U~^T - S^T W^T and O^T = S^T (gamma Q)^T on the tensor cores.
+//  8  U^T -> fp16 smem; S += Khat^T U and O^T += U^T P^T.
+//  9  O^T -> bf16 out.
+//
+// Operand precision (chosen by emulating the chunk algebra against the fp64
+// oracle): intra-chunk decay blocks in bf16 (fp32 exponent range), everything
+// that multiplies T, S, U or P in fp16 (11-bit significand), accumulation and
+// the carried state in fp32.
+//
+// Exponent range: the diagonal-block factor e^{Gamma_s - Gamma_i} spans up to
+// 16 tokens of decay, so the kernel requires lower_bound >= -5.3 (16 x 5.3 =
+// 84.8 < 87, inside fp32 / bf16 range); steeper gates take the staged path.
 #pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "kda_common.cuh"
 #include "kda_internal.h"
+#include "umma.cuh"
 
 namespace kda {
+namespace fused {
 
-bool fused_supported(float) { return false; }
+using namespace umma;
 
-cudaError_t launch_fused(const StagedArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+constexpr int kThreads = 256;
+
+// ---- shared memory map (bytes from a 1024-aligned base) ----
+constexpr uint32_t IN_Q = 0;          // bf16 [64][128] row-major (TMA box)
+constexpr uint32_t IN_K = 16384;
+constexpr uint32_t IN_V = 32768;
+constexpr uint32_t IN_G = 49152;      // fp32 [64][128]
+constexpr uint32_t IN_BYTES = 81920;
+constexpr uint32_t X = 81920;         // phase-shared region, 73728 bytes
+constexpr uint32_t AP_A = X + 0;      // bf16 K-major [128 rows][128]: k*R rows 0-63, q*R rows 64-127
+constexpr uint32_t AP_B = X + 32768;  // bf16 K-major [160 rows][128]: XD | C1 | C2 | C3
+constexpr uint32_t A32 = X + 0;       // fp32 [64][65]      (phases 3-4)
+constexpr uint32_t T32 = X + 16640;   // fp32 [64][65]      (phase 4)
+constexpr uint32_t T16 = X + 33792;   // fp16 K-major [64][64]        (phases 4-5)
+constexpr uint32_t MSCR = X + 41984;  // fp32 [16][48] solve scratch  (phase 4)
+constexpr uint32_t W16 = X + 0;       // fp16 K-major [64 r][128 c]   (phases 6-7)
+constexpr uint32_t S16 = X + 16384;   // fp16 [128 c][128 v] (MN-major A)  (phase 7)
+constexpr uint32_t P16 = X + 65536;   // fp16 K-major [64 r][64 i]    (phases 3-8)
+constexpr uint32_t BGK = X + 73728;   // fp16 [64 i][128 c] beta*gamma*k  (MN-major B of W)
+constexpr uint32_t U16 = BGK;         // fp16 K-major [128 v][64 r]   (phase 8; BGK is dead)
+constexpr uint32_t BV = BGK + 16384;  // fp16 [64 i][128 v] beta*v    (MN-major A of U~^T)
+constexpr uint32_t GQ = BV + 16384;   // fp16 K-major [64 r][128 c] gamma*q
+constexpr uint32_t KH = GQ + 16384;   // fp16 [64 i][128 c] Khat     (MN-major A of S update)
+constexpr uint32_t MISC = KH + 16384;
+constexpr uint32_t S_BETA = MISC;              // fp32 [64]
+constexpr uint32_t S_GAMMAC = S_BETA + 256;    // fp32 [128] e^{Gamma_last}
+constexpr uint32_t S_TOT = S_GAMMAC + 512;     // fp32 [4][128] per-block sums of log a
+constexpr uint32_t S_PDIAG = S_TOT + 2048;     // fp32 [2][64] halves of q_r . k_r
+constexpr uint32_t S_ORDER = S_PDIAG + 512;    // int16 [kSortLimit] sequences by length
+constexpr int kSortLimit = 512;
+constexpr uint32_t S_BARS = S_ORDER + 2 * kSortLimit;   // u64 [2]: inputs, mma
+constexpr uint32_t S_TMEM = S_BARS + 16;                // u32 tmem base, u32 abort flag
+constexpr uint32_t SMEM_BYTES = S_TMEM + 16;
+constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;      // + alignment slack
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+
+// ---- TMEM columns ----
+constexpr uint32_t TM_AP = 0;     // [128 lanes][160]  decayed K K^T | Q K^T
+constexpr uint32_t TM_W = 0;      // M=64 [64][128]    (after TM_AP is consumed)
+constexpr uint32_t TM_UT = 160;   // [128 v][64 r]     U~^T then U^T
+constexpr uint32_t TM_OT = 224;   // [128 v][64 r]     O^T
+constexpr uint32_t TM_S = 384;    // [128 c][128 v]    the state
+constexpr uint32_t TM_COLS = 512;
+
+constexpr uint32_t IDESC_AP = idesc_f16(128, 160, true, false, false);
+constexpr uint32_t IDESC_W = idesc_f16(64, 128, false, false, true);
+constexpr uint32_t IDESC_UT = idesc_f16(128, 64, false, true, false);
+constexpr uint32_t IDESC_U = idesc_f16(128, 64, false, true, false, true);   // negated B
+constexpr uint32_t IDESC_O1 = idesc_f16(128, 64, false, true, false);
+constexpr uint32_t IDESC_S = idesc_f16(128, 128, false, true, false);
+constexpr uint32_t IDESC_O2 = idesc_f16(128, 64, false, false, false);
+
+struct Params {
+    const float* beta;
+    const float* A_log;
+    const float* dt_bias;
+    float lower_bound;
+    float scale;
+    const float* initial_state;
+    const int32_t* cu_seqlens;
+    __nv_bfloat16* out;
+    float* final_state;
+    int64_t seqlen;
+    int64_t total_tokens;
+    int H;
+    int N;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ uint32_t pack_f16(float a, float b) {
+    __half2 v = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ void st_u32(unsigned char* base, uint32_t off, uint32_t v) {
+    *reinterpret_cast<uint32_t*>(base + off) = v;
+}
+__device__ __forceinline__ void st_v4(unsigned char* base, uint32_t off, uint32_t a, uint32_t b,
+                                      uint32_t c, uint32_t d) {
+    *reinterpret_cast<uint4*>(base + off) = make_uint4(a, b, c, d);
+}
+
+// Schedule: unit u = rank * H + head, rank = position of the sequence when
+// sorted by length (longest first, ties by index) if N <= kSortLimit.
+struct Unit {
+    int n, h;
+    int64_t bos, eos;
+};
+
+__device__ __forceinline__ int unit_of(int k, int b, int G) {
+    return (k & 1) ? (k + 1) * G - 1 - b : k * G + b;
+}
+
+__device__ __forceinline__ Unit decode_unit(const Params& p, const int16_t* order, int u) {
+    Unit x;
+    const int rank = u / p.H;
+    x.h = u - rank * p.H;
+    x.n = (p.N <= kSortLimit) ? order[rank] : rank;
+    seq_range(p.cu_seqlens, x.n, p.seqlen, p.total_tokens, &x.bos, &x.eos);
+    return x;
+}
+
+// Issues the four TMA loads of one chunk onto the input barrier (one thread).
+__device__ __forceinline__ void issue_chunk_loads(unsigned char* sm, uint64_t* bar,
+                                                  const CUtensorMap* tq, const CUtensorMap* tk,
+                                                  const CUtensorMap* tv, const CUtensorMap* tg,
+                                                  int h, int64_t t0) {
+    mbar_arrive_expect_tx(bar, IN_BYTES);
+    const int x = h * kHeadDim, y = (int)t0;
+    tma_load_2d(sm + IN_Q, tq, x, y, bar);
+    tma_load_2d(sm + IN_K, tk, x, y, bar);
+    tma_load_2d(sm + IN_V, tv, x, y, bar);
+    tma_load_2d(sm + IN_G, tg, x, y, bar);
+}
+
+// Finds the chunk after (k, j) on this CTA's schedule: next chunk of the same
+// unit or chunk 0 of the next non-empty unit.  Returns false if none.
+__device__ bool next_chunk(const Params& p, const int16_t* order, int b, int G, int units, int k,
+                           int64_t j, int64_t nch, int* k_out, int* h_out, int64_t* t0_out) {
+    if (j + 1 < nch) {
+        const Unit x = decode_unit(p, order, unit_of(k, b, G));
+        *k_out = k;
+        *h_out = x.h;
+        *t0_out = x.bos + (j + 1) * kChunk;
+        return true;
+    }
+    for (int kk = k + 1; (int64_t)kk * G < units; ++kk) {
+        const int u = unit_of(kk, b, G);
+        if (u >= units) continue;
+        const Unit x = decode_unit(p, order, u);
+        if (x.eos > x.bos) {
+            *k_out = kk;
+            *h_out = x.h;
+            *t0_out = x.bos;
+            return true;
+        }
+    }
+    return false;
+}
+
+// Waits (bounded) for an mbarrier phase; on expiry records the timeout and
+// raises the CTA-wide abort flag.  Returns true when the CTA should stop.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag) {
+    if (!mbar_wait_bounded(bar, parity)) {
+        record_error(KDA_DEVERR_TIMEOUT);
+        *abort_flag = 1u;
+    }
+    __syncthreads();
+    return *abort_flag != 0u;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                 const Params p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int G = gridDim.x, b = blockIdx.x;
+    const int H = p.H;
+    const int units = p.N * H;
+
+    float* sBeta = reinterpret_cast<float*>(sm + S_BETA);
+    float* sGammaC = reinterpret_cast<float*>(sm + S_GAMMAC);
+    float* sTot = reinterpret_cast<float*>(sm + S_TOT);
+    float* sPdiag = reinterpret_cast<float*>(sm + S_PDIAG);
+    int16_t* sOrder = reinterpret_cast<int16_t*>(sm + S_ORDER);
+    uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + S_BARS);
+    uint64_t* bar_mma = bar_in + 1;
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + S_TMEM);
+    volatile uint32_t* sAbort = sTmem + 1;
+
+    // ---- set-up: barriers, TMEM, length order ----
+    if (tid == 0) {
+        mbar_init(bar_in, 1);
+        mbar_init(bar_mma, 1);
+        mbar_init_fence();
+        *sAbort = 0u;
+    }
+    if (warp == 0) {
+        tmem_alloc(sTmem, TM_COLS);
+        tmem_relinquish();
+    }
+    if (p.N <= kSortLimit) {
+        for (int n = tid; n < p.N; n += kThreads) {
+            int64_t bn, en;
+            seq_range(p.cu_seqlens, n, p.seqlen, p.total_tokens, &bn, &en);
+            const int64_t ln = en - bn;
+            int rank = 0;
+            for (int m = 0; m < p.N; ++m) {
+                int64_t bm, em;
+                seq_range(p.cu_seqlens, m, p.seqlen, p.total_tokens, &bm, &em);
+                const int64_t lm = em - bm;
+                rank += (lm > ln) || (lm == ln && m < n);
+            }
+            sOrder[rank] = (int16_t)n;
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *sTmem;
+
+    uint32_t in_parity = 0, mma_parity = 0;
+    bool in_flight = false;
+
+    // first load
+    {
+        int k1, h1;
+        int64_t t1;
+        if (next_chunk(p, sOrder, b, G, units, -1, 0, 0, &k1, &h1, &t1)) {
+            if (tid == 0) issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
+            in_flight = true;
+        }
+    }
+
+    bool aborted = false;
+    for (int k = 0; (int64_t)k * G < units && !aborted; ++k) {
+        const int u = unit_of(k, b, G);
+        if (u >= units) continue;
+        const Unit x = decode_unit(p, sOrder, u);
+        const int h = x.h;
+        const int64_t state_off = ((int64_t)x.n * H + h) * kHeadDim * kHeadDim;
+
+        // state rows: lane quarter of this warp = channel rows c, half = column half
+        const int c_row = quarter * 32 + lane;
+        if (x.eos == x.bos) {   // empty sequence: final = initial
+            if (p.final_state) {
+                for (int v0 = half * 64; v0 < half * 64 + 64; v0 += 4) {
+                    float4 s = p.initial_state
+                        ? *reinterpret_cast<const float4*>(p.initial_state + state_off + c_row * kHeadDim + v0)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    *reinterpret_cast<float4*>(p.final_state + state_off + c_row * kHeadDim + v0) = s;
+                }
+            }
+            continue;
+        }
+        // load the initial state into TMEM
+        for (int v0 = half * 64; v0 < half * 64 + 64; v0 += 16) {
+            uint32_t r[16];
+            for (int j = 0; j < 16; j += 4) {
+                float4 s = p.initial_state
+                    ? *reinterpret_cast<const float4*>(p.initial_state + state_off + c_row * kHeadDim + v0 + j)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                r[j] = __float_as_uint(s.x);
+                r[j + 1] = __float_as_uint(s.y);
+                r[j + 2] = __float_as_uint(s.z);
+                r[j + 3] = __float_as_uint(s.w);
+            }
+            tmem_st16(taddr(tbase, quarter, TM_S + v0), r);
+        }
+        tmem_wait_st();
+        fence_before_sync();
+
+        // per-unit gate constants for this thread's two channels (phase-1 mapping)
+        const int cb = warp & 1, blk = warp >> 1;
+        const int c0 = cb * 64 + 2 * lane;
+        const float nexp = -expf(p.A_log[h]);
+        const float db0 = p.dt_bias[h * kHeadDim + c0];
+        const float db1 = p.dt_bias[h * kHeadDim + c0 + 1];
+
+        const int64_t nch = (x.eos - x.bos + kChunk - 1) / kChunk;
+        for (int64_t j = 0; j < nch; ++j) {
+            const int64_t t0 = x.bos + j * kChunk;
+            const int L = (int)(x.eos - t0 < kChunk ? x.eos - t0 : kChunk);
+
+            // ================= phase 1: gate + operands =================
+            if (tid < kChunk) sBeta[tid] = tid < L ? p.beta[(t0 + tid) * H + h] : 0.f;
+            if (wait_or_abort(bar_in, in_parity, sAbort)) { aborted = true; break; }
+            in_parity ^= 1u;
+            in_flight = false;
+            fence_after_sync();
+
+            float G0[16], G1[16];
+            {
+                float a0 = 0.f, a1 = 0.f;
+                const float* gin = reinterpret_cast<const float*>(sm + IN_G);
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int r = blk * 16 + rr;
+                    const float2 gv = *reinterpret_cast<const float2*>(gin + r * kHeadDim + c0);
+                    const bool ok = r < L;
+                    a0 += ok ? gate_log_decay(gv.x + db0, nexp, p.lower_bound) : 0.f;
+                    a1 += ok ? gate_log_decay(gv.y + db1, nexp, p.lower_bound) : 0.f;
+                    G0[rr] = a0;
+                    G1[rr] = a1;
+                }
+                sTot[blk * kHeadDim + c0] = a0;
+                sTot[blk * kHeadDim + c0 + 1] = a1;
+            }
+            __syncthreads();
+            {
+                float tot0[4], tot1[4];
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) {
+                    tot0[bb] = sTot[bb * kHeadDim + c0];
+                    tot1[bb] = sTot[bb * kHeadDim + c0 + 1];
+                }
+                float Ts0 = 0.f, Ts1 = 0.f, after0 = 0.f, after1 = 0.f;
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) {
+                    if (bb < blk) { Ts0 += tot0[bb]; Ts1 += tot1[bb]; }
+                    if (bb > blk) { after0 += tot0[bb]; after1 += tot1[bb]; }
+                }
+                const float tb0 = tot0[blk], tb1 = tot1[blk];
+                const float eTs0 = expf(Ts0), eTs1 = expf(Ts1);             // e^{Gamma_s(b)}
+                const float invB0 = expf(-tb0), invB1 = expf(-tb1);         // e^{Gamma_s - Gamma_e} >= 1
+                const float eA0 = expf(after0), eA1 = expf(after1);         // e^{Gamma_last - Gamma_e}
+                float F2_0 = 0.f, F2_1 = 0.f, F3_0 = 0.f, F3_1 = 0.f;
+                if (blk <= 1) { F2_0 = expf(tot0[blk + 1]); F2_1 = expf(tot1[blk + 1]); }
+                if (blk == 0) { F3_0 = expf(tot0[1] + tot0[2]); F3_1 = expf(tot1[1] + tot1[2]); }
+                if (blk == 0) {
+                    sGammaC[c0] = expf(Ts0 + tb0 + after0);
+                    sGammaC[c0 + 1] = expf(Ts1 + tb1 + after1);
+                }
+                const __nv_bfloat162* kin = reinterpret_cast<const __nv_bfloat162*>(sm + IN_K);
+                const __nv_bfloat162* qin = reinterpret_cast<const __nv_bfloat162*>(sm + IN_Q);
+                const __nv_bfloat162* vin = reinterpret_cast<const __nv_bfloat162*>(sm + IN_V);
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int r = blk * 16 + rr;
+                    const bool ok = r < L;
+                    float2 kk = __bfloat1622float2(kin[(r * kHeadDim + c0) >> 1]);
+                    float2 qq = __bfloat1622float2(qin[(r * kHeadDim + c0) >> 1]);
+                    float2 vv = __bfloat1622float2(vin[(r * kHeadDim + c0) >> 1]);
+                    if (!ok) { kk = make_float2(0.f, 0.f); qq = kk; vv = kk; }
+                    const float be = sBeta[r];
+                    const float R0 = expf(G0[rr]), R1 = expf(G1[rr]);          // e^{Gamma_r - Gamma_s}
+                    const float E0 = expf(tb0 - G0[rr]), E1 = expf(tb1 - G1[rr]); // e^{Gamma_e - Gamma_r}
+                    const float kE0 = kk.x * E0, kE1 = kk.y * E1;
+                    st_u32(sm, AP_A + sw128_off(r, c0, 128), pack_bf16(kk.x * R0, kk.y * R1));
+                    st_u32(sm, AP_A + sw128_off(64 + r, c0, 128), pack_bf16(qq.x * R0, qq.y * R1));
+                    st_u32(sm, AP_B + sw128_off(r, c0, 160), pack_bf16(kE0 * invB0, kE1 * invB1));
+                    if (blk <= 2) st_u32(sm, AP_B + sw128_off(64 + r, c0, 160), pack_bf16(kE0, kE1));
+                    if (blk <= 1) st_u32(sm, AP_B + sw128_off(112 + r, c0, 160), pack_bf16(kE0 * F2_0, kE1 * F2_1));
+                    if (blk == 0) st_u32(sm, AP_B + sw128_off(144 + r, c0, 160), pack_bf16(kE0 * F3_0, kE1 * F3_1));
+                    const float g0 = R0 * eTs0, g1 = R1 * eTs1;                 // gamma_r
+                    st_u32(sm, GQ + sw128_off(r, c0, 64), pack_f16(qq.x * g0, qq.y * g1));
+                    st_u32(sm, BGK + sw128_off(r, c0, 64), pack_f16(be * kk.x * g0, be * kk.y * g1));
+                    st_u32(sm, KH + sw128_off(r, c0, 64), pack_f16(kE0 * eA0, kE1 * eA1));
+                    st_u32(sm, BV + sw128_off(r, c0, 64), pack_f16(be * vv.x, be * vv.y));
+                    float pd = fmaf(qq.x, kk.x, qq.y * kk.y);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) pd += __shfl_xor_sync(0xffffffffu, pd, o);
+                    if (lane == 0) sPdiag[cb * 64 + r] = pd;
+                }
+            }
+            fence_proxy_async();
+            __syncthreads();
+
+            // inputs consumed: prefetch the next chunk; issue the A/P MMA
+            if (tid == 0) {
+                int k1, h1;
+                int64_t t1;
+                if (next_chunk(p, sOrder, b, G, units, k, j, nch, &k1, &h1, &t1)) {
+                    issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
+                }
+                fence_after_sync();
+                const uint32_t a0 = smem_u32(sm + AP_A), b0 = smem_u32(sm + AP_B);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
+                            ks > 0 ? 1u : 0u);
+                mma_commit(bar_mma);
+            }
+            {
+                int k1, h1;
+                int64_t t1;
+                in_flight = next_chunk(p, sOrder, b, G, units, k, j, nch, &k1, &h1, &t1);
+            }
+            if (wait_or_abort(bar_mma, mma_parity, sAbort)) { aborted = true; break; }
+            mma_parity ^= 1u;
+            fence_after_sync();
+
+            // ================= phase 3: A / P read-out =================
+            if (warp < 4) {
+                const bool isA = quarter < 2;
+                const int r = (quarter & 1) * 32 + lane;      // token row in the chunk
+                const int I = r >> 4;
+                float* a32 = reinterpret_cast<float*>(sm + A32);
+                const float be = sBeta[r];
+                const float pdiag = sPdiag[r] + sPdiag[64 + r];
+                auto put = [&](int i, float val) {
+                    if (isA) a32[r * 65 + i] = be * val;
+                    else *reinterpret_cast<__half*>(sm + P16 + sw128_off(r, i, 64)) = __float2half_rn(val);
+                };
+                auto tile = [&](int d, uint32_t col0, int i0) {
+                    uint32_t v[16];
+                    tmem_ld16(taddr(tbase, quarter, TM_AP + col0), v);
+                    tmem_wait_ld();
+                    if (I - d == (i0 >> 4)) {
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) {
+                            const int i = i0 + jj;
+                            const float val = __uint_as_float(v[jj]);
+                            if (d > 0) put(i, val);
+                            else if (i < r) put(i, val);
+                            else if (i == r && !isA) put(i, pdiag);
+                        }
+                    }
+                };
+                if ((quarter & 1) == 0) {
+                    tile(0, 0, 0);
+                    tile(0, 16, 16);
+                    tile(1, 64 + 0, 0);
+                } else {
+                    tile(0, 32, 32);
+                    tile(0, 48, 48);
+                    tile(1, 64 + 16, 16);
+                    tile(1, 64 + 32, 32);
+                    tile(2, 112 + 0, 0);
+                    tile(2, 112 + 16, 16);
+                    tile(3, 144 + 0, 0);
+                }
+                // zeros above the diagonal (and A's diagonal)
+                for (int i = 0; i < kChunk; ++i) {
+                    const bool zero = (i >> 4) > I || ((i >> 4) == I && (isA ? i >= r : i > r));
+                    if (zero) put(i, 0.f);
+                }
+            }
+            fence_before_sync();
+            __syncthreads();
+
+            // ================= phase 4: T = (I + A)^-1 =================
+            {
+                const float* a32 = reinterpret_cast<const float*>(sm + A32);
+                float* t32 = reinterpret_cast<float*>(sm + T32);
+                float* msc = reinterpret_cast<float*>(sm + MSCR);
+                if (tid < 64) {   // diagonal 16 x 16 blocks, one column each
+                    const int bI = tid >> 4, jc = tid & 15, o = bI * 16;
+                    float xv[16];
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) {
+                        float s = (rr == jc) ? 1.f : 0.f;
+#pragma unroll
+                        for (int ii = 0; ii < rr; ++ii)
+                            if (ii >= jc) s = fmaf(-a32[(o + rr) * 65 + o + ii], xv[ii], s);
+                        xv[rr] = (rr < jc) ? 0.f : s;
+                        t32[(o + rr) * 65 + o + jc] = xv[rr];
+                    }
+                }
+                __syncthreads();
+                for (int I = 1; I < 4; ++I) {
+                    const int ncol = 16 * I;
+                    // M[ii][col] = sum_{kk < 16 I} A[16 I + ii][kk] T[kk][col]
+                    for (int e = tid; e < 16 * ncol; e += kThreads) {
+                        const int ii = e / ncol, col = e % ncol;
+                        float s = 0.f;
+                        for (int kk = (col >> 4) << 4; kk < ncol; ++kk)
+                            s = fmaf(a32[(16 * I + ii) * 65 + kk], t32[kk * 65 + col], s);
+                        msc[ii * 48 + col] = s;
+                    }
+                    __syncthreads();
+                    // T[16 I + ii][col] = - sum_{jj <= ii} T_II[ii][jj] M[jj][col]
+                    for (int e = tid; e < 16 * ncol; e += kThreads) {
+                        const int ii = e / ncol, col = e % ncol;
+                        float s = 0.f;
+                        for (int jj = 0; jj <= ii; ++jj)
+                            s = fmaf(t32[(16 * I + ii) * 65 + 16 * I + jj], msc[jj * 48 + col], s);
+                        t32[(16 * I + ii) * 65 + col] = -s;
+                    }
+                    __syncthreads();
+                }
+                // T -> fp16 K-major tile (zeros above the diagonal blocks)
+                for (int e = tid; e < 64 * 8; e += kThreads) {
+                    const int r = e >> 3, ch = e & 7;
+                    uint32_t w[4];
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const int i = ch * 8 + 2 * q2;
+                        const bool live = (i >> 4) <= (r >> 4);
+                        w[q2] = pack_f16(live ? t32[r * 65 + i] : 0.f, live ? t32[r * 65 + i + 1] : 0.f);
+                    }
+                    st_v4(sm, T16 + sw128_chunk_off(r, ch, 64), w[0], w[1], w[2], w[3]);
+                }
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
+
+            // ================= phase 5: W and U~^T MMAs =================
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t t16 = smem_u32(sm + T16), bgk = smem_u32(sm + BGK), bv = smem_u32(sm + BV);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(tbase + TM_W, desc_kmajor(t16, 64, ks), desc_mnmajor(bgk, 64, ks), IDESC_W,
+                            ks > 0 ? 1u : 0u);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(tbase + TM_UT, desc_mnmajor(bv, 64, ks), desc_kmajor(t16, 64, ks), IDESC_UT,
+                            ks > 0 ? 1u : 0u);
+                mma_commit(bar_mma);
+            }
+            if (wait_or_abort(bar_mma, mma_parity, sAbort)) { aborted = true; break; }
+            mma_parity ^= 1u;
+            fence_after_sync();
+
+            // ================= phase 6: W -> fp16 smem =================
+            {
+                // M = 64 accumulator: row r lives in lane (r % 16) of quarter r / 16
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const uint32_t col = half * 64 + cc * 16;
+                    uint32_t v[16];
+                    tmem_ld16(taddr(tbase, quarter, TM_W + col), v);
+                    tmem_wait_ld();
+                    if (lane < 16) {
+                        const int r = quarter * 16 + lane;
+                        uint32_t w[8];
+#pragma unroll
+                        for (int q2 = 0; q2 < 8; ++q2)
+                            w[q2] = pack_f16(__uint_as_float(v[2 * q2]), __uint_as_float(v[2 * q2 + 1]));
+                        st_v4(sm, W16 + sw128_chunk_off(r, col / 8, 64), w[0], w[1], w[2], w[3]);
+                        st_v4(sm, W16 + sw128_chunk_off(r, col / 8 + 1, 64), w[4], w[5], w[6], w[7]);
+                    }
+                }
+            }
+
+            // ================= phase 7: S copy + decay, U and O MMAs =================
+            {
+                const float gC = sGammaC[c_row];
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const uint32_t v0 = half * 64 + cc * 16;
+                    uint32_t v[16];
+                    tmem_ld16(taddr(tbase, quarter, TM_S + v0), v);
+                    tmem_wait_ld();
+                    uint32_t w[8];
+#pragma unroll
+                    for (int q2 = 0; q2 < 8; ++q2)
+                        w[q2] = pack_f16(__uint_as_float(v[2 * q2]), __uint_as_float(v[2 * q2 + 1]));
+                    st_v4(sm, S16 + sw128_chunk_off(c_row, v0 / 8, 128), w[0], w[1], w[2], w[3]);
+                    st_v4(sm, S16 + sw128_chunk_off(c_row, v0 / 8 + 1, 128), w[4], w[5], w[6], w[7]);
+#pragma unroll
+                    for (int q2 = 0; q2 < 16; ++q2) v[q2] = __float_as_uint(__uint_as_float(v[q2]) * gC);
+                    tmem_st16(taddr(tbase, quarter, TM_S + v0), v);
+                }
+                tmem_wait_st();
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t s16 = smem_u32(sm + S16), w16 = smem_u32(sm + W16), gq = smem_u32(sm + GQ);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_f16(tbase + TM_UT, desc_mnmajor(s16, 128, ks), desc_kmajor(w16, 64, ks), IDESC_U, 1u);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_f16(tbase + TM_OT, desc_mnmajor(s16, 128, ks), desc_kmajor(gq, 64, ks), IDESC_O1,
+                            ks > 0 ? 1u : 0u);
+                mma_commit(bar_mma);
+            }
+            if (wait_or_abort(bar_mma, mma_parity, sAbort)) { aborted = true; break; }
+            mma_parity ^= 1u;
+            fence_after_sync();
+
+            // ================= phase 8: U -> fp16, S and O MMAs =================
+            {
+                const int v_row = c_row;   // lanes of U^T are value columns
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const uint32_t r0 = half * 32 + cc * 16;
+                    uint32_t v[16];
+                    tmem_ld16(taddr(tbase, quarter, TM_UT + r0), v);
+                    tmem_wait_ld();
+                    uint32_t w[8];
+#pragma unroll
+                    for (int q2 = 0; q2 < 8; ++q2)
+                        w[q2] = pack_f16(__uint_as_float(v[2 * q2]), __uint_as_float(v[2 * q2 + 1]));
+                    st_v4(sm, U16 + sw128_chunk_off(v_row, r0 / 8, 128), w[0], w[1], w[2], w[3]);
+                    st_v4(sm, U16 + sw128_chunk_off(v_row, r0 / 8 + 1, 128), w[4], w[5], w[6], w[7]);
+                }
+            }
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t kh = smem_u32(sm + KH), u16 = smem_u32(sm + U16), p16 = smem_u32(sm + P16);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(tbase + TM_S, desc_mnmajor(kh, 64, ks), desc_kmajor(u16, 128, ks), IDESC_S, 1u);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(tbase + TM_OT, desc_kmajor(u16, 128, ks), desc_kmajor(p16, 64, ks), IDESC_O2, 1u);
+                mma_commit(bar_mma);
+            }
+            if (wait_or_abort(bar_mma, mma_parity, sAbort)) { aborted = true; break; }
+            mma_parity ^= 1u;
+            fence_after_sync();
+
+            // ================= phase 9: O -> out =================
+            {
+                const int v_col = c_row;
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int r0 = half * 32 + cc * 16;
+                    uint32_t v[16];
+                    tmem_ld16(taddr(tbase, quarter, TM_OT + r0), v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) {
+                        const int r = r0 + jj;
+                        if (r < L)
+                            p.out[((t0 + r) * H + h) * kHeadDim + v_col] =
+                                __float2bfloat16_rn(p.scale * __uint_as_float(v[jj]));
+                    }
+                }
+            }
+            fence_before_sync();
+            __syncthreads();
+        }
+        if (aborted) break;
+        // final state
+        if (p.final_state) {
+            fence_after_sync();
+            for (int v0 = half * 64; v0 < half * 64 + 64; v0 += 16) {
+                uint32_t r[16];
+                tmem_ld16(taddr(tbase, quarter, TM_S + v0), r);
+                tmem_wait_ld();
+                for (int jj = 0; jj < 16; jj += 4)
+                    *reinterpret_cast<float4*>(p.final_state + state_off + c_row * kHeadDim + v0 + jj) =
+                        make_float4(__uint_as_float(r[jj]), __uint_as_float(r[jj + 1]),
+                                    __uint_as_float(r[jj + 2]), __uint_as_float(r[jj + 3]));
+            }
+        }
+        fence_before_sync();
+        __syncthreads();
+    }
+
+    // wind-down: never leave with a TMA load or an MMA in flight
+    if (aborted) {
+        if (tid == 0) {
+            if (in_flight) mbar_wait_bounded(bar_in, in_parity);
+            mbar_wait_bounded(bar_mma, mma_parity);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 0) tmem_dealloc(tbase, TM_COLS);
+}
+
+// ---- host side ----
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t elem, int64_t rows,
+              int64_t cols) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * elem};
+    cuuint32_t box[2] = {(cuuint32_t)kHeadDim, (cuuint32_t)kChunk};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace fused
+
+bool fused_supported(float lower_bound) { return lower_bound >= KDA_FUSED_MIN_LOWER_BOUND; }
+
+cudaError_t launch_fused(const StagedArgs& a, cudaStream_t stream) {
+    using namespace fused;
+    static int sm_count = 0;
+    static bool attr_set = false;
+    if (!sm_count) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev);
+        if (sm_count <= 0) return cudaErrorInvalidDevice;
+    }
+    if (!attr_set) {
+        cudaError_t err = cudaFuncSetAttribute(kda_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)SMEM_ALLOC);
+        if (err != cudaSuccess) return err;
+        attr_set = true;
+    }
+    CUtensorMap tq, tk, tv, tg;
+    const int64_t rows = a.total_tokens, cols = (int64_t)a.H * kHeadDim;
+    if (!make_map(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols) ||
+        !make_map(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols) ||
+        !make_map(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols) ||
+        !make_map(&tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols))
+        return cudaErrorInvalidValue;
+    Params p;
+    p.beta = a.beta;
+    p.A_log = a.A_log;
+    p.dt_bias = a.dt_bias;
+    p.lower_bound = a.lower_bound;
+    p.scale = a.scale;
+    p.initial_state = a.initial_state;
+    p.cu_seqlens = a.cu_seqlens;
+    p.out = static_cast<__nv_bfloat16*>(a.out);
+    p.final_state = a.final_state;
+    p.seqlen = a.seqlen;
+    p.total_tokens = a.total_tokens;
+    p.H = a.H;
+    p.N = a.N;
+    const int64_t units = (int64_t)a.N * a.H;
+    const int grid = (int)(units < sm_count ? units : sm_count);
+    if (grid <= 0) return cudaSuccess;
+    kda_fused_kernel<<<grid, kThreads, SMEM_ALLOC, stream>>>(tq, tk, tv, tg, p);
+    return cudaGetLastError();
+}
 
 }  // namespace kda
