@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""KDA chunked-prefill throughput on B200 (one JSON line on stdout).
+
+Workload (default): T = 8192 packed tokens, seq_lens [1300, 547, 2048, 963, 271,
+3063], H = 96, K = V = 128, bf16 q/k/v, fp32 gates, no initial state -- the
+varlen row of the FlashKDA H20 benchmark table (toolarium.ru post, section
+"Что показывают H20-бенчмарки"), with synthetic seeded inputs (kda_workloads).
+
+A step is one kda_fwd call over the whole batch (the fused tcgen05 kernel:
+gate pre-pass, intra-chunk WY, state propagation and output in one launch).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs an independent
+replica of the workload (the forward has no cross-GPU exchange); the value is
+the tokens of all ranks over the slowest rank's time.  --impl reference times
+the fp64 CPU oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kda_workloads as W  # noqa: E402
+
+BYTES_PER_TOKEN_HEAD = 1540          # q,k,v bf16 768 + g fp32 512 + beta 4 + out bf16 256
+STATE_BYTES = 128 * 128 * 4          # one (sequence, head) state, read or written
+FLOP_PER_TOKEN_HEAD = 180224         # 10 C D + 6 D^2 with C = 64, D = 128
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--workload", type=int, default=2, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(w: W.Workload) -> int:
+    b = BYTES_PER_TOKEN_HEAD * w.T * w.H
+    if w.init is not None:
+        b += STATE_BYTES * w.N * w.H
+    if w.final:
+        b += STATE_BYTES * w.N * w.H
+    return b
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_135_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic_from_profile(w: W.Workload):
+    """Per-launch DRAM bytes of the fused kernel from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "kda_fused_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    per_unit = d.get("dram_bytes_per_token_head")
+    if per_unit is None:
+        return None
+    return float(per_unit) * w.T * w.H
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x0000000000000004: "sw_power_cap",
+        0x0000000000000008: "hw_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000080: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                break
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "kda" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available() and args.impl == "kda":
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_sample(w: W.Workload, x: dict, target_s: float):
+    """Runs the fp64 oracle on the first h heads of every sequence, h sized so
+    the run takes about target_s seconds; returns (tokens-equivalent/s, desc)."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+
+    def run(h):
+        sub = dict(x)
+        for key in ("q", "k", "v", "g", "beta"):
+            sub[key] = x[key][:, :h].contiguous()
+        sub["A_log"] = x["A_log"][:h]
+        sub["dt_bias"] = x["dt_bias"][:h]
+        if x["initial_state"] is not None:
+            sub["initial_state"] = x["initial_state"][:, :h].contiguous()
+        t = time.perf_counter()
+        oracle.recurrent(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"], sub["A_log"],
+                         sub["dt_bias"], sub["lower_bound"], sub["scale"], sub["initial_state"],
+                         sub["cu_seqlens"], want_final=w.final)
+        return time.perf_counter() - t
+
+    # calibrate on one head: its N (sequence, head) units run on min(N, cores) threads
+    t1 = run(1)
+    per_token_head = t1 * min(w.N, cores) / w.T          # core-seconds per token-head
+    h = int(target_s * cores / max(per_token_head * w.T, 1e-9))
+    h = max(1, min(w.H, h))
+    t = run(h) if h > 1 else t1
+    rate = (w.T * h / w.H) / t          # whole-workload tokens per second equivalent
+    desc = (f"oracle over heads 0..{h - 1} of {w.H} (all {w.N} sequences, {w.T * h} token-heads) "
+            f"in {t:.2f} s on {oracle.max_threads()} OpenMP threads; scaled by {h}/{w.H}")
+    return rate, desc, cores, oracle.max_threads(), h
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = W.WORKLOADS[args.workload]
+    x = W.make_inputs(w)
+    import oracle
+    # size each step's sample so the whole run stays within a few minutes
+    per_step_target = max(0.5, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    rate, desc, cores, threads, h = oracle_sample(w, x, per_step_target)
+
+    def step():
+        sub = dict(x)
+        for key in ("q", "k", "v", "g", "beta"):
+            sub[key] = x[key][:, :h].contiguous()
+        sub["A_log"] = x["A_log"][:h]
+        sub["dt_bias"] = x["dt_bias"][:h]
+        if x["initial_state"] is not None:
+            sub["initial_state"] = x["initial_state"][:, :h].contiguous()
+        oracle.recurrent(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"], sub["A_log"],
+                         sub["dt_bias"], sub["lower_bound"], sub["scale"], sub["initial_state"],
+                         sub["cu_seqlens"], want_final=w.final)
+
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t
+    ms_per_step = el / args.steps * 1e3 * (w.H / h)     # whole-workload equivalent
+    value = w.T / (ms_per_step / 1e3) / 1e6
+    line = {
+        "impl": "reference", "metric": "KDA prefill throughput (Mtokens/s) at T=8192 H=96 D=128 varlen",
+        "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.describe(), "global_batch": w.N, "seq_len": w.T,
+                   "parallelism": "host cores (OpenMP over sequence x head)"},
+        "cpu_baseline": {"value": value, "unit": "Mtokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"each step: {desc.split(' in ')[0]}; scaled by {h}/{w.H}"},
+        "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        rc = run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
+
+    from gated_delta_rule_135_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(world)
+    import gated_delta_rule_135_b200 as kda
+
+    w = W.WORKLOADS[args.workload]
+    x = W.make_inputs(w)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    out = torch.empty_like(xd["q"])
+    fin = (torch.empty(w.N, w.H, 128, 128, device=dev) if w.final else None)
+    stream = torch.cuda.current_stream()
+    fused = x["lower_bound"] >= kda.FUSED_MIN_LOWER_BOUND
+    launches_per_step = 1 if fused else 5
+
+    def step():
+        kda.kda_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"],
+                    x["lower_bound"], x["scale"], xd["initial_state"], xd["cu_seqlens"], out=out,
+                    final_state=fin, batch=x["batch"])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if kda.kda_check_device_error() != 0:
+        raise RuntimeError("device error recorded during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = starts[0].elapsed_time(ends[-1])
+    total_ms = max_over_ranks(total_ms, world)
+    ms_per_step = total_ms / args.steps
+    tokens = w.T * world
+    value = tokens / (ms_per_step / 1e3) / 1e6
+    tflops = FLOP_PER_TOKEN_HEAD * w.T * w.H * world / (ms_per_step / 1e3) / 1e12
+    kernel_ms = statistics.mean(per_step)
+    alg_bytes = algorithmic_bytes(w)
+    peak, peak_kind = measured_hbm_peak()
+    achieved = alg_bytes / (kernel_ms / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "traffic": dram_traffic_from_profile(w),
+            "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
+            else "fallback 6650 GB/s",
+            "kernel": "kda_fused_kernel" if fused else "staged kernels",
+            "kernel_ms": kernel_ms, "algorithmic_bytes": alg_bytes,
+            "tflops": tflops}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        keys = ("q", "k", "v", "g", "beta")
+        host = {k: x[k].pin_memory() for k in keys}
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+        d2h = out_h.numel() * out_h.element_size()
+        for _ in range(2):
+            for k in keys:
+                xd[k].copy_(host[k], non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for k in keys:
+                xd[k].copy_(host[k], non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.e2e_steps
+        e2e = {"value": tokens / (e_ms / 1e3) / 1e6, "unit": "Mtokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc, cores, threads, _ = oracle_sample(w, x, args.cpu_seconds)
+        cpu = {"value": rate / 1e6, "unit": "Mtokens/s", "cores": threads, "kind": "oracle",
+               "sample": desc, "host_cores": cores}
+
+    if rank == 0:
+        line = {
+            "metric": "KDA prefill throughput (Mtokens/s) at T=8192 H=96 D=128 varlen",
+            "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded kda_workloads, no dataset)",
+            "config": {"workload": w.describe(), "model": "KDA layer forward (no weights)",
+                       "global_batch": w.N * world, "seq_len": w.T, "heads": w.H,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "precision": "bf16 q/k/v/out, fp32 gates and state; bf16/fp16 MMA operands, fp32 accumulate",
+                       "l2": f"inputs exceed L2 ({alg_bytes / 1e6:.0f} MB per step vs 126 MB); no flush"},
+            "tflops": tflops,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -15,7 +15,9 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkda.so")
+# KDA_LIBRARY may name another build of the same library (e.g. the
+# phase-clock instrumented libkda_phase.so); the default is libkda.so.
+LIB_PATH = os.environ.get("KDA_LIBRARY", os.path.join(_HERE, "libkda.so"))
 
 HEAD_DIM = 128
 CHUNK = 64

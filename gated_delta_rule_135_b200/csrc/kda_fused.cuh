@@ -39,6 +39,7 @@
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "umma.cuh"
+#include "warp_mma.cuh"
 
 namespace kda {
 namespace fused {
@@ -46,6 +47,22 @@ namespace fused {
 using namespace umma;
 
 constexpr int kThreads = 256;
+
+// Optional per-phase cycle accounting (debug builds with -DKDA_PHASE_CLOCKS).
+#ifdef KDA_PHASE_CLOCKS
+constexpr int kPhases = 18;
+__device__ unsigned long long g_phase_cycles[kPhases];
+#define PHASE_MARK(i)                                   \
+    do {                                                \
+        if (threadIdx.x == 0) {                         \
+            const long long now_ = clock64();           \
+            ph_acc[i] += (unsigned long long)(now_ - ph_last); \
+            ph_last = now_;                             \
+        }                                               \
+    } while (0)
+#else
+#define PHASE_MARK(i) do { } while (0)
+#endif
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
 constexpr uint32_t IN_Q = 0;          // bf16 [64][128] row-major (TMA box)
@@ -56,16 +73,17 @@ constexpr uint32_t IN_BYTES = 81920;
 constexpr uint32_t X = 81920;         // phase-shared region, 73728 bytes
 constexpr uint32_t AP_A = X + 0;      // bf16 K-major [128 rows][128]: k*R rows 0-63, q*R rows 64-127
 constexpr uint32_t AP_B = X + 32768;  // bf16 K-major [160 rows][128]: XD | C1 | C2 | C3
-constexpr uint32_t A32 = X + 0;       // fp32 [64][65]      (phases 3-4)
-constexpr uint32_t T32 = X + 16640;   // fp32 [64][65]      (phase 4)
-constexpr uint32_t T16 = X + 33792;   // fp16 K-major [64][64]        (phases 4-5)
-constexpr uint32_t MSCR = X + 41984;  // fp32 [16][48] solve scratch  (phase 4)
+constexpr int kF32Pitch = 68;         // fp32 row pitch of A32 / T32 (16-byte aligned rows)
+constexpr uint32_t A32 = X + 0;       // fp32 [64][68] beta-scaled A  (phases 3-4)
+constexpr uint32_t T32 = X + 17408;   // fp32 [64][68] T = (I + A)^-1 (phase 4)
+constexpr uint32_t T16 = X + 35840;   // fp16 K-major [64][64]        (phases 4-5)
 constexpr uint32_t W16 = X + 0;       // fp16 K-major [64 r][128 c]   (phases 6-7)
 constexpr uint32_t S16 = X + 16384;   // fp16 [128 c][128 v] (MN-major A)  (phase 7)
 constexpr uint32_t P16 = X + 65536;   // fp16 K-major [64 r][64 i]    (phases 3-8)
 constexpr uint32_t BGK = X + 73728;   // fp16 [64 i][128 c] beta*gamma*k  (MN-major B of W)
 constexpr uint32_t U16 = BGK;         // fp16 K-major [128 v][64 r]   (phase 8; BGK is dead)
 constexpr uint32_t BV = BGK + 16384;  // fp16 [64 i][128 v] beta*v    (MN-major A of U~^T)
+constexpr uint32_t OST = BV;          // bf16 [64 r][128 v] output staging (phase 9; BV is dead)
 constexpr uint32_t GQ = BV + 16384;   // fp16 K-major [64 r][128 c] gamma*q
 constexpr uint32_t KH = GQ + 16384;   // fp16 [64 i][128 c] Khat     (MN-major A of S update)
 constexpr uint32_t MISC = KH + 16384;
@@ -198,6 +216,26 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     return *abort_flag != 0u;
 }
 
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float fast_ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float fast_lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// Gate in base-2 units: log2 a = max(-exp(A_log) * log2(1 + 2^x2), lower_bound * log2 e)
+// with x2 = (g + dt_bias) * log2 e, i.e. softplus written as max(x2, 0) + log2(1 + 2^-|x2|).
+__device__ __forceinline__ float gate_log2_decay(float g, float db2, float nexpA, float lb2) {
+    const float x2 = fmaf(g, kLog2e, db2);
+    const float sp2 = fmaxf(x2, 0.f) + fast_lg2(1.f + fast_ex2(-fabsf(x2)));
+    return fmaxf(nexpA * sp2, lb2);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -251,9 +289,14 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     fence_after_sync();
     const uint32_t tbase = *sTmem;
+#ifdef KDA_PHASE_CLOCKS
+    unsigned long long ph_acc[kPhases] = {};
+    long long ph_last = clock64();
+#endif
 
     uint32_t in_parity = 0, mma_parity = 0;
     bool in_flight = false;
+    float beta_next = 0.f;   // beta of the chunk in flight (threads 0-63)
 
     // first load
     {
@@ -261,9 +304,21 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         int64_t t1;
         if (next_chunk(p, sOrder, b, G, units, -1, 0, 0, &k1, &h1, &t1)) {
             if (tid == 0) issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
+            if (tid < kChunk && t1 + tid < p.total_tokens) beta_next = p.beta[(t1 + tid) * H + h1];
             in_flight = true;
         }
     }
+
+    // phase-1 thread mapping: warp -> (64-channel block cb, 16-token block blk), lane -> channel pair
+    const int cb = warp & 1, blk = warp >> 1;
+    const int c0 = cb * 64 + 2 * lane;
+    const uint32_t lo = (uint32_t)(c0 & 7) * 2u;
+    const uint32_t chk = (uint32_t)(c0 & 63) >> 3;
+    const uint32_t off128 = (uint32_t)cb * 128u * 128u + (uint32_t)blk * 2048u + lo;
+    const uint32_t off160 = (uint32_t)cb * 160u * 128u + (uint32_t)blk * 2048u + lo;
+    const uint32_t off64 = (uint32_t)cb * 64u * 128u + (uint32_t)blk * 2048u + lo;
+    // state / TMEM mapping: lane quarter -> rows, half -> column half
+    const int c_row = quarter * 32 + lane;
 
     bool aborted = false;
     for (int k = 0; (int64_t)k * G < units && !aborted; ++k) {
@@ -273,8 +328,6 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int h = x.h;
         const int64_t state_off = ((int64_t)x.n * H + h) * kHeadDim * kHeadDim;
 
-        // state rows: lane quarter of this warp = channel rows c, half = column half
-        const int c_row = quarter * 32 + lane;
         if (x.eos == x.bos) {   // empty sequence: final = initial
             if (p.final_state) {
                 for (int v0 = half * 64; v0 < half * 64 + 64; v0 += 4) {
@@ -289,6 +342,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // load the initial state into TMEM
         for (int v0 = half * 64; v0 < half * 64 + 64; v0 += 16) {
             uint32_t r[16];
+#pragma unroll
             for (int j = 0; j < 16; j += 4) {
                 float4 s = p.initial_state
                     ? *reinterpret_cast<const float4*>(p.initial_state + state_off + c_row * kHeadDim + v0 + j)
@@ -303,12 +357,11 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_wait_st();
         fence_before_sync();
 
-        // per-unit gate constants for this thread's two channels (phase-1 mapping)
-        const int cb = warp & 1, blk = warp >> 1;
-        const int c0 = cb * 64 + 2 * lane;
-        const float nexp = -expf(p.A_log[h]);
-        const float db0 = p.dt_bias[h * kHeadDim + c0];
-        const float db1 = p.dt_bias[h * kHeadDim + c0 + 1];
+        // per-unit gate constants of this thread's two channels (base-2 units)
+        const float nexpA = -expf(p.A_log[h]);
+        const float lb2 = p.lower_bound * kLog2e;
+        const float db2_0 = p.dt_bias[h * kHeadDim + c0] * kLog2e;
+        const float db2_1 = p.dt_bias[h * kHeadDim + c0 + 1] * kLog2e;
 
         const int64_t nch = (x.eos - x.bos + kChunk - 1) / kChunk;
         for (int64_t j = 0; j < nch; ++j) {
@@ -316,13 +369,14 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int L = (int)(x.eos - t0 < kChunk ? x.eos - t0 : kChunk);
 
             // ================= phase 1: gate + operands =================
-            if (tid < kChunk) sBeta[tid] = tid < L ? p.beta[(t0 + tid) * H + h] : 0.f;
+            PHASE_MARK(0);
+            if (tid < kChunk) sBeta[tid] = tid < L ? beta_next : 0.f;
             if (wait_or_abort(bar_in, in_parity, sAbort)) { aborted = true; break; }
+            PHASE_MARK(1);
             in_parity ^= 1u;
             in_flight = false;
-            fence_after_sync();
 
-            float G0[16], G1[16];
+            float G0[16], G1[16];   // in-block inclusive cumsum of log2 a (two channels)
             {
                 float a0 = 0.f, a1 = 0.f;
                 const float* gin = reinterpret_cast<const float*>(sm + IN_G);
@@ -331,14 +385,17 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const int r = blk * 16 + rr;
                     const float2 gv = *reinterpret_cast<const float2*>(gin + r * kHeadDim + c0);
                     const bool ok = r < L;
-                    a0 += ok ? gate_log_decay(gv.x + db0, nexp, p.lower_bound) : 0.f;
-                    a1 += ok ? gate_log_decay(gv.y + db1, nexp, p.lower_bound) : 0.f;
+                    const float l0 = gate_log2_decay(gv.x, db2_0, nexpA, lb2);
+                    const float l1 = gate_log2_decay(gv.y, db2_1, nexpA, lb2);
+                    a0 += ok ? l0 : 0.f;
+                    a1 += ok ? l1 : 0.f;
                     G0[rr] = a0;
                     G1[rr] = a1;
                 }
                 sTot[blk * kHeadDim + c0] = a0;
                 sTot[blk * kHeadDim + c0 + 1] = a1;
             }
+            PHASE_MARK(12);
             __syncthreads();
             {
                 float tot0[4], tot1[4];
@@ -353,131 +410,172 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (bb < blk) { Ts0 += tot0[bb]; Ts1 += tot1[bb]; }
                     if (bb > blk) { after0 += tot0[bb]; after1 += tot1[bb]; }
                 }
-                const float tb0 = tot0[blk], tb1 = tot1[blk];
-                const float eTs0 = expf(Ts0), eTs1 = expf(Ts1);             // e^{Gamma_s(b)}
-                const float invB0 = expf(-tb0), invB1 = expf(-tb1);         // e^{Gamma_s - Gamma_e} >= 1
-                const float eA0 = expf(after0), eA1 = expf(after1);         // e^{Gamma_last - Gamma_e}
+                auto pick4 = [](const float (&a)[4], int i) {
+                    return i == 0 ? a[0] : (i == 1 ? a[1] : (i == 2 ? a[2] : a[3]));
+                };
+                const float tb0 = pick4(tot0, blk), tb1 = pick4(tot1, blk);
+                const float eTs0 = fast_ex2(Ts0), eTs1 = fast_ex2(Ts1);        // gamma at the block start
+                const float invB0 = fast_ex2(-tb0), invB1 = fast_ex2(-tb1);    // e^{Gamma_s - Gamma_e} >= 1
+                const float eA0 = fast_ex2(after0), eA1 = fast_ex2(after1);    // e^{Gamma_last - Gamma_e}
                 float F2_0 = 0.f, F2_1 = 0.f, F3_0 = 0.f, F3_1 = 0.f;
-                if (blk <= 1) { F2_0 = expf(tot0[blk + 1]); F2_1 = expf(tot1[blk + 1]); }
-                if (blk == 0) { F3_0 = expf(tot0[1] + tot0[2]); F3_1 = expf(tot1[1] + tot1[2]); }
+                if (blk <= 1) { F2_0 = fast_ex2(pick4(tot0, blk + 1)); F2_1 = fast_ex2(pick4(tot1, blk + 1)); }
+                if (blk == 0) { F3_0 = fast_ex2(tot0[1] + tot0[2]); F3_1 = fast_ex2(tot1[1] + tot1[2]); }
                 if (blk == 0) {
-                    sGammaC[c0] = expf(Ts0 + tb0 + after0);
-                    sGammaC[c0 + 1] = expf(Ts1 + tb1 + after1);
+                    sGammaC[c0] = fast_ex2(tb0 + after0);
+                    sGammaC[c0 + 1] = fast_ex2(tb1 + after1);
                 }
-                const __nv_bfloat162* kin = reinterpret_cast<const __nv_bfloat162*>(sm + IN_K);
-                const __nv_bfloat162* qin = reinterpret_cast<const __nv_bfloat162*>(sm + IN_Q);
-                const __nv_bfloat162* vin = reinterpret_cast<const __nv_bfloat162*>(sm + IN_V);
+                const uint32_t* kin = reinterpret_cast<const uint32_t*>(sm + IN_K);
+                const uint32_t* qin = reinterpret_cast<const uint32_t*>(sm + IN_Q);
+                const uint32_t* vin = reinterpret_cast<const uint32_t*>(sm + IN_V);
+                float pd[16];
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) {
                     const int r = blk * 16 + rr;
                     const bool ok = r < L;
-                    float2 kk = __bfloat1622float2(kin[(r * kHeadDim + c0) >> 1]);
-                    float2 qq = __bfloat1622float2(qin[(r * kHeadDim + c0) >> 1]);
-                    float2 vv = __bfloat1622float2(vin[(r * kHeadDim + c0) >> 1]);
-                    if (!ok) { kk = make_float2(0.f, 0.f); qq = kk; vv = kk; }
+                    const int idx = (r * kHeadDim + c0) >> 1;
+                    const uint32_t kw = ok ? kin[idx] : 0u, qw = ok ? qin[idx] : 0u, vw = ok ? vin[idx] : 0u;
+                    const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
+                    const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
+                    const float v0 = __uint_as_float(vw << 16), v1 = __uint_as_float(vw & 0xFFFF0000u);
                     const float be = sBeta[r];
-                    const float R0 = expf(G0[rr]), R1 = expf(G1[rr]);          // e^{Gamma_r - Gamma_s}
-                    const float E0 = expf(tb0 - G0[rr]), E1 = expf(tb1 - G1[rr]); // e^{Gamma_e - Gamma_r}
-                    const float kE0 = kk.x * E0, kE1 = kk.y * E1;
-                    st_u32(sm, AP_A + sw128_off(r, c0, 128), pack_bf16(kk.x * R0, kk.y * R1));
-                    st_u32(sm, AP_A + sw128_off(64 + r, c0, 128), pack_bf16(qq.x * R0, qq.y * R1));
-                    st_u32(sm, AP_B + sw128_off(r, c0, 160), pack_bf16(kE0 * invB0, kE1 * invB1));
-                    if (blk <= 2) st_u32(sm, AP_B + sw128_off(64 + r, c0, 160), pack_bf16(kE0, kE1));
-                    if (blk <= 1) st_u32(sm, AP_B + sw128_off(112 + r, c0, 160), pack_bf16(kE0 * F2_0, kE1 * F2_1));
-                    if (blk == 0) st_u32(sm, AP_B + sw128_off(144 + r, c0, 160), pack_bf16(kE0 * F3_0, kE1 * F3_1));
-                    const float g0 = R0 * eTs0, g1 = R1 * eTs1;                 // gamma_r
-                    st_u32(sm, GQ + sw128_off(r, c0, 64), pack_f16(qq.x * g0, qq.y * g1));
-                    st_u32(sm, BGK + sw128_off(r, c0, 64), pack_f16(be * kk.x * g0, be * kk.y * g1));
-                    st_u32(sm, KH + sw128_off(r, c0, 64), pack_f16(kE0 * eA0, kE1 * eA1));
-                    st_u32(sm, BV + sw128_off(r, c0, 64), pack_f16(be * vv.x, be * vv.y));
-                    float pd = fmaf(qq.x, kk.x, qq.y * kk.y);
+                    const float R0 = fast_ex2(G0[rr]), R1 = fast_ex2(G1[rr]);            // e^{Gamma_r - Gamma_s}
+                    const float E0 = fast_ex2(tb0 - G0[rr]), E1 = fast_ex2(tb1 - G1[rr]);  // e^{Gamma_e - Gamma_r}
+                    const float kE0 = k0 * E0, kE1 = k1 * E1;
+                    const uint32_t ro = (uint32_t)rr * 128u + ((chk ^ (uint32_t)(rr & 7)) << 4);
+                    st_u32(sm, AP_A + off128 + ro, pack_bf16(k0 * R0, k1 * R1));
+                    st_u32(sm, AP_A + off128 + 64u * 128u + ro, pack_bf16(q0 * R0, q1 * R1));
+                    st_u32(sm, AP_B + off160 + ro, pack_bf16(kE0 * invB0, kE1 * invB1));
+                    if (blk <= 2) st_u32(sm, AP_B + off160 + 64u * 128u + ro, pack_bf16(kE0, kE1));
+                    if (blk <= 1) st_u32(sm, AP_B + off160 + 112u * 128u + ro, pack_bf16(kE0 * F2_0, kE1 * F2_1));
+                    if (blk == 0) st_u32(sm, AP_B + off160 + 144u * 128u + ro, pack_bf16(kE0 * F3_0, kE1 * F3_1));
+                    const float g0 = R0 * eTs0, g1 = R1 * eTs1;                          // gamma_r
+                    const float bk0 = be * k0 * g0, bk1 = be * k1 * g1;
+                    st_u32(sm, GQ + off64 + ro, pack_f16(q0 * g0, q1 * g1));
+                    st_u32(sm, BGK + off64 + ro, pack_f16(bk0, bk1));
+                    st_u32(sm, KH + off64 + ro, pack_f16(kE0 * eA0, kE1 * eA1));
+                    st_u32(sm, BV + off64 + ro, pack_f16(be * v0, be * v1));
+                    pd[rr] = fmaf(q0, k0, q1 * k1);
+                }
+                PHASE_MARK(13);
+                // reduce pd over the 32 lanes for all 16 tokens at once (transposing butterfly):
+                // after the halving steps lanes 2m and 2m + 1 hold token m of the block
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) pd += __shfl_xor_sync(0xffffffffu, pd, o);
-                    if (lane == 0) sPdiag[cb * 64 + r] = pd;
+                for (int t = 0; t < 8; ++t) {
+                    const bool up = lane & 16;
+                    const float send = up ? pd[t] : pd[t + 8];
+                    const float keep = up ? pd[t + 8] : pd[t];
+                    pd[t] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const bool up = lane & 8;
+                    const float send = up ? pd[t] : pd[t + 4];
+                    const float keep = up ? pd[t + 4] : pd[t];
+                    pd[t] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                }
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const bool up = lane & 4;
+                    const float send = up ? pd[t] : pd[t + 2];
+                    const float keep = up ? pd[t + 2] : pd[t];
+                    pd[t] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+                }
+                {
+                    const bool up = lane & 2;
+                    const float send = up ? pd[0] : pd[1];
+                    const float keep = up ? pd[1] : pd[0];
+                    pd[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                }
+                pd[0] += __shfl_xor_sync(0xffffffffu, pd[0], 1);
+                // token held: bit3 of the token = lane bit4, bit2 = lane bit3, bit1 = lane bit2, bit0 = lane bit1
+                if ((lane & 1) == 0) {
+                    const int tk = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
+                                   ((lane >> 1) & 1);
+                    sPdiag[cb * 64 + blk * 16 + tk] = pd[0];
                 }
             }
             fence_proxy_async();
             __syncthreads();
+            PHASE_MARK(2);
 
             // inputs consumed: prefetch the next chunk; issue the A/P MMA
-            if (tid == 0) {
-                int k1, h1;
-                int64_t t1;
-                if (next_chunk(p, sOrder, b, G, units, k, j, nch, &k1, &h1, &t1)) {
-                    issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
-                }
-                fence_after_sync();
-                const uint32_t a0 = smem_u32(sm + AP_A), b0 = smem_u32(sm + AP_B);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
-                            ks > 0 ? 1u : 0u);
-                mma_commit(bar_mma);
-            }
             {
                 int k1, h1;
                 int64_t t1;
                 in_flight = next_chunk(p, sOrder, b, G, units, k, j, nch, &k1, &h1, &t1);
+                if (tid == 0) {
+                    if (in_flight) issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
+                    fence_after_sync();
+                    const uint32_t a0 = smem_u32(sm + AP_A), b0 = smem_u32(sm + AP_B);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
+                                ks > 0 ? 1u : 0u);
+                    mma_commit(bar_mma);
+                }
+                if (in_flight && tid < kChunk && t1 + tid < p.total_tokens)
+                    beta_next = p.beta[(t1 + tid) * H + h1];
             }
             if (wait_or_abort(bar_mma, mma_parity, sAbort)) { aborted = true; break; }
             mma_parity ^= 1u;
             fence_after_sync();
+            PHASE_MARK(3);
 
             // ================= phase 3: A / P read-out =================
             if (warp < 4) {
                 const bool isA = quarter < 2;
                 const int r = (quarter & 1) * 32 + lane;      // token row in the chunk
                 const int I = r >> 4;
-                float* a32 = reinterpret_cast<float*>(sm + A32);
-                const float be = sBeta[r];
-                const float pdiag = sPdiag[r] + sPdiag[64 + r];
-                auto put = [&](int i, float val) {
-                    if (isA) a32[r * 65 + i] = be * val;
-                    else *reinterpret_cast<__half*>(sm + P16 + sw128_off(r, i, 64)) = __float2half_rn(val);
-                };
-                auto tile = [&](int d, uint32_t col0, int i0) {
-                    uint32_t v[16];
-                    tmem_ld16(taddr(tbase, quarter, TM_AP + col0), v);
+                float row[64];
+                auto pick = [&](int J, uint32_t col_a, uint32_t col_b, int I_a) {
+                    // block J of the row: from TMEM columns col_a (rows with I == I_a) or col_b
+                    uint32_t ta[16], tb2[16];
+                    tmem_ld16(taddr(tbase, quarter, TM_AP + col_a), ta);
+                    tmem_ld16(taddr(tbase, quarter, TM_AP + col_b), tb2);
                     tmem_wait_ld();
-                    if (I - d == (i0 >> 4)) {
 #pragma unroll
-                        for (int jj = 0; jj < 16; ++jj) {
-                            const int i = i0 + jj;
-                            const float val = __uint_as_float(v[jj]);
-                            if (d > 0) put(i, val);
-                            else if (i < r) put(i, val);
-                            else if (i == r && !isA) put(i, pdiag);
-                        }
-                    }
+                    for (int jj = 0; jj < 16; ++jj)
+                        row[J * 16 + jj] = __uint_as_float(I == I_a ? ta[jj] : tb2[jj]);
                 };
-                if ((quarter & 1) == 0) {
-                    tile(0, 0, 0);
-                    tile(0, 16, 16);
-                    tile(1, 64 + 0, 0);
-                } else {
-                    tile(0, 32, 32);
-                    tile(0, 48, 48);
-                    tile(1, 64 + 16, 16);
-                    tile(1, 64 + 32, 32);
-                    tile(2, 112 + 0, 0);
-                    tile(2, 112 + 16, 16);
-                    tile(3, 144 + 0, 0);
+                if ((quarter & 1) == 0) {        // I in {0, 1}
+                    pick(0, 0, 64, 0);           // I=0: d=0 cols 0-15; I=1: d=1 cols 64-79
+                    pick(1, 16, 16, 1);          // I=1: d=0 cols 16-31 (I=0: masked below)
+#pragma unroll
+                    for (int jj = 32; jj < 64; ++jj) row[jj] = 0.f;
+                } else {                         // I in {2, 3}
+                    pick(0, 112, 144, 2);        // I=2: d=2 cols 112-127; I=3: d=3 cols 144-159
+                    pick(1, 80, 128, 2);         // I=2: d=1 cols 80-95;   I=3: d=2 cols 128-143
+                    pick(2, 32, 96, 2);          // I=2: d=0 cols 32-47;   I=3: d=1 cols 96-111
+                    pick(3, 48, 48, 3);          // I=3: d=0 cols 48-63 (I=2: masked below)
                 }
-                // zeros above the diagonal (and A's diagonal)
-                for (int i = 0; i < kChunk; ++i) {
-                    const bool zero = (i >> 4) > I || ((i >> 4) == I && (isA ? i >= r : i > r));
-                    if (zero) put(i, 0.f);
+                const float pdg = sPdiag[r] + sPdiag[64 + r];
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    row[i] = i < r ? row[i] : ((i == r && !isA) ? pdg : 0.f);
+                if (isA) {
+                    const float be = sBeta[r];
+                    float* a32 = reinterpret_cast<float*>(sm + A32) + r * kF32Pitch;
+#pragma unroll
+                    for (int i = 0; i < 64; i += 4)
+                        *reinterpret_cast<float4*>(a32 + i) =
+                            make_float4(be * row[i], be * row[i + 1], be * row[i + 2], be * row[i + 3]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        st_v4(sm, P16 + sw128_chunk_off(r, c, 64), pack_f16(row[8 * c], row[8 * c + 1]),
+                              pack_f16(row[8 * c + 2], row[8 * c + 3]), pack_f16(row[8 * c + 4], row[8 * c + 5]),
+                              pack_f16(row[8 * c + 6], row[8 * c + 7]));
                 }
             }
             fence_before_sync();
             __syncthreads();
+            PHASE_MARK(4);
 
             // ================= phase 4: T = (I + A)^-1 =================
             {
                 const float* a32 = reinterpret_cast<const float*>(sm + A32);
                 float* t32 = reinterpret_cast<float*>(sm + T32);
-                float* msc = reinterpret_cast<float*>(sm + MSCR);
-                if (tid < 64) {   // diagonal 16 x 16 blocks, one column each
+                if (tid < 64) {   // diagonal 16 x 16 blocks by forward substitution, one column each
                     const int bI = tid >> 4, jc = tid & 15, o = bI * 16;
                     float xv[16];
 #pragma unroll
@@ -485,49 +583,74 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         float s = (rr == jc) ? 1.f : 0.f;
 #pragma unroll
                         for (int ii = 0; ii < rr; ++ii)
-                            if (ii >= jc) s = fmaf(-a32[(o + rr) * 65 + o + ii], xv[ii], s);
+                            s = fmaf(-a32[(o + rr) * kF32Pitch + o + ii], xv[ii], s);
                         xv[rr] = (rr < jc) ? 0.f : s;
-                        t32[(o + rr) * 65 + o + jc] = xv[rr];
+                        t32[(o + rr) * kF32Pitch + o + jc] = xv[rr];
                     }
                 }
                 __syncthreads();
-                for (int I = 1; I < 4; ++I) {
-                    const int ncol = 16 * I;
-                    // M[ii][col] = sum_{kk < 16 I} A[16 I + ii][kk] T[kk][col]
-                    for (int e = tid; e < 16 * ncol; e += kThreads) {
-                        const int ii = e / ncol, col = e % ncol;
-                        float s = 0.f;
-                        for (int kk = (col >> 4) << 4; kk < ncol; ++kk)
-                            s = fmaf(a32[(16 * I + ii) * 65 + kk], t32[kk * 65 + col], s);
-                        msc[ii * 48 + col] = s;
+                PHASE_MARK(14);
+                // off-diagonal blocks: chain w on warp w (w < 6), 16x16 products on the warp
+                // tensor-core path (3xTF32, fp32 accuracy):  T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ.
+                // Partial sums Y_IJ are parked in the unused upper block (J, I) of t32.
+                auto Ab = [&](int I, int J) { return a32 + 16 * I * kF32Pitch + 16 * J; };
+                auto Tb = [&](int I, int J) { return t32 + 16 * I * kF32Pitch + 16 * J; };
+                float acc[2][4] = {};
+                // step 1: Y_10, Y_21, Y_32 -> T_10, T_21, T_32; partials Y_20, Y_31, Y_30
+                if (warp < 6) {
+                    const int Ii = (warp < 3) ? warp + 1 : (warp == 5 ? 3 : warp - 1);
+                    const int Jj = (warp < 3) ? warp : (warp == 5 ? 0 : warp - 3);
+                    warpmma::mm16_acc(Ab(Ii, Jj), kF32Pitch, Tb(Jj, Jj), kF32Pitch, acc);
+                    if (warp < 3) {
+                        warpmma::store16(Tb(Jj, Ii), kF32Pitch, acc, 1.f);
+                        __syncwarp();
+                        float acc2[2][4] = {};
+                        warpmma::mm16_acc(Tb(Ii, Ii), kF32Pitch, Tb(Jj, Ii), kF32Pitch, acc2);
+                        warpmma::store16(Tb(Ii, Jj), kF32Pitch, acc2, -1.f);
                     }
-                    __syncthreads();
-                    // T[16 I + ii][col] = - sum_{jj <= ii} T_II[ii][jj] M[jj][col]
-                    for (int e = tid; e < 16 * ncol; e += kThreads) {
-                        const int ii = e / ncol, col = e % ncol;
-                        float s = 0.f;
-                        for (int jj = 0; jj <= ii; ++jj)
-                            s = fmaf(t32[(16 * I + ii) * 65 + 16 * I + jj], msc[jj * 48 + col], s);
-                        t32[(16 * I + ii) * 65 + col] = -s;
-                    }
-                    __syncthreads();
                 }
+                __syncthreads();
+                PHASE_MARK(15);
+                // step 2: Y_20 += A_21 T_10 -> T_20;  Y_31 += A_32 T_21 -> T_31;  Y_30 += A_31 T_10
+                if (warp == 3 || warp == 4) {
+                    const int Ii = warp - 1, Jj = warp - 3;      // (2, 0) or (3, 1)
+                    warpmma::mm16_acc(Ab(Ii, Ii - 1), kF32Pitch, Tb(Ii - 1, Jj), kF32Pitch, acc);
+                    warpmma::store16(Tb(Jj, Ii), kF32Pitch, acc, 1.f);
+                    __syncwarp();
+                    float acc2[2][4] = {};
+                    warpmma::mm16_acc(Tb(Ii, Ii), kF32Pitch, Tb(Jj, Ii), kF32Pitch, acc2);
+                    warpmma::store16(Tb(Ii, Jj), kF32Pitch, acc2, -1.f);
+                } else if (warp == 5) {
+                    warpmma::mm16_acc(Ab(3, 1), kF32Pitch, Tb(1, 0), kF32Pitch, acc);
+                }
+                __syncthreads();
+                PHASE_MARK(16);
+                // step 3: Y_30 += A_32 T_20 -> T_30
+                if (warp == 5) {
+                    warpmma::mm16_acc(Ab(3, 2), kF32Pitch, Tb(2, 0), kF32Pitch, acc);
+                    warpmma::store16(Tb(0, 3), kF32Pitch, acc, 1.f);
+                    __syncwarp();
+                    float acc2[2][4] = {};
+                    warpmma::mm16_acc(Tb(3, 3), kF32Pitch, Tb(0, 3), kF32Pitch, acc2);
+                    warpmma::store16(Tb(3, 0), kF32Pitch, acc2, -1.f);
+                }
+                __syncthreads();
+                PHASE_MARK(17);
                 // T -> fp16 K-major tile (zeros above the diagonal blocks)
                 for (int e = tid; e < 64 * 8; e += kThreads) {
                     const int r = e >> 3, ch = e & 7;
-                    uint32_t w[4];
-#pragma unroll
-                    for (int q2 = 0; q2 < 4; ++q2) {
-                        const int i = ch * 8 + 2 * q2;
-                        const bool live = (i >> 4) <= (r >> 4);
-                        w[q2] = pack_f16(live ? t32[r * 65 + i] : 0.f, live ? t32[r * 65 + i + 1] : 0.f);
-                    }
-                    st_v4(sm, T16 + sw128_chunk_off(r, ch, 64), w[0], w[1], w[2], w[3]);
+                    const bool live = (ch >> 1) <= (r >> 4);
+                    const float4 lo4 = *reinterpret_cast<const float4*>(t32 + r * kF32Pitch + ch * 8);
+                    const float4 hi4 = *reinterpret_cast<const float4*>(t32 + r * kF32Pitch + ch * 8 + 4);
+                    st_v4(sm, T16 + sw128_chunk_off(r, ch, 64),
+                          live ? pack_f16(lo4.x, lo4.y) : 0u, live ? pack_f16(lo4.z, lo4.w) : 0u,
+                          live ? pack_f16(hi4.x, hi4.y) : 0u, live ? pack_f16(hi4.z, hi4.w) : 0u);
                 }
             }
             fence_proxy_async();
             fence_before_sync();
             __syncthreads();
+            PHASE_MARK(5);
 
             // ================= phase 5: W and U~^T MMAs =================
             if (tid == 0) {
@@ -546,22 +669,24 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (wait_or_abort(bar_mma, mma_parity, sAbort)) { aborted = true; break; }
             mma_parity ^= 1u;
             fence_after_sync();
+            PHASE_MARK(6);
 
             // ================= phase 6: W -> fp16 smem =================
             {
                 // M = 64 accumulator: row r lives in lane (r % 16) of quarter r / 16
+                uint32_t v[4][16];
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const uint32_t col = half * 64 + cc * 16;
-                    uint32_t v[16];
-                    tmem_ld16(taddr(tbase, quarter, TM_W + col), v);
-                    tmem_wait_ld();
-                    if (lane < 16) {
-                        const int r = quarter * 16 + lane;
+                for (int cc = 0; cc < 4; ++cc) tmem_ld16(taddr(tbase, quarter, TM_W + half * 64 + cc * 16), v[cc]);
+                tmem_wait_ld();
+                if (lane < 16) {
+                    const int r = quarter * 16 + lane;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        const uint32_t col = half * 64 + cc * 16;
                         uint32_t w[8];
 #pragma unroll
                         for (int q2 = 0; q2 < 8; ++q2)
-                            w[q2] = pack_f16(__uint_as_float(v[2 * q2]), __uint_as_float(v[2 * q2 + 1]));
+                            w[q2] = pack_f16(__uint_as_float(v[cc][2 * q2]), __uint_as_float(v[cc][2 * q2 + 1]));
                         st_v4(sm, W16 + sw128_chunk_off(r, col / 8, 64), w[0], w[1], w[2], w[3]);
                         st_v4(sm, W16 + sw128_chunk_off(r, col / 8 + 1, 64), w[4], w[5], w[6], w[7]);
                     }
@@ -592,6 +717,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             fence_proxy_async();
             fence_before_sync();
             __syncthreads();
+            PHASE_MARK(7);
             if (tid == 0) {
                 fence_after_sync();
                 const uint32_t s16 = smem_u32(sm + S16), w16 = smem_u32(sm + W16), gq = smem_u32(sm + GQ);
@@ -607,20 +733,22 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (wait_or_abort(bar_mma, mma_parity, sAbort)) { aborted = true; break; }
             mma_parity ^= 1u;
             fence_after_sync();
+            PHASE_MARK(8);
 
             // ================= phase 8: U -> fp16, S and O MMAs =================
             {
                 const int v_row = c_row;   // lanes of U^T are value columns
+                uint32_t v[2][16];
+                tmem_ld16(taddr(tbase, quarter, TM_UT + half * 32), v[0]);
+                tmem_ld16(taddr(tbase, quarter, TM_UT + half * 32 + 16), v[1]);
+                tmem_wait_ld();
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const uint32_t r0 = half * 32 + cc * 16;
-                    uint32_t v[16];
-                    tmem_ld16(taddr(tbase, quarter, TM_UT + r0), v);
-                    tmem_wait_ld();
                     uint32_t w[8];
 #pragma unroll
                     for (int q2 = 0; q2 < 8; ++q2)
-                        w[q2] = pack_f16(__uint_as_float(v[2 * q2]), __uint_as_float(v[2 * q2 + 1]));
+                        w[q2] = pack_f16(__uint_as_float(v[cc][2 * q2]), __uint_as_float(v[cc][2 * q2 + 1]));
                     st_v4(sm, U16 + sw128_chunk_off(v_row, r0 / 8, 128), w[0], w[1], w[2], w[3]);
                     st_v4(sm, U16 + sw128_chunk_off(v_row, r0 / 8 + 1, 128), w[4], w[5], w[6], w[7]);
                 }
@@ -628,6 +756,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             fence_proxy_async();
             fence_before_sync();
             __syncthreads();
+            PHASE_MARK(9);
             if (tid == 0) {
                 fence_after_sync();
                 const uint32_t kh = smem_u32(sm + KH), u16 = smem_u32(sm + U16), p16 = smem_u32(sm + P16);
@@ -642,27 +771,36 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (wait_or_abort(bar_mma, mma_parity, sAbort)) { aborted = true; break; }
             mma_parity ^= 1u;
             fence_after_sync();
+            PHASE_MARK(10);
 
-            // ================= phase 9: O -> out =================
+            // ================= phase 9: O -> out (through an smem tile, coalesced) =================
             {
                 const int v_col = c_row;
+                uint32_t v[2][16];
+                tmem_ld16(taddr(tbase, quarter, TM_OT + half * 32), v[0]);
+                tmem_ld16(taddr(tbase, quarter, TM_OT + half * 32 + 16), v[1]);
+                tmem_wait_ld();
+                __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + OST);
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int r0 = half * 32 + cc * 16;
-                    uint32_t v[16];
-                    tmem_ld16(taddr(tbase, quarter, TM_OT + r0), v);
-                    tmem_wait_ld();
+                for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const int r = r0 + jj;
-                        if (r < L)
-                            p.out[((t0 + r) * H + h) * kHeadDim + v_col] =
-                                __float2bfloat16_rn(p.scale * __uint_as_float(v[jj]));
-                    }
-                }
+                    for (int jj = 0; jj < 16; ++jj)
+                        ost[(half * 32 + cc * 16 + jj) * kHeadDim + v_col] =
+                            __float2bfloat16_rn(p.scale * __uint_as_float(v[cc][jj]));
             }
             fence_before_sync();
             __syncthreads();
+            {
+                const uint4* src = reinterpret_cast<const uint4*>(sm + OST);
+#pragma unroll
+                for (int e = tid; e < kChunk * 16; e += kThreads) {
+                    const int r = e >> 4, c = e & 15;
+                    if (r < L)
+                        *reinterpret_cast<uint4*>(p.out + ((t0 + r) * H + h) * kHeadDim + c * 8) = src[e];
+                }
+            }
+            __syncthreads();
+            PHASE_MARK(11);
         }
         if (aborted) break;
         // final state
@@ -672,6 +810,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 uint32_t r[16];
                 tmem_ld16(taddr(tbase, quarter, TM_S + v0), r);
                 tmem_wait_ld();
+#pragma unroll
                 for (int jj = 0; jj < 16; jj += 4)
                     *reinterpret_cast<float4*>(p.final_state + state_off + c_row * kHeadDim + v0 + jj) =
                         make_float4(__uint_as_float(r[jj]), __uint_as_float(r[jj + 1]),
@@ -693,6 +832,10 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     fence_after_sync();
     if (warp == 0) tmem_dealloc(tbase, TM_COLS);
+#ifdef KDA_PHASE_CLOCKS
+    if (tid == 0)
+        for (int i = 0; i < kPhases; ++i) atomicAdd(&g_phase_cycles[i], ph_acc[i]);
+#endif
 }
 
 // ---- host side ----
@@ -723,6 +866,17 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t
 }
 
 }  // namespace fused
+
+#ifdef KDA_PHASE_CLOCKS
+// Debug builds only: copies and clears the per-phase cycle totals.
+extern "C" int kda_debug_phase_cycles(unsigned long long* out) {
+    if (cudaMemcpyFromSymbol(out, fused::g_phase_cycles, sizeof(unsigned long long) * fused::kPhases) !=
+        cudaSuccess)
+        return -1;
+    unsigned long long zero[fused::kPhases] = {};
+    return cudaMemcpyToSymbol(fused::g_phase_cycles, zero, sizeof zero) == cudaSuccess ? fused::kPhases : -1;
+}
+#endif
 
 bool fused_supported(float lower_bound) { return lower_bound >= KDA_FUSED_MIN_LOWER_BOUND; }
 
