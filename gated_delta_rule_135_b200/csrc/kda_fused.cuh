@@ -370,6 +370,10 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
             // ================= phase 1: gate + operands =================
             PHASE_MARK(0);
+            // the chunk after this one (its global reads overlap the input wait)
+            int k1 = 0, h1 = 0;
+            int64_t t1 = 0;
+            const bool has_next = next_chunk(p, sOrder, b, G, units, k, j, nch, &k1, &h1, &t1);
             if (tid < kChunk) sBeta[tid] = tid < L ? beta_next : 0.f;
             if (wait_or_abort(bar_in, in_parity, sAbort)) { aborted = true; break; }
             PHASE_MARK(1);
@@ -428,16 +432,27 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const uint32_t* qin = reinterpret_cast<const uint32_t*>(sm + IN_Q);
                 const uint32_t* vin = reinterpret_cast<const uint32_t*>(sm + IN_V);
                 float pd[16];
+                // all loads of the block first: the stores below cannot be ordered
+                // before them by the compiler (one shared-memory base for both)
+                uint32_t kwv[16], qwv[16], vwv[16];
+                float bev[16];
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) {
                     const int r = blk * 16 + rr;
                     const bool ok = r < L;
                     const int idx = (r * kHeadDim + c0) >> 1;
-                    const uint32_t kw = ok ? kin[idx] : 0u, qw = ok ? qin[idx] : 0u, vw = ok ? vin[idx] : 0u;
+                    kwv[rr] = ok ? kin[idx] : 0u;
+                    qwv[rr] = ok ? qin[idx] : 0u;
+                    vwv[rr] = ok ? vin[idx] : 0u;
+                    bev[rr] = sBeta[r];
+                }
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    const uint32_t kw = kwv[rr], qw = qwv[rr], vw = vwv[rr];
                     const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
                     const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
                     const float v0 = __uint_as_float(vw << 16), v1 = __uint_as_float(vw & 0xFFFF0000u);
-                    const float be = sBeta[r];
+                    const float be = bev[rr];
                     const float R0 = fast_ex2(G0[rr]), R1 = fast_ex2(G1[rr]);            // e^{Gamma_r - Gamma_s}
                     const float E0 = fast_ex2(tb0 - G0[rr]), E1 = fast_ex2(tb1 - G1[rr]);  // e^{Gamma_e - Gamma_r}
                     const float kE0 = k0 * E0, kE1 = k1 * E1;
@@ -500,9 +515,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
             // inputs consumed: prefetch the next chunk; issue the A/P MMA
             {
-                int k1, h1;
-                int64_t t1;
-                in_flight = next_chunk(p, sOrder, b, G, units, k, j, nch, &k1, &h1, &t1);
+                in_flight = has_next;
                 if (tid == 0) {
                     if (in_flight) issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
                     fence_after_sync();
@@ -522,47 +535,57 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             PHASE_MARK(3);
 
             // ================= phase 3: A / P read-out =================
-            if (warp < 4) {
+            {
+                // quarter q holds rows 32 (q & 1) .. + 31 of A (q < 2) or P (q >= 2); warps 0-3
+                // assemble column blocks J = 0, 1 of their rows, warps 4-7 blocks J = 2, 3
                 const bool isA = quarter < 2;
                 const int r = (quarter & 1) * 32 + lane;      // token row in the chunk
                 const int I = r >> 4;
-                float row[64];
-                auto pick = [&](int J, uint32_t col_a, uint32_t col_b, int I_a) {
-                    // block J of the row: from TMEM columns col_a (rows with I == I_a) or col_b
+                const int jb = half * 2;                        // first column block of this warp
+                float row[32];
+                auto pick = [&](int Jl, uint32_t col_a, uint32_t col_b, int I_a) {
                     uint32_t ta[16], tb2[16];
                     tmem_ld16(taddr(tbase, quarter, TM_AP + col_a), ta);
                     tmem_ld16(taddr(tbase, quarter, TM_AP + col_b), tb2);
                     tmem_wait_ld();
 #pragma unroll
                     for (int jj = 0; jj < 16; ++jj)
-                        row[J * 16 + jj] = __uint_as_float(I == I_a ? ta[jj] : tb2[jj]);
+                        row[Jl * 16 + jj] = __uint_as_float(I == I_a ? ta[jj] : tb2[jj]);
                 };
                 if ((quarter & 1) == 0) {        // I in {0, 1}
-                    pick(0, 0, 64, 0);           // I=0: d=0 cols 0-15; I=1: d=1 cols 64-79
-                    pick(1, 16, 16, 1);          // I=1: d=0 cols 16-31 (I=0: masked below)
+                    if (half == 0) {
+                        pick(0, 0, 64, 0);       // J=0: I=0 d=0 cols 0-15; I=1 d=1 cols 64-79
+                        pick(1, 16, 16, 1);      // J=1: I=1 d=0 cols 16-31 (I=0: masked below)
+                    } else {
 #pragma unroll
-                    for (int jj = 32; jj < 64; ++jj) row[jj] = 0.f;
+                        for (int jj = 0; jj < 32; ++jj) row[jj] = 0.f;
+                    }
                 } else {                         // I in {2, 3}
-                    pick(0, 112, 144, 2);        // I=2: d=2 cols 112-127; I=3: d=3 cols 144-159
-                    pick(1, 80, 128, 2);         // I=2: d=1 cols 80-95;   I=3: d=2 cols 128-143
-                    pick(2, 32, 96, 2);          // I=2: d=0 cols 32-47;   I=3: d=1 cols 96-111
-                    pick(3, 48, 48, 3);          // I=3: d=0 cols 48-63 (I=2: masked below)
+                    if (half == 0) {
+                        pick(0, 112, 144, 2);    // J=0: I=2 d=2 cols 112-127; I=3 d=3 cols 144-159
+                        pick(1, 80, 128, 2);     // J=1: I=2 d=1 cols 80-95;   I=3 d=2 cols 128-143
+                    } else {
+                        pick(0, 32, 96, 2);      // J=2: I=2 d=0 cols 32-47;   I=3 d=1 cols 96-111
+                        pick(1, 48, 48, 3);      // J=3: I=3 d=0 cols 48-63 (I=2: masked below)
+                    }
                 }
                 const float pdg = sPdiag[r] + sPdiag[64 + r];
 #pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    row[i] = i < r ? row[i] : ((i == r && !isA) ? pdg : 0.f);
+                for (int ii = 0; ii < 32; ++ii) {
+                    const int i = jb * 16 + ii;
+                    row[ii] = i < r ? row[ii] : ((i == r && !isA) ? pdg : 0.f);
+                }
                 if (isA) {
                     const float be = sBeta[r];
-                    float* a32 = reinterpret_cast<float*>(sm + A32) + r * kF32Pitch;
+                    float* a32 = reinterpret_cast<float*>(sm + A32) + r * kF32Pitch + jb * 16;
 #pragma unroll
-                    for (int i = 0; i < 64; i += 4)
+                    for (int i = 0; i < 32; i += 4)
                         *reinterpret_cast<float4*>(a32 + i) =
                             make_float4(be * row[i], be * row[i + 1], be * row[i + 2], be * row[i + 3]);
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        st_v4(sm, P16 + sw128_chunk_off(r, c, 64), pack_f16(row[8 * c], row[8 * c + 1]),
+                    for (int c = 0; c < 4; ++c)
+                        st_v4(sm, P16 + sw128_chunk_off(r, jb * 2 + c, 64), pack_f16(row[8 * c], row[8 * c + 1]),
                               pack_f16(row[8 * c + 2], row[8 * c + 3]), pack_f16(row[8 * c + 4], row[8 * c + 5]),
                               pack_f16(row[8 * c + 6], row[8 * c + 7]));
                 }
@@ -575,76 +598,135 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             {
                 const float* a32 = reinterpret_cast<const float*>(sm + A32);
                 float* t32 = reinterpret_cast<float*>(sm + T32);
+                auto Ab = [&](int I, int J) { return a32 + 16 * I * kF32Pitch + 16 * J; };
+                auto Tb = [&](int I, int J) { return t32 + 16 * I * kF32Pitch + 16 * J; };
+                // one warp writes the fp16 copy of finished block (I, J): lane -> (row, 8-col chunk)
+                auto to_t16 = [&](int I, int J) {
+                    const int rr = lane >> 1, ch = lane & 1;
+                    const float* src = Tb(I, J) + rr * kF32Pitch + ch * 8;
+                    const float4 lo4 = *reinterpret_cast<const float4*>(src);
+                    const float4 hi4 = *reinterpret_cast<const float4*>(src + 4);
+                    st_v4(sm, T16 + sw128_chunk_off(16 * I + rr, 2 * J + ch, 64), pack_f16(lo4.x, lo4.y),
+                          pack_f16(lo4.z, lo4.w), pack_f16(hi4.x, hi4.y), pack_f16(hi4.z, hi4.w));
+                };
                 if (tid < 64) {   // diagonal 16 x 16 blocks by forward substitution, one column each
                     const int bI = tid >> 4, jc = tid & 15, o = bI * 16;
                     float xv[16];
 #pragma unroll
                     for (int rr = 0; rr < 16; ++rr) {
-                        float s = (rr == jc) ? 1.f : 0.f;
+                        float s0 = (rr == jc) ? 1.f : 0.f;
 #pragma unroll
                         for (int ii = 0; ii < rr; ++ii)
-                            s = fmaf(-a32[(o + rr) * kF32Pitch + o + ii], xv[ii], s);
-                        xv[rr] = (rr < jc) ? 0.f : s;
-                        t32[(o + rr) * kF32Pitch + o + jc] = xv[rr];
+                            s0 = fmaf(-a32[(o + rr) * kF32Pitch + o + ii], xv[ii], s0);
+                        xv[rr] = (rr < jc) ? 0.f : s0;
+                    }
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) t32[(o + rr) * kF32Pitch + o + jc] = xv[rr];
+                } else if (tid >= 128) {
+                    // zero fp16 blocks above the diagonal: 6 blocks x 32 chunks over 128 threads
+                    for (int e = tid - 128; e < 6 * 32; e += 128) {
+                        const int blkid = e >> 5, c = e & 31;
+                        const int I = blkid < 3 ? 0 : (blkid < 5 ? 1 : 2);
+                        const int J = blkid < 3 ? blkid + 1 : (blkid < 5 ? blkid - 1 : 3);
+                        st_v4(sm, T16 + sw128_chunk_off(16 * I + (c >> 1), 2 * J + (c & 1), 64), 0u, 0u, 0u, 0u);
                     }
                 }
                 __syncthreads();
                 PHASE_MARK(14);
-                // off-diagonal blocks: chain w on warp w (w < 6), 16x16 products on the warp
-                // tensor-core path (3xTF32, fp32 accuracy):  T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ.
-                // Partial sums Y_IJ are parked in the unused upper block (J, I) of t32.
-                auto Ab = [&](int I, int J) { return a32 + 16 * I * kF32Pitch + 16 * J; };
-                auto Tb = [&](int I, int J) { return t32 + 16 * I * kF32Pitch + 16 * J; };
+                // Off-diagonal blocks by recursive doubling on 16 x 16 blocks; products on the
+                // warp tensor-core path (3xTF32, fp32 accuracy).  Intermediates are parked in
+                // the unused upper blocks of t32.
+                //   T10 = -T11 A10 T00, T32 = -T33 A32 T22, T21 = -T22 A21 T11,
+                //   X20 = A20 T00 + A21 T10, X30 = A30 T00 + A31 T10,
+                //   T20 = -T22 X20, T31 = -(T32 A21 T11 + T33 A31 T11), T30 = -(T32 X20 + T33 X30).
                 float acc[2][4] = {};
-                // step 1: Y_10, Y_21, Y_32 -> T_10, T_21, T_32; partials Y_20, Y_31, Y_30
-                if (warp < 6) {
-                    const int Ii = (warp < 3) ? warp + 1 : (warp == 5 ? 3 : warp - 1);
-                    const int Jj = (warp < 3) ? warp : (warp == 5 ? 0 : warp - 3);
+                // step A: T10, T32 (two products each); X21 = A21 T11, X31 = A31 T11;
+                //         partial X20 = A20 T00, X30 = A30 T00; fp16 copies of the diagonal blocks
+                if (warp == 0 || warp == 1) {
+                    const int Ii = warp == 0 ? 1 : 3, Jj = Ii - 1;
                     warpmma::mm16_acc(Ab(Ii, Jj), kF32Pitch, Tb(Jj, Jj), kF32Pitch, acc);
-                    if (warp < 3) {
-                        warpmma::store16(Tb(Jj, Ii), kF32Pitch, acc, 1.f);
-                        __syncwarp();
-                        float acc2[2][4] = {};
-                        warpmma::mm16_acc(Tb(Ii, Ii), kF32Pitch, Tb(Jj, Ii), kF32Pitch, acc2);
-                        warpmma::store16(Tb(Ii, Jj), kF32Pitch, acc2, -1.f);
-                    }
-                }
-                __syncthreads();
-                PHASE_MARK(15);
-                // step 2: Y_20 += A_21 T_10 -> T_20;  Y_31 += A_32 T_21 -> T_31;  Y_30 += A_31 T_10
-                if (warp == 3 || warp == 4) {
-                    const int Ii = warp - 1, Jj = warp - 3;      // (2, 0) or (3, 1)
-                    warpmma::mm16_acc(Ab(Ii, Ii - 1), kF32Pitch, Tb(Ii - 1, Jj), kF32Pitch, acc);
                     warpmma::store16(Tb(Jj, Ii), kF32Pitch, acc, 1.f);
                     __syncwarp();
                     float acc2[2][4] = {};
                     warpmma::mm16_acc(Tb(Ii, Ii), kF32Pitch, Tb(Jj, Ii), kF32Pitch, acc2);
                     warpmma::store16(Tb(Ii, Jj), kF32Pitch, acc2, -1.f);
-                } else if (warp == 5) {
-                    warpmma::mm16_acc(Ab(3, 1), kF32Pitch, Tb(1, 0), kF32Pitch, acc);
+                    __syncwarp();
+                    to_t16(Ii, Jj);
+                } else if (warp == 2) {
+                    warpmma::mm16_acc(Ab(2, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc);
+                    warpmma::store16(Tb(1, 2), kF32Pitch, acc, 1.f);           // X21
+                    float acc2[2][4] = {};
+                    warpmma::mm16_acc(Ab(3, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc2);
+                    warpmma::store16(Tb(1, 3), kF32Pitch, acc2, 1.f);          // X31
+                } else if (warp == 3) {
+                    warpmma::mm16_acc(Ab(2, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);   // X20 partial
+                } else if (warp == 4) {
+                    warpmma::mm16_acc(Ab(3, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);   // X30 partial
+                } else {
+                    for (int d = warp - 5; d < 4; d += 3) to_t16(d, d);               // diagonal blocks
+                }
+                __syncthreads();
+                PHASE_MARK(15);
+                // step B: X20, X30 complete; T21 = -T22 X21; P31a = T32 X21, P31b = T33 X31
+                if (warp == 3 || warp == 4) {
+                    warpmma::mm16_acc(Ab(warp - 1, 1), kF32Pitch, Tb(1, 0), kF32Pitch, acc);
+                    warpmma::store16(Tb(0, warp - 1), kF32Pitch, acc, 1.f);   // X20 -> (0,2), X30 -> (0,3)
+                } else if (warp == 0) {
+                    float a2[2][4] = {};
+                    warpmma::mm16_acc(Tb(2, 2), kF32Pitch, Tb(1, 2), kF32Pitch, a2);
+                    warpmma::store16(Tb(2, 1), kF32Pitch, a2, -1.f);           // T21
+                    __syncwarp();
+                    to_t16(2, 1);
+                } else if (warp == 1) {
+                    float a2[2][4] = {};
+                    warpmma::mm16_acc(Tb(3, 2), kF32Pitch, Tb(1, 2), kF32Pitch, a2);
+                    warpmma::store16(Tb(0, 1), kF32Pitch, a2, 1.f);            // P31a -> (0,1)
+                } else if (warp == 2) {
+                    float a2[2][4] = {};
+                    warpmma::mm16_acc(Tb(3, 3), kF32Pitch, Tb(1, 3), kF32Pitch, a2);
+                    warpmma::store16(Tb(2, 3), kF32Pitch, a2, 1.f);            // P31b -> (2,3)
                 }
                 __syncthreads();
                 PHASE_MARK(16);
-                // step 3: Y_30 += A_32 T_20 -> T_30
-                if (warp == 5) {
-                    warpmma::mm16_acc(Ab(3, 2), kF32Pitch, Tb(2, 0), kF32Pitch, acc);
-                    warpmma::store16(Tb(0, 3), kF32Pitch, acc, 1.f);
+                // step C: T20 = -T22 X20; P30a = T32 X20, P30b = T33 X30; T31 = -(P31a + P31b)
+                if (warp == 0) {
+                    float a2[2][4] = {};
+                    warpmma::mm16_acc(Tb(2, 2), kF32Pitch, Tb(0, 2), kF32Pitch, a2);
+                    warpmma::store16(Tb(2, 0), kF32Pitch, a2, -1.f);           // T20
                     __syncwarp();
-                    float acc2[2][4] = {};
-                    warpmma::mm16_acc(Tb(3, 3), kF32Pitch, Tb(0, 3), kF32Pitch, acc2);
-                    warpmma::store16(Tb(3, 0), kF32Pitch, acc2, -1.f);
+                    to_t16(2, 0);
+                } else if (warp == 1) {
+                    float a2[2][4] = {};
+                    warpmma::mm16_acc(Tb(3, 2), kF32Pitch, Tb(0, 2), kF32Pitch, a2);
+                    warpmma::store16(Tb(1, 2), kF32Pitch, a2, 1.f);            // P30a -> (1,2)
+                } else if (warp == 2) {
+                    float a2[2][4] = {};
+                    warpmma::mm16_acc(Tb(3, 3), kF32Pitch, Tb(0, 3), kF32Pitch, a2);
+                    warpmma::store16(Tb(1, 3), kF32Pitch, a2, 1.f);            // P30b -> (1,3)
+                } else if (warp == 3) {
+                    for (int e = lane; e < 64; e += 32) {                      // T31 = -(P31a + P31b)
+                        const int rr = e >> 2, c4 = (e & 3) * 4;
+                        const float4 x1 = *reinterpret_cast<const float4*>(Tb(0, 1) + rr * kF32Pitch + c4);
+                        const float4 x2 = *reinterpret_cast<const float4*>(Tb(2, 3) + rr * kF32Pitch + c4);
+                        *reinterpret_cast<float4*>(Tb(3, 1) + rr * kF32Pitch + c4) =
+                            make_float4(-(x1.x + x2.x), -(x1.y + x2.y), -(x1.z + x2.z), -(x1.w + x2.w));
+                    }
+                    __syncwarp();
+                    to_t16(3, 1);
                 }
                 __syncthreads();
                 PHASE_MARK(17);
-                // T -> fp16 K-major tile (zeros above the diagonal blocks)
-                for (int e = tid; e < 64 * 8; e += kThreads) {
-                    const int r = e >> 3, ch = e & 7;
-                    const bool live = (ch >> 1) <= (r >> 4);
-                    const float4 lo4 = *reinterpret_cast<const float4*>(t32 + r * kF32Pitch + ch * 8);
-                    const float4 hi4 = *reinterpret_cast<const float4*>(t32 + r * kF32Pitch + ch * 8 + 4);
-                    st_v4(sm, T16 + sw128_chunk_off(r, ch, 64),
-                          live ? pack_f16(lo4.x, lo4.y) : 0u, live ? pack_f16(lo4.z, lo4.w) : 0u,
-                          live ? pack_f16(hi4.x, hi4.y) : 0u, live ? pack_f16(hi4.z, hi4.w) : 0u);
+                // step D: T30 = -(P30a + P30b)
+                if (warp == 0) {
+                    for (int e = lane; e < 64; e += 32) {
+                        const int rr = e >> 2, c4 = (e & 3) * 4;
+                        const float4 x1 = *reinterpret_cast<const float4*>(Tb(1, 2) + rr * kF32Pitch + c4);
+                        const float4 x2 = *reinterpret_cast<const float4*>(Tb(1, 3) + rr * kF32Pitch + c4);
+                        *reinterpret_cast<float4*>(Tb(3, 0) + rr * kF32Pitch + c4) =
+                            make_float4(-(x1.x + x2.x), -(x1.y + x2.y), -(x1.z + x2.z), -(x1.w + x2.w));
+                    }
+                    __syncwarp();
+                    to_t16(3, 0);
                 }
             }
             fence_proxy_async();
