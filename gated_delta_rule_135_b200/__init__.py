@@ -26,7 +26,7 @@ FUSED_MIN_LOWER_BOUND = -5.3
 KDA_OK = 0
 STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
                 3: "KDA_ERR_ALIGNMENT", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_DEVICE",
-                6: "KDA_ERR_WORKSPACE"}
+                6: "KDA_ERR_WORKSPACE", 7: "KDA_ERR_SCRATCH_LIMIT"}
 
 
 class KdaError(RuntimeError):
@@ -70,6 +70,10 @@ def _load():
     lib.kda_last_device_error_bits.argtypes = []
     lib.kda_version.restype = ctypes.c_char_p
     lib.kda_version.argtypes = []
+    lib.kda_fwd_staged_noalloc.restype = ctypes.c_int
+    lib.kda_fwd_staged_noalloc.argtypes = fwd_args + [vp]
+    lib.kda_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.kda_noalloc_scratch_bytes.argtypes = []
     return lib
 
 
@@ -78,7 +82,8 @@ _lib = _load()
 # Symbols include/kda.h declares (checked by the ABI test).
 EXPORTED = ("kda_fwd", "kda_fwd_staged", "kda_staged_workspace_size",
             "kda_staged_workspace_layout", "kda_strerror", "kda_check_device_error",
-            "kda_last_device_error_bits", "kda_version")
+            "kda_last_device_error_bits", "kda_version", "kda_fwd_staged_noalloc",
+            "kda_noalloc_scratch_bytes")
 
 
 def lib() -> ctypes.CDLL:
@@ -213,6 +218,28 @@ def kda_fwd_staged(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, scale: 
     if st != KDA_OK:
         raise KdaError(st, "kda_fwd_staged")
     return out, final_state, workspace
+
+
+def kda_fwd_staged_noalloc(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, scale: float,
+                           initial_state=None, cu_seqlens=None, out=None, final_state=None, *,
+                           batch: int = 1, stream=None):
+    """Calls kda_fwd_staged_noalloc: the staged forward on the library's fixed
+    16 MiB device scratch (no device allocation; small problems only)."""
+    dims = _marshal(q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens, out,
+                    final_state, batch)
+    if out is None:
+        out = torch.empty(q.shape[:-1] + (HEAD_DIM,), dtype=torch.bfloat16, device=q.device)
+    st = _lib.kda_fwd_staged_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log),
+                                     _ptr(dt_bias), float(lower_bound), float(scale),
+                                     _ptr(initial_state), _ptr(cu_seqlens), _ptr(out),
+                                     _ptr(final_state), dims, _stream_ptr(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_fwd_staged_noalloc")
+    return out, final_state
+
+
+def kda_noalloc_scratch_bytes() -> int:
+    return int(_lib.kda_noalloc_scratch_bytes())
 
 
 def kda_check_device_error(stream=None) -> int:

@@ -6,6 +6,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -93,7 +95,68 @@ kda_status copy_states_only(const StagedArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// kda_fwd_staged_noalloc: the staged forward on a library-owned scratch buffer.
+//
+// For callers that cannot allocate device memory: code whose device memory is
+// entirely owned by another allocator (a framework's caching allocator or a
+// pre-reserved arena, so that cudaMalloc fails or would fragment it) and code
+// on latency-critical paths that must not enter the driver's allocator.  The
+// scratch is a fixed array in device global memory that exists on every GPU
+// that loads this library, from load until process exit.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch on the current device, resolved once per
+// device (host code may not use the array's name as a device address).
+cudaError_t noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        err = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (err != cudaSuccess) return err;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
 extern "C" {
+
+size_t kda_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+kda_status kda_fwd_staged_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                  const float* beta, const float* A_log, const float* dt_bias,
+                                  float lower_bound, float scale, const float* initial_state,
+                                  const int32_t* cu_seqlens, void* out, float* final_state,
+                                  kda_dims dims, kda_stream_t stream) {
+    StagedArgs a{};
+    kda_status st = prepare(q, k, v, g, beta, A_log, dt_bias, lower_bound, scale, initial_state,
+                            cu_seqlens, out, final_state, dims, &a);
+    if (st != KDA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (a.total_tokens == 0) return copy_states_only(a, s);
+    const kda::StagedLayout L = kda::staged_layout(a.total_tokens, a.H, a.N);
+    if (L.total > kNoAllocScratchBytes) return KDA_ERR_SCRATCH_LIMIT;
+    void* ws = nullptr;
+    if (noalloc_scratch(&ws) != cudaSuccess) return KDA_ERR_CUDA;
+    // Every byte the staged kernels read is written earlier in the same call
+    // (chunk table, Gamma, W, U~, P, U, chunk states), so nothing is cleared.
+    return kda::launch_staged(a, static_cast<char*>(ws), L, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 
 kda_status kda_staged_workspace_layout(kda_dims dims, int varlen, kda_staged_layout* layout) {
     if (!layout) return KDA_ERR_INVALID_ARG;
@@ -169,6 +232,9 @@ const char* kda_strerror(kda_status status) {
         case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA call or kernel launch failed";
         case KDA_ERR_DEVICE: return "KDA_ERR_DEVICE: a kernel recorded a device-side error";
         case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
+        case KDA_ERR_SCRATCH_LIMIT:
+            return "KDA_ERR_SCRATCH_LIMIT: the problem needs more than the 16 MiB scratch of "
+                   "kda_fwd_staged_noalloc (use kda_fwd_staged with a workspace)";
     }
     return "KDA_ERR_UNKNOWN";
 }

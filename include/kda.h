@@ -60,7 +60,8 @@ typedef enum {
     KDA_ERR_ALIGNMENT = 3,     /* a base address not 16-byte aligned */
     KDA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
     KDA_ERR_DEVICE = 5,        /* a kernel recorded a device-side error (see kda_check_device_error) */
-    KDA_ERR_WORKSPACE = 6      /* workspace missing or smaller than required */
+    KDA_ERR_WORKSPACE = 6,     /* workspace missing or smaller than required */
+    KDA_ERR_SCRATCH_LIMIT = 7  /* kda_fwd_staged_noalloc: problem exceeds its fixed scratch */
 } kda_status;
 
 typedef struct {
@@ -140,6 +141,41 @@ kda_status kda_fwd_staged(const void* q, const void* k, const void* v,
                           void* out, float* final_state,
                           kda_dims dims, void* workspace, size_t workspace_bytes,
                           kda_stream_t stream);
+
+/*
+ * kda_fwd_staged_noalloc -- the staged forward (same kernels and results as
+ * kda_fwd_staged) without any device allocation.  No page describes this entry
+ * point; it exists for callers that cannot allocate device memory: callers
+ * whose device memory is entirely owned by another allocator (a framework's
+ * caching allocator, a pre-reserved arena), where cudaMalloc would fail or
+ * fragment that pool, and latency-critical callers that must not enter the
+ * driver's allocator.
+ *
+ * Scratch: a fixed 16 MiB array in device global memory (see
+ * kda_noalloc_scratch_bytes), present on every GPU that loads the library
+ * until the process exits.  The call neither allocates nor frees anything.
+ * Limit: problems whose staged workspace (kda_staged_workspace_size) exceeds
+ * the scratch are rejected with KDA_ERR_SCRATCH_LIMIT before any launch
+ * (roughly T * H <= 4500 tokens x heads at N = 1).
+ * Set-up: the first call on each device resolves the scratch's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before capturing a stream.
+ * Sharing: all calls share the one scratch, which keeps the last call's
+ * contents (nothing in it needs to start at zero).  Calls that overlap on the
+ * GPU -- on different streams or from different host threads -- race on it;
+ * serialise them.
+ * Arguments, layouts and other errors are those of kda_fwd.
+ */
+kda_status kda_fwd_staged_noalloc(const void* q, const void* k, const void* v,
+                                  const float* g, const float* beta,
+                                  const float* A_log, const float* dt_bias,
+                                  float lower_bound, float scale,
+                                  const float* initial_state, const int32_t* cu_seqlens,
+                                  void* out, float* final_state,
+                                  kda_dims dims, kda_stream_t stream);
+
+/* Size in bytes of the scratch kda_fwd_staged_noalloc uses (16 MiB). */
+size_t kda_noalloc_scratch_bytes(void);
 
 /* Human-readable name of a status code (static storage; never NULL). */
 const char* kda_strerror(kda_status status);
