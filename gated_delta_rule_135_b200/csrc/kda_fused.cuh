@@ -364,6 +364,10 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float db2_1 = p.dt_bias[h * kHeadDim + c0 + 1] * kLog2e;
 
         const int64_t nch = (x.eos - x.bos + kChunk - 1) / kChunk;
+        // chunk 0 of the next non-empty unit of this CTA (global reads once per unit)
+        int kn = 0, hn = 0;
+        int64_t tn = 0;
+        const bool unit_has_next = next_chunk(p, sOrder, b, G, units, k, nch - 1, nch, &kn, &hn, &tn);
         for (int64_t j = 0; j < nch; ++j) {
             const int64_t t0 = x.bos + j * kChunk;
             const int L = (int)(x.eos - t0 < kChunk ? x.eos - t0 : kChunk);
@@ -371,9 +375,10 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // ================= phase 1: gate + operands =================
             PHASE_MARK(0);
             // the chunk after this one (its global reads overlap the input wait)
-            int k1 = 0, h1 = 0;
-            int64_t t1 = 0;
-            const bool has_next = next_chunk(p, sOrder, b, G, units, k, j, nch, &k1, &h1, &t1);
+            const bool last = (j + 1 == nch);
+            const bool has_next = last ? unit_has_next : true;
+            const int h1 = last ? hn : h;
+            const int64_t t1 = last ? tn : t0 + kChunk;
             if (tid < kChunk) sBeta[tid] = tid < L ? beta_next : 0.f;
             if (wait_or_abort(bar_in, in_parity, sAbort)) { aborted = true; break; }
             PHASE_MARK(1);
@@ -446,13 +451,12 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     vwv[rr] = ok ? vin[idx] : 0u;
                     bev[rr] = sBeta[r];
                 }
+                // (a) operands of the A/P MMA, then issue it; (b) the other operand tiles while it runs
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) {
-                    const uint32_t kw = kwv[rr], qw = qwv[rr], vw = vwv[rr];
+                    const uint32_t kw = kwv[rr], qw = qwv[rr];
                     const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
                     const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
-                    const float v0 = __uint_as_float(vw << 16), v1 = __uint_as_float(vw & 0xFFFF0000u);
-                    const float be = bev[rr];
                     const float R0 = fast_ex2(G0[rr]), R1 = fast_ex2(G1[rr]);            // e^{Gamma_r - Gamma_s}
                     const float E0 = fast_ex2(tb0 - G0[rr]), E1 = fast_ex2(tb1 - G1[rr]);  // e^{Gamma_e - Gamma_r}
                     const float kE0 = k0 * E0, kE1 = k1 * E1;
@@ -463,13 +467,35 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (blk <= 2) st_u32(sm, AP_B + off160 + 64u * 128u + ro, pack_bf16(kE0, kE1));
                     if (blk <= 1) st_u32(sm, AP_B + off160 + 112u * 128u + ro, pack_bf16(kE0 * F2_0, kE1 * F2_1));
                     if (blk == 0) st_u32(sm, AP_B + off160 + 144u * 128u + ro, pack_bf16(kE0 * F3_0, kE1 * F3_1));
+                    pd[rr] = fmaf(q0, k0, q1 * k1);
+                }
+                fence_proxy_async();
+                __syncthreads();
+                if (tid == 0) {
+                    fence_after_sync();
+                    const uint32_t a0 = smem_u32(sm + AP_A), b0 = smem_u32(sm + AP_B);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
+                                ks > 0 ? 1u : 0u);
+                    mma_commit(bar_mma);
+                }
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    const uint32_t kw = kwv[rr], qw = qwv[rr], vw = vwv[rr];
+                    const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
+                    const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
+                    const float v0 = __uint_as_float(vw << 16), v1 = __uint_as_float(vw & 0xFFFF0000u);
+                    const float be = bev[rr];
+                    const float R0 = fast_ex2(G0[rr]), R1 = fast_ex2(G1[rr]);
+                    const float E0 = fast_ex2(tb0 - G0[rr]), E1 = fast_ex2(tb1 - G1[rr]);
+                    const float kE0 = k0 * E0, kE1 = k1 * E1;
+                    const uint32_t ro = (uint32_t)rr * 128u + ((chk ^ (uint32_t)(rr & 7)) << 4);
                     const float g0 = R0 * eTs0, g1 = R1 * eTs1;                          // gamma_r
-                    const float bk0 = be * k0 * g0, bk1 = be * k1 * g1;
                     st_u32(sm, GQ + off64 + ro, pack_f16(q0 * g0, q1 * g1));
-                    st_u32(sm, BGK + off64 + ro, pack_f16(bk0, bk1));
+                    st_u32(sm, BGK + off64 + ro, pack_f16(be * k0 * g0, be * k1 * g1));
                     st_u32(sm, KH + off64 + ro, pack_f16(kE0 * eA0, kE1 * eA1));
                     st_u32(sm, BV + off64 + ro, pack_f16(be * v0, be * v1));
-                    pd[rr] = fmaf(q0, k0, q1 * k1);
                 }
                 PHASE_MARK(13);
                 // reduce pd over the 32 lanes for all 16 tokens at once (transposing butterfly):
@@ -513,19 +539,10 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             __syncthreads();
             PHASE_MARK(2);
 
-            // inputs consumed: prefetch the next chunk; issue the A/P MMA
+            // inputs consumed: prefetch the next chunk (the A/P MMA is already running)
             {
                 in_flight = has_next;
-                if (tid == 0) {
-                    if (in_flight) issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
-                    fence_after_sync();
-                    const uint32_t a0 = smem_u32(sm + AP_A), b0 = smem_u32(sm + AP_B);
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
-                                ks > 0 ? 1u : 0u);
-                    mma_commit(bar_mma);
-                }
+                if (tid == 0 && in_flight) issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
                 if (in_flight && tid < kChunk && t1 + tid < p.total_tokens)
                     beta_next = p.beta[(t1 + tid) * H + h1];
             }
@@ -634,8 +651,9 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 __syncthreads();
                 PHASE_MARK(14);
                 // Off-diagonal blocks by recursive doubling on 16 x 16 blocks; products on the
-                // warp tensor-core path (3xTF32, fp32 accuracy).  Intermediates are parked in
-                // the unused upper blocks of t32.
+                // warp tensor-core path (mma.sync, fp16 operands, fp32 accumulation -- T is
+                // rounded to fp16 for the W / U~ MMAs in any case).  Intermediates are parked
+                // in the unused upper blocks of t32.
                 //   T10 = -T11 A10 T00, T32 = -T33 A32 T22, T21 = -T22 A21 T11,
                 //   X20 = A20 T00 + A21 T10, X30 = A30 T00 + A31 T10,
                 //   T20 = -T22 X20, T31 = -(T32 A21 T11 + T33 A31 T11), T30 = -(T32 X20 + T33 X30).
@@ -644,24 +662,24 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 //         partial X20 = A20 T00, X30 = A30 T00; fp16 copies of the diagonal blocks
                 if (warp == 0 || warp == 1) {
                     const int Ii = warp == 0 ? 1 : 3, Jj = Ii - 1;
-                    warpmma::mm16_acc(Ab(Ii, Jj), kF32Pitch, Tb(Jj, Jj), kF32Pitch, acc);
+                    warpmma::mm16_acc_h(Ab(Ii, Jj), kF32Pitch, Tb(Jj, Jj), kF32Pitch, acc);
                     warpmma::store16(Tb(Jj, Ii), kF32Pitch, acc, 1.f);
                     __syncwarp();
                     float acc2[2][4] = {};
-                    warpmma::mm16_acc(Tb(Ii, Ii), kF32Pitch, Tb(Jj, Ii), kF32Pitch, acc2);
+                    warpmma::mm16_acc_h(Tb(Ii, Ii), kF32Pitch, Tb(Jj, Ii), kF32Pitch, acc2);
                     warpmma::store16(Tb(Ii, Jj), kF32Pitch, acc2, -1.f);
                     __syncwarp();
                     to_t16(Ii, Jj);
                 } else if (warp == 2) {
-                    warpmma::mm16_acc(Ab(2, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc);
+                    warpmma::mm16_acc_h(Ab(2, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc);
                     warpmma::store16(Tb(1, 2), kF32Pitch, acc, 1.f);           // X21
                     float acc2[2][4] = {};
-                    warpmma::mm16_acc(Ab(3, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc2);
+                    warpmma::mm16_acc_h(Ab(3, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc2);
                     warpmma::store16(Tb(1, 3), kF32Pitch, acc2, 1.f);          // X31
                 } else if (warp == 3) {
-                    warpmma::mm16_acc(Ab(2, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);   // X20 partial
+                    warpmma::mm16_acc_h(Ab(2, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);   // X20 partial
                 } else if (warp == 4) {
-                    warpmma::mm16_acc(Ab(3, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);   // X30 partial
+                    warpmma::mm16_acc_h(Ab(3, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);   // X30 partial
                 } else {
                     for (int d = warp - 5; d < 4; d += 3) to_t16(d, d);               // diagonal blocks
                 }
@@ -669,21 +687,21 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 PHASE_MARK(15);
                 // step B: X20, X30 complete; T21 = -T22 X21; P31a = T32 X21, P31b = T33 X31
                 if (warp == 3 || warp == 4) {
-                    warpmma::mm16_acc(Ab(warp - 1, 1), kF32Pitch, Tb(1, 0), kF32Pitch, acc);
+                    warpmma::mm16_acc_h(Ab(warp - 1, 1), kF32Pitch, Tb(1, 0), kF32Pitch, acc);
                     warpmma::store16(Tb(0, warp - 1), kF32Pitch, acc, 1.f);   // X20 -> (0,2), X30 -> (0,3)
                 } else if (warp == 0) {
                     float a2[2][4] = {};
-                    warpmma::mm16_acc(Tb(2, 2), kF32Pitch, Tb(1, 2), kF32Pitch, a2);
+                    warpmma::mm16_acc_h(Tb(2, 2), kF32Pitch, Tb(1, 2), kF32Pitch, a2);
                     warpmma::store16(Tb(2, 1), kF32Pitch, a2, -1.f);           // T21
                     __syncwarp();
                     to_t16(2, 1);
                 } else if (warp == 1) {
                     float a2[2][4] = {};
-                    warpmma::mm16_acc(Tb(3, 2), kF32Pitch, Tb(1, 2), kF32Pitch, a2);
+                    warpmma::mm16_acc_h(Tb(3, 2), kF32Pitch, Tb(1, 2), kF32Pitch, a2);
                     warpmma::store16(Tb(0, 1), kF32Pitch, a2, 1.f);            // P31a -> (0,1)
                 } else if (warp == 2) {
                     float a2[2][4] = {};
-                    warpmma::mm16_acc(Tb(3, 3), kF32Pitch, Tb(1, 3), kF32Pitch, a2);
+                    warpmma::mm16_acc_h(Tb(3, 3), kF32Pitch, Tb(1, 3), kF32Pitch, a2);
                     warpmma::store16(Tb(2, 3), kF32Pitch, a2, 1.f);            // P31b -> (2,3)
                 }
                 __syncthreads();
@@ -691,17 +709,17 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // step C: T20 = -T22 X20; P30a = T32 X20, P30b = T33 X30; T31 = -(P31a + P31b)
                 if (warp == 0) {
                     float a2[2][4] = {};
-                    warpmma::mm16_acc(Tb(2, 2), kF32Pitch, Tb(0, 2), kF32Pitch, a2);
+                    warpmma::mm16_acc_h(Tb(2, 2), kF32Pitch, Tb(0, 2), kF32Pitch, a2);
                     warpmma::store16(Tb(2, 0), kF32Pitch, a2, -1.f);           // T20
                     __syncwarp();
                     to_t16(2, 0);
                 } else if (warp == 1) {
                     float a2[2][4] = {};
-                    warpmma::mm16_acc(Tb(3, 2), kF32Pitch, Tb(0, 2), kF32Pitch, a2);
+                    warpmma::mm16_acc_h(Tb(3, 2), kF32Pitch, Tb(0, 2), kF32Pitch, a2);
                     warpmma::store16(Tb(1, 2), kF32Pitch, a2, 1.f);            // P30a -> (1,2)
                 } else if (warp == 2) {
                     float a2[2][4] = {};
-                    warpmma::mm16_acc(Tb(3, 3), kF32Pitch, Tb(0, 3), kF32Pitch, a2);
+                    warpmma::mm16_acc_h(Tb(3, 3), kF32Pitch, Tb(0, 3), kF32Pitch, a2);
                     warpmma::store16(Tb(1, 3), kF32Pitch, a2, 1.f);            // P30b -> (1,3)
                 } else if (warp == 3) {
                     for (int e = lane; e < 64; e += 32) {                      // T31 = -(P31a + P31b)

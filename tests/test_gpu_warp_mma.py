@@ -24,7 +24,7 @@ def _lib():
                        check=True)
     lib = ctypes.CDLL(OUT)
     lib.mma_sync_probe.restype = ctypes.c_int
-    lib.mma_sync_probe.argtypes = [ctypes.c_void_p] * 3
+    lib.mma_sync_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int]
     return lib
 
 
@@ -36,8 +36,22 @@ def test_3xtf32_block_product(seed):
     Q = rng.normal(size=(16, 16)).astype(np.float32)
     dP, dQ = torch.from_numpy(P).cuda(), torch.from_numpy(Q).cuda()
     dD = torch.full((16, 16), float("nan"), device="cuda")
-    assert lib.mma_sync_probe(dP.data_ptr(), dQ.data_ptr(), dD.data_ptr()) == 0
+    assert lib.mma_sync_probe(dP.data_ptr(), dQ.data_ptr(), dD.data_ptr(), 0) == 0
     ref = P.astype(np.float64) @ Q.astype(np.float64)
     D = dD.cpu().numpy().astype(np.float64)
     # fp32-level agreement (a plain single-tf32 product would be off by ~1e-3)
     assert np.max(np.abs(D - ref)) <= 2e-5 * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_fp16_block_product(seed):
+    """Single-pass fp16 m16n8k16 product: exact on fp16-representable inputs."""
+    lib = _lib()
+    rng = np.random.default_rng(10 + seed)
+    P = (rng.integers(-64, 65, size=(16, 16)) / 64).astype(np.float32)
+    Q = (rng.integers(-64, 65, size=(16, 16)) / 64).astype(np.float32)
+    dP, dQ = torch.from_numpy(P).cuda(), torch.from_numpy(Q).cuda()
+    dD = torch.full((16, 16), float("nan"), device="cuda")
+    assert lib.mma_sync_probe(dP.data_ptr(), dQ.data_ptr(), dD.data_ptr(), 1) == 0
+    np.testing.assert_array_equal(dD.cpu().numpy().astype(np.float64),
+                                  P.astype(np.float64) @ Q.astype(np.float64))
