@@ -46,7 +46,7 @@ namespace fused {
 
 using namespace umma;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 
 // Optional per-phase cycle accounting (debug builds with -DKDA_PHASE_CLOCKS).
 #ifdef KDA_PHASE_CLOCKS
@@ -89,8 +89,8 @@ constexpr uint32_t KH = GQ + 16384;   // fp16 [64 i][128 c] Khat     (MN-major A
 constexpr uint32_t MISC = KH + 16384;
 constexpr uint32_t S_BETA = MISC;              // fp32 [64]
 constexpr uint32_t S_GAMMAC = S_BETA + 256;    // fp32 [128] e^{Gamma_last}
-constexpr uint32_t S_TOT = S_GAMMAC + 512;     // fp32 [4][128] per-block sums of log a
-constexpr uint32_t S_PDIAG = S_TOT + 2048;     // fp32 [2][64] halves of q_r . k_r
+constexpr uint32_t S_TOT = S_GAMMAC + 512;     // fp32 [8][128] per-half-block sums of log2 a
+constexpr uint32_t S_PDIAG = S_TOT + 4096;     // fp32 [2][64] halves of q_r . k_r
 constexpr uint32_t S_ORDER = S_PDIAG + 512;    // int16 [kSortLimit] sequences by length
 constexpr int kSortLimit = 512;
 constexpr uint32_t S_BARS = S_ORDER + 2 * kSortLimit;   // u64 [2]: inputs, mma
@@ -244,7 +244,9 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quarter = warp & 3, half = warp >> 2;
+    // TMEM access: warp w reads lane quarter (w % 4); `sub` splits columns between the four
+    // warps that share a quarter
+    const int quarter = warp & 3, sub = warp >> 2;
     const int G = gridDim.x, b = blockIdx.x;
     const int H = p.H;
     const int units = p.N * H;
@@ -309,15 +311,18 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
     }
 
-    // phase-1 thread mapping: warp -> (64-channel block cb, 16-token block blk), lane -> channel pair
-    const int cb = warp & 1, blk = warp >> 1;
+    // phase-1 mapping: warp -> (64-channel block cb, 16-token block blk, 8-token half hf),
+    // lane -> channel pair; each thread owns 2 channels x 8 tokens
+    const int cb = warp & 1, blk = (warp >> 1) & 3, hf = warp >> 3;
     const int c0 = cb * 64 + 2 * lane;
+    const int rbase = blk * 16 + hf * 8;                 // first token row of this thread
     const uint32_t lo = (uint32_t)(c0 & 7) * 2u;
     const uint32_t chk = (uint32_t)(c0 & 63) >> 3;
-    const uint32_t off128 = (uint32_t)cb * 128u * 128u + (uint32_t)blk * 2048u + lo;
-    const uint32_t off160 = (uint32_t)cb * 160u * 128u + (uint32_t)blk * 2048u + lo;
-    const uint32_t off64 = (uint32_t)cb * 64u * 128u + (uint32_t)blk * 2048u + lo;
-    // state / TMEM mapping: lane quarter -> rows, half -> column half
+    const uint32_t roff = (uint32_t)rbase * 128u + lo;
+    const uint32_t off128 = (uint32_t)cb * 128u * 128u + roff;
+    const uint32_t off160 = (uint32_t)cb * 160u * 128u + roff;
+    const uint32_t off64 = (uint32_t)cb * 64u * 128u + roff;
+    // state / TMEM mapping: lane quarter -> rows, sub -> 32-column quarter
     const int c_row = quarter * 32 + lane;
 
     bool aborted = false;
@@ -330,7 +335,8 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
         if (x.eos == x.bos) {   // empty sequence: final = initial
             if (p.final_state) {
-                for (int v0 = half * 64; v0 < half * 64 + 64; v0 += 4) {
+#pragma unroll
+                for (int v0 = sub * 32; v0 < sub * 32 + 32; v0 += 4) {
                     float4 s = p.initial_state
                         ? *reinterpret_cast<const float4*>(p.initial_state + state_off + c_row * kHeadDim + v0)
                         : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -340,7 +346,8 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             continue;
         }
         // load the initial state into TMEM
-        for (int v0 = half * 64; v0 < half * 64 + 64; v0 += 16) {
+#pragma unroll
+        for (int v0 = sub * 32; v0 < sub * 32 + 32; v0 += 16) {
             uint32_t r[16];
 #pragma unroll
             for (int j = 0; j < 16; j += 4) {
@@ -374,7 +381,6 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
             // ================= phase 1: gate + operands =================
             PHASE_MARK(0);
-            // the chunk after this one (its global reads overlap the input wait)
             const bool last = (j + 1 == nch);
             const bool has_next = last ? unit_has_next : true;
             const int h1 = last ? hn : h;
@@ -385,33 +391,37 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             in_parity ^= 1u;
             in_flight = false;
 
-            float G0[16], G1[16];   // in-block inclusive cumsum of log2 a (two channels)
+            float G0[8], G1[8];   // inclusive cumsum of log2 a over this thread's 8 tokens
             {
                 float a0 = 0.f, a1 = 0.f;
                 const float* gin = reinterpret_cast<const float*>(sm + IN_G);
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int r = blk * 16 + rr;
+                for (int i = 0; i < 8; ++i) {
+                    const int r = rbase + i;
                     const float2 gv = *reinterpret_cast<const float2*>(gin + r * kHeadDim + c0);
                     const bool ok = r < L;
                     const float l0 = gate_log2_decay(gv.x, db2_0, nexpA, lb2);
                     const float l1 = gate_log2_decay(gv.y, db2_1, nexpA, lb2);
                     a0 += ok ? l0 : 0.f;
                     a1 += ok ? l1 : 0.f;
-                    G0[rr] = a0;
-                    G1[rr] = a1;
+                    G0[i] = a0;
+                    G1[i] = a1;
                 }
-                sTot[blk * kHeadDim + c0] = a0;
-                sTot[blk * kHeadDim + c0 + 1] = a1;
+                sTot[(blk * 2 + hf) * kHeadDim + c0] = a0;
+                sTot[(blk * 2 + hf) * kHeadDim + c0 + 1] = a1;
             }
-            PHASE_MARK(12);
             __syncthreads();
+            PHASE_MARK(12);
             {
-                float tot0[4], tot1[4];
+                // block sums (16-token blocks) from the half-block sums
+                float tot0[4], tot1[4], half0 = 0.f, half1 = 0.f;
 #pragma unroll
                 for (int bb = 0; bb < 4; ++bb) {
-                    tot0[bb] = sTot[bb * kHeadDim + c0];
-                    tot1[bb] = sTot[bb * kHeadDim + c0 + 1];
+                    const float x00 = sTot[(2 * bb) * kHeadDim + c0], x01 = sTot[(2 * bb + 1) * kHeadDim + c0];
+                    const float x10 = sTot[(2 * bb) * kHeadDim + c0 + 1], x11 = sTot[(2 * bb + 1) * kHeadDim + c0 + 1];
+                    tot0[bb] = x00 + x01;
+                    tot1[bb] = x10 + x11;
+                    if (bb == blk && hf == 1) { half0 = x00; half1 = x10; }
                 }
                 float Ts0 = 0.f, Ts1 = 0.f, after0 = 0.f, after1 = 0.f;
 #pragma unroll
@@ -429,45 +439,52 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float F2_0 = 0.f, F2_1 = 0.f, F3_0 = 0.f, F3_1 = 0.f;
                 if (blk <= 1) { F2_0 = fast_ex2(pick4(tot0, blk + 1)); F2_1 = fast_ex2(pick4(tot1, blk + 1)); }
                 if (blk == 0) { F3_0 = fast_ex2(tot0[1] + tot0[2]); F3_1 = fast_ex2(tot1[1] + tot1[2]); }
-                if (blk == 0) {
+                if (blk == 0 && hf == 0) {
                     sGammaC[c0] = fast_ex2(tb0 + after0);
                     sGammaC[c0 + 1] = fast_ex2(tb1 + after1);
                 }
                 const uint32_t* kin = reinterpret_cast<const uint32_t*>(sm + IN_K);
                 const uint32_t* qin = reinterpret_cast<const uint32_t*>(sm + IN_Q);
                 const uint32_t* vin = reinterpret_cast<const uint32_t*>(sm + IN_V);
-                float pd[16];
-                // all loads of the block first: the stores below cannot be ordered
-                // before them by the compiler (one shared-memory base for both)
-                uint32_t kwv[16], qwv[16], vwv[16];
-                float bev[16];
+                // all loads of the thread's 8 tokens first (one shared-memory base for loads
+                // and stores: the compiler could not move loads above the stores)
+                uint32_t kwv[8], qwv[8], vwv[8];
+                float bev[8];
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int r = blk * 16 + rr;
+                for (int i = 0; i < 8; ++i) {
+                    const int r = rbase + i;
                     const bool ok = r < L;
                     const int idx = (r * kHeadDim + c0) >> 1;
-                    kwv[rr] = ok ? kin[idx] : 0u;
-                    qwv[rr] = ok ? qin[idx] : 0u;
-                    vwv[rr] = ok ? vin[idx] : 0u;
-                    bev[rr] = sBeta[r];
+                    kwv[i] = ok ? kin[idx] : 0u;
+                    qwv[i] = ok ? qin[idx] : 0u;
+                    vwv[i] = ok ? vin[idx] : 0u;
+                    bev[i] = sBeta[r];
                 }
-                // (a) operands of the A/P MMA, then issue it; (b) the other operand tiles while it runs
+                // (a) A/P MMA operands (+ K-hat, gamma*q which need the same factors), then the
+                //     MMA is issued; (b) beta*gamma*k and beta*v while it runs
+                float g0v[8], g1v[8], pd[8];
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    const uint32_t kw = kwv[rr], qw = qwv[rr];
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t kw = kwv[i], qw = qwv[i];
                     const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
                     const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
-                    const float R0 = fast_ex2(G0[rr]), R1 = fast_ex2(G1[rr]);            // e^{Gamma_r - Gamma_s}
-                    const float E0 = fast_ex2(tb0 - G0[rr]), E1 = fast_ex2(tb1 - G1[rr]);  // e^{Gamma_e - Gamma_r}
+                    const float ls0 = half0 + G0[i], ls1 = half1 + G1[i];             // Gamma_r - Gamma_s (log2)
+                    const float R0 = fast_ex2(ls0), R1 = fast_ex2(ls1);                 // e^{Gamma_r - Gamma_s}
+                    const float E0 = fast_ex2(tb0 - ls0), E1 = fast_ex2(tb1 - ls1);     // e^{Gamma_e - Gamma_r}
                     const float kE0 = k0 * E0, kE1 = k1 * E1;
-                    const uint32_t ro = (uint32_t)rr * 128u + ((chk ^ (uint32_t)(rr & 7)) << 4);
+                    const uint32_t ro = (uint32_t)i * 128u + ((chk ^ (uint32_t)i) << 4);
                     st_u32(sm, AP_A + off128 + ro, pack_bf16(k0 * R0, k1 * R1));
                     st_u32(sm, AP_A + off128 + 64u * 128u + ro, pack_bf16(q0 * R0, q1 * R1));
                     st_u32(sm, AP_B + off160 + ro, pack_bf16(kE0 * invB0, kE1 * invB1));
                     if (blk <= 2) st_u32(sm, AP_B + off160 + 64u * 128u + ro, pack_bf16(kE0, kE1));
                     if (blk <= 1) st_u32(sm, AP_B + off160 + 112u * 128u + ro, pack_bf16(kE0 * F2_0, kE1 * F2_1));
                     if (blk == 0) st_u32(sm, AP_B + off160 + 144u * 128u + ro, pack_bf16(kE0 * F3_0, kE1 * F3_1));
-                    pd[rr] = fmaf(q0, k0, q1 * k1);
+                    st_u32(sm, KH + off64 + ro, pack_f16(kE0 * eA0, kE1 * eA1));
+                    const float g0 = R0 * eTs0, g1 = R1 * eTs1;                          // gamma_r
+                    st_u32(sm, GQ + off64 + ro, pack_f16(q0 * g0, q1 * g1));
+                    g0v[i] = g0;
+                    g1v[i] = g1;
+                    pd[i] = fmaf(q0, k0, q1 * k1);
                 }
                 fence_proxy_async();
                 __syncthreads();
@@ -481,58 +498,44 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mma_commit(bar_mma);
                 }
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    const uint32_t kw = kwv[rr], qw = qwv[rr], vw = vwv[rr];
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t kw = kwv[i], vw = vwv[i];
                     const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
-                    const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
                     const float v0 = __uint_as_float(vw << 16), v1 = __uint_as_float(vw & 0xFFFF0000u);
-                    const float be = bev[rr];
-                    const float R0 = fast_ex2(G0[rr]), R1 = fast_ex2(G1[rr]);
-                    const float E0 = fast_ex2(tb0 - G0[rr]), E1 = fast_ex2(tb1 - G1[rr]);
-                    const float kE0 = k0 * E0, kE1 = k1 * E1;
-                    const uint32_t ro = (uint32_t)rr * 128u + ((chk ^ (uint32_t)(rr & 7)) << 4);
-                    const float g0 = R0 * eTs0, g1 = R1 * eTs1;                          // gamma_r
-                    st_u32(sm, GQ + off64 + ro, pack_f16(q0 * g0, q1 * g1));
-                    st_u32(sm, BGK + off64 + ro, pack_f16(be * k0 * g0, be * k1 * g1));
-                    st_u32(sm, KH + off64 + ro, pack_f16(kE0 * eA0, kE1 * eA1));
+                    const float be = bev[i];
+                    const uint32_t ro = (uint32_t)i * 128u + ((chk ^ (uint32_t)i) << 4);
+                    st_u32(sm, BGK + off64 + ro, pack_f16(be * k0 * g0v[i], be * k1 * g1v[i]));
                     st_u32(sm, BV + off64 + ro, pack_f16(be * v0, be * v1));
                 }
                 PHASE_MARK(13);
-                // reduce pd over the 32 lanes for all 16 tokens at once (transposing butterfly):
-                // after the halving steps lanes 2m and 2m + 1 hold token m of the block
+                // reduce pd over the 32 lanes for the 8 tokens at once (transposing butterfly);
+                // afterwards lanes 4m .. 4m + 3 hold the sum of token m
 #pragma unroll
-                for (int t = 0; t < 8; ++t) {
+                for (int t = 0; t < 4; ++t) {
                     const bool up = lane & 16;
-                    const float send = up ? pd[t] : pd[t + 8];
-                    const float keep = up ? pd[t + 8] : pd[t];
+                    const float send = up ? pd[t] : pd[t + 4];
+                    const float keep = up ? pd[t + 4] : pd[t];
                     pd[t] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
                 }
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const bool up = lane & 8;
-                    const float send = up ? pd[t] : pd[t + 4];
-                    const float keep = up ? pd[t + 4] : pd[t];
-                    pd[t] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-                }
-#pragma unroll
                 for (int t = 0; t < 2; ++t) {
-                    const bool up = lane & 4;
+                    const bool up = lane & 8;
                     const float send = up ? pd[t] : pd[t + 2];
                     const float keep = up ? pd[t + 2] : pd[t];
-                    pd[t] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+                    pd[t] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
                 }
                 {
-                    const bool up = lane & 2;
+                    const bool up = lane & 4;
                     const float send = up ? pd[0] : pd[1];
                     const float keep = up ? pd[1] : pd[0];
-                    pd[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                    pd[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
                 }
+                pd[0] += __shfl_xor_sync(0xffffffffu, pd[0], 2);
                 pd[0] += __shfl_xor_sync(0xffffffffu, pd[0], 1);
-                // token held: bit3 of the token = lane bit4, bit2 = lane bit3, bit1 = lane bit2, bit0 = lane bit1
-                if ((lane & 1) == 0) {
-                    const int tk = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
-                                   ((lane >> 1) & 1);
-                    sPdiag[cb * 64 + blk * 16 + tk] = pd[0];
+                // token held: bit2 = lane bit4, bit1 = lane bit3, bit0 = lane bit2
+                if ((lane & 3) == 0) {
+                    const int tk = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+                    sPdiag[cb * 64 + rbase + tk] = pd[0];
                 }
             }
             fence_proxy_async();
@@ -553,56 +556,51 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
             // ================= phase 3: A / P read-out =================
             {
-                // quarter q holds rows 32 (q & 1) .. + 31 of A (q < 2) or P (q >= 2); warps 0-3
-                // assemble column blocks J = 0, 1 of their rows, warps 4-7 blocks J = 2, 3
+                // quarter q holds rows 32 (q & 1) .. + 31 of A (q < 2) or P (q >= 2); warp `sub`
+                // assembles column block J = sub of those rows
                 const bool isA = quarter < 2;
                 const int r = (quarter & 1) * 32 + lane;      // token row in the chunk
                 const int I = r >> 4;
-                const int jb = half * 2;                        // first column block of this warp
-                float row[32];
-                auto pick = [&](int Jl, uint32_t col_a, uint32_t col_b, int I_a) {
+                const int J = sub;
+                float row[16];
+                auto pick = [&](uint32_t col_a, uint32_t col_b, int I_a) {
                     uint32_t ta[16], tb2[16];
                     tmem_ld16(taddr(tbase, quarter, TM_AP + col_a), ta);
                     tmem_ld16(taddr(tbase, quarter, TM_AP + col_b), tb2);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj)
-                        row[Jl * 16 + jj] = __uint_as_float(I == I_a ? ta[jj] : tb2[jj]);
+                    for (int jj = 0; jj < 16; ++jj) row[jj] = __uint_as_float(I == I_a ? ta[jj] : tb2[jj]);
                 };
                 if ((quarter & 1) == 0) {        // I in {0, 1}
-                    if (half == 0) {
-                        pick(0, 0, 64, 0);       // J=0: I=0 d=0 cols 0-15; I=1 d=1 cols 64-79
-                        pick(1, 16, 16, 1);      // J=1: I=1 d=0 cols 16-31 (I=0: masked below)
-                    } else {
+                    if (J == 0) pick(0, 64, 0);            // I=0: d=0 cols 0-15; I=1: d=1 cols 64-79
+                    else if (J == 1) pick(16, 16, 1);      // I=1: d=0 cols 16-31 (I=0: masked below)
+                    else {
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) row[jj] = 0.f;
+                        for (int jj = 0; jj < 16; ++jj) row[jj] = 0.f;
                     }
                 } else {                         // I in {2, 3}
-                    if (half == 0) {
-                        pick(0, 112, 144, 2);    // J=0: I=2 d=2 cols 112-127; I=3 d=3 cols 144-159
-                        pick(1, 80, 128, 2);     // J=1: I=2 d=1 cols 80-95;   I=3 d=2 cols 128-143
-                    } else {
-                        pick(0, 32, 96, 2);      // J=2: I=2 d=0 cols 32-47;   I=3 d=1 cols 96-111
-                        pick(1, 48, 48, 3);      // J=3: I=3 d=0 cols 48-63 (I=2: masked below)
-                    }
+                    if (J == 0) pick(112, 144, 2);         // I=2: d=2 cols 112-127; I=3: d=3 cols 144-159
+                    else if (J == 1) pick(80, 128, 2);     // I=2: d=1 cols 80-95;   I=3: d=2 cols 128-143
+                    else if (J == 2) pick(32, 96, 2);      // I=2: d=0 cols 32-47;   I=3: d=1 cols 96-111
+                    else pick(48, 48, 3);                  // I=3: d=0 cols 48-63 (I=2: masked below)
                 }
                 const float pdg = sPdiag[r] + sPdiag[64 + r];
 #pragma unroll
-                for (int ii = 0; ii < 32; ++ii) {
-                    const int i = jb * 16 + ii;
+                for (int ii = 0; ii < 16; ++ii) {
+                    const int i = J * 16 + ii;
                     row[ii] = i < r ? row[ii] : ((i == r && !isA) ? pdg : 0.f);
                 }
                 if (isA) {
                     const float be = sBeta[r];
-                    float* a32 = reinterpret_cast<float*>(sm + A32) + r * kF32Pitch + jb * 16;
+                    float* a32 = reinterpret_cast<float*>(sm + A32) + r * kF32Pitch + J * 16;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4)
+                    for (int i = 0; i < 16; i += 4)
                         *reinterpret_cast<float4*>(a32 + i) =
                             make_float4(be * row[i], be * row[i + 1], be * row[i + 2], be * row[i + 3]);
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        st_v4(sm, P16 + sw128_chunk_off(r, jb * 2 + c, 64), pack_f16(row[8 * c], row[8 * c + 1]),
+                    for (int c = 0; c < 2; ++c)
+                        st_v4(sm, P16 + sw128_chunk_off(r, J * 2 + c, 64), pack_f16(row[8 * c], row[8 * c + 1]),
                               pack_f16(row[8 * c + 2], row[8 * c + 3]), pack_f16(row[8 * c + 4], row[8 * c + 5]),
                               pack_f16(row[8 * c + 6], row[8 * c + 7]));
                 }
@@ -640,8 +638,8 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                     for (int rr = 0; rr < 16; ++rr) t32[(o + rr) * kF32Pitch + o + jc] = xv[rr];
                 } else if (tid >= 128) {
-                    // zero fp16 blocks above the diagonal: 6 blocks x 32 chunks over 128 threads
-                    for (int e = tid - 128; e < 6 * 32; e += 128) {
+                    // zero fp16 blocks above the diagonal: 6 blocks x 32 chunks
+                    for (int e = tid - 128; e < 6 * 32; e += kThreads - 128) {
                         const int blkid = e >> 5, c = e & 31;
                         const int I = blkid < 3 ? 0 : (blkid < 5 ? 1 : 2);
                         const int J = blkid < 3 ? blkid + 1 : (blkid < 5 ? blkid - 1 : 3);
@@ -680,7 +678,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     warpmma::mm16_acc_h(Ab(2, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);   // X20 partial
                 } else if (warp == 4) {
                     warpmma::mm16_acc_h(Ab(3, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);   // X30 partial
-                } else {
+                } else if (warp < 8) {
                     for (int d = warp - 5; d < 4; d += 3) to_t16(d, d);               // diagonal blocks
                 }
                 __syncthreads();
@@ -774,15 +772,15 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // ================= phase 6: W -> fp16 smem =================
             {
                 // M = 64 accumulator: row r lives in lane (r % 16) of quarter r / 16
-                uint32_t v[4][16];
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) tmem_ld16(taddr(tbase, quarter, TM_W + half * 64 + cc * 16), v[cc]);
+                uint32_t v[2][16];
+                tmem_ld16(taddr(tbase, quarter, TM_W + sub * 32), v[0]);
+                tmem_ld16(taddr(tbase, quarter, TM_W + sub * 32 + 16), v[1]);
                 tmem_wait_ld();
                 if (lane < 16) {
                     const int r = quarter * 16 + lane;
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        const uint32_t col = half * 64 + cc * 16;
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const uint32_t col = sub * 32 + cc * 16;
                         uint32_t w[8];
 #pragma unroll
                         for (int q2 = 0; q2 < 8; ++q2)
@@ -796,21 +794,22 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // ================= phase 7: S copy + decay, U and O MMAs =================
             {
                 const float gC = sGammaC[c_row];
+                uint32_t v[2][16];
+                tmem_ld16(taddr(tbase, quarter, TM_S + sub * 32), v[0]);
+                tmem_ld16(taddr(tbase, quarter, TM_S + sub * 32 + 16), v[1]);
+                tmem_wait_ld();
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const uint32_t v0 = half * 64 + cc * 16;
-                    uint32_t v[16];
-                    tmem_ld16(taddr(tbase, quarter, TM_S + v0), v);
-                    tmem_wait_ld();
+                for (int cc = 0; cc < 2; ++cc) {
+                    const uint32_t v0 = sub * 32 + cc * 16;
                     uint32_t w[8];
 #pragma unroll
                     for (int q2 = 0; q2 < 8; ++q2)
-                        w[q2] = pack_f16(__uint_as_float(v[2 * q2]), __uint_as_float(v[2 * q2 + 1]));
+                        w[q2] = pack_f16(__uint_as_float(v[cc][2 * q2]), __uint_as_float(v[cc][2 * q2 + 1]));
                     st_v4(sm, S16 + sw128_chunk_off(c_row, v0 / 8, 128), w[0], w[1], w[2], w[3]);
                     st_v4(sm, S16 + sw128_chunk_off(c_row, v0 / 8 + 1, 128), w[4], w[5], w[6], w[7]);
 #pragma unroll
-                    for (int q2 = 0; q2 < 16; ++q2) v[q2] = __float_as_uint(__uint_as_float(v[q2]) * gC);
-                    tmem_st16(taddr(tbase, quarter, TM_S + v0), v);
+                    for (int q2 = 0; q2 < 16; ++q2) v[cc][q2] = __float_as_uint(__uint_as_float(v[cc][q2]) * gC);
+                    tmem_st16(taddr(tbase, quarter, TM_S + v0), v[cc]);
                 }
                 tmem_wait_st();
             }
@@ -838,20 +837,15 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // ================= phase 8: U -> fp16, S and O MMAs =================
             {
                 const int v_row = c_row;   // lanes of U^T are value columns
-                uint32_t v[2][16];
-                tmem_ld16(taddr(tbase, quarter, TM_UT + half * 32), v[0]);
-                tmem_ld16(taddr(tbase, quarter, TM_UT + half * 32 + 16), v[1]);
+                uint32_t v[16];
+                tmem_ld16(taddr(tbase, quarter, TM_UT + sub * 16), v);
                 tmem_wait_ld();
+                uint32_t w[8];
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const uint32_t r0 = half * 32 + cc * 16;
-                    uint32_t w[8];
-#pragma unroll
-                    for (int q2 = 0; q2 < 8; ++q2)
-                        w[q2] = pack_f16(__uint_as_float(v[cc][2 * q2]), __uint_as_float(v[cc][2 * q2 + 1]));
-                    st_v4(sm, U16 + sw128_chunk_off(v_row, r0 / 8, 128), w[0], w[1], w[2], w[3]);
-                    st_v4(sm, U16 + sw128_chunk_off(v_row, r0 / 8 + 1, 128), w[4], w[5], w[6], w[7]);
-                }
+                for (int q2 = 0; q2 < 8; ++q2)
+                    w[q2] = pack_f16(__uint_as_float(v[2 * q2]), __uint_as_float(v[2 * q2 + 1]));
+                st_v4(sm, U16 + sw128_chunk_off(v_row, sub * 2, 128), w[0], w[1], w[2], w[3]);
+                st_v4(sm, U16 + sw128_chunk_off(v_row, sub * 2 + 1, 128), w[4], w[5], w[6], w[7]);
             }
             fence_proxy_async();
             fence_before_sync();
@@ -876,17 +870,13 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // ================= phase 9: O -> out (through an smem tile, coalesced) =================
             {
                 const int v_col = c_row;
-                uint32_t v[2][16];
-                tmem_ld16(taddr(tbase, quarter, TM_OT + half * 32), v[0]);
-                tmem_ld16(taddr(tbase, quarter, TM_OT + half * 32 + 16), v[1]);
+                uint32_t v[16];
+                tmem_ld16(taddr(tbase, quarter, TM_OT + sub * 16), v);
                 tmem_wait_ld();
                 __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + OST);
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-                    for (int jj = 0; jj < 16; ++jj)
-                        ost[(half * 32 + cc * 16 + jj) * kHeadDim + v_col] =
-                            __float2bfloat16_rn(p.scale * __uint_as_float(v[cc][jj]));
+                for (int jj = 0; jj < 16; ++jj)
+                    ost[(sub * 16 + jj) * kHeadDim + v_col] = __float2bfloat16_rn(p.scale * __uint_as_float(v[jj]));
             }
             fence_before_sync();
             __syncthreads();
@@ -906,7 +896,8 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // final state
         if (p.final_state) {
             fence_after_sync();
-            for (int v0 = half * 64; v0 < half * 64 + 64; v0 += 16) {
+#pragma unroll
+            for (int v0 = sub * 32; v0 < sub * 32 + 32; v0 += 16) {
                 uint32_t r[16];
                 tmem_ld16(taddr(tbase, quarter, TM_S + v0), r);
                 tmem_wait_ld();
