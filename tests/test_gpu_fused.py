@@ -102,9 +102,10 @@ def test_fused_split_and_resume():
     check(torch.cat([oa, ob]), fb, ref_o, ref_f, "split/resume")
 
 
-@pytest.mark.parametrize("wid", [3, 2])
+@pytest.mark.parametrize("wid", [3, 2, 1, 4])
 def test_fused_full_size_workloads(wid):
-    """8 x 1024 stateful (H=64) and the T=8192 H=96 varlen workload, compared in full."""
+    """The four large workloads compared in full against the oracle: 8 x 1024 stateful
+    (H=64), T=8192 H=96 varlen, T=8192 H=64 fixed, and T=131072 H=32 with states."""
     kda = _kda()
     w = W.WORKLOADS[wid]
     x = W.make_inputs(w)
