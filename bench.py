@@ -44,7 +44,7 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--workload", type=int, default=2, choices=sorted(W.WORKLOADS))
@@ -52,6 +52,10 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", action="store_true",
+                    help="time kda_decode (one token per sequence) instead of the prefill")
+    ap.add_argument("--decode-batch", type=int, default=256)
+    ap.add_argument("--decode-heads", type=int, default=96)
     return ap.parse_args()
 
 
@@ -131,18 +135,31 @@ class ClockSampler:
         except Exception:
             pass
 
-    def _run(self):
+    def sample(self):
+        if not self._ok:
+            return
         nv = self.nv
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+            mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for bit, name in self.REASONS.items():
+                if mask & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
-                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if mask & bit:
-                        self.reasons.add(name)
-            except Exception:
-                break
+            self.sample()
             time.sleep(0.002)
+
+    def wait(self, event):
+        """Samples from the calling thread until ``event`` has completed (the
+        launches are queued already, so the GPU stays busy meanwhile)."""
+        while not event.query():
+            self.sample()
+            time.sleep(0.0005)
+        torch.cuda.synchronize()
 
     def __enter__(self):
         if self._ok:
@@ -271,6 +288,110 @@ def run_reference(args, world, rank):
     return 0
 
 
+DECODE_BYTES_PER_SEQ_HEAD = 2 * STATE_BYTES + 768 + 512 + 4 + 256   # state in + out, q/k/v, g, beta, o
+
+
+def run_decode(args, world, rank, kda):
+    """kda_decode over B sequences x H heads per step: one token each, the fp32
+    states updated in place (B H 128 KiB of state traffic per step)."""
+    B, H = args.decode_batch, args.decode_heads
+    gen = torch.Generator("cpu").manual_seed(2000)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = W.custom([1] * B, H=H, packed=False, init="normal", wid=60)
+    x = W.make_inputs(w)
+    xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    state = (torch.randn(B, H, 128, 128, generator=gen) * 0.02).to(dev)
+    out = torch.empty(B, H, 128, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kda.kda_decode(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"],
+                       x["lower_bound"], x["scale"], state, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if kda.kda_check_device_error() != 0:
+        raise RuntimeError("device error recorded during warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        sampler.wait(ends[-1])
+    barrier(world)
+    kernel_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    total_ms = max_over_ranks(starts[0].elapsed_time(ends[-1]), world)
+    ms_per_step = total_ms / args.steps
+    value = B * world / (ms_per_step / 1e3) / 1e6
+    alg_bytes = DECODE_BYTES_PER_SEQ_HEAD * B * H
+    peak, peak_kind = measured_hbm_peak()
+    achieved = alg_bytes / (kernel_ms / 1e3) / 1e9
+
+    e2e = None
+    if args.e2e_steps > 0:
+        keys = ("q", "k", "v", "g", "beta")
+        host = {k: x[k].pin_memory() for k in keys}
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+        d2h = out_h.numel() * out_h.element_size()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for k in keys:
+                xd[k].copy_(host[k], non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.e2e_steps
+        e2e = {"value": B * world / (e_ms / 1e3) / 1e6, "unit": "Mtokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        sub_b = max(1, min(B, 32))
+        xs = {k: x[k][:sub_b] for k in ("q", "k", "v", "g", "beta")}
+        st = state[:sub_b].cpu()
+        t = time.perf_counter()
+        oracle.recurrent(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], x["A_log"], x["dt_bias"],
+                         x["lower_bound"], x["scale"], st, oracle.fixed_offsets(sub_b, 1))
+        el = time.perf_counter() - t
+        cpu = {"value": sub_b / el / 1e6, "unit": "Mtokens/s", "cores": oracle.max_threads(),
+               "kind": "oracle", "sample": f"{sub_b} of {B} sequences x {H} heads, one token each"}
+
+    if rank == 0:
+        line = {
+            "metric": f"KDA decode throughput (Mtokens/s) at B={B} H={H} D=128",
+            "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded kda_workloads, no dataset)",
+            "config": {"workload": f"decode B={B} H={H} K=V=128, fp32 state in place",
+                       "global_batch": B * world, "seq_len": 1, "heads": H,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": f"state {B * H * STATE_BYTES / 1e9:.2f} GB exceeds L2; no flush"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
+                         "kernel": "kda_decode_kernel", "kernel_ms": kernel_ms,
+                         "algorithmic_bytes": alg_bytes},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     assert args.warmup >= 3, "at least 3 warm-up steps"
@@ -287,6 +408,12 @@ def main():
         build.build()
     barrier(world)
     import gated_delta_rule_135_b200 as kda
+    if args.decode:
+        rc = run_decode(args, world, rank, kda)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
 
     w = W.WORKLOADS[args.workload]
     x = W.make_inputs(w)
@@ -319,7 +446,7 @@ def main():
             starts[i].record(stream)
             step()
             ends[i].record(stream)
-        torch.cuda.synchronize()
+        sampler.wait(ends[-1])
     barrier(world)
     per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = starts[0].elapsed_time(ends[-1])

@@ -74,6 +74,8 @@ def _load():
     lib.kda_fwd_staged_noalloc.argtypes = fwd_args + [vp]
     lib.kda_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.kda_noalloc_scratch_bytes.argtypes = []
+    lib.kda_decode.restype = ctypes.c_int
+    lib.kda_decode.argtypes = [vp] * 7 + [f32, f32, vp, vp, ctypes.c_int32, ctypes.c_int32, vp]
     return lib
 
 
@@ -83,7 +85,7 @@ _lib = _load()
 EXPORTED = ("kda_fwd", "kda_fwd_staged", "kda_staged_workspace_size",
             "kda_staged_workspace_layout", "kda_strerror", "kda_check_device_error",
             "kda_last_device_error_bits", "kda_version", "kda_fwd_staged_noalloc",
-            "kda_noalloc_scratch_bytes")
+            "kda_noalloc_scratch_bytes", "kda_decode")
 
 
 def lib() -> ctypes.CDLL:
@@ -240,6 +242,28 @@ def kda_fwd_staged_noalloc(q, k, v, g, beta, A_log, dt_bias, lower_bound: float,
 
 def kda_noalloc_scratch_bytes() -> int:
     return int(_lib.kda_noalloc_scratch_bytes())
+
+
+def kda_decode(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, scale: float, state,
+               out=None, *, stream=None):
+    """Calls kda_decode: one recurrent step per sequence.  q/k/v: bf16 [B, H, 128];
+    g: fp32 [B, H, 128]; beta: fp32 [B, H]; state: fp32 [B, H, 128, 128], updated in
+    place.  Returns out (bf16 [B, H, 128])."""
+    dev = q.device
+    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16), ("v", v, torch.bfloat16),
+                        ("g", g, torch.float32), ("beta", beta, torch.float32),
+                        ("A_log", A_log, torch.float32), ("dt_bias", dt_bias, torch.float32),
+                        ("state", state, torch.float32)):
+        _check_tensor(name, t, dt, dev)
+    B, H = q.shape[0], q.shape[1]
+    if out is None:
+        out = torch.empty(B, H, HEAD_DIM, dtype=torch.bfloat16, device=dev)
+    st = _lib.kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias),
+                         float(lower_bound), float(scale), _ptr(state), _ptr(out), int(B), int(H),
+                         _stream_ptr(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode")
+    return out
 
 
 def kda_check_device_error(stream=None) -> int:

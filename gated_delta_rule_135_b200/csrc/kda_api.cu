@@ -13,6 +13,7 @@
 
 #include "kda_staged.cuh"
 #include "kda_fused.cuh"
+#include "kda_decode.cuh"
 
 namespace {
 
@@ -221,6 +222,29 @@ kda_status kda_fwd(const void* q, const void* k, const void* v, const float* g, 
     cudaError_t err = kda::launch_staged(a, static_cast<char*>(ws), L, s);
     cudaError_t err2 = cudaFreeAsync(ws, s);
     return (err == cudaSuccess && err2 == cudaSuccess) ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                      const float* A_log, const float* dt_bias, float lower_bound, float scale,
+                      float* state, void* out, int32_t batch, int32_t num_heads, kda_stream_t stream) {
+    if (batch < 0 || num_heads < 1) return KDA_ERR_INVALID_ARG;
+    if (isnan(lower_bound) || lower_bound > 0.f || !isfinite(scale)) return KDA_ERR_INVALID_ARG;
+    if (batch == 0) return KDA_OK;
+    if (!q || !k || !v || !g || !beta || !A_log || !dt_bias || !state || !out) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, beta, A_log, dt_bias, state, out};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+    const size_t bh = (size_t)batch * num_heads;
+    const size_t ob = bh * kda::kHeadDim * 2;
+    if (overlaps(out, ob, q, ob) || overlaps(out, ob, k, ob) || overlaps(out, ob, v, ob) ||
+        overlaps(out, ob, g, bh * kda::kHeadDim * 4) || overlaps(out, ob, beta, bh * 4) ||
+        overlaps(out, ob, state, bh * kda::kHeadDim * kda::kHeadDim * 4))
+        return KDA_ERR_INVALID_ARG;
+    kda_status st = device_ok();
+    if (st != KDA_OK) return st;
+    return kda::launch_decode(q, k, v, g, beta, A_log, dt_bias, lower_bound, scale, state, out, batch,
+                              num_heads, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? KDA_OK : KDA_ERR_CUDA;
 }
 
 const char* kda_strerror(kda_status status) {

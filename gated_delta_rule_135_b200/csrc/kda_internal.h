@@ -36,6 +36,10 @@ StagedLayout staged_layout(int64_t total_tokens, int H, int N);
 cudaError_t launch_staged(const StagedArgs& a, char* workspace, const StagedLayout& L,
                           cudaStream_t stream);
 
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                          const float* A_log, const float* dt_bias, float lower_bound, float scale,
+                          float* state, void* out, int batch, int H, cudaStream_t stream);
+
 // The fused persistent tcgen05 kernel (same arguments; no workspace).
 cudaError_t launch_fused(const StagedArgs& a, cudaStream_t stream);
 bool fused_supported(float lower_bound);

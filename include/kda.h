@@ -177,6 +177,25 @@ kda_status kda_fwd_staged_noalloc(const void* q, const void* k, const void* v,
 /* Size in bytes of the scratch kda_fwd_staged_noalloc uses (16 MiB). */
 size_t kda_noalloc_scratch_bytes(void);
 
+/*
+ * kda_decode -- one recurrent step (decode) per sequence, in place on the state.
+ * The token-by-token form of the same KDA recurrence; the FlashKDA post
+ * (donniechu.com, sections "Hạn chế & điều kiện" and "What's next") lists
+ * decode as not yet tuned and a decode kernel as future work of that release.
+ *   q, k, v  bf16 [batch, H, 128]     g fp32 [batch, H, 128]     beta fp32 [batch, H]
+ *   A_log fp32 [H], dt_bias fp32 [H, 128]
+ *   state    fp32 [batch, H, 128, 128] ([k][v]); read and overwritten with the new state
+ *   out      bf16 [batch, H, 128] = scale * S_new^T q
+ * Errors as for kda_fwd (checked before the launch); out must not overlap any
+ * input or the state.  Asynchronous on `stream`.
+ */
+kda_status kda_decode(const void* q, const void* k, const void* v,
+                      const float* g, const float* beta,
+                      const float* A_log, const float* dt_bias,
+                      float lower_bound, float scale,
+                      float* state, void* out,
+                      int32_t batch, int32_t num_heads, kda_stream_t stream);
+
 /* Human-readable name of a status code (static storage; never NULL). */
 const char* kda_strerror(kda_status status);
 

@@ -124,3 +124,19 @@ def test_staged_workspace_layout_is_consistent():
         assert L.u - L.p >= 4 * T * H * 64
         assert L.total - L.chunk_states >= 4 * L.max_chunks * H * 128 * 128
         assert kda.lib().kda_staged_workspace_size(dims, varlen) == L.total
+
+
+def test_decode_rejects_bad_arguments():
+    lib = kda.lib()
+    p = [FAKE + i * (1 << 28) for i in range(9)]
+    call = lambda pp, lb=-5.0, scale=0.1, B=2, H=2: lib.kda_decode(  # noqa: E731
+        *pp[:7], ctypes.c_float(lb), ctypes.c_float(scale), pp[7], pp[8], B, H, None)
+    assert call(p, lb=1.0) == 1
+    assert call(p, scale=float("inf")) == 1
+    assert call(p, H=0) == 1
+    assert call(p, B=-1) == 1
+    bad = list(p)
+    bad[3] += 4
+    assert call(bad) == 3
+    assert call(p[:8] + [p[0]]) == 1          # out aliases q
+    assert call(p, B=0) == 0                  # nothing to do
