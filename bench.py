@@ -77,31 +77,45 @@ def algorithmic_bytes(w: W.Workload) -> int:
     return b
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "kda_fused_kernel": ("kda_fused.cuh", "umma.cuh", "warp_mma.cuh", "kda_common.cuh"),
+    "kda_decode_kernel": ("kda_decode.cuh", "kda_common.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str = "kda_fused_kernel") -> str:
+    """Hash of the device sources one kernel is compiled from (profiles carry it
+    so that stale DRAM counters are not reported against a changed kernel)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_135_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def dram_traffic_from_profile(w: W.Workload):
-    """Per-launch DRAM bytes of the fused kernel from the committed ncu summary,
-    if it was taken on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", "kda_fused_traffic.json")
+TRAFFIC_FILES = {"kda_fused_kernel": "kda_fused_traffic.json",
+                 "kda_decode_kernel": "kda_decode_traffic.json"}
+
+
+def dram_traffic_from_profile(kernel: str, units: float):
+    """Per-launch DRAM bytes (read + write) of ``kernel`` from its committed ncu
+    summary, scaled to ``units`` (token-heads for the prefill, sequence-heads
+    for decode), if the counters were taken on the current kernel source; else
+    None."""
+    path = os.path.join(ROOT, "profiles", TRAFFIC_FILES[kernel])
     try:
         with open(path) as f:
             d = json.load(f)
     except Exception:
         return None
-    if d.get("kernel_source_hash") != kernel_source_hash():
+    if d.get("kernel_source_hash") != kernel_source_hash(kernel):
         return None
-    per_unit = d.get("dram_bytes_per_token_head")
+    per_unit = d.get("dram_bytes_per_unit")
     if per_unit is None:
         return None
-    return float(per_unit) * w.T * w.H
+    return float(per_unit) * units
 
 
 class ClockSampler:
@@ -381,7 +395,8 @@ def run_decode(args, world, rank, kda):
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": f"state {B * H * STATE_BYTES / 1e9:.2f} GB exceeds L2; no flush"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak,
+                         "traffic": dram_traffic_from_profile("kda_decode_kernel", B * H),
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
                          "kernel": "kda_decode_kernel", "kernel_ms": kernel_ms,
                          "algorithmic_bytes": alg_bytes},
@@ -460,7 +475,7 @@ def main():
     peak, peak_kind = measured_hbm_peak()
     achieved = alg_bytes / (kernel_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "traffic": dram_traffic_from_profile(w),
+            "frac": achieved / peak, "traffic": dram_traffic_from_profile("kda_fused_kernel", w.T * w.H) if fused else None,
             "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
             else "fallback 6650 GB/s",
             "kernel": "kda_fused_kernel" if fused else "staged kernels",
