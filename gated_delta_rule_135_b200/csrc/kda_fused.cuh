@@ -52,13 +52,15 @@ constexpr int kThreads = 512;
 #ifdef KDA_PHASE_CLOCKS
 constexpr int kPhases = 18;
 __device__ unsigned long long g_phase_cycles[kPhases];
-#define PHASE_MARK(i)                                   \
-    do {                                                \
-        if (threadIdx.x == 0) {                         \
-            const long long now_ = clock64();           \
-            ph_acc[i] += (unsigned long long)(now_ - ph_last); \
-            ph_last = now_;                             \
-        }                                               \
+// thread 0 adds the cycles since the previous mark to a shared-memory slot (no
+// registers held across the kernel, so the instrumented build keeps its allocation)
+#define PHASE_MARK(i)                                                      \
+    do {                                                                   \
+        if (threadIdx.x == 0) {                                            \
+            const long long now_ = clock64();                              \
+            sPh[i] += (unsigned long long)(now_ - sPh[kPhases]);           \
+            sPh[kPhases] = (unsigned long long)now_;                       \
+        }                                                                  \
     } while (0)
 #else
 #define PHASE_MARK(i) do { } while (0)
@@ -77,8 +79,8 @@ constexpr int kF32Pitch = 68;         // fp32 row pitch of A32 / T32 (16-byte al
 constexpr uint32_t A32 = X + 0;       // fp32 [64][68] beta-scaled A  (phases 3-4)
 constexpr uint32_t T32 = X + 17408;   // fp32 [64][68] T = (I + A)^-1 (phase 4)
 constexpr uint32_t T16 = X + 35840;   // fp16 K-major [64][64]        (phases 4-5)
-constexpr uint32_t W16 = X + 0;       // fp16 K-major [64 r][128 c]   (phases 6-7)
-constexpr uint32_t S16 = X + 16384;   // fp16 [128 c][128 v] (MN-major A)  (phase 7)
+constexpr uint32_t S16 = X + 0;       // fp16 [128 c][128 v] (MN-major A)  (phases 5-7; A32/T32 dead)
+constexpr uint32_t W16 = X + 44032;   // fp16 K-major [64 r][128 c]   (phases 6-7; after T16)
 constexpr uint32_t P16 = X + 65536;   // fp16 K-major [64 r][64 i]    (phases 3-8)
 constexpr uint32_t BGK = X + 73728;   // fp16 [64 i][128 c] beta*gamma*k  (MN-major B of W)
 constexpr uint32_t U16 = BGK;         // fp16 K-major [128 v][64 r]   (phase 8; BGK is dead)
@@ -93,9 +95,14 @@ constexpr uint32_t S_TOT = S_GAMMAC + 512;     // fp32 [8][128] per-half-block s
 constexpr uint32_t S_PDIAG = S_TOT + 4096;     // fp32 [2][64] halves of q_r . k_r
 constexpr uint32_t S_ORDER = S_PDIAG + 512;    // int16 [kSortLimit] sequences by length
 constexpr int kSortLimit = 512;
-constexpr uint32_t S_BARS = S_ORDER + 2 * kSortLimit;   // u64 [2]: inputs, mma
-constexpr uint32_t S_TMEM = S_BARS + 16;                // u32 tmem base, u32 abort flag
-constexpr uint32_t SMEM_BYTES = S_TMEM + 16;
+constexpr uint32_t S_BARS = S_ORDER + 2 * kSortLimit;   // u64 [6]: inputs, then one per MMA group
+constexpr uint32_t S_TMEM = S_BARS + 48;                // u32 tmem base, u32 abort flag
+constexpr uint32_t S_PH = S_TMEM + 16;                  // u64 [kPhases + 1] (phase-clock builds)
+#ifdef KDA_PHASE_CLOCKS
+constexpr uint32_t SMEM_BYTES = S_PH + 8 * (kPhases + 1);
+#else
+constexpr uint32_t SMEM_BYTES = S_PH;
+#endif
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;      // + alignment slack
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
@@ -183,12 +190,14 @@ __device__ __forceinline__ void issue_chunk_loads(unsigned char* sm, uint64_t* b
 // Finds the chunk after (k, j) on this CTA's schedule: next chunk of the same
 // unit or chunk 0 of the next non-empty unit.  Returns false if none.
 __device__ bool next_chunk(const Params& p, const int16_t* order, int b, int G, int units, int k,
-                           int64_t j, int64_t nch, int* k_out, int* h_out, int64_t* t0_out) {
+                           int64_t j, int64_t nch, int* k_out, int* h_out, int64_t* t0_out,
+                           int64_t* eos_out) {
     if (j + 1 < nch) {
         const Unit x = decode_unit(p, order, unit_of(k, b, G));
         *k_out = k;
         *h_out = x.h;
         *t0_out = x.bos + (j + 1) * kChunk;
+        *eos_out = x.eos;
         return true;
     }
     for (int kk = k + 1; (int64_t)kk * G < units; ++kk) {
@@ -199,6 +208,7 @@ __device__ bool next_chunk(const Params& p, const int16_t* order, int b, int G, 
             *k_out = kk;
             *h_out = x.h;
             *t0_out = x.bos;
+            *eos_out = x.eos;
             return true;
         }
     }
@@ -206,17 +216,34 @@ __device__ bool next_chunk(const Params& p, const int16_t* order, int b, int G, 
 }
 
 // Waits (bounded) for an mbarrier phase; on expiry records the timeout and
-// raises the CTA-wide abort flag.  Returns true when the CTA should stop.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag) {
-    if (!mbar_wait_bounded(bar, parity)) {
-        record_error(KDA_DEVERR_TIMEOUT);
-        *abort_flag = 1u;
+// raises the CTA-wide abort flag.  Returns true when the CTA should stop.  One
+// thread polls; the others wait at the block barrier, which orders the
+// barrier's completion (and the data it guards) before their accesses.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                              uint64_t* bar2 = nullptr, uint32_t parity2 = 0u) {
+    if (threadIdx.x == 0) {
+        bool ok = mbar_wait_bounded(bar, parity);
+        if (ok && bar2 != nullptr) ok = mbar_wait_bounded(bar2, parity2);
+        if (!ok) {
+            record_error(KDA_DEVERR_TIMEOUT);
+            *abort_flag = 1u;
+        }
     }
     __syncthreads();
     return *abort_flag != 0u;
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
+
+// Warp roles while warps 0-3 solve for T: warps 4-11 compute the next chunk's gate,
+// warps 12-15 prepare its remaining inputs.
+constexpr int kSolveWarps = 4;
+constexpr int kGateWarp0 = 4, kGateThreads = 256;
+constexpr int kPrepWarp0 = 12, kPrepThreads = 128;
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 __device__ __forceinline__ float fast_ex2(float x) {
     float y;
@@ -230,19 +257,102 @@ __device__ __forceinline__ float fast_lg2(float x) {
 }
 // Gate in base-2 units: log2 a = max(-exp(A_log) * log2(1 + 2^x2), lower_bound * log2 e)
 // with x2 = (g + dt_bias) * log2 e, i.e. softplus written as max(x2, 0) + log2(1 + 2^-|x2|).
-__device__ __forceinline__ float gate_log2_decay(float g, float db2, float nexpA, float lb2) {
-    const float x2 = fmaf(g, kLog2e, db2);
-    const float sp2 = fmaxf(x2, 0.f) + fast_lg2(1.f + fast_ex2(-fabsf(x2)));
-    return fmaxf(nexpA * sp2, lb2);
+__device__ __forceinline__ float2 gate_log2_decay2(float2 g, float2 db2, float nexpA, float lb2) {
+    const float2 x2 = __ffma2_rn(g, make_float2(kLog2e, kLog2e), db2);
+    const float2 t = __fadd2_rn(make_float2(1.f, 1.f),
+                                make_float2(fast_ex2(-fabsf(x2.x)), fast_ex2(-fabsf(x2.y))));
+    const float2 sp2 = __fadd2_rn(make_float2(fmaxf(x2.x, 0.f), fmaxf(x2.y, 0.f)),
+                                  make_float2(fast_lg2(t.x), fast_lg2(t.y)));
+    const float2 l = __fmul2_rn(make_float2(nexpA, nexpA), sp2);
+    return make_float2(fmaxf(l.x, lb2), fmaxf(l.y, lb2));
+}
+
+// Packed fp32 pairs (two IEEE round-to-nearest operations per instruction).
+__device__ __forceinline__ float2 mul2(float2 a, float2 b);
+__device__ __forceinline__ float2 add2(float2 a, float2 b);
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    return __fadd2_rn(a, make_float2(-b.x, -b.y));
+}
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float2 a) { return pack_bf16(a.x, a.y); }
+__device__ __forceinline__ uint32_t pack_f16(float2 a) { return pack_f16(a.x, a.y); }
+
+// Gate of one chunk in place (threads gt = 0..255 of the gate warps; lane = channel quad,
+// warp = 8-token octet o): the g tile becomes, per (token r, channel c), the inclusive sum of
+// log2 a over r's octet up to r, and sTot[o][c] the octet total.  Rows r >= L (past the
+// sequence end) get log a = 0; r >= L is uniform across a warp.
+__device__ __forceinline__ void gate_chunk(unsigned char* sm, const Params& p, int h, int L, int gt) {
+    const int c = (gt & 31) * 4, o = gt >> 5;
+    const float nexpA = -expf(p.A_log[h]);
+    const float lb2 = p.lower_bound * kLog2e;
+    const float4 db = *reinterpret_cast<const float4*>(p.dt_bias + h * kHeadDim + c);
+    const float2 l2e = make_float2(kLog2e, kLog2e);
+    const float2 db01 = mul2(make_float2(db.x, db.y), l2e), db23 = mul2(make_float2(db.z, db.w), l2e);
+    float* gbuf = reinterpret_cast<float*>(sm + IN_G);
+    float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = o * 8 + i;
+        float4* gp = reinterpret_cast<float4*>(gbuf + r * kHeadDim + c);
+        if (r < L) {
+            const float4 gv = *gp;
+            a01 = add2(a01, gate_log2_decay2(make_float2(gv.x, gv.y), db01, nexpA, lb2));
+            a23 = add2(a23, gate_log2_decay2(make_float2(gv.z, gv.w), db23, nexpA, lb2));
+        }
+        *gp = make_float4(a01.x, a01.y, a23.x, a23.y);
+    }
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(sm + S_TOT) + o * kHeadDim + c) =
+        make_float4(a01.x, a01.y, a23.x, a23.y);
+}
+
+// The rest of a chunk's preparation (threads pt = 0..127 of the prep warps): beta of its
+// rows (0 past the sequence end) and k = q = v = 0 on rows r >= L.
+__device__ __forceinline__ void prep_chunk(unsigned char* sm, const Params& p, int h, int64_t t0, int L,
+                                           int pt) {
+    float* sBeta = reinterpret_cast<float*>(sm + S_BETA);
+    if (pt < kChunk) sBeta[pt] = pt < L ? p.beta[(t0 + pt) * p.H + h] : 0.f;
+    for (int e = L * 16 + pt; e < kChunk * 16; e += kPrepThreads) {
+        const uint32_t o = (uint32_t)e * 16u;   // row e / 16, 16-byte piece e % 16
+        *reinterpret_cast<uint4*>(sm + IN_Q + o) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(sm + IN_K + o) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(sm + IN_V + o) = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// Warps 4-15: wait (bounded) for the chunk's inputs, then gate / prepare it.  Returns
+// false on a timeout (the abort flag is raised).
+__device__ __forceinline__ bool stage_next_chunk(unsigned char* sm, const Params& p, uint64_t* bar_in,
+                                                 uint32_t parity, volatile uint32_t* abort_flag, int h,
+                                                 int64_t t0, int L) {
+    const int warp = threadIdx.x >> 5;
+    if (warp < kGateWarp0) return true;
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar_in, parity);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    if (!ok) {
+        if ((threadIdx.x & 31) == 0) {
+            record_error(KDA_DEVERR_TIMEOUT);
+            *abort_flag = 1u;
+        }
+        return false;
+    }
+    if (warp < kPrepWarp0) gate_chunk(sm, p, h, L, threadIdx.x - kGateWarp0 * 32);
+    else prep_chunk(sm, p, h, t0, L, threadIdx.x - kPrepWarp0 * 32);
+    return true;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                  const Params p) {
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // 1024-byte aligned base, derived by pointer arithmetic so that every access
+    // below stays in the shared state space (ld/st.shared, 32-bit addresses)
+    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // TMEM access: warp w reads lane quarter (w % 4); `sub` splits columns between the four
     // warps that share a quarter
@@ -256,15 +366,20 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float* sTot = reinterpret_cast<float*>(sm + S_TOT);
     float* sPdiag = reinterpret_cast<float*>(sm + S_PDIAG);
     int16_t* sOrder = reinterpret_cast<int16_t*>(sm + S_ORDER);
+    // one barrier per MMA commit group; each completes once per chunk:
+    //   ap = A/P, w = W (U~ follows uncommitted), u = U (O1 follows), o = O2, s = S update
     uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + S_BARS);
-    uint64_t* bar_mma = bar_in + 1;
+    uint64_t* bar_ap = bar_in + 1;
+    uint64_t* bar_w = bar_in + 2;
+    uint64_t* bar_u = bar_in + 3;
+    uint64_t* bar_o = bar_in + 4;
+    uint64_t* bar_s = bar_in + 5;
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + S_TMEM);
     volatile uint32_t* sAbort = sTmem + 1;
 
     // ---- set-up: barriers, TMEM, length order ----
     if (tid == 0) {
-        mbar_init(bar_in, 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < 6; ++i) mbar_init(bar_in + i, 1);
         mbar_init_fence();
         *sAbort = 0u;
     }
@@ -292,22 +407,40 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     fence_after_sync();
     const uint32_t tbase = *sTmem;
 #ifdef KDA_PHASE_CLOCKS
-    unsigned long long ph_acc[kPhases] = {};
-    long long ph_last = clock64();
+    volatile unsigned long long* sPh = reinterpret_cast<volatile unsigned long long*>(sm + S_PH);
+    if (tid == 0) {
+        for (int i = 0; i < kPhases; ++i) sPh[i] = 0ull;
+        sPh[kPhases] = (unsigned long long)clock64();
+    }
 #endif
 
-    uint32_t in_parity = 0, mma_parity = 0;
+    // barrier bookkeeping in one word (uniform across the CTA): bit i = phase parity of
+    // barrier i (0 inputs, 1 A/P, 2 W, 3 U, 4 O, 5 S); bit 8 + i = commit issued on barrier
+    // i and not yet waited for
+    enum : uint32_t { B_IN = 0, B_AP = 1, B_W = 2, B_U = 3, B_O = 4, B_S = 5 };
+    uint32_t bk = 0u;
+    auto par = [&](uint32_t b) { return (bk >> b) & 1u; };
+    auto pending = [&](uint32_t b) { return ((bk >> (8 + b)) & 1u) != 0u; };
+    auto issued = [&](uint32_t b) { bk |= 1u << (8 + b); };
+    auto waited = [&](uint32_t b) { bk = (bk ^ (1u << b)) & ~(1u << (8 + b)); };
     bool in_flight = false;
-    float beta_next = 0.f;   // beta of the chunk in flight (threads 0-63)
+    bool aborted = false;
 
-    // first load
+    // first chunk: load, then gate and prepare it (warps 4-15)
     {
         int k1, h1;
-        int64_t t1;
-        if (next_chunk(p, sOrder, b, G, units, -1, 0, 0, &k1, &h1, &t1)) {
+        int64_t t1, e1;
+        if (next_chunk(p, sOrder, b, G, units, -1, 0, 0, &k1, &h1, &t1, &e1)) {
             if (tid == 0) issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
-            if (tid < kChunk && t1 + tid < p.total_tokens) beta_next = p.beta[(t1 + tid) * H + h1];
             in_flight = true;
+            const int L1 = (int)(e1 - t1 < kChunk ? e1 - t1 : kChunk);
+            stage_next_chunk(sm, p, bar_in, par(B_IN), sAbort, h1, t1, L1);
+            __syncthreads();
+            if (*sAbort != 0u) aborted = true;
+            else {
+                waited(B_IN);
+                in_flight = false;
+            }
         }
     }
 
@@ -325,7 +458,6 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // state / TMEM mapping: lane quarter -> rows, sub -> 32-column quarter
     const int c_row = quarter * 32 + lane;
 
-    bool aborted = false;
     for (int k = 0; (int64_t)k * G < units && !aborted; ++k) {
         const int u = unit_of(k, b, G);
         if (u >= units) continue;
@@ -364,17 +496,12 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_wait_st();
         fence_before_sync();
 
-        // per-unit gate constants of this thread's two channels (base-2 units)
-        const float nexpA = -expf(p.A_log[h]);
-        const float lb2 = p.lower_bound * kLog2e;
-        const float db2_0 = p.dt_bias[h * kHeadDim + c0] * kLog2e;
-        const float db2_1 = p.dt_bias[h * kHeadDim + c0 + 1] * kLog2e;
 
         const int64_t nch = (x.eos - x.bos + kChunk - 1) / kChunk;
         // chunk 0 of the next non-empty unit of this CTA (global reads once per unit)
         int kn = 0, hn = 0;
-        int64_t tn = 0;
-        const bool unit_has_next = next_chunk(p, sOrder, b, G, units, k, nch - 1, nch, &kn, &hn, &tn);
+        int64_t tn = 0, en = 0;
+        const bool unit_has_next = next_chunk(p, sOrder, b, G, units, k, nch - 1, nch, &kn, &hn, &tn, &en);
         for (int64_t j = 0; j < nch; ++j) {
             const int64_t t0 = x.bos + j * kChunk;
             const int L = (int)(x.eos - t0 < kChunk ? x.eos - t0 : kChunk);
@@ -385,64 +512,55 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const bool has_next = last ? unit_has_next : true;
             const int h1 = last ? hn : h;
             const int64_t t1 = last ? tn : t0 + kChunk;
-            if (tid < kChunk) sBeta[tid] = tid < L ? beta_next : 0.f;
-            if (wait_or_abort(bar_in, in_parity, sAbort)) { aborted = true; break; }
+            const int64_t e1 = last ? en : x.eos;
+            const int L1 = (int)(e1 - t1 < kChunk ? e1 - t1 : kChunk);
+            // this chunk was gated and prepared while the previous one solved for T; the
+            // previous chunk's S update must have finished reading KH / U16
+            if (pending(B_S)) {
+                if (wait_or_abort(bar_s, par(B_S), sAbort)) {
+                    aborted = true;
+                    break;
+                }
+                waited(B_S);
+            }
             PHASE_MARK(1);
-            in_parity ^= 1u;
-            in_flight = false;
-
-            float G0[8], G1[8];   // inclusive cumsum of log2 a over this thread's 8 tokens
+            float2 Gc[8];   // inclusive sum of log2 a over this thread's octet (channel pair)
             {
-                float a0 = 0.f, a1 = 0.f;
                 const float* gin = reinterpret_cast<const float*>(sm + IN_G);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int r = rbase + i;
-                    const float2 gv = *reinterpret_cast<const float2*>(gin + r * kHeadDim + c0);
-                    const bool ok = r < L;
-                    const float l0 = gate_log2_decay(gv.x, db2_0, nexpA, lb2);
-                    const float l1 = gate_log2_decay(gv.y, db2_1, nexpA, lb2);
-                    a0 += ok ? l0 : 0.f;
-                    a1 += ok ? l1 : 0.f;
-                    G0[i] = a0;
-                    G1[i] = a1;
-                }
-                sTot[(blk * 2 + hf) * kHeadDim + c0] = a0;
-                sTot[(blk * 2 + hf) * kHeadDim + c0 + 1] = a1;
+                for (int i = 0; i < 8; ++i)
+                    Gc[i] = *reinterpret_cast<const float2*>(gin + (rbase + i) * kHeadDim + c0);
             }
-            __syncthreads();
             PHASE_MARK(12);
             {
                 // block sums (16-token blocks) from the half-block sums
-                float tot0[4], tot1[4], half0 = 0.f, half1 = 0.f;
+                float2 tot[4], half = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int bb = 0; bb < 4; ++bb) {
-                    const float x00 = sTot[(2 * bb) * kHeadDim + c0], x01 = sTot[(2 * bb + 1) * kHeadDim + c0];
-                    const float x10 = sTot[(2 * bb) * kHeadDim + c0 + 1], x11 = sTot[(2 * bb + 1) * kHeadDim + c0 + 1];
-                    tot0[bb] = x00 + x01;
-                    tot1[bb] = x10 + x11;
-                    if (bb == blk && hf == 1) { half0 = x00; half1 = x10; }
+                    const float2 x0 = *reinterpret_cast<const float2*>(sTot + (2 * bb) * kHeadDim + c0);
+                    const float2 x1 = *reinterpret_cast<const float2*>(sTot + (2 * bb + 1) * kHeadDim + c0);
+                    tot[bb] = add2(x0, x1);
+                    if (bb == blk && hf == 1) half = x0;
                 }
-                float Ts0 = 0.f, Ts1 = 0.f, after0 = 0.f, after1 = 0.f;
+                float2 Ts = make_float2(0.f, 0.f), after = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int bb = 0; bb < 4; ++bb) {
-                    if (bb < blk) { Ts0 += tot0[bb]; Ts1 += tot1[bb]; }
-                    if (bb > blk) { after0 += tot0[bb]; after1 += tot1[bb]; }
+                    if (bb < blk) Ts = add2(Ts, tot[bb]);
+                    if (bb > blk) after = add2(after, tot[bb]);
                 }
-                auto pick4 = [](const float (&a)[4], int i) {
+                auto pick4 = [](const float2 (&a)[4], int i) {
                     return i == 0 ? a[0] : (i == 1 ? a[1] : (i == 2 ? a[2] : a[3]));
                 };
-                const float tb0 = pick4(tot0, blk), tb1 = pick4(tot1, blk);
-                const float eTs0 = fast_ex2(Ts0), eTs1 = fast_ex2(Ts1);        // gamma at the block start
-                const float invB0 = fast_ex2(-tb0), invB1 = fast_ex2(-tb1);    // e^{Gamma_s - Gamma_e} >= 1
-                const float eA0 = fast_ex2(after0), eA1 = fast_ex2(after1);    // e^{Gamma_last - Gamma_e}
-                float F2_0 = 0.f, F2_1 = 0.f, F3_0 = 0.f, F3_1 = 0.f;
-                if (blk <= 1) { F2_0 = fast_ex2(pick4(tot0, blk + 1)); F2_1 = fast_ex2(pick4(tot1, blk + 1)); }
-                if (blk == 0) { F3_0 = fast_ex2(tot0[1] + tot0[2]); F3_1 = fast_ex2(tot1[1] + tot1[2]); }
-                if (blk == 0 && hf == 0) {
-                    sGammaC[c0] = fast_ex2(tb0 + after0);
-                    sGammaC[c0 + 1] = fast_ex2(tb1 + after1);
-                }
+                auto ex2v = [](float2 x) { return make_float2(fast_ex2(x.x), fast_ex2(x.y)); };
+                const float2 tb = pick4(tot, blk);
+                const float2 eTs = ex2v(Ts);                                  // gamma at the block start
+                const float2 invB = ex2v(make_float2(-tb.x, -tb.y));          // e^{Gamma_s - Gamma_e} >= 1
+                const float2 eA = ex2v(after);                                // e^{Gamma_last - Gamma_e}
+                float2 F2 = make_float2(0.f, 0.f), F3 = make_float2(0.f, 0.f);
+                if (blk <= 1) F2 = ex2v(pick4(tot, blk + 1));
+                if (blk == 0) F3 = ex2v(add2(tot[1], tot[2]));
+                if (blk == 0 && hf == 0)
+                    *reinterpret_cast<float2*>(sGammaC + c0) = ex2v(add2(tb, after));
                 const uint32_t* kin = reinterpret_cast<const uint32_t*>(sm + IN_K);
                 const uint32_t* qin = reinterpret_cast<const uint32_t*>(sm + IN_Q);
                 const uint32_t* vin = reinterpret_cast<const uint32_t*>(sm + IN_V);
@@ -453,38 +571,35 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int r = rbase + i;
-                    const bool ok = r < L;
                     const int idx = (r * kHeadDim + c0) >> 1;
-                    kwv[i] = ok ? kin[idx] : 0u;
-                    qwv[i] = ok ? qin[idx] : 0u;
-                    vwv[i] = ok ? vin[idx] : 0u;
+                    kwv[i] = kin[idx];
+                    qwv[i] = qin[idx];
+                    vwv[i] = vin[idx];
                     bev[i] = sBeta[r];
                 }
                 // (a) A/P MMA operands (+ K-hat, gamma*q which need the same factors), then the
                 //     MMA is issued; (b) beta*gamma*k and beta*v while it runs
-                float g0v[8], g1v[8], pd[8];
+                float2 gv[8];
+                float pd[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const uint32_t kw = kwv[i], qw = qwv[i];
-                    const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
-                    const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
-                    const float ls0 = half0 + G0[i], ls1 = half1 + G1[i];             // Gamma_r - Gamma_s (log2)
-                    const float R0 = fast_ex2(ls0), R1 = fast_ex2(ls1);                 // e^{Gamma_r - Gamma_s}
-                    const float E0 = fast_ex2(tb0 - ls0), E1 = fast_ex2(tb1 - ls1);     // e^{Gamma_e - Gamma_r}
-                    const float kE0 = k0 * E0, kE1 = k1 * E1;
+                    const float2 kk = bf16x2_to_float2(kwv[i]), qq = bf16x2_to_float2(qwv[i]);
+                    const float2 ls = add2(half, Gc[i]);                       // Gamma_r - Gamma_s (log2)
+                    const float2 R = ex2v(ls);                                 // e^{Gamma_r - Gamma_s}
+                    const float2 E = ex2v(sub2(tb, ls));                       // e^{Gamma_e - Gamma_r}
+                    const float2 kE = mul2(kk, E);
                     const uint32_t ro = (uint32_t)i * 128u + ((chk ^ (uint32_t)i) << 4);
-                    st_u32(sm, AP_A + off128 + ro, pack_bf16(k0 * R0, k1 * R1));
-                    st_u32(sm, AP_A + off128 + 64u * 128u + ro, pack_bf16(q0 * R0, q1 * R1));
-                    st_u32(sm, AP_B + off160 + ro, pack_bf16(kE0 * invB0, kE1 * invB1));
-                    if (blk <= 2) st_u32(sm, AP_B + off160 + 64u * 128u + ro, pack_bf16(kE0, kE1));
-                    if (blk <= 1) st_u32(sm, AP_B + off160 + 112u * 128u + ro, pack_bf16(kE0 * F2_0, kE1 * F2_1));
-                    if (blk == 0) st_u32(sm, AP_B + off160 + 144u * 128u + ro, pack_bf16(kE0 * F3_0, kE1 * F3_1));
-                    st_u32(sm, KH + off64 + ro, pack_f16(kE0 * eA0, kE1 * eA1));
-                    const float g0 = R0 * eTs0, g1 = R1 * eTs1;                          // gamma_r
-                    st_u32(sm, GQ + off64 + ro, pack_f16(q0 * g0, q1 * g1));
-                    g0v[i] = g0;
-                    g1v[i] = g1;
-                    pd[i] = fmaf(q0, k0, q1 * k1);
+                    st_u32(sm, AP_A + off128 + ro, pack_bf16(mul2(kk, R)));
+                    st_u32(sm, AP_A + off128 + 64u * 128u + ro, pack_bf16(mul2(qq, R)));
+                    st_u32(sm, AP_B + off160 + ro, pack_bf16(mul2(kE, invB)));
+                    if (blk <= 2) st_u32(sm, AP_B + off160 + 64u * 128u + ro, pack_bf16(kE));
+                    if (blk <= 1) st_u32(sm, AP_B + off160 + 112u * 128u + ro, pack_bf16(mul2(kE, F2)));
+                    if (blk == 0) st_u32(sm, AP_B + off160 + 144u * 128u + ro, pack_bf16(mul2(kE, F3)));
+                    st_u32(sm, KH + off64 + ro, pack_f16(mul2(kE, eA)));
+                    const float2 g = mul2(R, eTs);                             // gamma_r
+                    st_u32(sm, GQ + off64 + ro, pack_f16(mul2(qq, g)));
+                    gv[i] = g;
+                    pd[i] = fmaf(qq.x, kk.x, qq.y * kk.y);
                 }
                 fence_proxy_async();
                 __syncthreads();
@@ -495,17 +610,16 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     for (int ks = 0; ks < 8; ++ks)
                         mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
                                 ks > 0 ? 1u : 0u);
-                    mma_commit(bar_mma);
+                    mma_commit(bar_ap);
                 }
+                issued(B_AP);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const uint32_t kw = kwv[i], vw = vwv[i];
-                    const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
-                    const float v0 = __uint_as_float(vw << 16), v1 = __uint_as_float(vw & 0xFFFF0000u);
-                    const float be = bev[i];
+                    const float2 kk = bf16x2_to_float2(kwv[i]), vv = bf16x2_to_float2(vwv[i]);
+                    const float2 be = make_float2(bev[i], bev[i]);
                     const uint32_t ro = (uint32_t)i * 128u + ((chk ^ (uint32_t)i) << 4);
-                    st_u32(sm, BGK + off64 + ro, pack_f16(be * k0 * g0v[i], be * k1 * g1v[i]));
-                    st_u32(sm, BV + off64 + ro, pack_f16(be * v0, be * v1));
+                    st_u32(sm, BGK + off64 + ro, pack_f16(mul2(mul2(be, kk), gv[i])));
+                    st_u32(sm, BV + off64 + ro, pack_f16(mul2(be, vv)));
                 }
                 PHASE_MARK(13);
                 // reduce pd over the 32 lanes for the 8 tokens at once (transposing butterfly);
@@ -543,14 +657,10 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             PHASE_MARK(2);
 
             // inputs consumed: prefetch the next chunk (the A/P MMA is already running)
-            {
-                in_flight = has_next;
-                if (tid == 0 && in_flight) issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
-                if (in_flight && tid < kChunk && t1 + tid < p.total_tokens)
-                    beta_next = p.beta[(t1 + tid) * H + h1];
-            }
-            if (wait_or_abort(bar_mma, mma_parity, sAbort)) { aborted = true; break; }
-            mma_parity ^= 1u;
+            in_flight = has_next;
+            if (tid == 0 && in_flight) issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
+            if (wait_or_abort(bar_ap, par(B_AP), sAbort)) { aborted = true; break; }
+            waited(B_AP);
             fence_after_sync();
             PHASE_MARK(3);
 
@@ -594,9 +704,13 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const float be = sBeta[r];
                     float* a32 = reinterpret_cast<float*>(sm + A32) + r * kF32Pitch + J * 16;
 #pragma unroll
-                    for (int i = 0; i < 16; i += 4)
-                        *reinterpret_cast<float4*>(a32 + i) =
-                            make_float4(be * row[i], be * row[i + 1], be * row[i + 2], be * row[i + 3]);
+                    const float2 be2 = make_float2(be, be);
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4) {
+                        const float2 lo2 = mul2(be2, make_float2(row[i], row[i + 1]));
+                        const float2 hi2 = mul2(be2, make_float2(row[i + 2], row[i + 3]));
+                        *reinterpret_cast<float4*>(a32 + i) = make_float4(lo2.x, lo2.y, hi2.x, hi2.y);
+                    }
                 } else {
 #pragma unroll
                     for (int c = 0; c < 2; ++c)
@@ -609,8 +723,10 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             __syncthreads();
             PHASE_MARK(4);
 
-            // ================= phase 4: T = (I + A)^-1 =================
-            {
+            // ================= phase 4: T = (I + A)^-1 on warps 0-3 =================
+            // Meanwhile warps 4-11 gate the next chunk and warps 12-15 prepare its other
+            // inputs (its loads were issued after phase 1).
+            if (warp < kSolveWarps) {
                 const float* a32 = reinterpret_cast<const float*>(sm + A32);
                 float* t32 = reinterpret_cast<float*>(sm + T32);
                 auto Ab = [&](int I, int J) { return a32 + 16 * I * kF32Pitch + 16 * J; };
@@ -624,7 +740,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     st_v4(sm, T16 + sw128_chunk_off(16 * I + rr, 2 * J + ch, 64), pack_f16(lo4.x, lo4.y),
                           pack_f16(lo4.z, lo4.w), pack_f16(hi4.x, hi4.y), pack_f16(hi4.z, hi4.w));
                 };
-                if (tid < 64) {   // diagonal 16 x 16 blocks by forward substitution, one column each
+                if (warp < 2) {   // diagonal 16 x 16 blocks by forward substitution, one column each
                     const int bI = tid >> 4, jc = tid & 15, o = bI * 16;
                     float xv[16];
 #pragma unroll
@@ -637,16 +753,8 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
 #pragma unroll
                     for (int rr = 0; rr < 16; ++rr) t32[(o + rr) * kF32Pitch + o + jc] = xv[rr];
-                } else if (tid >= 128) {
-                    // zero fp16 blocks above the diagonal: 6 blocks x 32 chunks
-                    for (int e = tid - 128; e < 6 * 32; e += kThreads - 128) {
-                        const int blkid = e >> 5, c = e & 31;
-                        const int I = blkid < 3 ? 0 : (blkid < 5 ? 1 : 2);
-                        const int J = blkid < 3 ? blkid + 1 : (blkid < 5 ? blkid - 1 : 3);
-                        st_v4(sm, T16 + sw128_chunk_off(16 * I + (c >> 1), 2 * J + (c & 1), 64), 0u, 0u, 0u, 0u);
-                    }
                 }
-                __syncthreads();
+                named_bar_sync(1, kSolveWarps * 32);
                 PHASE_MARK(14);
                 // Off-diagonal blocks by recursive doubling on 16 x 16 blocks; products on the
                 // warp tensor-core path (mma.sync, fp16 operands, fp32 accumulation -- T is
@@ -655,7 +763,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 //   T10 = -T11 A10 T00, T32 = -T33 A32 T22, T21 = -T22 A21 T11,
                 //   X20 = A20 T00 + A21 T10, X30 = A30 T00 + A31 T10,
                 //   T20 = -T22 X20, T31 = -(T32 A21 T11 + T33 A31 T11), T30 = -(T32 X20 + T33 X30).
-                float acc[2][4] = {};
+                float acc[2][4] = {}, acc2[2][4] = {};
                 // step A: T10, T32 (two products each); X21 = A21 T11, X31 = A31 T11;
                 //         partial X20 = A20 T00, X30 = A30 T00; fp16 copies of the diagonal blocks
                 if (warp == 0 || warp == 1) {
@@ -663,30 +771,30 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     warpmma::mm16_acc_h(Ab(Ii, Jj), kF32Pitch, Tb(Jj, Jj), kF32Pitch, acc);
                     warpmma::store16(Tb(Jj, Ii), kF32Pitch, acc, 1.f);
                     __syncwarp();
-                    float acc2[2][4] = {};
-                    warpmma::mm16_acc_h(Tb(Ii, Ii), kF32Pitch, Tb(Jj, Ii), kF32Pitch, acc2);
-                    warpmma::store16(Tb(Ii, Jj), kF32Pitch, acc2, -1.f);
+                    float a3[2][4] = {};
+                    warpmma::mm16_acc_h(Tb(Ii, Ii), kF32Pitch, Tb(Jj, Ii), kF32Pitch, a3);
+                    warpmma::store16(Tb(Ii, Jj), kF32Pitch, a3, -1.f);
                     __syncwarp();
                     to_t16(Ii, Jj);
                 } else if (warp == 2) {
                     warpmma::mm16_acc_h(Ab(2, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc);
                     warpmma::store16(Tb(1, 2), kF32Pitch, acc, 1.f);           // X21
-                    float acc2[2][4] = {};
                     warpmma::mm16_acc_h(Ab(3, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc2);
                     warpmma::store16(Tb(1, 3), kF32Pitch, acc2, 1.f);          // X31
-                } else if (warp == 3) {
-                    warpmma::mm16_acc_h(Ab(2, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);   // X20 partial
-                } else if (warp == 4) {
-                    warpmma::mm16_acc_h(Ab(3, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);   // X30 partial
-                } else if (warp < 8) {
-                    for (int d = warp - 5; d < 4; d += 3) to_t16(d, d);               // diagonal blocks
+                } else {
+                    warpmma::mm16_acc_h(Ab(2, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);    // X20 partial
+                    warpmma::mm16_acc_h(Ab(3, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc2);   // X30 partial
+#pragma unroll
+                    for (int d = 0; d < 4; ++d) to_t16(d, d);                            // diagonal blocks
                 }
-                __syncthreads();
+                named_bar_sync(1, kSolveWarps * 32);
                 PHASE_MARK(15);
                 // step B: X20, X30 complete; T21 = -T22 X21; P31a = T32 X21, P31b = T33 X31
-                if (warp == 3 || warp == 4) {
-                    warpmma::mm16_acc_h(Ab(warp - 1, 1), kF32Pitch, Tb(1, 0), kF32Pitch, acc);
-                    warpmma::store16(Tb(0, warp - 1), kF32Pitch, acc, 1.f);   // X20 -> (0,2), X30 -> (0,3)
+                if (warp == 3) {
+                    warpmma::mm16_acc_h(Ab(2, 1), kF32Pitch, Tb(1, 0), kF32Pitch, acc);
+                    warpmma::store16(Tb(0, 2), kF32Pitch, acc, 1.f);            // X20 -> (0,2)
+                    warpmma::mm16_acc_h(Ab(3, 1), kF32Pitch, Tb(1, 0), kF32Pitch, acc2);
+                    warpmma::store16(Tb(0, 3), kF32Pitch, acc2, 1.f);           // X30 -> (0,3)
                 } else if (warp == 0) {
                     float a2[2][4] = {};
                     warpmma::mm16_acc_h(Tb(2, 2), kF32Pitch, Tb(1, 2), kF32Pitch, a2);
@@ -697,12 +805,12 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     float a2[2][4] = {};
                     warpmma::mm16_acc_h(Tb(3, 2), kF32Pitch, Tb(1, 2), kF32Pitch, a2);
                     warpmma::store16(Tb(0, 1), kF32Pitch, a2, 1.f);            // P31a -> (0,1)
-                } else if (warp == 2) {
+                } else {
                     float a2[2][4] = {};
                     warpmma::mm16_acc_h(Tb(3, 3), kF32Pitch, Tb(1, 3), kF32Pitch, a2);
                     warpmma::store16(Tb(2, 3), kF32Pitch, a2, 1.f);            // P31b -> (2,3)
                 }
-                __syncthreads();
+                named_bar_sync(1, kSolveWarps * 32);
                 PHASE_MARK(16);
                 // step C: T20 = -T22 X20; P30a = T32 X20, P30b = T33 X30; T31 = -(P31a + P31b)
                 if (warp == 0) {
@@ -719,7 +827,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     float a2[2][4] = {};
                     warpmma::mm16_acc_h(Tb(3, 3), kF32Pitch, Tb(0, 3), kF32Pitch, a2);
                     warpmma::store16(Tb(1, 3), kF32Pitch, a2, 1.f);            // P30b -> (1,3)
-                } else if (warp == 3) {
+                } else {
                     for (int e = lane; e < 64; e += 32) {                      // T31 = -(P31a + P31b)
                         const int rr = e >> 2, c4 = (e & 3) * 4;
                         const float4 x1 = *reinterpret_cast<const float4*>(Tb(0, 1) + rr * kF32Pitch + c4);
@@ -730,7 +838,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     __syncwarp();
                     to_t16(3, 1);
                 }
-                __syncthreads();
+                named_bar_sync(1, kSolveWarps * 32);
                 PHASE_MARK(17);
                 // step D: T30 = -(P30a + P30b)
                 if (warp == 0) {
@@ -744,13 +852,32 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     __syncwarp();
                     to_t16(3, 0);
                 }
+            } else {
+                if (warp >= kPrepWarp0) {
+                    // zero fp16 blocks above the diagonal: 6 blocks x 32 chunks
+                    for (int e = tid - kPrepWarp0 * 32; e < 6 * 32; e += kPrepThreads) {
+                        const int blkid = e >> 5, c = e & 31;
+                        const int I = blkid < 3 ? 0 : (blkid < 5 ? 1 : 2);
+                        const int J = blkid < 3 ? blkid + 1 : (blkid < 5 ? blkid - 1 : 3);
+                        st_v4(sm, T16 + sw128_chunk_off(16 * I + (c >> 1), 2 * J + (c & 1), 64), 0u, 0u, 0u, 0u);
+                    }
+                }
+                if (has_next) stage_next_chunk(sm, p, bar_in, par(B_IN), sAbort, h1, t1, L1);
             }
             fence_proxy_async();
             fence_before_sync();
             __syncthreads();
             PHASE_MARK(5);
+            if (*sAbort != 0u) {
+                aborted = true;
+                break;
+            }
+            if (has_next) {
+                waited(B_IN);
+                in_flight = false;
+            }
 
-            // ================= phase 5: W and U~^T MMAs =================
+            // ================= phase 5: W and U~^T MMAs; state copy while they run =================
             if (tid == 0) {
                 fence_after_sync();
                 const uint32_t t16 = smem_u32(sm + T16), bgk = smem_u32(sm + BGK), bv = smem_u32(sm + BV);
@@ -758,16 +885,49 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 for (int ks = 0; ks < 4; ++ks)
                     mma_f16(tbase + TM_W, desc_kmajor(t16, 64, ks), desc_mnmajor(bgk, 64, ks), IDESC_W,
                             ks > 0 ? 1u : 0u);
+                mma_commit(bar_w);
+                // U~^T needs no commit of its own: the U^T MMA that accumulates onto it is
+                // issued later by this thread, and one thread's MMAs execute in order
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_f16(tbase + TM_UT, desc_mnmajor(bv, 64, ks), desc_kmajor(t16, 64, ks), IDESC_UT,
                             ks > 0 ? 1u : 0u);
-                mma_commit(bar_mma);
             }
-            if (wait_or_abort(bar_mma, mma_parity, sAbort)) { aborted = true; break; }
-            mma_parity ^= 1u;
-            fence_after_sync();
+            issued(B_W);
             PHASE_MARK(6);
+            {
+                // S (TMEM, fp32) -> fp16 smem operand; S <- Diag(gamma_last) S in TMEM.  The
+                // previous chunk's S update finished before this chunk's inputs were consumed.
+                const float gC = sGammaC[c_row];
+                uint32_t v[2][16];
+                tmem_ld16(taddr(tbase, quarter, TM_S + sub * 32), v[0]);
+                tmem_ld16(taddr(tbase, quarter, TM_S + sub * 32 + 16), v[1]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const uint32_t v0 = sub * 32 + cc * 16;
+                    uint32_t w[8];
+#pragma unroll
+                    for (int q2 = 0; q2 < 8; ++q2)
+                        w[q2] = pack_f16(__uint_as_float(v[cc][2 * q2]), __uint_as_float(v[cc][2 * q2 + 1]));
+                    st_v4(sm, S16 + sw128_chunk_off(c_row, v0 / 8, 128), w[0], w[1], w[2], w[3]);
+                    st_v4(sm, S16 + sw128_chunk_off(c_row, v0 / 8 + 1, 128), w[4], w[5], w[6], w[7]);
+#pragma unroll
+                    for (int q2 = 0; q2 < 16; q2 += 2) {
+                        const float2 d = mul2(make_float2(__uint_as_float(v[cc][q2]), __uint_as_float(v[cc][q2 + 1])),
+                                              make_float2(gC, gC));
+                        v[cc][q2] = __float_as_uint(d.x);
+                        v[cc][q2 + 1] = __float_as_uint(d.y);
+                    }
+                    tmem_st16(taddr(tbase, quarter, TM_S + v0), v[cc]);
+                }
+                tmem_wait_st();
+            }
+            fence_before_sync();
+            if (wait_or_abort(bar_w, par(B_W), sAbort)) { aborted = true; break; }
+            waited(B_W);
+            fence_after_sync();
+            PHASE_MARK(7);
 
             // ================= phase 6: W -> fp16 smem =================
             {
@@ -790,51 +950,30 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                 }
             }
-
-            // ================= phase 7: S copy + decay, U and O MMAs =================
-            {
-                const float gC = sGammaC[c_row];
-                uint32_t v[2][16];
-                tmem_ld16(taddr(tbase, quarter, TM_S + sub * 32), v[0]);
-                tmem_ld16(taddr(tbase, quarter, TM_S + sub * 32 + 16), v[1]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const uint32_t v0 = sub * 32 + cc * 16;
-                    uint32_t w[8];
-#pragma unroll
-                    for (int q2 = 0; q2 < 8; ++q2)
-                        w[q2] = pack_f16(__uint_as_float(v[cc][2 * q2]), __uint_as_float(v[cc][2 * q2 + 1]));
-                    st_v4(sm, S16 + sw128_chunk_off(c_row, v0 / 8, 128), w[0], w[1], w[2], w[3]);
-                    st_v4(sm, S16 + sw128_chunk_off(c_row, v0 / 8 + 1, 128), w[4], w[5], w[6], w[7]);
-#pragma unroll
-                    for (int q2 = 0; q2 < 16; ++q2) v[cc][q2] = __float_as_uint(__uint_as_float(v[cc][q2]) * gC);
-                    tmem_st16(taddr(tbase, quarter, TM_S + v0), v[cc]);
-                }
-                tmem_wait_st();
-            }
             fence_proxy_async();
             fence_before_sync();
             __syncthreads();
-            PHASE_MARK(7);
+
+            // ================= phase 7: U and O MMAs =================
             if (tid == 0) {
                 fence_after_sync();
                 const uint32_t s16 = smem_u32(sm + S16), w16 = smem_u32(sm + W16), gq = smem_u32(sm + GQ);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     mma_f16(tbase + TM_UT, desc_mnmajor(s16, 128, ks), desc_kmajor(w16, 64, ks), IDESC_U, 1u);
+                mma_commit(bar_u);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     mma_f16(tbase + TM_OT, desc_mnmajor(s16, 128, ks), desc_kmajor(gq, 64, ks), IDESC_O1,
                             ks > 0 ? 1u : 0u);
-                mma_commit(bar_mma);
             }
-            if (wait_or_abort(bar_mma, mma_parity, sAbort)) { aborted = true; break; }
-            mma_parity ^= 1u;
+            issued(B_U);
+            if (wait_or_abort(bar_u, par(B_U), sAbort)) { aborted = true; break; }
+            waited(B_U);
             fence_after_sync();
             PHASE_MARK(8);
 
-            // ================= phase 8: U -> fp16, S and O MMAs =================
+            // ================= phase 8: U -> fp16, O and S MMAs =================
             {
                 const int v_row = c_row;   // lanes of U^T are value columns
                 uint32_t v[16];
@@ -854,16 +993,21 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (tid == 0) {
                 fence_after_sync();
                 const uint32_t kh = smem_u32(sm + KH), u16 = smem_u32(sm + U16), p16 = smem_u32(sm + P16);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tbase + TM_S, desc_mnmajor(kh, 64, ks), desc_kmajor(u16, 128, ks), IDESC_S, 1u);
+                // O first (the output waits for it), then the state update, which the next
+                // chunk needs only after its own inputs have been consumed
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_f16(tbase + TM_OT, desc_kmajor(u16, 128, ks), desc_kmajor(p16, 64, ks), IDESC_O2, 1u);
-                mma_commit(bar_mma);
+                mma_commit(bar_o);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16(tbase + TM_S, desc_mnmajor(kh, 64, ks), desc_kmajor(u16, 128, ks), IDESC_S, 1u);
+                mma_commit(bar_s);
             }
-            if (wait_or_abort(bar_mma, mma_parity, sAbort)) { aborted = true; break; }
-            mma_parity ^= 1u;
+            issued(B_O);
+            issued(B_S);
+            if (wait_or_abort(bar_o, par(B_O), sAbort)) { aborted = true; break; }
+            waited(B_O);
             fence_after_sync();
             PHASE_MARK(10);
 
@@ -875,8 +1019,12 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tmem_wait_ld();
                 __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + OST);
 #pragma unroll
-                for (int jj = 0; jj < 16; ++jj)
-                    ost[(sub * 16 + jj) * kHeadDim + v_col] = __float2bfloat16_rn(p.scale * __uint_as_float(v[jj]));
+                for (int jj = 0; jj < 16; jj += 2) {
+                    const float2 o2 = mul2(make_float2(p.scale, p.scale),
+                                           make_float2(__uint_as_float(v[jj]), __uint_as_float(v[jj + 1])));
+                    ost[(sub * 16 + jj) * kHeadDim + v_col] = __float2bfloat16_rn(o2.x);
+                    ost[(sub * 16 + jj + 1) * kHeadDim + v_col] = __float2bfloat16_rn(o2.y);
+                }
             }
             fence_before_sync();
             __syncthreads();
@@ -893,6 +1041,11 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             PHASE_MARK(11);
         }
         if (aborted) break;
+        // the last state update must land before the state is read out or replaced
+        if (pending(B_S)) {
+            if (wait_or_abort(bar_s, par(B_S), sAbort)) { aborted = true; break; }
+            waited(B_S);
+        }
         // final state
         if (p.final_state) {
             fence_after_sync();
@@ -915,8 +1068,9 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // wind-down: never leave with a TMA load or an MMA in flight
     if (aborted) {
         if (tid == 0) {
-            if (in_flight) mbar_wait_bounded(bar_in, in_parity);
-            mbar_wait_bounded(bar_mma, mma_parity);
+            if (in_flight) mbar_wait_bounded(bar_in, par(B_IN));
+            for (uint32_t b = B_AP; b <= B_S; ++b)
+                if (pending(b)) mbar_wait_bounded(bar_in + b, par(b));
         }
     }
     fence_before_sync();
@@ -925,7 +1079,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (warp == 0) tmem_dealloc(tbase, TM_COLS);
 #ifdef KDA_PHASE_CLOCKS
     if (tid == 0)
-        for (int i = 0; i < kPhases; ++i) atomicAdd(&g_phase_cycles[i], ph_acc[i]);
+        for (int i = 0; i < kPhases; ++i) atomicAdd(&g_phase_cycles[i], (unsigned long long)sPh[i]);
 #endif
 }
 
