@@ -78,16 +78,24 @@ constexpr uint32_t AP_B = X + 32768;  // bf16 K-major [160 rows][128]: XD | C1 |
 constexpr int kF32Pitch = 68;         // fp32 row pitch of A32 / T32 (16-byte aligned rows)
 constexpr uint32_t A32 = X + 0;       // fp32 [64][68] beta-scaled A  (phases 3-4)
 constexpr uint32_t T32 = X + 17408;   // fp32 [64][68] T = (I + A)^-1 (phase 4)
-constexpr uint32_t T16 = X + 35840;   // fp16 K-major [64][64]        (phases 4-5)
-constexpr uint32_t S16 = X + 0;       // fp16 [128 c][128 v] (MN-major A)  (phases 5-7; A32/T32 dead)
-constexpr uint32_t W16 = X + 44032;   // fp16 K-major [64 r][128 c]   (phases 6-7; after T16)
-constexpr uint32_t P16 = X + 65536;   // fp16 K-major [64 r][64 i]    (phases 3-8)
-constexpr uint32_t BGK = X + 73728;   // fp16 [64 i][128 c] beta*gamma*k  (MN-major B of W)
-constexpr uint32_t U16 = BGK;         // fp16 K-major [128 v][64 r]   (phase 8; BGK is dead)
-constexpr uint32_t BV = BGK + 16384;  // fp16 [64 i][128 v] beta*v    (MN-major A of U~^T)
-constexpr uint32_t OST = BV;          // bf16 [64 r][128 v] output staging (phase 9; BV is dead)
-constexpr uint32_t GQ = BV + 16384;   // fp16 K-major [64 r][128 c] gamma*q
-constexpr uint32_t KH = GQ + 16384;   // fp16 [64 i][128 c] Khat     (MN-major A of S update)
+// [T ; 0] is the 128-row K-major A of the W | U~ MMA and [0 ; P] that of the O += P U MMA:
+// T16, Z16 (zeros) and P16 are consecutive 64-row K-major fp16 tiles.
+constexpr uint32_t T16 = X + 35840;   // fp16 K-major [64 r][64 i]    (phases 4-5)
+constexpr uint32_t Z16 = X + 44032;   // zeros [64][64]               (phases 4-8)
+constexpr uint32_t P16 = X + 52224;   // fp16 K-major [64 r][64 i]    (phases 3-8)
+constexpr uint32_t S16 = X + 0;       // fp16 [128 c][128 v] (MN-major B)  (phases 5-7; A32/T32 dead)
+// [-W ; gamma q] is the 128-row K-major A of the U | O MMA, one piece per 64-channel block:
+// piece 0 = W0 | GQ0, piece 1 = W1 | GQ1 (each W half directly before its gamma q half).
+constexpr uint32_t W0 = X + 65536;    // fp16 K-major [64 r][c 0..63]   (phases 6-7)
+constexpr uint32_t GQ0 = X + 73728;   // fp16 K-major [64 r][c 0..63]   gamma q (phases 1-7)
+constexpr uint32_t BGK = X + 81920;   // fp16 [64 i][128 c] beta*gamma*k  (MN-major B of W | U~)
+constexpr uint32_t BV = BGK + 16384;  // fp16 [64 i][128 v] beta*v        (follows BGK in that B)
+constexpr uint32_t U16 = BGK;         // fp16 [64 r][128 v] (MN-major B)  (phase 8; BGK is dead)
+constexpr uint32_t W1 = BV + 8192;    // fp16 K-major [64 r][c 64..127] (phases 6-7; BV is dead)
+constexpr uint32_t OST = BV;          // bf16 [64 r][128 v] output staging, 16-byte chunks
+                                      // swizzled by row (phase 9; BV and W1 are dead)
+constexpr uint32_t GQ1 = BV + 16384;  // fp16 K-major [64 r][c 64..127] gamma q (phases 1-7)
+constexpr uint32_t KH = GQ1 + 8192;   // fp16 [64 i][128 c] Khat     (MN-major A of S update)
 constexpr uint32_t MISC = KH + 16384;
 constexpr uint32_t S_BETA = MISC;              // fp32 [64]
 constexpr uint32_t S_GAMMAC = S_BETA + 256;    // fp32 [128] e^{Gamma_last}
@@ -107,20 +115,20 @@ constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;      // + alignment slack
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
 // ---- TMEM columns ----
+// TM_WU after the W | U~ MMA: lanes 0-63 = rows r of [W (cols 0-127) | U~ (cols 128-255)],
+// lanes 64-127 = 0.  The U | O MMA then accumulates U = U~ - W S into lanes 0-63 and
+// O = gamma q S into lanes 64-127 of cols 128-255; O += P U follows in lanes 64-127.
 constexpr uint32_t TM_AP = 0;     // [128 lanes][160]  decayed K K^T | Q K^T
-constexpr uint32_t TM_W = 0;      // M=64 [64][128]    (after TM_AP is consumed)
-constexpr uint32_t TM_UT = 160;   // [128 v][64 r]     U~^T then U^T
-constexpr uint32_t TM_OT = 224;   // [128 v][64 r]     O^T
+constexpr uint32_t TM_WU = 0;     // [128 lanes][256]  (after TM_AP is consumed)
+constexpr uint32_t TM_UO = 128;   // [128 lanes][128]  U (lanes 0-63) | O (lanes 64-127)
 constexpr uint32_t TM_S = 384;    // [128 c][128 v]    the state
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t IDESC_AP = idesc_f16(128, 160, true, false, false);
-constexpr uint32_t IDESC_W = idesc_f16(64, 128, false, false, true);
-constexpr uint32_t IDESC_UT = idesc_f16(128, 64, false, true, false);
-constexpr uint32_t IDESC_U = idesc_f16(128, 64, false, true, false, true);   // negated B
-constexpr uint32_t IDESC_O1 = idesc_f16(128, 64, false, true, false);
-constexpr uint32_t IDESC_S = idesc_f16(128, 128, false, true, false);
-constexpr uint32_t IDESC_O2 = idesc_f16(128, 64, false, false, false);
+constexpr uint32_t IDESC_WU = idesc_f16(128, 256, false, false, true);
+constexpr uint32_t IDESC_UO = idesc_f16(128, 128, false, false, true);
+constexpr uint32_t IDESC_O2 = idesc_f16(128, 128, false, false, true);
+constexpr uint32_t IDESC_S = idesc_f16(128, 128, false, true, true);
 
 struct Params {
     const float* beta;
@@ -455,6 +463,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t off128 = (uint32_t)cb * 128u * 128u + roff;
     const uint32_t off160 = (uint32_t)cb * 160u * 128u + roff;
     const uint32_t off64 = (uint32_t)cb * 64u * 128u + roff;
+    const uint32_t gq_off = (cb ? GQ1 : GQ0) + roff;
     // state / TMEM mapping: lane quarter -> rows, sub -> 32-column quarter
     const int c_row = quarter * 32 + lane;
 
@@ -597,7 +606,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (blk == 0) st_u32(sm, AP_B + off160 + 144u * 128u + ro, pack_bf16(mul2(kE, F3)));
                     st_u32(sm, KH + off64 + ro, pack_f16(mul2(kE, eA)));
                     const float2 g = mul2(R, eTs);                             // gamma_r
-                    st_u32(sm, GQ + off64 + ro, pack_f16(mul2(qq, g)));
+                    st_u32(sm, gq_off + ro, pack_f16(mul2(qq, g)));
                     gv[i] = g;
                     pd[i] = fmaf(qq.x, kk.x, qq.y * kk.y);
                 }
@@ -854,13 +863,15 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
             } else {
                 if (warp >= kPrepWarp0) {
-                    // zero fp16 blocks above the diagonal: 6 blocks x 32 chunks
+                    // zero fp16 blocks above the diagonal (6 blocks x 32 chunks) and the zero tile
                     for (int e = tid - kPrepWarp0 * 32; e < 6 * 32; e += kPrepThreads) {
                         const int blkid = e >> 5, c = e & 31;
                         const int I = blkid < 3 ? 0 : (blkid < 5 ? 1 : 2);
                         const int J = blkid < 3 ? blkid + 1 : (blkid < 5 ? blkid - 1 : 3);
                         st_v4(sm, T16 + sw128_chunk_off(16 * I + (c >> 1), 2 * J + (c & 1), 64), 0u, 0u, 0u, 0u);
                     }
+                    for (int e = tid - kPrepWarp0 * 32; e < 8192 / 16; e += kPrepThreads)
+                        st_v4(sm, Z16 + (uint32_t)e * 16u, 0u, 0u, 0u, 0u);
                 }
                 if (has_next) stage_next_chunk(sm, p, bar_in, par(B_IN), sAbort, h1, t1, L1);
             }
@@ -877,21 +888,15 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 in_flight = false;
             }
 
-            // ================= phase 5: W and U~^T MMAs; state copy while they run =================
+            // ================= phase 5: [W | U~] = [T ; 0] [beta gamma K | beta V]; state copy meanwhile
             if (tid == 0) {
                 fence_after_sync();
-                const uint32_t t16 = smem_u32(sm + T16), bgk = smem_u32(sm + BGK), bv = smem_u32(sm + BV);
+                const uint32_t t16 = smem_u32(sm + T16), bgk = smem_u32(sm + BGK);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tbase + TM_W, desc_kmajor(t16, 64, ks), desc_mnmajor(bgk, 64, ks), IDESC_W,
+                    mma_f16(tbase + TM_WU, desc_kmajor(t16, 128, ks), desc_mnmajor(bgk, 64, ks), IDESC_WU,
                             ks > 0 ? 1u : 0u);
                 mma_commit(bar_w);
-                // U~^T needs no commit of its own: the U^T MMA that accumulates onto it is
-                // issued later by this thread, and one thread's MMAs execute in order
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tbase + TM_UT, desc_mnmajor(bv, 64, ks), desc_kmajor(t16, 64, ks), IDESC_UT,
-                            ks > 0 ? 1u : 0u);
             }
             issued(B_W);
             PHASE_MARK(6);
@@ -929,43 +934,38 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             fence_after_sync();
             PHASE_MARK(7);
 
-            // ================= phase 6: W -> fp16 smem =================
-            {
-                // M = 64 accumulator: row r lives in lane (r % 16) of quarter r / 16
+            // ================= phase 6: -W -> fp16 smem (lanes 0-63 hold the rows of W) =================
+            if (quarter < 2) {
+                const int r = quarter * 32 + lane;
                 uint32_t v[2][16];
-                tmem_ld16(taddr(tbase, quarter, TM_W + sub * 32), v[0]);
-                tmem_ld16(taddr(tbase, quarter, TM_W + sub * 32 + 16), v[1]);
+                tmem_ld16(taddr(tbase, quarter, TM_WU + sub * 32), v[0]);
+                tmem_ld16(taddr(tbase, quarter, TM_WU + sub * 32 + 16), v[1]);
                 tmem_wait_ld();
-                if (lane < 16) {
-                    const int r = quarter * 16 + lane;
+                const uint32_t piece = (sub < 2 ? W0 : W1) + (uint32_t)r * 128u;
 #pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        const uint32_t col = sub * 32 + cc * 16;
-                        uint32_t w[8];
+                for (int cc = 0; cc < 2; ++cc) {
+                    const uint32_t ch = (uint32_t)((sub & 1) * 4 + cc * 2);   // 8-column chunk in the piece
+                    uint32_t w[8];
 #pragma unroll
-                        for (int q2 = 0; q2 < 8; ++q2)
-                            w[q2] = pack_f16(__uint_as_float(v[cc][2 * q2]), __uint_as_float(v[cc][2 * q2 + 1]));
-                        st_v4(sm, W16 + sw128_chunk_off(r, col / 8, 64), w[0], w[1], w[2], w[3]);
-                        st_v4(sm, W16 + sw128_chunk_off(r, col / 8 + 1, 64), w[4], w[5], w[6], w[7]);
-                    }
+                    for (int q2 = 0; q2 < 8; ++q2)
+                        w[q2] = pack_f16(-__uint_as_float(v[cc][2 * q2]), -__uint_as_float(v[cc][2 * q2 + 1]));
+                    st_v4(sm, piece + ((ch ^ (uint32_t)(r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                    st_v4(sm, piece + (((ch + 1u) ^ (uint32_t)(r & 7)) << 4), w[4], w[5], w[6], w[7]);
                 }
             }
             fence_proxy_async();
             fence_before_sync();
             __syncthreads();
 
-            // ================= phase 7: U and O MMAs =================
+            // ================= phase 7: [U ; O] = [U~ ; 0] + [-W ; gamma Q] S =================
             if (tid == 0) {
                 fence_after_sync();
-                const uint32_t s16 = smem_u32(sm + S16), w16 = smem_u32(sm + W16), gq = smem_u32(sm + GQ);
+                const uint32_t s16 = smem_u32(sm + S16), w0 = smem_u32(sm + W0), w1 = smem_u32(sm + W1);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_f16(tbase + TM_UT, desc_mnmajor(s16, 128, ks), desc_kmajor(w16, 64, ks), IDESC_U, 1u);
+                    mma_f16(tbase + TM_UO, sdesc((ks < 4 ? w0 : w1) + (uint32_t)(ks & 3) * 32u, 16u, 1024u),
+                            desc_mnmajor(s16, 128, ks), IDESC_UO, 1u);
                 mma_commit(bar_u);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_f16(tbase + TM_OT, desc_mnmajor(s16, 128, ks), desc_kmajor(gq, 64, ks), IDESC_O1,
-                            ks > 0 ? 1u : 0u);
             }
             issued(B_U);
             if (wait_or_abort(bar_u, par(B_U), sAbort)) { aborted = true; break; }
@@ -973,18 +973,24 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             fence_after_sync();
             PHASE_MARK(8);
 
-            // ================= phase 8: U -> fp16, O and S MMAs =================
-            {
-                const int v_row = c_row;   // lanes of U^T are value columns
-                uint32_t v[16];
-                tmem_ld16(taddr(tbase, quarter, TM_UT + sub * 16), v);
+            // ================= phase 8: U -> fp16 (MN-major [r][v]); O += P U and S update =================
+            if (quarter < 2) {
+                const int r = quarter * 32 + lane;
+                uint32_t v[2][16];
+                tmem_ld16(taddr(tbase, quarter, TM_UO + sub * 32), v[0]);
+                tmem_ld16(taddr(tbase, quarter, TM_UO + sub * 32 + 16), v[1]);
                 tmem_wait_ld();
-                uint32_t w[8];
+                const uint32_t row = U16 + (uint32_t)(sub >> 1) * 8192u + (uint32_t)r * 128u;
 #pragma unroll
-                for (int q2 = 0; q2 < 8; ++q2)
-                    w[q2] = pack_f16(__uint_as_float(v[2 * q2]), __uint_as_float(v[2 * q2 + 1]));
-                st_v4(sm, U16 + sw128_chunk_off(v_row, sub * 2, 128), w[0], w[1], w[2], w[3]);
-                st_v4(sm, U16 + sw128_chunk_off(v_row, sub * 2 + 1, 128), w[4], w[5], w[6], w[7]);
+                for (int cc = 0; cc < 2; ++cc) {
+                    const uint32_t ch = (uint32_t)((sub & 1) * 4 + cc * 2);
+                    uint32_t w[8];
+#pragma unroll
+                    for (int q2 = 0; q2 < 8; ++q2)
+                        w[q2] = pack_f16(__uint_as_float(v[cc][2 * q2]), __uint_as_float(v[cc][2 * q2 + 1]));
+                    st_v4(sm, row + ((ch ^ (uint32_t)(r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                    st_v4(sm, row + (((ch + 1u) ^ (uint32_t)(r & 7)) << 4), w[4], w[5], w[6], w[7]);
+                }
             }
             fence_proxy_async();
             fence_before_sync();
@@ -992,16 +998,16 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             PHASE_MARK(9);
             if (tid == 0) {
                 fence_after_sync();
-                const uint32_t kh = smem_u32(sm + KH), u16 = smem_u32(sm + U16), p16 = smem_u32(sm + P16);
-                // O first (the output waits for it), then the state update, which the next
-                // chunk needs only after its own inputs have been consumed
+                const uint32_t kh = smem_u32(sm + KH), u16 = smem_u32(sm + U16), z16 = smem_u32(sm + Z16);
+                // O first (the output waits for it); its A is [0 ; P], so lanes 0-63 (U) get + 0
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tbase + TM_OT, desc_kmajor(u16, 128, ks), desc_kmajor(p16, 64, ks), IDESC_O2, 1u);
+                    mma_f16(tbase + TM_UO, desc_kmajor(z16, 128, ks), desc_mnmajor(u16, 64, ks), IDESC_O2, 1u);
                 mma_commit(bar_o);
+                // the state update; the next chunk waits for it before rewriting KH / U16
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_f16(tbase + TM_S, desc_mnmajor(kh, 64, ks), desc_kmajor(u16, 128, ks), IDESC_S, 1u);
+                    mma_f16(tbase + TM_S, desc_mnmajor(kh, 64, ks), desc_mnmajor(u16, 64, ks), IDESC_S, 1u);
                 mma_commit(bar_s);
             }
             issued(B_O);
@@ -1011,31 +1017,38 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             fence_after_sync();
             PHASE_MARK(10);
 
-            // ================= phase 9: O -> out (through an smem tile, coalesced) =================
-            {
-                const int v_col = c_row;
-                uint32_t v[16];
-                tmem_ld16(taddr(tbase, quarter, TM_OT + sub * 16), v);
+            // ================= phase 9: O -> out (lanes 64-127 hold the rows of O) =================
+            // rows go to a swizzled smem tile (16-byte chunk c of row r at chunk c ^ (r & 7)),
+            // then every thread copies 16-byte pieces out so that each warp writes whole rows
+            if (quarter >= 2) {
+                const int r = (quarter - 2) * 32 + lane;
+                uint32_t v[2][16];
+                tmem_ld16(taddr(tbase, quarter, TM_UO + sub * 32), v[0]);
+                tmem_ld16(taddr(tbase, quarter, TM_UO + sub * 32 + 16), v[1]);
                 tmem_wait_ld();
-                __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + OST);
+                const float2 sc = make_float2(p.scale, p.scale);
+                const uint32_t row = OST + (uint32_t)r * 256u;
 #pragma unroll
-                for (int jj = 0; jj < 16; jj += 2) {
-                    const float2 o2 = mul2(make_float2(p.scale, p.scale),
-                                           make_float2(__uint_as_float(v[jj]), __uint_as_float(v[jj + 1])));
-                    ost[(sub * 16 + jj) * kHeadDim + v_col] = __float2bfloat16_rn(o2.x);
-                    ost[(sub * 16 + jj + 1) * kHeadDim + v_col] = __float2bfloat16_rn(o2.y);
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint32_t w[8];
+#pragma unroll
+                    for (int q2 = 0; q2 < 8; ++q2)
+                        w[q2] = pack_bf16(mul2(sc, make_float2(__uint_as_float(v[cc][2 * q2]),
+                                                               __uint_as_float(v[cc][2 * q2 + 1]))));
+                    const uint32_t c16 = (uint32_t)(sub * 4 + cc * 2);   // 16-byte chunk of the row
+                    st_v4(sm, row + ((c16 ^ (uint32_t)(r & 7)) << 4), w[0], w[1], w[2], w[3]);
+                    st_v4(sm, row + (((c16 + 1u) ^ (uint32_t)(r & 7)) << 4), w[4], w[5], w[6], w[7]);
                 }
             }
             fence_before_sync();
             __syncthreads();
-            {
-                const uint4* src = reinterpret_cast<const uint4*>(sm + OST);
 #pragma unroll
-                for (int e = tid; e < kChunk * 16; e += kThreads) {
-                    const int r = e >> 4, c = e & 15;
-                    if (r < L)
-                        *reinterpret_cast<uint4*>(p.out + ((t0 + r) * H + h) * kHeadDim + c * 8) = src[e];
-                }
+            for (int e = tid; e < kChunk * 16; e += kThreads) {
+                const int r = e >> 4, c16 = e & 15;
+                if (r < L)
+                    *reinterpret_cast<uint4*>(p.out + ((t0 + r) * H + h) * kHeadDim + c16 * 8) =
+                        *reinterpret_cast<const uint4*>(sm + OST + (uint32_t)r * 256u +
+                                                         (((uint32_t)c16 ^ (uint32_t)(r & 7)) << 4));
             }
             __syncthreads();
             PHASE_MARK(11);
