@@ -195,6 +195,18 @@ __device__ __forceinline__ void issue_chunk_loads(unsigned char* sm, uint64_t* b
     tma_load_2d(sm + IN_G, tg, x, y, bar);
 }
 
+// Prefetches one chunk's four tiles into L2 (one thread), so that its later TMA load does
+// not wait on DRAM: the loads of all CTAs otherwise arrive in bursts at the same phase.
+__device__ __forceinline__ void prefetch_chunk(const CUtensorMap* tq, const CUtensorMap* tk,
+                                               const CUtensorMap* tv, const CUtensorMap* tg, int h,
+                                               int64_t t0) {
+    const int x = h * kHeadDim, y = (int)t0;
+    tma_prefetch_2d(tq, x, y);
+    tma_prefetch_2d(tk, x, y);
+    tma_prefetch_2d(tv, x, y);
+    tma_prefetch_2d(tg, x, y);
+}
+
 // Finds the chunk after (k, j) on this CTA's schedule: next chunk of the same
 // unit or chunk 0 of the next non-empty unit.  Returns false if none.
 __device__ bool next_chunk(const Params& p, const int16_t* order, int b, int G, int units, int k,
@@ -523,6 +535,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int64_t t1 = last ? tn : t0 + kChunk;
             const int64_t e1 = last ? en : x.eos;
             const int L1 = (int)(e1 - t1 < kChunk ? e1 - t1 : kChunk);
+            if (tid == 0 && has_next) prefetch_chunk(&tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
             // this chunk was gated and prepared while the previous one solved for T; the
             // previous chunk's S update must have finished reading KH / U16
             if (pending(B_S)) {
@@ -749,118 +762,100 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     st_v4(sm, T16 + sw128_chunk_off(16 * I + rr, 2 * J + ch, 64), pack_f16(lo4.x, lo4.y),
                           pack_f16(lo4.z, lo4.w), pack_f16(hi4.x, hi4.y), pack_f16(hi4.z, hi4.w));
                 };
-                if (warp < 2) {   // diagonal 16 x 16 blocks by forward substitution, one column each
+                // sign * (a 16 x 16 warp-MMA accumulator) straight into block (I, J) of the fp16 tile
+                auto acc_to_t16 = [&](int I, int J, const float (&acc)[2][4], float sign) {
+                    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+                    for (int nh = 0; nh < 2; ++nh) {
+                        const uint32_t col = (uint32_t)(16 * J + 8 * nh + 2 * t);
+                        st_u32(sm, T16 + sw128_off((uint32_t)(16 * I + g), col, 64u),
+                               pack_f16(sign * acc[nh][0], sign * acc[nh][1]));
+                        st_u32(sm, T16 + sw128_off((uint32_t)(16 * I + g + 8), col, 64u),
+                               pack_f16(sign * acc[nh][2], sign * acc[nh][3]));
+                    }
+                };
+                // L0: the four 16 x 16 diagonal blocks of T by forward substitution in fp32, one
+                // column per thread (threads 0-63), right-looking: once x_ii is final it
+                // updates every later row, so each step is independent FMAs on broadcast loads.
+                if (warp < 2) {
                     const int bI = tid >> 4, jc = tid & 15, o = bI * 16;
-                    float xv[16];
+                    float x[16];
 #pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) {
-                        float s0 = (rr == jc) ? 1.f : 0.f;
+                    for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == jc) ? 1.f : 0.f;
 #pragma unroll
-                        for (int ii = 0; ii < rr; ++ii)
-                            s0 = fmaf(-a32[(o + rr) * kF32Pitch + o + ii], xv[ii], s0);
-                        xv[rr] = (rr < jc) ? 0.f : s0;
+                    for (int ii = 0; ii < 15; ++ii) {
+                        const float xi = x[ii];
+#pragma unroll
+                        for (int rr = ii + 1; rr < 16; ++rr)
+                            x[rr] = fmaf(-a32[(o + rr) * kF32Pitch + o + ii], xi, x[rr]);
                     }
 #pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) t32[(o + rr) * kF32Pitch + o + jc] = xv[rr];
+                    for (int rr = 0; rr < 16; ++rr) t32[(o + rr) * kF32Pitch + o + jc] = x[rr];
                 }
                 named_bar_sync(1, kSolveWarps * 32);
                 PHASE_MARK(14);
-                // Off-diagonal blocks by recursive doubling on 16 x 16 blocks; products on the
-                // warp tensor-core path (mma.sync, fp16 operands, fp32 accumulation -- T is
-                // rounded to fp16 for the W / U~ MMAs in any case).  Intermediates are parked
-                // in the unused upper blocks of t32.
-                //   T10 = -T11 A10 T00, T32 = -T33 A32 T22, T21 = -T22 A21 T11,
-                //   X20 = A20 T00 + A21 T10, X30 = A30 T00 + A31 T10,
-                //   T20 = -T22 X20, T31 = -(T32 A21 T11 + T33 A31 T11), T30 = -(T32 X20 + T33 X30).
-                float acc[2][4] = {}, acc2[2][4] = {};
-                // step A: T10, T32 (two products each); X21 = A21 T11, X31 = A31 T11;
-                //         partial X20 = A20 T00, X30 = A30 T00; fp16 copies of the diagonal blocks
-                if (warp == 0 || warp == 1) {
-                    const int Ii = warp == 0 ? 1 : 3, Jj = Ii - 1;
-                    warpmma::mm16_acc_h(Ab(Ii, Jj), kF32Pitch, Tb(Jj, Jj), kF32Pitch, acc);
-                    warpmma::store16(Tb(Jj, Ii), kF32Pitch, acc, 1.f);
-                    __syncwarp();
-                    float a3[2][4] = {};
-                    warpmma::mm16_acc_h(Tb(Ii, Ii), kF32Pitch, Tb(Jj, Ii), kF32Pitch, a3);
-                    warpmma::store16(Tb(Ii, Jj), kF32Pitch, a3, -1.f);
-                    __syncwarp();
-                    to_t16(Ii, Jj);
-                } else if (warp == 2) {
-                    warpmma::mm16_acc_h(Ab(2, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc);
-                    warpmma::store16(Tb(1, 2), kF32Pitch, acc, 1.f);           // X21
-                    warpmma::mm16_acc_h(Ab(3, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc2);
-                    warpmma::store16(Tb(1, 3), kF32Pitch, acc2, 1.f);          // X31
-                } else {
-                    warpmma::mm16_acc_h(Ab(2, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);    // X20 partial
-                    warpmma::mm16_acc_h(Ab(3, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc2);   // X30 partial
+                // L1 (16 x 16 warp-MMA products, fp16 operands, fp32 accumulation):
+                //   T10 = -T11 (A10 T00), T32 = -T33 (A32 T22),
+                //   X20 = A20 T00 + A21 T10, X30 = A30 T00 + A31 T10, X21 = A21 T11, X31 = A31 T11.
+                // Warps 0 and 2 both form T10 (in their own scratch) so that neither waits for the
+                // other.  Scratch: T's upper blocks and A's upper blocks (A is zero there and
+                // is not read again).
+                {
+                    float* const a32w = reinterpret_cast<float*>(sm + A32);
+                    auto Aw = [&](int I, int J) { return a32w + 16 * I * kF32Pitch + 16 * J; };
+                    float acc[2][4] = {};
+                    if (warp == 0 || warp == 2) {
+                        float* ysc = warp == 0 ? Tb(0, 1) : Aw(0, 1);     // A10 T00
+                        float* t10 = warp == 0 ? Tb(1, 0) : Aw(0, 2);     // T10
+                        warpmma::mm16_acc_h(Ab(1, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);
+                        warpmma::store16(ysc, kF32Pitch, acc, 1.f);
+                        __syncwarp();
+                        float a2[2][4] = {};
+                        warpmma::mm16_acc_h(Tb(1, 1), kF32Pitch, ysc, kF32Pitch, a2);
+                        warpmma::store16(t10, kF32Pitch, a2, -1.f);
+                        __syncwarp();
+                        if (warp == 0) to_t16(1, 0);
+                        const int I = warp == 0 ? 2 : 3;
+                        float a3[2][4] = {};
+                        warpmma::mm16_acc_h(Ab(I, 0), kF32Pitch, Tb(0, 0), kF32Pitch, a3);
+                        warpmma::mm16_acc_h(Ab(I, 1), kF32Pitch, t10, kF32Pitch, a3);
+                        warpmma::store16(Tb(0, I), kF32Pitch, a3, 1.f);            // X20 / X30
+                    } else if (warp == 1) {
+                        warpmma::mm16_acc_h(Ab(3, 2), kF32Pitch, Tb(2, 2), kF32Pitch, acc);
+                        warpmma::store16(Tb(2, 3), kF32Pitch, acc, 1.f);            // A32 T22
+                        __syncwarp();
+                        float a2[2][4] = {};
+                        warpmma::mm16_acc_h(Tb(3, 3), kF32Pitch, Tb(2, 3), kF32Pitch, a2);
+                        warpmma::store16(Tb(3, 2), kF32Pitch, a2, -1.f);           // T32
+                        __syncwarp();
+                        to_t16(3, 2);
+                        float a3[2][4] = {};
+                        warpmma::mm16_acc_h(Ab(2, 1), kF32Pitch, Tb(1, 1), kF32Pitch, a3);
+                        warpmma::store16(Tb(1, 2), kF32Pitch, a3, 1.f);            // X21
+                    } else {
+                        warpmma::mm16_acc_h(Ab(3, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc);
+                        warpmma::store16(Tb(1, 3), kF32Pitch, acc, 1.f);            // X31
 #pragma unroll
-                    for (int d = 0; d < 4; ++d) to_t16(d, d);                            // diagonal blocks
+                        for (int d = 0; d < 4; ++d) to_t16(d, d);
+                    }
                 }
                 named_bar_sync(1, kSolveWarps * 32);
                 PHASE_MARK(15);
-                // step B: X20, X30 complete; T21 = -T22 X21; P31a = T32 X21, P31b = T33 X31
-                if (warp == 3) {
-                    warpmma::mm16_acc_h(Ab(2, 1), kF32Pitch, Tb(1, 0), kF32Pitch, acc);
-                    warpmma::store16(Tb(0, 2), kF32Pitch, acc, 1.f);            // X20 -> (0,2)
-                    warpmma::mm16_acc_h(Ab(3, 1), kF32Pitch, Tb(1, 0), kF32Pitch, acc2);
-                    warpmma::store16(Tb(0, 3), kF32Pitch, acc2, 1.f);           // X30 -> (0,3)
-                } else if (warp == 0) {
-                    float a2[2][4] = {};
-                    warpmma::mm16_acc_h(Tb(2, 2), kF32Pitch, Tb(1, 2), kF32Pitch, a2);
-                    warpmma::store16(Tb(2, 1), kF32Pitch, a2, -1.f);           // T21
-                    __syncwarp();
-                    to_t16(2, 1);
-                } else if (warp == 1) {
-                    float a2[2][4] = {};
-                    warpmma::mm16_acc_h(Tb(3, 2), kF32Pitch, Tb(1, 2), kF32Pitch, a2);
-                    warpmma::store16(Tb(0, 1), kF32Pitch, a2, 1.f);            // P31a -> (0,1)
-                } else {
-                    float a2[2][4] = {};
-                    warpmma::mm16_acc_h(Tb(3, 3), kF32Pitch, Tb(1, 3), kF32Pitch, a2);
-                    warpmma::store16(Tb(2, 3), kF32Pitch, a2, 1.f);            // P31b -> (2,3)
+                // L2: T_LL = -T_LR X, written straight to the fp16 tile:
+                //   T20 = -T22 X20, T21 = -T22 X21, T30 = -(T32 X20 + T33 X30), T31 = -(T32 X21 + T33 X31)
+                {
+                    float acc[2][4] = {};
+                    const int J = warp & 1;               // column block of the result
+                    if (warp < 2) {
+                        warpmma::mm16_acc_h(Tb(2, 2), kF32Pitch, Tb(J, 2), kF32Pitch, acc);
+                        acc_to_t16(2, J, acc, -1.f);
+                    } else {
+                        warpmma::mm16_acc_h(Tb(3, 2), kF32Pitch, Tb(J, 2), kF32Pitch, acc);
+                        warpmma::mm16_acc_h(Tb(3, 3), kF32Pitch, Tb(J, 3), kF32Pitch, acc);
+                        acc_to_t16(3, J, acc, -1.f);
+                    }
                 }
-                named_bar_sync(1, kSolveWarps * 32);
                 PHASE_MARK(16);
-                // step C: T20 = -T22 X20; P30a = T32 X20, P30b = T33 X30; T31 = -(P31a + P31b)
-                if (warp == 0) {
-                    float a2[2][4] = {};
-                    warpmma::mm16_acc_h(Tb(2, 2), kF32Pitch, Tb(0, 2), kF32Pitch, a2);
-                    warpmma::store16(Tb(2, 0), kF32Pitch, a2, -1.f);           // T20
-                    __syncwarp();
-                    to_t16(2, 0);
-                } else if (warp == 1) {
-                    float a2[2][4] = {};
-                    warpmma::mm16_acc_h(Tb(3, 2), kF32Pitch, Tb(0, 2), kF32Pitch, a2);
-                    warpmma::store16(Tb(1, 2), kF32Pitch, a2, 1.f);            // P30a -> (1,2)
-                } else if (warp == 2) {
-                    float a2[2][4] = {};
-                    warpmma::mm16_acc_h(Tb(3, 3), kF32Pitch, Tb(0, 3), kF32Pitch, a2);
-                    warpmma::store16(Tb(1, 3), kF32Pitch, a2, 1.f);            // P30b -> (1,3)
-                } else {
-                    for (int e = lane; e < 64; e += 32) {                      // T31 = -(P31a + P31b)
-                        const int rr = e >> 2, c4 = (e & 3) * 4;
-                        const float4 x1 = *reinterpret_cast<const float4*>(Tb(0, 1) + rr * kF32Pitch + c4);
-                        const float4 x2 = *reinterpret_cast<const float4*>(Tb(2, 3) + rr * kF32Pitch + c4);
-                        *reinterpret_cast<float4*>(Tb(3, 1) + rr * kF32Pitch + c4) =
-                            make_float4(-(x1.x + x2.x), -(x1.y + x2.y), -(x1.z + x2.z), -(x1.w + x2.w));
-                    }
-                    __syncwarp();
-                    to_t16(3, 1);
-                }
-                named_bar_sync(1, kSolveWarps * 32);
-                PHASE_MARK(17);
-                // step D: T30 = -(P30a + P30b)
-                if (warp == 0) {
-                    for (int e = lane; e < 64; e += 32) {
-                        const int rr = e >> 2, c4 = (e & 3) * 4;
-                        const float4 x1 = *reinterpret_cast<const float4*>(Tb(1, 2) + rr * kF32Pitch + c4);
-                        const float4 x2 = *reinterpret_cast<const float4*>(Tb(1, 3) + rr * kF32Pitch + c4);
-                        *reinterpret_cast<float4*>(Tb(3, 0) + rr * kF32Pitch + c4) =
-                            make_float4(-(x1.x + x2.x), -(x1.y + x2.y), -(x1.z + x2.z), -(x1.w + x2.w));
-                    }
-                    __syncwarp();
-                    to_t16(3, 0);
-                }
             } else {
                 if (warp >= kPrepWarp0) {
                     // zero fp16 blocks above the diagonal (6 blocks x 32 chunks) and the zero tile
