@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gdn", action="store_true",
+                    help="time kda_gdn_fwd, the scalar-gate variant, on the same workload")
     ap.add_argument("--decode", action="store_true",
                     help="time kda_decode (one token per sequence) instead of the prefill")
     ap.add_argument("--decode-batch", type=int, default=256)
@@ -68,8 +70,11 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def algorithmic_bytes(w: W.Workload) -> int:
-    b = BYTES_PER_TOKEN_HEAD * w.T * w.H
+GDN_BYTES_PER_TOKEN_HEAD = 1032    # q,k,v bf16 768 + g fp32 4 + beta 4 + out bf16 256
+
+
+def algorithmic_bytes(w: W.Workload, gdn: bool = False) -> int:
+    b = (GDN_BYTES_PER_TOKEN_HEAD if gdn else BYTES_PER_TOKEN_HEAD) * w.T * w.H
     if w.init is not None:
         b += STATE_BYTES * w.N * w.H
     if w.final:
@@ -225,7 +230,7 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
-def oracle_sample(w: W.Workload, x: dict, target_s: float):
+def oracle_sample(w: W.Workload, x: dict, target_s: float, gdn: bool = False):
     """Runs the fp64 oracle on the first h heads of every sequence, h sized so
     the run takes about target_s seconds; returns (tokens-equivalent/s, desc)."""
     import oracle
@@ -237,10 +242,11 @@ def oracle_sample(w: W.Workload, x: dict, target_s: float):
             sub[key] = x[key][:, :h].contiguous()
         sub["A_log"] = x["A_log"][:h]
         sub["dt_bias"] = x["dt_bias"][:h]
+        fwd = oracle.gdn_recurrent if gdn else oracle.recurrent
         if x["initial_state"] is not None:
             sub["initial_state"] = x["initial_state"][:, :h].contiguous()
         t = time.perf_counter()
-        oracle.recurrent(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"], sub["A_log"],
+        fwd(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"], sub["A_log"],
                          sub["dt_bias"], sub["lower_bound"], sub["scale"], sub["initial_state"],
                          sub["cu_seqlens"], want_final=w.final)
         return time.perf_counter() - t
@@ -418,7 +424,7 @@ def main():
             dist.destroy_process_group()
         return rc
 
-    from gated_delta_rule_135_b200 import build
+    import kda_build as build
     if rank == 0:
         build.build()
     barrier(world)
@@ -432,18 +438,21 @@ def main():
 
     w = W.WORKLOADS[args.workload]
     x = W.make_inputs(w)
+    if args.gdn:
+        x = W.gdn_inputs(x)
     dev = torch.device("cuda", torch.cuda.current_device())
     xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
     out = torch.empty_like(xd["q"])
     fin = (torch.empty(w.N, w.H, 128, 128, device=dev) if w.final else None)
     stream = torch.cuda.current_stream()
-    fused = x["lower_bound"] >= kda.FUSED_MIN_LOWER_BOUND
+    fused = args.gdn or x["lower_bound"] >= kda.FUSED_MIN_LOWER_BOUND
     launches_per_step = 1 if fused else 5
+    fwd = kda.kda_gdn_fwd if args.gdn else kda.kda_fwd
 
     def step():
-        kda.kda_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"],
-                    x["lower_bound"], x["scale"], xd["initial_state"], xd["cu_seqlens"], out=out,
-                    final_state=fin, batch=x["batch"])
+        fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"],
+            x["lower_bound"], x["scale"], xd["initial_state"], xd["cu_seqlens"], out=out,
+            final_state=fin, batch=x["batch"])
 
     for _ in range(args.warmup):
         step()
@@ -471,14 +480,16 @@ def main():
     value = tokens / (ms_per_step / 1e3) / 1e6
     tflops = FLOP_PER_TOKEN_HEAD * w.T * w.H * world / (ms_per_step / 1e3) / 1e12
     kernel_ms = statistics.mean(per_step)
-    alg_bytes = algorithmic_bytes(w)
+    alg_bytes = algorithmic_bytes(w, args.gdn)
     peak, peak_kind = measured_hbm_peak()
     achieved = alg_bytes / (kernel_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "traffic": dram_traffic_from_profile("kda_fused_kernel", w.T * w.H) if fused else None,
+            "frac": achieved / peak,
+            "traffic": (dram_traffic_from_profile("kda_fused_kernel", w.T * w.H) if fused and not args.gdn else None),
             "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
             else "fallback 6650 GB/s",
-            "kernel": "kda_fused_kernel" if fused else "staged kernels",
+            "kernel": ("kda_fused_kernel<scalar gate>" if args.gdn else "kda_fused_kernel") if fused
+            else "staged kernels",
             "kernel_ms": kernel_ms, "algorithmic_bytes": alg_bytes,
             "tflops": tflops}
 
@@ -513,18 +524,19 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, desc, cores, threads, _ = oracle_sample(w, x, args.cpu_seconds)
+        rate, desc, cores, threads, _ = oracle_sample(w, x, args.cpu_seconds, args.gdn)
         cpu = {"value": rate / 1e6, "unit": "Mtokens/s", "cores": threads, "kind": "oracle",
                "sample": desc, "host_cores": cores}
 
     if rank == 0:
         line = {
-            "metric": "KDA prefill throughput (Mtokens/s) at T=8192 H=96 D=128 varlen",
+            "metric": ("GDN (scalar-gate) prefill throughput (Mtokens/s) at T=8192 H=96 D=128 varlen"
+                       if args.gdn else "KDA prefill throughput (Mtokens/s) at T=8192 H=96 D=128 varlen"),
             "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded kda_workloads, no dataset)",
-            "config": {"workload": w.describe(), "model": "KDA layer forward (no weights)",
+            "config": {"workload": ("GDN (one gate per token-head) " if args.gdn else "") + w.describe(), "model": "KDA layer forward (no weights)",
                        "global_batch": w.N * world, "seq_len": w.T, "heads": w.H,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "precision": "bf16 q/k/v/out, fp32 gates and state; bf16/fp16 MMA operands, fp32 accumulate",

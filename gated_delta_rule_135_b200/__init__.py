@@ -74,6 +74,8 @@ def _load():
     lib.kda_fwd_staged_noalloc.argtypes = fwd_args + [vp]
     lib.kda_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.kda_noalloc_scratch_bytes.argtypes = []
+    lib.kda_gdn_fwd.restype = ctypes.c_int
+    lib.kda_gdn_fwd.argtypes = fwd_args + [vp]
     lib.kda_decode.restype = ctypes.c_int
     lib.kda_decode.argtypes = [vp] * 7 + [f32, f32, vp, vp, ctypes.c_int32, ctypes.c_int32, vp]
     return lib
@@ -85,7 +87,7 @@ _lib = _load()
 EXPORTED = ("kda_fwd", "kda_fwd_staged", "kda_staged_workspace_size",
             "kda_staged_workspace_layout", "kda_strerror", "kda_check_device_error",
             "kda_last_device_error_bits", "kda_version", "kda_fwd_staged_noalloc",
-            "kda_noalloc_scratch_bytes", "kda_decode")
+            "kda_noalloc_scratch_bytes", "kda_decode", "kda_gdn_fwd")
 
 
 def lib() -> ctypes.CDLL:
@@ -242,6 +244,25 @@ def kda_fwd_staged_noalloc(q, k, v, g, beta, A_log, dt_bias, lower_bound: float,
 
 def kda_noalloc_scratch_bytes() -> int:
     return int(_lib.kda_noalloc_scratch_bytes())
+
+
+def kda_gdn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                beta: torch.Tensor, A_log: torch.Tensor, dt_bias: torch.Tensor,
+                lower_bound: float, scale: float, initial_state: Optional[torch.Tensor] = None,
+                cu_seqlens: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                final_state: Optional[torch.Tensor] = None, *, batch: int = 1, stream=None):
+    """Calls kda_gdn_fwd (scalar gate).  q/k/v as for kda_fwd; g and beta: fp32 [.., H];
+    A_log and dt_bias: fp32 [H].  Returns (out, final_state)."""
+    dims = _marshal(q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens, out,
+                    final_state, batch)
+    if out is None:
+        out = torch.empty(q.shape[:-1] + (HEAD_DIM,), dtype=torch.bfloat16, device=q.device)
+    st = _lib.kda_gdn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias),
+                          float(lower_bound), float(scale), _ptr(initial_state), _ptr(cu_seqlens),
+                          _ptr(out), _ptr(final_state), dims, _stream_ptr(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_gdn_fwd")
+    return out, final_state
 
 
 def kda_decode(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, scale: float, state,

@@ -38,11 +38,12 @@ kda_status device_ok() {
     return major == 10 ? KDA_OK : KDA_ERR_UNSUPPORTED;
 }
 
-// Validates arguments and fills the kernel argument block.
+// Validates arguments and fills the kernel argument block.  g_per_head is the number of
+// gate values per (token, head): 128 (one per key channel) or 1 (the scalar-gate variant).
 kda_status prepare(const void* q, const void* k, const void* v, const float* g, const float* beta,
                    const float* A_log, const float* dt_bias, float lower_bound, float scale,
                    const float* initial_state, const int32_t* cu_seqlens, void* out,
-                   float* final_state, const kda_dims& d, StagedArgs* a) {
+                   float* final_state, const kda_dims& d, StagedArgs* a, size_t g_per_head = kda::kHeadDim) {
     if (d.head_dim_k != kda::kHeadDim || d.head_dim_v != kda::kHeadDim) return KDA_ERR_UNSUPPORTED;
     if (d.num_heads < 1 || d.seqlen < 0) return KDA_ERR_INVALID_ARG;
     if (isnan(lower_bound) || lower_bound > 0.f) return KDA_ERR_INVALID_ARG;
@@ -68,7 +69,7 @@ kda_status prepare(const void* q, const void* k, const void* v, const float* g, 
     const size_t out_bytes = tok * kda::kHeadDim * 2;
     const size_t st_bytes = (size_t)N * H * kda::kHeadDim * kda::kHeadDim * 4;
     if (overlaps(out, out_bytes, q, out_bytes) || overlaps(out, out_bytes, k, out_bytes) ||
-        overlaps(out, out_bytes, v, out_bytes) || overlaps(out, out_bytes, g, tok * kda::kHeadDim * 4) ||
+        overlaps(out, out_bytes, v, out_bytes) || overlaps(out, out_bytes, g, tok * g_per_head * 4) ||
         overlaps(out, out_bytes, beta, tok * 4) || overlaps(out, out_bytes, initial_state, st_bytes) ||
         overlaps(out, out_bytes, final_state, st_bytes))
         return KDA_ERR_INVALID_ARG;
@@ -222,6 +223,19 @@ kda_status kda_fwd(const void* q, const void* k, const void* v, const float* g, 
     cudaError_t err = kda::launch_staged(a, static_cast<char*>(ws), L, s);
     cudaError_t err2 = cudaFreeAsync(ws, s);
     return (err == cudaSuccess && err2 == cudaSuccess) ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_gdn_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                       const float* A_log, const float* dt_bias, float lower_bound, float scale,
+                       const float* initial_state, const int32_t* cu_seqlens, void* out,
+                       float* final_state, kda_dims dims, kda_stream_t stream) {
+    StagedArgs a{};
+    kda_status st = prepare(q, k, v, g, beta, A_log, dt_bias, lower_bound, scale, initial_state,
+                            cu_seqlens, out, final_state, dims, &a, 1);
+    if (st != KDA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (a.total_tokens == 0) return copy_states_only(a, s);
+    return kda::launch_fused_gdn(a, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 kda_status kda_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,

@@ -72,6 +72,13 @@ constexpr uint32_t IN_K = 16384;
 constexpr uint32_t IN_V = 32768;
 constexpr uint32_t IN_G = 49152;      // fp32 [64][128]
 constexpr uint32_t IN_BYTES = 81920;
+// Scalar-gate variant: q, k, v arrive as 128-byte-swizzled 64-channel blocks of 64 rows
+// (8 KB each) laid out k0 | q0 | k1 | q1 | v0 | v1, so that [k ; q] is the 128-row
+// K-major A operand of the A/P MMA and k its B operand; the g tile holds per-token data.
+constexpr uint32_t IN_S_BYTES = 49152;
+constexpr uint32_t S_GAM = IN_G;            // fp32 [64] Gamma (log2, inclusive in-chunk sum)
+constexpr uint32_t S_GE = IN_G + 256;       // fp32 [64] 2^Gamma
+constexpr uint32_t S_KF = IN_G + 512;       // fp32 [64] 2^(Gamma_63 - Gamma)
 constexpr uint32_t X = 81920;         // phase-shared region, 73728 bytes
 constexpr uint32_t AP_A = X + 0;      // bf16 K-major [128 rows][128]: k*R rows 0-63, q*R rows 64-127
 constexpr uint32_t AP_B = X + 32768;  // bf16 K-major [160 rows][128]: XD | C1 | C2 | C3
@@ -125,6 +132,7 @@ constexpr uint32_t TM_S = 384;    // [128 c][128 v]    the state
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t IDESC_AP = idesc_f16(128, 160, true, false, false);
+constexpr uint32_t IDESC_AP_S = idesc_f16(128, 64, true, false, false);   // scalar gate: [K ; Q] K^T
 constexpr uint32_t IDESC_WU = idesc_f16(128, 256, false, false, true);
 constexpr uint32_t IDESC_UO = idesc_f16(128, 128, false, false, true);
 constexpr uint32_t IDESC_O2 = idesc_f16(128, 128, false, false, true);
@@ -144,6 +152,7 @@ struct Params {
     int64_t total_tokens;
     int H;
     int N;
+    const float* g_scalar;   // scalar-gate variant: g [Ttot][H] (dt_bias is then [H])
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -195,16 +204,40 @@ __device__ __forceinline__ void issue_chunk_loads(unsigned char* sm, uint64_t* b
     tma_load_2d(sm + IN_G, tg, x, y, bar);
 }
 
-// Prefetches one chunk's four tiles into L2 (one thread), so that its later TMA load does
-// not wait on DRAM: the loads of all CTAs otherwise arrive in bursts at the same phase.
+// Scalar-gate variant: six 64 x 64 swizzled blocks (see IN_S_BYTES).
+__device__ __forceinline__ void issue_chunk_loads_s(unsigned char* sm, uint64_t* bar,
+                                                    const CUtensorMap* tq, const CUtensorMap* tk,
+                                                    const CUtensorMap* tv, int h, int64_t t0) {
+    mbar_arrive_expect_tx(bar, IN_S_BYTES);
+    const int x = h * kHeadDim, y = (int)t0;
+#pragma unroll
+    for (int cb = 0; cb < 2; ++cb) {
+        tma_load_2d(sm + (uint32_t)cb * 16384u, tk, x + 64 * cb, y, bar);
+        tma_load_2d(sm + (uint32_t)cb * 16384u + 8192u, tq, x + 64 * cb, y, bar);
+        tma_load_2d(sm + 32768u + (uint32_t)cb * 8192u, tv, x + 64 * cb, y, bar);
+    }
+}
+
+// Prefetches one chunk's tiles into L2 (one thread), so that its later TMA load does not
+// wait on DRAM: the loads of all CTAs otherwise arrive in bursts at the same phase.
+template <bool kScalar>
 __device__ __forceinline__ void prefetch_chunk(const CUtensorMap* tq, const CUtensorMap* tk,
                                                const CUtensorMap* tv, const CUtensorMap* tg, int h,
                                                int64_t t0) {
     const int x = h * kHeadDim, y = (int)t0;
-    tma_prefetch_2d(tq, x, y);
-    tma_prefetch_2d(tk, x, y);
-    tma_prefetch_2d(tv, x, y);
-    tma_prefetch_2d(tg, x, y);
+    if constexpr (kScalar) {
+#pragma unroll
+        for (int cb = 0; cb < 2; ++cb) {
+            tma_prefetch_2d(tq, x + 64 * cb, y);
+            tma_prefetch_2d(tk, x + 64 * cb, y);
+            tma_prefetch_2d(tv, x + 64 * cb, y);
+        }
+    } else {
+        tma_prefetch_2d(tq, x, y);
+        tma_prefetch_2d(tk, x, y);
+        tma_prefetch_2d(tv, x, y);
+        tma_prefetch_2d(tg, x, y);
+    }
 }
 
 // Finds the chunk after (k, j) on this CTA's schedule: next chunk of the same
@@ -343,13 +376,60 @@ __device__ __forceinline__ void prep_chunk(unsigned char* sm, const Params& p, i
     }
 }
 
+// Scalar-gate variant, one warp: lane l handles tokens 2l and 2l + 1.  S_GAM gets the
+// inclusive in-chunk sum Gamma of log2 a (flat past the sequence end), S_GE 2^Gamma and
+// S_KF 2^(Gamma_63 - Gamma).
+__device__ __forceinline__ void gate_chunk_s(unsigned char* sm, const Params& p, int h, int64_t t0, int L) {
+    const int lane = threadIdx.x & 31;
+    const float nexpA = -expf(p.A_log[h]);
+    const float lb2 = p.lower_bound * kLog2e;
+    const float db2 = p.dt_bias[h] * kLog2e;
+    const int r0 = 2 * lane;
+    float2 gv = make_float2(0.f, 0.f);
+    if (r0 < L) gv.x = p.g_scalar[(t0 + r0) * p.H + h];
+    if (r0 + 1 < L) gv.y = p.g_scalar[(t0 + r0 + 1) * p.H + h];
+    float2 l = gate_log2_decay2(gv, make_float2(db2, db2), nexpA, lb2);
+    if (r0 >= L) l.x = 0.f;
+    if (r0 + 1 >= L) l.y = 0.f;
+    const float pair = l.x + l.y;
+    float incl = pair;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+    }
+    const float g0 = incl - pair + l.x, g1 = incl;
+    const float glast = __shfl_sync(0xffffffffu, incl, 31);
+    float* gam = reinterpret_cast<float*>(sm + S_GAM);
+    float* ge = reinterpret_cast<float*>(sm + S_GE);
+    float* kf = reinterpret_cast<float*>(sm + S_KF);
+    *reinterpret_cast<float2*>(gam + r0) = make_float2(g0, g1);
+    *reinterpret_cast<float2*>(ge + r0) = make_float2(fast_ex2(g0), fast_ex2(g1));
+    *reinterpret_cast<float2*>(kf + r0) = make_float2(fast_ex2(glast - g0), fast_ex2(glast - g1));
+}
+
+// Scalar-gate variant of prep_chunk: beta, and k = q = v = 0 on rows r >= L of all six
+// blocks (a block row is 128 contiguous bytes).
+__device__ __forceinline__ void prep_chunk_s(unsigned char* sm, const Params& p, int h, int64_t t0, int L,
+                                             int pt) {
+    float* sBeta = reinterpret_cast<float*>(sm + S_BETA);
+    if (pt < kChunk) sBeta[pt] = pt < L ? p.beta[(t0 + pt) * p.H + h] : 0.f;
+    for (int e = L * 8 + pt; e < kChunk * 8; e += kPrepThreads) {
+#pragma unroll
+        for (int b6 = 0; b6 < 6; ++b6)
+            *reinterpret_cast<uint4*>(sm + (uint32_t)b6 * 8192u + (uint32_t)e * 16u) = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
 // Warps 4-15: wait (bounded) for the chunk's inputs, then gate / prepare it.  Returns
 // false on a timeout (the abort flag is raised).
+template <bool kScalar>
 __device__ __forceinline__ bool stage_next_chunk(unsigned char* sm, const Params& p, uint64_t* bar_in,
                                                  uint32_t parity, volatile uint32_t* abort_flag, int h,
                                                  int64_t t0, int L) {
     const int warp = threadIdx.x >> 5;
     if (warp < kGateWarp0) return true;
+    if (kScalar && warp > kGateWarp0 && warp < kPrepWarp0) return true;   // one gate warp suffices
     bool ok = true;
     if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar_in, parity);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -360,11 +440,18 @@ __device__ __forceinline__ bool stage_next_chunk(unsigned char* sm, const Params
         }
         return false;
     }
-    if (warp < kPrepWarp0) gate_chunk(sm, p, h, L, threadIdx.x - kGateWarp0 * 32);
-    else prep_chunk(sm, p, h, t0, L, threadIdx.x - kPrepWarp0 * 32);
+    if constexpr (kScalar) {
+        if (warp < kPrepWarp0) gate_chunk_s(sm, p, h, t0, L);
+        else prep_chunk_s(sm, p, h, t0, L, threadIdx.x - kPrepWarp0 * 32);
+        fence_proxy_async();   // the zeroed rows are MMA operands
+    } else {
+        if (warp < kPrepWarp0) gate_chunk(sm, p, h, L, threadIdx.x - kGateWarp0 * 32);
+        else prep_chunk(sm, p, h, t0, L, threadIdx.x - kPrepWarp0 * 32);
+    }
     return true;
 }
 
+template <bool kScalar>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -451,10 +538,13 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         int k1, h1;
         int64_t t1, e1;
         if (next_chunk(p, sOrder, b, G, units, -1, 0, 0, &k1, &h1, &t1, &e1)) {
-            if (tid == 0) issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
+            if (tid == 0) {
+                if constexpr (kScalar) issue_chunk_loads_s(sm, bar_in, &tm_q, &tm_k, &tm_v, h1, t1);
+                else issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
+            }
             in_flight = true;
             const int L1 = (int)(e1 - t1 < kChunk ? e1 - t1 : kChunk);
-            stage_next_chunk(sm, p, bar_in, par(B_IN), sAbort, h1, t1, L1);
+            stage_next_chunk<kScalar>(sm, p, bar_in, par(B_IN), sAbort, h1, t1, L1);
             __syncthreads();
             if (*sAbort != 0u) aborted = true;
             else {
@@ -535,7 +625,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int64_t t1 = last ? tn : t0 + kChunk;
             const int64_t e1 = last ? en : x.eos;
             const int L1 = (int)(e1 - t1 < kChunk ? e1 - t1 : kChunk);
-            if (tid == 0 && has_next) prefetch_chunk(&tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
+            if (tid == 0 && has_next) prefetch_chunk<kScalar>(&tm_q, &tm_k, &tm_v, &tm_g, h1, t1);
             // this chunk was gated and prepared while the previous one solved for T; the
             // previous chunk's S update must have finished reading KH / U16
             if (pending(B_S)) {
@@ -546,6 +636,66 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 waited(B_S);
             }
             PHASE_MARK(1);
+            if constexpr (kScalar) {
+                // A/P straight from the inputs: [K ; Q] K^T, bf16, the decay applied at read-out
+                if (tid == 0) {
+                    fence_after_sync();
+                    const uint32_t a0 = smem_u32(sm + IN_Q);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(a0, 128, ks), IDESC_AP_S,
+                                ks > 0 ? 1u : 0u);
+                    mma_commit(bar_ap);
+                }
+                issued(B_AP);
+                PHASE_MARK(12);
+                // per-token scalings of the operand tiles; inputs and outputs share the
+                // swizzled geometry, so each thread works on one 16-byte position per block
+                {
+                    const int r = tid >> 3;
+                    const uint32_t off = (uint32_t)r * 128u + (uint32_t)(tid & 7) * 16u;
+                    const float be = sBeta[r];
+                    const float ge = reinterpret_cast<const float*>(sm + S_GE)[r];
+                    const float kf = reinterpret_cast<const float*>(sm + S_KF)[r];
+                    const float2 bg2 = make_float2(be * ge, be * ge), kf2 = make_float2(kf, kf);
+                    const float2 ge2 = make_float2(ge, ge), be2 = make_float2(be, be);
+#pragma unroll
+                    for (int cbk = 0; cbk < 2; ++cbk) {
+                        const uint4 kw = *reinterpret_cast<const uint4*>(sm + (uint32_t)cbk * 16384u + off);
+                        const uint4 qw = *reinterpret_cast<const uint4*>(sm + (uint32_t)cbk * 16384u + 8192u + off);
+                        const uint4 vw = *reinterpret_cast<const uint4*>(sm + 32768u + (uint32_t)cbk * 8192u + off);
+                        const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, qq[4] = {qw.x, qw.y, qw.z, qw.w},
+                                       vv[4] = {vw.x, vw.y, vw.z, vw.w};
+                        uint32_t obgk[4], okh[4], ogq[4], obv[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 kx = bf16x2_to_float2(kk[e]);
+                            obgk[e] = pack_f16(mul2(bg2, kx));
+                            okh[e] = pack_f16(mul2(kf2, kx));
+                            ogq[e] = pack_f16(mul2(ge2, bf16x2_to_float2(qq[e])));
+                            obv[e] = pack_f16(mul2(be2, bf16x2_to_float2(vv[e])));
+                        }
+                        const uint32_t cboff = (uint32_t)cbk * 8192u + off;
+                        st_v4(sm, BGK + cboff, obgk[0], obgk[1], obgk[2], obgk[3]);
+                        st_v4(sm, KH + cboff, okh[0], okh[1], okh[2], okh[3]);
+                        st_v4(sm, (cbk ? GQ1 : GQ0) + off, ogq[0], ogq[1], ogq[2], ogq[3]);
+                        st_v4(sm, BV + cboff, obv[0], obv[1], obv[2], obv[3]);
+                    }
+                    if (tid < kHeadDim)
+                        sGammaC[tid] = fast_ex2(reinterpret_cast<const float*>(sm + S_GAM)[kChunk - 1]);
+                }
+                PHASE_MARK(13);
+                fence_proxy_async();
+                __syncthreads();
+                PHASE_MARK(2);
+                if (wait_or_abort(bar_ap, par(B_AP), sAbort)) { aborted = true; break; }
+                waited(B_AP);
+                fence_after_sync();
+                // the A/P MMA has finished reading the inputs: load the next chunk
+                in_flight = has_next;
+                if (tid == 0 && in_flight) issue_chunk_loads_s(sm, bar_in, &tm_q, &tm_k, &tm_v, h1, t1);
+                PHASE_MARK(3);
+            } else {
             float2 Gc[8];   // inclusive sum of log2 a over this thread's octet (channel pair)
             {
                 const float* gin = reinterpret_cast<const float*>(sm + IN_G);
@@ -685,9 +835,50 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             waited(B_AP);
             fence_after_sync();
             PHASE_MARK(3);
+            }
 
             // ================= phase 3: A / P read-out =================
-            {
+            if constexpr (kScalar) {
+                // rows 0-63 of the accumulator are K K^T, rows 64-127 Q K^T; the scalar decay
+                // 2^(Gamma_r - Gamma_i) (<= 1 on and below the diagonal) is applied here
+                const bool isA = quarter < 2;
+                const int r = (quarter & 1) * 32 + lane;
+                const int J = sub;
+                uint32_t raw[16];
+                tmem_ld16(taddr(tbase, quarter, TM_AP + (uint32_t)J * 16u), raw);
+                tmem_wait_ld();
+                const float* gam = reinterpret_cast<const float*>(sm + S_GAM);
+                const float gr = gam[r];
+                float row[16];
+#pragma unroll
+                for (int q4 = 0; q4 < 16; q4 += 4) {
+                    const float4 gi = *reinterpret_cast<const float4*>(gam + J * 16 + q4);
+                    const float gvals[4] = {gi.x, gi.y, gi.z, gi.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = J * 16 + q4 + e;
+                        const bool keep = isA ? (i < r) : (i <= r);
+                        const float dec = fast_ex2(gr - gvals[e]);
+                        row[q4 + e] = keep ? __uint_as_float(raw[q4 + e]) * dec : 0.f;
+                    }
+                }
+                if (isA) {
+                    const float2 be2 = make_float2(sBeta[r], sBeta[r]);
+                    float* a32 = reinterpret_cast<float*>(sm + A32) + r * kF32Pitch + J * 16;
+#pragma unroll
+                    for (int i = 0; i < 16; i += 4) {
+                        const float2 lo2 = mul2(be2, make_float2(row[i], row[i + 1]));
+                        const float2 hi2 = mul2(be2, make_float2(row[i + 2], row[i + 3]));
+                        *reinterpret_cast<float4*>(a32 + i) = make_float4(lo2.x, lo2.y, hi2.x, hi2.y);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+                        st_v4(sm, P16 + sw128_chunk_off(r, J * 2 + c, 64), pack_f16(row[8 * c], row[8 * c + 1]),
+                              pack_f16(row[8 * c + 2], row[8 * c + 3]), pack_f16(row[8 * c + 4], row[8 * c + 5]),
+                              pack_f16(row[8 * c + 6], row[8 * c + 7]));
+                }
+            } else {
                 // quarter q holds rows 32 (q & 1) .. + 31 of A (q < 2) or P (q >= 2); warp `sub`
                 // assembles column block J = sub of those rows
                 const bool isA = quarter < 2;
@@ -725,7 +916,6 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (isA) {
                     const float be = sBeta[r];
                     float* a32 = reinterpret_cast<float*>(sm + A32) + r * kF32Pitch + J * 16;
-#pragma unroll
                     const float2 be2 = make_float2(be, be);
 #pragma unroll
                     for (int i = 0; i < 16; i += 4) {
@@ -868,7 +1058,7 @@ kda_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     for (int e = tid - kPrepWarp0 * 32; e < 8192 / 16; e += kPrepThreads)
                         st_v4(sm, Z16 + (uint32_t)e * 16u, 0u, 0u, 0u, 0u);
                 }
-                if (has_next) stage_next_chunk(sm, p, bar_in, par(B_IN), sAbort, h1, t1, L1);
+                if (has_next) stage_next_chunk<kScalar>(sm, p, bar_in, par(B_IN), sAbort, h1, t1, L1);
             }
             fence_proxy_async();
             fence_before_sync();
@@ -1105,17 +1295,19 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
+// 2-D map over [rows][cols] with a box of box_cols x 64 rows; swizzled maps put each box in
+// the 128-byte-swizzled K-major layout of the MMA operands.
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t elem, int64_t rows,
-              int64_t cols) {
+              int64_t cols, uint32_t box_cols = kHeadDim, bool swizzle128 = false) {
     auto fn = get_encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)cols * elem};
-    cuuint32_t box[2] = {(cuuint32_t)kHeadDim, (cuuint32_t)kChunk};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)kChunk};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace fused
@@ -1133,8 +1325,10 @@ extern "C" int kda_debug_phase_cycles(unsigned long long* out) {
 
 bool fused_supported(float lower_bound) { return lower_bound >= KDA_FUSED_MIN_LOWER_BOUND; }
 
-cudaError_t launch_fused(const StagedArgs& a, cudaStream_t stream) {
-    using namespace fused;
+namespace fused {
+
+template <bool kScalar>
+cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
     static int sm_count = 0;
     static bool attr_set = false;
     if (!sm_count) {
@@ -1144,18 +1338,23 @@ cudaError_t launch_fused(const StagedArgs& a, cudaStream_t stream) {
         if (sm_count <= 0) return cudaErrorInvalidDevice;
     }
     if (!attr_set) {
-        cudaError_t err = cudaFuncSetAttribute(kda_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)SMEM_ALLOC);
+        cudaError_t err = cudaFuncSetAttribute(kda_fused_kernel<kScalar>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
         if (err != cudaSuccess) return err;
         attr_set = true;
     }
     CUtensorMap tq, tk, tv, tg;
     const int64_t rows = a.total_tokens, cols = (int64_t)a.H * kHeadDim;
-    if (!make_map(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols) ||
-        !make_map(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols) ||
-        !make_map(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols) ||
-        !make_map(&tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols))
+    const uint32_t box = kScalar ? 64u : (uint32_t)kHeadDim;
+    if (!make_map(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box, kScalar) ||
+        !make_map(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box, kScalar) ||
+        !make_map(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box, kScalar))
         return cudaErrorInvalidValue;
+    if (kScalar) {
+        tg = tq;   // unused
+    } else if (!make_map(&tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols)) {
+        return cudaErrorInvalidValue;
+    }
     Params p;
     p.beta = a.beta;
     p.A_log = a.A_log;
@@ -1170,11 +1369,17 @@ cudaError_t launch_fused(const StagedArgs& a, cudaStream_t stream) {
     p.total_tokens = a.total_tokens;
     p.H = a.H;
     p.N = a.N;
+    p.g_scalar = kScalar ? a.g : nullptr;
     const int64_t units = (int64_t)a.N * a.H;
     const int grid = (int)(units < sm_count ? units : sm_count);
     if (grid <= 0) return cudaSuccess;
-    kda_fused_kernel<<<grid, kThreads, SMEM_ALLOC, stream>>>(tq, tk, tv, tg, p);
+    kda_fused_kernel<kScalar><<<grid, kThreads, SMEM_ALLOC, stream>>>(tq, tk, tv, tg, p);
     return cudaGetLastError();
 }
+
+}  // namespace fused
+
+cudaError_t launch_fused(const StagedArgs& a, cudaStream_t stream) { return fused::launch<false>(a, stream); }
+cudaError_t launch_fused_gdn(const StagedArgs& a, cudaStream_t stream) { return fused::launch<true>(a, stream); }
 
 }  // namespace kda

@@ -42,6 +42,8 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
 
 // The fused persistent tcgen05 kernel (same arguments; no workspace).
 cudaError_t launch_fused(const StagedArgs& a, cudaStream_t stream);
+// Scalar-gate (Gated DeltaNet) variant: a.g is [Ttot][H], a.dt_bias [H]; any lower bound.
+cudaError_t launch_fused_gdn(const StagedArgs& a, cudaStream_t stream);
 bool fused_supported(float lower_bound);
 
 }  // namespace kda

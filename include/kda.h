@@ -196,6 +196,28 @@ kda_status kda_decode(const void* q, const void* k, const void* v,
                       float* state, void* out,
                       int32_t batch, int32_t num_heads, kda_stream_t stream);
 
+/*
+ * kda_gdn_fwd -- the scalar-gate variant (Gated DeltaNet): the same recurrence with
+ * one decay per (token, head) instead of one per key channel,
+ *   log a_t = max(-exp(A_log_h) * softplus(g_t,h + dt_bias_h), lower_bound),
+ * applied to every channel of the state.  The FlashKDA H20 benchmark table
+ * (toolarium.ru, section "Что показывают H20-бенчмарки") compares against such a
+ * "gdn" kernel in its second column.
+ *   q, k, v, out, initial_state, final_state, cu_seqlens, dims: as for kda_fwd
+ *   g        fp32 [B*T, H]   (one gate input per token and head)
+ *   beta     fp32 [B*T, H]
+ *   A_log    fp32 [H],  dt_bias fp32 [H]
+ * Any lower_bound <= 0 is accepted (the intra-chunk decays are formed pairwise).
+ * Errors, alignment, aliasing and asynchrony as for kda_fwd.
+ */
+kda_status kda_gdn_fwd(const void* q, const void* k, const void* v,
+                       const float* g, const float* beta,
+                       const float* A_log, const float* dt_bias,
+                       float lower_bound, float scale,
+                       const float* initial_state, const int32_t* cu_seqlens,
+                       void* out, float* final_state,
+                       kda_dims dims, kda_stream_t stream);
+
 /* Human-readable name of a status code (static storage; never NULL). */
 const char* kda_strerror(kda_status status);
 

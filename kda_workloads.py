@@ -129,3 +129,12 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> dict:
                 initial_state=init, cu_seqlens=cu,
                 batch=1 if w.packed else w.N,
                 seqlen=w.T if w.packed else w.seq_lens[0], N=w.N)
+
+
+def gdn_inputs(x: dict) -> dict:
+    """Inputs of the scalar-gate variant drawn from the same seeded tensors: the gate
+    input and dt_bias of channel 0 (same distributions, one value per token-head / head)."""
+    y = dict(x)
+    y["g"] = x["g"][..., 0].contiguous()
+    y["dt_bias"] = x["dt_bias"][:, 0].contiguous()
+    return y

@@ -182,6 +182,24 @@ def recurrent(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, scale: float
 # ----------------------------------------------------------------------------
 # the chunked form (second, independent formulation)
 
+def gdn_recurrent(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, scale: float,
+                  initial_state=None, cu_seqlens=None, **kw):
+    """Scalar-gate variant (Gated DeltaNet): the recurrence above with one decay per
+    (token, head), log a_t = max(-exp(A_log_h) softplus(g_t,h + dt_bias_h), lower_bound),
+    shared by all K channels.  g: [T, H] (or leading batch dims); dt_bias: [H].  It is
+    ``recurrent`` with g and dt_bias repeated over the channel axis.  The FlashKDA H20
+    table (toolarium.ru, section "Что показывают H20-бенчмарки") compares against
+    such a "gdn" kernel.
+    """
+    g32 = _f32(g)
+    H = g32.shape[-1]
+    K = (q.shape[-1] if hasattr(q, "shape") else 128)
+    g3 = np.repeat(g32.reshape(-1, H)[:, :, None], K, axis=2)
+    db = np.repeat(_f32(dt_bias).reshape(H, 1), K, axis=1)
+    return recurrent(q, k, v, g3, beta, A_log, db, lower_bound, scale, initial_state,
+                     cu_seqlens, **kw)
+
+
 def _softplus_np(x: np.ndarray) -> np.ndarray:
     return np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))
 

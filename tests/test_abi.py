@@ -11,7 +11,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _build():
-    from gated_delta_rule_135_b200 import build
+    import kda_build as build
     build.build()
 
 
@@ -140,3 +140,14 @@ def test_decode_rejects_bad_arguments():
     assert call(bad) == 3
     assert call(p[:8] + [p[0]]) == 1          # out aliases q
     assert call(p, B=0) == 0                  # nothing to do
+
+
+def test_gdn_rejects_bad_arguments():
+    assert kda.lib().kda_gdn_fwd(*([FAKE + i * (1 << 28) for i in range(7)]), ctypes.c_float(0.5),
+                                 ctypes.c_float(0.1), None, None, FAKE + (7 << 28), None, _dims(), None) == 1
+    assert kda.lib().kda_gdn_fwd(*([FAKE + i * (1 << 28) for i in range(7)]), ctypes.c_float(-1.0),
+                                 ctypes.c_float(0.1), None, None, FAKE + (7 << 28), None, _dims(hk=64), None) == 2
+    p = [FAKE + i * (1 << 28) for i in range(7)]
+    p[3] += 4
+    assert kda.lib().kda_gdn_fwd(*p, ctypes.c_float(-1.0), ctypes.c_float(0.1), None, None,
+                                 FAKE + (7 << 28), None, _dims(), None) == 3

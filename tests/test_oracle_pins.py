@@ -227,6 +227,25 @@ def test_channel_uniform_alpha_is_gated_deltanet():
         np.testing.assert_allclose(fin[0, h], s_ref, rtol=1e-10, atol=1e-12)
 
 
+def test_gdn_wrapper_is_scalar_decay_chunked_form():
+    """gdn_recurrent (one gate input per token-head, dt_bias per head) equals the
+    independent chunked Gated DeltaNet form with the gate evaluated token by token."""
+    rng = np.random.default_rng(11)
+    q, k, v, beta, S0 = _small_case(rng, T=45)
+    T, H, K = q.shape
+    g = rng.normal(size=(T, H)).astype(np.float32)
+    A_log = np.log(rng.uniform(1, 16, size=H)).astype(np.float32)
+    dt_bias = (0.1 * rng.normal(size=H)).astype(np.float32)
+    out, fin = oracle.gdn_recurrent(q, k, v, g, beta, A_log, dt_bias, -4.0, 0.5, S0)
+    la = oracle.gate_np(g[:, :, None], A_log, dt_bias[:, None], -4.0)[:, :, 0]
+    qf, kf, vf = (x.double().numpy() for x in (q, k, v))
+    for h in range(H):
+        o_ref, s_ref = _gdn_chunked(qf[:, h], kf[:, h], vf[:, h], beta[:, h].astype(np.float64),
+                                    la[:, h], S0[0, h], 0.5)
+        np.testing.assert_allclose(out[:, h], o_ref, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(fin[0, h], s_ref, rtol=1e-10, atol=1e-12)
+
+
 def test_additive_update_is_linear_attention():
     rng = np.random.default_rng(6)
     q, k, v, beta, S0 = _small_case(rng, T=33)

@@ -22,7 +22,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _kda():
-    from gated_delta_rule_135_b200 import build
+    import kda_build as build
     build.build()
     import gated_delta_rule_135_b200 as kda
     return kda
