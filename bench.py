@@ -84,6 +84,7 @@ def algorithmic_bytes(w: W.Workload, gdn: bool = False) -> int:
 
 KERNEL_SOURCES = {
     "kda_fused_kernel": ("kda_fused.cuh", "umma.cuh", "warp_mma.cuh", "kda_common.cuh"),
+    "kda_fused_kernel<scalar gate>": ("kda_fused.cuh", "umma.cuh", "warp_mma.cuh", "kda_common.cuh"),
     "kda_decode_kernel": ("kda_decode.cuh", "kda_common.cuh"),
 }
 
@@ -101,6 +102,7 @@ def kernel_source_hash(kernel: str = "kda_fused_kernel") -> str:
 
 
 TRAFFIC_FILES = {"kda_fused_kernel": "kda_fused_traffic.json",
+                 "kda_fused_kernel<scalar gate>": "kda_gdn_traffic.json",
                  "kda_decode_kernel": "kda_decode_traffic.json"}
 
 
@@ -485,7 +487,8 @@ def main():
     achieved = alg_bytes / (kernel_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak,
-            "traffic": (dram_traffic_from_profile("kda_fused_kernel", w.T * w.H) if fused and not args.gdn else None),
+            "traffic": (dram_traffic_from_profile("kda_fused_kernel<scalar gate>" if args.gdn else "kda_fused_kernel",
+                                                  w.T * w.H) if fused else None),
             "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
             else "fallback 6650 GB/s",
             "kernel": ("kda_fused_kernel<scalar gate>" if args.gdn else "kda_fused_kernel") if fused
