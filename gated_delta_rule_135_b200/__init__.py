@@ -74,6 +74,10 @@ def _load():
     lib.kda_fwd_staged_noalloc.argtypes = fwd_args + [vp]
     lib.kda_noalloc_scratch_bytes.restype = ctypes.c_size_t
     lib.kda_noalloc_scratch_bytes.argtypes = []
+    lib.kda_state_affine.restype = ctypes.c_int
+    lib.kda_state_affine.argtypes = [vp, vp, vp, vp, ctypes.c_int32, vp]
+    lib.kda_gdn_decode.restype = ctypes.c_int
+    lib.kda_gdn_decode.argtypes = [vp] * 7 + [f32, f32, vp, vp, ctypes.c_int32, ctypes.c_int32, vp]
     lib.kda_gdn_fwd.restype = ctypes.c_int
     lib.kda_gdn_fwd.argtypes = fwd_args + [vp]
     lib.kda_decode.restype = ctypes.c_int
@@ -87,7 +91,8 @@ _lib = _load()
 EXPORTED = ("kda_fwd", "kda_fwd_staged", "kda_staged_workspace_size",
             "kda_staged_workspace_layout", "kda_strerror", "kda_check_device_error",
             "kda_last_device_error_bits", "kda_version", "kda_fwd_staged_noalloc",
-            "kda_noalloc_scratch_bytes", "kda_decode", "kda_gdn_fwd")
+            "kda_noalloc_scratch_bytes", "kda_decode", "kda_gdn_fwd", "kda_gdn_decode",
+            "kda_state_affine")
 
 
 def lib() -> ctypes.CDLL:
@@ -284,6 +289,43 @@ def kda_decode(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, scale: floa
                          _stream_ptr(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_decode")
+    return out
+
+
+def kda_gdn_decode(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, scale: float, state,
+               out=None, *, stream=None):
+    """Calls kda_gdn_decode, the scalar-gate decode step.  q/k/v: bf16 [B, H, 128];
+    g: fp32 [B, H]; beta: fp32 [B, H]; dt_bias: fp32 [H]; state: fp32 [B, H, 128, 128],
+    updated in place.  Returns out (bf16 [B, H, 128])."""
+    dev = q.device
+    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16), ("v", v, torch.bfloat16),
+                        ("g", g, torch.float32), ("beta", beta, torch.float32),
+                        ("A_log", A_log, torch.float32), ("dt_bias", dt_bias, torch.float32),
+                        ("state", state, torch.float32)):
+        _check_tensor(name, t, dt, dev)
+    B, H = q.shape[0], q.shape[1]
+    if out is None:
+        out = torch.empty(B, H, HEAD_DIM, dtype=torch.bfloat16, device=dev)
+    st = _lib.kda_gdn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias),
+                         float(lower_bound), float(scale), _ptr(state), _ptr(out), int(B), int(H),
+                         _stream_ptr(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_gdn_decode")
+    return out
+
+
+def kda_state_affine(A: torch.Tensor, S: torch.Tensor, B: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     *, stream=None) -> torch.Tensor:
+    """Calls kda_state_affine: out[h] = A[h] @ S[h] + B[h]; all fp32 [H, 128, 128]."""
+    dev = A.device
+    for name, t in (("A", A), ("S", S), ("B", B)):
+        _check_tensor(name, t, torch.float32, dev)
+    if out is None:
+        out = torch.empty_like(B)
+    H = A.numel() // (HEAD_DIM * HEAD_DIM)
+    st = _lib.kda_state_affine(_ptr(A), _ptr(S), _ptr(B), _ptr(out), int(H), _stream_ptr(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_state_affine")
     return out
 
 

@@ -14,6 +14,7 @@
 #include "kda_staged.cuh"
 #include "kda_fused.cuh"
 #include "kda_decode.cuh"
+#include "kda_cp.cuh"
 
 namespace {
 
@@ -22,6 +23,7 @@ using kda::StagedArgs;
 thread_local uint32_t t_last_device_bits = 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
     if (!a || !b || an == 0 || bn == 0) return false;
@@ -62,9 +64,13 @@ kda_status prepare(const void* q, const void* k, const void* v, const float* g, 
     const int64_t H = d.num_heads;
     if (total > 0 && (!q || !k || !v || !g || !beta || !out)) return KDA_ERR_INVALID_ARG;
     if (!A_log || !dt_bias) return KDA_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens, out, final_state};
+    // TMA-loaded and vector-accessed arrays need 16-byte bases; beta (and the scalar-gate
+    // g) are read one element at a time, so 4 bytes suffice and token-offset slices work
+    const void* ptrs[] = {q, k, v, g_per_head > 1 ? (const void*)g : nullptr, A_log, dt_bias, initial_state,
+                          cu_seqlens, out, final_state};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return KDA_ERR_ALIGNMENT;
+    if ((beta && !aligned4(beta)) || (g_per_head == 1 && g && !aligned4(g))) return KDA_ERR_ALIGNMENT;
     const size_t tok = (size_t)total * (size_t)H;
     const size_t out_bytes = tok * kda::kHeadDim * 2;
     const size_t st_bytes = (size_t)N * H * kda::kHeadDim * kda::kHeadDim * 4;
@@ -238,9 +244,12 @@ kda_status kda_gdn_fwd(const void* q, const void* k, const void* v, const float*
     return kda::launch_fused_gdn(a, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
-kda_status kda_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                      const float* A_log, const float* dt_bias, float lower_bound, float scale,
-                      float* state, void* out, int32_t batch, int32_t num_heads, kda_stream_t stream) {
+namespace {
+
+kda_status decode_common(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                         const float* A_log, const float* dt_bias, float lower_bound, float scale,
+                         float* state, void* out, int32_t batch, int32_t num_heads, kda_stream_t stream,
+                         bool scalar_gate) {
     if (batch < 0 || num_heads < 1) return KDA_ERR_INVALID_ARG;
     if (isnan(lower_bound) || lower_bound > 0.f || !isfinite(scale)) return KDA_ERR_INVALID_ARG;
     if (batch == 0) return KDA_OK;
@@ -251,14 +260,48 @@ kda_status kda_decode(const void* q, const void* k, const void* v, const float* 
     const size_t bh = (size_t)batch * num_heads;
     const size_t ob = bh * kda::kHeadDim * 2;
     if (overlaps(out, ob, q, ob) || overlaps(out, ob, k, ob) || overlaps(out, ob, v, ob) ||
-        overlaps(out, ob, g, bh * kda::kHeadDim * 4) || overlaps(out, ob, beta, bh * 4) ||
+        overlaps(out, ob, g, bh * (scalar_gate ? 1 : kda::kHeadDim) * 4) || overlaps(out, ob, beta, bh * 4) ||
         overlaps(out, ob, state, bh * kda::kHeadDim * kda::kHeadDim * 4))
         return KDA_ERR_INVALID_ARG;
     kda_status st = device_ok();
     if (st != KDA_OK) return st;
     return kda::launch_decode(q, k, v, g, beta, A_log, dt_bias, lower_bound, scale, state, out, batch,
-                              num_heads, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+                              num_heads, reinterpret_cast<cudaStream_t>(stream), scalar_gate) == cudaSuccess
                ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace
+
+kda_status kda_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                      const float* A_log, const float* dt_bias, float lower_bound, float scale,
+                      float* state, void* out, int32_t batch, int32_t num_heads, kda_stream_t stream) {
+    return decode_common(q, k, v, g, beta, A_log, dt_bias, lower_bound, scale, state, out, batch, num_heads,
+                         stream, false);
+}
+
+kda_status kda_state_affine(const float* A, const float* S, const float* B, float* out, int32_t num_heads,
+                            kda_stream_t stream) {
+    if (num_heads < 0) return KDA_ERR_INVALID_ARG;
+    if (num_heads == 0) return KDA_OK;
+    if (!A || !S || !B || !out) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {A, S, B, out};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+    const size_t bytes = (size_t)num_heads * kda::kHeadDim * kda::kHeadDim * 4;
+    if (overlaps(out, bytes, A, bytes) || overlaps(out, bytes, S, bytes)) return KDA_ERR_INVALID_ARG;
+    kda_status st = device_ok();
+    if (st != KDA_OK) return st;
+    return kda::launch_state_affine(A, S, B, out, num_heads, reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? KDA_OK
+               : KDA_ERR_CUDA;
+}
+
+kda_status kda_gdn_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                          const float* A_log, const float* dt_bias, float lower_bound, float scale,
+                          float* state, void* out, int32_t batch, int32_t num_heads, kda_stream_t stream) {
+    return decode_common(q, k, v, g, beta, A_log, dt_bias, lower_bound, scale, state, out, batch, num_heads,
+                         stream, true);
 }
 
 const char* kda_strerror(kda_status status) {

@@ -19,6 +19,8 @@ namespace decode {
 
 constexpr int kThreads = kHeadDim;   // one thread per state column
 
+// kScalar: the scalar-gate variant, with g [B*H] and dt_bias [H] (one decay for all channels).
+template <bool kScalar>
 __global__ void __launch_bounds__(kThreads) kda_decode_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, const float* __restrict__ g, const float* __restrict__ beta,
@@ -33,7 +35,8 @@ __global__ void __launch_bounds__(kThreads) kda_decode_kernel(
     __shared__ float s_q[kHeadDim];          // q_c
     {
         const int64_t idx = (int64_t)bh * kHeadDim + tid;   // channel c = tid
-        const float la = gate_log_decay(g[idx] + dt_bias[h * kHeadDim + tid], -expf(A_log[h]), lower_bound);
+        const float gin = kScalar ? g[bh] + dt_bias[h] : g[idx] + dt_bias[h * kHeadDim + tid];
+        const float la = gate_log_decay(gin, -expf(A_log[h]), lower_bound);
         const float a = expf(la);
         const float kc = __bfloat162float(k[idx]);
         s_a[tid] = a;
@@ -65,10 +68,11 @@ __global__ void __launch_bounds__(kThreads) kda_decode_kernel(
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
                           const float* A_log, const float* dt_bias, float lower_bound, float scale,
-                          float* state, void* out, int batch, int H, cudaStream_t stream) {
+                          float* state, void* out, int batch, int H, cudaStream_t stream, bool scalar_gate) {
     const int64_t blocks = (int64_t)batch * H;
     if (blocks == 0) return cudaSuccess;
-    decode::kda_decode_kernel<<<(unsigned)blocks, decode::kThreads, 0, stream>>>(
+    auto kernel = scalar_gate ? decode::kda_decode_kernel<true> : decode::kda_decode_kernel<false>;
+    kernel<<<(unsigned)blocks, decode::kThreads, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
         static_cast<const __nv_bfloat16*>(v), g, beta, A_log, dt_bias, lower_bound, scale, state,
         static_cast<__nv_bfloat16*>(out), H);

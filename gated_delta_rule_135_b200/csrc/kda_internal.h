@@ -38,7 +38,12 @@ cudaError_t launch_staged(const StagedArgs& a, char* workspace, const StagedLayo
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
                           const float* A_log, const float* dt_bias, float lower_bound, float scale,
-                          float* state, void* out, int batch, int H, cudaStream_t stream);
+                          float* state, void* out, int batch, int H, cudaStream_t stream,
+                          bool scalar_gate = false);
+
+// out_h = A_h S_h + B_h for h < H (all [128][128] fp32); out must not overlap A or S.
+cudaError_t launch_state_affine(const float* A, const float* S, const float* B, float* out, int H,
+                                cudaStream_t stream);
 
 // The fused persistent tcgen05 kernel (same arguments; no workspace).
 cudaError_t launch_fused(const StagedArgs& a, cudaStream_t stream);

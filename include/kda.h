@@ -31,7 +31,8 @@
  * (empty sequences are allowed: their final state is their initial state).
  * cu_seqlens is read only on the device: no call synchronises with the host.
  *
- * Alignment: every tensor base address must be 16-byte aligned.
+ * Alignment: every tensor base address must be 16-byte aligned, except beta (and the
+ * scalar-gate g of kda_gdn_fwd), which need 4 bytes: slices at any token offset.
  * Aliasing: final_state may alias initial_state (in-place state update); out
  * must not overlap any input.
  * Streams: every compute call is asynchronous on `stream` (a cudaStream_t;
@@ -197,6 +198,17 @@ kda_status kda_decode(const void* q, const void* k, const void* v,
                       int32_t batch, int32_t num_heads, kda_stream_t stream);
 
 /*
+ * kda_gdn_decode -- one decode step of the scalar-gate variant: as kda_decode, with
+ * g fp32 [batch, H] and dt_bias fp32 [H] (one decay per sequence and head).
+ */
+kda_status kda_gdn_decode(const void* q, const void* k, const void* v,
+                          const float* g, const float* beta,
+                          const float* A_log, const float* dt_bias,
+                          float lower_bound, float scale,
+                          float* state, void* out,
+                          int32_t batch, int32_t num_heads, kda_stream_t stream);
+
+/*
  * kda_gdn_fwd -- the scalar-gate variant (Gated DeltaNet): the same recurrence with
  * one decay per (token, head) instead of one per key channel,
  *   log a_t = max(-exp(A_log_h) * softplus(g_t,h + dt_bias_h), lower_bound),
@@ -217,6 +229,18 @@ kda_status kda_gdn_fwd(const void* q, const void* k, const void* v,
                        const float* initial_state, const int32_t* cu_seqlens,
                        void* out, float* final_state,
                        kda_dims dims, kda_stream_t stream);
+
+/*
+ * kda_state_affine -- one step of the context-parallel state fold:
+ *   out[h] = A[h] S[h] + B[h]   for h < num_heads, all fp32 [num_heads][128][128] ([k][v]).
+ * The forward is affine in the state a segment starts from.  For a segment, A is its final
+ * state from initial state I with v = 0, and B its final state from initial state 0.  So
+ * when one long sequence is split into segments (one per rank, for the 128k-1M contexts the
+ * FlashKDA posts target: donniechu.com, "Số liệu kỹ thuật"), segment r starts from
+ * S_r = A_{r-1} S_{r-1} + B_{r-1}.  out may alias B but not A or S.  Errors as for kda_fwd.
+ */
+kda_status kda_state_affine(const float* A, const float* S, const float* B, float* out,
+                            int32_t num_heads, kda_stream_t stream);
 
 /* Human-readable name of a status code (static storage; never NULL). */
 const char* kda_strerror(kda_status status);

@@ -88,9 +88,21 @@ def test_rejects_bad_dims():
     assert _call(_dims(batch=2), cu=FAKE + (1 << 33)) == 1
 
 
-@pytest.mark.parametrize("which", range(8))
+@pytest.mark.parametrize("which", [0, 1, 2, 3, 5, 6, 7])
 def test_rejects_misaligned_pointers(which):
     assert _call(_dims(), misalign=which) == 3
+
+
+def test_beta_needs_only_element_alignment():
+    # beta (index 4) is read element by element: +8 bytes passes validation (the call then
+    # stops at the device check, with no GPU here); +2 bytes is rejected
+    p = [FAKE + i * (1 << 28) for i in range(8)]
+    p[4] += 2
+    assert kda.lib().kda_fwd(*p[:7], ctypes.c_float(-5.0), ctypes.c_float(0.1), None, None, p[7], None,
+                             _dims(), None) == 3
+    p[4] += 6
+    assert kda.lib().kda_fwd(*p[:7], ctypes.c_float(-5.0), ctypes.c_float(0.1), None, None, p[7], None,
+                             _dims(), None) != 3
 
 
 def test_rejects_output_aliasing_an_input():
@@ -148,6 +160,6 @@ def test_gdn_rejects_bad_arguments():
     assert kda.lib().kda_gdn_fwd(*([FAKE + i * (1 << 28) for i in range(7)]), ctypes.c_float(-1.0),
                                  ctypes.c_float(0.1), None, None, FAKE + (7 << 28), None, _dims(hk=64), None) == 2
     p = [FAKE + i * (1 << 28) for i in range(7)]
-    p[3] += 4
+    p[3] += 2          # the scalar gate needs element (4-byte) alignment
     assert kda.lib().kda_gdn_fwd(*p, ctypes.c_float(-1.0), ctypes.c_float(0.1), None, None,
                                  FAKE + (7 << 28), None, _dims(), None) == 3

@@ -69,3 +69,25 @@ def test_prefill_then_decode_equals_longer_prefill():
     o = o.float().cpu().numpy().astype(np.float64)
     assert oracle.rel_l2(o, ref_last) <= OUT_REL_L2
     assert oracle.rel_l2(state.cpu().numpy(), ref_f) <= STATE_REL_L2
+
+
+@pytest.mark.parametrize("B,T,H", [(3, 6, 4)])
+def test_gdn_decode_steps_match_recurrence(B, T, H):
+    kda = _kda()
+    w = W.custom([T] * B, H=H, packed=False, init="normal", wid=53)
+    x = W.gdn_inputs(W.make_inputs(w))
+    xd = to_device(x)
+    ref_o, ref_f = oracle.gdn_recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], x["A_log"],
+                                        x["dt_bias"], x["lower_bound"], x["scale"], x["initial_state"],
+                                        oracle.fixed_offsets(B, T))
+    state = xd["initial_state"].clone()
+    outs = []
+    for t in range(T):
+        s = _step_inputs(xd, B, T, t)
+        outs.append(kda.kda_gdn_decode(s["q"], s["k"], s["v"], s["g"], s["beta"], xd["A_log"], xd["dt_bias"],
+                                       x["lower_bound"], x["scale"], state))
+    torch.cuda.synchronize()
+    o = torch.stack(outs, dim=1).reshape(B * T, H, 128).float().cpu().numpy().astype(np.float64)
+    assert oracle.rel_l2(o, ref_o) <= OUT_REL_L2
+    assert oracle.max_abs(o, ref_o) <= OUT_MAX_ABS
+    assert oracle.rel_l2(state.cpu().numpy(), ref_f) <= STATE_REL_L2
