@@ -48,6 +48,11 @@ class kda_staged_layout(ctypes.Structure):
                 ("total", ctypes.c_size_t), ("max_chunks", ctypes.c_int64)]
 
 
+class kda_grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dq", "dk", "dv", "dg", "dbeta", "dA_log", "ddt_bias",
+                                               "d_initial_state")]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libkda.so not built ({LIB_PATH}); run gated_delta_rule_135_b200/build.py")
@@ -80,6 +85,11 @@ def _load():
     lib.kda_gdn_decode.argtypes = [vp] * 7 + [f32, f32, vp, vp, ctypes.c_int32, ctypes.c_int32, vp]
     lib.kda_gdn_fwd.restype = ctypes.c_int
     lib.kda_gdn_fwd.argtypes = fwd_args + [vp]
+    lib.kda_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.kda_bwd_workspace_size.argtypes = [kda_dims, ctypes.c_int]
+    lib.kda_bwd.restype = ctypes.c_int
+    lib.kda_bwd.argtypes = [vp] * 7 + [f32, f32, vp, vp, vp, vp, ctypes.POINTER(kda_grads), kda_dims, vp,
+                                       ctypes.c_size_t, vp]
     lib.kda_decode.restype = ctypes.c_int
     lib.kda_decode.argtypes = [vp] * 7 + [f32, f32, vp, vp, ctypes.c_int32, ctypes.c_int32, vp]
     return lib
@@ -92,7 +102,7 @@ EXPORTED = ("kda_fwd", "kda_fwd_staged", "kda_staged_workspace_size",
             "kda_staged_workspace_layout", "kda_strerror", "kda_check_device_error",
             "kda_last_device_error_bits", "kda_version", "kda_fwd_staged_noalloc",
             "kda_noalloc_scratch_bytes", "kda_decode", "kda_gdn_fwd", "kda_gdn_decode",
-            "kda_state_affine")
+            "kda_state_affine", "kda_bwd", "kda_bwd_workspace_size")
 
 
 def lib() -> ctypes.CDLL:
@@ -327,6 +337,53 @@ def kda_state_affine(A: torch.Tensor, S: torch.Tensor, B: torch.Tensor, out: Opt
     if st != KDA_OK:
         raise KdaError(st, "kda_state_affine")
     return out
+
+
+GRAD_NAMES = ("dq", "dk", "dv", "dg", "dbeta", "dA_log", "ddt_bias", "d_initial_state")
+
+
+def kda_bwd(q, k, v, g, beta, A_log, dt_bias, lower_bound: float, scale: float, d_out,
+            initial_state=None, cu_seqlens=None, d_final_state=None, *, want_d_initial: bool = True,
+            grads: Optional[dict] = None, workspace: Optional[torch.Tensor] = None, batch: int = 1,
+            stream=None) -> dict:
+    """Calls kda_bwd: the gradients of <d_out, out> + <d_final_state, final_state> for the
+    forward kda_fwd computes from the same arguments.  d_out: bf16 like q;
+    d_final_state: fp32 [N, H, 128, 128] or None.  Returns a dict of fp32 tensors
+    (GRAD_NAMES; d_initial_state only with want_d_initial).  `grads` may supply some or all
+    output tensors; `workspace` a uint8 device buffer of kda_bwd_workspace_size bytes."""
+    dims = _marshal(q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens, d_out, None, batch)
+    _check_tensor("d_final_state", d_final_state, torch.float32, q.device)
+    H = q.shape[-2]
+    shapes = {"dq": q.shape, "dk": q.shape, "dv": v.shape, "dg": g.shape, "dbeta": beta.shape,
+              "dA_log": A_log.shape, "ddt_bias": dt_bias.shape}
+    if want_d_initial:
+        N = dims.num_seqs if cu_seqlens is not None else dims.batch
+        shapes["d_initial_state"] = (N, H, HEAD_DIM, HEAD_DIM)
+    out = dict(grads or {})
+    for name, shape in shapes.items():
+        if out.get(name) is None:
+            out[name] = torch.empty(shape, dtype=torch.float32, device=q.device)
+        _check_tensor(name, out[name], torch.float32, q.device)
+    gr = kda_grads(*[None if out.get(n) is None else out[n].data_ptr() for n in GRAD_NAMES])
+    if workspace is None:
+        nbytes = _lib.kda_bwd_workspace_size(dims, int(cu_seqlens is not None))
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    st = _lib.kda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(A_log), _ptr(dt_bias),
+                      float(lower_bound), float(scale), _ptr(initial_state), _ptr(cu_seqlens), _ptr(d_out),
+                      _ptr(d_final_state), ctypes.byref(gr), dims, _ptr(workspace),
+                      ctypes.c_size_t(workspace.numel()), _stream_ptr(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_bwd")
+    return out
+
+
+def kda_bwd_workspace_size(q: torch.Tensor, cu_seqlens: Optional[torch.Tensor] = None, batch: int = 1) -> int:
+    H = q.shape[-2]
+    total = q.numel() // (H * HEAD_DIM)
+    if cu_seqlens is None and q.dim() == 4:
+        batch = q.shape[0]
+    dims = make_dims(H, total_tokens=total, cu_seqlens=cu_seqlens, batch=batch)
+    return int(_lib.kda_bwd_workspace_size(dims, int(cu_seqlens is not None)))
 
 
 def kda_check_device_error(stream=None) -> int:

@@ -15,6 +15,7 @@
 #include "kda_fused.cuh"
 #include "kda_decode.cuh"
 #include "kda_cp.cuh"
+#include "kda_backward.cuh"
 
 namespace {
 
@@ -45,7 +46,8 @@ kda_status device_ok() {
 kda_status prepare(const void* q, const void* k, const void* v, const float* g, const float* beta,
                    const float* A_log, const float* dt_bias, float lower_bound, float scale,
                    const float* initial_state, const int32_t* cu_seqlens, void* out,
-                   float* final_state, const kda_dims& d, StagedArgs* a, size_t g_per_head = kda::kHeadDim) {
+                   float* final_state, const kda_dims& d, StagedArgs* a, size_t g_per_head = kda::kHeadDim,
+                   bool check_device = true) {
     if (d.head_dim_k != kda::kHeadDim || d.head_dim_v != kda::kHeadDim) return KDA_ERR_UNSUPPORTED;
     if (d.num_heads < 1 || d.seqlen < 0) return KDA_ERR_INVALID_ARG;
     if (isnan(lower_bound) || lower_bound > 0.f) return KDA_ERR_INVALID_ARG;
@@ -87,7 +89,7 @@ kda_status prepare(const void* q, const void* k, const void* v, const float* g, 
     a->initial_state = initial_state; a->cu_seqlens = cu_seqlens;
     a->out = out; a->final_state = final_state;
     a->seqlen = d.seqlen; a->total_tokens = total; a->H = (int)H; a->N = (int)N;
-    return device_ok();
+    return check_device ? device_ok() : KDA_OK;
 }
 
 // Carries the initial state to the final state when no token is processed.
@@ -246,6 +248,72 @@ kda_status kda_gdn_fwd(const void* q, const void* k, const void* v, const float*
 
 namespace {
 
+struct Span {
+    const void* p;
+    size_t n;
+};
+
+// Validates the backward's arguments: the forward's (with d_out in the place of out) and the
+// gradient outputs, which must be aligned and overlap neither an input nor one another.
+kda_status prepare_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                       const float* A_log, const float* dt_bias, float lower_bound, float scale,
+                       const float* initial_state, const int32_t* cu_seqlens, const void* d_out,
+                       const float* d_final, const kda_grads* gr, const kda_dims& d, StagedArgs* a,
+                       kda::BwdArgs* b) {
+    if (!gr) return KDA_ERR_INVALID_ARG;
+    kda_status st = prepare(q, k, v, g, beta, A_log, dt_bias, lower_bound, scale, initial_state, cu_seqlens,
+                            const_cast<void*>(d_out), nullptr, d, a, kda::kHeadDim, false);
+    if (st != KDA_OK) return st;
+    const size_t tok = (size_t)a->total_tokens * a->H, D = kda::kHeadDim;
+    const size_t st_bytes = (size_t)a->N * a->H * D * D * 4;
+    if (tok > 0 && (!gr->dq || !gr->dk || !gr->dv || !gr->dg || !gr->dbeta)) return KDA_ERR_INVALID_ARG;
+    if (!gr->dA_log || !gr->ddt_bias) return KDA_ERR_INVALID_ARG;
+    const void* a16[] = {gr->dq, gr->dk, gr->dv, gr->dg, gr->dA_log, gr->ddt_bias, gr->d_initial_state, d_final};
+    for (const void* p : a16)
+        if (p && !aligned16(p)) return KDA_ERR_ALIGNMENT;
+    if (gr->dbeta && !aligned4(gr->dbeta)) return KDA_ERR_ALIGNMENT;
+    const Span outs[] = {{gr->dq, tok * D * 4}, {gr->dk, tok * D * 4}, {gr->dv, tok * D * 4},
+                         {gr->dg, tok * D * 4}, {gr->dbeta, tok * 4}, {gr->dA_log, (size_t)a->H * 4},
+                         {gr->ddt_bias, (size_t)a->H * D * 4}, {gr->d_initial_state, st_bytes}};
+    const Span ins[] = {{q, tok * D * 2}, {k, tok * D * 2}, {v, tok * D * 2}, {g, tok * D * 4},
+                        {beta, tok * 4}, {A_log, (size_t)a->H * 4}, {dt_bias, (size_t)a->H * D * 4},
+                        {initial_state, st_bytes}, {cu_seqlens, cu_seqlens ? ((size_t)a->N + 1) * 4 : 0},
+                        {d_out, tok * D * 2}};
+    const int n_out = sizeof(outs) / sizeof(outs[0]);
+    for (int i = 0; i < n_out; ++i) {
+        for (const Span& in : ins)
+            if (overlaps(outs[i].p, outs[i].n, in.p, in.n)) return KDA_ERR_INVALID_ARG;
+        for (int j = i + 1; j < n_out; ++j)
+            if (overlaps(outs[i].p, outs[i].n, outs[j].p, outs[j].n)) return KDA_ERR_INVALID_ARG;
+    }
+    // d_initial_state may alias d_final_state exactly, not partially
+    if (gr->d_initial_state && d_final && (const void*)gr->d_initial_state != (const void*)d_final &&
+        overlaps(gr->d_initial_state, st_bytes, d_final, st_bytes))
+        return KDA_ERR_INVALID_ARG;
+    for (int i = 0; i < n_out - 1; ++i)
+        if (overlaps(outs[i].p, outs[i].n, d_final, st_bytes)) return KDA_ERR_INVALID_ARG;
+    a->out = nullptr;
+    b->d_out = d_out;
+    b->d_final = d_final;
+    b->dq = gr->dq; b->dk = gr->dk; b->dv = gr->dv; b->dg = gr->dg; b->dbeta = gr->dbeta;
+    b->dA_log = gr->dA_log; b->ddt_bias = gr->ddt_bias; b->d_initial = gr->d_initial_state;
+    return device_ok();
+}
+
+// With no token to process: the parameter gradients are zero and d_initial = d_final.
+kda_status bwd_no_tokens(const StagedArgs& a, const kda::BwdArgs& b, cudaStream_t s) {
+    const size_t D = kda::kHeadDim;
+    if (cudaMemsetAsync(b.dA_log, 0, (size_t)a.H * 4, s) != cudaSuccess) return KDA_ERR_CUDA;
+    if (cudaMemsetAsync(b.ddt_bias, 0, (size_t)a.H * D * 4, s) != cudaSuccess) return KDA_ERR_CUDA;
+    if (!b.d_initial || a.N == 0) return KDA_OK;
+    const size_t bytes = (size_t)a.N * a.H * D * D * 4;
+    cudaError_t err = b.d_final
+        ? ((const void*)b.d_final == (const void*)b.d_initial ? cudaSuccess
+           : cudaMemcpyAsync(b.d_initial, b.d_final, bytes, cudaMemcpyDeviceToDevice, s))
+        : cudaMemsetAsync(b.d_initial, 0, bytes, s);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status decode_common(const void* q, const void* k, const void* v, const float* g, const float* beta,
                          const float* A_log, const float* dt_bias, float lower_bound, float scale,
                          float* state, void* out, int32_t batch, int32_t num_heads, kda_stream_t stream,
@@ -302,6 +370,43 @@ kda_status kda_gdn_decode(const void* q, const void* k, const void* v, const flo
                           float* state, void* out, int32_t batch, int32_t num_heads, kda_stream_t stream) {
     return decode_common(q, k, v, g, beta, A_log, dt_bias, lower_bound, scale, state, out, batch, num_heads,
                          stream, true);
+}
+
+size_t kda_bwd_workspace_size(kda_dims dims, int varlen) {
+    if (dims.num_heads < 1 || dims.seqlen < 0 || dims.batch < 0 || dims.num_seqs < 0) return 0;
+    int64_t N = dims.num_seqs, total = dims.seqlen;
+    if (!varlen) {
+        N = dims.batch;
+        total = (int64_t)dims.batch * dims.seqlen;
+    }
+    return kda::bwd_layout(total, dims.num_heads, (int)N).total;
+}
+
+kda_status kda_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                   const float* A_log, const float* dt_bias, float lower_bound, float scale,
+                   const float* initial_state, const int32_t* cu_seqlens, const void* d_out,
+                   const float* d_final_state, const kda_grads* grads, kda_dims dims, void* workspace,
+                   size_t workspace_bytes, kda_stream_t stream) {
+    StagedArgs a{};
+    kda::BwdArgs b{};
+    kda_status st = prepare_bwd(q, k, v, g, beta, A_log, dt_bias, lower_bound, scale, initial_state,
+                                cu_seqlens, d_out, d_final_state, grads, dims, &a, &b);
+    if (st != KDA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (a.total_tokens == 0) return bwd_no_tokens(a, b, s);
+    const kda::BwdLayout B = kda::bwd_layout(a.total_tokens, a.H, a.N);
+    if (workspace) {
+        if (workspace_bytes < B.total) return KDA_ERR_WORKSPACE;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_ALIGNMENT;
+        return kda::launch_bwd(a, b, static_cast<char*>(workspace), B, s) == cudaSuccess ? KDA_OK
+                                                                                       : KDA_ERR_CUDA;
+    }
+    if (workspace_bytes != 0) return KDA_ERR_WORKSPACE;
+    void* ws = nullptr;
+    if (cudaMallocAsync(&ws, B.total, s) != cudaSuccess) return KDA_ERR_CUDA;
+    cudaError_t err = kda::launch_bwd(a, b, static_cast<char*>(ws), B, s);
+    cudaError_t err2 = cudaFreeAsync(ws, s);
+    return (err == cudaSuccess && err2 == cudaSuccess) ? KDA_OK : KDA_ERR_CUDA;
 }
 
 const char* kda_strerror(kda_status status) {

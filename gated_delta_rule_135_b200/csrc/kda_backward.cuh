@@ -1,0 +1,643 @@
+// kda_backward.cuh -- the KDA backward: gradients of L = <dO, out> + <dS_final, final_state>
+// with respect to q, k, v, g, beta, A_log, dt_bias and the initial state.
+//
+// Staged, fp32 on CUDA cores, on top of the staged forward's workspace (Gamma, W, U~, P, U
+// and the state at every chunk start).  Per chunk (restated from the chain rule through
+// the forward's chunk algebra; the oracle's chunk_step_bwd follows the same steps):
+//   from S' = Diag(gC) S + Khat^T U:   dS = Diag(gC) dS',  dgC = rowsum(S * dS'),
+//                                      dKhat = U dS'^T,     dU = Khat dS'
+//   from O = scale((gamma q) S + P U):  d(gamma q) = scale dO S^T,  dS += scale (gamma q)^T dO,
+//                                      dP = scale dO U^T (i <= r),  dU += scale P^T dO
+//   from U = T Xu - W S, W = T Xw:     dW = -dU S^T, dS -= W^T dU, dT = dU Xu^T + dW Xw^T,
+//                                      dXu = T^T dU, dXw = T^T dW
+//   from T = (I + A)^-1:               dA = -T^T dT T^T (i < r)
+//   then the decay products (A_ri = beta_r sum_c k_rc k_ic e^{G_rc - G_ic}, P likewise with
+//   q_r), Xu = beta v, Xw = beta gamma k, Khat = k e^{G_last - G}, gamma = e^G; the chunk's
+//   dGamma summed from the end gives d log a, and the gate's derivative gives dg, dA_log and
+//   ddt_bias (zero where the lower-bound clamp is active).
+#pragma once
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+namespace bwd {
+
+constexpr int kPitch = kHeadDim + 1;
+constexpr int kPitchC = kChunk + 1;
+constexpr int kSlab = 32;
+
+__device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162float(x); }
+
+// global chunk id of sequence n's first chunk (one block; sums the earlier sequences)
+__device__ int64_t first_chunk_id(const int32_t* cu_seqlens, int n, int64_t seqlen, int64_t total_tokens) {
+    __shared__ int64_t warp_part[32];
+    __shared__ int64_t result;
+    int64_t part = 0;
+    for (int m = threadIdx.x; m < n; m += blockDim.x) {
+        int64_t mb, me;
+        seq_range(cu_seqlens, m, seqlen, total_tokens, &mb, &me);
+        part += (me - mb + kChunk - 1) / kChunk;
+    }
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if ((threadIdx.x & 31) == 0) warp_part[threadIdx.x >> 5] = part;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int64_t s = 0;
+        for (int x = 0; x < (int)(blockDim.x >> 5); ++x) s += warp_part[x];
+        result = s;
+    }
+    __syncthreads();
+    return result;
+}
+
+// ---------------------------------------------------------------------------
+// B1: dS backwards over a sequence's chunks; per chunk stores dS' (the gradient of the
+// state after it) and dU.  grid (N, H, 128 / kSlab), 256 threads.
+constexpr int kB1Threads = 256;
+constexpr size_t kB1Smem = sizeof(float) * (kHeadDim * (kSlab + 1) + 3 * kChunk * kPitch + kChunk * kPitchC +
+                                            2 * kChunk * (kSlab + 1) + kHeadDim);
+
+__global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const float* __restrict__ gamma,
+    const float* __restrict__ w, const float* __restrict__ p, const __nv_bfloat16* __restrict__ d_out,
+    const float* __restrict__ d_final, const int32_t* __restrict__ cu_seqlens, int64_t seqlen,
+    int64_t total_tokens, int H, float scale, int64_t max_chunks, float* __restrict__ dsn_out,
+    float* __restrict__ du_out, float* __restrict__ d_initial) {
+    const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kSlab, tid = threadIdx.x;
+    extern __shared__ float sm[];
+    float* sdS = sm;                                   // [128][33]
+    float* sKh = sdS + kHeadDim * (kSlab + 1);         // [64][129] Khat
+    float* sQt = sKh + kChunk * kPitch;                // [64][129] gamma * q
+    float* sW = sQt + kChunk * kPitch;                 // [64][129] W
+    float* sP = sW + kChunk * kPitch;                  // [64][65]  P
+    float* sdO = sP + kChunk * kPitchC;                // [64][33]
+    float* sdU = sdO + kChunk * (kSlab + 1);           // [64][33]
+    float* sgC = sdU + kChunk * (kSlab + 1);           // [128] Gamma_last
+    int64_t b, e;
+    seq_range(cu_seqlens, n, seqlen, total_tokens, &b, &e);
+    const int64_t c_first = first_chunk_id(cu_seqlens, n, seqlen, total_tokens);
+    for (int x = tid; x < kHeadDim * kSlab; x += kB1Threads) {
+        const int c = x / kSlab, j = x % kSlab;
+        sdS[c * (kSlab + 1) + j] = d_final ? d_final[(((int64_t)n * H + h) * kHeadDim + c) * kHeadDim + j0 + j] : 0.f;
+    }
+    __syncthreads();
+    const int64_t nch = (e - b + kChunk - 1) / kChunk;
+    for (int64_t jc = nch - 1; jc >= 0; --jc) {
+        const int64_t t0 = b + jc * kChunk, cid = c_first + jc;
+        const int len = (int)(e - t0 < kChunk ? e - t0 : kChunk);
+        if (cid >= max_chunks) {
+            if (tid == 0) record_error(KDA_DEVERR_BOUNDS);
+            break;
+        }
+        // dS' of this chunk
+        for (int x = tid; x < kHeadDim * kSlab; x += kB1Threads) {
+            const int c = x / kSlab, j = x % kSlab;
+            dsn_out[((cid * H + h) * kHeadDim + c) * kHeadDim + j0 + j] = sdS[c * (kSlab + 1) + j];
+        }
+        if (tid < kHeadDim) sgC[tid] = gamma[((t0 + len - 1) * H + h) * kHeadDim + tid];
+        __syncthreads();
+        for (int x = tid; x < kChunk * kHeadDim; x += kB1Threads) {
+            const int r = x / kHeadDim, c = x % kHeadDim;
+            float kh = 0.f, qt = 0.f, wv = 0.f;
+            if (r < len) {
+                const int64_t idx = ((t0 + r) * H + h) * kHeadDim + c;
+                const float G = gamma[idx];
+                kh = bf(k[idx]) * expf(sgC[c] - G);
+                qt = bf(q[idx]) * expf(G);
+                wv = w[idx];
+            }
+            sKh[r * kPitch + c] = kh;
+            sQt[r * kPitch + c] = qt;
+            sW[r * kPitch + c] = wv;
+        }
+        for (int x = tid; x < kChunk * kChunk; x += kB1Threads) {
+            const int r = x / kChunk, i = x % kChunk;
+            sP[r * kPitchC + i] = r < len ? p[((t0 + r) * H + h) * kChunk + i] : 0.f;
+        }
+        for (int x = tid; x < kChunk * kSlab; x += kB1Threads) {
+            const int r = x / kSlab, j = x % kSlab;
+            sdO[r * (kSlab + 1) + j] = r < len ? bf(d_out[((t0 + r) * H + h) * kHeadDim + j0 + j]) : 0.f;
+        }
+        __syncthreads();
+        // dU = scale P^T dO + Khat dS'
+        {
+            const int j = tid % kSlab;
+            for (int r = tid / kSlab; r < kChunk; r += kB1Threads / kSlab) {
+                float acc = 0.f;
+                if (r < len) {
+                    for (int i = r; i < len; ++i) acc = fmaf(sP[i * kPitchC + r], sdO[i * (kSlab + 1) + j], acc);
+                    acc *= scale;
+                    for (int c = 0; c < kHeadDim; ++c)
+                        acc = fmaf(sKh[r * kPitch + c], sdS[c * (kSlab + 1) + j], acc);
+                    du_out[((t0 + r) * H + h) * kHeadDim + j0 + j] = acc;
+                }
+                sdU[r * (kSlab + 1) + j] = acc;
+            }
+        }
+        __syncthreads();
+        // dS = Diag(gC) dS' + scale (gamma q)^T dO - W^T dU
+        {
+            const int j = tid % kSlab;
+            for (int c = tid / kSlab; c < kHeadDim; c += kB1Threads / kSlab) {
+                float a1 = 0.f, a2 = 0.f;
+                for (int r = 0; r < len; ++r) {
+                    a1 = fmaf(sQt[r * kPitch + c], sdO[r * (kSlab + 1) + j], a1);
+                    a2 = fmaf(sW[r * kPitch + c], sdU[r * (kSlab + 1) + j], a2);
+                }
+                sdS[c * (kSlab + 1) + j] = expf(sgC[c]) * sdS[c * (kSlab + 1) + j] + scale * a1 - a2;
+            }
+        }
+        __syncthreads();
+    }
+    if (d_initial) {
+        for (int x = tid; x < kHeadDim * kSlab; x += kB1Threads) {
+            const int c = x / kSlab, j = x % kSlab;
+            d_initial[(((int64_t)n * H + h) * kHeadDim + c) * kHeadDim + j0 + j] = sdS[c * (kSlab + 1) + j];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// B2: per chunk and 32-channel tile: dKhat = U dS'^T, d(gamma q) = scale dO S^T,
+// dW = -dU S^T (rows r, channels c of the tile) and dgC_c = sum_j S_cj dS'_cj.
+// grid (max_chunks, H, 128 / 32), 256 threads.
+constexpr int kB2Threads = 256;
+constexpr int kCT = 32;
+constexpr size_t kB2Smem = sizeof(float) * (2 * kCT * kPitch + 3 * kChunk * kPitch);
+
+__global__ void __launch_bounds__(kB2Threads) chunk_products_bwd_kernel(
+    const float* __restrict__ u, const float* __restrict__ du, const __nv_bfloat16* __restrict__ d_out,
+    const float* __restrict__ chunk_states, const float* __restrict__ dsn, const int4* __restrict__ table,
+    const int32_t* __restrict__ count, int H, float scale, float* __restrict__ dkhat, float* __restrict__ dqg,
+    float* __restrict__ dw, float* __restrict__ dgc) {
+    const int ci = blockIdx.x;
+    if (ci >= *count) return;
+    const int4 e = table[ci];
+    const int h = blockIdx.y, c0 = blockIdx.z * kCT, tid = threadIdx.x, len = e.z;
+    extern __shared__ float sm[];
+    float* sS = sm;                        // [32 c][129 j] S rows of the tile
+    float* sN = sS + kCT * kPitch;         // [32 c][129 j] dS' rows of the tile
+    float* sU = sN + kCT * kPitch;         // [64][129] U
+    float* sO = sU + kChunk * kPitch;      // [64][129] dO
+    float* sD = sO + kChunk * kPitch;      // [64][129] dU
+    const int64_t sbase = ((int64_t)ci * H + h) * kHeadDim * kHeadDim;
+    for (int x = tid; x < kCT * kHeadDim; x += kB2Threads) {
+        const int c = x / kHeadDim, j = x % kHeadDim;
+        sS[c * kPitch + j] = chunk_states[sbase + (int64_t)(c0 + c) * kHeadDim + j];
+        sN[c * kPitch + j] = dsn[sbase + (int64_t)(c0 + c) * kHeadDim + j];
+    }
+    for (int x = tid; x < kChunk * kHeadDim; x += kB2Threads) {
+        const int r = x / kHeadDim, j = x % kHeadDim;
+        float uv = 0.f, ov = 0.f, dv = 0.f;
+        if (r < len) {
+            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + j;
+            uv = u[idx];
+            ov = bf(d_out[idx]);
+            dv = du[idx];
+        }
+        sU[r * kPitch + j] = uv;
+        sO[r * kPitch + j] = ov;
+        sD[r * kPitch + j] = dv;
+    }
+    __syncthreads();
+    for (int x = tid; x < len * kCT; x += kB2Threads) {
+        const int r = x / kCT, c = x % kCT;
+        float a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        for (int j = 0; j < kHeadDim; ++j) {
+            a1 = fmaf(sU[r * kPitch + j], sN[c * kPitch + j], a1);
+            a2 = fmaf(sO[r * kPitch + j], sS[c * kPitch + j], a2);
+            a3 = fmaf(sD[r * kPitch + j], sS[c * kPitch + j], a3);
+        }
+        const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c0 + c;
+        dkhat[idx] = a1;
+        dqg[idx] = scale * a2;
+        dw[idx] = -a3;
+    }
+    if (tid < kCT) {
+        float a = 0.f;
+        for (int j = 0; j < kHeadDim; ++j) a = fmaf(sS[tid * kPitch + j], sN[tid * kPitch + j], a);
+        dgc[((int64_t)ci * H + h) * kHeadDim + c0 + tid] = a;
+    }
+}
+
+// Loads k, Gamma and beta of chunk `e` into smem (zero past the sequence end) and
+// forms A (beta-scaled, strictly lower) and T = (I + A)^-1 there; sA is scratch for A.
+__device__ void recompute_T(const __nv_bfloat16* __restrict__ k, const float* __restrict__ gamma,
+                            const float* __restrict__ beta, int4 e, int H, int h, float* sk, float* sG,
+                            float* sb, float* sA, float* sT, int nthreads) {
+    const int tid = threadIdx.x, len = e.z;
+    for (int x = tid; x < kChunk * kHeadDim; x += nthreads) {
+        const int r = x / kHeadDim, c = x % kHeadDim;
+        float kv = 0.f, gv = 0.f;
+        if (r < len) {
+            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c;
+            kv = bf(k[idx]);
+            gv = gamma[idx];
+        }
+        sk[r * kPitch + c] = kv;
+        sG[r * kPitch + c] = gv;
+    }
+    if (tid < kChunk) sb[tid] = tid < len ? beta[((int64_t)e.y + tid) * H + h] : 0.f;
+    for (int x = tid; x < kChunk * kPitchC; x += nthreads) { sA[x] = 0.f; sT[x] = 0.f; }
+    __syncthreads();
+    for (int x = tid; x < kChunk * kChunk; x += nthreads) {
+        const int r = x / kChunk, i = x % kChunk;
+        if (i >= r || r >= len) continue;
+        float acc = 0.f;
+        for (int c = 0; c < kHeadDim; ++c)
+            acc = fmaf(sk[r * kPitch + c] * sk[i * kPitch + c], expf(sG[r * kPitch + c] - sG[i * kPitch + c]), acc);
+        sA[r * kPitchC + i] = sb[r] * acc;
+    }
+    __syncthreads();
+    if (tid < kChunk) {
+        const int j = tid;
+        for (int r = j; r < kChunk; ++r) {
+            float s0 = (r == j) ? 1.f : 0.f;
+            for (int i = j; i < r; ++i) s0 = fmaf(-sA[r * kPitchC + i], sT[i * kPitchC + j], s0);
+            sT[r * kPitchC + j] = s0;
+        }
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// B3a: the T-side gradients of one chunk.  grid (max_chunks, H), 256 threads.
+//   dT = dU (beta v)^T + dW (beta gamma k)^T,  dXu = T^T dU -> dv, dbeta,
+//   dXw = T^T dW -> dk, dGamma, dbeta (partial sums, overwritten: first writer),
+//   dA = -T^T (dT T^T) (strictly lower) -> da_out [chunk][64][64].
+constexpr int kB3Threads = 256;
+constexpr size_t kB3aSmem = sizeof(float) * (4 * kChunk * kPitch + 3 * kChunk * kPitchC + 2 * kChunk);
+
+__global__ void __launch_bounds__(kB3Threads) t_side_bwd_kernel(
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, const float* __restrict__ beta,
+    const float* __restrict__ gamma, const float* __restrict__ du, const float* __restrict__ dw,
+    const int4* __restrict__ table, const int32_t* __restrict__ count, int H, float* __restrict__ dk_out,
+    float* __restrict__ dv_out, float* __restrict__ dG_out, float* __restrict__ dbeta_out,
+    float* __restrict__ da_out) {
+    const int ci = blockIdx.x;
+    if (ci >= *count) return;
+    const int4 e = table[ci];
+    const int h = blockIdx.y, tid = threadIdx.x, len = e.z;
+    extern __shared__ float sm[];
+    float* sk = sm;                          // [64][129]
+    float* sG = sk + kChunk * kPitch;        // [64][129]
+    float* s1 = sG + kChunk * kPitch;        // [64][129] dU, later dW
+    float* s2 = s1 + kChunk * kPitch;        // [64][129] v
+    float* sA = s2 + kChunk * kPitch;        // [64][65] A, later dT T^T
+    float* sT = sA + kChunk * kPitchC;       // [64][65]
+    float* sdT = sT + kChunk * kPitchC;      // [64][65] dT, later dA
+    float* sbt = sdT + kChunk * kPitchC;     // [64] dbeta of the value side
+    float* sb = sbt + kChunk;                // [64]
+    recompute_T(k, gamma, beta, e, H, h, sk, sG, sb, sA, sT, kB3Threads);
+    for (int x = tid; x < kChunk * kHeadDim; x += kB3Threads) {
+        const int r = x / kHeadDim, c = x % kHeadDim;
+        float a = 0.f, b2 = 0.f;
+        if (r < len) {
+            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c;
+            a = du[idx];
+            b2 = bf(v[idx]);
+        }
+        s1[r * kPitch + c] = a;
+        s2[r * kPitch + c] = b2;
+    }
+    __syncthreads();
+    // dT (value part) and dXu = T^T dU
+    for (int x = tid; x < kChunk * kChunk; x += kB3Threads) {
+        const int r = x / kChunk, i = x % kChunk;
+        float acc = 0.f;
+        for (int j = 0; j < kHeadDim; ++j) acc = fmaf(s1[r * kPitch + j], s2[i * kPitch + j], acc);
+        sdT[r * kPitchC + i] = sb[i] * acc;
+    }
+    __syncthreads();   // the dT loop reads v from s2, which the next loop overwrites
+    for (int x = tid; x < len * kHeadDim; x += kB3Threads) {
+        const int i = x / kHeadDim, j = x % kHeadDim;
+        float acc = 0.f;
+        for (int r = i; r < len; ++r) acc = fmaf(sT[r * kPitchC + i], s1[r * kPitch + j], acc);
+        const int64_t idx = (((int64_t)e.y + i) * H + h) * kHeadDim + j;
+        dv_out[idx] = sb[i] * acc;
+        s2[i * kPitch + j] *= acc;                 // dXu * v, summed into dbeta below
+    }
+    __syncthreads();
+    if (tid < kChunk) {
+        float a = 0.f;
+        for (int j = 0; j < kHeadDim; ++j) a += s2[tid * kPitch + j];
+        sbt[tid] = a;
+    }
+    __syncthreads();
+    for (int x = tid; x < kChunk * kHeadDim; x += kB3Threads) {
+        const int r = x / kHeadDim, c = x % kHeadDim;
+        s1[r * kPitch + c] = r < len ? dw[(((int64_t)e.y + r) * H + h) * kHeadDim + c] : 0.f;
+    }
+    // s2 <- Xw / beta = gamma * k
+    for (int x = tid; x < kChunk * kHeadDim; x += kB3Threads) {
+        const int r = x / kHeadDim, c = x % kHeadDim;
+        s2[r * kPitch + c] = expf(sG[r * kPitch + c]) * sk[r * kPitch + c];
+    }
+    __syncthreads();
+    // dT += dW (beta gamma k)^T
+    for (int x = tid; x < kChunk * kChunk; x += kB3Threads) {
+        const int r = x / kChunk, i = x % kChunk;
+        float acc = 0.f;
+        for (int c = 0; c < kHeadDim; ++c) acc = fmaf(s1[r * kPitch + c], s2[i * kPitch + c], acc);
+        sdT[r * kPitchC + i] += sb[i] * acc;
+    }
+    // dXw = T^T dW -> dk = dXw beta gamma, dGamma = dXw beta gamma k, dbeta += sum_c dXw gamma k
+    for (int x = tid; x < len * kHeadDim; x += kB3Threads) {
+        const int i = x / kHeadDim, c = x % kHeadDim;
+        float acc = 0.f;
+        for (int r = i; r < len; ++r) acc = fmaf(sT[r * kPitchC + i], s1[r * kPitch + c], acc);
+        const int64_t idx = (((int64_t)e.y + i) * H + h) * kHeadDim + c;
+        const float gk = s2[i * kPitch + c];
+        const float gam = expf(sG[i * kPitch + c]);
+        dk_out[idx] = acc * sb[i] * gam;
+        dG_out[idx] = acc * sb[i] * gk;
+        sG[i * kPitch + c] = acc * gk;             // Gamma is no longer needed: dbeta terms
+    }
+    __syncthreads();
+    if (tid < kChunk) {
+        float a = sbt[tid];
+        for (int c = 0; c < kHeadDim; ++c) a += sG[tid * kPitch + c];
+        if (tid < len) dbeta_out[((int64_t)e.y + tid) * H + h] = a;
+    }
+    // dA = -T^T (dT T^T), strictly lower
+    for (int x = tid; x < kChunk * kChunk; x += kB3Threads) {
+        const int r = x / kChunk, i = x % kChunk;
+        float acc = 0.f;
+        for (int m = 0; m <= i; ++m) acc = fmaf(sdT[r * kPitchC + m], sT[i * kPitchC + m], acc);
+        sA[r * kPitchC + i] = acc;                 // Y = dT T^T
+    }
+    __syncthreads();
+    for (int x = tid; x < kChunk * kChunk; x += kB3Threads) {
+        const int r = x / kChunk, i = x % kChunk;
+        float acc = 0.f;
+        if (i < r && r < len)
+            for (int m = r; m < kChunk; ++m) acc = fmaf(sT[m * kPitchC + r], sA[m * kPitchC + i], acc);
+        da_out[((int64_t)ci * H + h) * kChunk * kChunk + r * kChunk + i] = -acc;
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// B3b: the decay-side gradients of one chunk and the gate.  grid (max_chunks, H), 512 threads.
+// With dP = scale dO U^T (i <= r) and the B3a outputs, thread (t, c) forms
+//   RA = sum_{i<t} dA_ti k_ic D_tic,  RP = sum_{i<=t} dP_ti k_ic D_tic          (row terms)
+//   CA = sum_{r>t} beta_r dA_rt k_rc D_rtc,  CP = sum_{r>=t} dP_rt q_rc D_rtc  (column terms)
+// where D_ric = prod_{i<s<=r} a_sc is built one factor at a time (no exponentials, and it
+// underflows to 0 exactly when the decay does), then
+//   dq = d(gamma q) gamma + RP,  dk += beta RA + CA + CP + dKhat e^{G_last - G},
+//   dGamma = [T side] + d(gamma q) gamma q + beta k RA + q RP - k (CA + CP) - dKhat Khat,
+//   dbeta += sum_c k RA,
+// with sum_r dKhat Khat + dgC gamma_C added to the last row's dGamma.  d log a is dGamma
+// summed from the chunk's end; the gate's chain rule gives dg and per-chunk partial sums of
+// dA_log and ddt_bias (reduced by param_reduce_kernel).
+constexpr int kB3bThreads = 512;
+constexpr size_t kB3bSmem = sizeof(float) * (5 * kChunk * kPitch + 2 * kChunk * kPitchC + kChunk + kHeadDim +
+                                             kChunk * 4 + 4);
+
+__global__ void __launch_bounds__(kB3bThreads) decay_bwd_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const float* __restrict__ g,
+    const float* __restrict__ beta, const float* __restrict__ A_log, const float* __restrict__ dt_bias,
+    float lower_bound, float scale, const float* __restrict__ gamma, const float* __restrict__ u,
+    const __nv_bfloat16* __restrict__ d_out, const float* __restrict__ da, const float* __restrict__ dqg,
+    const float* __restrict__ dkhat, const float* __restrict__ dgc, const float* __restrict__ dG_t,
+    const int4* __restrict__ table, const int32_t* __restrict__ count, int H, float* __restrict__ dq_out,
+    float* __restrict__ dk_io, float* __restrict__ dg_out, float* __restrict__ dbeta_io,
+    float* __restrict__ dalog_part, float* __restrict__ ddt_part) {
+    const int ci = blockIdx.x;
+    if (ci >= *count) return;
+    const int4 e = table[ci];
+    const int h = blockIdx.y, tid = threadIdx.x, len = e.z;
+    extern __shared__ float sm[];
+    float* sX = sm;                          // [64][129] dO, then k
+    float* sY = sX + kChunk * kPitch;        // [64][129] U, then q
+    float* sa = sY + kChunk * kPitch;        // [64][129] a = e^{log a}
+    float* sT1 = sa + kChunk * kPitch;       // [64][129] dGamma without the dKhat Khat term
+    float* sT2 = sT1 + kChunk * kPitch;      // [64][129] dKhat Khat
+    float* sdP = sT2 + kChunk * kPitch;      // [64][65]
+    float* sdA = sdP + kChunk * kPitchC;     // [64][65]
+    float* sb = sdA + kChunk * kPitchC;      // [64]
+    float* sgC = sb + kChunk;                // [128] Gamma of the last row
+    float* sbp = sgC + kHeadDim;             // [64][4] dbeta partials (one per warp of a row)
+    float* sred = sbp + kChunk * 4;          // [4]
+    const float nexp = -expf(A_log[h]);
+    // phase 1: dP, dA, beta, a, Gamma_last
+    for (int x = tid; x < kChunk * kHeadDim; x += kB3bThreads) {
+        const int r = x / kHeadDim, c = x % kHeadDim;
+        float ov = 0.f, uv = 0.f, av = 0.f;
+        if (r < len) {
+            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c;
+            ov = bf(d_out[idx]);
+            uv = u[idx];
+            av = expf(gate_log_decay(g[idx] + dt_bias[h * kHeadDim + c], nexp, lower_bound));
+        }
+        sX[r * kPitch + c] = ov;
+        sY[r * kPitch + c] = uv;
+        sa[r * kPitch + c] = av;
+    }
+    for (int x = tid; x < kChunk * kChunk; x += kB3bThreads) {
+        const int r = x / kChunk, i = x % kChunk;
+        sdA[r * kPitchC + i] = da[((int64_t)ci * H + h) * kChunk * kChunk + x];
+    }
+    if (tid < kChunk) sb[tid] = tid < len ? beta[((int64_t)e.y + tid) * H + h] : 0.f;
+    if (tid < kHeadDim) sgC[tid] = gamma[(((int64_t)e.y + len - 1) * H + h) * kHeadDim + tid];
+    __syncthreads();
+    for (int x = tid; x < kChunk * kChunk; x += kB3bThreads) {
+        const int r = x / kChunk, i = x % kChunk;
+        float acc = 0.f;
+        if (i <= r && r < len) {
+            for (int j = 0; j < kHeadDim; ++j) acc = fmaf(sX[r * kPitch + j], sY[i * kPitch + j], acc);
+            acc *= scale;
+        }
+        sdP[r * kPitchC + i] = acc;
+    }
+    __syncthreads();
+    // phase 2: k and q
+    for (int x = tid; x < kChunk * kHeadDim; x += kB3bThreads) {
+        const int r = x / kHeadDim, c = x % kHeadDim;
+        float kv = 0.f, qv = 0.f;
+        if (r < len) {
+            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c;
+            kv = bf(k[idx]);
+            qv = bf(q[idx]);
+        }
+        sX[r * kPitch + c] = kv;
+        sY[r * kPitch + c] = qv;
+    }
+    __syncthreads();
+    const int c = tid % kHeadDim;
+    for (int t = tid / kHeadDim; t < len; t += kB3bThreads / kHeadDim) {
+        const float kt = sX[t * kPitch + c], qt = sY[t * kPitch + c];
+        float RA = 0.f, RP = sdP[t * kPitchC + t] * kt, D = 1.f;
+        for (int i = t - 1; i >= 0; --i) {
+            D *= sa[(i + 1) * kPitch + c];
+            const float kd = sX[i * kPitch + c] * D;
+            RA = fmaf(sdA[t * kPitchC + i], kd, RA);
+            RP = fmaf(sdP[t * kPitchC + i], kd, RP);
+        }
+        float CA = 0.f, CP = sdP[t * kPitchC + t] * qt;
+        D = 1.f;
+        for (int r = t + 1; r < len; ++r) {
+            D *= sa[r * kPitch + c];
+            CA = fmaf(sb[r] * sdA[r * kPitchC + t], sX[r * kPitch + c] * D, CA);
+            CP = fmaf(sdP[r * kPitchC + t], sY[r * kPitch + c] * D, CP);
+        }
+        const int64_t idx = (((int64_t)e.y + t) * H + h) * kHeadDim + c;
+        const float G = gamma[idx];
+        const float gam = expf(G), eK = expf(sgC[c] - G);
+        const float dQ = dqg[idx], dKh = dkhat[idx];
+        const float bt = sb[t];
+        dq_out[idx] = fmaf(dQ, gam, RP);
+        dk_io[idx] = dk_io[idx] + bt * RA + CA + CP + dKh * eK;
+        sT1[t * kPitch + c] = dG_t[idx] + dQ * gam * qt + bt * kt * RA + qt * RP - kt * (CA + CP);
+        sT2[t * kPitch + c] = dKh * kt * eK;
+        float pb = kt * RA;
+        for (int o = 16; o > 0; o >>= 1) pb += __shfl_xor_sync(0xffffffffu, pb, o);
+        if ((tid & 31) == 0) sbp[t * 4 + c / 32] = pb;
+    }
+    __syncthreads();
+    if (tid < kChunk && tid < len) {
+        const int64_t bi = ((int64_t)e.y + tid) * H + h;
+        dbeta_io[bi] = dbeta_io[bi] + ((sbp[tid * 4] + sbp[tid * 4 + 1]) + (sbp[tid * 4 + 2] + sbp[tid * 4 + 3]));
+    }
+    // gate: d log a_s = sum_{t >= s} dGamma_t (the dKhat Khat terms of rows t < s, which the last
+    // row's sum adds back, remain) + dgC gamma_C
+    if (tid < kHeadDim) {
+        float yall = 0.f;
+        for (int t = 0; t < len; ++t) yall += sT2[t * kPitch + c];
+        float R = yall + dgc[((int64_t)ci * H + h) * kHeadDim + c] * expf(sgC[c]);
+        const float db = dt_bias[h * kHeadDim + c];
+        float p_dt = 0.f, p_al = 0.f;
+        for (int s = len - 1; s >= 0; --s) {
+            R += sT1[s * kPitch + c] - sT2[s * kPitch + c];
+            const int64_t idx = (((int64_t)e.y + s) * H + h) * kHeadDim + c;
+            const float x = g[idx] + db;
+            const float raw = nexp * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))));
+            float dgv = 0.f;
+            if (raw >= lower_bound) {
+                dgv = R * nexp / (1.f + expf(-x));
+                p_al = fmaf(R, raw, p_al);
+            }
+            dg_out[idx] = dgv;
+            p_dt += dgv;
+        }
+        ddt_part[((int64_t)ci * H + h) * kHeadDim + c] = p_dt;
+        for (int o = 16; o > 0; o >>= 1) p_al += __shfl_xor_sync(0xffffffffu, p_al, o);
+        if ((tid & 31) == 0) sred[tid / 32] = p_al;
+    }
+    __syncthreads();
+    if (tid == 0) dalog_part[(int64_t)ci * H + h] = (sred[0] + sred[1]) + (sred[2] + sred[3]);
+}
+
+// dA_log[h] and ddt_bias[h][c]: the per-chunk partials summed in chunk order.  grid H, 128 threads.
+__global__ void __launch_bounds__(kHeadDim) param_reduce_kernel(
+    const float* __restrict__ dalog_part, const float* __restrict__ ddt_part, const int32_t* __restrict__ count,
+    int H, float* __restrict__ dA_log, float* __restrict__ ddt_bias) {
+    const int h = blockIdx.x, c = threadIdx.x, n = *count;
+    float s = 0.f, sa = 0.f;
+    for (int ci = 0; ci < n; ++ci) s += ddt_part[((int64_t)ci * H + h) * kHeadDim + c];
+    ddt_bias[h * kHeadDim + c] = s;
+    __shared__ float part[kHeadDim];
+    for (int ci = c; ci < n; ci += kHeadDim) sa += dalog_part[(int64_t)ci * H + h];
+    part[c] = sa;
+    __syncthreads();
+    if (c == 0) {
+        float t = 0.f;
+        for (int x = 0; x < kHeadDim; ++x) t += part[x];
+        dA_log[h] = t;
+    }
+}
+
+}  // namespace bwd
+
+// ---------------------------------------------------------------------------
+// host side
+
+BwdLayout bwd_layout(int64_t total_tokens, int H, int N) {
+    BwdLayout B{};
+    auto align = [](size_t x) { return (x + 255) & ~size_t(255); };
+    B.fwd = staged_layout(total_tokens, H, N);
+    const size_t tok = (size_t)total_tokens * (size_t)H, mc = (size_t)B.fwd.max_chunks;
+    size_t off = B.fwd.total;
+    B.dsn = off;       off = align(off + sizeof(float) * mc * H * kHeadDim * kHeadDim);
+    B.du = off;        off = align(off + sizeof(float) * tok * kHeadDim);
+    B.dkhat = off;     off = align(off + sizeof(float) * tok * kHeadDim);
+    B.dqg = off;       off = align(off + sizeof(float) * tok * kHeadDim);
+    B.dw = off;        off = align(off + sizeof(float) * tok * kHeadDim);
+    B.dG = off;        off = align(off + sizeof(float) * tok * kHeadDim);
+    B.da = off;        off = align(off + sizeof(float) * mc * H * kChunk * kChunk);
+    B.dgc = off;       off = align(off + sizeof(float) * mc * H * kHeadDim);
+    B.dalog_part = off; off = align(off + sizeof(float) * mc * H);
+    B.ddt_part = off;  off = align(off + sizeof(float) * mc * H * kHeadDim);
+    B.total = off;
+    return B;
+}
+
+cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const BwdLayout& B,
+                       cudaStream_t stream) {
+    static bool attrs_set = false;
+    if (!attrs_set) {
+        cudaError_t err;
+        if ((err = cudaFuncSetAttribute(bwd::state_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)bwd::kB1Smem)) != cudaSuccess) return err;
+        if ((err = cudaFuncSetAttribute(bwd::chunk_products_bwd_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd::kB2Smem)) !=
+            cudaSuccess) return err;
+        if ((err = cudaFuncSetAttribute(bwd::t_side_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)bwd::kB3aSmem)) != cudaSuccess) return err;
+        if ((err = cudaFuncSetAttribute(bwd::decay_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)bwd::kB3bSmem)) != cudaSuccess) return err;
+        attrs_set = true;
+    }
+    // the forward's intermediates (Gamma, W, P, U, chunk-start states); out is not needed
+    StagedArgs f = a;
+    f.out = nullptr;
+    f.final_state = nullptr;
+    cudaError_t err = launch_staged(f, ws, B.fwd, stream);
+    if (err != cudaSuccess) return err;
+    const StagedLayout& L = B.fwd;
+    const int4* table = reinterpret_cast<const int4*>(ws + L.chunk_table);
+    const int32_t* count = reinterpret_cast<const int32_t*>(ws + L.chunk_table + sizeof(int4) * L.max_chunks);
+    const float* gamma = reinterpret_cast<const float*>(ws + L.gamma);
+    const float* w = reinterpret_cast<const float*>(ws + L.w);
+    const float* p = reinterpret_cast<const float*>(ws + L.p);
+    const float* u = reinterpret_cast<const float*>(ws + L.u);
+    const float* cs = reinterpret_cast<const float*>(ws + L.chunk_states);
+    float* dsn = reinterpret_cast<float*>(ws + B.dsn);
+    float* du = reinterpret_cast<float*>(ws + B.du);
+    float* dkhat = reinterpret_cast<float*>(ws + B.dkhat);
+    float* dqg = reinterpret_cast<float*>(ws + B.dqg);
+    float* dw = reinterpret_cast<float*>(ws + B.dw);
+    float* dG = reinterpret_cast<float*>(ws + B.dG);
+    float* da = reinterpret_cast<float*>(ws + B.da);
+    float* dgc = reinterpret_cast<float*>(ws + B.dgc);
+    float* dalog_part = reinterpret_cast<float*>(ws + B.dalog_part);
+    float* ddt_part = reinterpret_cast<float*>(ws + B.ddt_part);
+    const auto* q = static_cast<const __nv_bfloat16*>(a.q);
+    const auto* k = static_cast<const __nv_bfloat16*>(a.k);
+    const auto* v = static_cast<const __nv_bfloat16*>(a.v);
+    const auto* dO = static_cast<const __nv_bfloat16*>(d.d_out);
+    const int H = a.H;
+    if (a.N > 0) {
+        dim3 g1((unsigned)a.N, (unsigned)H, kHeadDim / bwd::kSlab);
+        bwd::state_bwd_kernel<<<g1, bwd::kB1Threads, bwd::kB1Smem, stream>>>(
+            q, k, gamma, w, p, dO, d.d_final, a.cu_seqlens, a.seqlen, a.total_tokens, H, a.scale, L.max_chunks,
+            dsn, du, d.d_initial);
+    }
+    if (L.max_chunks > 0) {
+        dim3 g2((unsigned)L.max_chunks, (unsigned)H, kHeadDim / bwd::kCT);
+        bwd::chunk_products_bwd_kernel<<<g2, bwd::kB2Threads, bwd::kB2Smem, stream>>>(
+            u, du, dO, cs, dsn, table, count, H, a.scale, dkhat, dqg, dw, dgc);
+        dim3 g3((unsigned)L.max_chunks, (unsigned)H);
+        bwd::t_side_bwd_kernel<<<g3, bwd::kB3Threads, bwd::kB3aSmem, stream>>>(
+            k, v, a.beta, gamma, du, dw, table, count, H, d.dk, d.dv, dG, d.dbeta, da);
+        bwd::decay_bwd_kernel<<<g3, bwd::kB3bThreads, bwd::kB3bSmem, stream>>>(
+            q, k, a.g, a.beta, a.A_log, a.dt_bias, a.lower_bound, a.scale, gamma, u, dO, da, dqg, dkhat, dgc, dG,
+            table, count, H, d.dq, d.dk, d.dg, d.dbeta, dalog_part, ddt_part);
+    }
+    bwd::param_reduce_kernel<<<(unsigned)H, kHeadDim, 0, stream>>>(dalog_part, ddt_part, count, H, d.dA_log,
+                                                                   d.ddt_bias);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

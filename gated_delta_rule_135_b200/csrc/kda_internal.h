@@ -36,6 +36,30 @@ StagedLayout staged_layout(int64_t total_tokens, int H, int N);
 cudaError_t launch_staged(const StagedArgs& a, char* workspace, const StagedLayout& L,
                           cudaStream_t stream);
 
+// The backward: gradients of <dO, out> + <dS_final, final_state>.
+struct BwdArgs {
+    const void* d_out;       // bf16 [Ttot, H, 128]
+    const float* d_final;    // fp32 [N, H, 128, 128] or null (zero)
+    float* dq;               // fp32 [Ttot, H, 128]
+    float* dk;
+    float* dv;
+    float* dg;
+    float* dbeta;            // fp32 [Ttot, H]
+    float* dA_log;           // fp32 [H]
+    float* ddt_bias;         // fp32 [H, 128]
+    float* d_initial;        // fp32 [N, H, 128, 128] or null (not written)
+};
+
+// The staged forward's workspace followed by the backward's own buffers.
+struct BwdLayout {
+    StagedLayout fwd;
+    size_t dsn, du, dkhat, dqg, dw, dG, da, dgc, dalog_part, ddt_part, total;
+};
+
+BwdLayout bwd_layout(int64_t total_tokens, int H, int N);
+cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* workspace, const BwdLayout& B,
+                       cudaStream_t stream);
+
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* g, const float* beta,
                           const float* A_log, const float* dt_bias, float lower_bound, float scale,
                           float* state, void* out, int batch, int H, cudaStream_t stream,

@@ -446,7 +446,7 @@ cudaError_t launch_staged(const StagedArgs& a, char* ws, const StagedLayout& L, 
             k, gamma, w, ut, a.initial_state, a.cu_seqlens, a.seqlen, a.total_tokens, H, u, cs,
             L.max_chunks, a.final_state);
     }
-    if (L.max_chunks > 0) {
+    if (L.max_chunks > 0 && a.out) {   // the backward runs the forward for its intermediates only
         dim3 gc((unsigned)L.max_chunks, (unsigned)H);
         chunk_out_kernel<<<gc, kOutThreads, kOutSmem, stream>>>(
             q, gamma, cs, p, u, table, count, H, a.scale, static_cast<__nv_bfloat16*>(a.out));

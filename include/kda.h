@@ -242,6 +242,59 @@ kda_status kda_gdn_fwd(const void* q, const void* k, const void* v,
 kda_status kda_state_affine(const float* A, const float* S, const float* B, float* out,
                             int32_t num_heads, kda_stream_t stream);
 
+/*
+ * kda_bwd -- the backward of kda_fwd: gradients of the scalar
+ *   L = <d_out, out> + <d_final_state, final_state>
+ * with respect to every input of the forward.  The pages describe the forward only (the
+ * FlashKDA posts: donniechu.com, "Hạn chế & điều kiện" -- the release targets prefill); the
+ * backward is the chain rule taken through the same chunked form (WY / UT representation
+ * of each 64-token chunk and the chunk-to-chunk state recurrence), stage by stage:
+ *   (1) the staged forward into the workspace (Gamma, W, P, U, the state at every chunk start);
+ *   (2) dS backwards over each sequence's chunks, storing dS' per chunk and dU;
+ *   (3) per chunk: dKhat, d(gamma q), dW and d gamma_C from U, dU, dO, S, dS';
+ *   (4) per chunk: T = (I + A)^-1 recomputed; dT, dA, dv and the T-side dk, dGamma, dbeta;
+ *   (5) per chunk: dP and the pairwise decay terms (products of a, never exponentials of
+ *       differences), dq, dk, dbeta, then d log a (dGamma summed from the chunk's end) and
+ *       the gate's chain rule (zero where the lower_bound clamp is active);
+ *   (6) dA_log and ddt_bias summed over chunks in a fixed order (deterministic).
+ * fp32 CUDA-core arithmetic; no atomics, so results are bitwise reproducible.
+ *
+ * Inputs q ... cu_seqlens, lower_bound, scale, dims: exactly those of the kda_fwd call.
+ *   d_out          bf16 [Ttot, H, 128]       gradient of out
+ *   d_final_state  fp32 [N, H, 128, 128]     gradient of final_state; NULL means zero
+ * Outputs (device, caller-owned, written in full; none may overlap an input or another):
+ *   dq, dk, dv, dg fp32 [Ttot, H, 128]       dbeta fp32 [Ttot, H]
+ *   dA_log         fp32 [H]                  ddt_bias fp32 [H, 128]
+ *   d_initial_state fp32 [N, H, 128, 128]    NULL means "do not write"; may alias
+ *                                            d_final_state exactly (in place)
+ * workspace: at least kda_bwd_workspace_size(dims, varlen) bytes, 256-byte aligned; or
+ * NULL with workspace_bytes = 0, and the call allocates it stream-ordered
+ * (cudaMallocAsync / cudaFreeAsync).  Alignment as for kda_fwd: 16 bytes, except beta and
+ * dbeta (4 bytes).  Errors are reported before any launch.  Asynchronous on `stream`.
+ */
+typedef struct {
+    float* dq;
+    float* dk;
+    float* dv;
+    float* dg;
+    float* dbeta;
+    float* dA_log;
+    float* ddt_bias;
+    float* d_initial_state;
+} kda_grads;
+
+size_t kda_bwd_workspace_size(kda_dims dims, int varlen);
+
+kda_status kda_bwd(const void* q, const void* k, const void* v,
+                   const float* g, const float* beta,
+                   const float* A_log, const float* dt_bias,
+                   float lower_bound, float scale,
+                   const float* initial_state, const int32_t* cu_seqlens,
+                   const void* d_out, const float* d_final_state,
+                   const kda_grads* grads,
+                   kda_dims dims, void* workspace, size_t workspace_bytes,
+                   kda_stream_t stream);
+
 /* Human-readable name of a status code (static storage; never NULL). */
 const char* kda_strerror(kda_status status);
 

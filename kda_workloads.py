@@ -131,6 +131,16 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> dict:
                 seqlen=w.T if w.packed else w.seq_lens[0], N=w.N)
 
 
+def cotangents(w: Workload, seed: Optional[int] = None):
+    """Seeded gradients of the forward's outputs for the backward: d_out (bf16 [T, H, V],
+    standard normal) and d_final_state (fp32 [N, H, K, V], normal with std 0.1)."""
+    gen = torch.Generator("cpu")
+    gen.manual_seed(5000 + w.wid if seed is None else seed)
+    d_out = torch.randn(w.T, w.H, w.V, generator=gen).to(torch.bfloat16)
+    d_final = torch.randn(w.N, w.H, w.K, w.V, generator=gen) * 0.1
+    return d_out, d_final
+
+
 def gdn_inputs(x: dict) -> dict:
     """Inputs of the scalar-gate variant drawn from the same seeded tensors: the gate
     input and dt_bias of channel 0 (same distributions, one value per token-head / head)."""

@@ -163,3 +163,58 @@ def test_gdn_rejects_bad_arguments():
     p[3] += 2          # the scalar gate needs element (4-byte) alignment
     assert kda.lib().kda_gdn_fwd(*p, ctypes.c_float(-1.0), ctypes.c_float(0.1), None, None,
                                  FAKE + (7 << 28), None, _dims(), None) == 3
+
+
+def _bwd_call(dims=None, grads_override=None, drop=None, dfinal=None, ws=None, ws_bytes=0):
+    dims = dims or _dims()
+    p = [FAKE + i * (1 << 28) for i in range(8)]          # q k v g beta A_log dt_bias d_out
+    gp = [FAKE + (1 << 32) + i * (1 << 28) for i in range(8)]
+    fields = dict(zip(kda.GRAD_NAMES, gp))
+    fields.update(grads_override or {})
+    if drop:
+        fields[drop] = None
+    gr = kda.kda_grads(*[fields[n] for n in kda.GRAD_NAMES])
+    return kda.lib().kda_bwd(*p[:7], ctypes.c_float(-5.0), ctypes.c_float(0.1), None, None, p[7], dfinal,
+                             ctypes.byref(gr), dims, ws, ctypes.c_size_t(ws_bytes), None)
+
+
+def test_bwd_rejects_bad_arguments():
+    lib = kda.lib()
+    # no gradient block
+    assert lib.kda_bwd(*([FAKE] * 7), ctypes.c_float(-5.0), ctypes.c_float(0.1), None, None, FAKE, None,
+                       None, _dims(), None, ctypes.c_size_t(0), None) == 1
+    for name in ("dq", "dk", "dv", "dg", "dbeta", "dA_log", "ddt_bias"):
+        assert _bwd_call(drop=name) == 1, name
+    base = FAKE + (1 << 32)
+    assert _bwd_call(grads_override={"dq": base + 8}) == 3           # misaligned
+    assert _bwd_call(grads_override={"dbeta": base + 4 * (1 << 28) + 2}) == 3
+    assert _bwd_call(grads_override={"dq": FAKE}) == 1               # dq overlaps q
+    assert _bwd_call(grads_override={"dk": base + 4096}) == 1         # dk overlaps dq
+    assert _bwd_call(grads_override={"dA_log": FAKE + 7 * (1 << 28)}) == 1   # overlaps d_out
+    dfin = FAKE + (1 << 34)
+    assert _bwd_call(grads_override={"d_initial_state": dfin + 4096}, dfinal=dfin) == 1
+    assert _bwd_call(dims=_dims(hk=64)) == 2
+    assert _bwd_call(dims=_dims(H=0)) == 1
+
+
+def test_bwd_argument_checks_pass_before_the_device_check():
+    # valid arguments (beta-like dbeta at +4 bytes, d_initial aliasing d_final exactly, no
+    # d_initial at all) get past validation: with no GPU here the call then fails the device
+    # check (KDA_ERR_CUDA or KDA_ERR_UNSUPPORTED), never an argument error
+    base = FAKE + (1 << 32)
+    dfin = FAKE + (1 << 34)
+    for kw in (dict(), dict(grads_override={"dbeta": base + 4 * (1 << 28) + 4}),
+               dict(grads_override={"d_initial_state": dfin}, dfinal=dfin), dict(drop="d_initial_state")):
+        assert _bwd_call(**kw) in (2, 4), kw
+
+
+def test_bwd_workspace_extends_the_staged_layout():
+    for varlen, dims in ((0, _dims(H=3, T=1000)), (1, _dims(H=96, T=8192, nseq=6))):
+        T, H = dims.seqlen * (1 if varlen else dims.batch), dims.num_heads
+        N = dims.num_seqs if varlen else dims.batch
+        mc = math.ceil(T / 64) + N
+        extra = 4 * (mc * H * 128 * 128 + 5 * T * H * 128 + mc * H * 64 * 64 + mc * H * 128 + mc * H
+                     + mc * H * 128)
+        staged = kda.lib().kda_staged_workspace_size(dims, varlen)
+        assert kda.lib().kda_bwd_workspace_size(dims, varlen) >= staged + extra
+        assert kda.lib().kda_bwd_workspace_size(dims, varlen) <= staged + extra + 16 * 256
