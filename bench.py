@@ -56,6 +56,8 @@ def parse():
                     help="time kda_gdn_fwd, the scalar-gate variant, on the same workload")
     ap.add_argument("--decode", action="store_true",
                     help="time kda_decode (one token per sequence) instead of the prefill")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward kda_bwd (all gradients) instead of the forward")
     ap.add_argument("--decode-batch", type=int, default=256)
     ap.add_argument("--decode-heads", type=int, default=96)
     return ap.parse_args()
@@ -415,6 +417,134 @@ def run_decode(args, world, rank, kda):
     return 0
 
 
+BWD_BYTES_PER_TOKEN_HEAD = 3592   # reads q,k,v bf16 768, g 512, beta 4, d_out bf16 256; writes dq,dk,dv,dg fp32 2048, dbeta 4
+BWD_LAUNCHES_PER_STEP = 9         # staged forward 4 (no output kernel) + backward 5
+
+
+def run_backward(args, world, rank, kda):
+    """kda_bwd over the workload: every gradient (dq, dk, dv, dg, dbeta, dA_log, ddt_bias
+    and the initial-state gradient when the workload has states) per step."""
+    w = W.WORKLOADS[args.workload]
+    x = W.make_inputs(w)
+    dO, dF = W.cotangents(w)
+    if not w.final:
+        dF = None
+    dev = torch.device("cuda", torch.cuda.current_device())
+    xd = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    dOd = dO.to(dev)
+    dFd = dF.to(dev) if dF is not None else None
+    want_dinit = w.init is not None
+    grads = kda.kda_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"],
+                        x["lower_bound"], x["scale"], dOd, xd["initial_state"], xd["cu_seqlens"], dFd,
+                        want_d_initial=want_dinit, batch=x["batch"])
+    ws = torch.empty(kda.kda_bwd_workspace_size(xd["q"], xd["cu_seqlens"], x["batch"]), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kda.kda_bwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"],
+                    x["lower_bound"], x["scale"], dOd, xd["initial_state"], xd["cu_seqlens"], dFd,
+                    want_d_initial=want_dinit, grads=grads, workspace=ws, batch=x["batch"])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if kda.kda_check_device_error() != 0:
+        raise RuntimeError("device error recorded during warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        sampler.wait(ends[-1])
+    barrier(world)
+    step_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    total_ms = max_over_ranks(starts[0].elapsed_time(ends[-1]), world)
+    ms_per_step = total_ms / args.steps
+    value = w.T * world / (ms_per_step / 1e3) / 1e6
+    alg_bytes = BWD_BYTES_PER_TOKEN_HEAD * w.T * w.H + STATE_BYTES * w.N * w.H * (
+        (w.init is not None) + (dF is not None) + want_dinit)
+    peak, peak_kind = measured_hbm_peak()
+    achieved = alg_bytes / (step_ms / 1e3) / 1e9
+
+    e2e = None
+    if args.e2e_steps > 0:
+        keys = ("q", "k", "v", "g", "beta")
+        host = {k: x[k].pin_memory() for k in keys}
+        dO_h = dO.pin_memory()
+        outs = ("dq", "dk", "dv", "dg", "dbeta")
+        out_h = {n: torch.empty(grads[n].shape, dtype=grads[n].dtype).pin_memory() for n in outs}
+        h2d = sum(host[k].numel() * host[k].element_size() for k in keys) + dO_h.numel() * dO_h.element_size()
+        d2h = sum(t.numel() * t.element_size() for t in out_h.values())
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for k in keys:
+                xd[k].copy_(host[k], non_blocking=True)
+            dOd.copy_(dO_h, non_blocking=True)
+            step()
+            for n in outs:
+                out_h[n].copy_(grads[n], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.e2e_steps
+        e2e = {"value": w.T * world / (e_ms / 1e3) / 1e6, "unit": "Mtokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from threadpoolctl import threadpool_limits
+        from oracle import backward as OB
+        h = max(1, min(w.H, int(args.cpu_seconds / 4.0)))     # about 4 s of oracle per head at T = 8192
+        sub = {key: x[key][:, :h].contiguous() for key in ("q", "k", "v", "g", "beta")}
+        init = x["initial_state"][:, :h].contiguous() if x["initial_state"] is not None else None
+        dsub = dF[:, :h].contiguous() if dF is not None else None
+        cu = x["cu_seqlens"] if x["cu_seqlens"] is not None else \
+            torch.arange(x["batch"] + 1, dtype=torch.int32) * x["seqlen"]
+        with threadpool_limits(1):
+            t = time.perf_counter()
+            OB.grads_chunked(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"], x["A_log"][:h],
+                             x["dt_bias"][:h], x["lower_bound"], x["scale"], init, cu,
+                             dO[:, :h].contiguous(), dsub)
+            el = time.perf_counter() - t
+        cpu = {"value": (w.T * h / w.H) / el / 1e6, "unit": "Mtokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"chunked fp64 backward oracle over heads 0..{h - 1} of {w.H} ({w.T * h} token-heads) "
+                         f"in {el:.2f} s on one thread; scaled by {h}/{w.H}"}
+
+    if rank == 0:
+        line = {
+            "metric": "KDA backward throughput (Mtokens/s) at T=8192 H=96 D=128 varlen"
+            if args.workload == 2 else f"KDA backward throughput (Mtokens/s), {w.name}",
+            "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded kda_workloads, no dataset)",
+            "config": {"workload": "backward (all gradients) of " + w.describe(),
+                       "model": "KDA layer backward (no weights)",
+                       "global_batch": w.N * world, "seq_len": w.T, "heads": w.H,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "precision": "bf16 q/k/v/d_out, fp32 gates, states and gradients; fp32 CUDA cores",
+                       "l2": f"inputs and gradients exceed L2 ({alg_bytes / 1e6:.0f} MB per step); no flush"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)",
+                         "kernel": f"whole backward step ({BWD_LAUNCHES_PER_STEP} launches)",
+                         "kernel_ms": step_ms, "algorithmic_bytes": alg_bytes},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": BWD_LAUNCHES_PER_STEP * args.steps,
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     assert args.warmup >= 3, "at least 3 warm-up steps"
@@ -431,8 +561,8 @@ def main():
         build.build()
     barrier(world)
     import gated_delta_rule_135_b200 as kda
-    if args.decode:
-        rc = run_decode(args, world, rank, kda)
+    if args.decode or args.bwd:
+        rc = (run_decode if args.decode else run_backward)(args, world, rank, kda)
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()

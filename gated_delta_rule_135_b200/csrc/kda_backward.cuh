@@ -19,6 +19,7 @@
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "kda_tile.cuh"
 
 namespace kda {
 namespace bwd {
@@ -53,10 +54,12 @@ __device__ int64_t first_chunk_id(const int32_t* cu_seqlens, int n, int64_t seql
 
 // ---------------------------------------------------------------------------
 // B1: dS backwards over a sequence's chunks; per chunk stores dS' (the gradient of the
-// state after it) and dU.  grid (N, H, 128 / kSlab), 256 threads.
+// state after it) and dU.  grid (N, H, 128 / kSlab), 256 threads; each block owns a
+// 128 x kSlab column slab of dS.  Register tiles: dU 2 x 4 and dS 4 x 4 per thread.
 constexpr int kB1Threads = 256;
-constexpr size_t kB1Smem = sizeof(float) * (kHeadDim * (kSlab + 1) + 3 * kChunk * kPitch + kChunk * kPitchC +
-                                            2 * kChunk * (kSlab + 1) + kHeadDim);
+constexpr int kSP = kSlab + 1;
+constexpr size_t kB1Smem = sizeof(float) * (kHeadDim * kSP + 3 * kChunk * kPitch + kChunk * kPitchC +
+                                            2 * kChunk * kSP + 2 * kHeadDim);
 
 __global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const float* __restrict__ gamma,
@@ -67,21 +70,22 @@ __global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
     const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kSlab, tid = threadIdx.x;
     extern __shared__ float sm[];
     float* sdS = sm;                                   // [128][33]
-    float* sKh = sdS + kHeadDim * (kSlab + 1);         // [64][129] Khat
-    float* sQt = sKh + kChunk * kPitch;                // [64][129] gamma * q
-    float* sW = sQt + kChunk * kPitch;                 // [64][129] W
-    float* sP = sW + kChunk * kPitch;                  // [64][65]  P
+    float* sKh = sdS + kHeadDim * kSP;                 // [64][129] Khat
+    float* sQt = sKh + kChunk * kPitch;                // [64][129] scale * gamma * q
+    float* sW = sQt + kChunk * kPitch;                 // [64][129] -W
+    float* sP = sW + kChunk * kPitch;                  // [64][65]  scale * P
     float* sdO = sP + kChunk * kPitchC;                // [64][33]
-    float* sdU = sdO + kChunk * (kSlab + 1);           // [64][33]
-    float* sgC = sdU + kChunk * (kSlab + 1);           // [128] Gamma_last
+    float* sdU = sdO + kChunk * kSP;                   // [64][33]
+    float* sgC = sdU + kChunk * kSP;                   // [128] e^{Gamma_last}
+    float* sgL = sgC + kHeadDim;                       // [128] Gamma_last
     int64_t b, e;
     seq_range(cu_seqlens, n, seqlen, total_tokens, &b, &e);
     const int64_t c_first = first_chunk_id(cu_seqlens, n, seqlen, total_tokens);
     for (int x = tid; x < kHeadDim * kSlab; x += kB1Threads) {
         const int c = x / kSlab, j = x % kSlab;
-        sdS[c * (kSlab + 1) + j] = d_final ? d_final[(((int64_t)n * H + h) * kHeadDim + c) * kHeadDim + j0 + j] : 0.f;
+        sdS[c * kSP + j] = d_final ? d_final[(((int64_t)n * H + h) * kHeadDim + c) * kHeadDim + j0 + j] : 0.f;
     }
-    __syncthreads();
+    const int tx = tid % 8, ty = tid / 8;      // tile columns tx + 8 jj, rows ty + 32 ii
     const int64_t nch = (e - b + kChunk - 1) / kChunk;
     for (int64_t jc = nch - 1; jc >= 0; --jc) {
         const int64_t t0 = b + jc * kChunk, cid = c_first + jc;
@@ -90,70 +94,67 @@ __global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
             if (tid == 0) record_error(KDA_DEVERR_BOUNDS);
             break;
         }
+        __syncthreads();   // the previous chunk's dS is complete; its operands are consumed
         // dS' of this chunk
         for (int x = tid; x < kHeadDim * kSlab; x += kB1Threads) {
             const int c = x / kSlab, j = x % kSlab;
-            dsn_out[((cid * H + h) * kHeadDim + c) * kHeadDim + j0 + j] = sdS[c * (kSlab + 1) + j];
+            dsn_out[((cid * H + h) * kHeadDim + c) * kHeadDim + j0 + j] = sdS[c * kSP + j];
         }
-        if (tid < kHeadDim) sgC[tid] = gamma[((t0 + len - 1) * H + h) * kHeadDim + tid];
+        const float* gl = gamma + ((t0 + len - 1) * H + h) * kHeadDim;
+        if (tid < kHeadDim) sgL[tid] = gl[tid];
+        const int64_t base = (t0 * H + h) * kHeadDim, ld = (int64_t)H * kHeadDim;
+        stage<kChunk, kHeadDim, kB1Threads>(sW, kPitch, w + base, ld, len,
+                                            [](int, int, float x) { return -x; });
+        stage<kChunk, kChunk, kB1Threads>(sP, kPitchC, p + (t0 * H + h) * kChunk, (int64_t)H * kChunk, len,
+                                          [scale](int, int, float x) { return scale * x; });
+        stage<kChunk, kSlab, kB1Threads>(sdO, kSP, d_out + base + j0, ld, len, Identity{});
         __syncthreads();
-        for (int x = tid; x < kChunk * kHeadDim; x += kB1Threads) {
-            const int r = x / kHeadDim, c = x % kHeadDim;
-            float kh = 0.f, qt = 0.f, wv = 0.f;
-            if (r < len) {
-                const int64_t idx = ((t0 + r) * H + h) * kHeadDim + c;
-                const float G = gamma[idx];
-                kh = bf(k[idx]) * expf(sgC[c] - G);
-                qt = bf(q[idx]) * expf(G);
-                wv = w[idx];
-            }
-            sKh[r * kPitch + c] = kh;
-            sQt[r * kPitch + c] = qt;
-            sW[r * kPitch + c] = wv;
-        }
-        for (int x = tid; x < kChunk * kChunk; x += kB1Threads) {
-            const int r = x / kChunk, i = x % kChunk;
-            sP[r * kPitchC + i] = r < len ? p[((t0 + r) * H + h) * kChunk + i] : 0.f;
-        }
-        for (int x = tid; x < kChunk * kSlab; x += kB1Threads) {
-            const int r = x / kSlab, j = x % kSlab;
-            sdO[r * (kSlab + 1) + j] = r < len ? bf(d_out[((t0 + r) * H + h) * kHeadDim + j0 + j]) : 0.f;
-        }
+        stage2<kChunk, kHeadDim, kB1Threads>(sKh, kPitch, gamma + base, k + base, ld, len,
+                                             [sgL](int, int c, float G, float kv) { return kv * expf(sgL[c] - G); });
+        stage2<kChunk, kHeadDim, kB1Threads>(sQt, kPitch, gamma + base, q + base, ld, len,
+                                             [scale](int, int, float G, float qv) { return scale * qv * expf(G); });
+        if (tid < kHeadDim) sgC[tid] = expf(sgL[tid]);
         __syncthreads();
-        // dU = scale P^T dO + Khat dS'
+        // dU = scale P^T dO + Khat dS'   (rows >= len come out 0: P is lower triangular)
         {
-            const int j = tid % kSlab;
-            for (int r = tid / kSlab; r < kChunk; r += kB1Threads / kSlab) {
-                float acc = 0.f;
-                if (r < len) {
-                    for (int i = r; i < len; ++i) acc = fmaf(sP[i * kPitchC + r], sdO[i * (kSlab + 1) + j], acc);
-                    acc *= scale;
-                    for (int c = 0; c < kHeadDim; ++c)
-                        acc = fmaf(sKh[r * kPitch + c], sdS[c * (kSlab + 1) + j], acc);
-                    du_out[((t0 + r) * H + h) * kHeadDim + j0 + j] = acc;
+            float acc[2][4];
+            tile_zero(acc);
+            tile_fma<2, 4, 32, 8, 1, kPitchC, kSP, 1>(acc, sP, sdO, ty, tx, 0, len);
+            tile_fma<2, 4, 32, 8, kPitch, 1, kSP, 1>(acc, sKh, sdS, ty, tx, 0, kHeadDim);
+#pragma unroll
+            for (int ii = 0; ii < 2; ++ii) {
+                const int r = ty + 32 * ii;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = tx + 8 * jj;
+                    sdU[r * kSP + j] = acc[ii][jj];
+                    if (r < len) du_out[((t0 + r) * H + h) * kHeadDim + j0 + j] = acc[ii][jj];
                 }
-                sdU[r * (kSlab + 1) + j] = acc;
             }
         }
         __syncthreads();
         // dS = Diag(gC) dS' + scale (gamma q)^T dO - W^T dU
         {
-            const int j = tid % kSlab;
-            for (int c = tid / kSlab; c < kHeadDim; c += kB1Threads / kSlab) {
-                float a1 = 0.f, a2 = 0.f;
-                for (int r = 0; r < len; ++r) {
-                    a1 = fmaf(sQt[r * kPitch + c], sdO[r * (kSlab + 1) + j], a1);
-                    a2 = fmaf(sW[r * kPitch + c], sdU[r * (kSlab + 1) + j], a2);
+            float acc[4][4];
+            tile_zero(acc);
+            tile_fma<4, 4, 32, 8, 1, kPitch, kSP, 1>(acc, sQt, sdO, ty, tx, 0, len);
+            tile_fma<4, 4, 32, 8, 1, kPitch, kSP, 1>(acc, sW, sdU, ty, tx, 0, len);
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) {
+                const int c = ty + 32 * ii;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = tx + 8 * jj;
+                    sdS[c * kSP + j] = fmaf(sgC[c], sdS[c * kSP + j], acc[ii][jj]);
                 }
-                sdS[c * (kSlab + 1) + j] = expf(sgC[c]) * sdS[c * (kSlab + 1) + j] + scale * a1 - a2;
             }
         }
-        __syncthreads();
     }
+    __syncthreads();
     if (d_initial) {
         for (int x = tid; x < kHeadDim * kSlab; x += kB1Threads) {
             const int c = x / kSlab, j = x % kSlab;
-            d_initial[(((int64_t)n * H + h) * kHeadDim + c) * kHeadDim + j0 + j] = sdS[c * (kSlab + 1) + j];
+            d_initial[(((int64_t)n * H + h) * kHeadDim + c) * kHeadDim + j0 + j] = sdS[c * kSP + j];
         }
     }
 }
@@ -181,38 +182,58 @@ __global__ void __launch_bounds__(kB2Threads) chunk_products_bwd_kernel(
     float* sU = sN + kCT * kPitch;         // [64][129] U
     float* sO = sU + kChunk * kPitch;      // [64][129] dO
     float* sD = sO + kChunk * kPitch;      // [64][129] dU
-    const int64_t sbase = ((int64_t)ci * H + h) * kHeadDim * kHeadDim;
-    for (int x = tid; x < kCT * kHeadDim; x += kB2Threads) {
-        const int c = x / kHeadDim, j = x % kHeadDim;
-        sS[c * kPitch + j] = chunk_states[sbase + (int64_t)(c0 + c) * kHeadDim + j];
-        sN[c * kPitch + j] = dsn[sbase + (int64_t)(c0 + c) * kHeadDim + j];
-    }
-    for (int x = tid; x < kChunk * kHeadDim; x += kB2Threads) {
-        const int r = x / kHeadDim, j = x % kHeadDim;
-        float uv = 0.f, ov = 0.f, dv = 0.f;
-        if (r < len) {
-            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + j;
-            uv = u[idx];
-            ov = bf(d_out[idx]);
-            dv = du[idx];
-        }
-        sU[r * kPitch + j] = uv;
-        sO[r * kPitch + j] = ov;
-        sD[r * kPitch + j] = dv;
-    }
+    const int64_t sbase = ((int64_t)ci * H + h) * kHeadDim * kHeadDim + (int64_t)c0 * kHeadDim;
+    stage<kCT, kHeadDim, kB2Threads>(sS, kPitch, chunk_states + sbase, kHeadDim, kCT, Identity{});
+    stage<kCT, kHeadDim, kB2Threads>(sN, kPitch, dsn + sbase, kHeadDim, kCT, Identity{});
+    const int64_t base = ((int64_t)e.y * H + h) * kHeadDim, ld = (int64_t)H * kHeadDim;
+    stage<kChunk, kHeadDim, kB2Threads>(sU, kPitch, u + base, ld, len, Identity{});
+    stage<kChunk, kHeadDim, kB2Threads>(sO, kPitch, d_out + base, ld, len, Identity{});
+    stage<kChunk, kHeadDim, kB2Threads>(sD, kPitch, du + base, ld, len, Identity{});
     __syncthreads();
-    for (int x = tid; x < len * kCT; x += kB2Threads) {
-        const int r = x / kCT, c = x % kCT;
-        float a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    // 2 x 4 register tiles of the three products: rows ty + 32 ii, channels tx + 8 jj
+    {
+        const int tx = tid % 8, ty = tid / 8;
+        float a1[2][4], a2[2][4], a3[2][4];
+        tile_zero(a1);
+        tile_zero(a2);
+        tile_zero(a3);
+#pragma unroll 2
         for (int j = 0; j < kHeadDim; ++j) {
-            a1 = fmaf(sU[r * kPitch + j], sN[c * kPitch + j], a1);
-            a2 = fmaf(sO[r * kPitch + j], sS[c * kPitch + j], a2);
-            a3 = fmaf(sD[r * kPitch + j], sS[c * kPitch + j], a3);
+            float u0[2], o0[2], d0[2], nv[4], sv[4];
+#pragma unroll
+            for (int ii = 0; ii < 2; ++ii) {
+                const int r = ty + 32 * ii;
+                u0[ii] = sU[r * kPitch + j];
+                o0[ii] = sO[r * kPitch + j];
+                d0[ii] = sD[r * kPitch + j];
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int c = tx + 8 * jj;
+                nv[jj] = sN[c * kPitch + j];
+                sv[jj] = sS[c * kPitch + j];
+            }
+#pragma unroll
+            for (int ii = 0; ii < 2; ++ii)
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    a1[ii][jj] = fmaf(u0[ii], nv[jj], a1[ii][jj]);
+                    a2[ii][jj] = fmaf(o0[ii], sv[jj], a2[ii][jj]);
+                    a3[ii][jj] = fmaf(d0[ii], sv[jj], a3[ii][jj]);
+                }
         }
-        const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c0 + c;
-        dkhat[idx] = a1;
-        dqg[idx] = scale * a2;
-        dw[idx] = -a3;
+#pragma unroll
+        for (int ii = 0; ii < 2; ++ii) {
+            const int r = ty + 32 * ii;
+            if (r >= len) continue;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c0 + tx + 8 * jj;
+                dkhat[idx] = a1[ii][jj];
+                dqg[idx] = scale * a2[ii][jj];
+                dw[idx] = -a3[ii][jj];
+            }
+        }
     }
     if (tid < kCT) {
         float a = 0.f;
@@ -221,162 +242,114 @@ __global__ void __launch_bounds__(kB2Threads) chunk_products_bwd_kernel(
     }
 }
 
-// Loads k, Gamma and beta of chunk `e` into smem (zero past the sequence end) and
-// forms A (beta-scaled, strictly lower) and T = (I + A)^-1 there; sA is scratch for A.
-__device__ void recompute_T(const __nv_bfloat16* __restrict__ k, const float* __restrict__ gamma,
-                            const float* __restrict__ beta, int4 e, int H, int h, float* sk, float* sG,
-                            float* sb, float* sA, float* sT, int nthreads) {
-    const int tid = threadIdx.x, len = e.z;
-    for (int x = tid; x < kChunk * kHeadDim; x += nthreads) {
-        const int r = x / kHeadDim, c = x % kHeadDim;
-        float kv = 0.f, gv = 0.f;
-        if (r < len) {
-            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c;
-            kv = bf(k[idx]);
-            gv = gamma[idx];
-        }
-        sk[r * kPitch + c] = kv;
-        sG[r * kPitch + c] = gv;
-    }
-    if (tid < kChunk) sb[tid] = tid < len ? beta[((int64_t)e.y + tid) * H + h] : 0.f;
-    for (int x = tid; x < kChunk * kPitchC; x += nthreads) { sA[x] = 0.f; sT[x] = 0.f; }
-    __syncthreads();
-    for (int x = tid; x < kChunk * kChunk; x += nthreads) {
-        const int r = x / kChunk, i = x % kChunk;
-        if (i >= r || r >= len) continue;
-        float acc = 0.f;
-        for (int c = 0; c < kHeadDim; ++c)
-            acc = fmaf(sk[r * kPitch + c] * sk[i * kPitch + c], expf(sG[r * kPitch + c] - sG[i * kPitch + c]), acc);
-        sA[r * kPitchC + i] = sb[r] * acc;
-    }
-    __syncthreads();
-    if (tid < kChunk) {
-        const int j = tid;
-        for (int r = j; r < kChunk; ++r) {
-            float s0 = (r == j) ? 1.f : 0.f;
-            for (int i = j; i < r; ++i) s0 = fmaf(-sA[r * kPitchC + i], sT[i * kPitchC + j], s0);
-            sT[r * kPitchC + j] = s0;
-        }
-    }
-    __syncthreads();
-}
-
 // ---------------------------------------------------------------------------
 // B3a: the T-side gradients of one chunk.  grid (max_chunks, H), 256 threads.
-//   dT = dU (beta v)^T + dW (beta gamma k)^T,  dXu = T^T dU -> dv, dbeta,
-//   dXw = T^T dW -> dk, dGamma, dbeta (partial sums, overwritten: first writer),
-//   dA = -T^T (dT T^T) (strictly lower) -> da_out [chunk][64][64].
+// T = (I + A)^-1 comes from the forward (stored per chunk); with Xu = beta v, Xw = beta gamma k:
+//   dT = dU Xu^T + dW Xw^T,  dXu = T^T dU -> dv = beta dXu,  dXw = T^T dW -> dk = dXw beta gamma,
+//   dGamma = dXw beta gamma k,  dbeta = sum_j dXu v + sum_c dXw gamma k   (the T-side parts),
+//   dA = -T^T (dT T^T), strictly lower -> da_out [chunk][64][64].
 constexpr int kB3Threads = 256;
-constexpr size_t kB3aSmem = sizeof(float) * (4 * kChunk * kPitch + 3 * kChunk * kPitchC + 2 * kChunk);
+constexpr size_t kB3aSmem = sizeof(float) * (4 * kChunk * kPitch + 3 * kChunk * kPitchC + kChunk);
 
 __global__ void __launch_bounds__(kB3Threads) t_side_bwd_kernel(
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, const float* __restrict__ beta,
-    const float* __restrict__ gamma, const float* __restrict__ du, const float* __restrict__ dw,
-    const int4* __restrict__ table, const int32_t* __restrict__ count, int H, float* __restrict__ dk_out,
-    float* __restrict__ dv_out, float* __restrict__ dG_out, float* __restrict__ dbeta_out,
-    float* __restrict__ da_out) {
+    const float* __restrict__ gamma, const float* __restrict__ t_mat, const float* __restrict__ du,
+    const float* __restrict__ dw, const int4* __restrict__ table, const int32_t* __restrict__ count, int H,
+    float* __restrict__ dk_out, float* __restrict__ dv_out, float* __restrict__ dG_out,
+    float* __restrict__ dbeta_out, float* __restrict__ da_out) {
     const int ci = blockIdx.x;
     if (ci >= *count) return;
     const int4 e = table[ci];
     const int h = blockIdx.y, tid = threadIdx.x, len = e.z;
     extern __shared__ float sm[];
-    float* sk = sm;                          // [64][129]
-    float* sG = sk + kChunk * kPitch;        // [64][129]
-    float* s1 = sG + kChunk * kPitch;        // [64][129] dU, later dW
-    float* s2 = s1 + kChunk * kPitch;        // [64][129] v
-    float* sA = s2 + kChunk * kPitch;        // [64][65] A, later dT T^T
-    float* sT = sA + kChunk * kPitchC;       // [64][65]
-    float* sdT = sT + kChunk * kPitchC;      // [64][65] dT, later dA
-    float* sbt = sdT + kChunk * kPitchC;     // [64] dbeta of the value side
-    float* sb = sbt + kChunk;                // [64]
-    recompute_T(k, gamma, beta, e, H, h, sk, sG, sb, sA, sT, kB3Threads);
-    for (int x = tid; x < kChunk * kHeadDim; x += kB3Threads) {
-        const int r = x / kHeadDim, c = x % kHeadDim;
-        float a = 0.f, b2 = 0.f;
-        if (r < len) {
-            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c;
-            a = du[idx];
-            b2 = bf(v[idx]);
+    float* sXw = sm;                         // [64][129] beta gamma k
+    float* sXu = sXw + kChunk * kPitch;      // [64][129] beta v
+    float* sdU = sXu + kChunk * kPitch;      // [64][129]
+    float* sdW = sdU + kChunk * kPitch;      // [64][129]
+    float* sT = sdW + kChunk * kPitch;       // [64][65]
+    float* sdT = sT + kChunk * kPitchC;      // [64][65]
+    float* sY = sdT + kChunk * kPitchC;      // [64][65] dT T^T
+    float* sb = sY + kChunk * kPitchC;       // [64]
+    if (tid < kChunk) sb[tid] = tid < len ? beta[((int64_t)e.y + tid) * H + h] : 0.f;
+    stage<kChunk, kChunk, kB3Threads>(sT, kPitchC, t_mat + ((int64_t)ci * H + h) * kChunk * kChunk, kChunk, kChunk,
+                                      Identity{});
+    const int64_t base = ((int64_t)e.y * H + h) * kHeadDim, ld = (int64_t)H * kHeadDim;
+    stage<kChunk, kHeadDim, kB3Threads>(sdU, kPitch, du + base, ld, len, Identity{});
+    stage<kChunk, kHeadDim, kB3Threads>(sdW, kPitch, dw + base, ld, len, Identity{});
+    __syncthreads();
+    stage2<kChunk, kHeadDim, kB3Threads>(sXw, kPitch, gamma + base, k + base, ld, len,
+                                         [sb](int r, int, float G, float kv) { return sb[r] * expf(G) * kv; });
+    stage<kChunk, kHeadDim, kB3Threads>(sXu, kPitch, v + base, ld, len,
+                                        [sb](int r, int, float x) { return sb[r] * x; });
+    __syncthreads();
+    const int tx = tid % 16, ty = tid / 16;   // tiles: rows ty + 16 ii, columns tx + 16 jj
+    {   // dT = dU Xu^T + dW Xw^T
+        float acc[4][4];
+        tile_zero(acc);
+        tile_fma<4, 4, 16, 16, kPitch, 1, 1, kPitch>(acc, sdU, sXu, ty, tx, 0, kHeadDim);
+        tile_fma<4, 4, 16, 16, kPitch, 1, 1, kPitch>(acc, sdW, sXw, ty, tx, 0, kHeadDim);
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) sdT[(ty + 16 * ii) * kPitchC + tx + 16 * jj] = acc[ii][jj];
+    }
+    {   // dXu = T^T dU, dXw = T^T dW and their epilogues
+        float au[4][8], aw[4][8];
+        tile_zero(au);
+        tile_zero(aw);
+        tile_fma<4, 8, 16, 16, 1, kPitchC, kPitch, 1>(au, sT, sdU, ty, tx, 0, len);
+        tile_fma<4, 8, 16, 16, 1, kPitchC, kPitch, 1>(aw, sT, sdW, ty, tx, 0, len);
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) {
+            const int i = ty + 16 * ii;
+            float pb = 0.f;
+            if (i < len) {
+                const float bi = sb[i];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const int j = tx + 16 * jj;
+                    const int64_t idx = (((int64_t)e.y + i) * H + h) * kHeadDim + j;
+                    const float gam = expf(gamma[idx]), kk = bf(k[idx]);
+                    const float dkv = aw[ii][jj] * bi * gam;
+                    dv_out[idx] = bi * au[ii][jj];
+                    dk_out[idx] = dkv;
+                    dG_out[idx] = dkv * kk;
+                    pb = fmaf(au[ii][jj], bf(v[idx]), pb);
+                    pb = fmaf(aw[ii][jj], gam * kk, pb);
+                }
+            }
+            // the 16 lanes of a half-warp share row i
+            for (int o = 8; o > 0; o >>= 1) pb += __shfl_xor_sync(0xffffffffu, pb, o);
+            if (tx == 0 && i < len) dbeta_out[((int64_t)e.y + i) * H + h] = pb;
         }
-        s1[r * kPitch + c] = a;
-        s2[r * kPitch + c] = b2;
     }
     __syncthreads();
-    // dT (value part) and dXu = T^T dU
-    for (int x = tid; x < kChunk * kChunk; x += kB3Threads) {
-        const int r = x / kChunk, i = x % kChunk;
-        float acc = 0.f;
-        for (int j = 0; j < kHeadDim; ++j) acc = fmaf(s1[r * kPitch + j], s2[i * kPitch + j], acc);
-        sdT[r * kPitchC + i] = sb[i] * acc;
-    }
-    __syncthreads();   // the dT loop reads v from s2, which the next loop overwrites
-    for (int x = tid; x < len * kHeadDim; x += kB3Threads) {
-        const int i = x / kHeadDim, j = x % kHeadDim;
-        float acc = 0.f;
-        for (int r = i; r < len; ++r) acc = fmaf(sT[r * kPitchC + i], s1[r * kPitch + j], acc);
-        const int64_t idx = (((int64_t)e.y + i) * H + h) * kHeadDim + j;
-        dv_out[idx] = sb[i] * acc;
-        s2[i * kPitch + j] *= acc;                 // dXu * v, summed into dbeta below
+    {   // Y = dT T^T
+        float acc[4][4];
+        tile_zero(acc);
+        tile_fma<4, 4, 16, 16, kPitchC, 1, 1, kPitchC>(acc, sdT, sT, ty, tx, 0, kChunk);
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) sY[(ty + 16 * ii) * kPitchC + tx + 16 * jj] = acc[ii][jj];
     }
     __syncthreads();
-    if (tid < kChunk) {
-        float a = 0.f;
-        for (int j = 0; j < kHeadDim; ++j) a += s2[tid * kPitch + j];
-        sbt[tid] = a;
-    }
-    __syncthreads();
-    for (int x = tid; x < kChunk * kHeadDim; x += kB3Threads) {
-        const int r = x / kHeadDim, c = x % kHeadDim;
-        s1[r * kPitch + c] = r < len ? dw[(((int64_t)e.y + r) * H + h) * kHeadDim + c] : 0.f;
-    }
-    // s2 <- Xw / beta = gamma * k
-    for (int x = tid; x < kChunk * kHeadDim; x += kB3Threads) {
-        const int r = x / kHeadDim, c = x % kHeadDim;
-        s2[r * kPitch + c] = expf(sG[r * kPitch + c]) * sk[r * kPitch + c];
-    }
-    __syncthreads();
-    // dT += dW (beta gamma k)^T
-    for (int x = tid; x < kChunk * kChunk; x += kB3Threads) {
-        const int r = x / kChunk, i = x % kChunk;
-        float acc = 0.f;
-        for (int c = 0; c < kHeadDim; ++c) acc = fmaf(s1[r * kPitch + c], s2[i * kPitch + c], acc);
-        sdT[r * kPitchC + i] += sb[i] * acc;
-    }
-    // dXw = T^T dW -> dk = dXw beta gamma, dGamma = dXw beta gamma k, dbeta += sum_c dXw gamma k
-    for (int x = tid; x < len * kHeadDim; x += kB3Threads) {
-        const int i = x / kHeadDim, c = x % kHeadDim;
-        float acc = 0.f;
-        for (int r = i; r < len; ++r) acc = fmaf(sT[r * kPitchC + i], s1[r * kPitch + c], acc);
-        const int64_t idx = (((int64_t)e.y + i) * H + h) * kHeadDim + c;
-        const float gk = s2[i * kPitch + c];
-        const float gam = expf(sG[i * kPitch + c]);
-        dk_out[idx] = acc * sb[i] * gam;
-        dG_out[idx] = acc * sb[i] * gk;
-        sG[i * kPitch + c] = acc * gk;             // Gamma is no longer needed: dbeta terms
-    }
-    __syncthreads();
-    if (tid < kChunk) {
-        float a = sbt[tid];
-        for (int c = 0; c < kHeadDim; ++c) a += sG[tid * kPitch + c];
-        if (tid < len) dbeta_out[((int64_t)e.y + tid) * H + h] = a;
-    }
-    // dA = -T^T (dT T^T), strictly lower
-    for (int x = tid; x < kChunk * kChunk; x += kB3Threads) {
-        const int r = x / kChunk, i = x % kChunk;
-        float acc = 0.f;
-        for (int m = 0; m <= i; ++m) acc = fmaf(sdT[r * kPitchC + m], sT[i * kPitchC + m], acc);
-        sA[r * kPitchC + i] = acc;                 // Y = dT T^T
-    }
-    __syncthreads();
-    for (int x = tid; x < kChunk * kChunk; x += kB3Threads) {
-        const int r = x / kChunk, i = x % kChunk;
-        float acc = 0.f;
-        if (i < r && r < len)
-            for (int m = r; m < kChunk; ++m) acc = fmaf(sT[m * kPitchC + r], sA[m * kPitchC + i], acc);
-        da_out[((int64_t)ci * H + h) * kChunk * kChunk + r * kChunk + i] = -acc;
+    {   // dA = -T^T Y, strictly lower
+        float acc[4][4];
+        tile_zero(acc);
+        tile_fma<4, 4, 16, 16, 1, kPitchC, kPitchC, 1>(acc, sT, sY, ty, tx, 0, kChunk);
+        float* dst = da_out + ((int64_t)ci * H + h) * kChunk * kChunk;
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) {
+            const int r = ty + 16 * ii;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int i = tx + 16 * jj;
+                dst[r * kChunk + i] = (i < r && r < len) ? -acc[ii][jj] : 0.f;
+            }
+        }
     }
 }
-
 
 // ---------------------------------------------------------------------------
 // B3b: the decay-side gradients of one chunk and the gate.  grid (max_chunks, H), 512 threads.
@@ -392,7 +365,7 @@ __global__ void __launch_bounds__(kB3Threads) t_side_bwd_kernel(
 // summed from the chunk's end; the gate's chain rule gives dg and per-chunk partial sums of
 // dA_log and ddt_bias (reduced by param_reduce_kernel).
 constexpr int kB3bThreads = 512;
-constexpr size_t kB3bSmem = sizeof(float) * (5 * kChunk * kPitch + 2 * kChunk * kPitchC + kChunk + kHeadDim +
+constexpr size_t kB3bSmem = sizeof(float) * (5 * kChunk * kPitch + 2 * kChunk * kPitchC + kChunk + 2 * kHeadDim +
                                              kChunk * 4 + 4);
 
 __global__ void __launch_bounds__(kB3bThreads) decay_bwd_kernel(
@@ -420,53 +393,48 @@ __global__ void __launch_bounds__(kB3bThreads) decay_bwd_kernel(
     float* sgC = sb + kChunk;                // [128] Gamma of the last row
     float* sbp = sgC + kHeadDim;             // [64][4] dbeta partials (one per warp of a row)
     float* sred = sbp + kChunk * 4;          // [4]
+    float* sdb = sred + 4;                   // [128] dt_bias of the head
     const float nexp = -expf(A_log[h]);
     // phase 1: dP, dA, beta, a, Gamma_last
-    for (int x = tid; x < kChunk * kHeadDim; x += kB3bThreads) {
-        const int r = x / kHeadDim, c = x % kHeadDim;
-        float ov = 0.f, uv = 0.f, av = 0.f;
-        if (r < len) {
-            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c;
-            ov = bf(d_out[idx]);
-            uv = u[idx];
-            av = expf(gate_log_decay(g[idx] + dt_bias[h * kHeadDim + c], nexp, lower_bound));
-        }
-        sX[r * kPitch + c] = ov;
-        sY[r * kPitch + c] = uv;
-        sa[r * kPitch + c] = av;
-    }
-    for (int x = tid; x < kChunk * kChunk; x += kB3bThreads) {
-        const int r = x / kChunk, i = x % kChunk;
-        sdA[r * kPitchC + i] = da[((int64_t)ci * H + h) * kChunk * kChunk + x];
-    }
     if (tid < kChunk) sb[tid] = tid < len ? beta[((int64_t)e.y + tid) * H + h] : 0.f;
-    if (tid < kHeadDim) sgC[tid] = gamma[(((int64_t)e.y + len - 1) * H + h) * kHeadDim + tid];
+    if (tid < kHeadDim) {
+        sgC[tid] = gamma[(((int64_t)e.y + len - 1) * H + h) * kHeadDim + tid];
+        sdb[tid] = dt_bias[h * kHeadDim + tid];
+    }
+    const int64_t base = ((int64_t)e.y * H + h) * kHeadDim, ld = (int64_t)H * kHeadDim;
+    stage<kChunk, kHeadDim, kB3bThreads>(sX, kPitch, d_out + base, ld, len, Identity{});
+    stage<kChunk, kHeadDim, kB3bThreads>(sY, kPitch, u + base, ld, len, Identity{});
+    stage<kChunk, kChunk, kB3bThreads>(sdA, kPitchC, da + ((int64_t)ci * H + h) * kChunk * kChunk, kChunk, kChunk,
+                                       Identity{});
     __syncthreads();
-    for (int x = tid; x < kChunk * kChunk; x += kB3bThreads) {
-        const int r = x / kChunk, i = x % kChunk;
-        float acc = 0.f;
-        if (i <= r && r < len) {
-            for (int j = 0; j < kHeadDim; ++j) acc = fmaf(sX[r * kPitch + j], sY[i * kPitch + j], acc);
-            acc *= scale;
+    stage<kChunk, kHeadDim, kB3bThreads>(sa, kPitch, g + base, ld, len, [sdb, nexp, lower_bound](int, int c, float x) {
+        return expf(gate_log_decay(x + sdb[c], nexp, lower_bound));
+    });
+    {   // dP = scale dO U^T (i <= r < len): 2 x 4 tiles, rows ty + 32 ii, columns tx + 16 jj
+        const int tx = tid % 16, ty = tid / 16;
+        float acc[2][4];
+        tile_zero(acc);
+        tile_fma<2, 4, 32, 16, kPitch, 1, 1, kPitch>(acc, sX, sY, ty, tx, 0, kHeadDim);
+#pragma unroll
+        for (int ii = 0; ii < 2; ++ii) {
+            const int r = ty + 32 * ii;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int i = tx + 16 * jj;
+                sdP[r * kPitchC + i] = (i <= r && r < len) ? scale * acc[ii][jj] : 0.f;
+            }
         }
-        sdP[r * kPitchC + i] = acc;
     }
     __syncthreads();
     // phase 2: k and q
-    for (int x = tid; x < kChunk * kHeadDim; x += kB3bThreads) {
-        const int r = x / kHeadDim, c = x % kHeadDim;
-        float kv = 0.f, qv = 0.f;
-        if (r < len) {
-            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c;
-            kv = bf(k[idx]);
-            qv = bf(q[idx]);
-        }
-        sX[r * kPitch + c] = kv;
-        sY[r * kPitch + c] = qv;
-    }
+    stage<kChunk, kHeadDim, kB3bThreads>(sX, kPitch, k + base, ld, len, Identity{});
+    stage<kChunk, kHeadDim, kB3bThreads>(sY, kPitch, q + base, ld, len, Identity{});
     __syncthreads();
     const int c = tid % kHeadDim;
     for (int t = tid / kHeadDim; t < len; t += kB3bThreads / kHeadDim) {
+        const int64_t idx = (((int64_t)e.y + t) * H + h) * kHeadDim + c;
+        // issued before the pair loops so that their latency is hidden behind them
+        const float G = gamma[idx], dQ = dqg[idx], dKh = dkhat[idx], dkT = dk_io[idx], dGT = dG_t[idx];
         const float kt = sX[t * kPitch + c], qt = sY[t * kPitch + c];
         float RA = 0.f, RP = sdP[t * kPitchC + t] * kt, D = 1.f;
         for (int i = t - 1; i >= 0; --i) {
@@ -482,14 +450,11 @@ __global__ void __launch_bounds__(kB3bThreads) decay_bwd_kernel(
             CA = fmaf(sb[r] * sdA[r * kPitchC + t], sX[r * kPitch + c] * D, CA);
             CP = fmaf(sdP[r * kPitchC + t], sY[r * kPitch + c] * D, CP);
         }
-        const int64_t idx = (((int64_t)e.y + t) * H + h) * kHeadDim + c;
-        const float G = gamma[idx];
         const float gam = expf(G), eK = expf(sgC[c] - G);
-        const float dQ = dqg[idx], dKh = dkhat[idx];
         const float bt = sb[t];
         dq_out[idx] = fmaf(dQ, gam, RP);
-        dk_io[idx] = dk_io[idx] + bt * RA + CA + CP + dKh * eK;
-        sT1[t * kPitch + c] = dG_t[idx] + dQ * gam * qt + bt * kt * RA + qt * RP - kt * (CA + CP);
+        dk_io[idx] = dkT + bt * RA + CA + CP + dKh * eK;
+        sT1[t * kPitch + c] = dGT + dQ * gam * qt + bt * kt * RA + qt * RP - kt * (CA + CP);
         sT2[t * kPitch + c] = dKh * kt * eK;
         float pb = kt * RA;
         for (int o = 16; o > 0; o >>= 1) pb += __shfl_xor_sync(0xffffffffu, pb, o);
@@ -506,7 +471,7 @@ __global__ void __launch_bounds__(kB3bThreads) decay_bwd_kernel(
         float yall = 0.f;
         for (int t = 0; t < len; ++t) yall += sT2[t * kPitch + c];
         float R = yall + dgc[((int64_t)ci * H + h) * kHeadDim + c] * expf(sgC[c]);
-        const float db = dt_bias[h * kHeadDim + c];
+        const float db = sdb[c];
         float p_dt = 0.f, p_al = 0.f;
         for (int s = len - 1; s >= 0; --s) {
             R += sT1[s * kPitch + c] - sT2[s * kPitch + c];
@@ -559,6 +524,7 @@ BwdLayout bwd_layout(int64_t total_tokens, int H, int N) {
     B.fwd = staged_layout(total_tokens, H, N);
     const size_t tok = (size_t)total_tokens * (size_t)H, mc = (size_t)B.fwd.max_chunks;
     size_t off = B.fwd.total;
+    B.t_mat = off;     off = align(off + sizeof(float) * mc * H * kChunk * kChunk);
     B.dsn = off;       off = align(off + sizeof(float) * mc * H * kHeadDim * kHeadDim);
     B.du = off;        off = align(off + sizeof(float) * tok * kHeadDim);
     B.dkhat = off;     off = align(off + sizeof(float) * tok * kHeadDim);
@@ -593,6 +559,7 @@ cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const Bw
     StagedArgs f = a;
     f.out = nullptr;
     f.final_state = nullptr;
+    f.t_mat = reinterpret_cast<float*>(ws + B.t_mat);
     cudaError_t err = launch_staged(f, ws, B.fwd, stream);
     if (err != cudaSuccess) return err;
     const StagedLayout& L = B.fwd;
@@ -603,6 +570,7 @@ cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const Bw
     const float* p = reinterpret_cast<const float*>(ws + L.p);
     const float* u = reinterpret_cast<const float*>(ws + L.u);
     const float* cs = reinterpret_cast<const float*>(ws + L.chunk_states);
+    const float* tm = reinterpret_cast<const float*>(ws + B.t_mat);
     float* dsn = reinterpret_cast<float*>(ws + B.dsn);
     float* du = reinterpret_cast<float*>(ws + B.du);
     float* dkhat = reinterpret_cast<float*>(ws + B.dkhat);
@@ -630,7 +598,7 @@ cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const Bw
             u, du, dO, cs, dsn, table, count, H, a.scale, dkhat, dqg, dw, dgc);
         dim3 g3((unsigned)L.max_chunks, (unsigned)H);
         bwd::t_side_bwd_kernel<<<g3, bwd::kB3Threads, bwd::kB3aSmem, stream>>>(
-            k, v, a.beta, gamma, du, dw, table, count, H, d.dk, d.dv, dG, d.dbeta, da);
+            k, v, a.beta, gamma, tm, du, dw, table, count, H, d.dk, d.dv, dG, d.dbeta, da);
         bwd::decay_bwd_kernel<<<g3, bwd::kB3bThreads, bwd::kB3bSmem, stream>>>(
             q, k, a.g, a.beta, a.A_log, a.dt_bias, a.lower_bound, a.scale, gamma, u, dO, da, dqg, dkhat, dgc, dG,
             table, count, H, d.dq, d.dk, d.dg, d.dbeta, dalog_part, ddt_part);

@@ -25,6 +25,7 @@ struct StagedArgs {
     int64_t total_tokens;  // Ttot
     int H;
     int N;                 // number of sequences
+    float* t_mat;          // optional: T = (I + A)^-1 of every chunk, [max_chunks][H][64][64]
 };
 
 struct StagedLayout {
@@ -53,7 +54,7 @@ struct BwdArgs {
 // The staged forward's workspace followed by the backward's own buffers.
 struct BwdLayout {
     StagedLayout fwd;
-    size_t dsn, du, dkhat, dqg, dw, dG, da, dgc, dalog_part, ddt_part, total;
+    size_t t_mat, dsn, du, dkhat, dqg, dw, dG, da, dgc, dalog_part, ddt_part, total;
 };
 
 BwdLayout bwd_layout(int64_t total_tokens, int H, int N);

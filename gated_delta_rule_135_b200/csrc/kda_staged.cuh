@@ -16,6 +16,7 @@
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "kda_tile.cuh"
 
 namespace kda {
 
@@ -109,7 +110,8 @@ __global__ void __launch_bounds__(kIntraThreads) intra_chunk_kernel(
     const __nv_bfloat16* __restrict__ v, const float* __restrict__ beta,
     const float* __restrict__ gamma, const int4* __restrict__ table,
     const int32_t* __restrict__ count, int H,
-    float* __restrict__ w_out, float* __restrict__ ut_out, float* __restrict__ p_out) {
+    float* __restrict__ w_out, float* __restrict__ ut_out, float* __restrict__ p_out,
+    float* __restrict__ t_out) {
     const int ci = blockIdx.x;
     if (ci >= *count) return;
     const int4 e = table[ci];
@@ -124,46 +126,52 @@ __global__ void __launch_bounds__(kIntraThreads) intra_chunk_kernel(
     float* sT = sP + kChunk * kPitchC;       // [64][65]
     float* sb = sT + kChunk * kPitchC;       // [64] beta
 
-    for (int x = tid; x < kChunk * kHeadDim; x += kIntraThreads) {
-        const int r = x / kHeadDim, c = x % kHeadDim;
-        float kv = 0.f, qv = 0.f, gv = 0.f;
-        if (r < len) {
-            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c;
-            kv = bf16_to_f32(k[idx]);
-            qv = bf16_to_f32(q[idx]);
-            gv = gamma[idx];
-        }
-        sk[r * kPitch + c] = kv;
-        sq[r * kPitch + c] = qv;
-        sG[r * kPitch + c] = gv;
-    }
+    const int64_t base = ((int64_t)e.y * H + h) * kHeadDim, ld = (int64_t)H * kHeadDim;
+    stage<kChunk, kHeadDim, kIntraThreads>(sk, kPitch, k + base, ld, len, Identity{});
+    stage<kChunk, kHeadDim, kIntraThreads>(sq, kPitch, q + base, ld, len, Identity{});
+    stage<kChunk, kHeadDim, kIntraThreads>(sG, kPitch, gamma + base, ld, len, Identity{});
     for (int x = tid; x < kChunk * kPitchC; x += kIntraThreads) { sA[x] = 0.f; sP[x] = 0.f; sT[x] = 0.f; }
     if (tid < kChunk) sb[tid] = tid < len ? beta[((int64_t)e.y + tid) * H + h] : 0.f;
     __syncthreads();
 
-    // lower-triangle pairs (r, i), i <= r, enumerated row-major
-    constexpr int kPairs = kChunk * (kChunk + 1) / 2;
-    for (int p = tid; p < kPairs; p += kIntraThreads) {
-        int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
-        while (r * (r + 1) / 2 > p) --r;
-        while ((r + 1) * (r + 2) / 2 <= p) ++r;
-        const int i = p - r * (r + 1) / 2;
-        if (r >= len) continue;
-        const float* kr = sk + r * kPitch;
-        const float* ki = sk + i * kPitch;
-        const float* qr = sq + r * kPitch;
-        const float* Gr = sG + r * kPitch;
-        const float* Gi = sG + i * kPitch;
-        float acc_a = 0.f, acc_p = 0.f;
+    // A and P on 2 x 2 tiles of (r, i) pairs, tiles (tr, ti) with ti <= tr enumerated row-major:
+    // rows 2 tr + {0, 1}, columns 2 ti + {0, 1}; every decay formed pair by pair
+    constexpr int kTiles = (kChunk / 2) * (kChunk / 2 + 1) / 2;
+    for (int p = tid; p < kTiles; p += kIntraThreads) {
+        int tr = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
+        while (tr * (tr + 1) / 2 > p) --tr;
+        while ((tr + 1) * (tr + 2) / 2 <= p) ++tr;
+        const int ti = p - tr * (tr + 1) / 2;
+        const int r0 = 2 * tr, i0 = 2 * ti;
+        if (r0 >= len) continue;
+        float aa[2][2] = {}, ap[2][2] = {};
         for (int cc = 0; cc < kHeadDim; ++cc) {
             const int c = (cc + tid) & (kHeadDim - 1);
-            const float dec = expf(Gr[c] - Gi[c]);   // <= 1: Gamma is non-increasing in r
-            const float kd = ki[c] * dec;
-            acc_a = fmaf(kr[c], kd, acc_a);
-            acc_p = fmaf(qr[c], kd, acc_p);
+            const float kr[2] = {sk[r0 * kPitch + c], sk[(r0 + 1) * kPitch + c]};
+            const float qr[2] = {sq[r0 * kPitch + c], sq[(r0 + 1) * kPitch + c]};
+            const float Gr[2] = {sG[r0 * kPitch + c], sG[(r0 + 1) * kPitch + c]};
+            const float ki[2] = {sk[i0 * kPitch + c], sk[(i0 + 1) * kPitch + c]};
+            const float Gi[2] = {sG[i0 * kPitch + c], sG[(i0 + 1) * kPitch + c]};
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int b2 = 0; b2 < 2; ++b2) {
+                    // e^{Gamma_r - Gamma_i} <= 1 for i <= r (Gamma is non-increasing); the pairs
+                    // above the diagonal of a diagonal tile are discarded below
+                    const float kd = ki[b2] * expf(fminf(Gr[a] - Gi[b2], 0.f));
+                    aa[a][b2] = fmaf(kr[a], kd, aa[a][b2]);
+                    ap[a][b2] = fmaf(qr[a], kd, ap[a][b2]);
+                }
         }
-        if (i < r) sA[r * kPitchC + i] = sb[r] * acc_a;
-        sP[r * kPitchC + i] = acc_p;
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int b2 = 0; b2 < 2; ++b2) {
+                const int r = r0 + a, i = i0 + b2;
+                if (r >= len || i > r) continue;
+                if (i < r) sA[r * kPitchC + i] = sb[r] * aa[a][b2];
+                sP[r * kPitchC + i] = ap[a][b2];
+            }
     }
     __syncthreads();
 
@@ -183,31 +191,35 @@ __global__ void __launch_bounds__(kIntraThreads) intra_chunk_kernel(
         sq[r * kPitch + c] = sb[r] * expf(sG[r * kPitch + c]) * sk[r * kPitch + c];
     }
     __syncthreads();
-    for (int x = tid; x < kChunk * kHeadDim; x += kIntraThreads) {
-        const int r = x / kHeadDim, c = x % kHeadDim;
-        float vv = 0.f;
-        if (r < len) vv = bf16_to_f32(v[(((int64_t)e.y + r) * H + h) * kHeadDim + c]);
-        sG[r * kPitch + c] = sb[r] * vv;
-    }
+    stage<kChunk, kHeadDim, kIntraThreads>(sG, kPitch, v + base, ld, len, [sb](int r, int, float x) { return sb[r] * x; });
     __syncthreads();
-    // W = T (beta gamma K), U~ = T (beta V): column c = tid % 128, rows tid/128 + 2m
+    // W = T (beta gamma K), U~ = T (beta V): 4 x 8 register tiles, rows ty + 16 ii, columns tx + 16 jj
     {
-        const int c = tid % kHeadDim;
-        for (int r = tid / kHeadDim; r < len; r += kIntraThreads / kHeadDim) {
-            float aw = 0.f, au = 0.f;
-            for (int i = 0; i <= r; ++i) {
-                const float t = sT[r * kPitchC + i];
-                aw = fmaf(t, sq[i * kPitch + c], aw);
-                au = fmaf(t, sG[i * kPitch + c], au);
+        const int tx = tid % 16, ty = tid / 16;
+        float aw[4][8], au[4][8];
+        tile_zero(aw);
+        tile_zero(au);
+        tile_fma<4, 8, 16, 16, kPitchC, 1, kPitch, 1>(aw, sT, sq, ty, tx, 0, len);
+        tile_fma<4, 8, 16, 16, kPitchC, 1, kPitch, 1>(au, sT, sG, ty, tx, 0, len);
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) {
+            const int r = ty + 16 * ii;
+            if (r >= len) continue;
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                const int64_t idx = base + (int64_t)r * ld + tx + 16 * jj;
+                w_out[idx] = aw[ii][jj];
+                ut_out[idx] = au[ii][jj];
             }
-            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c;
-            w_out[idx] = aw;
-            ut_out[idx] = au;
         }
     }
     for (int x = tid; x < len * kChunk; x += kIntraThreads) {
         const int r = x / kChunk, i = x % kChunk;
         p_out[(((int64_t)e.y + r) * H + h) * kChunk + i] = sP[r * kPitchC + i];
+    }
+    if (t_out) {   // kept for the backward
+        float* dst = t_out + ((int64_t)ci * H + h) * kChunk * kChunk;
+        for (int x = tid; x < kChunk * kChunk; x += kIntraThreads) dst[x] = sT[(x / kChunk) * kPitchC + x % kChunk];
     }
 }
 
@@ -217,7 +229,7 @@ __global__ void __launch_bounds__(kIntraThreads) intra_chunk_kernel(
 constexpr int kSlab = 32;
 constexpr int kStateThreads = 256;
 constexpr size_t kStateSmem =
-    sizeof(float) * (kHeadDim * (kSlab + 1) + 2 * kChunk * kPitch + kChunk * (kSlab + 1) + kHeadDim);
+    sizeof(float) * (kHeadDim * (kSlab + 1) + 2 * kChunk * kPitch + kChunk * (kSlab + 1) + 2 * kHeadDim);
 
 __global__ void __launch_bounds__(kStateThreads) state_prop_kernel(
     const __nv_bfloat16* __restrict__ k, const float* __restrict__ gamma,
@@ -233,7 +245,8 @@ __global__ void __launch_bounds__(kStateThreads) state_prop_kernel(
     float* sW = sS + kHeadDim * (kSlab + 1);         // [64][129] W, later Khat
     float* sK = sW + kChunk * kPitch;                // [64][129] k -> Khat
     float* sU = sK + kChunk * kPitch;                // [64][33]
-    float* sgC = sU + kChunk * (kSlab + 1);          // [128] gamma_last
+    float* sgC = sU + kChunk * (kSlab + 1);          // [128] e^{Gamma_last}
+    float* sgL = sgC + kHeadDim;                     // [128] Gamma_last
     __shared__ int64_t s_first_chunk;
 
     int64_t b, e;
@@ -264,28 +277,10 @@ __global__ void __launch_bounds__(kStateThreads) state_prop_kernel(
     }
     __syncthreads();
     int64_t chunk_id = s_first_chunk;
+    const int tx = tid % 8, ty = tid / 8;   // register tiles: columns tx + 8 jj, rows ty + 32 ii
     for (int64_t t0 = b; t0 < e; t0 += kChunk, ++chunk_id) {
         const int len = (int)(e - t0 < kChunk ? e - t0 : kChunk);
-        // stage W and k/Gamma of the chunk
-        for (int x = tid; x < kChunk * kHeadDim; x += kStateThreads) {
-            const int r = x / kHeadDim, c = x % kHeadDim;
-            float wv = 0.f, kv = 0.f;
-            if (r < len) {
-                const int64_t idx = ((t0 + r) * H + h) * kHeadDim + c;
-                wv = w[idx];
-                kv = bf16_to_f32(k[idx]);
-            }
-            sW[r * kPitch + c] = wv;
-            sK[r * kPitch + c] = kv;
-        }
-        if (tid < kHeadDim) sgC[tid] = gamma[((t0 + len - 1) * H + h) * kHeadDim + tid];
-        __syncthreads();
-        // Khat_ic = k_ic e^{Gamma_last,c - Gamma_ic}
-        for (int x = tid; x < len * kHeadDim; x += kStateThreads) {
-            const int r = x / kHeadDim, c = x % kHeadDim;
-            const float G = gamma[((t0 + r) * H + h) * kHeadDim + c];
-            sK[r * kPitch + c] *= expf(sgC[c] - G);
-        }
+        __syncthreads();   // the previous chunk's state update is complete
         // record the chunk's starting state
         if (chunk_id < max_chunks) {
             for (int x = tid; x < kHeadDim * kSlab; x += kStateThreads) {
@@ -296,34 +291,52 @@ __global__ void __launch_bounds__(kStateThreads) state_prop_kernel(
         } else if (tid == 0) {
             record_error(KDA_DEVERR_BOUNDS);
         }
+        if (tid < kHeadDim) sgL[tid] = gamma[((t0 + len - 1) * H + h) * kHeadDim + tid];
+        const int64_t base = (t0 * H + h) * kHeadDim, ld = (int64_t)H * kHeadDim;
+        stage<kChunk, kHeadDim, kStateThreads>(sW, kPitch, w + base, ld, len, [](int, int, float x) { return -x; });
+        stage<kChunk, kSlab, kStateThreads>(sU, kSlab + 1, ut + base + j0, ld, len, Identity{});
         __syncthreads();
-        // U = U~ - W S   (rows r, slab columns j)
+        // Khat_ic = k_ic e^{Gamma_last,c - Gamma_ic}
+        stage2<kChunk, kHeadDim, kStateThreads>(sK, kPitch, gamma + base, k + base, ld, len,
+                                                [sgL](int, int c, float G, float kv) { return kv * expf(sgL[c] - G); });
+        if (tid < kHeadDim) sgC[tid] = expf(sgL[tid]);
+        // U = U~ - W S   (rows r, slab columns j; rows >= len stay 0)
         {
-            const int j = tid % kSlab;
-            for (int r = tid / kSlab; r < kChunk; r += kStateThreads / kSlab) {
-                float acc = 0.f;
-                if (r < len) {
-                    acc = ut[((t0 + r) * H + h) * kHeadDim + j0 + j];
-                    for (int c = 0; c < kHeadDim; ++c)
-                        acc = fmaf(-sW[r * kPitch + c], sS[c * (kSlab + 1) + j], acc);
-                    u_out[((t0 + r) * H + h) * kHeadDim + j0 + j] = acc;
+            float acc[2][4];
+#pragma unroll
+            for (int ii = 0; ii < 2; ++ii)
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) acc[ii][jj] = sU[(ty + 32 * ii) * (kSlab + 1) + tx + 8 * jj];
+            tile_fma<2, 4, 32, 8, kPitch, 1, kSlab + 1, 1>(acc, sW, sS, ty, tx, 0, kHeadDim);
+#pragma unroll
+            for (int ii = 0; ii < 2; ++ii) {
+                const int r = ty + 32 * ii;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = tx + 8 * jj;
+                    sU[r * (kSlab + 1) + j] = acc[ii][jj];
+                    if (r < len) u_out[((t0 + r) * H + h) * kHeadDim + j0 + j] = acc[ii][jj];
                 }
-                sU[r * (kSlab + 1) + j] = acc;
             }
         }
         __syncthreads();
         // S = Diag(gamma_last) S + Khat^T U
         {
-            const int j = tid % kSlab;
-            for (int c = tid / kSlab; c < kHeadDim; c += kStateThreads / kSlab) {
-                float acc = expf(sgC[c]) * sS[c * (kSlab + 1) + j];
-                for (int r = 0; r < len; ++r)
-                    acc = fmaf(sK[r * kPitch + c], sU[r * (kSlab + 1) + j], acc);
-                sS[c * (kSlab + 1) + j] = acc;
+            float acc[4][4];
+            tile_zero(acc);
+            tile_fma<4, 4, 32, 8, 1, kPitch, kSlab + 1, 1>(acc, sK, sU, ty, tx, 0, len);
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) {
+                const int c = ty + 32 * ii;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int j = tx + 8 * jj;
+                    sS[c * (kSlab + 1) + j] = fmaf(sgC[c], sS[c * (kSlab + 1) + j], acc[ii][jj]);
+                }
             }
         }
-        __syncthreads();
     }
+    __syncthreads();
     if (final_state) {
         for (int x = tid; x < kHeadDim * kSlab; x += kStateThreads) {
             const int c = x / kSlab, j = x % kSlab;
@@ -438,7 +451,7 @@ cudaError_t launch_staged(const StagedArgs& a, char* ws, const StagedLayout& L, 
         gate_cumsum_kernel<<<gc, 128, 0, stream>>>(a.g, a.A_log, a.dt_bias, a.lower_bound, table,
                                                    count, H, gamma);
         intra_chunk_kernel<<<gc, kIntraThreads, kIntraSmem, stream>>>(q, k, v, a.beta, gamma, table,
-                                                                      count, H, w, ut, p);
+                                                                      count, H, w, ut, p, a.t_mat);
     }
     if (a.N > 0) {
         dim3 gs((unsigned)a.N, (unsigned)H, kHeadDim / kSlab);
