@@ -162,10 +162,13 @@ __global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
 // ---------------------------------------------------------------------------
 // B2: per chunk and 32-channel tile: dKhat = U dS'^T, d(gamma q) = scale dO S^T,
 // dW = -dU S^T (rows r, channels c of the tile) and dgC_c = sum_j S_cj dS'_cj.
-// grid (max_chunks, H, 128 / 32), 256 threads.
+// grid (max_chunks, H, 128 / 32), 256 threads.  The sum over j runs in two halves of 64,
+// so that the staged operands take 66.5 KB and three blocks share an SM.
 constexpr int kB2Threads = 256;
 constexpr int kCT = 32;
-constexpr size_t kB2Smem = sizeof(float) * (2 * kCT * kPitch + 3 * kChunk * kPitch);
+constexpr int kJH = 64;                 // j columns staged at a time
+constexpr int kPH = kJH + 1;
+constexpr size_t kB2Smem = sizeof(float) * (2 * kCT * kPH + 3 * kChunk * kPH);
 
 __global__ void __launch_bounds__(kB2Threads) chunk_products_bwd_kernel(
     const float* __restrict__ u, const float* __restrict__ du, const __nv_bfloat16* __restrict__ d_out,
@@ -177,41 +180,42 @@ __global__ void __launch_bounds__(kB2Threads) chunk_products_bwd_kernel(
     const int4 e = table[ci];
     const int h = blockIdx.y, c0 = blockIdx.z * kCT, tid = threadIdx.x, len = e.z;
     extern __shared__ float sm[];
-    float* sS = sm;                        // [32 c][129 j] S rows of the tile
-    float* sN = sS + kCT * kPitch;         // [32 c][129 j] dS' rows of the tile
-    float* sU = sN + kCT * kPitch;         // [64][129] U
-    float* sO = sU + kChunk * kPitch;      // [64][129] dO
-    float* sD = sO + kChunk * kPitch;      // [64][129] dU
+    float* sS = sm;                        // [32 c][65 j] S rows of the tile
+    float* sN = sS + kCT * kPH;            // [32 c][65 j] dS' rows of the tile
+    float* sU = sN + kCT * kPH;            // [64][65] U
+    float* sO = sU + kChunk * kPH;         // [64][65] dO
+    float* sD = sO + kChunk * kPH;         // [64][65] dU
     const int64_t sbase = ((int64_t)ci * H + h) * kHeadDim * kHeadDim + (int64_t)c0 * kHeadDim;
-    stage<kCT, kHeadDim, kB2Threads>(sS, kPitch, chunk_states + sbase, kHeadDim, kCT, Identity{});
-    stage<kCT, kHeadDim, kB2Threads>(sN, kPitch, dsn + sbase, kHeadDim, kCT, Identity{});
     const int64_t base = ((int64_t)e.y * H + h) * kHeadDim, ld = (int64_t)H * kHeadDim;
-    stage<kChunk, kHeadDim, kB2Threads>(sU, kPitch, u + base, ld, len, Identity{});
-    stage<kChunk, kHeadDim, kB2Threads>(sO, kPitch, d_out + base, ld, len, Identity{});
-    stage<kChunk, kHeadDim, kB2Threads>(sD, kPitch, du + base, ld, len, Identity{});
-    __syncthreads();
-    // 2 x 4 register tiles of the three products: rows ty + 32 ii, channels tx + 8 jj
-    {
-        const int tx = tid % 8, ty = tid / 8;
-        float a1[2][4], a2[2][4], a3[2][4];
-        tile_zero(a1);
-        tile_zero(a2);
-        tile_zero(a3);
+    const int tx = tid % 8, ty = tid / 8;  // 2 x 4 tiles: rows ty + 32 ii, channels tx + 8 jj
+    float a1[2][4], a2[2][4], a3[2][4];
+    tile_zero(a1);
+    tile_zero(a2);
+    tile_zero(a3);
+    float gsum = 0.f;
+    for (int jh = 0; jh < kHeadDim; jh += kJH) {
+        if (jh) __syncthreads();           // the previous half is consumed
+        stage<kCT, kJH, kB2Threads>(sS, kPH, chunk_states + sbase + jh, kHeadDim, kCT, Identity{});
+        stage<kCT, kJH, kB2Threads>(sN, kPH, dsn + sbase + jh, kHeadDim, kCT, Identity{});
+        stage<kChunk, kJH, kB2Threads>(sU, kPH, u + base + jh, ld, len, Identity{});
+        stage<kChunk, kJH, kB2Threads>(sO, kPH, d_out + base + jh, ld, len, Identity{});
+        stage<kChunk, kJH, kB2Threads>(sD, kPH, du + base + jh, ld, len, Identity{});
+        __syncthreads();
 #pragma unroll 2
-        for (int j = 0; j < kHeadDim; ++j) {
+        for (int j = 0; j < kJH; ++j) {
             float u0[2], o0[2], d0[2], nv[4], sv[4];
 #pragma unroll
             for (int ii = 0; ii < 2; ++ii) {
                 const int r = ty + 32 * ii;
-                u0[ii] = sU[r * kPitch + j];
-                o0[ii] = sO[r * kPitch + j];
-                d0[ii] = sD[r * kPitch + j];
+                u0[ii] = sU[r * kPH + j];
+                o0[ii] = sO[r * kPH + j];
+                d0[ii] = sD[r * kPH + j];
             }
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
                 const int c = tx + 8 * jj;
-                nv[jj] = sN[c * kPitch + j];
-                sv[jj] = sS[c * kPitch + j];
+                nv[jj] = sN[c * kPH + j];
+                sv[jj] = sS[c * kPH + j];
             }
 #pragma unroll
             for (int ii = 0; ii < 2; ++ii)
@@ -222,24 +226,22 @@ __global__ void __launch_bounds__(kB2Threads) chunk_products_bwd_kernel(
                     a3[ii][jj] = fmaf(d0[ii], sv[jj], a3[ii][jj]);
                 }
         }
+        if (tid < kCT)
+            for (int j = 0; j < kJH; ++j) gsum = fmaf(sS[tid * kPH + j], sN[tid * kPH + j], gsum);
+    }
 #pragma unroll
-        for (int ii = 0; ii < 2; ++ii) {
-            const int r = ty + 32 * ii;
-            if (r >= len) continue;
+    for (int ii = 0; ii < 2; ++ii) {
+        const int r = ty + 32 * ii;
+        if (r >= len) continue;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c0 + tx + 8 * jj;
-                dkhat[idx] = a1[ii][jj];
-                dqg[idx] = scale * a2[ii][jj];
-                dw[idx] = -a3[ii][jj];
-            }
+        for (int jj = 0; jj < 4; ++jj) {
+            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c0 + tx + 8 * jj;
+            dkhat[idx] = a1[ii][jj];
+            dqg[idx] = scale * a2[ii][jj];
+            dw[idx] = -a3[ii][jj];
         }
     }
-    if (tid < kCT) {
-        float a = 0.f;
-        for (int j = 0; j < kHeadDim; ++j) a = fmaf(sS[tid * kPitch + j], sN[tid * kPitch + j], a);
-        dgc[((int64_t)ci * H + h) * kHeadDim + c0 + tid] = a;
-    }
+    if (tid < kCT) dgc[((int64_t)ci * H + h) * kHeadDim + c0 + tid] = gsum;
 }
 
 // ---------------------------------------------------------------------------
