@@ -39,6 +39,8 @@ BYTES_PER_TOKEN_HEAD = 1540          # q,k,v bf16 768 + g fp32 512 + beta 4 + ou
 STATE_BYTES = 128 * 128 * 4          # one (sequence, head) state, read or written
 FLOP_PER_TOKEN_HEAD = 180224         # 10 C D + 6 D^2 with C = 64, D = 128
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0             # the spec sheet's HBM3e figure, for context
+NOMINAL_BF16_TFLOPS = 2250.0         # dense bf16 tensor peak, spec sheet, for context
 
 
 def parse():
@@ -70,6 +72,14 @@ def measured_hbm_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_bf16_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
 
 
 GDN_BYTES_PER_TOKEN_HEAD = 1032    # q,k,v bf16 768 + g fp32 4 + beta 4 + out bf16 256
@@ -624,7 +634,12 @@ def main():
             "kernel": ("kda_fused_kernel<scalar gate>" if args.gdn else "kda_fused_kernel") if fused
             else "staged kernels",
             "kernel_ms": kernel_ms, "algorithmic_bytes": alg_bytes,
-            "tflops": tflops}
+            "tflops": tflops,
+            "frac_nominal_hbm": achieved / NOMINAL_HBM_GBS,
+            "tensor": {"achieved_tflops": tflops, "peak_tflops": measured_bf16_peak(),
+                       "frac": tflops / measured_bf16_peak(),
+                       "frac_nominal": tflops / NOMINAL_BF16_TFLOPS,
+                       "flop_per_token_head": FLOP_PER_TOKEN_HEAD}}
 
     # end to end through the public API with host buffers
     e2e = None

@@ -65,6 +65,8 @@ def _load():
     lib.kda_fwd_staged.argtypes = fwd_args + [vp, ctypes.c_size_t, vp]
     lib.kda_staged_workspace_size.restype = ctypes.c_size_t
     lib.kda_staged_workspace_size.argtypes = [kda_dims, ctypes.c_int]
+    lib.kda_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.kda_fwd_workspace_size.argtypes = [kda_dims]
     lib.kda_staged_workspace_layout.restype = ctypes.c_int
     lib.kda_staged_workspace_layout.argtypes = [kda_dims, ctypes.c_int, ctypes.POINTER(kda_staged_layout)]
     lib.kda_strerror.restype = ctypes.c_char_p
@@ -102,7 +104,7 @@ EXPORTED = ("kda_fwd", "kda_fwd_staged", "kda_staged_workspace_size",
             "kda_staged_workspace_layout", "kda_strerror", "kda_check_device_error",
             "kda_last_device_error_bits", "kda_version", "kda_fwd_staged_noalloc",
             "kda_noalloc_scratch_bytes", "kda_decode", "kda_gdn_fwd", "kda_gdn_decode",
-            "kda_state_affine", "kda_bwd", "kda_bwd_workspace_size")
+            "kda_state_affine", "kda_bwd", "kda_bwd_workspace_size", "kda_fwd_workspace_size")
 
 
 def lib() -> ctypes.CDLL:

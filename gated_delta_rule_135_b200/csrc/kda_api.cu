@@ -195,6 +195,11 @@ size_t kda_staged_workspace_size(kda_dims dims, int varlen) {
     return kda_staged_workspace_layout(dims, varlen, &L) == KDA_OK ? L.total : 0;
 }
 
+size_t kda_fwd_workspace_size(kda_dims dims) {
+    const size_t a = kda_staged_workspace_size(dims, 1), b = kda_staged_workspace_size(dims, 0);
+    return a > b ? a : b;
+}
+
 kda_status kda_fwd_staged(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, const float* A_log, const float* dt_bias,
                           float lower_bound, float scale, const float* initial_state,

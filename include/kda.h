@@ -130,6 +130,12 @@ typedef struct {
     int64_t max_chunks;   /* ceil(Ttot / 64) + N */
 } kda_staged_layout;
 
+/* Bytes of workspace kda_fwd_staged needs for `dims`, whichever layout the call uses: the
+ * larger of the varlen reading (N = num_seqs, Ttot = seqlen) and the fixed one (N = batch,
+ * Ttot = batch * seqlen).  kda_fwd itself takes no workspace (its staged fallback allocates
+ * stream-ordered).  0 for invalid dims. */
+size_t kda_fwd_workspace_size(kda_dims dims);
+
 /* varlen != 0: the call passes cu_seqlens (N = num_seqs, Ttot = seqlen);
  * varlen == 0: fixed layout (N = batch, Ttot = batch * seqlen). */
 kda_status kda_staged_workspace_layout(kda_dims dims, int varlen, kda_staged_layout* layout);

@@ -136,6 +136,7 @@ def test_staged_workspace_layout_is_consistent():
         assert L.u - L.p >= 4 * T * H * 64
         assert L.total - L.chunk_states >= 4 * L.max_chunks * H * 128 * 128
         assert kda.lib().kda_staged_workspace_size(dims, varlen) == L.total
+        assert kda.lib().kda_fwd_workspace_size(dims) >= L.total
 
 
 def test_decode_rejects_bad_arguments():
@@ -213,8 +214,9 @@ def test_bwd_workspace_extends_the_staged_layout():
         T, H = dims.seqlen * (1 if varlen else dims.batch), dims.num_heads
         N = dims.num_seqs if varlen else dims.batch
         mc = math.ceil(T / 64) + N
-        extra = 4 * (mc * H * 128 * 128 + 5 * T * H * 128 + mc * H * 64 * 64 + mc * H * 128 + mc * H
-                     + mc * H * 128)
+        # T per chunk, dS' per chunk, dU dKhat d(gamma q) dW dGamma, dA per chunk, dgC, partials
+        extra = 4 * (mc * H * 64 * 64 + mc * H * 128 * 128 + 5 * T * H * 128 + mc * H * 64 * 64
+                     + mc * H * 128 + mc * H + mc * H * 128)
         staged = kda.lib().kda_staged_workspace_size(dims, varlen)
         assert kda.lib().kda_bwd_workspace_size(dims, varlen) >= staged + extra
         assert kda.lib().kda_bwd_workspace_size(dims, varlen) <= staged + extra + 16 * 256
