@@ -60,6 +60,9 @@ def parse():
                     help="time kda_decode (one token per sequence) instead of the prefill")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward kda_bwd (all gradients) instead of the forward")
+    ap.add_argument("--segments", type=int, default=0,
+                    help="one-sequence workloads: run the forward as R segments per pass "
+                         "(cp.segmented_prefill) instead of one kda_fwd call; -1 = cp.choose_segments")
     ap.add_argument("--decode-batch", type=int, default=256)
     ap.add_argument("--decode-heads", type=int, default=96)
     return ap.parse_args()
@@ -590,8 +593,22 @@ def main():
     fused = args.gdn or x["lower_bound"] >= kda.FUSED_MIN_LOWER_BOUND
     launches_per_step = 1 if fused else 5
     fwd = kda.kda_gdn_fwd if args.gdn else kda.kda_fwd
+    seg_ws = {}
+    if args.segments:
+        assert w.N == 1 and fused, "--segments takes a one-sequence workload on the fused path"
+        from gated_delta_rule_135_b200 import cp
+        from gated_delta_rule_135_b200.cp import choose_segments, segment_offsets
+        if args.segments < 0:     # the library's choice
+            args.segments = choose_segments(w.T, w.H, torch.cuda.get_device_properties(dev).multi_processor_count)
+        n_seg = len(segment_offsets(w.T, args.segments)) - 1
+        launches_per_step = 1 if n_seg == 1 else 3 + (n_seg - 1)
 
     def step():
+        if args.segments:
+            o, f = cp.segmented_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"],
+                                        xd["dt_bias"], x["lower_bound"], x["scale"], xd["initial_state"],
+                                        segments=args.segments, gdn=args.gdn, out=out, workspace=seg_ws)
+            return
         fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"],
             x["lower_bound"], x["scale"], xd["initial_state"], xd["cu_seqlens"], out=out,
             final_state=fin, batch=x["batch"])
@@ -628,11 +645,12 @@ def main():
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak,
             "traffic": (dram_traffic_from_profile("kda_fused_kernel<scalar gate>" if args.gdn else "kda_fused_kernel",
-                                                  w.T * w.H) if fused else None),
+                                                  w.T * w.H) if fused and not args.segments else None),
             "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
             else "fallback 6650 GB/s",
-            "kernel": ("kda_fused_kernel<scalar gate>" if args.gdn else "kda_fused_kernel") if fused
-            else "staged kernels",
+            "kernel": (f"segmented prefill ({args.segments} segments: 3 fused launches + folds)" if args.segments
+                       else ("kda_fused_kernel<scalar gate>" if args.gdn else "kda_fused_kernel") if fused
+                       else "staged kernels"),
             "kernel_ms": kernel_ms, "algorithmic_bytes": alg_bytes,
             "tflops": tflops,
             "frac_nominal_hbm": achieved / NOMINAL_HBM_GBS,
@@ -678,13 +696,17 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": ("GDN (scalar-gate) prefill throughput (Mtokens/s) at T=8192 H=96 D=128 varlen"
-                       if args.gdn else "KDA prefill throughput (Mtokens/s) at T=8192 H=96 D=128 varlen"),
+            "metric": (("GDN (scalar-gate) prefill throughput (Mtokens/s) at T=8192 H=96 D=128 varlen"
+                        if args.gdn else "KDA prefill throughput (Mtokens/s) at T=8192 H=96 D=128 varlen")
+                       if args.workload == 2 else
+                       f"{'GDN (scalar-gate)' if args.gdn else 'KDA'} prefill throughput (Mtokens/s), {w.name}"),
             "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded kda_workloads, no dataset)",
-            "config": {"workload": ("GDN (one gate per token-head) " if args.gdn else "") + w.describe(), "model": "KDA layer forward (no weights)",
+            "config": {"workload": ("GDN (one gate per token-head) " if args.gdn else "") + w.describe()
+                       + (f"; run as {args.segments} segments (maps, fold, final pass)" if args.segments else ""),
+                       "model": "KDA layer forward (no weights)",
                        "global_batch": w.N * world, "seq_len": w.T, "heads": w.H,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "precision": "bf16 q/k/v/out, fp32 gates and state; bf16/fp16 MMA operands, fp32 accumulate",

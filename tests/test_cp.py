@@ -99,3 +99,27 @@ def test_cp_two_ranks_equals_unsplit_run():
 
 def test_cp_two_ranks_scalar_gate():
     _check(gdn=True)
+
+
+def test_segment_offsets_are_chunk_aligned_and_cover():
+    import kda_build
+    kda_build.build()
+    from gated_delta_rule_135_b200.cp import segment_offsets
+    for T, R in ((700, 3), (131072, 8), (131072, 37), (64, 5), (1, 4), (1000, 1)):
+        cuts = segment_offsets(T, R)
+        assert cuts[0] == 0 and cuts[-1] == T
+        assert all(b > a for a, b in zip(cuts, cuts[1:]))
+        assert all(c % 64 == 0 for c in cuts[:-1])
+        assert len(cuts) - 1 <= R
+
+
+def test_choose_segments_fills_the_sms_only_when_heads_do_not():
+    import kda_build
+    kda_build.build()
+    from gated_delta_rule_135_b200.cp import choose_segments
+    # many (sequence, head) units already fill 148 SMs: no split
+    assert choose_segments(8192, 96, 148) == 1
+    assert choose_segments(1024, 64, 148) == 1
+    # one long sequence with 32 heads: a split that fills the SMs
+    R = choose_segments(131072, 32, 148)
+    assert R >= 4 and R * 32 >= 128

@@ -63,3 +63,45 @@ def test_state_affine_matches_matmul():
     out = kda.kda_state_affine(A.cuda(), S.cuda(), B.cuda())
     ref = (A.double() @ S.double() + B.double())
     assert torch.allclose(out.cpu().double(), ref, rtol=1e-5, atol=1e-4)
+
+
+@pytest.mark.parametrize("gdn", [False, True], ids=["kda", "scalar_gate"])
+def test_segmented_prefill_matches_oracle(gdn):
+    """One sequence split into segments run as one varlen batch per pass (maps, fold, final)."""
+    kda, cp = _kda()
+    H = 3
+    x = W.make_inputs(W.custom([700], H=H, packed=False, init="normal", wid=73))
+    if gdn:
+        x = W.gdn_inputs(x)
+    xd = to_device(x)
+    assert cp.segment_offsets(700, 3) == [0, 256, 512, 700]
+    ws = {}
+    for _ in range(2):          # the second call reuses the cached buffers
+        out, fin = cp.segmented_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"],
+                                        xd["dt_bias"], x["lower_bound"], x["scale"], xd["initial_state"],
+                                        segments=3, gdn=gdn, workspace=ws)
+    assert kda.kda_check_device_error() == 0
+    f = oracle.gdn_recurrent if gdn else oracle.recurrent
+    ref_o, ref_f = f(x["q"], x["k"], x["v"], x["g"], x["beta"], x["A_log"], x["dt_bias"], x["lower_bound"],
+                     x["scale"], x["initial_state"], None)
+    o = out.float().cpu().numpy().astype(np.float64)
+    assert oracle.rel_l2(o, ref_o) <= OUT_REL_L2
+    assert oracle.max_abs(o, ref_o) <= OUT_MAX_ABS
+    assert oracle.rel_l2(fin.cpu().numpy(), ref_f) <= STATE_REL_L2
+
+
+def test_segmented_prefill_long_sequence_full_size():
+    """T = 131072, H = 32 with states, split in 8 segments, against the fp64 oracle."""
+    kda, cp = _kda()
+    w = W.WORKLOADS[4]
+    x = W.make_inputs(w)
+    xd = to_device(x)
+    out, fin = cp.segmented_prefill(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"],
+                                    x["lower_bound"], x["scale"], xd["initial_state"], segments=8)
+    assert kda.kda_check_device_error() == 0
+    ref_o, ref_f = oracle.recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], x["A_log"], x["dt_bias"],
+                                    x["lower_bound"], x["scale"], x["initial_state"], None)
+    o = out.float().cpu().numpy().astype(np.float64)
+    assert oracle.rel_l2(o, ref_o) <= OUT_REL_L2
+    assert oracle.max_abs(o, ref_o) <= OUT_MAX_ABS
+    assert oracle.rel_l2(fin.cpu().numpy(), ref_f) <= STATE_REL_L2
