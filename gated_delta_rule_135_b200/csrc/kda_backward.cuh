@@ -95,6 +95,16 @@ __global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
             break;
         }
         __syncthreads();   // the previous chunk's dS is complete; its operands are consumed
+        if (jc > 0) {      // the next chunk in this scan (full: only a sequence's last chunk is short)
+            const int64_t nb = ((t0 - kChunk) * H + h) * kHeadDim, ldb = (int64_t)H * kHeadDim;
+            prefetch_rows_l2(gamma + nb, ldb * 4, kChunk, kHeadDim * 4, kB1Threads);
+            prefetch_rows_l2(w + nb, ldb * 4, kChunk, kHeadDim * 4, kB1Threads);
+            prefetch_rows_l2(k + nb, ldb * 2, kChunk, kHeadDim * 2, kB1Threads);
+            prefetch_rows_l2(q + nb, ldb * 2, kChunk, kHeadDim * 2, kB1Threads);
+            prefetch_rows_l2(p + ((t0 - kChunk) * H + h) * kChunk, (int64_t)H * kChunk * 4, kChunk, kChunk * 4,
+                             kB1Threads);
+            prefetch_rows_l2(d_out + nb + j0, ldb * 2, kChunk, kSlab * 2, kB1Threads);
+        }
         // dS' of this chunk
         for (int x = tid; x < kHeadDim * kSlab; x += kB1Threads) {
             const int c = x / kSlab, j = x % kSlab;
@@ -366,10 +376,18 @@ __global__ void __launch_bounds__(kB3Threads) t_side_bwd_kernel(
 // with sum_r dKhat Khat + dgC gamma_C added to the last row's dGamma.  d log a is dGamma
 // summed from the chunk's end; the gate's chain rule gives dg and per-chunk partial sums of
 // dA_log and ddt_bias (reduced by param_reduce_kernel).
+//
+// kFactored (gates clamped at lower_bound >= -5.3): the four pair sums become register-tiled
+// products.  With s the start of a 16-token block, e^{G_r - G_i} = e^{G_r - G_s} e^{G_s - G_i},
+// both factors inside the fp32 range when r, i lie in or after that block (16 x 5.3 < 87):
+//   row terms:    sum over column blocks b of e^{G_r - G_sb} (dA or dP)[r, b] (k e^{G_sb - G})[b]
+//   column terms: sum over row blocks b of e^{G_sb - G_i} (beta dA or dP)[b, i]^T (k or q e^{G - G_sb})[b]
+// The operands k e^{G_s - G} and k, q e^{G - G_s} take s as the row's own block start.
 constexpr int kB3bThreads = 512;
 constexpr size_t kB3bSmem = sizeof(float) * (5 * kChunk * kPitch + 2 * kChunk * kPitchC + kChunk + 2 * kHeadDim +
                                              kChunk * 4 + 4);
 
+template <bool kFactored>
 __global__ void __launch_bounds__(kB3bThreads) decay_bwd_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const float* __restrict__ g,
     const float* __restrict__ beta, const float* __restrict__ A_log, const float* __restrict__ dt_bias,
@@ -386,8 +404,9 @@ __global__ void __launch_bounds__(kB3bThreads) decay_bwd_kernel(
     extern __shared__ float sm[];
     float* sX = sm;                          // [64][129] dO, then k
     float* sY = sX + kChunk * kPitch;        // [64][129] U, then q
-    float* sa = sY + kChunk * kPitch;        // [64][129] a = e^{log a}
+    float* sa = sY + kChunk * kPitch;        // [64][129] a = e^{log a} (kFactored: Gamma)
     float* sT1 = sa + kChunk * kPitch;       // [64][129] dGamma without the dKhat Khat term
+                                             //           (kFactored: first k e^{G_s - G})
     float* sT2 = sT1 + kChunk * kPitch;      // [64][129] dKhat Khat
     float* sdP = sT2 + kChunk * kPitch;      // [64][65]
     float* sdA = sdP + kChunk * kPitchC;     // [64][65]
@@ -409,9 +428,12 @@ __global__ void __launch_bounds__(kB3bThreads) decay_bwd_kernel(
     stage<kChunk, kChunk, kB3bThreads>(sdA, kPitchC, da + ((int64_t)ci * H + h) * kChunk * kChunk, kChunk, kChunk,
                                        Identity{});
     __syncthreads();
-    stage<kChunk, kHeadDim, kB3bThreads>(sa, kPitch, g + base, ld, len, [sdb, nexp, lower_bound](int, int c, float x) {
-        return expf(gate_log_decay(x + sdb[c], nexp, lower_bound));
-    });
+    if constexpr (kFactored)
+        stage<kChunk, kHeadDim, kB3bThreads>(sa, kPitch, gamma + base, ld, len, Identity{});
+    else
+        stage<kChunk, kHeadDim, kB3bThreads>(sa, kPitch, g + base, ld, len, [sdb, nexp, lower_bound](int, int c, float x) {
+            return expf(gate_log_decay(x + sdb[c], nexp, lower_bound));
+        });
     {   // dP = scale dO U^T (i <= r < len): 2 x 4 tiles, rows ty + 32 ii, columns tx + 16 jj
         const int tx = tid % 16, ty = tid / 16;
         float acc[2][4];
@@ -432,6 +454,124 @@ __global__ void __launch_bounds__(kB3bThreads) decay_bwd_kernel(
     stage<kChunk, kHeadDim, kB3bThreads>(sX, kPitch, k + base, ld, len, Identity{});
     stage<kChunk, kHeadDim, kB3bThreads>(sY, kPitch, q + base, ld, len, Identity{});
     __syncthreads();
+    if constexpr (kFactored) {
+        // operands: sT1 <- k e^{G_s - G}, sX <- k e^{G - G_s}, sY <- q e^{G - G_s}, s = r's block start
+        for (int x = tid; x < kChunk * kHeadDim; x += kB3bThreads) {
+            const int r = x / kHeadDim, cc = x % kHeadDim;
+            float up = 0.f, down = 0.f;
+            if (r < len) {
+                const float gr = sa[r * kPitch + cc], gs = sa[(r & ~15) * kPitch + cc];
+                up = expf(gs - gr);
+                down = expf(gr - gs);
+            }
+            const float kv = sX[r * kPitch + cc];
+            sT1[r * kPitch + cc] = kv * up;
+            sX[r * kPitch + cc] = kv * down;
+            sY[r * kPitch + cc] *= down;
+        }
+        __syncthreads();
+        const int tx = tid % 32, ty = tid / 32;   // rows ty + 16 ii (block ii), channels tx + 32 jj
+        float RA[4][4], RP[4][4], CA[4][4], CP[4][4];
+        tile_zero(RA);
+        tile_zero(RP);
+        tile_zero(CA);
+        tile_zero(CP);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            if (16 * b >= len) break;
+            float pa[4][4], pp[4][4];
+            // row terms from column block b (rows in blocks >= b)
+            tile_zero(pa);
+            tile_zero(pp);
+            for (int i = 16 * b; i < 16 * b + 16; ++i) {
+                float kc[4];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) kc[jj] = sT1[i * kPitch + tx + 32 * jj];
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) {
+                    if (ii < b) continue;
+                    const float va = sdA[(ty + 16 * ii) * kPitchC + i], vp = sdP[(ty + 16 * ii) * kPitchC + i];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        pa[ii][jj] = fmaf(va, kc[jj], pa[ii][jj]);
+                        pp[ii][jj] = fmaf(vp, kc[jj], pp[ii][jj]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) {
+                if (ii < b) continue;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int r = ty + 16 * ii, cc = tx + 32 * jj;
+                    const float sc = expf(fminf(sa[r * kPitch + cc] - sa[16 * b * kPitch + cc], 0.f));
+                    RA[ii][jj] = fmaf(sc, pa[ii][jj], RA[ii][jj]);
+                    RP[ii][jj] = fmaf(sc, pp[ii][jj], RP[ii][jj]);
+                }
+            }
+            // column terms from row block b (columns in blocks <= b)
+            tile_zero(pa);
+            tile_zero(pp);
+            for (int r = 16 * b; r < 16 * b + 16; ++r) {
+                float kr[4], qr[4];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    kr[jj] = sX[r * kPitch + tx + 32 * jj];
+                    qr[jj] = sY[r * kPitch + tx + 32 * jj];
+                }
+                const float br = sb[r];
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) {
+                    if (ii > b) continue;
+                    const float va = br * sdA[r * kPitchC + ty + 16 * ii], vp = sdP[r * kPitchC + ty + 16 * ii];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        pa[ii][jj] = fmaf(va, kr[jj], pa[ii][jj]);
+                        pp[ii][jj] = fmaf(vp, qr[jj], pp[ii][jj]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int ii = 0; ii < 4; ++ii) {
+                if (ii > b) continue;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int i = ty + 16 * ii, cc = tx + 32 * jj;
+                    const float sc = expf(sa[16 * b * kPitch + cc] - sa[i * kPitch + cc]);
+                    CA[ii][jj] = fmaf(sc, pa[ii][jj], CA[ii][jj]);
+                    CP[ii][jj] = fmaf(sc, pp[ii][jj], CP[ii][jj]);
+                }
+            }
+        }
+        __syncthreads();   // sT1 (an operand until here) now receives dGamma
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) {
+            const int t = ty + 16 * ii;
+            float pb[4] = {0.f, 0.f, 0.f, 0.f};
+            if (t < len) {
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int cc = tx + 32 * jj;
+                    const int64_t idx = (((int64_t)e.y + t) * H + h) * kHeadDim + cc;
+                    const float G = sa[t * kPitch + cc], kt = bf(k[idx]), qt = bf(q[idx]);
+                    const float dQ = dqg[idx], dKh = dkhat[idx];
+                    const float gam = expf(G), eK = expf(sgC[cc] - G), bt = sb[t];
+                    const float ra = RA[ii][jj], rp = RP[ii][jj], cs = CA[ii][jj] + CP[ii][jj];
+                    dq_out[idx] = fmaf(dQ, gam, rp);
+                    dk_io[idx] = dk_io[idx] + bt * ra + cs + dKh * eK;
+                    sT1[t * kPitch + cc] = dG_t[idx] + dQ * gam * qt + bt * kt * ra + qt * rp - kt * cs;
+                    sT2[t * kPitch + cc] = dKh * kt * eK;
+                    pb[jj] = kt * ra;
+                }
+            }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                float v = pb[jj];
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (tx == 0) sbp[t * 4 + jj] = v;
+            }
+        }
+    } else {
     const int c = tid % kHeadDim;
     for (int t = tid / kHeadDim; t < len; t += kB3bThreads / kHeadDim) {
         const int64_t idx = (((int64_t)e.y + t) * H + h) * kHeadDim + c;
@@ -462,38 +602,69 @@ __global__ void __launch_bounds__(kB3bThreads) decay_bwd_kernel(
         for (int o = 16; o > 0; o >>= 1) pb += __shfl_xor_sync(0xffffffffu, pb, o);
         if ((tid & 31) == 0) sbp[t * 4 + c / 32] = pb;
     }
+    }
     __syncthreads();
     if (tid < kChunk && tid < len) {
         const int64_t bi = ((int64_t)e.y + tid) * H + h;
         dbeta_io[bi] = dbeta_io[bi] + ((sbp[tid * 4] + sbp[tid * 4 + 1]) + (sbp[tid * 4 + 2] + sbp[tid * 4 + 3]));
     }
     // gate: d log a_s = sum_{t >= s} dGamma_t (the dKhat Khat terms of rows t < s, which the last
-    // row's sum adds back, remain) + dgC gamma_C
-    if (tid < kHeadDim) {
-        float yall = 0.f;
-        for (int t = 0; t < len; ++t) yall += sT2[t * kPitch + c];
-        float R = yall + dgc[((int64_t)ci * H + h) * kHeadDim + c] * expf(sgC[c]);
-        const float db = sdb[c];
+    // row's sum adds back, remain) + dgC gamma_C.  The raw gate input is staged into sX (free
+    // now); each channel's reverse sum runs as four 16-row segments, one thread each.
+    stage<kChunk, kHeadDim, kB3bThreads>(sX, kPitch, g + base, ld, len, Identity{});
+    float* segD = sY;                        // [4][128] segment sums of dGamma - dKhat Khat
+    float* segY = sY + 4 * kHeadDim;         // [4][128] segment sums of dKhat Khat
+    float* segT = sY + 8 * kHeadDim;         // [4][128] ddt_bias partials
+    float* warpA = sY + 12 * kHeadDim;       // [16] dA_log partials
+    const int gc = tid % kHeadDim, seg = tid / kHeadDim;
+    const int r0 = seg * 16, r1 = min(r0 + 16, len);
+    {
+        float sd = 0.f, sy = 0.f;
+        for (int r = r0; r < r1; ++r) {
+            sd += sT1[r * kPitch + gc] - sT2[r * kPitch + gc];
+            sy += sT2[r * kPitch + gc];
+        }
+        segD[seg * kHeadDim + gc] = sd;
+        segY[seg * kHeadDim + gc] = sy;
+    }
+    __syncthreads();
+    {
+        float R = ((segY[gc] + segY[kHeadDim + gc]) + (segY[2 * kHeadDim + gc] + segY[3 * kHeadDim + gc])) +
+                  dgc[((int64_t)ci * H + h) * kHeadDim + gc] * expf(sgC[gc]);
+        for (int sg = 3; sg > seg; --sg) R += segD[sg * kHeadDim + gc];
+        const float db = sdb[gc];
         float p_dt = 0.f, p_al = 0.f;
-        for (int s = len - 1; s >= 0; --s) {
-            R += sT1[s * kPitch + c] - sT2[s * kPitch + c];
-            const int64_t idx = (((int64_t)e.y + s) * H + h) * kHeadDim + c;
-            const float x = g[idx] + db;
+        for (int r = r1 - 1; r >= r0; --r) {
+            R += sT1[r * kPitch + gc] - sT2[r * kPitch + gc];
+            const float x = sX[r * kPitch + gc] + db;
             const float raw = nexp * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))));
             float dgv = 0.f;
             if (raw >= lower_bound) {
                 dgv = R * nexp / (1.f + expf(-x));
                 p_al = fmaf(R, raw, p_al);
             }
-            dg_out[idx] = dgv;
+            sa[r * kPitch + gc] = dgv;     // staged for vector stores
             p_dt += dgv;
         }
-        ddt_part[((int64_t)ci * H + h) * kHeadDim + c] = p_dt;
+        __syncthreads();                   // segD / segY are consumed
+        segT[seg * kHeadDim + gc] = p_dt;
         for (int o = 16; o > 0; o >>= 1) p_al += __shfl_xor_sync(0xffffffffu, p_al, o);
-        if ((tid & 31) == 0) sred[tid / 32] = p_al;
+        if ((tid & 31) == 0) warpA[tid / 32] = p_al;
     }
     __syncthreads();
-    if (tid == 0) dalog_part[(int64_t)ci * H + h] = (sred[0] + sred[1]) + (sred[2] + sred[3]);
+    for (int x = tid; x < len * (kHeadDim / 4); x += kB3bThreads) {
+        const int r = x / (kHeadDim / 4), c4 = 4 * (x % (kHeadDim / 4));
+        const float* src = sa + r * kPitch + c4;
+        *reinterpret_cast<float4*>(dg_out + base + (int64_t)r * ld + c4) = make_float4(src[0], src[1], src[2], src[3]);
+    }
+    if (tid < kHeadDim)
+        ddt_part[((int64_t)ci * H + h) * kHeadDim + tid] =
+            (segT[tid] + segT[kHeadDim + tid]) + (segT[2 * kHeadDim + tid] + segT[3 * kHeadDim + tid]);
+    if (tid == 0) {
+        float t = 0.f;
+        for (int w = 0; w < kB3bThreads / 32; ++w) t += warpA[w];
+        dalog_part[(int64_t)ci * H + h] = t;
+    }
 }
 
 // dA_log[h] and ddt_bias[h][c]: the per-chunk partials summed in chunk order.  grid H, 128 threads.
@@ -553,7 +724,9 @@ cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const Bw
             cudaSuccess) return err;
         if ((err = cudaFuncSetAttribute(bwd::t_side_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)bwd::kB3aSmem)) != cudaSuccess) return err;
-        if ((err = cudaFuncSetAttribute(bwd::decay_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if ((err = cudaFuncSetAttribute(bwd::decay_bwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)bwd::kB3bSmem)) != cudaSuccess) return err;
+        if ((err = cudaFuncSetAttribute(bwd::decay_bwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)bwd::kB3bSmem)) != cudaSuccess) return err;
         attrs_set = true;
     }
@@ -601,7 +774,8 @@ cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const Bw
         dim3 g3((unsigned)L.max_chunks, (unsigned)H);
         bwd::t_side_bwd_kernel<<<g3, bwd::kB3Threads, bwd::kB3aSmem, stream>>>(
             k, v, a.beta, gamma, tm, du, dw, table, count, H, d.dk, d.dv, dG, d.dbeta, da);
-        bwd::decay_bwd_kernel<<<g3, bwd::kB3bThreads, bwd::kB3bSmem, stream>>>(
+        auto decay = fused_supported(a.lower_bound) ? bwd::decay_bwd_kernel<true> : bwd::decay_bwd_kernel<false>;
+        decay<<<g3, bwd::kB3bThreads, bwd::kB3bSmem, stream>>>(
             q, k, a.g, a.beta, a.A_log, a.dt_bias, a.lower_bound, a.scale, gamma, u, dO, da, dqg, dkhat, dgc, dG,
             table, count, H, d.dq, d.dk, d.dg, d.dbeta, dalog_part, ddt_part);
     }

@@ -281,6 +281,14 @@ __global__ void __launch_bounds__(kStateThreads) state_prop_kernel(
     for (int64_t t0 = b; t0 < e; t0 += kChunk, ++chunk_id) {
         const int len = (int)(e - t0 < kChunk ? e - t0 : kChunk);
         __syncthreads();   // the previous chunk's state update is complete
+        if (t0 + kChunk < e) {   // the next chunk's rows into L2
+            const int nlen = (int)(e - t0 - kChunk < kChunk ? e - t0 - kChunk : kChunk);
+            const int64_t nb = ((t0 + kChunk) * H + h) * kHeadDim, ldb = (int64_t)H * kHeadDim;
+            prefetch_rows_l2(w + nb, ldb * 4, nlen, kHeadDim * 4, kStateThreads);
+            prefetch_rows_l2(gamma + nb, ldb * 4, nlen, kHeadDim * 4, kStateThreads);
+            prefetch_rows_l2(k + nb, ldb * 2, nlen, kHeadDim * 2, kStateThreads);
+            prefetch_rows_l2(ut + nb + j0, ldb * 4, nlen, kSlab * 4, kStateThreads);
+        }
         // record the chunk's starting state
         if (chunk_id < max_chunks) {
             for (int x = tid; x < kHeadDim * kSlab; x += kStateThreads) {

@@ -124,6 +124,18 @@ __device__ __forceinline__ void stage2(float* __restrict__ dst, int pitch, const
     }
 }
 
+// Pulls `rows` rows of `row_bytes` bytes, row r at base + r * ld_bytes, into L2: one
+// prefetch per 128-byte line, spread over the block.  The serial chunk scans call it for the
+// next chunk so that its staging loads hit L2.
+__device__ __forceinline__ void prefetch_rows_l2(const void* base, int64_t ld_bytes, int rows, int row_bytes,
+                                                 int nthreads) {
+    const int lines = (row_bytes + 127) / 128;
+    for (int x = threadIdx.x; x < rows * lines; x += nthreads) {
+        const char* ptr = static_cast<const char*>(base) + (int64_t)(x / lines) * ld_bytes + (x % lines) * 128;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+    }
+}
+
 struct Identity {
     __device__ float operator()(int, int, float v) const { return v; }
 };
