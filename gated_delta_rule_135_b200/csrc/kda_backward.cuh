@@ -54,10 +54,11 @@ __device__ int64_t first_chunk_id(const int32_t* cu_seqlens, int n, int64_t seql
 
 // ---------------------------------------------------------------------------
 // B1: dS backwards over a sequence's chunks; per chunk stores dS' (the gradient of the
-// state after it) and dU.  grid (N, H, 128 / kSlab), 256 threads; each block owns a
-// 128 x kSlab column slab of dS.  Register tiles: dU 2 x 4 and dS 4 x 4 per thread.
-constexpr int kB1Threads = 256;
-constexpr int kSP = kSlab + 1;
+// state after it) and dU.  grid (N, H, 2), 512 threads; each block owns a 128 x 64 column
+// slab of dS.  Register tiles: dU 2 x 4 and dS 4 x 4 per thread.
+constexpr int kB1Threads = 512;
+constexpr int kB1Slab = 64;              // dS columns per block
+constexpr int kSP = kB1Slab + 1;
 constexpr size_t kB1Smem = sizeof(float) * (kHeadDim * kSP + 3 * kChunk * kPitch + kChunk * kPitchC +
                                             2 * kChunk * kSP + 2 * kHeadDim);
 
@@ -67,25 +68,25 @@ __global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
     const float* __restrict__ d_final, const int32_t* __restrict__ cu_seqlens, int64_t seqlen,
     int64_t total_tokens, int H, float scale, int64_t max_chunks, float* __restrict__ dsn_out,
     float* __restrict__ du_out, float* __restrict__ d_initial) {
-    const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kSlab, tid = threadIdx.x;
+    const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kB1Slab, tid = threadIdx.x;
     extern __shared__ float sm[];
-    float* sdS = sm;                                   // [128][33]
+    float* sdS = sm;                                   // [128][65]
     float* sKh = sdS + kHeadDim * kSP;                 // [64][129] Khat
     float* sQt = sKh + kChunk * kPitch;                // [64][129] scale * gamma * q
     float* sW = sQt + kChunk * kPitch;                 // [64][129] -W
     float* sP = sW + kChunk * kPitch;                  // [64][65]  scale * P
-    float* sdO = sP + kChunk * kPitchC;                // [64][33]
-    float* sdU = sdO + kChunk * kSP;                   // [64][33]
+    float* sdO = sP + kChunk * kPitchC;                // [64][65]
+    float* sdU = sdO + kChunk * kSP;                   // [64][65]
     float* sgC = sdU + kChunk * kSP;                   // [128] e^{Gamma_last}
     float* sgL = sgC + kHeadDim;                       // [128] Gamma_last
     int64_t b, e;
     seq_range(cu_seqlens, n, seqlen, total_tokens, &b, &e);
     const int64_t c_first = first_chunk_id(cu_seqlens, n, seqlen, total_tokens);
-    for (int x = tid; x < kHeadDim * kSlab; x += kB1Threads) {
-        const int c = x / kSlab, j = x % kSlab;
+    for (int x = tid; x < kHeadDim * kB1Slab; x += kB1Threads) {
+        const int c = x / kB1Slab, j = x % kB1Slab;
         sdS[c * kSP + j] = d_final ? d_final[(((int64_t)n * H + h) * kHeadDim + c) * kHeadDim + j0 + j] : 0.f;
     }
-    const int tx = tid % 8, ty = tid / 8;      // tile columns tx + 8 jj, rows ty + 32 ii
+    const int tx = tid % 16, ty = tid / 16;    // tile columns tx + 16 jj, rows ty + 32 ii
     const int64_t nch = (e - b + kChunk - 1) / kChunk;
     for (int64_t jc = nch - 1; jc >= 0; --jc) {
         const int64_t t0 = b + jc * kChunk, cid = c_first + jc;
@@ -103,11 +104,11 @@ __global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
             prefetch_rows_l2(q + nb, ldb * 2, kChunk, kHeadDim * 2, kB1Threads);
             prefetch_rows_l2(p + ((t0 - kChunk) * H + h) * kChunk, (int64_t)H * kChunk * 4, kChunk, kChunk * 4,
                              kB1Threads);
-            prefetch_rows_l2(d_out + nb + j0, ldb * 2, kChunk, kSlab * 2, kB1Threads);
+            prefetch_rows_l2(d_out + nb + j0, ldb * 2, kChunk, kB1Slab * 2, kB1Threads);
         }
         // dS' of this chunk
-        for (int x = tid; x < kHeadDim * kSlab; x += kB1Threads) {
-            const int c = x / kSlab, j = x % kSlab;
+        for (int x = tid; x < kHeadDim * kB1Slab; x += kB1Threads) {
+            const int c = x / kB1Slab, j = x % kB1Slab;
             dsn_out[((cid * H + h) * kHeadDim + c) * kHeadDim + j0 + j] = sdS[c * kSP + j];
         }
         const float* gl = gamma + ((t0 + len - 1) * H + h) * kHeadDim;
@@ -117,7 +118,7 @@ __global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
                                             [](int, int, float x) { return -x; });
         stage<kChunk, kChunk, kB1Threads>(sP, kPitchC, p + (t0 * H + h) * kChunk, (int64_t)H * kChunk, len,
                                           [scale](int, int, float x) { return scale * x; });
-        stage<kChunk, kSlab, kB1Threads>(sdO, kSP, d_out + base + j0, ld, len, Identity{});
+        stage<kChunk, kB1Slab, kB1Threads>(sdO, kSP, d_out + base + j0, ld, len, Identity{});
         __syncthreads();
         stage2<kChunk, kHeadDim, kB1Threads>(sKh, kPitch, gamma + base, k + base, ld, len,
                                              [sgL](int, int c, float G, float kv) { return kv * expf(sgL[c] - G); });
@@ -129,14 +130,14 @@ __global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
         {
             float acc[2][4];
             tile_zero(acc);
-            tile_fma<2, 4, 32, 8, 1, kPitchC, kSP, 1>(acc, sP, sdO, ty, tx, 0, len);
-            tile_fma<2, 4, 32, 8, kPitch, 1, kSP, 1>(acc, sKh, sdS, ty, tx, 0, kHeadDim);
+            tile_fma<2, 4, 32, 16, 1, kPitchC, kSP, 1>(acc, sP, sdO, ty, tx, 0, len);
+            tile_fma<2, 4, 32, 16, kPitch, 1, kSP, 1>(acc, sKh, sdS, ty, tx, 0, kHeadDim);
 #pragma unroll
             for (int ii = 0; ii < 2; ++ii) {
                 const int r = ty + 32 * ii;
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    const int j = tx + 8 * jj;
+                    const int j = tx + 16 * jj;
                     sdU[r * kSP + j] = acc[ii][jj];
                     if (r < len) du_out[((t0 + r) * H + h) * kHeadDim + j0 + j] = acc[ii][jj];
                 }
@@ -147,14 +148,14 @@ __global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
         {
             float acc[4][4];
             tile_zero(acc);
-            tile_fma<4, 4, 32, 8, 1, kPitch, kSP, 1>(acc, sQt, sdO, ty, tx, 0, len);
-            tile_fma<4, 4, 32, 8, 1, kPitch, kSP, 1>(acc, sW, sdU, ty, tx, 0, len);
+            tile_fma<4, 4, 32, 16, 1, kPitch, kSP, 1>(acc, sQt, sdO, ty, tx, 0, len);
+            tile_fma<4, 4, 32, 16, 1, kPitch, kSP, 1>(acc, sW, sdU, ty, tx, 0, len);
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii) {
                 const int c = ty + 32 * ii;
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    const int j = tx + 8 * jj;
+                    const int j = tx + 16 * jj;
                     sdS[c * kSP + j] = fmaf(sgC[c], sdS[c * kSP + j], acc[ii][jj]);
                 }
             }
@@ -162,8 +163,8 @@ __global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
     }
     __syncthreads();
     if (d_initial) {
-        for (int x = tid; x < kHeadDim * kSlab; x += kB1Threads) {
-            const int c = x / kSlab, j = x % kSlab;
+        for (int x = tid; x < kHeadDim * kB1Slab; x += kB1Threads) {
+            const int c = x / kB1Slab, j = x % kB1Slab;
             d_initial[(((int64_t)n * H + h) * kHeadDim + c) * kHeadDim + j0 + j] = sdS[c * kSP + j];
         }
     }
@@ -762,7 +763,7 @@ cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const Bw
     const auto* dO = static_cast<const __nv_bfloat16*>(d.d_out);
     const int H = a.H;
     if (a.N > 0) {
-        dim3 g1((unsigned)a.N, (unsigned)H, kHeadDim / bwd::kSlab);
+        dim3 g1((unsigned)a.N, (unsigned)H, kHeadDim / bwd::kB1Slab);
         bwd::state_bwd_kernel<<<g1, bwd::kB1Threads, bwd::kB1Smem, stream>>>(
             q, k, gamma, w, p, dO, d.d_final, a.cu_seqlens, a.seqlen, a.total_tokens, H, a.scale, L.max_chunks,
             dsn, du, d.d_initial);

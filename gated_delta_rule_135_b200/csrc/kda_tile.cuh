@@ -16,7 +16,7 @@ namespace kda {
 template <int TM, int TN, int RS, int CS, int AR, int AK, int BK, int BC>
 __device__ __forceinline__ void tile_fma(float (&acc)[TM][TN], const float* __restrict__ a,
                                          const float* __restrict__ b, int r0, int c0, int k0, int k1) {
-#pragma unroll 2
+#pragma unroll 4
     for (int k = k0; k < k1; ++k) {
         float av[TM], bv[TN];
 #pragma unroll
