@@ -43,6 +43,15 @@ NOMINAL_HBM_GBS = 8000.0             # the spec sheet's HBM3e figure, for contex
 NOMINAL_BF16_TFLOPS = 2250.0         # dense bf16 tensor peak, spec sheet, for context
 
 
+def workload(args) -> "W.Workload":
+    """The workload of --workload, with --heads applied (same sequences, seed and values)."""
+    import dataclasses
+    w = W.WORKLOADS[args.workload]
+    if args.heads:
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
+    return w
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -60,6 +69,8 @@ def parse():
                     help="time kda_decode (one token per sequence) instead of the prefill")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward kda_bwd (all gradients) instead of the forward")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the workload's head count (small cases for profiling)")
     ap.add_argument("--segments", type=int, default=0,
                     help="one-sequence workloads: run the forward as R segments per pass "
                          "(cp.segmented_prefill) instead of one kda_fwd call; -1 = cp.choose_segments")
@@ -283,7 +294,7 @@ def oracle_sample(w: W.Workload, x: dict, target_s: float, gdn: bool = False):
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
-    w = W.WORKLOADS[args.workload]
+    w = workload(args)
     x = W.make_inputs(w)
     import oracle
     # size each step's sample so the whole run stays within a few minutes
@@ -437,7 +448,7 @@ BWD_LAUNCHES_PER_STEP = 9         # staged forward 4 (no output kernel) + backwa
 def run_backward(args, world, rank, kda):
     """kda_bwd over the workload: every gradient (dq, dk, dv, dg, dbeta, dA_log, ddt_bias
     and the initial-state gradient when the workload has states) per step."""
-    w = W.WORKLOADS[args.workload]
+    w = workload(args)
     x = W.make_inputs(w)
     dO, dF = W.cotangents(w)
     if not w.final:
@@ -581,7 +592,7 @@ def main():
             dist.destroy_process_group()
         return rc
 
-    w = W.WORKLOADS[args.workload]
+    w = workload(args)
     x = W.make_inputs(w)
     if args.gdn:
         x = W.gdn_inputs(x)

@@ -256,12 +256,12 @@ __global__ void __launch_bounds__(kB2Threads) chunk_products_bwd_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// B3a: the T-side gradients of one chunk.  grid (max_chunks, H), 256 threads.
+// B3a: the T-side gradients of one chunk.  grid (max_chunks, H), 512 threads.
 // T = (I + A)^-1 comes from the forward (stored per chunk); with Xu = beta v, Xw = beta gamma k:
 //   dT = dU Xu^T + dW Xw^T,  dXu = T^T dU -> dv = beta dXu,  dXw = T^T dW -> dk = dXw beta gamma,
 //   dGamma = dXw beta gamma k,  dbeta = sum_j dXu v + sum_c dXw gamma k   (the T-side parts),
 //   dA = -T^T (dT T^T), strictly lower -> da_out [chunk][64][64].
-constexpr int kB3Threads = 256;
+constexpr int kB3Threads = 512;
 constexpr size_t kB3aSmem = sizeof(float) * (4 * kChunk * kPitch + 3 * kChunk * kPitchC + kChunk);
 
 __global__ void __launch_bounds__(kB3Threads) t_side_bwd_kernel(
@@ -295,26 +295,26 @@ __global__ void __launch_bounds__(kB3Threads) t_side_bwd_kernel(
     stage<kChunk, kHeadDim, kB3Threads>(sXu, kPitch, v + base, ld, len,
                                         [sb](int r, int, float x) { return sb[r] * x; });
     __syncthreads();
-    const int tx = tid % 16, ty = tid / 16;   // tiles: rows ty + 16 ii, columns tx + 16 jj
+    const int tx = tid % 16, ty = tid / 16;   // tiles: rows ty + 32 ii, columns tx + 16 jj
     {   // dT = dU Xu^T + dW Xw^T
-        float acc[4][4];
+        float acc[2][4];
         tile_zero(acc);
-        tile_fma<4, 4, 16, 16, kPitch, 1, 1, kPitch>(acc, sdU, sXu, ty, tx, 0, kHeadDim);
-        tile_fma<4, 4, 16, 16, kPitch, 1, 1, kPitch>(acc, sdW, sXw, ty, tx, 0, kHeadDim);
+        tile_fma<2, 4, 32, 16, kPitch, 1, 1, kPitch>(acc, sdU, sXu, ty, tx, 0, kHeadDim);
+        tile_fma<2, 4, 32, 16, kPitch, 1, 1, kPitch>(acc, sdW, sXw, ty, tx, 0, kHeadDim);
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
+        for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) sdT[(ty + 16 * ii) * kPitchC + tx + 16 * jj] = acc[ii][jj];
+            for (int jj = 0; jj < 4; ++jj) sdT[(ty + 32 * ii) * kPitchC + tx + 16 * jj] = acc[ii][jj];
     }
     {   // dXu = T^T dU, dXw = T^T dW and their epilogues
-        float au[4][8], aw[4][8];
+        float au[2][8], aw[2][8];
         tile_zero(au);
         tile_zero(aw);
-        tile_fma<4, 8, 16, 16, 1, kPitchC, kPitch, 1>(au, sT, sdU, ty, tx, 0, len);
-        tile_fma<4, 8, 16, 16, 1, kPitchC, kPitch, 1>(aw, sT, sdW, ty, tx, 0, len);
+        tile_fma<2, 8, 32, 16, 1, kPitchC, kPitch, 1>(au, sT, sdU, ty, tx, 0, len);
+        tile_fma<2, 8, 32, 16, 1, kPitchC, kPitch, 1>(aw, sT, sdW, ty, tx, 0, len);
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-            const int i = ty + 16 * ii;
+        for (int ii = 0; ii < 2; ++ii) {
+            const int i = ty + 32 * ii;
             float pb = 0.f;
             if (i < len) {
                 const float bi = sb[i];
@@ -338,23 +338,23 @@ __global__ void __launch_bounds__(kB3Threads) t_side_bwd_kernel(
     }
     __syncthreads();
     {   // Y = dT T^T
-        float acc[4][4];
+        float acc[2][4];
         tile_zero(acc);
-        tile_fma<4, 4, 16, 16, kPitchC, 1, 1, kPitchC>(acc, sdT, sT, ty, tx, 0, kChunk);
+        tile_fma<2, 4, 32, 16, kPitchC, 1, 1, kPitchC>(acc, sdT, sT, ty, tx, 0, kChunk);
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
+        for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) sY[(ty + 16 * ii) * kPitchC + tx + 16 * jj] = acc[ii][jj];
+            for (int jj = 0; jj < 4; ++jj) sY[(ty + 32 * ii) * kPitchC + tx + 16 * jj] = acc[ii][jj];
     }
     __syncthreads();
     {   // dA = -T^T Y, strictly lower
-        float acc[4][4];
+        float acc[2][4];
         tile_zero(acc);
-        tile_fma<4, 4, 16, 16, 1, kPitchC, kPitchC, 1>(acc, sT, sY, ty, tx, 0, kChunk);
+        tile_fma<2, 4, 32, 16, 1, kPitchC, kPitchC, 1>(acc, sT, sY, ty, tx, 0, kChunk);
         float* dst = da_out + ((int64_t)ci * H + h) * kChunk * kChunk;
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-            const int r = ty + 16 * ii;
+        for (int ii = 0; ii < 2; ++ii) {
+            const int r = ty + 32 * ii;
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
                 const int i = tx + 16 * jj;

@@ -100,8 +100,8 @@ __global__ void __launch_bounds__(128) gate_cumsum_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// (b) intra-chunk WY: A, P, T = (I + A)^-1, W, U~.  grid (max_chunks, H), 256 threads.
-constexpr int kIntraThreads = 256;
+// (b) intra-chunk WY: A, P, T = (I + A)^-1, W, U~.  grid (max_chunks, H), 512 threads.
+constexpr int kIntraThreads = 512;
 constexpr size_t kIntraSmem =
     sizeof(float) * (3 * kChunk * kPitch + 3 * kChunk * kPitchC + kChunk);
 
@@ -135,18 +135,20 @@ __global__ void __launch_bounds__(kIntraThreads) intra_chunk_kernel(
     __syncthreads();
 
     // A and P on 2 x 2 tiles of (r, i) pairs, tiles (tr, ti) with ti <= tr enumerated row-major:
-    // rows 2 tr + {0, 1}, columns 2 ti + {0, 1}; every decay formed pair by pair
+    // rows 2 tr + {0, 1}, columns 2 ti + {0, 1}; every decay formed pair by pair.  Thread t takes
+    // tile t over all channels; the tiles past the thread count go one per warp, its lanes
+    // splitting the channels (reduced by shuffles, in a fixed order).
     constexpr int kTiles = (kChunk / 2) * (kChunk / 2 + 1) / 2;
-    for (int p = tid; p < kTiles; p += kIntraThreads) {
-        int tr = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
+    static_assert(kTiles <= kIntraThreads + kIntraThreads / 32, "pair tiles exceed one round");
+    auto tile_coords = [](int p, int& tr, int& ti) {
+        tr = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
         while (tr * (tr + 1) / 2 > p) --tr;
         while ((tr + 1) * (tr + 2) / 2 <= p) ++tr;
-        const int ti = p - tr * (tr + 1) / 2;
-        const int r0 = 2 * tr, i0 = 2 * ti;
-        if (r0 >= len) continue;
-        float aa[2][2] = {}, ap[2][2] = {};
-        for (int cc = 0; cc < kHeadDim; ++cc) {
-            const int c = (cc + tid) & (kHeadDim - 1);
+        ti = p - tr * (tr + 1) / 2;
+    };
+    auto pair_sums = [&](int r0, int i0, int c_begin, int c_step, int n_c, float (&aa)[2][2], float (&ap)[2][2]) {
+        for (int m = 0; m < n_c; ++m) {
+            const int c = (c_begin + m * c_step) & (kHeadDim - 1);
             const float kr[2] = {sk[r0 * kPitch + c], sk[(r0 + 1) * kPitch + c]};
             const float qr[2] = {sq[r0 * kPitch + c], sq[(r0 + 1) * kPitch + c]};
             const float Gr[2] = {sG[r0 * kPitch + c], sG[(r0 + 1) * kPitch + c]};
@@ -163,6 +165,8 @@ __global__ void __launch_bounds__(kIntraThreads) intra_chunk_kernel(
                     ap[a][b2] = fmaf(qr[a], kd, ap[a][b2]);
                 }
         }
+    };
+    auto store_tile = [&](int r0, int i0, const float (&aa)[2][2], const float (&ap)[2][2]) {
 #pragma unroll
         for (int a = 0; a < 2; ++a)
 #pragma unroll
@@ -172,19 +176,68 @@ __global__ void __launch_bounds__(kIntraThreads) intra_chunk_kernel(
                 if (i < r) sA[r * kPitchC + i] = sb[r] * aa[a][b2];
                 sP[r * kPitchC + i] = ap[a][b2];
             }
+    };
+    if (tid < kTiles) {
+        int tr, ti;
+        tile_coords(tid, tr, ti);
+        if (2 * tr < len) {
+            float aa[2][2] = {}, ap[2][2] = {};
+            pair_sums(2 * tr, 2 * ti, tid, 1, kHeadDim, aa, ap);
+            store_tile(2 * tr, 2 * ti, aa, ap);
+        }
     }
-    __syncthreads();
-
-    // T = (I + A)^-1 by forward substitution, one column per thread
-    if (tid < kChunk) {
-        const int j = tid;
-        for (int r = j; r < kChunk; ++r) {
-            float s = (r == j) ? 1.f : 0.f;
-            for (int i = j; i < r; ++i) s = fmaf(-sA[r * kPitchC + i], sT[i * kPitchC + j], s);
-            sT[r * kPitchC + j] = s;
+    {
+        const int p = kIntraThreads + tid / 32, lane = tid % 32;
+        int tr = 0, ti = 0;
+        if (p < kTiles) tile_coords(p, tr, ti);
+        if (p < kTiles && 2 * tr < len) {           // uniform across the warp
+            float aa[2][2] = {}, ap[2][2] = {};
+            pair_sums(2 * tr, 2 * ti, lane, 32, kHeadDim / 32, aa, ap);
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int b2 = 0; b2 < 2; ++b2)
+                    for (int o = 16; o > 0; o >>= 1) {
+                        aa[a][b2] += __shfl_xor_sync(0xffffffffu, aa[a][b2], o);
+                        ap[a][b2] += __shfl_xor_sync(0xffffffffu, ap[a][b2], o);
+                    }
+            if (lane == 0) store_tile(2 * tr, 2 * ti, aa, ap);
         }
     }
     __syncthreads();
+
+    // T = (I + A)^-1 in 16 x 16 blocks.  Level 0: the diagonal blocks by forward substitution,
+    // one column per thread.  Level d = 1..3: blocks (j + d, j) as T_ij = -T_ii sum_{j<=m<i} A_im T_mj,
+    // the sum into scratch (sq: q is consumed) and then the product with T_ii.
+    if (tid < kChunk) {
+        const int o = tid & ~15, j = tid & 15;
+        for (int r = 0; r < 16; ++r) {
+            float acc = (r == j) ? 1.f : 0.f;
+            for (int i = j; i < r; ++i) acc = fmaf(-sA[(o + r) * kPitchC + o + i], sT[(o + i) * kPitchC + o + j], acc);
+            if (r >= j) sT[(o + r) * kPitchC + o + j] = acc;
+        }
+    }
+    __syncthreads();
+    float* scratch = sq;
+    for (int d = 1; d < 4; ++d) {
+        const int n = (4 - d) * 256;
+        for (int x = tid; x < n; x += kIntraThreads) {
+            const int bj = x / 256, bi = bj + d, r = (x / 16) % 16, cc = x % 16;
+            float acc = 0.f;
+            for (int m = 16 * bj; m < 16 * bi; ++m)
+                acc = fmaf(sA[(16 * bi + r) * kPitchC + m], sT[m * kPitchC + 16 * bj + cc], acc);
+            scratch[x] = acc;
+        }
+        __syncthreads();
+        for (int x = tid; x < n; x += kIntraThreads) {
+            const int bj = x / 256, bi = bj + d, r = (x / 16) % 16, cc = x % 16;
+            float acc = 0.f;
+            for (int m = 0; m <= r; ++m)
+                acc = fmaf(sT[(16 * bi + r) * kPitchC + 16 * bi + m], scratch[bj * 256 + m * 16 + cc], acc);
+            sT[(16 * bi + r) * kPitchC + 16 * bj + cc] = -acc;
+        }
+        __syncthreads();
+    }
     // sq <- beta * gamma * k ; sG <- beta * v   (Gamma is consumed first)
     for (int x = tid; x < kChunk * kHeadDim; x += kIntraThreads) {
         const int r = x / kHeadDim, c = x % kHeadDim;
@@ -193,17 +246,17 @@ __global__ void __launch_bounds__(kIntraThreads) intra_chunk_kernel(
     __syncthreads();
     stage<kChunk, kHeadDim, kIntraThreads>(sG, kPitch, v + base, ld, len, [sb](int r, int, float x) { return sb[r] * x; });
     __syncthreads();
-    // W = T (beta gamma K), U~ = T (beta V): 4 x 8 register tiles, rows ty + 16 ii, columns tx + 16 jj
+    // W = T (beta gamma K), U~ = T (beta V): 2 x 8 register tiles, rows ty + 32 ii, columns tx + 16 jj
     {
         const int tx = tid % 16, ty = tid / 16;
-        float aw[4][8], au[4][8];
+        float aw[2][8], au[2][8];
         tile_zero(aw);
         tile_zero(au);
-        tile_fma<4, 8, 16, 16, kPitchC, 1, kPitch, 1>(aw, sT, sq, ty, tx, 0, len);
-        tile_fma<4, 8, 16, 16, kPitchC, 1, kPitch, 1>(au, sT, sG, ty, tx, 0, len);
+        tile_fma<2, 8, 32, 16, kPitchC, 1, kPitch, 1>(aw, sT, sq, ty, tx, 0, len);
+        tile_fma<2, 8, 32, 16, kPitchC, 1, kPitch, 1>(au, sT, sG, ty, tx, 0, len);
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-            const int r = ty + 16 * ii;
+        for (int ii = 0; ii < 2; ++ii) {
+            const int r = ty + 32 * ii;
             if (r >= len) continue;
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) {
