@@ -49,6 +49,8 @@ def workload(args) -> "W.Workload":
     w = W.WORKLOADS[args.workload]
     if args.heads:
         w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
+    if args.lower_bound is not None:
+        w = dataclasses.replace(w, lower_bound=args.lower_bound, name=f"{w.name}_lb{args.lower_bound:g}")
     return w
 
 
@@ -69,6 +71,8 @@ def parse():
                     help="time kda_decode (one token per sequence) instead of the prefill")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward kda_bwd (all gradients) instead of the forward")
+    ap.add_argument("--lower-bound", type=float, default=None,
+                    help="override the workload's gate clamp (below -5.3 kda_fwd takes the staged kernels)")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the workload's head count (small cases for profiling)")
     ap.add_argument("--segments", type=int, default=0,
@@ -709,7 +713,7 @@ def main():
         line = {
             "metric": (("GDN (scalar-gate) prefill throughput (Mtokens/s) at T=8192 H=96 D=128 varlen"
                         if args.gdn else "KDA prefill throughput (Mtokens/s) at T=8192 H=96 D=128 varlen")
-                       if args.workload == 2 else
+                       if args.workload == 2 and not args.heads and args.lower_bound is None else
                        f"{'GDN (scalar-gate)' if args.gdn else 'KDA'} prefill throughput (Mtokens/s), {w.name}"),
             "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,

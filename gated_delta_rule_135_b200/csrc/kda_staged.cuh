@@ -408,8 +408,8 @@ __global__ void __launch_bounds__(kStateThreads) state_prop_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// (d) output: O = scale ((gamma * Q) S_c + P U), bf16.  grid (max_chunks, H), 256 threads.
-constexpr int kOutThreads = 256;
+// (d) output: O = scale ((gamma * Q) S_c + P U), bf16.  grid (max_chunks, H), 512 threads.
+constexpr int kOutThreads = 512;
 constexpr size_t kOutSmem =
     sizeof(float) * (kChunk * kPitch + kHeadDim * kPitch + kChunk * kPitchC + kChunk * kPitch);
 
@@ -427,32 +427,28 @@ __global__ void __launch_bounds__(kOutThreads) chunk_out_kernel(
     float* sS = sQ + kChunk * kPitch;        // [128][129]
     float* sP = sS + kHeadDim * kPitch;      // [64][65]
     float* sU = sP + kChunk * kPitchC;       // [64][129]
-    for (int x = tid; x < kChunk * kHeadDim; x += kOutThreads) {
-        const int r = x / kHeadDim, c = x % kHeadDim;
-        float qv = 0.f, uv = 0.f;
-        if (r < len) {
-            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c;
-            qv = bf16_to_f32(q[idx]) * expf(gamma[idx]);
-            uv = u[idx];
-        }
-        sQ[r * kPitch + c] = qv;
-        sU[r * kPitch + c] = uv;
-    }
-    for (int x = tid; x < kHeadDim * kHeadDim; x += kOutThreads) {
-        const int c = x / kHeadDim, j = x % kHeadDim;
-        sS[c * kPitch + j] = chunk_states[(((int64_t)ci * H + h) * kHeadDim + c) * kHeadDim + j];
-    }
-    for (int x = tid; x < kChunk * kChunk; x += kOutThreads) {
-        const int r = x / kChunk, i = x % kChunk;
-        sP[r * kPitchC + i] = r < len ? p[(((int64_t)e.y + r) * H + h) * kChunk + i] : 0.f;
-    }
+    const int64_t base = ((int64_t)e.y * H + h) * kHeadDim, ld = (int64_t)H * kHeadDim;
+    stage<kHeadDim, kHeadDim, kOutThreads>(sS, kPitch, chunk_states + ((int64_t)ci * H + h) * kHeadDim * kHeadDim,
+                                           kHeadDim, kHeadDim, Identity{});
+    stage2<kChunk, kHeadDim, kOutThreads>(sQ, kPitch, gamma + base, q + base, ld, len,
+                                          [](int, int, float G, float qv) { return qv * expf(G); });
+    stage<kChunk, kHeadDim, kOutThreads>(sU, kPitch, u + base, ld, len, Identity{});
+    stage<kChunk, kChunk, kOutThreads>(sP, kPitchC, p + ((int64_t)e.y * H + h) * kChunk, (int64_t)H * kChunk, len,
+                                       Identity{});
     __syncthreads();
-    const int j = tid % kHeadDim;
-    for (int r = tid / kHeadDim; r < len; r += kOutThreads / kHeadDim) {
-        float acc = 0.f;
-        for (int c = 0; c < kHeadDim; ++c) acc = fmaf(sQ[r * kPitch + c], sS[c * kPitch + j], acc);
-        for (int i = 0; i <= r; ++i) acc = fmaf(sP[r * kPitchC + i], sU[i * kPitch + j], acc);
-        out[(((int64_t)e.y + r) * H + h) * kHeadDim + j] = __float2bfloat16_rn(scale * acc);
+    // 2 x 8 register tiles: rows ty + 32 ii, columns tx + 16 jj
+    const int tx = tid % 16, ty = tid / 16;
+    float acc[2][8];
+    tile_zero(acc);
+    tile_fma<2, 8, 32, 16, kPitch, 1, kPitch, 1>(acc, sQ, sS, ty, tx, 0, kHeadDim);
+    tile_fma<2, 8, 32, 16, kPitchC, 1, kPitch, 1>(acc, sP, sU, ty, tx, 0, len);
+#pragma unroll
+    for (int ii = 0; ii < 2; ++ii) {
+        const int r = ty + 32 * ii;
+        if (r >= len) continue;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+            out[base + (int64_t)r * ld + tx + 16 * jj] = __float2bfloat16_rn(scale * acc[ii][jj]);
     }
 }
 
