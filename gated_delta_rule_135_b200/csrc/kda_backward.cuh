@@ -26,31 +26,8 @@ namespace bwd {
 
 constexpr int kPitch = kHeadDim + 1;
 constexpr int kPitchC = kChunk + 1;
-constexpr int kSlab = 32;
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162float(x); }
-
-// global chunk id of sequence n's first chunk (one block; sums the earlier sequences)
-__device__ int64_t first_chunk_id(const int32_t* cu_seqlens, int n, int64_t seqlen, int64_t total_tokens) {
-    __shared__ int64_t warp_part[32];
-    __shared__ int64_t result;
-    int64_t part = 0;
-    for (int m = threadIdx.x; m < n; m += blockDim.x) {
-        int64_t mb, me;
-        seq_range(cu_seqlens, m, seqlen, total_tokens, &mb, &me);
-        part += (me - mb + kChunk - 1) / kChunk;
-    }
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if ((threadIdx.x & 31) == 0) warp_part[threadIdx.x >> 5] = part;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int64_t s = 0;
-        for (int x = 0; x < (int)(blockDim.x >> 5); ++x) s += warp_part[x];
-        result = s;
-    }
-    __syncthreads();
-    return result;
-}
 
 // ---------------------------------------------------------------------------
 // B1: dS backwards over a sequence's chunks; per chunk stores dS' (the gradient of the
@@ -386,7 +363,7 @@ __global__ void __launch_bounds__(kB3Threads) t_side_bwd_kernel(
 // The operands k e^{G_s - G} and k, q e^{G - G_s} take s as the row's own block start.
 constexpr int kB3bThreads = 512;
 constexpr size_t kB3bSmem = sizeof(float) * (5 * kChunk * kPitch + 2 * kChunk * kPitchC + kChunk + 2 * kHeadDim +
-                                             kChunk * 4 + 4);
+                                             kChunk * 4);
 
 template <bool kFactored>
 __global__ void __launch_bounds__(kB3bThreads) decay_bwd_kernel(
@@ -414,8 +391,7 @@ __global__ void __launch_bounds__(kB3bThreads) decay_bwd_kernel(
     float* sb = sdA + kChunk * kPitchC;      // [64]
     float* sgC = sb + kChunk;                // [128] Gamma of the last row
     float* sbp = sgC + kHeadDim;             // [64][4] dbeta partials (one per warp of a row)
-    float* sred = sbp + kChunk * 4;          // [4]
-    float* sdb = sred + 4;                   // [128] dt_bias of the head
+    float* sdb = sbp + kChunk * 4;           // [128] dt_bias of the head
     const float nexp = -expf(A_log[h]);
     // phase 1: dP, dA, beta, a, Gamma_last
     if (tid < kChunk) sb[tid] = tid < len ? beta[((int64_t)e.y + tid) * H + h] : 0.f;

@@ -300,29 +300,10 @@ __global__ void __launch_bounds__(kStateThreads) state_prop_kernel(
     float* sU = sK + kChunk * kPitch;                // [64][33]
     float* sgC = sU + kChunk * (kSlab + 1);          // [128] e^{Gamma_last}
     float* sgL = sgC + kHeadDim;                     // [128] Gamma_last
-    __shared__ int64_t s_first_chunk;
 
     int64_t b, e;
     seq_range(cu_seqlens, n, seqlen, total_tokens, &b, &e);
-    // global chunk id of this sequence's first chunk: sum over earlier sequences
-    {
-        int64_t part = 0;
-        for (int m = tid; m < n; m += kStateThreads) {
-            int64_t mb, me;
-            seq_range(cu_seqlens, m, seqlen, total_tokens, &mb, &me);
-            part += (me - mb + kChunk - 1) / kChunk;
-        }
-        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        __shared__ int64_t warp_part[kStateThreads / 32];
-        if ((tid & 31) == 0) warp_part[tid >> 5] = part;
-        __syncthreads();
-        if (tid == 0) {
-            int64_t s = 0;
-            for (int x = 0; x < kStateThreads / 32; ++x) s += warp_part[x];
-            s_first_chunk = s;
-        }
-        __syncthreads();
-    }
+    const int64_t s_first_chunk = first_chunk_id(cu_seqlens, n, seqlen, total_tokens);
     for (int x = tid; x < kHeadDim * kSlab; x += kStateThreads) {
         const int c = x / kSlab, j = x % kSlab;
         sS[c * (kSlab + 1) + j] = initial_state
