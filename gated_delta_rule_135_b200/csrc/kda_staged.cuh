@@ -278,9 +278,9 @@ __global__ void __launch_bounds__(kIntraThreads) intra_chunk_kernel(
 
 // ---------------------------------------------------------------------------
 // (c) inter-chunk state propagation, serial over a sequence's chunks.
-// grid (N, H, 128 / kSlab), 256 threads; each block owns a 128 x kSlab column slab of S.
-constexpr int kSlab = 32;
-constexpr int kStateThreads = 256;
+// grid (N, H, 128 / kSlab), 512 threads; each block owns a 128 x kSlab column slab of S.
+constexpr int kSlab = 64;
+constexpr int kStateThreads = 512;
 constexpr size_t kStateSmem =
     sizeof(float) * (kHeadDim * (kSlab + 1) + 2 * kChunk * kPitch + kChunk * (kSlab + 1) + 2 * kHeadDim);
 
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(kStateThreads) state_prop_kernel(
     }
     __syncthreads();
     int64_t chunk_id = s_first_chunk;
-    const int tx = tid % 8, ty = tid / 8;   // register tiles: columns tx + 8 jj, rows ty + 32 ii
+    const int tx = tid % 16, ty = tid / 16;   // register tiles: columns tx + 16 jj, rows ty + 32 ii
     for (int64_t t0 = b; t0 < e; t0 += kChunk, ++chunk_id) {
         const int len = (int)(e - t0 < kChunk ? e - t0 : kChunk);
         __syncthreads();   // the previous chunk's state update is complete
@@ -348,14 +348,14 @@ __global__ void __launch_bounds__(kStateThreads) state_prop_kernel(
 #pragma unroll
             for (int ii = 0; ii < 2; ++ii)
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) acc[ii][jj] = sU[(ty + 32 * ii) * (kSlab + 1) + tx + 8 * jj];
-            tile_fma<2, 4, 32, 8, kPitch, 1, kSlab + 1, 1>(acc, sW, sS, ty, tx, 0, kHeadDim);
+                for (int jj = 0; jj < 4; ++jj) acc[ii][jj] = sU[(ty + 32 * ii) * (kSlab + 1) + tx + 16 * jj];
+            tile_fma<2, 4, 32, 16, kPitch, 1, kSlab + 1, 1>(acc, sW, sS, ty, tx, 0, kHeadDim);
 #pragma unroll
             for (int ii = 0; ii < 2; ++ii) {
                 const int r = ty + 32 * ii;
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    const int j = tx + 8 * jj;
+                    const int j = tx + 16 * jj;
                     sU[r * (kSlab + 1) + j] = acc[ii][jj];
                     if (r < len) u_out[((t0 + r) * H + h) * kHeadDim + j0 + j] = acc[ii][jj];
                 }
@@ -366,13 +366,13 @@ __global__ void __launch_bounds__(kStateThreads) state_prop_kernel(
         {
             float acc[4][4];
             tile_zero(acc);
-            tile_fma<4, 4, 32, 8, 1, kPitch, kSlab + 1, 1>(acc, sK, sU, ty, tx, 0, len);
+            tile_fma<4, 4, 32, 16, 1, kPitch, kSlab + 1, 1>(acc, sK, sU, ty, tx, 0, len);
 #pragma unroll
             for (int ii = 0; ii < 4; ++ii) {
                 const int c = ty + 32 * ii;
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
-                    const int j = tx + 8 * jj;
+                    const int j = tx + 16 * jj;
                     sS[c * (kSlab + 1) + j] = fmaf(sgC[c], sS[c * (kSlab + 1) + j], acc[ii][jj]);
                 }
             }
