@@ -1,8 +1,9 @@
 // kda_backward.cuh -- the KDA backward: gradients of L = <dO, out> + <dS_final, final_state>
 // with respect to q, k, v, g, beta, A_log, dt_bias and the initial state.
 //
-// Staged, fp32 on CUDA cores, on top of the staged forward's workspace (Gamma, W, U~, P, U
-// and the state at every chunk start).  Per chunk (restated from the chain rule through
+// Staged through HBM on top of the staged forward's workspace (Gamma, W, U~, P, U, T and the
+// state at every chunk start): fp32 CUDA-core products, except the three state products of B2,
+// which run on the tensor cores with split-bf16 operands and fp32 accumulation.  Per chunk (restated from the chain rule through
 // the forward's chunk algebra; the oracle's chunk_step_bwd follows the same steps):
 //   from S' = Diag(gC) S + Khat^T U:   dS = Diag(gC) dS',  dgC = rowsum(S * dS'),
 //                                      dKhat = U dS'^T,     dU = Khat dS'
@@ -20,6 +21,7 @@
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_tile.cuh"
+#include "umma.cuh"
 
 namespace kda {
 namespace bwd {
@@ -148,88 +150,208 @@ __global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// B2: per chunk and 32-channel tile: dKhat = U dS'^T, d(gamma q) = scale dO S^T,
-// dW = -dU S^T (rows r, channels c of the tile) and dgC_c = sum_j S_cj dS'_cj.
-// grid (max_chunks, H, 128 / 32), 256 threads.  The sum over j runs in two halves of 64,
-// so that the staged operands take 66.5 KB and three blocks share an SM.
-constexpr int kB2Threads = 256;
-constexpr int kCT = 32;
-constexpr int kJH = 64;                 // j columns staged at a time
-constexpr int kPH = kJH + 1;
-constexpr size_t kB2Smem = sizeof(float) * (2 * kCT * kPH + 3 * kChunk * kPH);
+// B2 (tensor cores): per chunk and head (one CTA; two share an SM)
+//   D1 = S [dO ; dU]^T   (M = 128 state rows c, N = 128: the chunk's dO rows, then its dU rows)
+//   D2 = dS' U^T         (M = 128, N = 64)
+// i.e. the transposes of d(gamma q) / scale, -dW and dKhat, summed over j in two halves of 64.
+// fp32 operands enter as bf16 high and low parts (x = hi + lo, |lo| <= 2^-9 |x|) and every
+// product as hi.hi + hi.lo + lo.hi with fp32 accumulation in TMEM: about 16 mantissa bits.
+// dO is bf16 already (its low part is 0).  Lane c of the accumulators is state row c, so each
+// warp stores 32 consecutive channels of a token row.  dgC = rowsum(S * dS') on the CUDA cores
+// from the fp32 values being staged.
+namespace tc {
+using namespace umma;
+constexpr uint32_t S_HI = 0, S_LO = 16384, N_HI = 32768, N_LO = 49152, B_HI = 65536, B_LO = 81920,
+                   U_HI = 98304, U_LO = 106496, BAR = 114688, TSLOT = BAR + 8, ABORT = BAR + 12;
+constexpr uint32_t BYTES = BAR + 16;
+constexpr uint32_t ALLOC = BYTES + 1008;   // + alignment slack (the dynamic base is 16-byte aligned)
+constexpr uint32_t TM_COLS = 256;          // D1 in columns 0-127, D2 in 128-191
+constexpr uint32_t IDESC_N128 = idesc_f16(128, 128, true, false, false);
+constexpr uint32_t IDESC_N64 = idesc_f16(128, 64, true, false, false);
+constexpr int kThreads = 256;
 
-__global__ void __launch_bounds__(kB2Threads) chunk_products_bwd_kernel(
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * i]), h1 = __float2bfloat16_rn(x[2 * i + 1]);
+        const __nv_bfloat16 l0 = __float2bfloat16_rn(x[2 * i] - __bfloat162float(h0));
+        const __nv_bfloat16 l1 = __float2bfloat16_rn(x[2 * i + 1] - __bfloat162float(h1));
+        h[i] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+        l[i] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__device__ __forceinline__ void load8(const float* src, float (&x)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+}  // namespace tc
+
+__global__ void __launch_bounds__(tc::kThreads, 2) chunk_products_tc_kernel(
     const float* __restrict__ u, const float* __restrict__ du, const __nv_bfloat16* __restrict__ d_out,
     const float* __restrict__ chunk_states, const float* __restrict__ dsn, const int4* __restrict__ table,
     const int32_t* __restrict__ count, int H, float scale, float* __restrict__ dkhat, float* __restrict__ dqg,
     float* __restrict__ dw, float* __restrict__ dgc) {
+    using namespace tc;
     const int ci = blockIdx.x;
-    if (ci >= *count) return;
+    if (ci >= *count) return;                  // before any TMEM is taken
     const int4 e = table[ci];
-    const int h = blockIdx.y, c0 = blockIdx.z * kCT, tid = threadIdx.x, len = e.z;
-    extern __shared__ float sm[];
-    float* sS = sm;                        // [32 c][65 j] S rows of the tile
-    float* sN = sS + kCT * kPH;            // [32 c][65 j] dS' rows of the tile
-    float* sU = sN + kCT * kPH;            // [64][65] U
-    float* sO = sU + kChunk * kPH;         // [64][65] dO
-    float* sD = sO + kChunk * kPH;         // [64][65] dU
-    const int64_t sbase = ((int64_t)ci * H + h) * kHeadDim * kHeadDim + (int64_t)c0 * kHeadDim;
+    const int h = blockIdx.y, tid = threadIdx.x, warp = tid / 32, lane = tid % 32, len = e.z;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);
+    uint32_t* slot = reinterpret_cast<uint32_t*>(sm + TSLOT);
+    volatile uint32_t* sAbort = reinterpret_cast<volatile uint32_t*>(sm + ABORT);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init_fence();
+        *sAbort = 0u;
+    }
+    if (warp == 0) {
+        tmem_alloc(slot, TM_COLS);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *slot;
+    const int64_t sbase = ((int64_t)ci * H + h) * kHeadDim * kHeadDim;
     const int64_t base = ((int64_t)e.y * H + h) * kHeadDim, ld = (int64_t)H * kHeadDim;
-    const int tx = tid % 8, ty = tid / 8;  // 2 x 4 tiles: rows ty + 32 ii, channels tx + 8 jj
-    float a1[2][4], a2[2][4], a3[2][4];
-    tile_zero(a1);
-    tile_zero(a2);
-    tile_zero(a3);
-    float gsum = 0.f;
-    for (int jh = 0; jh < kHeadDim; jh += kJH) {
-        if (jh) __syncthreads();           // the previous half is consumed
-        stage<kCT, kJH, kB2Threads>(sS, kPH, chunk_states + sbase + jh, kHeadDim, kCT, Identity{});
-        stage<kCT, kJH, kB2Threads>(sN, kPH, dsn + sbase + jh, kHeadDim, kCT, Identity{});
-        stage<kChunk, kJH, kB2Threads>(sU, kPH, u + base + jh, ld, len, Identity{});
-        stage<kChunk, kJH, kB2Threads>(sO, kPH, d_out + base + jh, ld, len, Identity{});
-        stage<kChunk, kJH, kB2Threads>(sD, kPH, du + base + jh, ld, len, Identity{});
+    float gpart[4] = {0.f, 0.f, 0.f, 0.f};     // dgC partials of this thread's state rows
+    bool aborted = false;
+    uint32_t failed_parity = 0u;
+    for (int hj = 0; hj < 2 && !aborted; ++hj) {
+        failed_parity = (uint32_t)hj;
+        const int col0 = hj * 64;
+        // S and dS' (128 rows each), with the dgC partial sums
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int x = tid + kThreads * m, c = x >> 3, ch = x & 7;
+            float a[8], b[8];
+            load8(chunk_states + sbase + (int64_t)c * kHeadDim + col0 + 8 * ch, a);
+            load8(dsn + sbase + (int64_t)c * kHeadDim + col0 + 8 * ch, b);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) gpart[m] = fmaf(a[i], b[i], gpart[m]);
+            uint4 hi, lo;
+            split8(a, hi, lo);
+            *reinterpret_cast<uint4*>(sm + S_HI + sw128_chunk_off(c, ch, 128)) = hi;
+            *reinterpret_cast<uint4*>(sm + S_LO + sw128_chunk_off(c, ch, 128)) = lo;
+            split8(b, hi, lo);
+            *reinterpret_cast<uint4*>(sm + N_HI + sw128_chunk_off(c, ch, 128)) = hi;
+            *reinterpret_cast<uint4*>(sm + N_LO + sw128_chunk_off(c, ch, 128)) = lo;
+        }
+        // [dO ; dU] (rows r < 64: dO, r >= 64: dU of token r - 64) and U, zero past the chunk
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int x = tid + kThreads * m, r = x >> 3, ch = x & 7;
+            uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = make_uint4(0u, 0u, 0u, 0u);
+            if (r < 64) {
+                if (r < len) hi = *reinterpret_cast<const uint4*>(d_out + base + (int64_t)r * ld + col0 + 8 * ch);
+            } else if (r - 64 < len) {
+                float a[8];
+                load8(du + base + (int64_t)(r - 64) * ld + col0 + 8 * ch, a);
+                split8(a, hi, lo);
+            }
+            *reinterpret_cast<uint4*>(sm + B_HI + sw128_chunk_off(r, ch, 128)) = hi;
+            *reinterpret_cast<uint4*>(sm + B_LO + sw128_chunk_off(r, ch, 128)) = lo;
+        }
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const int x = tid + kThreads * m, r = x >> 3, ch = x & 7;
+            uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = make_uint4(0u, 0u, 0u, 0u);
+            if (r < len) {
+                float a[8];
+                load8(u + base + (int64_t)r * ld + col0 + 8 * ch, a);
+                split8(a, hi, lo);
+            }
+            *reinterpret_cast<uint4*>(sm + U_HI + sw128_chunk_off(r, ch, 64)) = hi;
+            *reinterpret_cast<uint4*>(sm + U_LO + sw128_chunk_off(r, ch, 64)) = lo;
+        }
+        fence_proxy_async();
+        fence_before_sync();
         __syncthreads();
-#pragma unroll 2
-        for (int j = 0; j < kJH; ++j) {
-            float u0[2], o0[2], d0[2], nv[4], sv[4];
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t s_hi = smem_u32(sm + S_HI), s_lo = smem_u32(sm + S_LO), n_hi = smem_u32(sm + N_HI),
+                           n_lo = smem_u32(sm + N_LO), b_hi = smem_u32(sm + B_HI), b_lo = smem_u32(sm + B_LO),
+                           u_hi = smem_u32(sm + U_HI), u_lo = smem_u32(sm + U_LO);
 #pragma unroll
-            for (int ii = 0; ii < 2; ++ii) {
-                const int r = ty + 32 * ii;
-                u0[ii] = sU[r * kPH + j];
-                o0[ii] = sO[r * kPH + j];
-                d0[ii] = sD[r * kPH + j];
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint32_t acc = (hj > 0 || ks > 0) ? 1u : 0u;
+                mma_f16(tbase, desc_kmajor(s_hi, 128, ks), desc_kmajor(b_hi, 128, ks), IDESC_N128, acc);
+                mma_f16(tbase, desc_kmajor(s_hi, 128, ks), desc_kmajor(b_lo, 128, ks), IDESC_N128, 1u);
+                mma_f16(tbase, desc_kmajor(s_lo, 128, ks), desc_kmajor(b_hi, 128, ks), IDESC_N128, 1u);
+                mma_f16(tbase + 128, desc_kmajor(n_hi, 128, ks), desc_kmajor(u_hi, 64, ks), IDESC_N64, acc);
+                mma_f16(tbase + 128, desc_kmajor(n_hi, 128, ks), desc_kmajor(u_lo, 64, ks), IDESC_N64, 1u);
+                mma_f16(tbase + 128, desc_kmajor(n_lo, 128, ks), desc_kmajor(u_hi, 64, ks), IDESC_N64, 1u);
             }
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int c = tx + 8 * jj;
-                nv[jj] = sN[c * kPH + j];
-                sv[jj] = sS[c * kPH + j];
+            mma_commit(bar);
+            // one thread polls (bounded); the block barrier below orders the completion for all
+            if (!mbar_wait_bounded(bar, (uint32_t)hj)) {
+                record_error(KDA_DEVERR_TIMEOUT);
+                *sAbort = 1u;
             }
+        }
+        __syncthreads();
+        fence_after_sync();
+        aborted = *sAbort != 0u;
+    }
+    if (aborted) {
+        // the MMAs may still be reading shared memory and writing TMEM: give them (bounded)
+        // time before the columns are released
+        if (tid == 0) mbar_wait_bounded(bar, failed_parity);
+        fence_before_sync();
+        __syncthreads();
+    } else {
+        // dgC: the 8 lanes holding one state row's chunks sum their partials
 #pragma unroll
-            for (int ii = 0; ii < 2; ++ii)
+        for (int m = 0; m < 4; ++m) {
+            float v = gpart[m];
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            const int x = tid + kThreads * m;
+            if ((x & 7) == 0) dgc[((int64_t)ci * H + h) * kHeadDim + (x >> 3)] = v;
+        }
+        const int q = warp & 3, c = q * 32 + lane;
+        if (warp < 4) {        // D1: columns 0-63 are d(gamma q) / scale, 64-127 are -dW
+#pragma unroll 1
+            for (int cb = 0; cb < 8; ++cb) {
+                uint32_t v[16];
+                tmem_ld16(taddr(tbase, q, 16 * cb), v);
+                tmem_wait_ld();
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    a1[ii][jj] = fmaf(u0[ii], nv[jj], a1[ii][jj]);
-                    a2[ii][jj] = fmaf(o0[ii], sv[jj], a2[ii][jj]);
-                    a3[ii][jj] = fmaf(d0[ii], sv[jj], a3[ii][jj]);
+                for (int i = 0; i < 16; ++i) {
+                    const int col = 16 * cb + i, r = col & 63;
+                    if (r >= len) continue;
+                    const int64_t idx = base + (int64_t)r * ld + c;
+                    if (col < 64) dqg[idx] = scale * __uint_as_float(v[i]);
+                    else dw[idx] = -__uint_as_float(v[i]);
                 }
-        }
-        if (tid < kCT)
-            for (int j = 0; j < kJH; ++j) gsum = fmaf(sS[tid * kPH + j], sN[tid * kPH + j], gsum);
-    }
+            }
+        } else {               // D2: columns 128-191 are dKhat
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t v[16];
+                tmem_ld16(taddr(tbase, q, 128 + 16 * cb), v);
+                tmem_wait_ld();
 #pragma unroll
-    for (int ii = 0; ii < 2; ++ii) {
-        const int r = ty + 32 * ii;
-        if (r >= len) continue;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const int64_t idx = (((int64_t)e.y + r) * H + h) * kHeadDim + c0 + tx + 8 * jj;
-            dkhat[idx] = a1[ii][jj];
-            dqg[idx] = scale * a2[ii][jj];
-            dw[idx] = -a3[ii][jj];
+                for (int i = 0; i < 16; ++i) {
+                    const int r = 16 * cb + i;
+                    if (r < len) dkhat[base + (int64_t)r * ld + c] = __uint_as_float(v[i]);
+                }
+            }
         }
+        fence_before_sync();
+        __syncthreads();
     }
-    if (tid < kCT) dgc[((int64_t)ci * H + h) * kHeadDim + c0 + tid] = gsum;
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tbase, TM_COLS);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -696,8 +818,8 @@ cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const Bw
         cudaError_t err;
         if ((err = cudaFuncSetAttribute(bwd::state_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)bwd::kB1Smem)) != cudaSuccess) return err;
-        if ((err = cudaFuncSetAttribute(bwd::chunk_products_bwd_kernel,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd::kB2Smem)) !=
+        if ((err = cudaFuncSetAttribute(bwd::chunk_products_tc_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd::tc::ALLOC)) !=
             cudaSuccess) return err;
         if ((err = cudaFuncSetAttribute(bwd::t_side_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)bwd::kB3aSmem)) != cudaSuccess) return err;
@@ -745,10 +867,9 @@ cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const Bw
             dsn, du, d.d_initial);
     }
     if (L.max_chunks > 0) {
-        dim3 g2((unsigned)L.max_chunks, (unsigned)H, kHeadDim / bwd::kCT);
-        bwd::chunk_products_bwd_kernel<<<g2, bwd::kB2Threads, bwd::kB2Smem, stream>>>(
-            u, du, dO, cs, dsn, table, count, H, a.scale, dkhat, dqg, dw, dgc);
         dim3 g3((unsigned)L.max_chunks, (unsigned)H);
+        bwd::chunk_products_tc_kernel<<<g3, bwd::tc::kThreads, bwd::tc::ALLOC, stream>>>(
+            u, du, dO, cs, dsn, table, count, H, a.scale, dkhat, dqg, dw, dgc);
         bwd::t_side_bwd_kernel<<<g3, bwd::kB3Threads, bwd::kB3aSmem, stream>>>(
             k, v, a.beta, gamma, tm, du, dw, table, count, H, d.dk, d.dv, dG, d.dbeta, da);
         auto decay = fused_supported(a.lower_bound) ? bwd::decay_bwd_kernel<true> : bwd::decay_bwd_kernel<false>;
