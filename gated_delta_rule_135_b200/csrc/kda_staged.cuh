@@ -2,7 +2,9 @@
 //
 // fp32 CUDA-core arithmetic, every intra-chunk decay exp(Gamma_r - Gamma_i)
 // formed pair by pair (never as a product of two exponentials), so the path
-// is exact for any gate, including an unclamped one.  It is the fallback of
+// is exact for any gate, including an unclamped one.  The state propagation
+// runs on the tensor cores with split-bf16 operands (about 16 mantissa bits
+// per product) and the state in fp32 TMEM.  It is the fallback of
 // kda_fwd for gates too steep for the fused kernel's factored decays, and its
 // workspace exposes every stage's output for checking.
 //
@@ -17,6 +19,7 @@
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_tile.cuh"
+#include "umma.cuh"
 
 namespace kda {
 
@@ -277,114 +280,242 @@ __global__ void __launch_bounds__(kIntraThreads) intra_chunk_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// (c) inter-chunk state propagation, serial over a sequence's chunks.
-// grid (N, H, 128 / kSlab), 512 threads; each block owns a 128 x kSlab column slab of S.
-constexpr int kSlab = 64;
-constexpr int kStateThreads = 512;
-constexpr size_t kStateSmem =
-    sizeof(float) * (kHeadDim * (kSlab + 1) + 2 * kChunk * kPitch + kChunk * (kSlab + 1) + 2 * kHeadDim);
+// (c) inter-chunk state propagation on the tensor cores, serial over a sequence's chunks.  grid (N, H), 256 threads, one sequence and
+// head per CTA with the fp32 state transposed in TMEM (lane j = state column, column c = state
+// row).  Per chunk:
+//   1. one pass over the TMEM state writes the chunk-start state, writes its split-bf16 copy
+//      (the MN-major A operand S^T) and scales the TMEM state by gamma_C;
+//   2. U^T = U~^T - S^T W^T         (M = 128 state columns j, N = 64 tokens, K = 128 rows c);
+//   3. U = U~ + (that product) is written out and staged split-bf16 as the A operand U^T;
+//   4. S^T += U^T Khat              (M = 128, N = 128 state rows c, K = 64 tokens).
+// Operands are bf16 high and low parts of the fp32 values (hi.hi + hi.lo + lo.hi, fp32
+// accumulation): about 16 mantissa bits per product, the state itself kept in fp32.
+namespace stc {
+using namespace umma;
+constexpr uint32_t SH = 0, SL = 32768, WH = 65536, WL = 81920, UH = 98304, UL = 114688, KH = 131072,
+                   KL = 147456, GC = 163840, BAR = GC + 512, TSLOT = BAR + 8, ABORT = BAR + 12;
+constexpr uint32_t BYTES = BAR + 16;
+constexpr uint32_t ALLOC = BYTES + 1008;
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_COLS = 256;
+constexpr uint32_t IDESC_U = idesc_f16(128, 64, true, true, false);
+constexpr uint32_t IDESC_S = idesc_f16(128, 128, true, true, true);
+constexpr int kThreads = 256;
 
-__global__ void __launch_bounds__(kStateThreads) state_prop_kernel(
+__device__ __forceinline__ void split1(float x, uint16_t& hi, uint16_t& lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    hi = __bfloat16_as_ushort(h);
+    lo = __bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(h)));
+}
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+    uint16_t h[8], l[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) split1(x[i], h[i], l[i]);
+    hi = make_uint4(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16), h[4] | ((uint32_t)h[5] << 16),
+                    h[6] | ((uint32_t)h[7] << 16));
+    lo = make_uint4(l[0] | ((uint32_t)l[1] << 16), l[2] | ((uint32_t)l[3] << 16), l[4] | ((uint32_t)l[5] << 16),
+                    l[6] | ((uint32_t)l[7] << 16));
+}
+}  // namespace stc
+
+__global__ void __launch_bounds__(stc::kThreads, 1) state_prop_tc_kernel(
     const __nv_bfloat16* __restrict__ k, const float* __restrict__ gamma,
     const float* __restrict__ w, const float* __restrict__ ut,
     const float* __restrict__ initial_state, const int32_t* __restrict__ cu_seqlens,
     int64_t seqlen, int64_t total_tokens, int H,
     float* __restrict__ u_out, float* __restrict__ chunk_states, int64_t max_chunks,
     float* __restrict__ final_state) {
-    const int n = blockIdx.x, h = blockIdx.y, slab = blockIdx.z, tid = threadIdx.x;
-    const int j0 = slab * kSlab;
-    extern __shared__ float sm[];
-    float* sS = sm;                                  // [128][33]
-    float* sW = sS + kHeadDim * (kSlab + 1);         // [64][129] W, later Khat
-    float* sK = sW + kChunk * kPitch;                // [64][129] k -> Khat
-    float* sU = sK + kChunk * kPitch;                // [64][33]
-    float* sgC = sU + kChunk * (kSlab + 1);          // [128] e^{Gamma_last}
-    float* sgL = sgC + kHeadDim;                     // [128] Gamma_last
-
+    using namespace stc;
+    const int n = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);
+    uint32_t* slot = reinterpret_cast<uint32_t*>(sm + TSLOT);
+    volatile uint32_t* sAbort = reinterpret_cast<volatile uint32_t*>(sm + ABORT);
+    float* sGC = reinterpret_cast<float*>(sm + GC);            // [128] e^{Gamma_last}
     int64_t b, e;
     seq_range(cu_seqlens, n, seqlen, total_tokens, &b, &e);
-    const int64_t s_first_chunk = first_chunk_id(cu_seqlens, n, seqlen, total_tokens);
-    for (int x = tid; x < kHeadDim * kSlab; x += kStateThreads) {
-        const int c = x / kSlab, j = x % kSlab;
-        sS[c * (kSlab + 1) + j] = initial_state
-            ? initial_state[(((int64_t)n * H + h) * kHeadDim + c) * kHeadDim + j0 + j] : 0.f;
+    const int64_t first = first_chunk_id(cu_seqlens, n, seqlen, total_tokens);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init_fence();
+        *sAbort = 0u;
     }
+    if (warp == 0) {
+        tmem_alloc(slot, TM_COLS);
+        tmem_relinquish();
+    }
+    fence_before_sync();
     __syncthreads();
-    int64_t chunk_id = s_first_chunk;
-    const int tx = tid % 16, ty = tid / 16;   // register tiles: columns tx + 16 jj, rows ty + 32 ii
-    for (int64_t t0 = b; t0 < e; t0 += kChunk, ++chunk_id) {
+    fence_after_sync();
+    const uint32_t tbase = *slot;
+    // thread -> state column j (TMEM lane) and a half of the 128 state rows
+    const int q = warp & 3, j = q * 32 + lane, c_half = warp >> 2;   // rows c in [64 c_half, 64 c_half + 64)
+    const int64_t st_base = ((int64_t)n * H + h) * kHeadDim * kHeadDim;
+    // the initial state into TMEM: S^T[j][c] = S[c][j]
+#pragma unroll 1
+    for (int cb = 0; cb < 4; ++cb) {
+        uint32_t v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int c = 64 * c_half + 16 * cb + i;
+            v[i] = __float_as_uint(initial_state ? initial_state[st_base + (int64_t)c * kHeadDim + j] : 0.f);
+        }
+        tmem_st16(taddr(tbase, q, TM_S + 64 * c_half + 16 * cb), v);
+    }
+    tmem_wait_st();
+    uint32_t phase = 0u;
+    bool aborted = false;
+    const int64_t ld = (int64_t)H * kHeadDim;
+    int64_t chunk_id = first;
+    for (int64_t t0 = b; t0 < e && !aborted; t0 += kChunk, ++chunk_id) {
         const int len = (int)(e - t0 < kChunk ? e - t0 : kChunk);
-        __syncthreads();   // the previous chunk's state update is complete
-        if (t0 + kChunk < e) {   // the next chunk's rows into L2
-            const int nlen = (int)(e - t0 - kChunk < kChunk ? e - t0 - kChunk : kChunk);
-            const int64_t nb = ((t0 + kChunk) * H + h) * kHeadDim, ldb = (int64_t)H * kHeadDim;
-            prefetch_rows_l2(w + nb, ldb * 4, nlen, kHeadDim * 4, kStateThreads);
-            prefetch_rows_l2(gamma + nb, ldb * 4, nlen, kHeadDim * 4, kStateThreads);
-            prefetch_rows_l2(k + nb, ldb * 2, nlen, kHeadDim * 2, kStateThreads);
-            prefetch_rows_l2(ut + nb + j0, ldb * 4, nlen, kSlab * 4, kStateThreads);
-        }
-        // record the chunk's starting state
-        if (chunk_id < max_chunks) {
-            for (int x = tid; x < kHeadDim * kSlab; x += kStateThreads) {
-                const int c = x / kSlab, j = x % kSlab;
-                chunk_states[((chunk_id * H + h) * kHeadDim + c) * kHeadDim + j0 + j] =
-                    sS[c * (kSlab + 1) + j];
-            }
-        } else if (tid == 0) {
-            record_error(KDA_DEVERR_BOUNDS);
-        }
-        if (tid < kHeadDim) sgL[tid] = gamma[((t0 + len - 1) * H + h) * kHeadDim + tid];
-        const int64_t base = (t0 * H + h) * kHeadDim, ld = (int64_t)H * kHeadDim;
-        stage<kChunk, kHeadDim, kStateThreads>(sW, kPitch, w + base, ld, len, [](int, int, float x) { return -x; });
-        stage<kChunk, kSlab, kStateThreads>(sU, kSlab + 1, ut + base + j0, ld, len, Identity{});
-        __syncthreads();
-        // Khat_ic = k_ic e^{Gamma_last,c - Gamma_ic}
-        stage2<kChunk, kHeadDim, kStateThreads>(sK, kPitch, gamma + base, k + base, ld, len,
-                                                [sgL](int, int c, float G, float kv) { return kv * expf(sgL[c] - G); });
-        if (tid < kHeadDim) sgC[tid] = expf(sgL[tid]);
-        // U = U~ - W S   (rows r, slab columns j; rows >= len stay 0)
-        {
-            float acc[2][4];
+        const int64_t base = (t0 * H + h) * kHeadDim;
+        if (tid < kHeadDim) sGC[tid] = expf(gamma[base + (int64_t)(len - 1) * ld + tid]);
+        // -W (K-major B of step 2: rows r, columns c) and Khat (MN-major B of step 4: rows r, columns c)
 #pragma unroll
-            for (int ii = 0; ii < 2; ++ii)
+        for (int m = 0; m < 4; ++m) {
+            const int x = tid + kThreads * m, r = x >> 4, ch = x & 15;   // 64 rows x 16 chunks of 8
+            float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, kk[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (r < len) {
+                const int64_t off = base + (int64_t)r * ld + 8 * ch;
+                const float4 w0 = *reinterpret_cast<const float4*>(w + off), w1 = *reinterpret_cast<const float4*>(w + off + 4);
+                const float4 g0 = *reinterpret_cast<const float4*>(gamma + off), g1 = *reinterpret_cast<const float4*>(gamma + off + 4);
+                const uint4 kb = *reinterpret_cast<const uint4*>(k + off);
+                const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                const uint32_t kw[4] = {kb.x, kb.y, kb.z, kb.w};
+                const float* gl = gamma + base + (int64_t)(len - 1) * ld + 8 * ch;
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) acc[ii][jj] = sU[(ty + 32 * ii) * (kSlab + 1) + tx + 16 * jj];
-            tile_fma<2, 4, 32, 16, kPitch, 1, kSlab + 1, 1>(acc, sW, sS, ty, tx, 0, kHeadDim);
-#pragma unroll
-            for (int ii = 0; ii < 2; ++ii) {
-                const int r = ty + 32 * ii;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int j = tx + 16 * jj;
-                    sU[r * (kSlab + 1) + j] = acc[ii][jj];
-                    if (r < len) u_out[((t0 + r) * H + h) * kHeadDim + j0 + j] = acc[ii][jj];
+                for (int i = 0; i < 8; ++i) {
+                    const float kv = __uint_as_float((i & 1) ? (kw[i >> 1] & 0xffff0000u) : (kw[i >> 1] << 16));
+                    a[i] = -wv[i];
+                    kk[i] = kv * expf(gl[i] - gv[i]);
                 }
             }
+            uint4 hi, lo;
+            stc::split8(a, hi, lo);
+            *reinterpret_cast<uint4*>(sm + WH + sw128_chunk_off(r, ch, 64)) = hi;
+            *reinterpret_cast<uint4*>(sm + WL + sw128_chunk_off(r, ch, 64)) = lo;
+            stc::split8(kk, hi, lo);
+            *reinterpret_cast<uint4*>(sm + KH + sw128_chunk_off(r, ch, 64)) = hi;
+            *reinterpret_cast<uint4*>(sm + KL + sw128_chunk_off(r, ch, 64)) = lo;
+        }
+        __syncthreads();   // sGC
+        // 1. the chunk-start state: out, split copy (MN-major A: rows c, columns j), scaled in TMEM
+        const bool store_cs = chunk_id < max_chunks;
+        if (!store_cs && tid == 0) record_error(KDA_DEVERR_BOUNDS);
+#pragma unroll 1
+        for (int cb = 0; cb < 4; ++cb) {
+            uint32_t v[16];
+            const uint32_t col = TM_S + 64 * c_half + 16 * cb;
+            tmem_ld16(taddr(tbase, q, col), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int c = 64 * c_half + 16 * cb + i;
+                const float sv = __uint_as_float(v[i]);
+                if (store_cs) chunk_states[(chunk_id * H + h) * kHeadDim * kHeadDim + (int64_t)c * kHeadDim + j] = sv;
+                uint16_t hi, lo;
+                stc::split1(sv, hi, lo);
+                *reinterpret_cast<uint16_t*>(sm + SH + sw128_off(c, j, 128)) = hi;
+                *reinterpret_cast<uint16_t*>(sm + SL + sw128_off(c, j, 128)) = lo;
+                v[i] = __float_as_uint(sv * sGC[c]);
+            }
+            tmem_st16(taddr(tbase, q, col), v);
+        }
+        tmem_wait_st();
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        // 2. U^T (columns TM_U..) = S^T (-W)^T
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t sh = smem_u32(sm + SH), sl = smem_u32(sm + SL), wh = smem_u32(sm + WH),
+                           wl = smem_u32(sm + WL);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                mma_f16(tbase + TM_U, desc_mnmajor(sh, 128, ks), desc_kmajor(wh, 64, ks), IDESC_U, ks > 0 ? 1u : 0u);
+                mma_f16(tbase + TM_U, desc_mnmajor(sh, 128, ks), desc_kmajor(wl, 64, ks), IDESC_U, 1u);
+                mma_f16(tbase + TM_U, desc_mnmajor(sl, 128, ks), desc_kmajor(wh, 64, ks), IDESC_U, 1u);
+            }
+            mma_commit(bar);
+            if (!mbar_wait_bounded(bar, phase)) {
+                record_error(KDA_DEVERR_TIMEOUT);
+                *sAbort = 1u;
+            }
         }
         __syncthreads();
-        // S = Diag(gamma_last) S + Khat^T U
-        {
-            float acc[4][4];
-            tile_zero(acc);
-            tile_fma<4, 4, 32, 16, 1, kPitch, kSlab + 1, 1>(acc, sK, sU, ty, tx, 0, len);
+        fence_after_sync();
+        if (*sAbort != 0u) { aborted = true; break; }
+        phase ^= 1u;
+        // 3. U = U~ + U^T^T: out, and split as the MN-major A of step 4 (rows r, columns j)
+#pragma unroll 1
+        for (int rb = 0; rb < 2; ++rb) {
+            uint32_t v[16];
+            const int r0 = 32 * c_half + 16 * rb;                  // warps 0-3: r 0-31, warps 4-7: r 32-63
+            tmem_ld16(taddr(tbase, q, TM_U + r0), v);
+            tmem_wait_ld();
 #pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
-                const int c = ty + 32 * ii;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int j = tx + 16 * jj;
-                    sS[c * (kSlab + 1) + j] = fmaf(sgC[c], sS[c * (kSlab + 1) + j], acc[ii][jj]);
+            for (int i = 0; i < 16; ++i) {
+                const int r = r0 + i;
+                float uv = 0.f;
+                if (r < len) {
+                    const int64_t idx = base + (int64_t)r * ld + j;
+                    uv = ut[idx] + __uint_as_float(v[i]);
+                    u_out[idx] = uv;
                 }
+                uint16_t hi, lo;
+                stc::split1(uv, hi, lo);
+                *reinterpret_cast<uint16_t*>(sm + UH + sw128_off(r, j, 64)) = hi;
+                *reinterpret_cast<uint16_t*>(sm + UL + sw128_off(r, j, 64)) = lo;
             }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        // 4. S^T += U^T Khat
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t uh = smem_u32(sm + UH), ul = smem_u32(sm + UL), kh = smem_u32(sm + KH),
+                           kl = smem_u32(sm + KL);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                mma_f16(tbase + TM_S, desc_mnmajor(uh, 64, ks), desc_mnmajor(kh, 64, ks), IDESC_S, 1u);
+                mma_f16(tbase + TM_S, desc_mnmajor(uh, 64, ks), desc_mnmajor(kl, 64, ks), IDESC_S, 1u);
+                mma_f16(tbase + TM_S, desc_mnmajor(ul, 64, ks), desc_mnmajor(kh, 64, ks), IDESC_S, 1u);
+            }
+            mma_commit(bar);
+            if (!mbar_wait_bounded(bar, phase)) {
+                record_error(KDA_DEVERR_TIMEOUT);
+                *sAbort = 1u;
+            }
+        }
+        __syncthreads();
+        fence_after_sync();
+        if (*sAbort != 0u) { aborted = true; break; }
+        phase ^= 1u;
+    }
+    if (aborted) {
+        // the MMAs may still be running: give them (bounded) time before TMEM is released
+        if (tid == 0) mbar_wait_bounded(bar, phase);
+        fence_before_sync();
+        __syncthreads();
+    } else if (final_state) {
+#pragma unroll 1
+        for (int cb = 0; cb < 4; ++cb) {
+            uint32_t v[16];
+            tmem_ld16(taddr(tbase, q, TM_S + 64 * c_half + 16 * cb), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                final_state[st_base + (int64_t)(64 * c_half + 16 * cb + i) * kHeadDim + j] = __uint_as_float(v[i]);
         }
     }
+    fence_before_sync();
     __syncthreads();
-    if (final_state) {
-        for (int x = tid; x < kHeadDim * kSlab; x += kStateThreads) {
-            const int c = x / kSlab, j = x % kSlab;
-            final_state[(((int64_t)n * H + h) * kHeadDim + c) * kHeadDim + j0 + j] =
-                sS[c * (kSlab + 1) + j];
-        }
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tbase, TM_COLS);
     }
 }
 
@@ -463,8 +594,8 @@ cudaError_t launch_staged(const StagedArgs& a, char* ws, const StagedLayout& L, 
         cudaError_t err;
         if ((err = cudaFuncSetAttribute(intra_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)kIntraSmem)) != cudaSuccess) return err;
-        if ((err = cudaFuncSetAttribute(state_prop_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)kStateSmem)) != cudaSuccess) return err;
+        if ((err = cudaFuncSetAttribute(state_prop_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)stc::ALLOC)) != cudaSuccess) return err;
         if ((err = cudaFuncSetAttribute(chunk_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)kOutSmem)) != cudaSuccess) return err;
         attrs_set = true;
@@ -492,8 +623,8 @@ cudaError_t launch_staged(const StagedArgs& a, char* ws, const StagedLayout& L, 
                                                                       count, H, w, ut, p, a.t_mat);
     }
     if (a.N > 0) {
-        dim3 gs((unsigned)a.N, (unsigned)H, kHeadDim / kSlab);
-        state_prop_kernel<<<gs, kStateThreads, kStateSmem, stream>>>(
+        dim3 gs((unsigned)a.N, (unsigned)H);
+        state_prop_tc_kernel<<<gs, stc::kThreads, stc::ALLOC, stream>>>(
             k, gamma, w, ut, a.initial_state, a.cu_seqlens, a.seqlen, a.total_tokens, H, u, cs,
             L.max_chunks, a.final_state);
     }
