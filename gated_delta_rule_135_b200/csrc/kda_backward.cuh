@@ -2,8 +2,9 @@
 // with respect to q, k, v, g, beta, A_log, dt_bias and the initial state.
 //
 // Staged through HBM on top of the staged forward's workspace (Gamma, W, U~, P, U, T and the
-// state at every chunk start): fp32 CUDA-core products, except the three state products of B2,
-// which run on the tensor cores with split-bf16 operands and fp32 accumulation.  Per chunk (restated from the chain rule through
+// state at every chunk start).  The state-gradient scan (B1) and the state products (B2) run on
+// the tensor cores with split-bf16 operands and fp32 accumulation in TMEM; the per-chunk T-side
+// and decay-side stages (B3a, B3b) are fp32 CUDA-core products.  Per chunk (restated from the chain rule through
 // the forward's chunk algebra; the oracle's chunk_step_bwd follows the same steps):
 //   from S' = Diag(gC) S + Khat^T U:   dS = Diag(gC) dS',  dgC = rowsum(S * dS'),
 //                                      dKhat = U dS'^T,     dU = Khat dS'
@@ -32,120 +33,283 @@ constexpr int kPitchC = kChunk + 1;
 __device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162float(x); }
 
 // ---------------------------------------------------------------------------
-// B1: dS backwards over a sequence's chunks; per chunk stores dS' (the gradient of the
-// state after it) and dU.  grid (N, H, 2), 512 threads; each block owns a 128 x 64 column
-// slab of dS.  Register tiles: dU 2 x 4 and dS 4 x 4 per thread.
-constexpr int kB1Threads = 512;
-constexpr int kB1Slab = 64;              // dS columns per block
-constexpr int kSP = kB1Slab + 1;
-constexpr size_t kB1Smem = sizeof(float) * (kHeadDim * kSP + 3 * kChunk * kPitch + kChunk * kPitchC +
-                                            2 * kChunk * kSP + 2 * kHeadDim);
+// B1 (tensor cores): dS backwards over a sequence's chunks.  grid (N, H), 256 threads: one sequence and head per CTA, dS^T (the
+// gradient of the state after the current chunk, transposed: lane j, column c) in fp32 TMEM.
+// Per chunk, last to first:
+//   1. one pass over the TMEM state writes dS' out, stages its split-bf16 copy (the MN-major A
+//      operand dS'^T) and scales the TMEM state by gamma_C;
+//   2. dU^T = dO^T (scale P) + dS'^T Khat^T    (M = 128 columns j, N = 64 tokens);
+//   3. dU is written out and staged split-bf16 as the MN-major A operand dU^T;
+//   4. dS^T += dO^T (scale gamma q) - dU^T W   (M = 128, N = 128 state rows c).
+// dO is bf16 already (one part); every other operand enters as bf16 high and low parts.
+namespace btc {
+using namespace umma;
+constexpr uint32_t NH = 0, NL = 32768, KH = 65536, KL = 81920, PH = 98304, PL = 106496, DO = 114688,
+                   UH = 131072, UL = 147456, QH = 163840, QL = 180224, WH = 196608, WL = 212992,
+                   GC = 229376, BAR = GC + 512, TSLOT = BAR + 8, ABORT = BAR + 12;
+constexpr uint32_t BYTES = BAR + 16;
+constexpr uint32_t ALLOC = BYTES + 1008;
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_COLS = 256;
+constexpr uint32_t IDESC_UP = idesc_f16(128, 64, true, true, true);    // dO^T (scale P)
+constexpr uint32_t IDESC_UK = idesc_f16(128, 64, true, true, false);   // dS'^T Khat^T
+constexpr uint32_t IDESC_S = idesc_f16(128, 128, true, true, true);
+constexpr int kThreads = 256;
 
-__global__ void __launch_bounds__(kB1Threads) state_bwd_kernel(
+__device__ __forceinline__ void split1(float x, uint16_t& hi, uint16_t& lo) {
+    const __nv_bfloat16 hb = __float2bfloat16_rn(x);
+    hi = __bfloat16_as_ushort(hb);
+    lo = __bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(hb)));
+}
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+    uint16_t a[8], b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) split1(x[i], a[i], b[i]);
+    hi = make_uint4(a[0] | ((uint32_t)a[1] << 16), a[2] | ((uint32_t)a[3] << 16), a[4] | ((uint32_t)a[5] << 16),
+                    a[6] | ((uint32_t)a[7] << 16));
+    lo = make_uint4(b[0] | ((uint32_t)b[1] << 16), b[2] | ((uint32_t)b[3] << 16), b[4] | ((uint32_t)b[5] << 16),
+                    b[6] | ((uint32_t)b[7] << 16));
+}
+__device__ __forceinline__ void load8f(const float* src, float (&x)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ void load8b(const __nv_bfloat16* src, float (&x)[8]) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+}  // namespace btc
+
+__global__ void __launch_bounds__(btc::kThreads, 1) state_bwd_tc_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const float* __restrict__ gamma,
     const float* __restrict__ w, const float* __restrict__ p, const __nv_bfloat16* __restrict__ d_out,
     const float* __restrict__ d_final, const int32_t* __restrict__ cu_seqlens, int64_t seqlen,
     int64_t total_tokens, int H, float scale, int64_t max_chunks, float* __restrict__ dsn_out,
     float* __restrict__ du_out, float* __restrict__ d_initial) {
-    const int n = blockIdx.x, h = blockIdx.y, j0 = blockIdx.z * kB1Slab, tid = threadIdx.x;
-    extern __shared__ float sm[];
-    float* sdS = sm;                                   // [128][65]
-    float* sKh = sdS + kHeadDim * kSP;                 // [64][129] Khat
-    float* sQt = sKh + kChunk * kPitch;                // [64][129] scale * gamma * q
-    float* sW = sQt + kChunk * kPitch;                 // [64][129] -W
-    float* sP = sW + kChunk * kPitch;                  // [64][65]  scale * P
-    float* sdO = sP + kChunk * kPitchC;                // [64][65]
-    float* sdU = sdO + kChunk * kSP;                   // [64][65]
-    float* sgC = sdU + kChunk * kSP;                   // [128] e^{Gamma_last}
-    float* sgL = sgC + kHeadDim;                       // [128] Gamma_last
+    using namespace btc;
+    const int n = blockIdx.x, h = blockIdx.y, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + BAR);
+    uint32_t* slot = reinterpret_cast<uint32_t*>(sm + TSLOT);
+    volatile uint32_t* sAbort = reinterpret_cast<volatile uint32_t*>(sm + ABORT);
+    float* sGC = reinterpret_cast<float*>(sm + GC);
     int64_t b, e;
     seq_range(cu_seqlens, n, seqlen, total_tokens, &b, &e);
     const int64_t c_first = first_chunk_id(cu_seqlens, n, seqlen, total_tokens);
-    for (int x = tid; x < kHeadDim * kB1Slab; x += kB1Threads) {
-        const int c = x / kB1Slab, j = x % kB1Slab;
-        sdS[c * kSP + j] = d_final ? d_final[(((int64_t)n * H + h) * kHeadDim + c) * kHeadDim + j0 + j] : 0.f;
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init_fence();
+        *sAbort = 0u;
     }
-    const int tx = tid % 16, ty = tid / 16;    // tile columns tx + 16 jj, rows ty + 32 ii
+    if (warp == 0) {
+        tmem_alloc(slot, TM_COLS);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *slot;
+    const int q4 = warp & 3, j = q4 * 32 + lane, c_half = warp >> 2;
+    const int64_t st_base = ((int64_t)n * H + h) * kHeadDim * kHeadDim;
+#pragma unroll 1
+    for (int cb = 0; cb < 4; ++cb) {
+        uint32_t v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int c = 64 * c_half + 16 * cb + i;
+            v[i] = __float_as_uint(d_final ? d_final[st_base + (int64_t)c * kHeadDim + j] : 0.f);
+        }
+        tmem_st16(taddr(tbase, q4, TM_S + 64 * c_half + 16 * cb), v);
+    }
+    tmem_wait_st();
+    uint32_t phase = 0u;
+    bool aborted = false;
+    const int64_t ld = (int64_t)H * kHeadDim;
     const int64_t nch = (e - b + kChunk - 1) / kChunk;
-    for (int64_t jc = nch - 1; jc >= 0; --jc) {
+    for (int64_t jc = nch - 1; jc >= 0 && !aborted; --jc) {
         const int64_t t0 = b + jc * kChunk, cid = c_first + jc;
         const int len = (int)(e - t0 < kChunk ? e - t0 : kChunk);
-        if (cid >= max_chunks) {
-            if (tid == 0) record_error(KDA_DEVERR_BOUNDS);
-            break;
-        }
-        __syncthreads();   // the previous chunk's dS is complete; its operands are consumed
-        if (jc > 0) {      // the next chunk in this scan (full: only a sequence's last chunk is short)
-            const int64_t nb = ((t0 - kChunk) * H + h) * kHeadDim, ldb = (int64_t)H * kHeadDim;
-            prefetch_rows_l2(gamma + nb, ldb * 4, kChunk, kHeadDim * 4, kB1Threads);
-            prefetch_rows_l2(w + nb, ldb * 4, kChunk, kHeadDim * 4, kB1Threads);
-            prefetch_rows_l2(k + nb, ldb * 2, kChunk, kHeadDim * 2, kB1Threads);
-            prefetch_rows_l2(q + nb, ldb * 2, kChunk, kHeadDim * 2, kB1Threads);
-            prefetch_rows_l2(p + ((t0 - kChunk) * H + h) * kChunk, (int64_t)H * kChunk * 4, kChunk, kChunk * 4,
-                             kB1Threads);
-            prefetch_rows_l2(d_out + nb + j0, ldb * 2, kChunk, kB1Slab * 2, kB1Threads);
-        }
-        // dS' of this chunk
-        for (int x = tid; x < kHeadDim * kB1Slab; x += kB1Threads) {
-            const int c = x / kB1Slab, j = x % kB1Slab;
-            dsn_out[((cid * H + h) * kHeadDim + c) * kHeadDim + j0 + j] = sdS[c * kSP + j];
-        }
-        const float* gl = gamma + ((t0 + len - 1) * H + h) * kHeadDim;
-        if (tid < kHeadDim) sgL[tid] = gl[tid];
-        const int64_t base = (t0 * H + h) * kHeadDim, ld = (int64_t)H * kHeadDim;
-        stage<kChunk, kHeadDim, kB1Threads>(sW, kPitch, w + base, ld, len,
-                                            [](int, int, float x) { return -x; });
-        stage<kChunk, kChunk, kB1Threads>(sP, kPitchC, p + (t0 * H + h) * kChunk, (int64_t)H * kChunk, len,
-                                          [scale](int, int, float x) { return scale * x; });
-        stage<kChunk, kB1Slab, kB1Threads>(sdO, kSP, d_out + base + j0, ld, len, Identity{});
-        __syncthreads();
-        stage2<kChunk, kHeadDim, kB1Threads>(sKh, kPitch, gamma + base, k + base, ld, len,
-                                             [sgL](int, int c, float G, float kv) { return kv * expf(sgL[c] - G); });
-        stage2<kChunk, kHeadDim, kB1Threads>(sQt, kPitch, gamma + base, q + base, ld, len,
-                                             [scale](int, int, float G, float qv) { return scale * qv * expf(G); });
-        if (tid < kHeadDim) sgC[tid] = expf(sgL[tid]);
-        __syncthreads();
-        // dU = scale P^T dO + Khat dS'   (rows >= len come out 0: P is lower triangular)
-        {
-            float acc[2][4];
-            tile_zero(acc);
-            tile_fma<2, 4, 32, 16, 1, kPitchC, kSP, 1>(acc, sP, sdO, ty, tx, 0, len);
-            tile_fma<2, 4, 32, 16, kPitch, 1, kSP, 1>(acc, sKh, sdS, ty, tx, 0, kHeadDim);
+        const int64_t base = (t0 * H + h) * kHeadDim;
+        const float* gl = gamma + base + (int64_t)(len - 1) * ld;
+        if (tid < kHeadDim) sGC[tid] = expf(gl[tid]);
+        // Khat (K-major B of step 2), scale gamma q and -W (MN-major B of step 4), dO (A of 2 and 4);
+        // all [64 tokens][128 channels], zero past the chunk
+#pragma unroll 2
+        for (int m = 0; m < 4; ++m) {
+            const int x = tid + kThreads * m, r = x >> 4, ch = x & 15;
+            float kk[8] = {}, qq[8] = {}, ww[8] = {};
+            uint4 dob = make_uint4(0u, 0u, 0u, 0u);
+            if (r < len) {
+                const int64_t off = base + (int64_t)r * ld + 8 * ch;
+                float g8[8], k8[8], q8[8], w8[8];
+                load8f(gamma + off, g8);
+                load8b(k + off, k8);
+                load8b(q + off, q8);
+                load8f(w + off, w8);
+                dob = *reinterpret_cast<const uint4*>(d_out + off);
 #pragma unroll
-            for (int ii = 0; ii < 2; ++ii) {
-                const int r = ty + 32 * ii;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int j = tx + 16 * jj;
-                    sdU[r * kSP + j] = acc[ii][jj];
-                    if (r < len) du_out[((t0 + r) * H + h) * kHeadDim + j0 + j] = acc[ii][jj];
+                for (int i = 0; i < 8; ++i) {
+                    kk[i] = k8[i] * expf(gl[8 * ch + i] - g8[i]);
+                    qq[i] = scale * q8[i] * expf(g8[i]);
+                    ww[i] = -w8[i];
                 }
+            }
+            const uint32_t o = sw128_chunk_off(r, ch, 64);
+            uint4 hi, lo;
+            split8(kk, hi, lo);
+            *reinterpret_cast<uint4*>(sm + KH + o) = hi;
+            *reinterpret_cast<uint4*>(sm + KL + o) = lo;
+            split8(qq, hi, lo);
+            *reinterpret_cast<uint4*>(sm + QH + o) = hi;
+            *reinterpret_cast<uint4*>(sm + QL + o) = lo;
+            split8(ww, hi, lo);
+            *reinterpret_cast<uint4*>(sm + WH + o) = hi;
+            *reinterpret_cast<uint4*>(sm + WL + o) = lo;
+            *reinterpret_cast<uint4*>(sm + DO + o) = dob;
+        }
+        // scale P: rows i (tokens, K), columns r (N)
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const int x = tid + kThreads * m, i = x >> 3, ch = x & 7;
+            float pp[8] = {};
+            if (i < len) {
+                load8f(p + (t0 * H + h) * kChunk + (int64_t)i * H * kChunk + 8 * ch, pp);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) pp[t] *= scale;
+            }
+            uint4 hi, lo;
+            split8(pp, hi, lo);
+            *reinterpret_cast<uint4*>(sm + PH + sw128_chunk_off(i, ch, 64)) = hi;
+            *reinterpret_cast<uint4*>(sm + PL + sw128_chunk_off(i, ch, 64)) = lo;
+        }
+        __syncthreads();   // sGC
+        // 1. dS' out, its split copy (rows c, columns j), and gamma_C dS' in TMEM
+        const bool in_range = cid < max_chunks;
+        if (!in_range && tid == 0) record_error(KDA_DEVERR_BOUNDS);
+#pragma unroll 1
+        for (int cb = 0; cb < 4; ++cb) {
+            uint32_t v[16];
+            const uint32_t col = TM_S + 64 * c_half + 16 * cb;
+            tmem_ld16(taddr(tbase, q4, col), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int c = 64 * c_half + 16 * cb + i;
+                const float sv = __uint_as_float(v[i]);
+                if (in_range) dsn_out[(cid * H + h) * kHeadDim * kHeadDim + (int64_t)c * kHeadDim + j] = sv;
+                uint16_t hi, lo;
+                split1(sv, hi, lo);
+                *reinterpret_cast<uint16_t*>(sm + NH + sw128_off(c, j, 128)) = hi;
+                *reinterpret_cast<uint16_t*>(sm + NL + sw128_off(c, j, 128)) = lo;
+                v[i] = __float_as_uint(sv * sGC[c]);
+            }
+            tmem_st16(taddr(tbase, q4, col), v);
+        }
+        tmem_wait_st();
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        // 2. dU^T = dO^T (scale P) + dS'^T Khat^T
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t d0 = smem_u32(sm + DO), ph = smem_u32(sm + PH), pl = smem_u32(sm + PL),
+                           nh = smem_u32(sm + NH), nl = smem_u32(sm + NL), kh = smem_u32(sm + KH),
+                           kl = smem_u32(sm + KL);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                mma_f16(tbase + TM_U, desc_mnmajor(d0, 64, ks), desc_mnmajor(ph, 64, ks), IDESC_UP, ks > 0 ? 1u : 0u);
+                mma_f16(tbase + TM_U, desc_mnmajor(d0, 64, ks), desc_mnmajor(pl, 64, ks), IDESC_UP, 1u);
+            }
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                mma_f16(tbase + TM_U, desc_mnmajor(nh, 128, ks), desc_kmajor(kh, 64, ks), IDESC_UK, 1u);
+                mma_f16(tbase + TM_U, desc_mnmajor(nh, 128, ks), desc_kmajor(kl, 64, ks), IDESC_UK, 1u);
+                mma_f16(tbase + TM_U, desc_mnmajor(nl, 128, ks), desc_kmajor(kh, 64, ks), IDESC_UK, 1u);
+            }
+            mma_commit(bar);
+            if (!mbar_wait_bounded(bar, phase)) {
+                record_error(KDA_DEVERR_TIMEOUT);
+                *sAbort = 1u;
             }
         }
         __syncthreads();
-        // dS = Diag(gC) dS' + scale (gamma q)^T dO - W^T dU
-        {
-            float acc[4][4];
-            tile_zero(acc);
-            tile_fma<4, 4, 32, 16, 1, kPitch, kSP, 1>(acc, sQt, sdO, ty, tx, 0, len);
-            tile_fma<4, 4, 32, 16, 1, kPitch, kSP, 1>(acc, sW, sdU, ty, tx, 0, len);
+        fence_after_sync();
+        if (*sAbort != 0u) { aborted = true; break; }
+        phase ^= 1u;
+        // 3. dU out and staged (rows r, columns j)
+#pragma unroll 1
+        for (int rb = 0; rb < 2; ++rb) {
+            uint32_t v[16];
+            const int r0 = 32 * c_half + 16 * rb;
+            tmem_ld16(taddr(tbase, q4, TM_U + r0), v);
+            tmem_wait_ld();
 #pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
-                const int c = ty + 32 * ii;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int j = tx + 16 * jj;
-                    sdS[c * kSP + j] = fmaf(sgC[c], sdS[c * kSP + j], acc[ii][jj]);
+            for (int i = 0; i < 16; ++i) {
+                const int r = r0 + i;
+                float dv = 0.f;
+                if (r < len) {
+                    dv = __uint_as_float(v[i]);
+                    du_out[base + (int64_t)r * ld + j] = dv;
                 }
+                uint16_t hi, lo;
+                split1(dv, hi, lo);
+                *reinterpret_cast<uint16_t*>(sm + UH + sw128_off(r, j, 64)) = hi;
+                *reinterpret_cast<uint16_t*>(sm + UL + sw128_off(r, j, 64)) = lo;
             }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        // 4. dS^T += dO^T (scale gamma q) - dU^T W
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t d0 = smem_u32(sm + DO), qh = smem_u32(sm + QH), ql = smem_u32(sm + QL),
+                           uh = smem_u32(sm + UH), ul = smem_u32(sm + UL), wh = smem_u32(sm + WH),
+                           wl = smem_u32(sm + WL);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                mma_f16(tbase + TM_S, desc_mnmajor(d0, 64, ks), desc_mnmajor(qh, 64, ks), IDESC_S, 1u);
+                mma_f16(tbase + TM_S, desc_mnmajor(d0, 64, ks), desc_mnmajor(ql, 64, ks), IDESC_S, 1u);
+                mma_f16(tbase + TM_S, desc_mnmajor(uh, 64, ks), desc_mnmajor(wh, 64, ks), IDESC_S, 1u);
+                mma_f16(tbase + TM_S, desc_mnmajor(uh, 64, ks), desc_mnmajor(wl, 64, ks), IDESC_S, 1u);
+                mma_f16(tbase + TM_S, desc_mnmajor(ul, 64, ks), desc_mnmajor(wh, 64, ks), IDESC_S, 1u);
+            }
+            mma_commit(bar);
+            if (!mbar_wait_bounded(bar, phase)) {
+                record_error(KDA_DEVERR_TIMEOUT);
+                *sAbort = 1u;
+            }
+        }
+        __syncthreads();
+        fence_after_sync();
+        if (*sAbort != 0u) { aborted = true; break; }
+        phase ^= 1u;
+    }
+    if (aborted) {
+        if (tid == 0) mbar_wait_bounded(bar, phase);
+        fence_before_sync();
+        __syncthreads();
+    } else if (d_initial) {
+#pragma unroll 1
+        for (int cb = 0; cb < 4; ++cb) {
+            uint32_t v[16];
+            tmem_ld16(taddr(tbase, q4, TM_S + 64 * c_half + 16 * cb), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                d_initial[st_base + (int64_t)(64 * c_half + 16 * cb + i) * kHeadDim + j] = __uint_as_float(v[i]);
         }
     }
+    fence_before_sync();
     __syncthreads();
-    if (d_initial) {
-        for (int x = tid; x < kHeadDim * kB1Slab; x += kB1Threads) {
-            const int c = x / kB1Slab, j = x % kB1Slab;
-            d_initial[(((int64_t)n * H + h) * kHeadDim + c) * kHeadDim + j0 + j] = sdS[c * kSP + j];
-        }
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tbase, TM_COLS);
     }
 }
 
@@ -816,8 +980,8 @@ cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const Bw
     static bool attrs_set = false;
     if (!attrs_set) {
         cudaError_t err;
-        if ((err = cudaFuncSetAttribute(bwd::state_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)bwd::kB1Smem)) != cudaSuccess) return err;
+        if ((err = cudaFuncSetAttribute(bwd::state_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)bwd::btc::ALLOC)) != cudaSuccess) return err;
         if ((err = cudaFuncSetAttribute(bwd::chunk_products_tc_kernel,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd::tc::ALLOC)) !=
             cudaSuccess) return err;
@@ -861,8 +1025,8 @@ cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const Bw
     const auto* dO = static_cast<const __nv_bfloat16*>(d.d_out);
     const int H = a.H;
     if (a.N > 0) {
-        dim3 g1((unsigned)a.N, (unsigned)H, kHeadDim / bwd::kB1Slab);
-        bwd::state_bwd_kernel<<<g1, bwd::kB1Threads, bwd::kB1Smem, stream>>>(
+        dim3 g1((unsigned)a.N, (unsigned)H);
+        bwd::state_bwd_tc_kernel<<<g1, bwd::btc::kThreads, bwd::btc::ALLOC, stream>>>(
             q, k, gamma, w, p, dO, d.d_final, a.cu_seqlens, a.seqlen, a.total_tokens, H, a.scale, L.max_chunks,
             dsn, du, d.d_initial);
     }
