@@ -22,6 +22,7 @@
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_tile.cuh"
+#include "kda_chunks.cuh"
 #include "umma.cuh"
 
 namespace kda {
