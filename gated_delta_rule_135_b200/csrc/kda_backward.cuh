@@ -978,8 +978,7 @@ BwdLayout bwd_layout(int64_t total_tokens, int H, int N) {
 
 cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const BwdLayout& B,
                        cudaStream_t stream) {
-    static bool attrs_set = false;
-    if (!attrs_set) {
+    cudaError_t setup_err = once_per_device([](int) {
         cudaError_t err;
         if ((err = cudaFuncSetAttribute(bwd::state_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)bwd::btc::ALLOC)) != cudaSuccess) return err;
@@ -992,8 +991,9 @@ cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const Bw
                                         (int)bwd::kB3bSmem)) != cudaSuccess) return err;
         if ((err = cudaFuncSetAttribute(bwd::decay_bwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)bwd::kB3bSmem)) != cudaSuccess) return err;
-        attrs_set = true;
-    }
+        return cudaSuccess;
+    });
+    if (setup_err != cudaSuccess) return setup_err;
     // the forward's intermediates (Gamma, W, P, U, chunk-start states); out is not needed
     StagedArgs f = a;
     f.out = nullptr;

@@ -1329,20 +1329,15 @@ namespace fused {
 
 template <bool kScalar>
 cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
-    static int sm_count = 0;
-    static bool attr_set = false;
-    if (!sm_count) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev);
-        if (sm_count <= 0) return cudaErrorInvalidDevice;
-    }
-    if (!attr_set) {
-        cudaError_t err = cudaFuncSetAttribute(kda_fused_kernel<kScalar>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
-        if (err != cudaSuccess) return err;
-        attr_set = true;
-    }
+    cudaError_t err = once_per_device([](int) {
+        return cudaFuncSetAttribute(kda_fused_kernel<kScalar>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)SMEM_ALLOC);
+    });
+    if (err != cudaSuccess) return err;
+    int dev = 0, sm_count = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+    if (sm_count <= 0) return cudaErrorInvalidDevice;
     CUtensorMap tq, tk, tv, tg;
     const int64_t rows = a.total_tokens, cols = (int64_t)a.H * kHeadDim;
     const uint32_t box = kScalar ? 64u : (uint32_t)kHeadDim;

@@ -5,7 +5,25 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace kda {
+
+// Runs `setup` (cudaFuncSetAttribute calls and the like) once for the current device: kernel
+// attributes belong to a device, so a process that drives several GPUs needs them on each.
+template <typename F>
+cudaError_t once_per_device(F setup) {
+    static std::mutex m;
+    static uint64_t done = 0;   // bit d: device d is set up (devices past 63 always run setup)
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lock(m);
+    if (dev < 64 && (done >> dev) & 1u) return cudaSuccess;
+    err = setup(dev);
+    if (err == cudaSuccess && dev < 64) done |= uint64_t(1) << dev;
+    return err;
+}
 
 struct StagedArgs {
     const void* q;

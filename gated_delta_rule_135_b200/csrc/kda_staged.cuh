@@ -590,8 +590,7 @@ StagedLayout staged_layout(int64_t total_tokens, int H, int N) {
 }
 
 cudaError_t launch_staged(const StagedArgs& a, char* ws, const StagedLayout& L, cudaStream_t stream) {
-    static bool attrs_set = false;
-    if (!attrs_set) {
+    cudaError_t setup_err = once_per_device([](int) {
         cudaError_t err;
         if ((err = cudaFuncSetAttribute(intra_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)kIntraSmem)) != cudaSuccess) return err;
@@ -599,8 +598,9 @@ cudaError_t launch_staged(const StagedArgs& a, char* ws, const StagedLayout& L, 
                                         (int)stc::ALLOC)) != cudaSuccess) return err;
         if ((err = cudaFuncSetAttribute(chunk_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)kOutSmem)) != cudaSuccess) return err;
-        attrs_set = true;
-    }
+        return cudaSuccess;
+    });
+    if (setup_err != cudaSuccess) return setup_err;
     int4* table = reinterpret_cast<int4*>(ws + L.chunk_table);
     int32_t* count = reinterpret_cast<int32_t*>(ws + L.chunk_table + sizeof(int4) * L.max_chunks);
     float* gamma = reinterpret_cast<float*>(ws + L.gamma);
