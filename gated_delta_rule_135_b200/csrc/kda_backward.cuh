@@ -56,33 +56,6 @@ constexpr uint32_t IDESC_UK = idesc_f16(128, 64, true, true, false);   // dS'^T 
 constexpr uint32_t IDESC_S = idesc_f16(128, 128, true, true, true);
 constexpr int kThreads = 256;
 
-__device__ __forceinline__ void split1(float x, uint16_t& hi, uint16_t& lo) {
-    const __nv_bfloat16 hb = __float2bfloat16_rn(x);
-    hi = __bfloat16_as_ushort(hb);
-    lo = __bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(hb)));
-}
-__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
-    uint16_t a[8], b[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) split1(x[i], a[i], b[i]);
-    hi = make_uint4(a[0] | ((uint32_t)a[1] << 16), a[2] | ((uint32_t)a[3] << 16), a[4] | ((uint32_t)a[5] << 16),
-                    a[6] | ((uint32_t)a[7] << 16));
-    lo = make_uint4(b[0] | ((uint32_t)b[1] << 16), b[2] | ((uint32_t)b[3] << 16), b[4] | ((uint32_t)b[5] << 16),
-                    b[6] | ((uint32_t)b[7] << 16));
-}
-__device__ __forceinline__ void load8f(const float* src, float (&x)[8]) {
-    const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-__device__ __forceinline__ void load8b(const __nv_bfloat16* src, float (&x)[8]) {
-    const uint4 v = *reinterpret_cast<const uint4*>(src);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        x[2 * i] = __uint_as_float(w[i] << 16);
-        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-}
 }  // namespace btc
 
 __global__ void __launch_bounds__(btc::kThreads, 1) state_bwd_tc_kernel(
@@ -148,10 +121,10 @@ __global__ void __launch_bounds__(btc::kThreads, 1) state_bwd_tc_kernel(
             if (r < len) {
                 const int64_t off = base + (int64_t)r * ld + 8 * ch;
                 float g8[8], k8[8], q8[8], w8[8];
-                load8f(gamma + off, g8);
-                load8b(k + off, k8);
-                load8b(q + off, q8);
-                load8f(w + off, w8);
+                load8_f32(gamma + off, g8);
+                load8_bf16(k + off, k8);
+                load8_bf16(q + off, q8);
+                load8_f32(w + off, w8);
                 dob = *reinterpret_cast<const uint4*>(d_out + off);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -162,13 +135,13 @@ __global__ void __launch_bounds__(btc::kThreads, 1) state_bwd_tc_kernel(
             }
             const uint32_t o = sw128_chunk_off(r, ch, 64);
             uint4 hi, lo;
-            split8(kk, hi, lo);
+            split_bf16x8(kk, hi, lo);
             *reinterpret_cast<uint4*>(sm + KH + o) = hi;
             *reinterpret_cast<uint4*>(sm + KL + o) = lo;
-            split8(qq, hi, lo);
+            split_bf16x8(qq, hi, lo);
             *reinterpret_cast<uint4*>(sm + QH + o) = hi;
             *reinterpret_cast<uint4*>(sm + QL + o) = lo;
-            split8(ww, hi, lo);
+            split_bf16x8(ww, hi, lo);
             *reinterpret_cast<uint4*>(sm + WH + o) = hi;
             *reinterpret_cast<uint4*>(sm + WL + o) = lo;
             *reinterpret_cast<uint4*>(sm + DO + o) = dob;
@@ -179,12 +152,12 @@ __global__ void __launch_bounds__(btc::kThreads, 1) state_bwd_tc_kernel(
             const int x = tid + kThreads * m, i = x >> 3, ch = x & 7;
             float pp[8] = {};
             if (i < len) {
-                load8f(p + (t0 * H + h) * kChunk + (int64_t)i * H * kChunk + 8 * ch, pp);
+                load8_f32(p + (t0 * H + h) * kChunk + (int64_t)i * H * kChunk + 8 * ch, pp);
 #pragma unroll
                 for (int t = 0; t < 8; ++t) pp[t] *= scale;
             }
             uint4 hi, lo;
-            split8(pp, hi, lo);
+            split_bf16x8(pp, hi, lo);
             *reinterpret_cast<uint4*>(sm + PH + sw128_chunk_off(i, ch, 64)) = hi;
             *reinterpret_cast<uint4*>(sm + PL + sw128_chunk_off(i, ch, 64)) = lo;
         }
@@ -204,7 +177,7 @@ __global__ void __launch_bounds__(btc::kThreads, 1) state_bwd_tc_kernel(
                 const float sv = __uint_as_float(v[i]);
                 if (in_range) dsn_out[(cid * H + h) * kHeadDim * kHeadDim + (int64_t)c * kHeadDim + j] = sv;
                 uint16_t hi, lo;
-                split1(sv, hi, lo);
+                split_bf16(sv, hi, lo);
                 *reinterpret_cast<uint16_t*>(sm + NH + sw128_off(c, j, 128)) = hi;
                 *reinterpret_cast<uint16_t*>(sm + NL + sw128_off(c, j, 128)) = lo;
                 v[i] = __float_as_uint(sv * sGC[c]);
@@ -258,7 +231,7 @@ __global__ void __launch_bounds__(btc::kThreads, 1) state_bwd_tc_kernel(
                     du_out[base + (int64_t)r * ld + j] = dv;
                 }
                 uint16_t hi, lo;
-                split1(dv, hi, lo);
+                split_bf16(dv, hi, lo);
                 *reinterpret_cast<uint16_t*>(sm + UH + sw128_off(r, j, 64)) = hi;
                 *reinterpret_cast<uint16_t*>(sm + UL + sw128_off(r, j, 64)) = lo;
             }
@@ -335,24 +308,6 @@ constexpr uint32_t IDESC_N128 = idesc_f16(128, 128, true, false, false);
 constexpr uint32_t IDESC_N64 = idesc_f16(128, 64, true, false, false);
 constexpr int kThreads = 256;
 
-__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
-    uint32_t h[4], l[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * i]), h1 = __float2bfloat16_rn(x[2 * i + 1]);
-        const __nv_bfloat16 l0 = __float2bfloat16_rn(x[2 * i] - __bfloat162float(h0));
-        const __nv_bfloat16 l1 = __float2bfloat16_rn(x[2 * i + 1] - __bfloat162float(h1));
-        h[i] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-        l[i] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
-    }
-    hi = make_uint4(h[0], h[1], h[2], h[3]);
-    lo = make_uint4(l[0], l[1], l[2], l[3]);
-}
-
-__device__ __forceinline__ void load8(const float* src, float (&x)[8]) {
-    const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
 }  // namespace tc
 
 __global__ void __launch_bounds__(tc::kThreads, 2) chunk_products_tc_kernel(
@@ -396,15 +351,15 @@ __global__ void __launch_bounds__(tc::kThreads, 2) chunk_products_tc_kernel(
         for (int m = 0; m < 4; ++m) {
             const int x = tid + kThreads * m, c = x >> 3, ch = x & 7;
             float a[8], b[8];
-            load8(chunk_states + sbase + (int64_t)c * kHeadDim + col0 + 8 * ch, a);
-            load8(dsn + sbase + (int64_t)c * kHeadDim + col0 + 8 * ch, b);
+            load8_f32(chunk_states + sbase + (int64_t)c * kHeadDim + col0 + 8 * ch, a);
+            load8_f32(dsn + sbase + (int64_t)c * kHeadDim + col0 + 8 * ch, b);
 #pragma unroll
             for (int i = 0; i < 8; ++i) gpart[m] = fmaf(a[i], b[i], gpart[m]);
             uint4 hi, lo;
-            split8(a, hi, lo);
+            split_bf16x8(a, hi, lo);
             *reinterpret_cast<uint4*>(sm + S_HI + sw128_chunk_off(c, ch, 128)) = hi;
             *reinterpret_cast<uint4*>(sm + S_LO + sw128_chunk_off(c, ch, 128)) = lo;
-            split8(b, hi, lo);
+            split_bf16x8(b, hi, lo);
             *reinterpret_cast<uint4*>(sm + N_HI + sw128_chunk_off(c, ch, 128)) = hi;
             *reinterpret_cast<uint4*>(sm + N_LO + sw128_chunk_off(c, ch, 128)) = lo;
         }
@@ -417,8 +372,8 @@ __global__ void __launch_bounds__(tc::kThreads, 2) chunk_products_tc_kernel(
                 if (r < len) hi = *reinterpret_cast<const uint4*>(d_out + base + (int64_t)r * ld + col0 + 8 * ch);
             } else if (r - 64 < len) {
                 float a[8];
-                load8(du + base + (int64_t)(r - 64) * ld + col0 + 8 * ch, a);
-                split8(a, hi, lo);
+                load8_f32(du + base + (int64_t)(r - 64) * ld + col0 + 8 * ch, a);
+                split_bf16x8(a, hi, lo);
             }
             *reinterpret_cast<uint4*>(sm + B_HI + sw128_chunk_off(r, ch, 128)) = hi;
             *reinterpret_cast<uint4*>(sm + B_LO + sw128_chunk_off(r, ch, 128)) = lo;
@@ -429,8 +384,8 @@ __global__ void __launch_bounds__(tc::kThreads, 2) chunk_products_tc_kernel(
             uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = make_uint4(0u, 0u, 0u, 0u);
             if (r < len) {
                 float a[8];
-                load8(u + base + (int64_t)r * ld + col0 + 8 * ch, a);
-                split8(a, hi, lo);
+                load8_f32(u + base + (int64_t)r * ld + col0 + 8 * ch, a);
+                split_bf16x8(a, hi, lo);
             }
             *reinterpret_cast<uint4*>(sm + U_HI + sw128_chunk_off(r, ch, 64)) = hi;
             *reinterpret_cast<uint4*>(sm + U_LO + sw128_chunk_off(r, ch, 64)) = lo;

@@ -302,20 +302,6 @@ constexpr uint32_t IDESC_U = idesc_f16(128, 64, true, true, false);
 constexpr uint32_t IDESC_S = idesc_f16(128, 128, true, true, true);
 constexpr int kThreads = 256;
 
-__device__ __forceinline__ void split1(float x, uint16_t& hi, uint16_t& lo) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    hi = __bfloat16_as_ushort(h);
-    lo = __bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(h)));
-}
-__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
-    uint16_t h[8], l[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) split1(x[i], h[i], l[i]);
-    hi = make_uint4(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16), h[4] | ((uint32_t)h[5] << 16),
-                    h[6] | ((uint32_t)h[7] << 16));
-    lo = make_uint4(l[0] | ((uint32_t)l[1] << 16), l[2] | ((uint32_t)l[3] << 16), l[4] | ((uint32_t)l[5] << 16),
-                    l[6] | ((uint32_t)l[7] << 16));
-}
 }  // namespace stc
 
 __global__ void __launch_bounds__(stc::kThreads, 1) state_prop_tc_kernel(
@@ -394,10 +380,10 @@ __global__ void __launch_bounds__(stc::kThreads, 1) state_prop_tc_kernel(
                 }
             }
             uint4 hi, lo;
-            stc::split8(a, hi, lo);
+            split_bf16x8(a, hi, lo);
             *reinterpret_cast<uint4*>(sm + WH + sw128_chunk_off(r, ch, 64)) = hi;
             *reinterpret_cast<uint4*>(sm + WL + sw128_chunk_off(r, ch, 64)) = lo;
-            stc::split8(kk, hi, lo);
+            split_bf16x8(kk, hi, lo);
             *reinterpret_cast<uint4*>(sm + KH + sw128_chunk_off(r, ch, 64)) = hi;
             *reinterpret_cast<uint4*>(sm + KL + sw128_chunk_off(r, ch, 64)) = lo;
         }
@@ -417,7 +403,7 @@ __global__ void __launch_bounds__(stc::kThreads, 1) state_prop_tc_kernel(
                 const float sv = __uint_as_float(v[i]);
                 if (store_cs) chunk_states[(chunk_id * H + h) * kHeadDim * kHeadDim + (int64_t)c * kHeadDim + j] = sv;
                 uint16_t hi, lo;
-                stc::split1(sv, hi, lo);
+                split_bf16(sv, hi, lo);
                 *reinterpret_cast<uint16_t*>(sm + SH + sw128_off(c, j, 128)) = hi;
                 *reinterpret_cast<uint16_t*>(sm + SL + sw128_off(c, j, 128)) = lo;
                 v[i] = __float_as_uint(sv * sGC[c]);
@@ -466,7 +452,7 @@ __global__ void __launch_bounds__(stc::kThreads, 1) state_prop_tc_kernel(
                     u_out[idx] = uv;
                 }
                 uint16_t hi, lo;
-                stc::split1(uv, hi, lo);
+                split_bf16(uv, hi, lo);
                 *reinterpret_cast<uint16_t*>(sm + UH + sw128_off(r, j, 64)) = hi;
                 *reinterpret_cast<uint16_t*>(sm + UL + sw128_off(r, j, 64)) = lo;
             }

@@ -136,6 +136,40 @@ __device__ __forceinline__ void prefetch_rows_l2(const void* base, int64_t ld_by
     }
 }
 
+// ---- split-bf16 operands of the tensor-core stages ----
+// x = hi + lo with hi = bf16(x) and lo = bf16(x - hi), both rounded to nearest even: a product
+// taken as hi.hi + hi.lo + lo.hi (fp32 accumulation) keeps about 16 mantissa bits.
+__device__ __forceinline__ void split_bf16(float x, uint16_t& hi, uint16_t& lo) {
+    const __nv_bfloat16 hb = __float2bfloat16_rn(x);
+    hi = __bfloat16_as_ushort(hb);
+    lo = __bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(hb)));
+}
+// Eight values -> the high and the low parts as two 16-byte chunks (element 0 in the low half).
+__device__ __forceinline__ void split_bf16x8(const float (&x)[8], uint4& hi, uint4& lo) {
+    uint16_t a[8], b[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) split_bf16(x[i], a[i], b[i]);
+    hi = make_uint4(a[0] | ((uint32_t)a[1] << 16), a[2] | ((uint32_t)a[3] << 16), a[4] | ((uint32_t)a[5] << 16),
+                    a[6] | ((uint32_t)a[7] << 16));
+    lo = make_uint4(b[0] | ((uint32_t)b[1] << 16), b[2] | ((uint32_t)b[3] << 16), b[4] | ((uint32_t)b[5] << 16),
+                    b[6] | ((uint32_t)b[7] << 16));
+}
+// Eight consecutive fp32 values (16-byte aligned source).
+__device__ __forceinline__ void load8_f32(const float* src, float (&x)[8]) {
+    const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+// Eight consecutive bf16 values widened to fp32 (16-byte aligned source).
+__device__ __forceinline__ void load8_bf16(const __nv_bfloat16* src, float (&x)[8]) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
 struct Identity {
     __device__ float operator()(int, int, float v) const { return v; }
 };
