@@ -105,12 +105,15 @@ kda_status kda_fwd(const void* q, const void* k, const void* v,
 #define KDA_FUSED_MIN_LOWER_BOUND (-5.3f)
 
 /*
- * kda_fwd_staged -- the same forward as four separate kernels with fp32 CUDA-core
- * arithmetic and intermediates in a caller-provided workspace:
+ * kda_fwd_staged -- the same forward as four separate kernels with intermediates in a
+ * caller-provided workspace:
  *   (a) gate pre-pass: Gamma = in-chunk inclusive cumsum of log a;
  *   (b) intra-chunk WY: A, T = (I + A)^-1, W = T diag(beta)(gamma*K), U~ = T diag(beta) V, P;
  *   (c) state propagation: U = U~ - W S_c, S_{c+1} = Diag(gamma_C) S_c + Khat^T U;
  *   (d) output: O = scale ((gamma*Q) S_c + P U).
+ * (a), (b) and (d) are fp32 CUDA-core kernels, every intra-chunk decay formed pair by pair (exact
+ * for any gate).  (c) runs on the tensor cores with the state in fp32 and bf16 high + low operand
+ * parts (about 16 mantissa bits per product).
  * Chunks are 64 tokens, restarting at every sequence start.
  * workspace: device buffer of at least kda_staged_workspace_size(dims) bytes,
  * 256-byte aligned.  Its layout (offsets from kda_staged_workspace_layout) is
@@ -263,7 +266,9 @@ kda_status kda_state_affine(const float* A, const float* S, const float* B, floa
  *       differences), dq, dk, dbeta, then d log a (dGamma summed from the chunk's end) and
  *       the gate's chain rule (zero where the lower_bound clamp is active);
  *   (6) dA_log and ddt_bias summed over chunks in a fixed order (deterministic).
- * fp32 CUDA-core arithmetic; no atomics, so results are bitwise reproducible.
+ * Stages (2), (3) and the state propagation of (1) run on the tensor cores with fp32
+ * accumulation and bf16 high + low operand parts (about 16 mantissa bits per product); the
+ * rest is fp32 CUDA-core arithmetic.  No atomics, so results are bitwise reproducible.
  *
  * Inputs q ... cu_seqlens, lower_bound, scale, dims: exactly those of the kda_fwd call.
  *   d_out          bf16 [Ttot, H, 128]       gradient of out
