@@ -3,7 +3,9 @@
 // TMEM read-back layout against a host matmul.  Not part of the library.
 //
 // D[M][N] = A[M][K] * B[N][K]^T (negated when neg_b), fp32 accumulation.
-// A, B arrive as fp32 values that 16-bit floats represent exactly.
+// A, B arrive as fp32 values that 16-bit floats represent exactly.  With a_tmem, A is
+// written to tensor memory (row m in lane m, elements 2j and 2j+1 packed into column j)
+// and the MMA reads it from there.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -19,7 +21,7 @@ constexpr int kMaxM = 128, kMaxN = 256, kMaxK = 128;
 
 __global__ void __launch_bounds__(128) probe_kernel(const float* A, const float* B, float* D,
                                                     int M, int N, int K, int a_mn, int b_mn,
-                                                    int bf16, int neg_b, int* status) {
+                                                    int bf16, int neg_b, int a_tmem, int* status) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -47,20 +49,49 @@ __global__ void __launch_bounds__(128) probe_kernel(const float* A, const float*
         mbar_init_fence();
     }
     if (warp == 0) {
-        tmem_alloc(&tmem_base, 256);
+        tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
     }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tbase = tmem_base;
+    constexpr uint32_t kAcol = 256;   // A's columns in TMEM (D uses 0 .. N-1)
+    if (a_tmem) {
+        // row 32 * warp + lane of A into lane quarter `warp`, two 16-bit elements per column
+        const int m = warp * 32 + lane;
+        for (int c0 = 0; c0 < K / 2; c0 += 16) {
+            uint32_t r[16];
+            for (int j = 0; j < 16; ++j) {
+                const float lo = A[m * K + 2 * (c0 + j)], hi = A[m * K + 2 * (c0 + j) + 1];
+                uint32_t w;
+                if (bf16) {
+                    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+                    w = *reinterpret_cast<uint32_t*>(&v);
+                } else {
+                    __half2 v = __floats2half2_rn(lo, hi);
+                    w = *reinterpret_cast<uint32_t*>(&v);
+                }
+                r[j] = w;
+            }
+            tmem_st16(taddr(tbase, warp, kAcol + c0), r);
+        }
+        tmem_wait_st();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
     if (tid == 0) {
         const uint32_t idesc = idesc_f16(M, N, bf16 != 0, a_mn != 0, b_mn != 0, neg_b != 0);
         const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
         for (int ks = 0; ks < K / 16; ++ks) {
-            const uint64_t ad = a_mn ? desc_mnmajor(a0, K, ks) : desc_kmajor(a0, M, ks);
             const uint64_t bd = b_mn ? desc_mnmajor(b0, K, ks) : desc_kmajor(b0, N, ks);
-            mma_f16(tbase, ad, bd, idesc, ks > 0 ? 1u : 0u);
+            if (a_tmem) {
+                mma_f16_ts(tbase, tbase + kAcol + (uint32_t)ks * 8u, bd, idesc, ks > 0 ? 1u : 0u);
+            } else {
+                const uint64_t ad = a_mn ? desc_mnmajor(a0, K, ks) : desc_kmajor(a0, M, ks);
+                mma_f16(tbase, ad, bd, idesc, ks > 0 ? 1u : 0u);
+            }
         }
         mma_commit(&bar);
     }
@@ -83,20 +114,21 @@ __global__ void __launch_bounds__(128) probe_kernel(const float* A, const float*
     }
     fence_before_sync();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tbase, 256);
+    if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
 }  // namespace
 
 extern "C" int umma_probe(const float* A, const float* B, float* D, int M, int N, int K, int a_mn,
-                          int b_mn, int bf16, int neg_b, int* status) {
+                          int b_mn, int bf16, int neg_b, int a_tmem, int* status) {
     if (!(M == 64 || M == 128) || N < 16 || N > kMaxN || N % 16 || K < 16 || K > kMaxK || K % 16)
         return -1;
+    if (a_tmem && (M != 128 || a_mn)) return -1;   // a TMEM operand is 128 lanes, one row per lane
     const int smem = kMaxM * kMaxK * 2 + kMaxN * kMaxK * 2 + 1024;
     if (cudaFuncSetAttribute(probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
         return -2;
-    probe_kernel<<<1, 128, smem>>>(A, B, D, M, N, K, a_mn, b_mn, bf16, neg_b, status);
+    probe_kernel<<<1, 128, smem>>>(A, B, D, M, N, K, a_mn, b_mn, bf16, neg_b, a_tmem, status);
     if (cudaGetLastError() != cudaSuccess) return -3;
     return cudaDeviceSynchronize() == cudaSuccess ? 0 : -4;
 }

@@ -29,25 +29,31 @@ def _lib():
                        check=True)
     lib = ctypes.CDLL(OUT)
     lib.umma_probe.restype = ctypes.c_int
-    lib.umma_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 + [ctypes.c_void_p]
+    lib.umma_probe.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 8 + [ctypes.c_void_p]
     return lib
 
 
-# (M, N, K, a_mn, b_mn, bf16, neg_b): the shapes and majors the fused kernel uses
+# (M, N, K, a_mn, b_mn, bf16, neg_b, a_tmem): the shapes, majors and operand sources the
+# kernels use
 CASES = [
-    (128, 160, 128, 0, 0, 1, 0),   # A/P: [RK;RQ] x [XD;C1;C2;C3]^T, bf16, both K-major
-    (64, 128, 64, 0, 1, 0, 0),     # W = T * BGK: A K-major, B MN-major, M = 64
-    (128, 64, 64, 1, 0, 0, 0),     # U~^T = BV^T T^T: A MN-major
-    (128, 64, 128, 1, 0, 0, 1),    # U^T -= S^T W^T: negated B
-    (128, 128, 64, 1, 0, 0, 0),    # S += Khat^T U
-    (128, 64, 64, 0, 0, 0, 0),     # O^T += U^T P^T
+    (128, 160, 128, 0, 0, 1, 0, 0),   # A/P: [RK;RQ] x [XD;C1;C2;C3]^T, bf16, both K-major
+    (64, 128, 64, 0, 1, 0, 0, 0),     # W = T * BGK: A K-major, B MN-major, M = 64
+    (128, 64, 64, 1, 0, 0, 0, 0),     # U~^T = BV^T T^T: A MN-major
+    (128, 64, 128, 1, 0, 0, 1, 0),    # U^T -= S^T W^T: negated B
+    (128, 128, 64, 1, 0, 0, 0, 0),    # S += Khat^T U
+    (128, 64, 64, 0, 0, 0, 0, 0),     # O^T += U^T P^T
+    # A read from tensor memory (the transposed state products)
+    (128, 128, 128, 0, 0, 0, 0, 1),   # [O | Y]^T = S^T [gamma Q ; -beta gamma K]^T
+    (128, 64, 64, 0, 0, 0, 0, 1),     # U^T = Y^T T^T
+    (128, 192, 64, 0, 1, 0, 0, 1),    # [S | O]^T += U^T [Khat | P^T], B MN-major with N = 192
+    (128, 64, 32, 0, 0, 1, 0, 1),     # bf16 operands from tensor memory
 ]
 
 
-@pytest.mark.parametrize("M,N,K,a_mn,b_mn,bf16,neg_b", CASES)
-def test_umma_layout(M, N, K, a_mn, b_mn, bf16, neg_b):
+@pytest.mark.parametrize("M,N,K,a_mn,b_mn,bf16,neg_b,a_tmem", CASES)
+def test_umma_layout(M, N, K, a_mn, b_mn, bf16, neg_b, a_tmem):
     lib = _lib()
-    rng = np.random.default_rng(M * 7 + N * 3 + K + a_mn * 11 + b_mn * 13 + neg_b)
+    rng = np.random.default_rng(M * 7 + N * 3 + K + a_mn * 11 + b_mn * 13 + neg_b + a_tmem * 17)
     A = rng.integers(-8, 9, size=(M, K)).astype(np.float32) / 8
     B = rng.integers(-8, 9, size=(N, K)).astype(np.float32) / 8
     dA = torch.from_numpy(A).cuda()
@@ -55,7 +61,7 @@ def test_umma_layout(M, N, K, a_mn, b_mn, bf16, neg_b):
     dD = torch.full((M, N), float("nan"), device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     rc = lib.umma_probe(dA.data_ptr(), dB.data_ptr(), dD.data_ptr(), M, N, K, a_mn, b_mn, bf16,
-                        neg_b, st.data_ptr())
+                        neg_b, a_tmem, st.data_ptr())
     assert rc == 0
     assert int(st.item()) == 0, "MMA completion wait timed out"
     ref = (A.astype(np.float64) @ B.astype(np.float64).T) * (-1 if neg_b else 1)
