@@ -94,6 +94,8 @@ def _load():
                                        ctypes.c_size_t, vp]
     lib.kda_decode.restype = ctypes.c_int
     lib.kda_decode.argtypes = [vp] * 7 + [f32, f32, vp, vp, ctypes.c_int32, ctypes.c_int32, vp]
+    lib.kda_selftest_wait_timeout.restype = ctypes.c_int
+    lib.kda_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp, vp]
     return lib
 
 
@@ -104,7 +106,8 @@ EXPORTED = ("kda_fwd", "kda_fwd_staged", "kda_staged_workspace_size",
             "kda_staged_workspace_layout", "kda_strerror", "kda_check_device_error",
             "kda_last_device_error_bits", "kda_version", "kda_fwd_staged_noalloc",
             "kda_noalloc_scratch_bytes", "kda_decode", "kda_gdn_fwd", "kda_gdn_decode",
-            "kda_state_affine", "kda_bwd", "kda_bwd_workspace_size", "kda_fwd_workspace_size")
+            "kda_state_affine", "kda_bwd", "kda_bwd_workspace_size", "kda_fwd_workspace_size",
+            "kda_selftest_wait_timeout")
 
 
 def lib() -> ctypes.CDLL:
@@ -386,6 +389,18 @@ def kda_bwd_workspace_size(q: torch.Tensor, cu_seqlens: Optional[torch.Tensor] =
         batch = q.shape[0]
     dims = make_dims(H, total_tokens=total, cu_seqlens=cu_seqlens, batch=batch)
     return int(_lib.kda_bwd_workspace_size(dims, int(cu_seqlens is not None)))
+
+
+def kda_selftest_wait_timeout(limit_ns: int, observed: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Makes one bounded device-side wait run out on purpose (diagnostics; see include/kda.h).
+    observed: optional int32 CUDA tensor of 2 elements."""
+    if observed is not None:
+        _check_tensor("observed", observed, torch.int32, observed.device)
+        if observed.numel() < 2:
+            raise ValueError("observed needs 2 elements")
+    st = _lib.kda_selftest_wait_timeout(int(limit_ns), _ptr(observed), _stream_ptr(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_selftest_wait_timeout")
 
 
 def kda_check_device_error(stream=None) -> int:

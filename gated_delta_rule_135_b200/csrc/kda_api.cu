@@ -13,9 +13,11 @@
 
 #include "kda_staged.cuh"
 #include "kda_fused.cuh"
+#include "kda_pipe.cuh"
 #include "kda_decode.cuh"
 #include "kda_cp.cuh"
 #include "kda_backward.cuh"
+#include "kda_selftest.cuh"
 
 namespace {
 
@@ -229,7 +231,7 @@ kda_status kda_fwd(const void* q, const void* k, const void* v, const float* g, 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (a.total_tokens == 0) return copy_states_only(a, s);
     if (kda::fused_supported(lower_bound))
-        return kda::launch_fused(a, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+        return kda::launch_pipe(a, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     kda::StagedLayout L = kda::staged_layout(a.total_tokens, a.H, a.N);
     void* ws = nullptr;
     if (cudaMallocAsync(&ws, L.total, s) != cudaSuccess) return KDA_ERR_CUDA;
@@ -412,6 +414,17 @@ kda_status kda_bwd(const void* q, const void* k, const void* v, const float* g, 
     cudaError_t err = kda::launch_bwd(a, b, static_cast<char*>(ws), B, s);
     cudaError_t err2 = cudaFreeAsync(ws, s);
     return (err == cudaSuccess && err2 == cudaSuccess) ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_selftest_wait_timeout(uint64_t limit_ns, uint32_t* observed, kda_stream_t stream) {
+    if (limit_ns < 1 || limit_ns > 1000000000ull) return KDA_ERR_INVALID_ARG;
+    if (observed && !aligned4(observed)) return KDA_ERR_ALIGNMENT;
+    kda_status st = device_ok();
+    if (st != KDA_OK) return st;
+    return kda::launch_wait_timeout_selftest(limit_ns, observed, reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? KDA_OK
+               : KDA_ERR_CUDA;
 }
 
 const char* kda_strerror(kda_status status) {

@@ -93,5 +93,7 @@ cudaError_t launch_fused(const StagedArgs& a, cudaStream_t stream);
 // Scalar-gate (Gated DeltaNet) variant: a.g is [Ttot][H], a.dt_bias [H]; any lower bound.
 cudaError_t launch_fused_gdn(const StagedArgs& a, cudaStream_t stream);
 bool fused_supported(float lower_bound);
+// The warp-specialised product kernel of kda_fwd (same arguments and requirement on lower_bound).
+cudaError_t launch_pipe(const StagedArgs& a, cudaStream_t stream);
 
 }  // namespace kda

@@ -1,0 +1,1392 @@
+// kda_pipe.cuh -- the product KDA chunked-prefill kernel (kda_fwd): persistent,
+// warp-specialised, sm_100a.
+//
+// One CTA per SM walks a static longest-first "snake" schedule of (sequence, head) units.
+// Its 16 warps have three roles that work on consecutive 64-token chunks at once:
+//
+//   chain warps 0-3     thread v owns value column v of the state.  The state lives in TMEM
+//                       transposed (S^T: lane v, column c) in fp32, lane v scaled by its own
+//                       power of two 2^-sigma_v: every column of S evolves on its own and the
+//                       recurrence is linear in it, so the scaling is exact and keeps every
+//                       fp16 MMA operand derived from the state inside the fp16 range.  Per
+//                       chunk (A operands read straight from TMEM, B operands from shared memory):
+//                         S^T -> fp16 (TMEM);  S^T <- S^T Diag(gamma_C)  (after the next MMA issues)
+//                         [O | Y]^T  = S^T [gamma Q ; -beta gamma K]^T                    K = 128
+//                         Y^T       += 2^-sigma (beta V)^T  -> fp16 (TMEM)
+//                         U^T        = Y^T T^T                                             K = 64
+//                         U^T -> fp16 (TMEM);  [S | O]^T += U^T [Khat | P^T]              N = 192
+//                         O^T -> bf16 out (times scale 2^sigma_v)
+//   aux warps 4-7       beta, V^T, the exact diagonal q_r . k_r of P, the A/P MMA issue, the
+//                       A / P read-out (with all front-end warps) and T = (I + A)^-1
+//   element warps 8-15  gate and decay factors (thread: 4 channels x 8 tokens) and every
+//                       decayed operand tile
+//
+// Y = beta V - beta gamma K S and U = T Y is the WY/UT form U = T diag(beta)(V - (gamma K) S)
+// of the chunk (U~ - W S with the product by T taken last), so that the part of the chain that
+// needs the state does not wait for the triangular solve: the front end (aux + element warps)
+// builds chunk j+1 while the chain warps finish chunk j.
+//
+// Decay factors (16-token blocks, R_r = e^{Gamma_r - Gamma_(block start)} <= 1 and
+// E_r = e^{Gamma_(block end) - Gamma_r} <= 1, formed as running products of a_t): the A/P MMA
+// (bf16, M = 128 x N = 160) multiplies [k R ; q R] by the diagonal-block operand k E / R_block
+// (>= 1, at most e^{16 |lower_bound|}) and the block-distance operands k E, k E F2, k E F3.
+// So the kernel requires lower_bound >= -5.3 (16 x 5.3 = 84.8 < 87); steeper gates take the
+// staged path.  P's main diagonal (no decay, the dominant output term) is taken exactly in fp32.
+//
+// Operand precision: decay blocks bf16, everything that multiplies T, S, Y, U or P in fp16,
+// accumulation and the carried state in fp32.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+#include "umma.cuh"
+#include "warp_mma.cuh"
+
+namespace kda {
+namespace pipe {
+
+using namespace umma;
+
+constexpr int kThreads = 512;
+constexpr int kFeThreads = 384;          // warps 4-15
+constexpr int kAuxWarp0 = 4, kElemWarp0 = 8;
+// named barriers (0 is __syncthreads)
+constexpr uint32_t BAR_FE = 1, BAR_CHAIN = 2, BAR_AUX = 3;
+
+// ---- shared memory (bytes from a 1024-aligned base) ----
+constexpr uint32_t IN_Q = 0;           // bf16 [64][128] row-major TMA boxes
+constexpr uint32_t IN_K = 16384;
+constexpr uint32_t IN_V = 32768;
+constexpr uint32_t IN_BYTES = 49152;
+constexpr uint32_t AP_A = 49152;       // bf16 K-major [128 rows][128]: k R rows 0-63, q R rows 64-127
+constexpr uint32_t AP_B = 81920;       // bf16 K-major [160 rows][128]: XD | C1 | C2 | C3
+constexpr int kF32Pitch = 68;          // fp32 row pitch of A32 / T32
+constexpr uint32_t A32 = AP_A;         // fp32 [64][68] beta-scaled A (after the A/P MMA)
+constexpr uint32_t T32 = AP_A + 17408; // fp32 [64][68] T
+constexpr uint32_t B1 = 122880;        // fp16 K-major [128 rows][128]: gamma q rows 0-63, -beta gamma k 64-127
+constexpr uint32_t B2 = 155648;        // fp16 MN-major, K = 64 tokens: Khat (c 0-63 | c 64-127) | P^T
+constexpr uint32_t KH = B2;
+constexpr uint32_t PT = B2 + 16384;
+constexpr uint32_t VT = 180224;        // bf16 [128 v][64 i]: 128-byte rows, 16-byte chunk j at j ^ (v & 7)
+constexpr uint32_t T16 = 196608;       // fp16 K-major [64 r][64 i]
+constexpr uint32_t MISC = 204800;
+constexpr uint32_t S_BETA = MISC;              // fp32 [2][64] (by chunk parity)
+constexpr uint32_t S_GC = MISC + 512;          // fp32 [2][128] gamma_C = e^{Gamma_63}
+constexpr uint32_t S_PTOT = MISC + 1536;       // fp32 [4][128] per-block products of a
+constexpr uint32_t S_PD = MISC + 3584;         // fp32 [2][64] halves of q_r . k_r
+constexpr uint32_t S_ORDER = MISC + 4096;      // int16 [kSortLimit]
+constexpr int kSortLimit = 512;
+constexpr uint32_t S_META = S_ORDER + 2 * kSortLimit;   // int32 [2][8] chunk metadata
+constexpr uint32_t S_BARS = S_META + 64;                // u64 [8]
+constexpr uint32_t S_TMEM = S_BARS + 64;                // u32 tmem base, u32 abort flag
+constexpr uint32_t S_PH = S_TMEM + 16;                  // u64 [kPhases + 2] (phase-clock builds)
+constexpr int kPhases = 18;
+#ifdef KDA_PHASE_CLOCKS
+constexpr uint32_t SMEM_BYTES = S_PH + 8 * (kPhases + 2);
+#else
+constexpr uint32_t SMEM_BYTES = S_PH;
+#endif
+constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+static_assert(T32 + 64 * kF32Pitch * 4 <= B1, "solve scratch inside the A/P operand region");
+
+// ---- TMEM columns ----
+constexpr uint32_t TM_S = 0;      // S^T fp32 [128 v][128 c]
+constexpr uint32_t TM_O = 128;    // O^T fp32 [v][64 r]
+constexpr uint32_t TM_Y = 192;    // Y^T then U^T, fp32 [v][64 i]
+constexpr uint32_t TM_H = 256;    // fp16 A operands: S^T (64 columns); then Y^T (+0) and U^T (+32)
+constexpr uint32_t TM_AP = 320;   // A/P accumulator [128 rows][160]
+constexpr uint32_t TM_COLS = 512;
+
+constexpr uint32_t IDESC_AP = idesc_f16(128, 160, true, false, false);
+constexpr uint32_t IDESC_OY = idesc_f16(128, 128, false, false, false);
+constexpr uint32_t IDESC_T = idesc_f16(128, 64, false, false, false);
+constexpr uint32_t IDESC_SO = idesc_f16(128, 192, false, false, true);
+
+// fp16 values at or above this magnitude trigger a rescale of the lane (2^15 leaves room below
+// the fp16 maximum 65504); a state lane below kSmall with sigma > 0 is scaled back up
+constexpr float kRangeHi = 32768.f;
+constexpr float kStateHi = 16384.f;
+constexpr float kStateLo = 64.f;
+constexpr int kSigmaMax = 100;
+
+struct Params {
+    const float* g;
+    const float* beta;
+    const float* A_log;
+    const float* dt_bias;
+    float lower_bound;
+    float scale;
+    const float* initial_state;
+    const int32_t* cu_seqlens;
+    __nv_bfloat16* out;
+    float* final_state;
+    int64_t seqlen;
+    int64_t total_tokens;
+    int H;
+    int N;
+};
+
+#ifdef KDA_PHASE_CLOCKS
+__device__ unsigned long long g_pipe_phase_cycles[kPhases];
+// thread `who` adds the cycles since its role's previous mark to slot i
+#define PIPE_MARK(who, slot, i)                                            \
+    do {                                                                   \
+        if (threadIdx.x == (who)) {                                        \
+            const long long now_ = clock64();                              \
+            sPh[i] += (unsigned long long)(now_ - sPh[kPhases + (slot)]);  \
+            sPh[kPhases + (slot)] = (unsigned long long)now_;              \
+        }                                                                  \
+    } while (0)
+#else
+#define PIPE_MARK(who, slot, i) do { } while (0)
+#endif
+
+// ---- small helpers ----
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+// fp16 pair, saturating at +-65504 (never inf)
+__device__ __forceinline__ uint32_t pack_f16s(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+// running max of |x| over fp16 pairs (sign bits of the result are meaningless)
+__device__ __forceinline__ uint32_t hmax_abs(uint32_t m, uint32_t h) {
+    uint32_t r;
+    asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(m), "r"(h));
+    return r;
+}
+__device__ __forceinline__ float hmax_to_float(uint32_t m) {
+    const __half2 h = *reinterpret_cast<const __half2*>(&m);
+    return fmaxf(fabsf(__low2float(h)), fabsf(__high2float(h)));
+}
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ float fast_ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float fast_lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float fast_rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// 2^e for an integer e in [-126, 127]
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+// floor(log2 |x|) for a normal nonzero x
+__device__ __forceinline__ int ilog2f(float x) { return (int)((__float_as_uint(x) >> 23) & 0xFFu) - 127; }
+
+__device__ __forceinline__ void st_v2(unsigned char* base, uint32_t off, uint32_t a, uint32_t b) {
+    *reinterpret_cast<uint2*>(base + off) = make_uint2(a, b);
+}
+// Shared-memory stores the compiler may move later shared loads above: the operand tiles
+// written in one phase are never read back in it (the phase ends with a fence and a barrier,
+// which order them before every later use).
+__device__ __forceinline__ void st_tile2(const unsigned char* base, uint32_t off, uint32_t a, uint32_t b) {
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(smem_u32(base) + off), "r"(a), "r"(b));
+}
+__device__ __forceinline__ void st_tile4(const unsigned char* base, uint32_t off, uint32_t a, uint32_t b,
+                                         uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(base) + off), "r"(a), "r"(b), "r"(c),
+                 "r"(d));
+}
+__device__ __forceinline__ void st_tile_h(const unsigned char* base, uint32_t off, uint16_t a) {
+    asm volatile("st.shared.b16 [%0], %1;" ::"r"(smem_u32(base) + off), "h"(a));
+}
+__device__ __forceinline__ void st_v4(unsigned char* base, uint32_t off, uint32_t a, uint32_t b,
+                                      uint32_t c, uint32_t d) {
+    *reinterpret_cast<uint4*>(base + off) = make_uint4(a, b, c, d);
+}
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Named barrier that also ORs a predicate over the participating threads (uniform result).
+__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0u;
+}
+
+// Every lane of the warp waits (bounded) for the phase, so each has acquired what the phase
+// guards; the warp agrees on the outcome.  A timeout is recorded in the device error word.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+    if (!ok && (threadIdx.x & 31) == 0) record_error(KDA_DEVERR_TIMEOUT);
+    return ok;
+}
+
+// ---- schedule ----
+// Slot k of CTA b over G CTAs (snake order: even slots forward, odd slots backward).
+__device__ __forceinline__ int unit_of(int k, int b, int G) {
+    return (k & 1) ? (k + 1) * G - 1 - b : k * G + b;
+}
+
+struct Cursor {
+    int k, h, n;
+    int64_t bos, eos, t0;
+    bool valid;
+};
+
+__device__ __forceinline__ void decode_unit(const Params& p, const int16_t* order, int u, int* n, int* h,
+                                            int64_t* bos, int64_t* eos) {
+    const int rank = u / p.H;
+    *h = u - rank * p.H;
+    *n = (p.N <= kSortLimit) ? order[rank] : rank;
+    seq_range(p.cu_seqlens, *n, p.seqlen, p.total_tokens, bos, eos);
+}
+
+// The first chunk of the first non-empty unit at slot >= k0 (invalid if none).
+__device__ __noinline__ Cursor unit_from(const Params& p, const int16_t* order, int b, int G, int units, int k0) {
+    Cursor c;
+    c.valid = false;
+    for (int k = k0; (int64_t)k * G < units; ++k) {
+        const int u = unit_of(k, b, G);
+        if (u >= units) continue;
+        decode_unit(p, order, u, &c.n, &c.h, &c.bos, &c.eos);
+        if (c.eos > c.bos) {
+            c.k = k;
+            c.t0 = c.bos;
+            c.valid = true;
+            return c;
+        }
+    }
+    return c;
+}
+
+__device__ __forceinline__ Cursor next_chunk(const Params& p, const int16_t* order, int b, int G, int units,
+                                             Cursor c) {
+    if (c.t0 + kChunk < c.eos) {
+        c.t0 += kChunk;
+        return c;
+    }
+    return unit_from(p, order, b, G, units, c.k + 1);
+}
+
+__device__ __forceinline__ void issue_chunk_loads(unsigned char* sm, uint64_t* bar, const CUtensorMap* tq,
+                                                  const CUtensorMap* tk, const CUtensorMap* tv, int h,
+                                                  int64_t t0) {
+    mbar_arrive_expect_tx(bar, IN_BYTES);
+    const int x = h * kHeadDim, y = (int)t0;
+    tma_load_2d(sm + IN_Q, tq, x, y, bar);
+    tma_load_2d(sm + IN_K, tk, x, y, bar);
+    tma_load_2d(sm + IN_V, tv, x, y, bar);
+}
+__device__ __forceinline__ void prefetch_chunk(const CUtensorMap* tq, const CUtensorMap* tk,
+                                               const CUtensorMap* tv, const CUtensorMap* tg, int h,
+                                               int64_t t0) {
+    const int x = h * kHeadDim, y = (int)t0;
+    tma_prefetch_2d(tq, x, y);
+    tma_prefetch_2d(tk, x, y);
+    tma_prefetch_2d(tv, x, y);
+    tma_prefetch_2d(tg, x, y);
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---- element warps: gate ----
+// a[i][e] = a_t for token r0 + i, channel c0 + e: a = max(2^(-e^A_log * log2(1 + 2^x2)), e^lb)
+// with x2 = (g + dt_bias) log2 e, i.e. e^(-e^A_log softplus(g + dt_bias)) clamped at e^lb.
+// Rows past the chunk's valid length get a = 1.
+__device__ __forceinline__ void gate_tokens(const Params& p, int h, int64_t t0, int L, int c0, int r0,
+                                            float (&a)[8][4]) {
+    const float nexpA = -expf(p.A_log[h]);
+    const float alb = fast_ex2(p.lower_bound * kLog2e);
+    const float4 db = *reinterpret_cast<const float4*>(p.dt_bias + h * kHeadDim + c0);
+    const float2 db01 = make_float2(db.x * kLog2e, db.y * kLog2e), db23 = make_float2(db.z * kLog2e, db.w * kLog2e);
+    const float2 l2e = make_float2(kLog2e, kLog2e);
+    float4 gv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = r0 + i;
+        gv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < L)
+            gv[i] = __ldg(reinterpret_cast<const float4*>(p.g + ((t0 + r) * p.H + h) * kHeadDim + c0));
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float2 x01 = __ffma2_rn(make_float2(gv[i].x, gv[i].y), l2e, db01);
+        const float2 x23 = __ffma2_rn(make_float2(gv[i].z, gv[i].w), l2e, db23);
+        const float2 s01 = __fadd2_rn(make_float2(1.f, 1.f), make_float2(fast_ex2(x01.x), fast_ex2(x01.y)));
+        const float2 s23 = __fadd2_rn(make_float2(1.f, 1.f), make_float2(fast_ex2(x23.x), fast_ex2(x23.y)));
+        const float2 l01 = __fmul2_rn(make_float2(nexpA, nexpA), make_float2(fast_lg2(s01.x), fast_lg2(s01.y)));
+        const float2 l23 = __fmul2_rn(make_float2(nexpA, nexpA), make_float2(fast_lg2(s23.x), fast_lg2(s23.y)));
+        const bool live = r0 + i < L;
+        a[i][0] = live ? fmaxf(fast_ex2(l01.x), alb) : 1.f;
+        a[i][1] = live ? fmaxf(fast_ex2(l01.y), alb) : 1.f;
+        a[i][2] = live ? fmaxf(fast_ex2(l23.x), alb) : 1.f;
+        a[i][3] = live ? fmaxf(fast_ex2(l23.y), alb) : 1.f;
+    }
+}
+
+// Decay factors of an element thread's 8 tokens (4 channels): E[i] = product of a over the
+// tokens after i up to the block end, and the initial value of the running product
+// R = a-product from the block start (R_i = R0 * a_0 * ... * a_i).  po is the product over the
+// other 8-token half of the block (before this half for the second half, after it for the first).
+__device__ __forceinline__ void decay_suffix(const float (&a)[8][4], const float (&po)[4], bool second_half,
+                                             float (&E)[8][4], float (&R0)[4]) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        E[7][e] = second_half ? 1.f : po[e];
+#pragma unroll
+        for (int i = 6; i >= 0; --i) E[i][e] = E[i + 1][e] * a[i + 1][e];
+        R0[e] = second_half ? po[e] : 1.f;
+    }
+}
+
+// ---- chain warps: rare range repairs (out of line: they cost no instruction-cache space on
+// the common path).  lane_base = TMEM address of the warp's lane quarter.
+
+// Every state lane value (TM_S) and O^T (TM_O) times 2^-d.
+__device__ __noinline__ void chain_rescale_state(uint32_t lane_base, int d) {
+    const float f = pow2i(-d);
+#pragma unroll 1
+    for (int cb = 0; cb < 6; ++cb) {
+        const uint32_t col = cb < 4 ? TM_S + 32u * cb : TM_O + 32u * (cb - 4);
+        uint32_t s[32];
+        tmem_ld32(lane_base + col, s);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s[j] = __float_as_uint(f * __uint_as_float(s[j]));
+        tmem_st32(lane_base + col, s);
+    }
+    tmem_wait_st();
+}
+
+// The TMEM loads and stores below are warp-collective (.sync.aligned): the whole warp calls these
+// repairs when any of its lanes needs one, and lanes that do not need it use a shift of 0.
+
+// A state lane left [kStateLo, kStateHi) (or saturated): choose the shift delta that brings its
+// fp32 maximum to [2^12, 2^13) (never below sigma = 0, never above kSigmaMax) and write the fp16
+// copy again.  Returns delta (0 where need is false); the caller adds it to sigma.
+__device__ __noinline__ int chain_state_reconvert(uint32_t lane_base, int sigma, bool need) {
+    float mx = 0.f;
+#pragma unroll 1
+    for (int cb = 0; cb < 4; ++cb) {
+        uint32_t s[32];
+        tmem_ld32(lane_base + TM_S + 32u * cb, s);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) mx = fmaxf(mx, fabsf(__uint_as_float(s[j])));
+    }
+    int delta = mx > 0.f ? ilog2f(mx) - 12 : -sigma;
+    if (delta < -sigma) delta = -sigma;
+    if (sigma + delta > kSigmaMax) delta = kSigmaMax - sigma;
+    if (!need) delta = 0;
+    const float f = pow2i(-delta);
+#pragma unroll 1
+    for (int cb = 0; cb < 4; ++cb) {
+        uint32_t s[32];
+        tmem_ld32(lane_base + TM_S + 32u * cb, s);
+        tmem_wait_ld();
+        uint32_t h16[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            h16[j] = pack_f16s(f * __uint_as_float(s[2 * j]), f * __uint_as_float(s[2 * j + 1]));
+        tmem_st16(lane_base + TM_H + 16u * cb, h16);
+    }
+    tmem_wait_st();
+    return delta;
+}
+
+// Y (with_beta_v: TM_Y plus 2^-sigma beta v of this lane's value column v) or U (TM_Y as is)
+// saturated its fp16 copy in a lane where need is true: shift that lane down so that its fp32
+// maximum lands in [2^12, 2^13), convert again into the fp16 columns at TM_H + col, and rescale
+// its state and O^T to match.  Returns the shift d (0 where need is false or the lane cannot move
+// further); the caller adds it to sigma.
+__device__ __noinline__ int chain_vals_reconvert(uint32_t lane_base, uint32_t col, const unsigned char* sm,
+                                                 int v, uint32_t slot, bool with_beta_v, int sigma, bool need) {
+    const float fs = pow2i(-sigma);
+    const float* be = reinterpret_cast<const float*>(sm + S_BETA) + slot * 64u;
+    float mx = 0.f;
+    int d = 0;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        const float f = pow2i(-d);
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+            uint32_t t[32];
+            tmem_ld32(lane_base + TM_Y + 32u * half, t);
+            tmem_wait_ld();
+            float x[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(t[j]);
+            if (with_beta_v) {
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const uint32_t c8 = (uint32_t)(4 * half + ch);
+                    const uint4 w = *reinterpret_cast<const uint4*>(sm + VT + (uint32_t)v * 128u +
+                                                                    ((c8 ^ ((uint32_t)v & 7u)) << 4));
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 vv = bf16x2_to_float2(ww[e]);
+                        x[8 * ch + 2 * e] = fmaf(fs * be[8 * c8 + 2 * e], vv.x, x[8 * ch + 2 * e]);
+                        x[8 * ch + 2 * e + 1] = fmaf(fs * be[8 * c8 + 2 * e + 1], vv.y, x[8 * ch + 2 * e + 1]);
+                    }
+                }
+            }
+            if (pass == 0) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) mx = fmaxf(mx, fabsf(x[j]));
+            } else {
+                uint32_t h16[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) h16[j] = pack_f16s(f * x[2 * j], f * x[2 * j + 1]);
+                tmem_st16(lane_base + col + 16u * half, h16);
+            }
+        }
+        if (pass == 0) {
+            d = ilog2f(mx) - 12;
+            if (sigma + d > kSigmaMax) d = kSigmaMax - sigma;
+            if (!need || d < 0) d = 0;
+        }
+    }
+    tmem_wait_st();
+    chain_rescale_state(lane_base, d);
+    return d;
+}
+
+// ---- the kernel ----
+__global__ void __launch_bounds__(kThreads, 1)
+kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                const Params p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = gridDim.x, b = blockIdx.x;
+    const int H = p.H;
+    const int units = p.N * H;
+
+    int16_t* sOrder = reinterpret_cast<int16_t*>(sm + S_ORDER);
+    int32_t* sMeta = reinterpret_cast<int32_t*>(sm + S_META);
+    uint64_t* bar_in = reinterpret_cast<uint64_t*>(sm + S_BARS);   // inputs landed (TMA)
+    uint64_t* bar_ap = bar_in + 1;       // A/P MMA done
+    uint64_t* bar_formed = bar_in + 2;   // chunk's B1, Khat, V^T, beta, gamma_C, metadata written
+    uint64_t* bar_t = bar_in + 3;        // chunk's P^T and T written
+    uint64_t* bar_y = bar_in + 4;        // [O | Y] MMA done
+    uint64_t* bar_u = bar_in + 5;        // U MMA done
+    uint64_t* bar_s = bar_in + 6;        // [S | O] MMA done (chunk's shared operands free again)
+    uint64_t* bar_apready = bar_in + 7;  // chunk's A/P operand tiles written (the chain issues the MMA)
+    uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + S_TMEM);
+    volatile uint32_t* sAbort = sTmem + 1;
+    volatile uint32_t* sEnd = sTmem + 2;   // set once the front end has no further chunk
+#ifdef KDA_PHASE_CLOCKS
+    volatile unsigned long long* sPh = reinterpret_cast<volatile unsigned long long*>(sm + S_PH);
+#endif
+
+    // ---- set-up ----
+    if (tid == 0) {
+        for (int i = 0; i < 8; ++i) mbar_init(bar_in + i, 1);
+        mbar_init_fence();
+        *sAbort = 0u;
+        *sEnd = 0u;
+    }
+    if (warp == 0) {
+        tmem_alloc(sTmem, TM_COLS);
+        tmem_relinquish();
+    }
+    if (p.N <= kSortLimit) {
+        for (int n = tid; n < p.N; n += kThreads) {
+            int64_t bn, en;
+            seq_range(p.cu_seqlens, n, p.seqlen, p.total_tokens, &bn, &en);
+            const int64_t ln = en - bn;
+            int rank = 0;
+            for (int m = 0; m < p.N; ++m) {
+                int64_t bm, em;
+                seq_range(p.cu_seqlens, m, p.seqlen, p.total_tokens, &bm, &em);
+                const int64_t lm = em - bm;
+                rank += (lm > ln) || (lm == ln && m < n);
+            }
+            sOrder[rank] = (int16_t)n;
+        }
+    }
+    // T16's blocks above the diagonal are never written by the solve: zero them once
+    for (int e = tid; e < 8192 / 16; e += kThreads) st_v4(sm, T16 + (uint32_t)e * 16u, 0u, 0u, 0u, 0u);
+#ifdef KDA_PHASE_CLOCKS
+    if (tid == 0)
+        for (int i = 0; i < kPhases + 2; ++i) sPh[i] = (i < kPhases) ? 0ull : (unsigned long long)clock64();
+#endif
+    __syncthreads();
+    // empty units: final state = initial state (the chain never sees them)
+    if (p.final_state) {
+        for (int k = 0; (int64_t)k * G < units; ++k) {
+            const int u = unit_of(k, b, G);
+            if (u >= units) continue;
+            int n, h;
+            int64_t bos, eos;
+            decode_unit(p, sOrder, u, &n, &h, &bos, &eos);
+            if (eos > bos) continue;
+            const int64_t off = ((int64_t)n * H + h) * kHeadDim * kHeadDim;
+            for (int e = tid; e < kHeadDim * kHeadDim / 4; e += kThreads) {
+                const float4 s = p.initial_state ? reinterpret_cast<const float4*>(p.initial_state + off)[e]
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                reinterpret_cast<float4*>(p.final_state + off)[e] = s;
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tbase = *sTmem;
+
+    if (warp < kAuxWarp0) {
+        // =============================== chain warps ===============================
+        const int v = tid;                       // value column = TMEM lane
+        const uint32_t lane_base = tbase + ((uint32_t)(warp * 32) << 16);
+        int sigma = 0;                           // this lane's state is stored times 2^-sigma
+        uint32_t cc = 0;                         // chunks started
+        bool have_prev = false;
+        int prev_h = 0, prev_n = 0, prev_L = 0, prev_last = 0;
+        int64_t prev_t0 = 0;
+        uint32_t issued_y = 0, issued_u = 0, issued_s = 0, done_s = 0, issued_ap = 0;   // thread 0's MMA commits
+        bool aborted = false;
+
+        // O^T (TMEM) of the previous chunk -> out, and its final state if it ended a unit.  Lane v
+        // holds column v of every output row; lanes v and v + 1 (v even) trade one value per pair of
+        // rows, so the even lane writes columns (v, v + 1) of even rows and the odd lane those of odd
+        // rows, as 4-byte stores (a warp writes 64 contiguous bytes per row).
+        auto retire_prev = [&]() {
+            const float sc = p.scale * pow2i(sigma);
+            const bool odd = (v & 1) != 0;
+            const int64_t row_stride = (int64_t)H * kHeadDim;
+            __nv_bfloat16* base = p.out + (prev_t0 * H + prev_h) * kHeadDim + (v & ~1) + (odd ? row_stride : 0);
+#pragma unroll 1
+            for (int cb = 0; cb < 2; ++cb) {
+                uint32_t o[32];
+                tmem_ld32(lane_base + TM_O + 32u * cb, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    const float e0 = sc * __uint_as_float(o[j]), e1 = sc * __uint_as_float(o[j + 1]);
+                    // even lane sends its odd-row value, odd lane its even-row value
+                    const float got = __shfl_xor_sync(0xffffffffu, odd ? e0 : e1, 1);
+                    const uint32_t w = odd ? pack_bf16(got, e1) : pack_bf16(e0, got);
+                    const int r = 32 * cb + j + (odd ? 1 : 0);
+                    if (r < prev_L)
+                        *reinterpret_cast<uint32_t*>(base + (int64_t)(32 * cb + j) * row_stride) = w;
+                }
+            }
+            if (prev_last && p.final_state) {
+                const float f = pow2i(sigma);
+                float* fs = p.final_state + ((int64_t)prev_n * H + prev_h) * kHeadDim * kHeadDim + v;
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
+                    uint32_t s[32];
+                    tmem_ld32(lane_base + TM_S + 32u * cb, s);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) fs[(32 * cb + j) * kHeadDim] = f * __uint_as_float(s[j]);
+                }
+            }
+        };
+        // fp32 values -> fp16 pairs at TMEM column `col` (count/2 columns) times 2^-d; returns max |fp16|
+        auto to_f16_tmem = [&](float (&x)[64], uint32_t col, float f) -> float {
+            uint32_t m = 0u;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t h16[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    h16[j] = pack_f16s(f * x[32 * half + 2 * j], f * x[32 * half + 2 * j + 1]);
+                    m = hmax_abs(m, h16[j]);
+                }
+                tmem_st16(lane_base + col + 16u * half, h16);
+            }
+            return hmax_to_float(m);
+        };
+
+        while (true) {
+            bool bad = false;
+            if (have_prev) {
+                bad |= !warp_wait(bar_s, (cc - 1) & 1u);
+                if (tid == 0 && !bad) done_s = issued_s;
+                fence_after_sync();
+                PIPE_MARK(0, 1, 9);
+                if (!bad) retire_prev();
+            }
+            PIPE_MARK(0, 1, 10);
+            // the front end's A/P MMA: its operand tiles are written early in the chunk, while
+            // the chain is idle here; issuing costs the issuing warp about 70 cycles per MMA
+            if (tid == 0) {
+                const bool ap_ok = mbar_wait_bounded(bar_apready, cc & 1u);
+                PIPE_MARK(0, 1, 11);
+                if (!ap_ok) {
+                    record_error(KDA_DEVERR_TIMEOUT);
+                    *sAbort = 1u;
+                } else if (*sEnd == 0u) {
+                    fence_after_sync();
+                    const uint32_t a0 = smem_u32(sm + AP_A), b0 = smem_u32(sm + AP_B);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
+                                ks > 0 ? 1u : 0u);
+                    mma_commit(bar_ap);
+                    ++issued_ap;
+                }
+            }
+            PIPE_MARK(0, 1, 12);
+            bad |= !warp_wait(bar_formed, cc & 1u);
+            const int32_t* meta = sMeta + (cc & 1u) * 8u;
+            const int m_valid = meta[0], m_h = meta[1], m_n = meta[2], m_t0 = meta[3], m_L = meta[4],
+                      m_first = meta[5], m_last = meta[6];
+            if (named_bar_or(BAR_CHAIN, 128, bad || *sAbort != 0u)) {
+                aborted = true;
+                break;
+            }
+            if (!m_valid) break;
+            PIPE_MARK(0, 1, 13);
+            if (m_first) {
+                // the unit's initial state (or zeros) into TMEM
+                sigma = 0;
+                const float* is = p.initial_state
+                    ? p.initial_state + ((int64_t)m_n * H + m_h) * kHeadDim * kHeadDim + v : nullptr;
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
+                    uint32_t s[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) s[j] = is ? __float_as_uint(is[(32 * cb + j) * kHeadDim]) : 0u;
+                    tmem_st32(lane_base + TM_S + 32u * cb, s);
+                }
+                tmem_wait_st();
+            }
+            // ---- S^T -> fp16 A operand (scale kept unless the lane leaves its range) ----
+            int delta = 0;
+            {
+                uint32_t m = 0u;
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
+                    uint32_t s[32];
+                    tmem_ld32(lane_base + TM_S + 32u * cb, s);
+                    tmem_wait_ld();
+                    uint32_t h16[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        h16[j] = pack_f16s(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1]));
+                        m = hmax_abs(m, h16[j]);
+                    }
+                    tmem_st16(lane_base + TM_H + 16u * cb, h16);
+                }
+                const float mh = hmax_to_float(m);
+                const bool need = mh >= kStateHi || (mh < kStateLo && sigma > 0);
+                if (__any_sync(0xffffffffu, need)) {   // rare; the whole warp takes part
+                    tmem_wait_st();
+                    delta = chain_state_reconvert(lane_base, sigma, need);
+                    sigma += delta;
+                }
+            }
+            tmem_wait_st();
+            fence_before_sync();
+            named_bar_sync(BAR_CHAIN, 128);
+            // [O | Y]^T = S^T [gamma Q ; -beta gamma K]^T
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t b1 = smem_u32(sm + B1);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_f16_ts(tbase + TM_O, tbase + TM_H + (uint32_t)ks * 8u, desc_kmajor(b1, 128, ks), IDESC_OY,
+                               ks > 0 ? 1u : 0u);
+                mma_commit(bar_y);
+                ++issued_y;
+            }
+            // S^T <- S^T Diag(gamma_C) 2^-delta (the MMA above reads only the fp16 copy)
+            {
+                const float* gc = reinterpret_cast<const float*>(sm + S_GC) + (cc & 1u) * kHeadDim;
+                const float f = pow2i(-delta);
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
+                    uint32_t s[32];
+                    tmem_ld32(lane_base + TM_S + 32u * cb, s);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 g4 = *reinterpret_cast<const float4*>(gc + 32 * cb + j);
+                        const float2 a = __fmul2_rn(make_float2(__uint_as_float(s[j]), __uint_as_float(s[j + 1])),
+                                                    make_float2(g4.x * f, g4.y * f));
+                        const float2 c = __fmul2_rn(make_float2(__uint_as_float(s[j + 2]), __uint_as_float(s[j + 3])),
+                                                    make_float2(g4.z * f, g4.w * f));
+                        s[j] = __float_as_uint(a.x);
+                        s[j + 1] = __float_as_uint(a.y);
+                        s[j + 2] = __float_as_uint(c.x);
+                        s[j + 3] = __float_as_uint(c.y);
+                    }
+                    tmem_st32(lane_base + TM_S + 32u * cb, s);
+                }
+                tmem_wait_st();
+            }
+            PIPE_MARK(0, 1, 14);
+            // ---- Y^T += 2^-sigma (beta V)^T -> fp16 ----
+            bad |= !warp_wait(bar_y, cc & 1u);
+            fence_after_sync();
+            {
+                float y[64];
+                {
+                    uint32_t t0r[32], t1r[32];
+                    tmem_ld32(lane_base + TM_Y, t0r);
+                    tmem_ld32(lane_base + TM_Y + 32u, t1r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        y[j] = __uint_as_float(t0r[j]);
+                        y[32 + j] = __uint_as_float(t1r[j]);
+                    }
+                }
+                const float fs = pow2i(-sigma);
+                const float* be = reinterpret_cast<const float*>(sm + S_BETA) + (cc & 1u) * 64u;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(sm + VT + (uint32_t)v * 128u +
+                                                                    (((uint32_t)ch ^ ((uint32_t)v & 7u)) << 4));
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                    const float4 b0 = *reinterpret_cast<const float4*>(be + 8 * ch);
+                    const float4 b1v = *reinterpret_cast<const float4*>(be + 8 * ch + 4);
+                    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1v.x, b1v.y, b1v.z, b1v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 vv = bf16x2_to_float2(ww[e]);
+                        y[8 * ch + 2 * e] = fmaf(fs * bb[2 * e], vv.x, y[8 * ch + 2 * e]);
+                        y[8 * ch + 2 * e + 1] = fmaf(fs * bb[2 * e + 1], vv.y, y[8 * ch + 2 * e + 1]);
+                    }
+                }
+                const bool need = to_f16_tmem(y, TM_H, 1.f) >= kRangeHi;
+                if (__any_sync(0xffffffffu, need)) {   // rare; the whole warp takes part
+                    tmem_wait_st();
+                    sigma += chain_vals_reconvert(lane_base, TM_H, sm, v, cc & 1u, true, sigma, need);
+                }
+            }
+            tmem_wait_st();
+            fence_before_sync();
+            if (named_bar_or(BAR_CHAIN, 128, bad || *sAbort != 0u)) {
+                aborted = true;
+                break;
+            }
+            PIPE_MARK(0, 1, 15);
+            // U^T = Y^T T^T, once the front end has T
+            if (tid == 0) {
+                if (mbar_wait_bounded(bar_t, cc & 1u)) {
+                    fence_after_sync();
+                    const uint32_t t16 = smem_u32(sm + T16);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_f16_ts(tbase + TM_Y, tbase + TM_H + (uint32_t)ks * 8u, desc_kmajor(t16, 64, ks), IDESC_T,
+                                   ks > 0 ? 1u : 0u);
+                    mma_commit(bar_u);
+                    ++issued_u;
+                } else {
+                    record_error(KDA_DEVERR_TIMEOUT);
+                    *sAbort = 1u;
+                }
+            }
+            bad |= !warp_wait(bar_u, cc & 1u);
+            fence_after_sync();
+            PIPE_MARK(0, 1, 16);
+            // ---- U^T -> fp16 ----
+            {
+                float u[64];
+                {
+                    uint32_t t0r[32], t1r[32];
+                    tmem_ld32(lane_base + TM_Y, t0r);
+                    tmem_ld32(lane_base + TM_Y + 32u, t1r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        u[j] = __uint_as_float(t0r[j]);
+                        u[32 + j] = __uint_as_float(t1r[j]);
+                    }
+                }
+                const bool need = to_f16_tmem(u, TM_H + 32u, 1.f) >= kRangeHi;
+                if (__any_sync(0xffffffffu, need)) {   // rare; the whole warp takes part
+                    tmem_wait_st();
+                    sigma += chain_vals_reconvert(lane_base, TM_H + 32u, sm, v, cc & 1u, false, sigma, need);
+                }
+            }
+            tmem_wait_st();
+            fence_before_sync();
+            if (named_bar_or(BAR_CHAIN, 128, bad || *sAbort != 0u)) {
+                aborted = true;
+                break;
+            }
+            // [S | O]^T += U^T [Khat | P^T]
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t b2 = smem_u32(sm + B2);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_f16_ts(tbase + TM_S, tbase + TM_H + 32u + (uint32_t)ks * 8u, desc_mnmajor(b2, 64, ks),
+                               IDESC_SO, 1u);
+                mma_commit(bar_s);
+                ++issued_s;
+            }
+            PIPE_MARK(0, 1, 17);
+            have_prev = true;
+            prev_h = m_h;
+            prev_n = m_n;
+            prev_t0 = m_t0;
+            prev_L = m_L;
+            prev_last = m_last;
+            ++cc;
+        }
+        // wind-down: no MMA of this thread may still run when TMEM is released
+        if (tid == 0 && aborted) {
+            if (issued_y > 0) mbar_wait_bounded(bar_y, (issued_y - 1) & 1u);
+            if (issued_u > 0) mbar_wait_bounded(bar_u, (issued_u - 1) & 1u);
+            if (issued_s > done_s) mbar_wait_bounded(bar_s, (issued_s - 1) & 1u);
+            if (issued_ap > 0) mbar_wait_bounded(bar_ap, (issued_ap - 1) & 1u);
+        }
+        if (aborted && tid == 0) *sAbort = 1u;
+    } else {
+        // =============================== front end ===============================
+        const bool is_aux = warp < kElemWarp0;
+        const int at = tid - 128;           // aux thread (warps 4-7)
+        const int et = tid - 256;           // element thread (warps 8-15)
+        const int ew = et >> 5;
+        const int eI = ew >> 1, ehf = ew & 1;
+        const int c0 = 64 * ehf + 4 * (lane & 15);
+        const int r0 = 16 * eI + 8 * (lane >> 4);
+        const int quarter = warp & 3;       // TMEM lane quarter of this warp
+        const int fsub = (warp - kAuxWarp0) >> 2;   // 0 aux, 1 warps 8-11, 2 warps 12-15
+        const bool issuer = tid == 128;
+        bool tma_pending = false;
+        uint32_t tma_parity = 0;
+        bool aborted = false;
+        uint32_t range_bad = 0u;
+
+        Cursor cur = unit_from(p, sOrder, b, G, units, 0);
+        float a[8][4];
+        float beta_reg = 0.f;   // aux threads 0-63: beta of their token of the next chunk to form
+        if (cur.valid) {
+            if (issuer) {
+                issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, cur.h, cur.t0);
+                const Cursor n2 = next_chunk(p, sOrder, b, G, units, cur);
+                if (n2.valid) prefetch_chunk(&tm_q, &tm_k, &tm_v, &tm_g, n2.h, n2.t0);
+            }
+            tma_pending = true;
+            const int L = (int)(cur.eos - cur.t0 < kChunk ? cur.eos - cur.t0 : kChunk);
+            if (!is_aux) gate_tokens(p, cur.h, cur.t0, L, c0, r0, a);
+            else if (at < kChunk && at < L) beta_reg = p.beta[(cur.t0 + at) * H + cur.h];
+        }
+        uint32_t ci = 0;
+        while (cur.valid) {
+            const Cursor nxt = next_chunk(p, sOrder, b, G, units, cur);
+            const int h = cur.h;
+            const int64_t t0 = cur.t0;
+            const int L = (int)(cur.eos - t0 < kChunk ? cur.eos - t0 : kChunk);
+            const uint32_t sl = ci & 1u;
+            bool bad = false;
+            PIPE_MARK(128, 0, 0);
+            // ================ F0: block products of a (element) / beta (aux) ================
+            // Each element thread keeps its 32 values a_t across the phases and rebuilds the
+            // factors R (running product from the block start) and E (product to the block end)
+            // where it needs them; po = product over the other 8-token half of its block.
+            float po[4];
+            if (!is_aux) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float own = a[0][e];
+#pragma unroll
+                    for (int i = 1; i < 8; ++i) own *= a[i][e];
+                    po[e] = __shfl_xor_sync(0xffffffffu, own, 16);
+                    if ((lane >> 4) == 0) own *= po[e];          // block product (both halves agree)
+                    if ((lane >> 4) == 0)
+                        reinterpret_cast<float*>(sm + S_PTOT)[eI * kHeadDim + c0 + e] = own;
+                }
+            } else if (at < kChunk) {
+                reinterpret_cast<float*>(sm + S_BETA)[sl * 64u + at] = beta_reg;
+            }
+            named_bar_sync(BAR_FE, kFeThreads);
+            PIPE_MARK(128, 0, 1);
+            // ================ F2: A/P operand tiles (element) / P diagonal (aux) ================
+            bad |= !warp_wait(bar_in, ci & 1u);
+            if (!is_aux) {
+                const float* ptot = reinterpret_cast<const float*>(sm + S_PTOT);
+                float4 pt[4];
+#pragma unroll
+                for (int J = 0; J < 4; ++J) pt[J] = *reinterpret_cast<const float4*>(ptot + J * kHeadDim + c0);
+                auto pick = [&](int J) { return J == 0 ? pt[0] : (J == 1 ? pt[1] : (J == 2 ? pt[2] : pt[3])); };
+                const float4 pbI = pick(eI);
+                const float invB[4] = {fast_rcp(pbI.x), fast_rcp(pbI.y), fast_rcp(pbI.z), fast_rcp(pbI.w)};
+                const float4 p1 = pick(eI < 3 ? eI + 1 : 3), p2 = pick(eI < 2 ? eI + 2 : 3);
+                const float F2[4] = {p1.x, p1.y, p1.z, p1.w};
+                const float F3[4] = {p1.x * p2.x, p1.y * p2.y, p1.z * p2.z, p1.w * p2.w};
+                uint32_t mq = 0u, mk = 0u;
+                float E[8][4], Rr[4];
+                decay_suffix(a, po, (lane >> 4) != 0, E, Rr);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = r0 + i;
+                    float R[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) R[e] = Rr[e] = Rr[e] * a[i][e];
+                    uint2 kk = *reinterpret_cast<const uint2*>(sm + IN_K + (uint32_t)r * 256u + (uint32_t)c0 * 2u);
+                    uint2 qq = *reinterpret_cast<const uint2*>(sm + IN_Q + (uint32_t)r * 256u + (uint32_t)c0 * 2u);
+                    if (r >= L) kk = qq = make_uint2(0u, 0u);
+                    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mk) : "r"(kk.x));
+                    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mk) : "r"(kk.y));
+                    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mq) : "r"(qq.x));
+                    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mq) : "r"(qq.y));
+                    const float2 k01 = bf16x2_to_float2(kk.x), k23 = bf16x2_to_float2(kk.y);
+                    const float2 q01 = bf16x2_to_float2(qq.x), q23 = bf16x2_to_float2(qq.y);
+                    const float kv[4] = {k01.x, k01.y, k23.x, k23.y}, qv[4] = {q01.x, q01.y, q23.x, q23.y};
+                    float kE[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) kE[e] = kv[e] * E[i][e];
+                    st_tile2(sm, AP_A + sw128_off(r, c0, 128), pack_bf16(kv[0] * R[0], kv[1] * R[1]),
+                          pack_bf16(kv[2] * R[2], kv[3] * R[3]));
+                    st_tile2(sm, AP_A + sw128_off(64 + r, c0, 128), pack_bf16(qv[0] * R[0], qv[1] * R[1]),
+                          pack_bf16(qv[2] * R[2], qv[3] * R[3]));
+                    st_tile2(sm, AP_B + sw128_off(r, c0, 160), pack_bf16(kE[0] * invB[0], kE[1] * invB[1]),
+                          pack_bf16(kE[2] * invB[2], kE[3] * invB[3]));
+                    if (eI <= 2)
+                        st_tile2(sm, AP_B + sw128_off(64 + r, c0, 160), pack_bf16(kE[0], kE[1]), pack_bf16(kE[2], kE[3]));
+                    if (eI <= 1)
+                        st_tile2(sm, AP_B + sw128_off(112 + r, c0, 160), pack_bf16(kE[0] * F2[0], kE[1] * F2[1]),
+                              pack_bf16(kE[2] * F2[2], kE[3] * F2[3]));
+                    if (eI == 0)
+                        st_tile2(sm, AP_B + sw128_off(144 + r, c0, 160), pack_bf16(kE[0] * F3[0], kE[1] * F3[1]),
+                              pack_bf16(kE[2] * F3[2], kE[3] * F3[3]));
+                }
+                // |q|, |k| bound every fp16 operand built from them (the decay factors are <= 1)
+                const float2 mkf = bf16x2_to_float2(mk), mqf = bf16x2_to_float2(mq);
+                if (fmaxf(fmaxf(fabsf(mkf.x), fabsf(mkf.y)), fmaxf(fabsf(mqf.x), fabsf(mqf.y))) >= kRangeHi)
+                    range_bad = 1u;
+            } else {
+                // q_r . k_r in fp32 over one 64-channel half; 16-byte chunks visited in a
+                // row-dependent order (conflict-free)
+                const int r = at & 63, hh = at >> 6;
+                float pd = 0.f;
+                if (r < L) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t off = (uint32_t)r * 256u + (uint32_t)hh * 128u + (((uint32_t)(j + r) & 7u) << 4);
+                        const uint4 qv = *reinterpret_cast<const uint4*>(sm + IN_Q + off);
+                        const uint4 kv = *reinterpret_cast<const uint4*>(sm + IN_K + off);
+                        const uint32_t qa[4] = {qv.x, qv.y, qv.z, qv.w}, ka[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 a2 = bf16x2_to_float2(qa[e]), b2 = bf16x2_to_float2(ka[e]);
+                            pd = fmaf(a2.x, b2.x, pd);
+                            pd = fmaf(a2.y, b2.y, pd);
+                        }
+                    }
+                }
+                reinterpret_cast<float*>(sm + S_PD)[hh * 64 + r] = pd;
+            }
+            fence_proxy_async();
+            if (named_bar_or(BAR_FE, kFeThreads, bad || *sAbort != 0u)) {
+                aborted = true;
+                break;
+            }
+            tma_pending = false;
+            PIPE_MARK(128, 0, 2);
+            // ================ F3: the A/P operands are ready (the chain issues the MMA) ================
+            if (issuer) mbar_arrive(bar_apready);
+            PIPE_MARK(128, 0, 3);
+            // ================ F4: the chain's operands (once it is done with the last chunk's) ================
+            if (ci > 0) bad |= !warp_wait(bar_s, (ci - 1) & 1u);
+            PIPE_MARK(128, 0, 4);
+            if (!is_aux) {
+                const float* ptot = reinterpret_cast<const float*>(sm + S_PTOT);
+                float before[4] = {1.f, 1.f, 1.f, 1.f}, after[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+                for (int J = 0; J < 4; ++J) {
+                    const float4 x = *reinterpret_cast<const float4*>(ptot + J * kHeadDim + c0);
+                    const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        if (J < eI) before[e] *= xv[e];
+                        if (J > eI) after[e] *= xv[e];
+                    }
+                }
+                const float* sb = reinterpret_cast<const float*>(sm + S_BETA) + sl * 64u;
+                float E[8][4], Rr[4];
+                decay_suffix(a, po, (lane >> 4) != 0, E, Rr);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = r0 + i;
+                    const float nb = -sb[r];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) Rr[e] *= a[i][e];
+                    // k, q again from the input tiles (still resident: the next chunk's loads are
+                    // issued after this phase); rows past the valid length are zero
+                    uint2 kk = *reinterpret_cast<const uint2*>(sm + IN_K + (uint32_t)r * 256u + (uint32_t)c0 * 2u);
+                    uint2 qq = *reinterpret_cast<const uint2*>(sm + IN_Q + (uint32_t)r * 256u + (uint32_t)c0 * 2u);
+                    if (r >= L) kk = qq = make_uint2(0u, 0u);
+                    const float2 k01 = bf16x2_to_float2(kk.x), k23 = bf16x2_to_float2(kk.y);
+                    const float2 q01 = bf16x2_to_float2(qq.x), q23 = bf16x2_to_float2(qq.y);
+                    const float kv[4] = {k01.x, k01.y, k23.x, k23.y}, qv[4] = {q01.x, q01.y, q23.x, q23.y};
+                    float gm[4], kh[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        gm[e] = Rr[e] * before[e];
+                        kh[e] = kv[e] * E[i][e] * after[e];
+                    }
+                    st_tile2(sm, B1 + sw128_off(r, c0, 128), pack_f16s(qv[0] * gm[0], qv[1] * gm[1]),
+                          pack_f16s(qv[2] * gm[2], qv[3] * gm[3]));
+                    st_tile2(sm, B1 + sw128_off(64 + r, c0, 128), pack_f16s(nb * kv[0] * gm[0], nb * kv[1] * gm[1]),
+                          pack_f16s(nb * kv[2] * gm[2], nb * kv[3] * gm[3]));
+                    st_tile2(sm, KH + sw128_off(r, c0, 64), pack_f16s(kh[0], kh[1]), pack_f16s(kh[2], kh[3]));
+                    if (fabsf(nb) > 1.f && fabsf(nb) * fmaxf(fmaxf(fabsf(kv[0]), fabsf(kv[1])),
+                                                             fmaxf(fabsf(kv[2]), fabsf(kv[3]))) >= kRangeHi)
+                        range_bad = 1u;
+                }
+                if (eI == 0 && (lane >> 4) == 0) {
+                    float gc[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+                    for (int J = 0; J < 4; ++J) {
+                        const float4 x = *reinterpret_cast<const float4*>(ptot + J * kHeadDim + c0);
+                        gc[0] *= x.x; gc[1] *= x.y; gc[2] *= x.z; gc[3] *= x.w;
+                    }
+                    *reinterpret_cast<float4*>(reinterpret_cast<float*>(sm + S_GC) + sl * kHeadDim + c0) =
+                        make_float4(gc[0], gc[1], gc[2], gc[3]);
+                }
+            } else {
+                // V^T: thread -> value columns 2 vp and 2 vp + 1, tokens 32 th .. 32 th + 31
+              {
+                const int vp = at & 63, th = at >> 6;
+                const uint32_t v0 = 2u * (uint32_t)vp, v1 = v0 + 1u;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t w[8];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        const int r = 32 * th + 8 * j + t;
+                        w[t] = r < L ? *reinterpret_cast<const uint32_t*>(sm + IN_V + (uint32_t)r * 256u + (uint32_t)vp * 4u)
+                                     : 0u;
+                    }
+                    const uint32_t ch = (uint32_t)(4 * th + j);
+                    st_tile4(sm, VT + v0 * 128u + ((ch ^ (v0 & 7u)) << 4), __byte_perm(w[0], w[1], 0x5410),
+                          __byte_perm(w[2], w[3], 0x5410), __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
+                    st_tile4(sm, VT + v1 * 128u + ((ch ^ (v1 & 7u)) << 4), __byte_perm(w[0], w[1], 0x7632),
+                          __byte_perm(w[2], w[3], 0x7632), __byte_perm(w[4], w[5], 0x7632), __byte_perm(w[6], w[7], 0x7632));
+                }
+              }
+                if (at == 0) {
+                    int32_t* meta = sMeta + sl * 8u;
+                    meta[0] = 1;
+                    meta[1] = h;
+                    meta[2] = cur.n;
+                    meta[3] = (int32_t)t0;
+                    meta[4] = L;
+                    meta[5] = t0 == cur.bos ? 1 : 0;
+                    meta[6] = t0 + kChunk >= cur.eos ? 1 : 0;
+                }
+            }
+            fence_proxy_async();
+            if (named_bar_or(BAR_FE, kFeThreads, bad || *sAbort != 0u)) {
+                aborted = true;
+                break;
+            }
+            PIPE_MARK(128, 0, 5);
+            // ================ F5: hand the chunk to the chain; load the next one ================
+            if (issuer) {
+                mbar_arrive(bar_formed);
+                if (nxt.valid) {
+                    issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, nxt.h, nxt.t0);
+                    const Cursor n2 = next_chunk(p, sOrder, b, G, units, nxt);
+                    if (n2.valid) prefetch_chunk(&tm_q, &tm_k, &tm_v, &tm_g, n2.h, n2.t0);
+                }
+            }
+            tma_pending = nxt.valid;
+            tma_parity = (ci + 1u) & 1u;
+            // beta of the next chunk: its latency is hidden behind the read-out and the solve
+            if (is_aux && at < kChunk) {
+                const int L1 = nxt.valid ? (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk) : 0;
+                beta_reg = at < L1 ? p.beta[(nxt.t0 + at) * H + nxt.h] : 0.f;
+            }
+            // ================ F6: A / P read-out (aux warps, one per TMEM lane quarter) ================
+            // The element warps meanwhile compute the next chunk's gate (it overlaps the read-out and
+            // the solve).
+            if (!is_aux) {
+                if (nxt.valid) {
+                    const int L1 = (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk);
+                    gate_tokens(p, nxt.h, nxt.t0, L1, c0, r0, a);
+                }
+            } else {
+                if (!warp_wait(bar_ap, ci & 1u)) *sAbort = 1u;
+                fence_after_sync();
+                PIPE_MARK(128, 0, 6);
+                const bool isA = quarter < 2;
+                const int r = (quarter & 1) * 32 + lane;      // token row of A (k rows) or P (q rows)
+                const int I = r >> 4;
+                const float be = reinterpret_cast<const float*>(sm + S_BETA)[sl * 64u + r];
+                const float pdg = reinterpret_cast<const float*>(sm + S_PD)[r] +
+                                  reinterpret_cast<const float*>(sm + S_PD)[64 + r];
+                float pmax = 0.f;
+#pragma unroll 1
+                for (int J = 0; J < 4; ++J) {
+                    float row[16];
+                    auto pick = [&](uint32_t col_a, uint32_t col_b, int I_a) {
+                        uint32_t ta[16], tb[16];
+                        tmem_ld16(taddr(tbase, quarter, TM_AP + col_a), ta);
+                        tmem_ld16(taddr(tbase, quarter, TM_AP + col_b), tb);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) row[x] = __uint_as_float(I == I_a ? ta[x] : tb[x]);
+                    };
+                    if ((quarter & 1) == 0) {        // I in {0, 1}
+                        if (J == 0) pick(0, 64, 0);            // I=0: diagonal; I=1: C1 of block 0
+                        else if (J == 1) pick(16, 16, 1);      // I=1: diagonal (I=0: masked)
+                        else {
+#pragma unroll
+                            for (int x = 0; x < 16; ++x) row[x] = 0.f;
+                        }
+                    } else {                         // I in {2, 3}
+                        if (J == 0) pick(112, 144, 2);         // I=2: C2 of block 0; I=3: C3 of block 0
+                        else if (J == 1) pick(80, 128, 2);     // I=2: C1 of block 1; I=3: C2 of block 1
+                        else if (J == 2) pick(32, 96, 2);      // I=2: diagonal; I=3: C1 of block 2
+                        else pick(48, 48, 3);                  // I=3: diagonal (I=2: masked)
+                    }
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) {
+                        const int i = J * 16 + x;
+                        row[x] = i < r ? row[x] : ((i == r && !isA) ? pdg : 0.f);
+                    }
+                    if (isA) {
+                        float* a32 = reinterpret_cast<float*>(sm + A32) + r * kF32Pitch + J * 16;
+#pragma unroll
+                        for (int x = 0; x < 16; x += 4)
+                            *reinterpret_cast<float4*>(a32 + x) =
+                                make_float4(be * row[x], be * row[x + 1], be * row[x + 2], be * row[x + 3]);
+                    } else {
+                        // P^T (MN-major, K = token i, N = row r): 16-bit stores, a warp writes 64
+                        // contiguous bytes per i
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            const int i = J * 16 + x;
+                            pmax = fmaxf(pmax, fabsf(row[x]));
+                            st_tile_h(sm, PT + sw128_off((uint32_t)i, (uint32_t)r, 64u),
+                                      __half_as_ushort(__float2half_rn(fminf(fmaxf(row[x], -65504.f), 65504.f))));
+                        }
+                    }
+                }
+                if (pmax >= kRangeHi) range_bad = 1u;
+                fence_proxy_async();
+                tmem_wait_ld();
+                fence_before_sync();
+                named_bar_sync(BAR_AUX, 128);
+                PIPE_MARK(128, 0, 7);
+                const int sw = warp - kAuxWarp0;
+                const float* a32 = reinterpret_cast<const float*>(sm + A32);
+                float* t32 = reinterpret_cast<float*>(sm + T32);
+                float tmax = 0.f;
+                auto Ab = [&](int I, int J) { return a32 + 16 * I * kF32Pitch + 16 * J; };
+                auto Tb = [&](int I, int J) { return t32 + 16 * I * kF32Pitch + 16 * J; };
+                // one warp writes the fp16 copy of finished block (I, J): lane -> (row, 8-col chunk)
+                auto to_t16 = [&](int I, int J) {
+                    const int rr = lane >> 1, ch = lane & 1;
+                    const float* src = Tb(I, J) + rr * kF32Pitch + ch * 8;
+                    const float4 lo4 = *reinterpret_cast<const float4*>(src);
+                    const float4 hi4 = *reinterpret_cast<const float4*>(src + 4);
+                    tmax = fmaxf(tmax, fmaxf(fmaxf(fmaxf(fabsf(lo4.x), fabsf(lo4.y)), fmaxf(fabsf(lo4.z), fabsf(lo4.w))),
+                                             fmaxf(fmaxf(fabsf(hi4.x), fabsf(hi4.y)), fmaxf(fabsf(hi4.z), fabsf(hi4.w)))));
+                    st_v4(sm, T16 + sw128_chunk_off(16 * I + rr, 2 * J + ch, 64), pack_f16s(lo4.x, lo4.y),
+                          pack_f16s(lo4.z, lo4.w), pack_f16s(hi4.x, hi4.y), pack_f16s(hi4.z, hi4.w));
+                };
+                // sign * (a 16 x 16 warp-MMA accumulator) straight into block (I, J) of the fp16 tile
+                auto acc_to_t16 = [&](int I, int J, const float (&acc)[2][4], float sign) {
+                    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+                    for (int nh = 0; nh < 2; ++nh) {
+                        const uint32_t col = (uint32_t)(16 * J + 8 * nh + 2 * t);
+                        tmax = fmaxf(tmax, fmaxf(fmaxf(fabsf(acc[nh][0]), fabsf(acc[nh][1])),
+                                                 fmaxf(fabsf(acc[nh][2]), fabsf(acc[nh][3]))));
+                        *reinterpret_cast<uint32_t*>(sm + T16 + sw128_off((uint32_t)(16 * I + g), col, 64u)) =
+                            pack_f16s(sign * acc[nh][0], sign * acc[nh][1]);
+                        *reinterpret_cast<uint32_t*>(sm + T16 + sw128_off((uint32_t)(16 * I + g + 8), col, 64u)) =
+                            pack_f16s(sign * acc[nh][2], sign * acc[nh][3]);
+                    }
+                };
+                // L0: the four 16 x 16 diagonal blocks by forward substitution in fp32, one column
+                // per thread (threads 0-63), right-looking
+                if (sw < 2) {
+                    const int bI = at >> 4, jc = at & 15, o = bI * 16;
+                    float x[16];
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == jc) ? 1.f : 0.f;
+#pragma unroll
+                    for (int ii = 0; ii < 15; ++ii) {
+                        const float xi = x[ii];
+#pragma unroll
+                        for (int rr = ii + 1; rr < 16; ++rr) x[rr] = fmaf(-a32[(o + rr) * kF32Pitch + o + ii], xi, x[rr]);
+                    }
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) t32[(o + rr) * kF32Pitch + o + jc] = x[rr];
+                }
+                named_bar_sync(BAR_AUX, 128);
+                PIPE_MARK(128, 0, 8);
+                // L1 (16 x 16 warp-MMA products, fp16 operands, fp32 accumulation):
+                //   T10 = -T11 (A10 T00), T32 = -T33 (A32 T22),
+                //   X20 = A20 T00 + A21 T10, X30 = A30 T00 + A31 T10, X21 = A21 T11, X31 = A31 T11.
+                // Aux warps 0 and 2 both form T10 (in their own scratch) so that neither waits for
+                // the other.  Scratch: T's and A's blocks above the diagonal.
+                {
+                    float* const a32w = reinterpret_cast<float*>(sm + A32);
+                    auto Aw = [&](int I, int J) { return a32w + 16 * I * kF32Pitch + 16 * J; };
+                    float acc[2][4] = {};
+                    if (sw == 0 || sw == 2) {
+                        float* ysc = sw == 0 ? Tb(0, 1) : Aw(0, 1);     // A10 T00
+                        float* t10 = sw == 0 ? Tb(1, 0) : Aw(0, 2);     // T10
+                        warpmma::mm16_acc_h(Ab(1, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);
+                        warpmma::store16(ysc, kF32Pitch, acc, 1.f);
+                        __syncwarp();
+                        float a2[2][4] = {};
+                        warpmma::mm16_acc_h(Tb(1, 1), kF32Pitch, ysc, kF32Pitch, a2);
+                        warpmma::store16(t10, kF32Pitch, a2, -1.f);
+                        __syncwarp();
+                        if (sw == 0) to_t16(1, 0);
+                        const int I = sw == 0 ? 2 : 3;
+                        float a3[2][4] = {};
+                        warpmma::mm16_acc_h(Ab(I, 0), kF32Pitch, Tb(0, 0), kF32Pitch, a3);
+                        warpmma::mm16_acc_h(Ab(I, 1), kF32Pitch, t10, kF32Pitch, a3);
+                        warpmma::store16(Tb(0, I), kF32Pitch, a3, 1.f);            // X20 / X30
+                    } else if (sw == 1) {
+                        warpmma::mm16_acc_h(Ab(3, 2), kF32Pitch, Tb(2, 2), kF32Pitch, acc);
+                        warpmma::store16(Tb(2, 3), kF32Pitch, acc, 1.f);            // A32 T22
+                        __syncwarp();
+                        float a2[2][4] = {};
+                        warpmma::mm16_acc_h(Tb(3, 3), kF32Pitch, Tb(2, 3), kF32Pitch, a2);
+                        warpmma::store16(Tb(3, 2), kF32Pitch, a2, -1.f);           // T32
+                        __syncwarp();
+                        to_t16(3, 2);
+                        float a3[2][4] = {};
+                        warpmma::mm16_acc_h(Ab(2, 1), kF32Pitch, Tb(1, 1), kF32Pitch, a3);
+                        warpmma::store16(Tb(1, 2), kF32Pitch, a3, 1.f);            // X21
+                    } else {
+                        warpmma::mm16_acc_h(Ab(3, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc);
+                        warpmma::store16(Tb(1, 3), kF32Pitch, acc, 1.f);            // X31
+#pragma unroll
+                        for (int d = 0; d < 4; ++d) to_t16(d, d);
+                    }
+                }
+                named_bar_sync(BAR_AUX, 128);
+                // L2: T_LL = -T_LR X, written straight to the fp16 tile:
+                //   T20 = -T22 X20, T21 = -T22 X21, T30 = -(T32 X20 + T33 X30), T31 = -(T32 X21 + T33 X31)
+                {
+                    float acc[2][4] = {};
+                    const int J = sw & 1;
+                    if (sw < 2) {
+                        warpmma::mm16_acc_h(Tb(2, 2), kF32Pitch, Tb(J, 2), kF32Pitch, acc);
+                        acc_to_t16(2, J, acc, -1.f);
+                    } else {
+                        warpmma::mm16_acc_h(Tb(3, 2), kF32Pitch, Tb(J, 2), kF32Pitch, acc);
+                        warpmma::mm16_acc_h(Tb(3, 3), kF32Pitch, Tb(J, 3), kF32Pitch, acc);
+                        acc_to_t16(3, J, acc, -1.f);
+                    }
+                }
+                if (tmax >= kRangeHi) range_bad = 1u;
+                fence_proxy_async();
+                named_bar_sync(BAR_AUX, 128);
+                if (at == 0) mbar_arrive(bar_t);
+            }
+            if (named_bar_or(BAR_FE, kFeThreads, *sAbort != 0u)) {
+                aborted = true;
+                break;
+            }
+            cur = nxt;
+            ++ci;
+        }
+        if (range_bad) record_error(KDA_DEVERR_RANGE);
+        if (!aborted) {
+            if (issuer) {
+                sMeta[(ci & 1u) * 8u] = 0;   // end of work for the chain
+                *sEnd = 1u;
+                mbar_arrive(bar_apready);
+                mbar_arrive(bar_formed);
+            }
+        } else {
+            *sAbort = 1u;
+            if (issuer) {
+                if (tma_pending) mbar_wait_bounded(bar_in, tma_parity);
+            }
+        }
+    }
+
+    // wind-down: every role has drained its own asynchronous operations
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 0) tmem_dealloc(tbase, TM_COLS);
+#ifdef KDA_PHASE_CLOCKS
+    if (tid == 0)
+        for (int i = 0; i < kPhases; ++i) atomicAdd(&g_pipe_phase_cycles[i], (unsigned long long)sPh[i]);
+#endif
+}
+
+// ---- host side ----
+
+cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
+    cudaError_t err = once_per_device([](int) {
+        return cudaFuncSetAttribute(kda_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
+    });
+    if (err != cudaSuccess) return err;
+    int dev = 0, sm_count = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+    if (sm_count <= 0) return cudaErrorInvalidDevice;
+    CUtensorMap tq, tk, tv, tg;
+    const int64_t rows = a.total_tokens, cols = (int64_t)a.H * kHeadDim;
+    if (!fused::make_map(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols) ||
+        !fused::make_map(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols) ||
+        !fused::make_map(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols) ||
+        !fused::make_map(&tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols))
+        return cudaErrorInvalidValue;
+    Params p;
+    p.g = a.g;
+    p.beta = a.beta;
+    p.A_log = a.A_log;
+    p.dt_bias = a.dt_bias;
+    p.lower_bound = a.lower_bound;
+    p.scale = a.scale;
+    p.initial_state = a.initial_state;
+    p.cu_seqlens = a.cu_seqlens;
+    p.out = static_cast<__nv_bfloat16*>(a.out);
+    p.final_state = a.final_state;
+    p.seqlen = a.seqlen;
+    p.total_tokens = a.total_tokens;
+    p.H = a.H;
+    p.N = a.N;
+    const int64_t units = (int64_t)a.N * a.H;
+    const int grid = (int)(units < sm_count ? units : sm_count);
+    if (grid <= 0) return cudaSuccess;
+    kda_pipe_kernel<<<grid, kThreads, SMEM_ALLOC, stream>>>(tq, tk, tv, tg, p);
+    return cudaGetLastError();
+}
+
+}  // namespace pipe
+
+#ifdef KDA_PHASE_CLOCKS
+// Debug builds only: copies and clears the per-phase cycle totals of the pipelined kernel
+// (slots 0-8: front end, thread 128; slots 9-17: chain, thread 0).
+extern "C" int kda_debug_pipe_phase_cycles(unsigned long long* out) {
+    if (cudaMemcpyFromSymbol(out, pipe::g_pipe_phase_cycles, sizeof(unsigned long long) * pipe::kPhases) !=
+        cudaSuccess)
+        return -1;
+    unsigned long long zero[pipe::kPhases] = {};
+    return cudaMemcpyToSymbol(pipe::g_pipe_phase_cycles, zero, sizeof zero) == cudaSuccess ? pipe::kPhases : -1;
+}
+#endif
+
+cudaError_t launch_pipe(const StagedArgs& a, cudaStream_t stream) { return pipe::launch(a, stream); }
+
+}  // namespace kda

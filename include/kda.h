@@ -79,15 +79,29 @@ typedef struct {
 #define KDA_DEVERR_BAD_OFFSETS 0x1u   /* cu_seqlens not monotone / out of [0, Ttot] */
 #define KDA_DEVERR_TIMEOUT     0x2u   /* a bounded wait ran out of iterations */
 #define KDA_DEVERR_BOUNDS      0x4u   /* an index outside its buffer was skipped */
+#define KDA_DEVERR_RANGE       0x8u   /* kda_fwd: an input outside the fused path's operating range
+                                         (see kda_fwd); the affected values were saturated */
 
 /*
  * kda_fwd -- the chunked prefill forward (the product path).
  *
- * Runs the fused persistent sm_100a kernel (tcgen05 tensor cores with TMEM
- * accumulators, TMA-staged inputs) when lower_bound >= KDA_FUSED_MIN_LOWER_BOUND,
- * and the staged exact-decay kernels otherwise (their intra-chunk decays are
- * formed pair by pair and cannot overflow for any gate).  The staged fallback
- * allocates its workspace stream-ordered (cudaMallocAsync).
+ * Runs the fused persistent sm_100a kernel when lower_bound >= KDA_FUSED_MIN_LOWER_BOUND, and
+ * the staged exact-decay kernels otherwise (their intra-chunk decays are formed pair by pair and
+ * cannot overflow for any gate).  The staged fallback allocates its workspace stream-ordered
+ * (cudaMallocAsync).
+ *
+ * The fused kernel: one CTA per SM carries each (sequence, head) state in tensor memory and
+ * runs the 64-token chunks through tcgen05 MMAs with fp16/bf16 operands and fp32 accumulation;
+ * warps 0-3 advance the state while the others build the next chunk.
+ * Operating range of the fused kernel:
+ *   - the initial state and v: any finite values.  The state is stored with a power-of-two
+ *     scale per value column (each column of S evolves independently and linearly), so no
+ *     fp16 operand derived from it can overflow;
+ *   - q, k and beta: |q|, |k|, |beta * k| elementwise and |q_r . k_i| below 2^15, which
+ *     L2-normalised q and k with beta <= 1 satisfy with a wide margin.
+ * An input outside that range is not an error before the launch: the kernel saturates the
+ * affected fp16 operands (never inf or NaN), records KDA_DEVERR_RANGE in the device error word
+ * and the output is then not guaranteed; kda_fwd_staged computes such inputs in fp32.
  *
  * lower_bound: <= 0 (may be -INFINITY: no clamp); NaN or > 0 is rejected.
  * scale: finite.  Returns KDA_OK or an error code; never aborts.
@@ -305,6 +319,21 @@ kda_status kda_bwd(const void* q, const void* k, const void* v,
                    const kda_grads* grads,
                    kda_dims dims, void* workspace, size_t workspace_bytes,
                    kda_stream_t stream);
+
+/*
+ * kda_selftest_wait_timeout -- diagnostics: exercises the recovery path of the library's bounded
+ * waits without any fault.  No page has a counterpart; every kernel here waits on mbarriers with a
+ * wall-clock limit, and this entry point makes one such wait run out on purpose.  It launches one
+ * CTA that allocates tensor memory, starts one tensor-core MMA, then waits (at most limit_ns
+ * nanoseconds) on an mbarrier that nothing arrives at.  As in the product kernels, the expired
+ * wait records KDA_DEVERR_TIMEOUT, the CTA waits (bounded) for its own MMA, frees its tensor
+ * memory and returns; the device stays usable.
+ *   limit_ns   in [1, 1e9]
+ *   observed   NULL, or device uint32 [2]: [0] = 1 if the wait ran out, [1] = 1 if the MMA had
+ *              completed before the tensor memory was freed
+ * Asynchronous on `stream`; read the result with kda_check_device_error.
+ */
+kda_status kda_selftest_wait_timeout(uint64_t limit_ns, uint32_t* observed, kda_stream_t stream);
 
 /* Human-readable name of a status code (static storage; never NULL). */
 const char* kda_strerror(kda_status status);

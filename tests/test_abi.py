@@ -220,3 +220,10 @@ def test_bwd_workspace_extends_the_staged_layout():
         staged = kda.lib().kda_staged_workspace_size(dims, varlen)
         assert kda.lib().kda_bwd_workspace_size(dims, varlen) >= staged + extra
         assert kda.lib().kda_bwd_workspace_size(dims, varlen) <= staged + extra + 16 * 256
+
+
+def test_selftest_rejects_bad_limits():
+    lib = kda.lib()
+    assert lib.kda_selftest_wait_timeout(0, None, None) == 1                  # KDA_ERR_INVALID_ARG
+    assert lib.kda_selftest_wait_timeout(2_000_000_000, None, None) == 1
+    assert lib.kda_selftest_wait_timeout(1000, ctypes.c_void_p(FAKE + 2), None) == 3   # KDA_ERR_ALIGNMENT
