@@ -113,13 +113,13 @@ def algorithmic_bytes(w: W.Workload, gdn: bool = False) -> int:
 
 
 KERNEL_SOURCES = {
-    "kda_fused_kernel": ("kda_fused.cuh", "umma.cuh", "warp_mma.cuh", "kda_common.cuh"),
+    "kda_pipe_kernel": ("kda_pipe.cuh", "umma.cuh", "warp_mma.cuh", "kda_common.cuh"),
     "kda_fused_kernel<scalar gate>": ("kda_fused.cuh", "umma.cuh", "warp_mma.cuh", "kda_common.cuh"),
     "kda_decode_kernel": ("kda_decode.cuh", "kda_common.cuh"),
 }
 
 
-def kernel_source_hash(kernel: str = "kda_fused_kernel") -> str:
+def kernel_source_hash(kernel: str = "kda_pipe_kernel") -> str:
     """Hash of the device sources one kernel is compiled from (profiles carry it
     so that stale DRAM counters are not reported against a changed kernel)."""
     h = hashlib.sha256()
@@ -131,7 +131,7 @@ def kernel_source_hash(kernel: str = "kda_fused_kernel") -> str:
     return h.hexdigest()[:16]
 
 
-TRAFFIC_FILES = {"kda_fused_kernel": "kda_fused_traffic.json",
+TRAFFIC_FILES = {"kda_pipe_kernel": "kda_pipe_traffic.json",
                  "kda_fused_kernel<scalar gate>": "kda_gdn_traffic.json",
                  "kda_decode_kernel": "kda_decode_traffic.json"}
 
@@ -295,6 +295,16 @@ def oracle_sample(w: W.Workload, x: dict, target_s: float, gdn: bool = False):
     return rate, desc, cores, oracle.max_threads(), h
 
 
+def workload_config(w: W.Workload, world: int, parallelism: str, gdn: bool = False, segments: int = 0) -> dict:
+    """The `config` object of a bench line: the workload and its sizes (the same keys on every
+    arm, so that lines of the same workload compare)."""
+    return {"workload": ("GDN (one gate per token-head) " if gdn else "") + w.describe()
+                        + (f"; run as {segments} segments (maps, fold, final pass)" if segments else ""),
+            "global_batch": w.N * world, "seq_len": w.T, "heads": w.H,
+            "parallelism": parallelism,
+            "l2": f"inputs exceed L2 ({algorithmic_bytes(w, gdn) / 1e6:.0f} MB per step vs 126 MB); no flush"}
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
@@ -330,8 +340,8 @@ def run_reference(args, world, rank):
         "value": value, "unit": "Mtokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.describe(), "global_batch": w.N, "seq_len": w.T,
-                   "parallelism": "host cores (OpenMP over sequence x head)"},
+        "config": workload_config(w, world, "host cores (OpenMP over sequence x head)"),
+        "precision": "fp64 token-by-token recurrence (the oracle)",
         "cpu_baseline": {"value": value, "unit": "Mtokens/s", "cores": threads, "kind": "oracle",
                          "sample": f"each step: {desc.split(' in ')[0]}; scaled by {h}/{w.H}"},
         "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -659,12 +669,12 @@ def main():
     achieved = alg_bytes / (kernel_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak,
-            "traffic": (dram_traffic_from_profile("kda_fused_kernel<scalar gate>" if args.gdn else "kda_fused_kernel",
+            "traffic": (dram_traffic_from_profile("kda_fused_kernel<scalar gate>" if args.gdn else "kda_pipe_kernel",
                                                   w.T * w.H) if fused and not args.segments else None),
             "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
             else "fallback 6650 GB/s",
             "kernel": (f"segmented prefill ({args.segments} segments: 3 fused launches + folds)" if args.segments
-                       else ("kda_fused_kernel<scalar gate>" if args.gdn else "kda_fused_kernel") if fused
+                       else ("kda_fused_kernel<scalar gate>" if args.gdn else "kda_pipe_kernel") if fused
                        else "staged kernels"),
             "kernel_ms": kernel_ms, "algorithmic_bytes": alg_bytes,
             "tflops": tflops,
@@ -719,13 +729,9 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded kda_workloads, no dataset)",
-            "config": {"workload": ("GDN (one gate per token-head) " if args.gdn else "") + w.describe()
-                       + (f"; run as {args.segments} segments (maps, fold, final pass)" if args.segments else ""),
-                       "model": "KDA layer forward (no weights)",
-                       "global_batch": w.N * world, "seq_len": w.T, "heads": w.H,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "precision": "bf16 q/k/v/out, fp32 gates and state; bf16/fp16 MMA operands, fp32 accumulate",
-                       "l2": f"inputs exceed L2 ({alg_bytes / 1e6:.0f} MB per step vs 126 MB); no flush"},
+            "config": workload_config(w, world, f"replicas x{world}" if world > 1 else "single GPU",
+                                      args.gdn, args.segments),
+            "precision": "bf16 q/k/v/out, fp32 gates and state; bf16/fp16 MMA operands, fp32 accumulate",
             "tflops": tflops,
             "roofline": roof,
             "cpu_baseline": cpu,

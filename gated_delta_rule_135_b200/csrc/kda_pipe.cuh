@@ -189,6 +189,14 @@ __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) 
 // floor(log2 |x|) for a normal nonzero x
 __device__ __forceinline__ int ilog2f(float x) { return (int)((__float_as_uint(x) >> 23) & 0xFFu) - 127; }
 
+// Byte offset of the 4-channel group starting at channel c0 (a multiple of 4) in row rowbase + i
+// of a 128-byte-swizzled 16-bit tile with `rows` rows, where rowbase is a multiple of 8 (so the
+// swizzle phase of the row is i): the same value as sw128_off(rowbase + i, c0, rows).
+__device__ __forceinline__ uint32_t quad_off(uint32_t rows, uint32_t rowbase, int i, uint32_t c0) {
+    return (c0 >> 6) * rows * 128u + (rowbase + (uint32_t)i) * 128u + (((((c0 & 63u) >> 3) ^ (uint32_t)i)) << 4) +
+           ((c0 & 7u) << 1);
+}
+
 __device__ __forceinline__ void st_v2(unsigned char* base, uint32_t off, uint32_t a, uint32_t b) {
     *reinterpret_cast<uint2*>(base + off) = make_uint2(a, b);
 }
@@ -393,17 +401,20 @@ __device__ __noinline__ int chain_state_reconvert(uint32_t lane_base, int sigma,
     if (delta < -sigma) delta = -sigma;
     if (sigma + delta > kSigmaMax) delta = kSigmaMax - sigma;
     if (!need) delta = 0;
+    // the fp16 copy and the fp32 state itself, both times 2^-delta
     const float f = pow2i(-delta);
 #pragma unroll 1
     for (int cb = 0; cb < 4; ++cb) {
         uint32_t s[32];
         tmem_ld32(lane_base + TM_S + 32u * cb, s);
         tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s[j] = __float_as_uint(f * __uint_as_float(s[j]));
         uint32_t h16[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            h16[j] = pack_f16s(f * __uint_as_float(s[2 * j]), f * __uint_as_float(s[2 * j + 1]));
+        for (int j = 0; j < 16; ++j) h16[j] = pack_f16s(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1]));
         tmem_st16(lane_base + TM_H + 16u * cb, h16);
+        tmem_st32(lane_base + TM_S + 32u * cb, s);
     }
     tmem_wait_st();
     return delta;
@@ -619,16 +630,9 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
         while (true) {
             bool bad = false;
-            if (have_prev) {
-                bad |= !warp_wait(bar_s, (cc - 1) & 1u);
-                if (tid == 0 && !bad) done_s = issued_s;
-                fence_after_sync();
-                PIPE_MARK(0, 1, 9);
-                if (!bad) retire_prev();
-            }
-            PIPE_MARK(0, 1, 10);
-            // the front end's A/P MMA: its operand tiles are written early in the chunk, while
-            // the chain is idle here; issuing costs the issuing warp about 70 cycles per MMA
+            // the front end's A/P MMA, issued as soon as its operand tiles are written (it does not
+            // depend on the state, so it goes before the previous chunk's retirement); issuing
+            // costs the issuing warp about 70 cycles per MMA
             if (tid == 0) {
                 const bool ap_ok = mbar_wait_bounded(bar_apready, cc & 1u);
                 PIPE_MARK(0, 1, 11);
@@ -646,6 +650,14 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     ++issued_ap;
                 }
             }
+            if (have_prev) {
+                bad |= !warp_wait(bar_s, (cc - 1) & 1u);
+                if (tid == 0 && !bad) done_s = issued_s;
+                fence_after_sync();
+                PIPE_MARK(0, 1, 9);
+                if (!bad) retire_prev();
+            }
+            PIPE_MARK(0, 1, 10);
             PIPE_MARK(0, 1, 12);
             bad |= !warp_wait(bar_formed, cc & 1u);
             const int32_t* meta = sMeta + (cc & 1u) * 8u;
@@ -710,10 +722,10 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mma_commit(bar_y);
                 ++issued_y;
             }
-            // S^T <- S^T Diag(gamma_C) 2^-delta (the MMA above reads only the fp16 copy)
+            // S^T <- S^T Diag(gamma_C) (the MMA above reads only the fp16 copy; a rescale of the lane
+            // was applied to the fp32 state already)
             {
                 const float* gc = reinterpret_cast<const float*>(sm + S_GC) + (cc & 1u) * kHeadDim;
-                const float f = pow2i(-delta);
 #pragma unroll 1
                 for (int cb = 0; cb < 4; ++cb) {
                     uint32_t s[32];
@@ -723,9 +735,9 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int j = 0; j < 32; j += 4) {
                         const float4 g4 = *reinterpret_cast<const float4*>(gc + 32 * cb + j);
                         const float2 a = __fmul2_rn(make_float2(__uint_as_float(s[j]), __uint_as_float(s[j + 1])),
-                                                    make_float2(g4.x * f, g4.y * f));
+                                                    make_float2(g4.x, g4.y));
                         const float2 c = __fmul2_rn(make_float2(__uint_as_float(s[j + 2]), __uint_as_float(s[j + 3])),
-                                                    make_float2(g4.z * f, g4.w * f));
+                                                    make_float2(g4.z, g4.w));
                         s[j] = __float_as_uint(a.x);
                         s[j + 1] = __float_as_uint(a.y);
                         s[j + 2] = __float_as_uint(c.x);
@@ -753,6 +765,7 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
                 const float fs = pow2i(-sigma);
+                const float2 fs2 = make_float2(fs, fs);
                 const float* be = reinterpret_cast<const float*>(sm + S_BETA) + (cc & 1u) * 64u;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
@@ -761,12 +774,14 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
                     const float4 b0 = *reinterpret_cast<const float4*>(be + 8 * ch);
                     const float4 b1v = *reinterpret_cast<const float4*>(be + 8 * ch + 4);
-                    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1v.x, b1v.y, b1v.z, b1v.w};
+                    const float2 bb[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1v.x, b1v.y),
+                                          make_float2(b1v.z, b1v.w)};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float2 vv = bf16x2_to_float2(ww[e]);
-                        y[8 * ch + 2 * e] = fmaf(fs * bb[2 * e], vv.x, y[8 * ch + 2 * e]);
-                        y[8 * ch + 2 * e + 1] = fmaf(fs * bb[2 * e + 1], vv.y, y[8 * ch + 2 * e + 1]);
+                        const float2 yy = __ffma2_rn(__fmul2_rn(fs2, bb[e]), bf16x2_to_float2(ww[e]),
+                                                     make_float2(y[8 * ch + 2 * e], y[8 * ch + 2 * e + 1]));
+                        y[8 * ch + 2 * e] = yy.x;
+                        y[8 * ch + 2 * e + 1] = yy.y;
                     }
                 }
                 const bool need = to_f16_tmem(y, TM_H, 1.f) >= kRangeHi;
@@ -951,19 +966,19 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     float kE[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) kE[e] = kv[e] * E[i][e];
-                    st_tile2(sm, AP_A + sw128_off(r, c0, 128), pack_bf16(kv[0] * R[0], kv[1] * R[1]),
+                    st_tile2(sm, AP_A + quad_off(128u, (uint32_t)r0, i, (uint32_t)c0), pack_bf16(kv[0] * R[0], kv[1] * R[1]),
                           pack_bf16(kv[2] * R[2], kv[3] * R[3]));
-                    st_tile2(sm, AP_A + sw128_off(64 + r, c0, 128), pack_bf16(qv[0] * R[0], qv[1] * R[1]),
+                    st_tile2(sm, AP_A + quad_off(128u, 64u + (uint32_t)r0, i, (uint32_t)c0), pack_bf16(qv[0] * R[0], qv[1] * R[1]),
                           pack_bf16(qv[2] * R[2], qv[3] * R[3]));
-                    st_tile2(sm, AP_B + sw128_off(r, c0, 160), pack_bf16(kE[0] * invB[0], kE[1] * invB[1]),
+                    st_tile2(sm, AP_B + quad_off(160u, (uint32_t)r0, i, (uint32_t)c0), pack_bf16(kE[0] * invB[0], kE[1] * invB[1]),
                           pack_bf16(kE[2] * invB[2], kE[3] * invB[3]));
                     if (eI <= 2)
-                        st_tile2(sm, AP_B + sw128_off(64 + r, c0, 160), pack_bf16(kE[0], kE[1]), pack_bf16(kE[2], kE[3]));
+                        st_tile2(sm, AP_B + quad_off(160u, 64u + (uint32_t)r0, i, (uint32_t)c0), pack_bf16(kE[0], kE[1]), pack_bf16(kE[2], kE[3]));
                     if (eI <= 1)
-                        st_tile2(sm, AP_B + sw128_off(112 + r, c0, 160), pack_bf16(kE[0] * F2[0], kE[1] * F2[1]),
+                        st_tile2(sm, AP_B + quad_off(160u, 112u + (uint32_t)r0, i, (uint32_t)c0), pack_bf16(kE[0] * F2[0], kE[1] * F2[1]),
                               pack_bf16(kE[2] * F2[2], kE[3] * F2[3]));
                     if (eI == 0)
-                        st_tile2(sm, AP_B + sw128_off(144 + r, c0, 160), pack_bf16(kE[0] * F3[0], kE[1] * F3[1]),
+                        st_tile2(sm, AP_B + quad_off(160u, 144u + (uint32_t)r0, i, (uint32_t)c0), pack_bf16(kE[0] * F3[0], kE[1] * F3[1]),
                               pack_bf16(kE[2] * F3[2], kE[3] * F3[3]));
                 }
                 // |q|, |k| bound every fp16 operand built from them (the decay factors are <= 1)
@@ -1041,11 +1056,11 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         gm[e] = Rr[e] * before[e];
                         kh[e] = kv[e] * E[i][e] * after[e];
                     }
-                    st_tile2(sm, B1 + sw128_off(r, c0, 128), pack_f16s(qv[0] * gm[0], qv[1] * gm[1]),
+                    st_tile2(sm, B1 + quad_off(128u, (uint32_t)r0, i, (uint32_t)c0), pack_f16s(qv[0] * gm[0], qv[1] * gm[1]),
                           pack_f16s(qv[2] * gm[2], qv[3] * gm[3]));
-                    st_tile2(sm, B1 + sw128_off(64 + r, c0, 128), pack_f16s(nb * kv[0] * gm[0], nb * kv[1] * gm[1]),
+                    st_tile2(sm, B1 + quad_off(128u, 64u + (uint32_t)r0, i, (uint32_t)c0), pack_f16s(nb * kv[0] * gm[0], nb * kv[1] * gm[1]),
                           pack_f16s(nb * kv[2] * gm[2], nb * kv[3] * gm[3]));
-                    st_tile2(sm, KH + sw128_off(r, c0, 64), pack_f16s(kh[0], kh[1]), pack_f16s(kh[2], kh[3]));
+                    st_tile2(sm, KH + quad_off(64u, (uint32_t)r0, i, (uint32_t)c0), pack_f16s(kh[0], kh[1]), pack_f16s(kh[2], kh[3]));
                     if (fabsf(nb) > 1.f && fabsf(nb) * fmaxf(fmaxf(fabsf(kv[0]), fabsf(kv[1])),
                                                              fmaxf(fabsf(kv[2]), fabsf(kv[3]))) >= kRangeHi)
                         range_bad = 1u;
