@@ -114,7 +114,7 @@ def algorithmic_bytes(w: W.Workload, gdn: bool = False) -> int:
 
 KERNEL_SOURCES = {
     "kda_pipe_kernel": ("kda_pipe.cuh", "umma.cuh", "warp_mma.cuh", "kda_common.cuh"),
-    "kda_fused_kernel<scalar gate>": ("kda_fused.cuh", "umma.cuh", "warp_mma.cuh", "kda_common.cuh"),
+    "kda_pipe_kernel<scalar gate>": ("kda_pipe.cuh", "umma.cuh", "warp_mma.cuh", "kda_common.cuh"),
     "kda_decode_kernel": ("kda_decode.cuh", "kda_common.cuh"),
 }
 
@@ -132,7 +132,7 @@ def kernel_source_hash(kernel: str = "kda_pipe_kernel") -> str:
 
 
 TRAFFIC_FILES = {"kda_pipe_kernel": "kda_pipe_traffic.json",
-                 "kda_fused_kernel<scalar gate>": "kda_gdn_traffic.json",
+                 "kda_pipe_kernel<scalar gate>": "kda_gdn_traffic.json",
                  "kda_decode_kernel": "kda_decode_traffic.json"}
 
 
@@ -669,12 +669,12 @@ def main():
     achieved = alg_bytes / (kernel_ms / 1e3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak,
-            "traffic": (dram_traffic_from_profile("kda_fused_kernel<scalar gate>" if args.gdn else "kda_pipe_kernel",
+            "traffic": (dram_traffic_from_profile("kda_pipe_kernel<scalar gate>" if args.gdn else "kda_pipe_kernel",
                                                   w.T * w.H) if fused and not args.segments else None),
             "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
             else "fallback 6650 GB/s",
             "kernel": (f"segmented prefill ({args.segments} segments: 3 fused launches + folds)" if args.segments
-                       else ("kda_fused_kernel<scalar gate>" if args.gdn else "kda_pipe_kernel") if fused
+                       else ("kda_pipe_kernel<scalar gate>" if args.gdn else "kda_pipe_kernel") if fused
                        else "staged kernels"),
             "kernel_ms": kernel_ms, "algorithmic_bytes": alg_bytes,
             "tflops": tflops,

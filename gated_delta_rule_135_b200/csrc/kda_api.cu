@@ -12,7 +12,6 @@
 #include "kda_internal.h"
 
 #include "kda_staged.cuh"
-#include "kda_fused.cuh"
 #include "kda_pipe.cuh"
 #include "kda_decode.cuh"
 #include "kda_cp.cuh"
@@ -250,7 +249,7 @@ kda_status kda_gdn_fwd(const void* q, const void* k, const void* v, const float*
     if (st != KDA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (a.total_tokens == 0) return copy_states_only(a, s);
-    return kda::launch_fused_gdn(a, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda::launch_pipe_gdn(a, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 namespace {

@@ -88,12 +88,11 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
 cudaError_t launch_state_affine(const float* A, const float* S, const float* B, float* out, int H,
                                 cudaStream_t stream);
 
-// The fused persistent tcgen05 kernel (same arguments; no workspace).
-cudaError_t launch_fused(const StagedArgs& a, cudaStream_t stream);
-// Scalar-gate (Gated DeltaNet) variant: a.g is [Ttot][H], a.dt_bias [H]; any lower bound.
-cudaError_t launch_fused_gdn(const StagedArgs& a, cudaStream_t stream);
-bool fused_supported(float lower_bound);
-// The warp-specialised product kernel of kda_fwd (same arguments and requirement on lower_bound).
+// The fused persistent tcgen05 kernel of kda_fwd (same arguments; no workspace); it needs
+// lower_bound >= KDA_FUSED_MIN_LOWER_BOUND (fused_supported).
 cudaError_t launch_pipe(const StagedArgs& a, cudaStream_t stream);
+bool fused_supported(float lower_bound);
+// Scalar-gate (Gated DeltaNet) variant: a.g is [Ttot][H], a.dt_bias [H]; any lower bound.
+cudaError_t launch_pipe_gdn(const StagedArgs& a, cudaStream_t stream);
 
 }  // namespace kda

@@ -102,6 +102,14 @@ constexpr uint32_t TM_AP = 320;   // A/P accumulator [128 rows][160]
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t IDESC_AP = idesc_f16(128, 160, true, false, false);
+constexpr uint32_t IDESC_AP_S = idesc_f16(128, 64, true, false, false);   // scalar gate: [K ; Q] K^T
+// Scalar-gate variant: q, k, v arrive as 128-byte-swizzled 64-channel blocks of 64 rows (8 KB
+// each), laid out k0 | q0 | k1 | q1 | v0 | v1 in the input region, so that [k ; q] is the 128-row
+// K-major A operand of the A/P MMA and k its B operand; its per-token gate quantities share the
+// block-product array.
+constexpr uint32_t S_GAM = S_PTOT;          // fp32 [64] Gamma (log2, inclusive in-chunk sum)
+constexpr uint32_t S_GE = S_PTOT + 256;     // fp32 [64] 2^Gamma
+constexpr uint32_t S_KF = S_PTOT + 512;     // fp32 [64] 2^(Gamma_63 - Gamma)
 constexpr uint32_t IDESC_OY = idesc_f16(128, 128, false, false, false);
 constexpr uint32_t IDESC_T = idesc_f16(128, 64, false, false, false);
 constexpr uint32_t IDESC_SO = idesc_f16(128, 192, false, false, true);
@@ -478,7 +486,64 @@ __device__ __noinline__ int chain_vals_reconvert(uint32_t lane_base, uint32_t co
     return d;
 }
 
+// ---- scalar-gate variant: gate and loads ----
+// One warp: lane l handles tokens 2l and 2l + 1 (gv = their raw gate inputs).  S_GAM gets the
+// inclusive in-chunk sum Gamma of log2 a (flat past the valid length), S_GE 2^Gamma and S_KF
+// 2^(Gamma_63 - Gamma).
+__device__ __forceinline__ void gate_scan_scalar(unsigned char* sm, const Params& p, int h, int L, float2 gv) {
+    const int lane = threadIdx.x & 31;
+    const float nexpA = -expf(p.A_log[h]);
+    const float lb2 = p.lower_bound * kLog2e;
+    const float db2 = p.dt_bias[h] * kLog2e;
+    const int r0 = 2 * lane;
+    float2 l;
+    {
+        const float x0 = fmaf(gv.x, kLog2e, db2), x1 = fmaf(gv.y, kLog2e, db2);
+        l.x = fmaxf(nexpA * fast_lg2(1.f + fast_ex2(x0)), lb2);
+        l.y = fmaxf(nexpA * fast_lg2(1.f + fast_ex2(x1)), lb2);
+    }
+    if (r0 >= L) l.x = 0.f;
+    if (r0 + 1 >= L) l.y = 0.f;
+    const float pair = l.x + l.y;
+    float incl = pair;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+    }
+    const float g0 = incl - pair + l.x, g1 = incl;
+    const float glast = __shfl_sync(0xffffffffu, incl, 31);
+    *reinterpret_cast<float2*>(reinterpret_cast<float*>(sm + S_GAM) + r0) = make_float2(g0, g1);
+    *reinterpret_cast<float2*>(reinterpret_cast<float*>(sm + S_GE) + r0) = make_float2(fast_ex2(g0), fast_ex2(g1));
+    *reinterpret_cast<float2*>(reinterpret_cast<float*>(sm + S_KF) + r0) =
+        make_float2(fast_ex2(glast - g0), fast_ex2(glast - g1));
+}
+
+__device__ __forceinline__ void issue_chunk_loads_s(unsigned char* sm, uint64_t* bar, const CUtensorMap* tq,
+                                                    const CUtensorMap* tk, const CUtensorMap* tv, int h,
+                                                    int64_t t0) {
+    mbar_arrive_expect_tx(bar, IN_BYTES);
+    const int x = h * kHeadDim, y = (int)t0;
+#pragma unroll
+    for (int cb = 0; cb < 2; ++cb) {
+        tma_load_2d(sm + IN_Q + (uint32_t)cb * 16384u, tk, x + 64 * cb, y, bar);
+        tma_load_2d(sm + IN_Q + (uint32_t)cb * 16384u + 8192u, tq, x + 64 * cb, y, bar);
+        tma_load_2d(sm + IN_V + (uint32_t)cb * 8192u, tv, x + 64 * cb, y, bar);
+    }
+}
+__device__ __forceinline__ void prefetch_chunk_s(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
+                                                 int h, int64_t t0) {
+    const int x = h * kHeadDim, y = (int)t0;
+#pragma unroll
+    for (int cb = 0; cb < 2; ++cb) {
+        tma_prefetch_2d(tq, x + 64 * cb, y);
+        tma_prefetch_2d(tk, x + 64 * cb, y);
+        tma_prefetch_2d(tv, x + 64 * cb, y);
+    }
+}
+
 // ---- the kernel ----
+template <bool kScalar>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -641,11 +706,21 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     *sAbort = 1u;
                 } else if (*sEnd == 0u) {
                     fence_after_sync();
-                    const uint32_t a0 = smem_u32(sm + AP_A), b0 = smem_u32(sm + AP_B);
+                    if constexpr (kScalar) {
+                        // [K ; Q] K^T straight from the swizzled input blocks (the decay is applied
+                        // at read-out)
+                        const uint32_t a0 = smem_u32(sm + IN_Q);
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
-                                ks > 0 ? 1u : 0u);
+                        for (int ks = 0; ks < 8; ++ks)
+                            mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(a0, 128, ks), IDESC_AP_S,
+                                    ks > 0 ? 1u : 0u);
+                    } else {
+                        const uint32_t a0 = smem_u32(sm + AP_A), b0 = smem_u32(sm + AP_B);
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks)
+                            mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
+                                    ks > 0 ? 1u : 0u);
+                    }
                     mma_commit(bar_ap);
                     ++issued_ap;
                 }
@@ -890,16 +965,33 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         Cursor cur = unit_from(p, sOrder, b, G, units, 0);
         float a[8][4];
         float beta_reg = 0.f;   // aux threads 0-63: beta of their token of the next chunk to form
+        float2 g_reg = make_float2(0.f, 0.f);   // scalar gate, warp 8: g of tokens 2 lane, 2 lane + 1
+        // the scalar gate's inputs of chunk c (rows past L read as 0)
+        auto load_g_scalar = [&](const Cursor& c) {
+            const int Lc = (int)(c.eos - c.t0 < kChunk ? c.eos - c.t0 : kChunk);
+            g_reg.x = 2 * lane < Lc ? p.g[(c.t0 + 2 * lane) * H + c.h] : 0.f;
+            g_reg.y = 2 * lane + 1 < Lc ? p.g[(c.t0 + 2 * lane + 1) * H + c.h] : 0.f;
+        };
         if (cur.valid) {
             if (issuer) {
-                issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, cur.h, cur.t0);
                 const Cursor n2 = next_chunk(p, sOrder, b, G, units, cur);
-                if (n2.valid) prefetch_chunk(&tm_q, &tm_k, &tm_v, &tm_g, n2.h, n2.t0);
+                if constexpr (kScalar) {
+                    issue_chunk_loads_s(sm, bar_in, &tm_q, &tm_k, &tm_v, cur.h, cur.t0);
+                    if (n2.valid) prefetch_chunk_s(&tm_q, &tm_k, &tm_v, n2.h, n2.t0);
+                } else {
+                    issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, cur.h, cur.t0);
+                    if (n2.valid) prefetch_chunk(&tm_q, &tm_k, &tm_v, &tm_g, n2.h, n2.t0);
+                }
             }
             tma_pending = true;
             const int L = (int)(cur.eos - cur.t0 < kChunk ? cur.eos - cur.t0 : kChunk);
-            if (!is_aux) gate_tokens(p, cur.h, cur.t0, L, c0, r0, a);
-            else if (at < kChunk && at < L) beta_reg = p.beta[(cur.t0 + at) * H + cur.h];
+            if (is_aux) {
+                if (at < kChunk && at < L) beta_reg = p.beta[(cur.t0 + at) * H + cur.h];
+            } else if constexpr (kScalar) {
+                if (warp == kElemWarp0) load_g_scalar(cur);
+            } else {
+                gate_tokens(p, cur.h, cur.t0, L, c0, r0, a);
+            }
         }
         uint32_t ci = 0;
         while (cur.valid) {
@@ -915,7 +1007,22 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // factors R (running product from the block start) and E (product to the block end)
             // where it needs them; po = product over the other 8-token half of its block.
             float po[4];
-            if (!is_aux) {
+            if constexpr (kScalar) {
+                // the inputs must have landed: rows past the valid length are zeroed in the tiles,
+                // which are MMA operands themselves
+                bad |= !warp_wait(bar_in, ci & 1u);
+                if (!is_aux) {
+                    for (int e = L * 8 + et; e < kChunk * 8; e += 256) {
+#pragma unroll
+                        for (int b6 = 0; b6 < 6; ++b6)
+                            st_v4(sm, IN_Q + (uint32_t)b6 * 8192u + (uint32_t)e * 16u, 0u, 0u, 0u, 0u);
+                    }
+                    if (warp == kElemWarp0) gate_scan_scalar(sm, p, h, L, g_reg);
+                } else if (at < kChunk) {
+                    reinterpret_cast<float*>(sm + S_BETA)[sl * 64u + at] = beta_reg;
+                }
+                fence_proxy_async();
+            } else if (!is_aux) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     float own = a[0][e];
@@ -932,8 +1039,10 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             named_bar_sync(BAR_FE, kFeThreads);
             PIPE_MARK(128, 0, 1);
             // ================ F2: A/P operand tiles (element) / P diagonal (aux) ================
-            bad |= !warp_wait(bar_in, ci & 1u);
-            if (!is_aux) {
+            if constexpr (!kScalar) bad |= !warp_wait(bar_in, ci & 1u);
+            if constexpr (kScalar) {
+                // the A/P MMA reads the input tiles directly; P's diagonal needs no correction
+            } else if (!is_aux) {
                 const float* ptot = reinterpret_cast<const float*>(sm + S_PTOT);
                 float4 pt[4];
 #pragma unroll
@@ -1020,7 +1129,47 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // ================ F4: the chain's operands (once it is done with the last chunk's) ================
             if (ci > 0) bad |= !warp_wait(bar_s, (ci - 1) & 1u);
             PIPE_MARK(128, 0, 4);
-            if (!is_aux) {
+            if (kScalar && !is_aux) {
+                // per-token scalings of the swizzled input blocks; inputs and outputs share the
+                // 128-byte-swizzled geometry, so an item is one 16-byte position of a row
+                const float* sb = reinterpret_cast<const float*>(sm + S_BETA) + sl * 64u;
+                const float* ge = reinterpret_cast<const float*>(sm + S_GE);
+                const float* kf = reinterpret_cast<const float*>(sm + S_KF);
+                uint32_t mq = 0u, mk = 0u;
+                float mbk = 0.f;
+#pragma unroll 1
+                for (int e = et; e < kChunk * 16; e += 256) {
+                    const int r = e >> 4;
+                    const uint32_t cb = (uint32_t)(e >> 3) & 1u, pos = (uint32_t)e & 7u;
+                    const uint32_t off = cb * 16384u + (uint32_t)r * 128u + pos * 16u;
+                    const uint4 kw = *reinterpret_cast<const uint4*>(sm + IN_Q + off);
+                    const uint4 qw = *reinterpret_cast<const uint4*>(sm + IN_Q + off + 8192u);
+                    const float g = ge[r], nbg = -sb[r] * g, kfr = kf[r];
+                    const float2 g2 = make_float2(g, g), nbg2 = make_float2(nbg, nbg), kf2 = make_float2(kfr, kfr);
+                    const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, qq[4] = {qw.x, qw.y, qw.z, qw.w};
+                    uint32_t oq[4], ok[4], oh[4];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mk) : "r"(kk[x]));
+                        asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mq) : "r"(qq[x]));
+                        const float2 kx = bf16x2_to_float2(kk[x]), qx = bf16x2_to_float2(qq[x]);
+                        const float2 gq = __fmul2_rn(g2, qx), bk = __fmul2_rn(nbg2, kx), kh = __fmul2_rn(kf2, kx);
+                        oq[x] = pack_f16s(gq.x, gq.y);
+                        ok[x] = pack_f16s(bk.x, bk.y);
+                        oh[x] = pack_f16s(kh.x, kh.y);
+                        mbk = fmaxf(mbk, fmaxf(fabsf(bk.x), fabsf(bk.y)));
+                    }
+                    st_tile4(sm, B1 + off, oq[0], oq[1], oq[2], oq[3]);
+                    st_tile4(sm, B1 + off + 8192u, ok[0], ok[1], ok[2], ok[3]);
+                    st_tile4(sm, KH + cb * 8192u + (uint32_t)r * 128u + pos * 16u, oh[0], oh[1], oh[2], oh[3]);
+                }
+                const float2 mkf = bf16x2_to_float2(mk), mqf = bf16x2_to_float2(mq);
+                if (fmaxf(fmaxf(fabsf(mkf.x), fabsf(mkf.y)), fmaxf(fabsf(mqf.x), fabsf(mqf.y))) >= kRangeHi ||
+                    mbk >= kRangeHi)
+                    range_bad = 1u;
+                if (et < kHeadDim)
+                    reinterpret_cast<float*>(sm + S_GC)[sl * kHeadDim + et] = ge[kChunk - 1];
+            } else if (!is_aux) {
                 const float* ptot = reinterpret_cast<const float*>(sm + S_PTOT);
                 float before[4] = {1.f, 1.f, 1.f, 1.f}, after[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
@@ -1086,8 +1235,13 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int t = 0; t < 8; ++t) {
                         const int r = 32 * th + 8 * j + t;
-                        w[t] = r < L ? *reinterpret_cast<const uint32_t*>(sm + IN_V + (uint32_t)r * 256u + (uint32_t)vp * 4u)
-                                     : 0u;
+                        uint32_t voff;
+                        if constexpr (kScalar)   // 64-channel swizzled blocks: element (r, v0) of block v0 / 64
+                            voff = (v0 >> 6) * 8192u + (uint32_t)r * 128u +
+                                   ((((v0 & 63u) >> 3) ^ ((uint32_t)r & 7u)) << 4) + (v0 & 7u) * 2u;
+                        else
+                            voff = (uint32_t)r * 256u + (uint32_t)vp * 4u;
+                        w[t] = r < L ? *reinterpret_cast<const uint32_t*>(sm + IN_V + voff) : 0u;
                     }
                     const uint32_t ch = (uint32_t)(4 * th + j);
                     st_tile4(sm, VT + v0 * 128u + ((ch ^ (v0 & 7u)) << 4), __byte_perm(w[0], w[1], 0x5410),
@@ -1114,16 +1268,27 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             PIPE_MARK(128, 0, 5);
             // ================ F5: hand the chunk to the chain; load the next one ================
-            if (issuer) {
-                mbar_arrive(bar_formed);
-                if (nxt.valid) {
+            // the next chunk's inputs: right away for the channel-wise gate (its A/P MMA reads the
+            // operand tiles); for the scalar gate once the A/P MMA, which reads the input tiles
+            // themselves, is done (in F6)
+            auto load_next = [&]() {
+                const Cursor n2 = next_chunk(p, sOrder, b, G, units, nxt);
+                if constexpr (kScalar) {
+                    issue_chunk_loads_s(sm, bar_in, &tm_q, &tm_k, &tm_v, nxt.h, nxt.t0);
+                    if (n2.valid) prefetch_chunk_s(&tm_q, &tm_k, &tm_v, n2.h, n2.t0);
+                } else {
                     issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, nxt.h, nxt.t0);
-                    const Cursor n2 = next_chunk(p, sOrder, b, G, units, nxt);
                     if (n2.valid) prefetch_chunk(&tm_q, &tm_k, &tm_v, &tm_g, n2.h, n2.t0);
                 }
+            };
+            if (issuer) {
+                mbar_arrive(bar_formed);
+                if (!kScalar && nxt.valid) load_next();
             }
-            tma_pending = nxt.valid;
-            tma_parity = (ci + 1u) & 1u;
+            if (!kScalar) {
+                tma_pending = nxt.valid;
+                tma_parity = (ci + 1u) & 1u;
+            }
             // beta of the next chunk: its latency is hidden behind the read-out and the solve
             if (is_aux && at < kChunk) {
                 const int L1 = nxt.valid ? (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk) : 0;
@@ -1134,11 +1299,21 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // the solve).
             if (!is_aux) {
                 if (nxt.valid) {
-                    const int L1 = (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk);
-                    gate_tokens(p, nxt.h, nxt.t0, L1, c0, r0, a);
+                    if constexpr (kScalar) {
+                        if (warp == kElemWarp0) load_g_scalar(nxt);
+                    } else {
+                        const int L1 = (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk);
+                        gate_tokens(p, nxt.h, nxt.t0, L1, c0, r0, a);
+                    }
                 }
             } else {
-                if (!warp_wait(bar_ap, ci & 1u)) *sAbort = 1u;
+                const bool ap_done = warp_wait(bar_ap, ci & 1u);
+                if (!ap_done) *sAbort = 1u;
+                if (kScalar && ap_done && nxt.valid) {
+                    if (issuer) load_next();
+                    tma_pending = true;
+                    tma_parity = (ci + 1u) & 1u;
+                }
                 fence_after_sync();
                 PIPE_MARK(128, 0, 6);
                 const bool isA = quarter < 2;
@@ -1159,6 +1334,21 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                         for (int x = 0; x < 16; ++x) row[x] = __uint_as_float(I == I_a ? ta[x] : tb[x]);
                     };
+                    if constexpr (kScalar) {
+                        // raw K K^T / Q K^T times the scalar decay 2^(Gamma_r - Gamma_i) (<= 1 on and
+                        // below the diagonal)
+                        uint32_t raw[16];
+                        tmem_ld16(taddr(tbase, quarter, TM_AP + (uint32_t)J * 16u), raw);
+                        tmem_wait_ld();
+                        const float* gam = reinterpret_cast<const float*>(sm + S_GAM);
+                        const float gr = gam[r];
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            const int i = J * 16 + x;
+                            const bool keep = isA ? (i < r) : (i <= r);
+                            row[x] = keep ? __uint_as_float(raw[x]) * fast_ex2(gr - gam[i]) : 0.f;
+                        }
+                    } else {
                     if ((quarter & 1) == 0) {        // I in {0, 1}
                         if (J == 0) pick(0, 64, 0);            // I=0: diagonal; I=1: C1 of block 0
                         else if (J == 1) pick(16, 16, 1);      // I=1: diagonal (I=0: masked)
@@ -1176,6 +1366,7 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     for (int x = 0; x < 16; ++x) {
                         const int i = J * 16 + x;
                         row[x] = i < r ? row[x] : ((i == r && !isA) ? pdg : 0.f);
+                    }
                     }
                     if (isA) {
                         float* a32 = reinterpret_cast<float*>(sm + A32) + r * kF32Pitch + J * 16;
@@ -1350,9 +1541,39 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
 // ---- host side ----
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda symbol).
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D map over [rows][cols] with a box of box_cols x 64 rows; swizzled maps put each box in the
+// 128-byte-swizzled K-major layout of the MMA operands.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t elem, int64_t rows, int64_t cols,
+              uint32_t box_cols = kHeadDim, bool swizzle128 = false) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * elem};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)kChunk};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kScalar>
 cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
     cudaError_t err = once_per_device([](int) {
-        return cudaFuncSetAttribute(kda_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
+        return cudaFuncSetAttribute(kda_pipe_kernel<kScalar>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)SMEM_ALLOC);
     });
     if (err != cudaSuccess) return err;
     int dev = 0, sm_count = 0;
@@ -1361,11 +1582,18 @@ cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
     if (sm_count <= 0) return cudaErrorInvalidDevice;
     CUtensorMap tq, tk, tv, tg;
     const int64_t rows = a.total_tokens, cols = (int64_t)a.H * kHeadDim;
-    if (!fused::make_map(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols) ||
-        !fused::make_map(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols) ||
-        !fused::make_map(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols) ||
-        !fused::make_map(&tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols))
+    // channel-wise gate: 128-channel unswizzled boxes (CUDA cores read them); scalar gate:
+    // 64-channel 128-byte-swizzled boxes (the MMA reads them)
+    const uint32_t box = kScalar ? 64u : (uint32_t)kHeadDim;
+    if (!make_map(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box, kScalar) ||
+        !make_map(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box, kScalar) ||
+        !make_map(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box, kScalar))
         return cudaErrorInvalidValue;
+    if (kScalar) {
+        tg = tq;   // unused: the scalar gate input is read with plain loads
+    } else if (!make_map(&tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols)) {
+        return cudaErrorInvalidValue;
+    }
     Params p;
     p.g = a.g;
     p.beta = a.beta;
@@ -1384,7 +1612,7 @@ cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
     const int64_t units = (int64_t)a.N * a.H;
     const int grid = (int)(units < sm_count ? units : sm_count);
     if (grid <= 0) return cudaSuccess;
-    kda_pipe_kernel<<<grid, kThreads, SMEM_ALLOC, stream>>>(tq, tk, tv, tg, p);
+    kda_pipe_kernel<kScalar><<<grid, kThreads, SMEM_ALLOC, stream>>>(tq, tk, tv, tg, p);
     return cudaGetLastError();
 }
 
@@ -1402,6 +1630,8 @@ extern "C" int kda_debug_pipe_phase_cycles(unsigned long long* out) {
 }
 #endif
 
-cudaError_t launch_pipe(const StagedArgs& a, cudaStream_t stream) { return pipe::launch(a, stream); }
+bool fused_supported(float lower_bound) { return lower_bound >= KDA_FUSED_MIN_LOWER_BOUND; }
+cudaError_t launch_pipe(const StagedArgs& a, cudaStream_t stream) { return pipe::launch<false>(a, stream); }
+cudaError_t launch_pipe_gdn(const StagedArgs& a, cudaStream_t stream) { return pipe::launch<true>(a, stream); }
 
 }  // namespace kda

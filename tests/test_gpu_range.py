@@ -147,3 +147,24 @@ def test_out_of_range_keys_are_flagged_not_inf():
     bits = kda.kda_check_device_error()
     assert bits & KDA_DEVERR_RANGE, f"expected the range bit, got bits {bits:#x}"
     assert torch.isfinite(out.float()).all() and torch.isfinite(fin).all()
+
+
+@pytest.mark.parametrize("lb", [-5.0, -20.0])
+def test_range_scalar_gate_matches_oracle(lb):
+    """kda_gdn_fwd (one decay per token-head) shares the state chain and its per-column scale:
+    huge initial states and v x 1e3 against the fp64 scalar-gate oracle."""
+    kda = _kda()
+    w = W.custom([300, 77, 130], H=3, init="normal", lower_bound=lb, wid=47)
+    x = W.gdn_inputs(W.make_inputs(w))
+    x["initial_state"] = _big_state(x, 11)
+    x["v"] = (x["v"].float() * 1e3).to(torch.bfloat16)
+    xd = to_device(x)
+    fin = alloc_final(xd, True)
+    out, fin = kda.kda_gdn_fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"],
+                               x["lower_bound"], x["scale"], xd["initial_state"], xd["cu_seqlens"],
+                               final_state=fin, batch=x["batch"])
+    bits = kda.kda_check_device_error()
+    assert bits == 0, f"device error bits {bits:#x}"
+    ref_o, ref_f = oracle.gdn_recurrent(x["q"], x["k"], x["v"], x["g"], x["beta"], x["A_log"], x["dt_bias"],
+                                        x["lower_bound"], x["scale"], x["initial_state"], x["cu_seqlens"])
+    _check(out, fin, ref_o, ref_f, f"scalar gate lb={lb}")
