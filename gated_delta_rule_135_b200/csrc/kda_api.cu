@@ -6,7 +6,6 @@
 #include <math.h>
 #include <string.h>
 
-#include <mutex>
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -120,25 +119,14 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of the scratch on the current device, resolved once per
-// device (host code may not use the array's name as a device address).
+// Device address of the scratch in the current context, looked up on every call (host code
+// may not use the array's name as a device address).  Nothing is cached, so a context created
+// after cudaDeviceReset gets its own array's address.
 cudaError_t noalloc_scratch(void** out) {
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
+    void* ptr = nullptr;
+    const cudaError_t err = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
     if (err != cudaSuccess) return err;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
-        void* ptr = nullptr;
-        err = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-        if (err != cudaSuccess) return err;
-        g_noalloc_ptr[dev] = ptr;
-    }
-    *out = g_noalloc_ptr[dev];
+    *out = ptr;
     return cudaSuccess;
 }
 

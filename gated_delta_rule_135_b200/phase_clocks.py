@@ -1,0 +1,102 @@
+"""Per-phase cycle counts of the fused prefill kernel (a profiling aid, not part of the ABI).
+
+Builds the instrumented library (``build.py --phase-clocks``: the same kernel with clock64()
+marks between its phases, accumulated per CTA), runs one workload through it and prints the
+average cycles per 64-token chunk of each phase, for the front end (thread 128) and the state
+chain (thread 0).  Run it by path from the repository root (importing the package loads the
+product library, so this script sets KDA_LIBRARY before it imports the package):
+
+    python gated_delta_rule_135_b200/phase_clocks.py [--workload 2] [--gdn]
+
+The instrumented build is slower than the product build (the marks serialise a little); compare
+phases with each other, not the printed kernel time with the bench.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import os
+import sys
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_ROOT = os.path.dirname(_HERE)
+
+# index = slot of the kernel's phase marks; each counts the cycles since the previous mark
+# of the same role
+PHASES = [
+    ("FE", "solve L1 + L2, loop to the next chunk"),
+    ("FE", "F0 block products of a / beta"),
+    ("FE", "F2 A/P operand tiles, P diagonal"),
+    ("FE", "F3 signal A/P operands ready"),
+    ("FE", "F4 wait for the previous state update"),
+    ("FE", "F4 B1, Khat, V^T tiles"),
+    ("FE", "F5/F6 hand-off, next TMA, wait for A/P"),
+    ("FE", "F6 A / P read-out"),
+    ("FE", "solve L0 (diagonal blocks)"),
+    ("chain", "wait for the previous [S|O] MMA"),
+    ("chain", "output of the previous chunk"),
+    ("chain", "wait for A/P operands, issue the A/P MMA"),
+    ("chain", "(between marks)"),
+    ("chain", "wait for the chunk's operands"),
+    ("chain", "S^T -> fp16, [O|Y] MMA, S <- S Diag(gamma_C)"),
+    ("chain", "wait [O|Y], Y^T += beta V^T -> fp16"),
+    ("chain", "wait T, U MMA, wait U"),
+    ("chain", "U -> fp16, [S|O] MMA issue"),
+]
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--gdn", action="store_true", help="the scalar-gate forward (kda_gdn_fwd)")
+    args = ap.parse_args(argv)
+
+    sys.path.insert(0, _ROOT)
+    import kda_build
+    lib_path = kda_build.build(phase_clocks=True)
+    os.environ["KDA_LIBRARY"] = lib_path
+    import torch
+
+    import gated_delta_rule_135_b200 as kda
+    import kda_workloads as W
+
+    w = W.WORKLOADS[args.workload]
+    x = W.make_inputs(w)
+    if args.gdn:
+        x = W.gdn_inputs(x)
+    xd = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    fin = torch.empty(w.N, w.H, 128, 128, device="cuda") if w.final else None
+    fwd = kda.kda_gdn_fwd if args.gdn else kda.kda_fwd
+
+    def step():
+        fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"], x["lower_bound"],
+            x["scale"], xd["initial_state"], xd["cu_seqlens"], final_state=fin, batch=x["batch"])
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    lib = kda.lib()
+    lib.kda_debug_pipe_phase_cycles.restype = ctypes.c_int
+    buf = (ctypes.c_ulonglong * len(PHASES))()
+    if lib.kda_debug_pipe_phase_cycles(buf) != len(PHASES):   # clears the counters
+        raise RuntimeError("phase counters not available in this build")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    step()
+    e1.record()
+    torch.cuda.synchronize()
+    if lib.kda_debug_pipe_phase_cycles(buf) != len(PHASES):
+        raise RuntimeError("reading the phase counters failed")
+    chunks = sum((s + 63) // 64 for s in w.seq_lens) * w.H
+    print(f"instrumented kernel {e0.elapsed_time(e1):.3f} ms, {chunks} chunk-heads")
+    tot = {"FE": 0.0, "chain": 0.0}
+    for (role, name), c in zip(PHASES, buf):
+        per = c / chunks
+        tot[role] += per
+        print(f"{role:5s}  {name:46s} {per:8.0f} cycles/chunk")
+    print(f"front end {tot['FE']:.0f}, chain {tot['chain']:.0f} cycles/chunk")
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -41,6 +41,10 @@
  * A kernel that detects a violated precondition on the device (offsets out of
  * range, a wait that ran out) records it in a device error word instead of
  * faulting; kda_check_device_error() reads and clears it.
+ * Contexts: the library sets its kernels' shared-memory attributes once per device and
+ * process.  Do not call it again after cudaDeviceReset in the same process: the attributes
+ * belong to the destroyed context, and the launches of the new one are refused (KDA_ERR_CUDA).
+ * Nothing else is cached across calls (kda_fwd_staged_noalloc looks its scratch up each time).
  */
 #ifndef KDA_H
 #define KDA_H
