@@ -154,6 +154,10 @@ __device__ unsigned long long g_pipe_phase_cycles[kPhases];
 #endif
 
 // ---- small helpers ----
+// Pulls the line holding `ptr` into L2 (no register result, never waited on).
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -307,15 +311,6 @@ __device__ __forceinline__ void issue_chunk_loads(unsigned char* sm, uint64_t* b
     tma_load_2d(sm + IN_Q, tq, x, y, bar);
     tma_load_2d(sm + IN_K, tk, x, y, bar);
     tma_load_2d(sm + IN_V, tv, x, y, bar);
-}
-__device__ __forceinline__ void prefetch_chunk(const CUtensorMap* tq, const CUtensorMap* tk,
-                                               const CUtensorMap* tv, const CUtensorMap* tg, int h,
-                                               int64_t t0) {
-    const int x = h * kHeadDim, y = (int)t0;
-    tma_prefetch_2d(tq, x, y);
-    tma_prefetch_2d(tk, x, y);
-    tma_prefetch_2d(tv, x, y);
-    tma_prefetch_2d(tg, x, y);
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -531,22 +526,12 @@ __device__ __forceinline__ void issue_chunk_loads_s(unsigned char* sm, uint64_t*
         tma_load_2d(sm + IN_V + (uint32_t)cb * 8192u, tv, x + 64 * cb, y, bar);
     }
 }
-__device__ __forceinline__ void prefetch_chunk_s(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
-                                                 int h, int64_t t0) {
-    const int x = h * kHeadDim, y = (int)t0;
-#pragma unroll
-    for (int cb = 0; cb < 2; ++cb) {
-        tma_prefetch_2d(tq, x + 64 * cb, y);
-        tma_prefetch_2d(tk, x + 64 * cb, y);
-        tma_prefetch_2d(tv, x + 64 * cb, y);
-    }
-}
 
 // ---- the kernel ----
 template <bool kScalar>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                const __grid_constant__ CUtensorMap tm_v,
                 const Params p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -955,8 +940,8 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int c0 = 64 * ehf + 4 * (lane & 15);
         const int r0 = 16 * eI + 8 * (lane >> 4);
         const int quarter = warp & 3;       // TMEM lane quarter of this warp
-        const int fsub = (warp - kAuxWarp0) >> 2;   // 0 aux, 1 warps 8-11, 2 warps 12-15
-        const bool issuer = tid == 128;
+        const bool issuer = tid == 128;      // barrier arrivals of the front end
+        const bool loader = tid == 256;      // TMA loads of the next chunk (element warp 8)
         bool tma_pending = false;
         uint32_t tma_parity = 0;
         bool aborted = false;
@@ -974,19 +959,15 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         };
         if (cur.valid) {
             if (issuer) {
-                const Cursor n2 = next_chunk(p, sOrder, b, G, units, cur);
-                if constexpr (kScalar) {
+                if constexpr (kScalar)
                     issue_chunk_loads_s(sm, bar_in, &tm_q, &tm_k, &tm_v, cur.h, cur.t0);
-                    if (n2.valid) prefetch_chunk_s(&tm_q, &tm_k, &tm_v, n2.h, n2.t0);
-                } else {
+                else
                     issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, cur.h, cur.t0);
-                    if (n2.valid) prefetch_chunk(&tm_q, &tm_k, &tm_v, &tm_g, n2.h, n2.t0);
-                }
             }
             tma_pending = true;
             const int L = (int)(cur.eos - cur.t0 < kChunk ? cur.eos - cur.t0 : kChunk);
             if (is_aux) {
-                if (at < kChunk && at < L) beta_reg = p.beta[(cur.t0 + at) * H + cur.h];
+                if (at < kChunk) beta_reg = p.beta[(cur.t0 + (at < L ? at : L - 1)) * H + cur.h];
             } else if constexpr (kScalar) {
                 if (warp == kElemWarp0) load_g_scalar(cur);
             } else {
@@ -1002,6 +983,20 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint32_t sl = ci & 1u;
             bool bad = false;
             PIPE_MARK(128, 0, 0);
+            // the next chunk's gate input into L2 (its q, k, v come by TMA once this chunk's are used)
+            if (nxt.valid) {
+                const int L1 = (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk);
+                if constexpr (kScalar) {
+                    if (warp == kElemWarp0) {
+                        if (2 * lane < L1) prefetch_l2(p.g + (nxt.t0 + 2 * lane) * H + nxt.h);
+                        if (2 * lane + 1 < L1) prefetch_l2(p.g + (nxt.t0 + 2 * lane + 1) * H + nxt.h);
+                    }
+                } else if (!is_aux) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        if (r0 + i < L1) prefetch_l2(p.g + ((nxt.t0 + r0 + i) * H + nxt.h) * kHeadDim + c0);
+                }
+            }
             // ================ F0: block products of a (element) / beta (aux) ================
             // Each element thread keeps its 32 values a_t across the phases and rebuilds the
             // factors R (running product from the block start) and E (product to the block end)
@@ -1019,7 +1014,7 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     if (warp == kElemWarp0) gate_scan_scalar(sm, p, h, L, g_reg);
                 } else if (at < kChunk) {
-                    reinterpret_cast<float*>(sm + S_BETA)[sl * 64u + at] = beta_reg;
+                    reinterpret_cast<float*>(sm + S_BETA)[sl * 64u + at] = at < L ? beta_reg : 0.f;
                 }
                 fence_proxy_async();
             } else if (!is_aux) {
@@ -1034,7 +1029,7 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         reinterpret_cast<float*>(sm + S_PTOT)[eI * kHeadDim + c0 + e] = own;
                 }
             } else if (at < kChunk) {
-                reinterpret_cast<float*>(sm + S_BETA)[sl * 64u + at] = beta_reg;
+                reinterpret_cast<float*>(sm + S_BETA)[sl * 64u + at] = at < L ? beta_reg : 0.f;
             }
             named_bar_sync(BAR_FE, kFeThreads);
             PIPE_MARK(128, 0, 1);
@@ -1271,49 +1266,50 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // the next chunk's inputs: right away for the channel-wise gate (its A/P MMA reads the
             // operand tiles); for the scalar gate once the A/P MMA, which reads the input tiles
             // themselves, is done (in F6)
+            // (issued by an element thread: a TMA issue blocks its thread for several hundred
+            // cycles, which the aux warps' read-out and solve cannot spare)
             auto load_next = [&]() {
-                const Cursor n2 = next_chunk(p, sOrder, b, G, units, nxt);
-                if constexpr (kScalar) {
+                if constexpr (kScalar)
                     issue_chunk_loads_s(sm, bar_in, &tm_q, &tm_k, &tm_v, nxt.h, nxt.t0);
-                    if (n2.valid) prefetch_chunk_s(&tm_q, &tm_k, &tm_v, n2.h, n2.t0);
-                } else {
+                else
                     issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, nxt.h, nxt.t0);
-                    if (n2.valid) prefetch_chunk(&tm_q, &tm_k, &tm_v, &tm_g, n2.h, n2.t0);
-                }
             };
-            if (issuer) {
-                mbar_arrive(bar_formed);
-                if (!kScalar && nxt.valid) load_next();
-            }
+            if (issuer) mbar_arrive(bar_formed);
+            if (!kScalar && loader && nxt.valid) load_next();
             if (!kScalar) {
                 tma_pending = nxt.valid;
                 tma_parity = (ci + 1u) & 1u;
             }
-            // beta of the next chunk: its latency is hidden behind the read-out and the solve
-            if (is_aux && at < kChunk) {
-                const int L1 = nxt.valid ? (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk) : 0;
-                beta_reg = at < L1 ? p.beta[(nxt.t0 + at) * H + nxt.h] : 0.f;
+            // beta of the next chunk: its latency is hidden behind the read-out and the solve (the
+            // load is unconditional, row clamped, so that nothing consumes it before the next F0)
+            if (is_aux && at < kChunk && nxt.valid) {
+                const int L1 = (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk);
+                beta_reg = p.beta[(nxt.t0 + (at < L1 ? at : L1 - 1)) * H + nxt.h];
             }
             // ================ F6: A / P read-out (aux warps, one per TMEM lane quarter) ================
             // The element warps meanwhile compute the next chunk's gate (it overlaps the read-out and
             // the solve).
             if (!is_aux) {
-                if (nxt.valid) {
-                    if constexpr (kScalar) {
-                        if (warp == kElemWarp0) load_g_scalar(nxt);
-                    } else {
-                        const int L1 = (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk);
-                        gate_tokens(p, nxt.h, nxt.t0, L1, c0, r0, a);
+                if constexpr (kScalar) {
+                    // warp 8: the next chunk's gate input, then (once the A/P MMA has read the input
+                    // tiles) the next chunk's TMA loads
+                    if (warp == kElemWarp0) {
+                        if (nxt.valid) load_g_scalar(nxt);
+                        const bool ap_done = warp_wait(bar_ap, ci & 1u);
+                        if (!ap_done) *sAbort = 1u;
+                        if (ap_done && nxt.valid) {
+                            if (loader) load_next();
+                            tma_pending = true;
+                            tma_parity = (ci + 1u) & 1u;
+                        }
                     }
+                } else if (nxt.valid) {
+                    const int L1 = (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk);
+                    gate_tokens(p, nxt.h, nxt.t0, L1, c0, r0, a);
                 }
             } else {
                 const bool ap_done = warp_wait(bar_ap, ci & 1u);
                 if (!ap_done) *sAbort = 1u;
-                if (kScalar && ap_done && nxt.valid) {
-                    if (issuer) load_next();
-                    tma_pending = true;
-                    tma_parity = (ci + 1u) & 1u;
-                }
                 fence_after_sync();
                 PIPE_MARK(128, 0, 6);
                 const bool isA = quarter < 2;
@@ -1522,9 +1518,7 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         } else {
             *sAbort = 1u;
-            if (issuer) {
-                if (tma_pending) mbar_wait_bounded(bar_in, tma_parity);
-            }
+            if ((issuer || loader) && tma_pending) mbar_wait_bounded(bar_in, tma_parity);
         }
     }
 
@@ -1580,7 +1574,7 @@ cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
     if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
     if ((err = cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
     if (sm_count <= 0) return cudaErrorInvalidDevice;
-    CUtensorMap tq, tk, tv, tg;
+    CUtensorMap tq, tk, tv;
     const int64_t rows = a.total_tokens, cols = (int64_t)a.H * kHeadDim;
     // channel-wise gate: 128-channel unswizzled boxes (CUDA cores read them); scalar gate:
     // 64-channel 128-byte-swizzled boxes (the MMA reads them)
@@ -1589,11 +1583,6 @@ cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
         !make_map(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box, kScalar) ||
         !make_map(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box, kScalar))
         return cudaErrorInvalidValue;
-    if (kScalar) {
-        tg = tq;   // unused: the scalar gate input is read with plain loads
-    } else if (!make_map(&tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols)) {
-        return cudaErrorInvalidValue;
-    }
     Params p;
     p.g = a.g;
     p.beta = a.beta;
@@ -1612,7 +1601,7 @@ cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
     const int64_t units = (int64_t)a.N * a.H;
     const int grid = (int)(units < sm_count ? units : sm_count);
     if (grid <= 0) return cudaSuccess;
-    kda_pipe_kernel<kScalar><<<grid, kThreads, SMEM_ALLOC, stream>>>(tq, tk, tv, tg, p);
+    kda_pipe_kernel<kScalar><<<grid, kThreads, SMEM_ALLOC, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 
