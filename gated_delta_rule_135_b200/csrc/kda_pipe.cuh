@@ -54,7 +54,7 @@ constexpr int kThreads = 512;
 constexpr int kFeThreads = 384;          // warps 4-15
 constexpr int kAuxWarp0 = 4, kElemWarp0 = 8;
 // named barriers (0 is __syncthreads)
-constexpr uint32_t BAR_FE = 1, BAR_CHAIN = 2, BAR_AUX = 3;
+constexpr uint32_t BAR_FE = 1, BAR_CHAIN = 2, BAR_AUX = 3, BAR_ELEM = 4;
 
 // ---- shared memory (bytes from a 1024-aligned base) ----
 constexpr uint32_t IN_Q = 0;           // bf16 [64][128] row-major TMA boxes
@@ -63,9 +63,6 @@ constexpr uint32_t IN_V = 32768;
 constexpr uint32_t IN_BYTES = 49152;
 constexpr uint32_t AP_A = 49152;       // bf16 K-major [128 rows][128]: k R rows 0-63, q R rows 64-127
 constexpr uint32_t AP_B = 81920;       // bf16 K-major [160 rows][128]: XD | C1 | C2 | C3
-constexpr int kF32Pitch = 68;          // fp32 row pitch of A32 / T32
-constexpr uint32_t A32 = AP_A;         // fp32 [64][68] beta-scaled A (after the A/P MMA)
-constexpr uint32_t T32 = AP_A + 17408; // fp32 [64][68] T
 constexpr uint32_t B1 = 122880;        // fp16 K-major [128 rows][128]: gamma q rows 0-63, -beta gamma k 64-127
 constexpr uint32_t B2 = 155648;        // fp16 MN-major, K = 64 tokens: Khat (c 0-63 | c 64-127) | P^T
 constexpr uint32_t KH = B2;
@@ -76,22 +73,34 @@ constexpr uint32_t MISC = 204800;
 constexpr uint32_t S_BETA = MISC;              // fp32 [2][64] (by chunk parity)
 constexpr uint32_t S_GC = MISC + 512;          // fp32 [2][128] gamma_C = e^{Gamma_63}
 constexpr uint32_t S_PTOT = MISC + 1536;       // fp32 [4][128] per-block products of a
-constexpr uint32_t S_PD = MISC + 3584;         // fp32 [2][64] halves of q_r . k_r
+constexpr uint32_t S_PD = MISC + 3584;         // fp32 [2][64] halves of q_r . k_r (of the chunk the aux
+                                               // warps formed last)
 constexpr uint32_t S_ORDER = MISC + 4096;      // int16 [kSortLimit]
 constexpr int kSortLimit = 512;
 constexpr uint32_t S_META = S_ORDER + 2 * kSortLimit;   // int32 [2][8] chunk metadata
-constexpr uint32_t S_BARS = S_META + 64;                // u64 [8]
-constexpr uint32_t S_TMEM = S_BARS + 64;                // u32 tmem base, u32 abort flag
-constexpr uint32_t S_PH = S_TMEM + 16;                  // u64 [kPhases + 2] (phase-clock builds)
-constexpr int kPhases = 18;
-#ifdef KDA_PHASE_CLOCKS
-constexpr uint32_t SMEM_BYTES = S_PH + 8 * (kPhases + 2);
-#else
-constexpr uint32_t SMEM_BYTES = S_PH;
-#endif
+constexpr uint32_t S_BARS = S_META + 64;                // u64 [16]
+constexpr int kNumBars = 9;
+constexpr uint32_t S_TMEM = S_BARS + 128;               // u32 tmem base, u32 abort flag
+constexpr uint32_t S_PH = S_TMEM + 16;                  // u64 [kPhases + 3] (phase-clock builds)
+constexpr int kPhases = 24;
+// The triangular solve's scratch, apart from the A/P operand tiles (which the element warps
+// rewrite for the next chunk while the aux warps solve): A's diagonal 16 x 16 blocks in fp32
+// (row pitch 20 floats), its six blocks below the diagonal and the solve's intermediate blocks
+// in fp16 (row pitch 24 halves; both pitches keep row accesses free of bank conflicts).
+constexpr uint32_t SV = 210432;
+constexpr int kAdPitch = 20;
+constexpr int kHp = 24;
+constexpr uint32_t kHBlk = 16 * kHp * 2;                // bytes of one fp16 block
+constexpr uint32_t SV_AD = SV;                          // fp32 [4][16][20]
+constexpr uint32_t SV_AL = SV_AD + 4 * 16 * kAdPitch * 4;   // fp16 [6][16][24]: A10 A20 A21 A30 A31 A32
+constexpr uint32_t SV_SC = SV_AL + 6 * kHBlk;           // fp16 [8][16][24] intermediates
+constexpr uint32_t SC_Y0 = SV_SC, SC_Y2 = SV_SC + kHBlk, SC_T10B = SV_SC + 2 * kHBlk, SC_X20 = SV_SC + 3 * kHBlk,
+                   SC_X30 = SV_SC + 4 * kHBlk, SC_X21 = SV_SC + 5 * kHBlk, SC_X31 = SV_SC + 6 * kHBlk,
+                   SC_Y32 = SV_SC + 7 * kHBlk;
+constexpr uint32_t SMEM_BYTES = SV_SC + 8 * kHBlk;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
+static_assert(S_PH + 8 * (kPhases + 3) <= SV, "phase slots below the solve scratch");
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
-static_assert(T32 + 64 * kF32Pitch * 4 <= B1, "solve scratch inside the A/P operand region");
 
 // ---- TMEM columns ----
 constexpr uint32_t TM_S = 0;      // S^T fp32 [128 v][128 c]
@@ -106,10 +115,11 @@ constexpr uint32_t IDESC_AP_S = idesc_f16(128, 64, true, false, false);   // sca
 // Scalar-gate variant: q, k, v arrive as 128-byte-swizzled 64-channel blocks of 64 rows (8 KB
 // each), laid out k0 | q0 | k1 | q1 | v0 | v1 in the input region, so that [k ; q] is the 128-row
 // K-major A operand of the A/P MMA and k its B operand; its per-token gate quantities share the
-// block-product array.
-constexpr uint32_t S_GAM = S_PTOT;          // fp32 [64] Gamma (log2, inclusive in-chunk sum)
-constexpr uint32_t S_GE = S_PTOT + 256;     // fp32 [64] 2^Gamma
-constexpr uint32_t S_KF = S_PTOT + 512;     // fp32 [64] 2^(Gamma_63 - Gamma)
+// block-product array, one set per chunk parity (the aux warps read a chunk's Gamma while the
+// element warps form the next chunk's).
+__host__ __device__ constexpr uint32_t s_gam(uint32_t sl) { return S_PTOT + sl * 768u; }   // fp32 [64] Gamma (log2)
+__host__ __device__ constexpr uint32_t s_ge(uint32_t sl) { return s_gam(sl) + 256u; }      // fp32 [64] 2^Gamma
+__host__ __device__ constexpr uint32_t s_kf(uint32_t sl) { return s_gam(sl) + 512u; }      // fp32 [64] 2^(Gamma_63 - Gamma)
 constexpr uint32_t IDESC_OY = idesc_f16(128, 128, false, false, false);
 constexpr uint32_t IDESC_T = idesc_f16(128, 64, false, false, false);
 constexpr uint32_t IDESC_SO = idesc_f16(128, 192, false, false, true);
@@ -256,6 +266,55 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
     return ok;
 }
 
+// ---- 16 x 16 fp16 block products of the triangular solve (mma.sync m16n8k16, fp32 accumulation) ----
+// Operands come from shared memory through ldmatrix: lane l gives the address of row (l & 15),
+// columns 8 (l >> 4) .. 8 (l >> 4) + 7 of the block.  Without .trans that yields the A fragment of
+// a row-major block; with .trans the B fragment of a row-major [k][n] block.
+__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
+}
+// acc (+)= P Q for 16 x 16 blocks at ldmatrix row addresses pa (P) and qa (Q)
+__device__ __forceinline__ void mm16h(float (&acc)[2][4], uint32_t pa, uint32_t qa) {
+    uint32_t a[4], b[4];
+    ldsm4(pa, a);
+    ldsm4t(qa, b);
+    const uint32_t b0[2] = {b[0], b[1]}, b1[2] = {b[2], b[3]};
+    warpmma::mma_f16_16816(acc[0], a, b0);
+    warpmma::mma_f16_16816(acc[1], a, b1);
+}
+// ldmatrix row address of a fp16 block at byte offset `off` (row pitch kHp halves)
+__device__ __forceinline__ uint32_t lm_blk(const unsigned char* sm, uint32_t off) {
+    const uint32_t lane = threadIdx.x & 31u;
+    return smem_u32(sm) + off + (lane & 15u) * (uint32_t)kHp * 2u + (lane >> 4) * 16u;
+}
+// ldmatrix row address of block (I, J) of the 128-byte-swizzled fp16 T tile [64 r][64 i]
+__device__ __forceinline__ uint32_t lm_t16(const unsigned char* sm, int I, int J) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t row = 16u * (uint32_t)I + (lane & 15u), chunk = 2u * (uint32_t)J + (lane >> 4);
+    return smem_u32(sm) + T16 + row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+// sign * accumulator -> fp16 block at byte offset `off` (round to nearest, as an operand load would)
+__device__ __forceinline__ void store16h(unsigned char* sm, uint32_t off, const float (&acc)[2][4], float sign) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+        const uint32_t col = (uint32_t)(8 * nh + 2 * t);
+        *reinterpret_cast<uint32_t*>(sm + off + ((uint32_t)g * kHp + col) * 2u) =
+            warpmma::pack_half2(sign * acc[nh][0], sign * acc[nh][1]);
+        *reinterpret_cast<uint32_t*>(sm + off + ((uint32_t)(g + 8) * kHp + col) * 2u) =
+            warpmma::pack_half2(sign * acc[nh][2], sign * acc[nh][3]);
+    }
+}
+// index of A's block (I, J), J < I, among the six below the diagonal
+__device__ __forceinline__ uint32_t al_off(int I, int J) {
+    return SV_AL + (uint32_t)(I * (I - 1) / 2 + J) * kHBlk;
+}
+
 // ---- schedule ----
 // Slot k of CTA b over G CTAs (snake order: even slots forward, odd slots backward).
 __device__ __forceinline__ int unit_of(int k, int b, int G) {
@@ -355,15 +414,17 @@ __device__ __forceinline__ void gate_tokens(const Params& p, int h, int64_t t0, 
 // R = a-product from the block start (R_i = R0 * a_0 * ... * a_i).  po is the product over the
 // other 8-token half of the block (before this half for the second half, after it for the first).
 __device__ __forceinline__ void decay_suffix(const float (&a)[8][4], const float (&po)[4], bool second_half,
-                                             float (&E)[8][4], float (&R0)[4]) {
+                                             float2 (&E)[8][2], float2 (&R0)[2]) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        E[7][e] = second_half ? 1.f : po[e];
+    for (int e = 0; e < 2; ++e) {
+        E[7][e] = second_half ? make_float2(1.f, 1.f) : make_float2(po[2 * e], po[2 * e + 1]);
 #pragma unroll
-        for (int i = 6; i >= 0; --i) E[i][e] = E[i + 1][e] * a[i + 1][e];
-        R0[e] = second_half ? po[e] : 1.f;
+        for (int i = 6; i >= 0; --i) E[i][e] = __fmul2_rn(E[i + 1][e], make_float2(a[i + 1][2 * e], a[i + 1][2 * e + 1]));
+        R0[e] = second_half ? make_float2(po[2 * e], po[2 * e + 1]) : make_float2(1.f, 1.f);
     }
 }
+__device__ __forceinline__ uint32_t pack_bf16v(float2 v) { return pack_bf16(v.x, v.y); }
+__device__ __forceinline__ uint32_t pack_f16v(float2 v) { return pack_f16s(v.x, v.y); }
 
 // ---- chain warps: rare range repairs (out of line: they cost no instruction-cache space on
 // the common path).  lane_base = TMEM address of the warp's lane quarter.
@@ -482,10 +543,11 @@ __device__ __noinline__ int chain_vals_reconvert(uint32_t lane_base, uint32_t co
 }
 
 // ---- scalar-gate variant: gate and loads ----
-// One warp: lane l handles tokens 2l and 2l + 1 (gv = their raw gate inputs).  S_GAM gets the
-// inclusive in-chunk sum Gamma of log2 a (flat past the valid length), S_GE 2^Gamma and S_KF
-// 2^(Gamma_63 - Gamma).
-__device__ __forceinline__ void gate_scan_scalar(unsigned char* sm, const Params& p, int h, int L, float2 gv) {
+// One warp: lane l handles tokens 2l and 2l + 1 (gv = their raw gate inputs).  s_gam(sl) gets the
+// inclusive in-chunk sum Gamma of log2 a (flat past the valid length), s_ge(sl) 2^Gamma and
+// s_kf(sl) 2^(Gamma_63 - Gamma).
+__device__ __forceinline__ void gate_scan_scalar(unsigned char* sm, const Params& p, int h, int L, float2 gv,
+                                                 uint32_t sl) {
     const int lane = threadIdx.x & 31;
     const float nexpA = -expf(p.A_log[h]);
     const float lb2 = p.lower_bound * kLog2e;
@@ -508,9 +570,9 @@ __device__ __forceinline__ void gate_scan_scalar(unsigned char* sm, const Params
     }
     const float g0 = incl - pair + l.x, g1 = incl;
     const float glast = __shfl_sync(0xffffffffu, incl, 31);
-    *reinterpret_cast<float2*>(reinterpret_cast<float*>(sm + S_GAM) + r0) = make_float2(g0, g1);
-    *reinterpret_cast<float2*>(reinterpret_cast<float*>(sm + S_GE) + r0) = make_float2(fast_ex2(g0), fast_ex2(g1));
-    *reinterpret_cast<float2*>(reinterpret_cast<float*>(sm + S_KF) + r0) =
+    *reinterpret_cast<float2*>(reinterpret_cast<float*>(sm + s_gam(sl)) + r0) = make_float2(g0, g1);
+    *reinterpret_cast<float2*>(reinterpret_cast<float*>(sm + s_ge(sl)) + r0) = make_float2(fast_ex2(g0), fast_ex2(g1));
+    *reinterpret_cast<float2*>(reinterpret_cast<float*>(sm + s_kf(sl)) + r0) =
         make_float2(fast_ex2(glast - g0), fast_ex2(glast - g1));
 }
 
@@ -550,19 +612,18 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t* bar_u = bar_in + 5;        // U MMA done
     uint64_t* bar_s = bar_in + 6;        // [S | O] MMA done (chunk's shared operands free again)
     uint64_t* bar_apready = bar_in + 7;  // chunk's A/P operand tiles written (the chain issues the MMA)
+    uint64_t* bar_ro = bar_in + 8;       // chunk's A/P product read out of TMEM (the accumulator is free)
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + S_TMEM);
     volatile uint32_t* sAbort = sTmem + 1;
-    volatile uint32_t* sEnd = sTmem + 2;   // set once the front end has no further chunk
 #ifdef KDA_PHASE_CLOCKS
     volatile unsigned long long* sPh = reinterpret_cast<volatile unsigned long long*>(sm + S_PH);
 #endif
 
     // ---- set-up ----
     if (tid == 0) {
-        for (int i = 0; i < 8; ++i) mbar_init(bar_in + i, 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(bar_in + i, 1);
         mbar_init_fence();
         *sAbort = 0u;
-        *sEnd = 0u;
     }
     if (warp == 0) {
         tmem_alloc(sTmem, TM_COLS);
@@ -587,7 +648,7 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int e = tid; e < 8192 / 16; e += kThreads) st_v4(sm, T16 + (uint32_t)e * 16u, 0u, 0u, 0u, 0u);
 #ifdef KDA_PHASE_CLOCKS
     if (tid == 0)
-        for (int i = 0; i < kPhases + 2; ++i) sPh[i] = (i < kPhases) ? 0ull : (unsigned long long)clock64();
+        for (int i = 0; i < kPhases + 3; ++i) sPh[i] = (i < kPhases) ? 0ull : (unsigned long long)clock64();
 #endif
     __syncthreads();
     // empty units: final state = initial state (the chain never sees them)
@@ -678,38 +739,72 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             return hmax_to_float(m);
         };
 
+        // The front end's A/P MMA of chunk cc (thread 0): its operand tiles are written and the
+        // previous chunk's product has been read out of TMEM.  It does not depend on the state, so it
+        // goes before the previous chunk's output when both barriers are already complete, and after
+        // it otherwise.  block = false only tests the barriers; ap_open stays set until the step is
+        // settled (the MMA issued, the end of the work seen, or a wait run out).
+        bool ap_open = false;   // thread 0: chunk cc's A/P step not settled yet
+        bool ap_seen = false;   // thread 0: chunk cc's A/P operand tiles seen ready
+        auto issue_ap = [&](bool block) {
+            if (!ap_seen) {
+                if (block) {
+                    if (!mbar_wait_bounded(bar_apready, cc & 1u)) {
+                        record_error(KDA_DEVERR_TIMEOUT);
+                        *sAbort = 1u;
+                        ap_open = false;
+                        return;
+                    }
+                } else if (!mbar_test_wait(bar_apready, cc & 1u)) {
+                    return;
+                }
+                ap_seen = true;
+            }
+            {
+                if (cc > 0) {
+                    if (block) {
+                        if (!mbar_wait_bounded(bar_ro, (cc - 1) & 1u)) {
+                            record_error(KDA_DEVERR_TIMEOUT);
+                            *sAbort = 1u;
+                            ap_open = false;
+                            return;
+                        }
+                    } else if (!mbar_test_wait(bar_ro, (cc - 1) & 1u)) {
+                        return;
+                    }
+                }
+                fence_after_sync();
+                if constexpr (kScalar) {
+                    // [K ; Q] K^T straight from the swizzled input blocks (the decay is applied at
+                    // read-out)
+                    const uint32_t a0 = smem_u32(sm + IN_Q);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(a0, 128, ks), IDESC_AP_S,
+                                ks > 0 ? 1u : 0u);
+                } else {
+                    const uint32_t a0 = smem_u32(sm + AP_A), b0 = smem_u32(sm + AP_B);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
+                                ks > 0 ? 1u : 0u);
+                }
+                mma_commit(bar_ap);
+                ++issued_ap;
+            }
+            ap_open = false;
+        };
+
+        // whether another chunk follows (the front end marks a CTA's last chunk in its metadata)
+        bool more = unit_from(p, sOrder, b, G, units, 0).valid;
         while (true) {
             bool bad = false;
-            // the front end's A/P MMA, issued as soon as its operand tiles are written (it does not
-            // depend on the state, so it goes before the previous chunk's retirement); issuing
-            // costs the issuing warp about 70 cycles per MMA
-            if (tid == 0) {
-                const bool ap_ok = mbar_wait_bounded(bar_apready, cc & 1u);
-                PIPE_MARK(0, 1, 11);
-                if (!ap_ok) {
-                    record_error(KDA_DEVERR_TIMEOUT);
-                    *sAbort = 1u;
-                } else if (*sEnd == 0u) {
-                    fence_after_sync();
-                    if constexpr (kScalar) {
-                        // [K ; Q] K^T straight from the swizzled input blocks (the decay is applied
-                        // at read-out)
-                        const uint32_t a0 = smem_u32(sm + IN_Q);
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks)
-                            mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(a0, 128, ks), IDESC_AP_S,
-                                    ks > 0 ? 1u : 0u);
-                    } else {
-                        const uint32_t a0 = smem_u32(sm + AP_A), b0 = smem_u32(sm + AP_B);
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks)
-                            mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
-                                    ks > 0 ? 1u : 0u);
-                    }
-                    mma_commit(bar_ap);
-                    ++issued_ap;
-                }
+            if (tid == 0 && more) {
+                ap_open = true;
+                ap_seen = false;
+                issue_ap(false);
             }
+            // the previous chunk's output (and final state), once its [S | O] MMA is done
             if (have_prev) {
                 bad |= !warp_wait(bar_s, (cc - 1) & 1u);
                 if (tid == 0 && !bad) done_s = issued_s;
@@ -718,16 +813,19 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (!bad) retire_prev();
             }
             PIPE_MARK(0, 1, 10);
+            if (!more) break;
+            if (tid == 0 && ap_open) issue_ap(true);
+            PIPE_MARK(0, 1, 11);
             PIPE_MARK(0, 1, 12);
             bad |= !warp_wait(bar_formed, cc & 1u);
             const int32_t* meta = sMeta + (cc & 1u) * 8u;
-            const int m_valid = meta[0], m_h = meta[1], m_n = meta[2], m_t0 = meta[3], m_L = meta[4],
-                      m_first = meta[5], m_last = meta[6];
+            const int m_h = meta[1], m_n = meta[2], m_t0 = meta[3], m_L = meta[4], m_first = meta[5],
+                      m_last = meta[6];
+            more = meta[7] != 0;
             if (named_bar_or(BAR_CHAIN, 128, bad || *sAbort != 0u)) {
                 aborted = true;
                 break;
             }
-            if (!m_valid) break;
             PIPE_MARK(0, 1, 13);
             if (m_first) {
                 // the unit's initial state (or zeros) into TMEM
@@ -932,6 +1030,10 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (aborted && tid == 0) *sAbort = 1u;
     } else {
         // =============================== front end ===============================
+        // Element warps 8-15 build chunk n (gate, decay factors, the A/P operand tiles, the chain's
+        // operand tiles) while aux warps 4-7 read out the A/P product of chunk n - 1 and solve
+        // T = (I + A)^-1 for it, then form chunk n's V^T and P diagonal.  The two groups meet once per
+        // chunk (BAR_FE), after both have written chunk n's chain operands.
         const bool is_aux = warp < kElemWarp0;
         const int at = tid - 128;           // aux thread (warps 4-7)
         const int et = tid - 256;           // element thread (warps 8-15)
@@ -940,586 +1042,599 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int c0 = 64 * ehf + 4 * (lane & 15);
         const int r0 = 16 * eI + 8 * (lane >> 4);
         const int quarter = warp & 3;       // TMEM lane quarter of this warp
-        const bool issuer = tid == 128;      // barrier arrivals of the front end
-        const bool loader = tid == 256;      // TMA loads of the next chunk (element warp 8)
+        const bool loader = tid == 128;     // TMA loads (aux warp 4: it has idle time, the element warps have none)
+        const bool elead = tid == 256;      // the element warps' barrier arrivals
         bool tma_pending = false;
         uint32_t tma_parity = 0;
         bool aborted = false;
         uint32_t range_bad = 0u;
+        auto chunk_len = [](const Cursor& c) { return (int)(c.eos - c.t0 < kChunk ? c.eos - c.t0 : kChunk); };
+
+        // chunk c's q, k, v into the input tiles
+        auto load_inputs = [&](const Cursor& c) {
+            if constexpr (kScalar)
+                issue_chunk_loads_s(sm, bar_in, &tm_q, &tm_k, &tm_v, c.h, c.t0);
+            else
+                issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, c.h, c.t0);
+        };
 
         Cursor cur = unit_from(p, sOrder, b, G, units, 0);
-        float a[8][4];
-        float beta_reg = 0.f;   // aux threads 0-63: beta of their token of the next chunk to form
-        float2 g_reg = make_float2(0.f, 0.f);   // scalar gate, warp 8: g of tokens 2 lane, 2 lane + 1
-        // the scalar gate's inputs of chunk c (rows past L read as 0)
-        auto load_g_scalar = [&](const Cursor& c) {
-            const int Lc = (int)(c.eos - c.t0 < kChunk ? c.eos - c.t0 : kChunk);
-            g_reg.x = 2 * lane < Lc ? p.g[(c.t0 + 2 * lane) * H + c.h] : 0.f;
-            g_reg.y = 2 * lane + 1 < Lc ? p.g[(c.t0 + 2 * lane + 1) * H + c.h] : 0.f;
-        };
-        if (cur.valid) {
-            if (issuer) {
-                if constexpr (kScalar)
-                    issue_chunk_loads_s(sm, bar_in, &tm_q, &tm_k, &tm_v, cur.h, cur.t0);
-                else
-                    issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, cur.h, cur.t0);
-            }
-            tma_pending = true;
-            const int L = (int)(cur.eos - cur.t0 < kChunk ? cur.eos - cur.t0 : kChunk);
-            if (is_aux) {
-                if (at < kChunk) beta_reg = p.beta[(cur.t0 + (at < L ? at : L - 1)) * H + cur.h];
-            } else if constexpr (kScalar) {
-                if (warp == kElemWarp0) load_g_scalar(cur);
-            } else {
-                gate_tokens(p, cur.h, cur.t0, L, c0, r0, a);
-            }
-        }
         uint32_t ci = 0;
-        while (cur.valid) {
-            const Cursor nxt = next_chunk(p, sOrder, b, G, units, cur);
-            const int h = cur.h;
-            const int64_t t0 = cur.t0;
-            const int L = (int)(cur.eos - t0 < kChunk ? cur.eos - t0 : kChunk);
-            const uint32_t sl = ci & 1u;
-            bool bad = false;
-            PIPE_MARK(128, 0, 0);
-            // the next chunk's gate input into L2 (its q, k, v come by TMA once this chunk's are used)
-            if (nxt.valid) {
-                const int L1 = (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk);
+        if (loader && cur.valid) {
+            load_inputs(cur);
+            tma_pending = true;
+            tma_parity = 0;
+        }
+        if (!is_aux) {
+            // ======================= element warps =======================
+            float a[8][4];
+            float beta_reg = 0.f;   // element threads 0-63: beta of their token of the next chunk
+            float2 g_reg = make_float2(0.f, 0.f);   // scalar gate, warp 8: g of tokens 2 lane, 2 lane + 1
+            // the scalar gate's inputs of chunk c (rows past its length read as 0)
+            auto load_g_scalar = [&](const Cursor& c) {
+                const int Lc = chunk_len(c);
+                g_reg.x = 2 * lane < Lc ? p.g[(c.t0 + 2 * lane) * H + c.h] : 0.f;
+                g_reg.y = 2 * lane + 1 < Lc ? p.g[(c.t0 + 2 * lane + 1) * H + c.h] : 0.f;
+            };
+            // beta of chunk c: unconditional, row clamped, so that nothing consumes the load before
+            // the next chunk's first phase (where rows past the length are masked)
+            auto load_beta = [&](const Cursor& c) {
+                if (et < kChunk) {
+                    const int Lc = chunk_len(c);
+                    beta_reg = p.beta[(c.t0 + (et < Lc ? et : Lc - 1)) * H + c.h];
+                }
+            };
+            if (cur.valid) {
+                load_beta(cur);
                 if constexpr (kScalar) {
-                    if (warp == kElemWarp0) {
-                        if (2 * lane < L1) prefetch_l2(p.g + (nxt.t0 + 2 * lane) * H + nxt.h);
-                        if (2 * lane + 1 < L1) prefetch_l2(p.g + (nxt.t0 + 2 * lane + 1) * H + nxt.h);
-                    }
-                } else if (!is_aux) {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        if (r0 + i < L1) prefetch_l2(p.g + ((nxt.t0 + r0 + i) * H + nxt.h) * kHeadDim + c0);
+                    if (warp == kElemWarp0) load_g_scalar(cur);
+                } else {
+                    gate_tokens(p, cur.h, cur.t0, chunk_len(cur), c0, r0, a);
                 }
             }
-            // ================ F0: block products of a (element) / beta (aux) ================
-            // Each element thread keeps its 32 values a_t across the phases and rebuilds the
-            // factors R (running product from the block start) and E (product to the block end)
-            // where it needs them; po = product over the other 8-token half of its block.
-            float po[4];
-            if constexpr (kScalar) {
-                // the inputs must have landed: rows past the valid length are zeroed in the tiles,
-                // which are MMA operands themselves
-                bad |= !warp_wait(bar_in, ci & 1u);
-                if (!is_aux) {
+            while (cur.valid) {
+                const Cursor nxt = next_chunk(p, sOrder, b, G, units, cur);
+                const int h = cur.h;
+                const int L = chunk_len(cur);
+                const uint32_t sl = ci & 1u;
+                bool bad = false;
+                // the next chunk's gate input into L2
+                if (nxt.valid) {
+                    const int L1 = chunk_len(nxt);
+                    if constexpr (kScalar) {
+                        if (warp == kElemWarp0) {
+                            if (2 * lane < L1) prefetch_l2(p.g + (nxt.t0 + 2 * lane) * H + nxt.h);
+                            if (2 * lane + 1 < L1) prefetch_l2(p.g + (nxt.t0 + 2 * lane + 1) * H + nxt.h);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            if (r0 + i < L1) prefetch_l2(p.g + ((nxt.t0 + r0 + i) * H + nxt.h) * kHeadDim + c0);
+                    }
+                }
+                // ================ E0: beta; block products of a / the scalar gate's scan ================
+                if (et < kChunk) reinterpret_cast<float*>(sm + S_BETA)[sl * 64u + et] = et < L ? beta_reg : 0.f;
+                float po[4];   // channel gate: product of a over the other 8-token half of the block
+                if constexpr (kScalar) {
+                    // the inputs must have landed: rows past the valid length are zeroed in the tiles,
+                    // which are MMA operands themselves
+                    bad |= !warp_wait(bar_in, ci & 1u);
                     for (int e = L * 8 + et; e < kChunk * 8; e += 256) {
 #pragma unroll
                         for (int b6 = 0; b6 < 6; ++b6)
                             st_v4(sm, IN_Q + (uint32_t)b6 * 8192u + (uint32_t)e * 16u, 0u, 0u, 0u, 0u);
                     }
-                    if (warp == kElemWarp0) gate_scan_scalar(sm, p, h, L, g_reg);
-                } else if (at < kChunk) {
-                    reinterpret_cast<float*>(sm + S_BETA)[sl * 64u + at] = at < L ? beta_reg : 0.f;
-                }
-                fence_proxy_async();
-            } else if (!is_aux) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float own = a[0][e];
-#pragma unroll
-                    for (int i = 1; i < 8; ++i) own *= a[i][e];
-                    po[e] = __shfl_xor_sync(0xffffffffu, own, 16);
-                    if ((lane >> 4) == 0) own *= po[e];          // block product (both halves agree)
-                    if ((lane >> 4) == 0)
-                        reinterpret_cast<float*>(sm + S_PTOT)[eI * kHeadDim + c0 + e] = own;
-                }
-            } else if (at < kChunk) {
-                reinterpret_cast<float*>(sm + S_BETA)[sl * 64u + at] = at < L ? beta_reg : 0.f;
-            }
-            named_bar_sync(BAR_FE, kFeThreads);
-            PIPE_MARK(128, 0, 1);
-            // ================ F2: A/P operand tiles (element) / P diagonal (aux) ================
-            if constexpr (!kScalar) bad |= !warp_wait(bar_in, ci & 1u);
-            if constexpr (kScalar) {
-                // the A/P MMA reads the input tiles directly; P's diagonal needs no correction
-            } else if (!is_aux) {
-                const float* ptot = reinterpret_cast<const float*>(sm + S_PTOT);
-                float4 pt[4];
-#pragma unroll
-                for (int J = 0; J < 4; ++J) pt[J] = *reinterpret_cast<const float4*>(ptot + J * kHeadDim + c0);
-                auto pick = [&](int J) { return J == 0 ? pt[0] : (J == 1 ? pt[1] : (J == 2 ? pt[2] : pt[3])); };
-                const float4 pbI = pick(eI);
-                const float invB[4] = {fast_rcp(pbI.x), fast_rcp(pbI.y), fast_rcp(pbI.z), fast_rcp(pbI.w)};
-                const float4 p1 = pick(eI < 3 ? eI + 1 : 3), p2 = pick(eI < 2 ? eI + 2 : 3);
-                const float F2[4] = {p1.x, p1.y, p1.z, p1.w};
-                const float F3[4] = {p1.x * p2.x, p1.y * p2.y, p1.z * p2.z, p1.w * p2.w};
-                uint32_t mq = 0u, mk = 0u;
-                float E[8][4], Rr[4];
-                decay_suffix(a, po, (lane >> 4) != 0, E, Rr);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int r = r0 + i;
-                    float R[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) R[e] = Rr[e] = Rr[e] * a[i][e];
-                    uint2 kk = *reinterpret_cast<const uint2*>(sm + IN_K + (uint32_t)r * 256u + (uint32_t)c0 * 2u);
-                    uint2 qq = *reinterpret_cast<const uint2*>(sm + IN_Q + (uint32_t)r * 256u + (uint32_t)c0 * 2u);
-                    if (r >= L) kk = qq = make_uint2(0u, 0u);
-                    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mk) : "r"(kk.x));
-                    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mk) : "r"(kk.y));
-                    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mq) : "r"(qq.x));
-                    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mq) : "r"(qq.y));
-                    const float2 k01 = bf16x2_to_float2(kk.x), k23 = bf16x2_to_float2(kk.y);
-                    const float2 q01 = bf16x2_to_float2(qq.x), q23 = bf16x2_to_float2(qq.y);
-                    const float kv[4] = {k01.x, k01.y, k23.x, k23.y}, qv[4] = {q01.x, q01.y, q23.x, q23.y};
-                    float kE[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) kE[e] = kv[e] * E[i][e];
-                    st_tile2(sm, AP_A + quad_off(128u, (uint32_t)r0, i, (uint32_t)c0), pack_bf16(kv[0] * R[0], kv[1] * R[1]),
-                          pack_bf16(kv[2] * R[2], kv[3] * R[3]));
-                    st_tile2(sm, AP_A + quad_off(128u, 64u + (uint32_t)r0, i, (uint32_t)c0), pack_bf16(qv[0] * R[0], qv[1] * R[1]),
-                          pack_bf16(qv[2] * R[2], qv[3] * R[3]));
-                    st_tile2(sm, AP_B + quad_off(160u, (uint32_t)r0, i, (uint32_t)c0), pack_bf16(kE[0] * invB[0], kE[1] * invB[1]),
-                          pack_bf16(kE[2] * invB[2], kE[3] * invB[3]));
-                    if (eI <= 2)
-                        st_tile2(sm, AP_B + quad_off(160u, 64u + (uint32_t)r0, i, (uint32_t)c0), pack_bf16(kE[0], kE[1]), pack_bf16(kE[2], kE[3]));
-                    if (eI <= 1)
-                        st_tile2(sm, AP_B + quad_off(160u, 112u + (uint32_t)r0, i, (uint32_t)c0), pack_bf16(kE[0] * F2[0], kE[1] * F2[1]),
-                              pack_bf16(kE[2] * F2[2], kE[3] * F2[3]));
-                    if (eI == 0)
-                        st_tile2(sm, AP_B + quad_off(160u, 144u + (uint32_t)r0, i, (uint32_t)c0), pack_bf16(kE[0] * F3[0], kE[1] * F3[1]),
-                              pack_bf16(kE[2] * F3[2], kE[3] * F3[3]));
-                }
-                // |q|, |k| bound every fp16 operand built from them (the decay factors are <= 1)
-                const float2 mkf = bf16x2_to_float2(mk), mqf = bf16x2_to_float2(mq);
-                if (fmaxf(fmaxf(fabsf(mkf.x), fabsf(mkf.y)), fmaxf(fabsf(mqf.x), fabsf(mqf.y))) >= kRangeHi)
-                    range_bad = 1u;
-            } else {
-                // q_r . k_r in fp32 over one 64-channel half; 16-byte chunks visited in a
-                // row-dependent order (conflict-free)
-                const int r = at & 63, hh = at >> 6;
-                float pd = 0.f;
-                if (r < L) {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint32_t off = (uint32_t)r * 256u + (uint32_t)hh * 128u + (((uint32_t)(j + r) & 7u) << 4);
-                        const uint4 qv = *reinterpret_cast<const uint4*>(sm + IN_Q + off);
-                        const uint4 kv = *reinterpret_cast<const uint4*>(sm + IN_K + off);
-                        const uint32_t qa[4] = {qv.x, qv.y, qv.z, qv.w}, ka[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 a2 = bf16x2_to_float2(qa[e]), b2 = bf16x2_to_float2(ka[e]);
-                            pd = fmaf(a2.x, b2.x, pd);
-                            pd = fmaf(a2.y, b2.y, pd);
-                        }
-                    }
-                }
-                reinterpret_cast<float*>(sm + S_PD)[hh * 64 + r] = pd;
-            }
-            fence_proxy_async();
-            if (named_bar_or(BAR_FE, kFeThreads, bad || *sAbort != 0u)) {
-                aborted = true;
-                break;
-            }
-            tma_pending = false;
-            PIPE_MARK(128, 0, 2);
-            // ================ F3: the A/P operands are ready (the chain issues the MMA) ================
-            if (issuer) mbar_arrive(bar_apready);
-            PIPE_MARK(128, 0, 3);
-            // ================ F4: the chain's operands (once it is done with the last chunk's) ================
-            if (ci > 0) bad |= !warp_wait(bar_s, (ci - 1) & 1u);
-            PIPE_MARK(128, 0, 4);
-            if (kScalar && !is_aux) {
-                // per-token scalings of the swizzled input blocks; inputs and outputs share the
-                // 128-byte-swizzled geometry, so an item is one 16-byte position of a row
-                const float* sb = reinterpret_cast<const float*>(sm + S_BETA) + sl * 64u;
-                const float* ge = reinterpret_cast<const float*>(sm + S_GE);
-                const float* kf = reinterpret_cast<const float*>(sm + S_KF);
-                uint32_t mq = 0u, mk = 0u;
-                float mbk = 0.f;
-#pragma unroll 1
-                for (int e = et; e < kChunk * 16; e += 256) {
-                    const int r = e >> 4;
-                    const uint32_t cb = (uint32_t)(e >> 3) & 1u, pos = (uint32_t)e & 7u;
-                    const uint32_t off = cb * 16384u + (uint32_t)r * 128u + pos * 16u;
-                    const uint4 kw = *reinterpret_cast<const uint4*>(sm + IN_Q + off);
-                    const uint4 qw = *reinterpret_cast<const uint4*>(sm + IN_Q + off + 8192u);
-                    const float g = ge[r], nbg = -sb[r] * g, kfr = kf[r];
-                    const float2 g2 = make_float2(g, g), nbg2 = make_float2(nbg, nbg), kf2 = make_float2(kfr, kfr);
-                    const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, qq[4] = {qw.x, qw.y, qw.z, qw.w};
-                    uint32_t oq[4], ok[4], oh[4];
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mk) : "r"(kk[x]));
-                        asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mq) : "r"(qq[x]));
-                        const float2 kx = bf16x2_to_float2(kk[x]), qx = bf16x2_to_float2(qq[x]);
-                        const float2 gq = __fmul2_rn(g2, qx), bk = __fmul2_rn(nbg2, kx), kh = __fmul2_rn(kf2, kx);
-                        oq[x] = pack_f16s(gq.x, gq.y);
-                        ok[x] = pack_f16s(bk.x, bk.y);
-                        oh[x] = pack_f16s(kh.x, kh.y);
-                        mbk = fmaxf(mbk, fmaxf(fabsf(bk.x), fabsf(bk.y)));
-                    }
-                    st_tile4(sm, B1 + off, oq[0], oq[1], oq[2], oq[3]);
-                    st_tile4(sm, B1 + off + 8192u, ok[0], ok[1], ok[2], ok[3]);
-                    st_tile4(sm, KH + cb * 8192u + (uint32_t)r * 128u + pos * 16u, oh[0], oh[1], oh[2], oh[3]);
-                }
-                const float2 mkf = bf16x2_to_float2(mk), mqf = bf16x2_to_float2(mq);
-                if (fmaxf(fmaxf(fabsf(mkf.x), fabsf(mkf.y)), fmaxf(fabsf(mqf.x), fabsf(mqf.y))) >= kRangeHi ||
-                    mbk >= kRangeHi)
-                    range_bad = 1u;
-                if (et < kHeadDim)
-                    reinterpret_cast<float*>(sm + S_GC)[sl * kHeadDim + et] = ge[kChunk - 1];
-            } else if (!is_aux) {
-                const float* ptot = reinterpret_cast<const float*>(sm + S_PTOT);
-                float before[4] = {1.f, 1.f, 1.f, 1.f}, after[4] = {1.f, 1.f, 1.f, 1.f};
-#pragma unroll
-                for (int J = 0; J < 4; ++J) {
-                    const float4 x = *reinterpret_cast<const float4*>(ptot + J * kHeadDim + c0);
-                    const float xv[4] = {x.x, x.y, x.z, x.w};
+                    if (warp == kElemWarp0) gate_scan_scalar(sm, p, h, L, g_reg, sl);
+                    fence_proxy_async();
+                } else {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        if (J < eI) before[e] *= xv[e];
-                        if (J > eI) after[e] *= xv[e];
+                        float own = a[0][e];
+#pragma unroll
+                        for (int i = 1; i < 8; ++i) own *= a[i][e];
+                        po[e] = __shfl_xor_sync(0xffffffffu, own, 16);
+                        if ((lane >> 4) == 0) own *= po[e];          // block product (both halves agree)
+                        if ((lane >> 4) == 0)
+                            reinterpret_cast<float*>(sm + S_PTOT)[eI * kHeadDim + c0 + e] = own;
                     }
                 }
-                const float* sb = reinterpret_cast<const float*>(sm + S_BETA) + sl * 64u;
-                float E[8][4], Rr[4];
-                decay_suffix(a, po, (lane >> 4) != 0, E, Rr);
+                named_bar_sync(BAR_ELEM, 256);
+                PIPE_MARK(256, 2, 18);
+                // ================ E2: the A/P operand tiles (channel gate) ================
+                if constexpr (!kScalar) {
+                    bad |= !warp_wait(bar_in, ci & 1u);
+                    // the previous chunk's A/P MMA has read the tiles this phase rewrites
+                    if (ci > 0) bad |= !warp_wait(bar_ap, (ci - 1) & 1u);
+                    PIPE_MARK(256, 2, 19);
+                    const float* ptot = reinterpret_cast<const float*>(sm + S_PTOT);
+                    float4 pt[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int r = r0 + i;
-                    const float nb = -sb[r];
+                    for (int J = 0; J < 4; ++J) pt[J] = *reinterpret_cast<const float4*>(ptot + J * kHeadDim + c0);
+                    auto pick = [&](int J) { return J == 0 ? pt[0] : (J == 1 ? pt[1] : (J == 2 ? pt[2] : pt[3])); };
+                    const float4 pbI = pick(eI);
+                    const float invB[4] = {fast_rcp(pbI.x), fast_rcp(pbI.y), fast_rcp(pbI.z), fast_rcp(pbI.w)};
+                    const float4 p1 = pick(eI < 3 ? eI + 1 : 3), p2 = pick(eI < 2 ? eI + 2 : 3);
+                    const float2 invB01 = make_float2(invB[0], invB[1]), invB23 = make_float2(invB[2], invB[3]);
+                    const float2 F2a = make_float2(p1.x, p1.y), F2b = make_float2(p1.z, p1.w);
+                    const float2 F3a = __fmul2_rn(F2a, make_float2(p2.x, p2.y)), F3b = __fmul2_rn(F2b, make_float2(p2.z, p2.w));
+                    uint32_t mq = 0u, mk = 0u;
+                    float2 E[8][2], Rr[2];
+                    decay_suffix(a, po, (lane >> 4) != 0, E, Rr);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) Rr[e] *= a[i][e];
-                    // k, q again from the input tiles (still resident: the next chunk's loads are
-                    // issued after this phase); rows past the valid length are zero
-                    uint2 kk = *reinterpret_cast<const uint2*>(sm + IN_K + (uint32_t)r * 256u + (uint32_t)c0 * 2u);
-                    uint2 qq = *reinterpret_cast<const uint2*>(sm + IN_Q + (uint32_t)r * 256u + (uint32_t)c0 * 2u);
-                    if (r >= L) kk = qq = make_uint2(0u, 0u);
-                    const float2 k01 = bf16x2_to_float2(kk.x), k23 = bf16x2_to_float2(kk.y);
-                    const float2 q01 = bf16x2_to_float2(qq.x), q23 = bf16x2_to_float2(qq.y);
-                    const float kv[4] = {k01.x, k01.y, k23.x, k23.y}, qv[4] = {q01.x, q01.y, q23.x, q23.y};
-                    float gm[4], kh[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        gm[e] = Rr[e] * before[e];
-                        kh[e] = kv[e] * E[i][e] * after[e];
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = r0 + i;
+                        Rr[0] = __fmul2_rn(Rr[0], make_float2(a[i][0], a[i][1]));
+                        Rr[1] = __fmul2_rn(Rr[1], make_float2(a[i][2], a[i][3]));
+                        uint2 kk = *reinterpret_cast<const uint2*>(sm + IN_K + (uint32_t)r * 256u + (uint32_t)c0 * 2u);
+                        uint2 qq = *reinterpret_cast<const uint2*>(sm + IN_Q + (uint32_t)r * 256u + (uint32_t)c0 * 2u);
+                        if (r >= L) kk = qq = make_uint2(0u, 0u);
+                        asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mk) : "r"(kk.x));
+                        asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mk) : "r"(kk.y));
+                        asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mq) : "r"(qq.x));
+                        asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mq) : "r"(qq.y));
+                        const float2 k01 = bf16x2_to_float2(kk.x), k23 = bf16x2_to_float2(kk.y);
+                        const float2 q01 = bf16x2_to_float2(qq.x), q23 = bf16x2_to_float2(qq.y);
+                        const float2 kE01 = __fmul2_rn(k01, E[i][0]), kE23 = __fmul2_rn(k23, E[i][1]);
+                        st_tile2(sm, AP_A + quad_off(128u, (uint32_t)r0, i, (uint32_t)c0),
+                                 pack_bf16v(__fmul2_rn(k01, Rr[0])), pack_bf16v(__fmul2_rn(k23, Rr[1])));
+                        st_tile2(sm, AP_A + quad_off(128u, 64u + (uint32_t)r0, i, (uint32_t)c0),
+                                 pack_bf16v(__fmul2_rn(q01, Rr[0])), pack_bf16v(__fmul2_rn(q23, Rr[1])));
+                        st_tile2(sm, AP_B + quad_off(160u, (uint32_t)r0, i, (uint32_t)c0),
+                                 pack_bf16v(__fmul2_rn(kE01, invB01)), pack_bf16v(__fmul2_rn(kE23, invB23)));
+                        if (eI <= 2)
+                            st_tile2(sm, AP_B + quad_off(160u, 64u + (uint32_t)r0, i, (uint32_t)c0), pack_bf16v(kE01),
+                                     pack_bf16v(kE23));
+                        if (eI <= 1)
+                            st_tile2(sm, AP_B + quad_off(160u, 112u + (uint32_t)r0, i, (uint32_t)c0),
+                                     pack_bf16v(__fmul2_rn(kE01, F2a)), pack_bf16v(__fmul2_rn(kE23, F2b)));
+                        if (eI == 0)
+                            st_tile2(sm, AP_B + quad_off(160u, 144u + (uint32_t)r0, i, (uint32_t)c0),
+                                     pack_bf16v(__fmul2_rn(kE01, F3a)), pack_bf16v(__fmul2_rn(kE23, F3b)));
                     }
-                    st_tile2(sm, B1 + quad_off(128u, (uint32_t)r0, i, (uint32_t)c0), pack_f16s(qv[0] * gm[0], qv[1] * gm[1]),
-                          pack_f16s(qv[2] * gm[2], qv[3] * gm[3]));
-                    st_tile2(sm, B1 + quad_off(128u, 64u + (uint32_t)r0, i, (uint32_t)c0), pack_f16s(nb * kv[0] * gm[0], nb * kv[1] * gm[1]),
-                          pack_f16s(nb * kv[2] * gm[2], nb * kv[3] * gm[3]));
-                    st_tile2(sm, KH + quad_off(64u, (uint32_t)r0, i, (uint32_t)c0), pack_f16s(kh[0], kh[1]), pack_f16s(kh[2], kh[3]));
-                    if (fabsf(nb) > 1.f && fabsf(nb) * fmaxf(fmaxf(fabsf(kv[0]), fabsf(kv[1])),
-                                                             fmaxf(fabsf(kv[2]), fabsf(kv[3]))) >= kRangeHi)
+                    // |q|, |k| bound every fp16 operand built from them (the decay factors are <= 1)
+                    const float2 mkf = bf16x2_to_float2(mk), mqf = bf16x2_to_float2(mq);
+                    if (fmaxf(fmaxf(fabsf(mkf.x), fabsf(mkf.y)), fmaxf(fabsf(mqf.x), fabsf(mqf.y))) >= kRangeHi)
                         range_bad = 1u;
+                    fence_proxy_async();
+                    named_bar_sync(BAR_ELEM, 256);
                 }
-                if (eI == 0 && (lane >> 4) == 0) {
-                    float gc[4] = {1.f, 1.f, 1.f, 1.f};
+                PIPE_MARK(256, 2, 20);
+                // the A/P operands are ready: the chain issues the MMA
+                if (elead) mbar_arrive(bar_apready);
+                // ================ E4: the chain's operands (once it is done with the last chunk's) ================
+                if (ci > 0) bad |= !warp_wait(bar_s, (ci - 1) & 1u);
+                PIPE_MARK(256, 2, 21);
+                if constexpr (kScalar) {
+                    // per-token scalings of the swizzled input blocks; inputs and outputs share the
+                    // 128-byte-swizzled geometry, so an item is one 16-byte position of a row
+                    const float* sb = reinterpret_cast<const float*>(sm + S_BETA) + sl * 64u;
+                    const float* ge = reinterpret_cast<const float*>(sm + s_ge(sl));
+                    const float* kf = reinterpret_cast<const float*>(sm + s_kf(sl));
+                    uint32_t mq = 0u, mk = 0u;
+                    float mbk = 0.f;
+#pragma unroll 1
+                    for (int e = et; e < kChunk * 16; e += 256) {
+                        const int r = e >> 4;
+                        const uint32_t cb = (uint32_t)(e >> 3) & 1u, pos = (uint32_t)e & 7u;
+                        const uint32_t off = cb * 16384u + (uint32_t)r * 128u + pos * 16u;
+                        const uint4 kw = *reinterpret_cast<const uint4*>(sm + IN_Q + off);
+                        const uint4 qw = *reinterpret_cast<const uint4*>(sm + IN_Q + off + 8192u);
+                        const float g = ge[r], nbg = -sb[r] * g, kfr = kf[r];
+                        const float2 g2 = make_float2(g, g), nbg2 = make_float2(nbg, nbg), kf2 = make_float2(kfr, kfr);
+                        const uint32_t kk[4] = {kw.x, kw.y, kw.z, kw.w}, qq[4] = {qw.x, qw.y, qw.z, qw.w};
+                        uint32_t oq[4], ok[4], oh[4];
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mk) : "r"(kk[x]));
+                            asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(mq) : "r"(qq[x]));
+                            const float2 kx = bf16x2_to_float2(kk[x]), qx = bf16x2_to_float2(qq[x]);
+                            const float2 gq = __fmul2_rn(g2, qx), bk = __fmul2_rn(nbg2, kx), kh = __fmul2_rn(kf2, kx);
+                            oq[x] = pack_f16s(gq.x, gq.y);
+                            ok[x] = pack_f16s(bk.x, bk.y);
+                            oh[x] = pack_f16s(kh.x, kh.y);
+                            mbk = fmaxf(mbk, fmaxf(fabsf(bk.x), fabsf(bk.y)));
+                        }
+                        st_tile4(sm, B1 + off, oq[0], oq[1], oq[2], oq[3]);
+                        st_tile4(sm, B1 + off + 8192u, ok[0], ok[1], ok[2], ok[3]);
+                        st_tile4(sm, KH + cb * 8192u + (uint32_t)r * 128u + pos * 16u, oh[0], oh[1], oh[2], oh[3]);
+                    }
+                    const float2 mkf = bf16x2_to_float2(mk), mqf = bf16x2_to_float2(mq);
+                    if (fmaxf(fmaxf(fabsf(mkf.x), fabsf(mkf.y)), fmaxf(fabsf(mqf.x), fabsf(mqf.y))) >= kRangeHi ||
+                        mbk >= kRangeHi)
+                        range_bad = 1u;
+                    if (et < kHeadDim)
+                        reinterpret_cast<float*>(sm + S_GC)[sl * kHeadDim + et] = ge[kChunk - 1];
+                } else {
+                    const float* ptot = reinterpret_cast<const float*>(sm + S_PTOT);
+                    float2 before[2] = {make_float2(1.f, 1.f), make_float2(1.f, 1.f)};
+                    float2 after[2] = {make_float2(1.f, 1.f), make_float2(1.f, 1.f)};
 #pragma unroll
                     for (int J = 0; J < 4; ++J) {
                         const float4 x = *reinterpret_cast<const float4*>(ptot + J * kHeadDim + c0);
-                        gc[0] *= x.x; gc[1] *= x.y; gc[2] *= x.z; gc[3] *= x.w;
+                        const float2 x01 = make_float2(x.x, x.y), x23 = make_float2(x.z, x.w);
+                        if (J < eI) {
+                            before[0] = __fmul2_rn(before[0], x01);
+                            before[1] = __fmul2_rn(before[1], x23);
+                        }
+                        if (J > eI) {
+                            after[0] = __fmul2_rn(after[0], x01);
+                            after[1] = __fmul2_rn(after[1], x23);
+                        }
                     }
-                    *reinterpret_cast<float4*>(reinterpret_cast<float*>(sm + S_GC) + sl * kHeadDim + c0) =
-                        make_float4(gc[0], gc[1], gc[2], gc[3]);
-                }
-            } else {
-                // V^T: thread -> value columns 2 vp and 2 vp + 1, tokens 32 th .. 32 th + 31
-              {
-                const int vp = at & 63, th = at >> 6;
-                const uint32_t v0 = 2u * (uint32_t)vp, v1 = v0 + 1u;
+                    const float* sb = reinterpret_cast<const float*>(sm + S_BETA) + sl * 64u;
+                    float2 E[8][2], Rr[2];
+                    decay_suffix(a, po, (lane >> 4) != 0, E, Rr);
+                    // E times the products of the later blocks: Khat's factor
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t w[8];
-#pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        const int r = 32 * th + 8 * j + t;
-                        uint32_t voff;
-                        if constexpr (kScalar)   // 64-channel swizzled blocks: element (r, v0) of block v0 / 64
-                            voff = (v0 >> 6) * 8192u + (uint32_t)r * 128u +
-                                   ((((v0 & 63u) >> 3) ^ ((uint32_t)r & 7u)) << 4) + (v0 & 7u) * 2u;
-                        else
-                            voff = (uint32_t)r * 256u + (uint32_t)vp * 4u;
-                        w[t] = r < L ? *reinterpret_cast<const uint32_t*>(sm + IN_V + voff) : 0u;
+                    for (int i = 0; i < 8; ++i) {
+                        E[i][0] = __fmul2_rn(E[i][0], after[0]);
+                        E[i][1] = __fmul2_rn(E[i][1], after[1]);
                     }
-                    const uint32_t ch = (uint32_t)(4 * th + j);
-                    st_tile4(sm, VT + v0 * 128u + ((ch ^ (v0 & 7u)) << 4), __byte_perm(w[0], w[1], 0x5410),
-                          __byte_perm(w[2], w[3], 0x5410), __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
-                    st_tile4(sm, VT + v1 * 128u + ((ch ^ (v1 & 7u)) << 4), __byte_perm(w[0], w[1], 0x7632),
-                          __byte_perm(w[2], w[3], 0x7632), __byte_perm(w[4], w[5], 0x7632), __byte_perm(w[6], w[7], 0x7632));
+                    Rr[0] = __fmul2_rn(Rr[0], before[0]);
+                    Rr[1] = __fmul2_rn(Rr[1], before[1]);
+                    float nbk = 0.f;   // max |beta k| over the thread's rows
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = r0 + i;
+                        const float nb = -sb[r];
+                        const float2 nb2 = make_float2(nb, nb);
+                        // gamma = R times the products of the earlier blocks
+                        Rr[0] = __fmul2_rn(Rr[0], make_float2(a[i][0], a[i][1]));
+                        Rr[1] = __fmul2_rn(Rr[1], make_float2(a[i][2], a[i][3]));
+                        // k, q again from the input tiles (still resident: the next chunk's loads are
+                        // issued after this phase); rows past the valid length are zero
+                        uint2 kk = *reinterpret_cast<const uint2*>(sm + IN_K + (uint32_t)r * 256u + (uint32_t)c0 * 2u);
+                        uint2 qq = *reinterpret_cast<const uint2*>(sm + IN_Q + (uint32_t)r * 256u + (uint32_t)c0 * 2u);
+                        if (r >= L) kk = qq = make_uint2(0u, 0u);
+                        const float2 k01 = bf16x2_to_float2(kk.x), k23 = bf16x2_to_float2(kk.y);
+                        const float2 q01 = bf16x2_to_float2(qq.x), q23 = bf16x2_to_float2(qq.y);
+                        const float2 kg01 = __fmul2_rn(k01, Rr[0]), kg23 = __fmul2_rn(k23, Rr[1]);
+                        st_tile2(sm, B1 + quad_off(128u, (uint32_t)r0, i, (uint32_t)c0),
+                                 pack_f16v(__fmul2_rn(q01, Rr[0])), pack_f16v(__fmul2_rn(q23, Rr[1])));
+                        st_tile2(sm, B1 + quad_off(128u, 64u + (uint32_t)r0, i, (uint32_t)c0),
+                                 pack_f16v(__fmul2_rn(nb2, kg01)), pack_f16v(__fmul2_rn(nb2, kg23)));
+                        st_tile2(sm, KH + quad_off(64u, (uint32_t)r0, i, (uint32_t)c0),
+                                 pack_f16v(__fmul2_rn(k01, E[i][0])), pack_f16v(__fmul2_rn(k23, E[i][1])));
+                        nbk = fmaxf(nbk, fabsf(nb) * fmaxf(fmaxf(fabsf(k01.x), fabsf(k01.y)), fmaxf(fabsf(k23.x), fabsf(k23.y))));
+                    }
+                    // |beta k| bounds the -beta gamma k operand (the decay factors are <= 1)
+                    if (nbk >= kRangeHi) range_bad = 1u;
+                    if (eI == 0 && (lane >> 4) == 0) {
+                        float gc[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+                        for (int J = 0; J < 4; ++J) {
+                            const float4 x = *reinterpret_cast<const float4*>(ptot + J * kHeadDim + c0);
+                            gc[0] *= x.x; gc[1] *= x.y; gc[2] *= x.z; gc[3] *= x.w;
+                        }
+                        *reinterpret_cast<float4*>(reinterpret_cast<float*>(sm + S_GC) + sl * kHeadDim + c0) =
+                            make_float4(gc[0], gc[1], gc[2], gc[3]);
+                    }
                 }
-              }
+                fence_proxy_async();
+                if (named_bar_or(BAR_FE, kFeThreads, bad || *sAbort != 0u)) {
+                    aborted = true;
+                    break;
+                }
+                PIPE_MARK(256, 2, 22);
+                // hand the chunk to the chain
+                if (elead) mbar_arrive(bar_formed);
+                // ================ E6: the next chunk's beta and gate ================
+                if (nxt.valid) {
+                    load_beta(nxt);
+                    if constexpr (kScalar) {
+                        if (warp == kElemWarp0) load_g_scalar(nxt);
+                    } else {
+                        gate_tokens(p, nxt.h, nxt.t0, chunk_len(nxt), c0, r0, a);
+                    }
+                }
+                PIPE_MARK(256, 2, 23);
+                cur = nxt;
+                ++ci;
+            }
+            if (aborted) *sAbort = 1u;
+        } else {
+            // ======================= aux warps =======================
+            // Iteration k: the read-out and solve of chunk k - 1, then chunk k's V^T, P diagonal and
+            // metadata.  One more iteration after the last chunk solves that chunk.
+            const int sw = warp - kAuxWarp0;
+            float tmax = 0.f;
+            Cursor next_in;         // the chunk whose inputs the next TMA loads bring (scalar gate)
+            next_in.valid = false;
+            // sign * (a 16 x 16 warp-MMA accumulator) into block (I, J) of the fp16 T tile
+            auto acc_to_t16 = [&](int I, int J, const float (&acc)[2][4], float sign) {
+                const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+                for (int nh = 0; nh < 2; ++nh) {
+                    const uint32_t col = (uint32_t)(16 * J + 8 * nh + 2 * t);
+                    tmax = fmaxf(tmax, fmaxf(fmaxf(fabsf(acc[nh][0]), fabsf(acc[nh][1])),
+                                             fmaxf(fabsf(acc[nh][2]), fabsf(acc[nh][3]))));
+                    *reinterpret_cast<uint32_t*>(sm + T16 + sw128_off((uint32_t)(16 * I + g), col, 64u)) =
+                        pack_f16s(sign * acc[nh][0], sign * acc[nh][1]);
+                    *reinterpret_cast<uint32_t*>(sm + T16 + sw128_off((uint32_t)(16 * I + g + 8), col, 64u)) =
+                        pack_f16s(sign * acc[nh][2], sign * acc[nh][3]);
+                }
+            };
+            while (true) {
+                bool bad = false;
+                if (ci > 0) {
+                    const uint32_t cj = ci - 1, slp = cj & 1u;
+                    // ================ A0: A / P read-out of chunk cj (one warp per TMEM lane quarter) ================
+                    const bool ap_done = warp_wait(bar_ap, cj & 1u);
+                    if (!ap_done) *sAbort = 1u;
+                    if constexpr (kScalar) {
+                        if (loader && ap_done && next_in.valid) {
+                            load_inputs(next_in);
+                            tma_pending = true;
+                            tma_parity = ci & 1u;
+                        }
+                    }
+                    fence_after_sync();
+                    PIPE_MARK(128, 0, 0);
+                    const bool isA = quarter < 2;
+                    const int r = (quarter & 1) * 32 + lane;      // token row of A (k rows) or P (q rows)
+                    const int I = r >> 4;
+                    const float be = reinterpret_cast<const float*>(sm + S_BETA)[slp * 64u + r];
+                    float pdg = 0.f;
+                    if constexpr (!kScalar)
+                        pdg = reinterpret_cast<const float*>(sm + S_PD)[r] + reinterpret_cast<const float*>(sm + S_PD)[64 + r];
+                    float pmax = 0.f;
+#pragma unroll 1
+                    for (int J = 0; J < 4; ++J) {
+                        float row[16];
+                        auto pick = [&](uint32_t col_a, uint32_t col_b, int I_a) {
+                            uint32_t ta[16], tb[16];
+                            tmem_ld16(taddr(tbase, quarter, TM_AP + col_a), ta);
+                            tmem_ld16(taddr(tbase, quarter, TM_AP + col_b), tb);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int x = 0; x < 16; ++x) row[x] = __uint_as_float(I == I_a ? ta[x] : tb[x]);
+                        };
+                        if constexpr (kScalar) {
+                            // raw K K^T / Q K^T times the scalar decay 2^(Gamma_r - Gamma_i) (<= 1 on
+                            // and below the diagonal)
+                            uint32_t raw[16];
+                            tmem_ld16(taddr(tbase, quarter, TM_AP + (uint32_t)J * 16u), raw);
+                            tmem_wait_ld();
+                            const float* gam = reinterpret_cast<const float*>(sm + s_gam(slp));
+                            const float gr = gam[r];
+#pragma unroll
+                            for (int x = 0; x < 16; ++x) {
+                                const int i = J * 16 + x;
+                                const bool keep = isA ? (i < r) : (i <= r);
+                                row[x] = keep ? __uint_as_float(raw[x]) * fast_ex2(gr - gam[i]) : 0.f;
+                            }
+                        } else {
+                            if ((quarter & 1) == 0) {        // I in {0, 1}
+                                if (J == 0) pick(0, 64, 0);            // I=0: diagonal; I=1: C1 of block 0
+                                else if (J == 1) pick(16, 16, 1);      // I=1: diagonal (I=0: masked)
+                                else {
+#pragma unroll
+                                    for (int x = 0; x < 16; ++x) row[x] = 0.f;
+                                }
+                            } else {                         // I in {2, 3}
+                                if (J == 0) pick(112, 144, 2);         // I=2: C2 of block 0; I=3: C3 of block 0
+                                else if (J == 1) pick(80, 128, 2);     // I=2: C1 of block 1; I=3: C2 of block 1
+                                else if (J == 2) pick(32, 96, 2);      // I=2: diagonal; I=3: C1 of block 2
+                                else pick(48, 48, 3);                  // I=3: diagonal (I=2: masked)
+                            }
+#pragma unroll
+                            for (int x = 0; x < 16; ++x) {
+                                const int i = J * 16 + x;
+                                row[x] = i < r ? row[x] : ((i == r && !isA) ? pdg : 0.f);
+                            }
+                        }
+                        if (isA) {
+                            // beta-scaled A: diagonal blocks in fp32 (the forward substitution), the
+                            // blocks below in fp16 (operands of the block products)
+                            if (J == I) {
+                                float* ad = reinterpret_cast<float*>(sm + SV_AD) + (I * 16 + (r & 15)) * kAdPitch;
+#pragma unroll
+                                for (int x = 0; x < 16; x += 4)
+                                    *reinterpret_cast<float4*>(ad + x) =
+                                        make_float4(be * row[x], be * row[x + 1], be * row[x + 2], be * row[x + 3]);
+                            } else if (J < I) {
+                                uint32_t hv[8];
+#pragma unroll
+                                for (int x = 0; x < 8; ++x) hv[x] = warpmma::pack_half2(be * row[2 * x], be * row[2 * x + 1]);
+                                const uint32_t off = al_off(I, J) + (uint32_t)(r & 15) * kHp * 2u;
+                                st_v4(sm, off, hv[0], hv[1], hv[2], hv[3]);
+                                st_v4(sm, off + 16u, hv[4], hv[5], hv[6], hv[7]);
+                            }
+                        } else {
+                            // P^T (MN-major, K = token i, N = row r): 16-bit stores, a warp writes 64
+                            // contiguous bytes per i
+#pragma unroll
+                            for (int x = 0; x < 16; ++x) {
+                                const int i = J * 16 + x;
+                                pmax = fmaxf(pmax, fabsf(row[x]));
+                                st_tile_h(sm, PT + sw128_off((uint32_t)i, (uint32_t)r, 64u),
+                                          __half_as_ushort(__float2half_rn(fminf(fmaxf(row[x], -65504.f), 65504.f))));
+                            }
+                        }
+                    }
+                    if (pmax >= kRangeHi) range_bad = 1u;
+                    fence_proxy_async();
+                    tmem_wait_ld();
+                    fence_before_sync();
+                    named_bar_sync(BAR_AUX, 128);
+                    // the accumulator is free for the next chunk's A/P MMA
+                    if (at == 0) mbar_arrive(bar_ro);
+                    PIPE_MARK(128, 0, 1);
+                    // ================ A1: T = (I + A)^-1 of chunk cj ================
+                    // L0: the four 16 x 16 diagonal blocks by forward substitution in fp32, one column
+                    // per thread (threads 0-63), right-looking; written to the fp16 T tile
+                    if (sw < 2) {
+                        const int bI = at >> 4, jc = at & 15, o = bI * 16;
+                        const float* ad = reinterpret_cast<const float*>(sm + SV_AD) + bI * 16 * kAdPitch;
+                        float x[16];
+#pragma unroll
+                        for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == jc) ? 1.f : 0.f;
+#pragma unroll
+                        for (int ii = 0; ii < 15; ++ii) {
+                            const float xi = x[ii];
+#pragma unroll
+                            for (int rr = ii + 1; rr < 16; ++rr) x[rr] = fmaf(-ad[rr * kAdPitch + ii], xi, x[rr]);
+                        }
+#pragma unroll
+                        for (int rr = 0; rr < 16; ++rr) {
+                            tmax = fmaxf(tmax, fabsf(x[rr]));
+                            st_tile_h(sm, T16 + sw128_off((uint32_t)(o + rr), (uint32_t)(o + jc), 64u),
+                                      __half_as_ushort(__float2half_rn(fminf(fmaxf(x[rr], -65504.f), 65504.f))));
+                        }
+                    }
+                    named_bar_sync(BAR_AUX, 128);
+                    PIPE_MARK(128, 0, 2);
+                    // L1 (16 x 16 warp-MMA products, fp16 operands, fp32 accumulation):
+                    //   T10 = -T11 (A10 T00), T32 = -T33 (A32 T22),
+                    //   X20 = A20 T00 + A21 T10, X30 = A30 T00 + A31 T10, X21 = A21 T11, X31 = A31 T11.
+                    // Aux warps 0 and 2 both form T10 (warp 2 in its own scratch) so that neither waits
+                    // for the other.
+                    {
+                        float acc[2][4] = {};
+                        if (sw == 0 || sw == 2) {
+                            const uint32_t ysc = sw == 0 ? SC_Y0 : SC_Y2;
+                            mm16h(acc, lm_blk(sm, al_off(1, 0)), lm_t16(sm, 0, 0));       // A10 T00
+                            store16h(sm, ysc, acc, 1.f);
+                            __syncwarp();
+                            float a2[2][4] = {};
+                            mm16h(a2, lm_t16(sm, 1, 1), lm_blk(sm, ysc));                 // T10
+                            if (sw == 0) acc_to_t16(1, 0, a2, -1.f);
+                            else store16h(sm, SC_T10B, a2, -1.f);
+                            __syncwarp();
+                            const int I = sw == 0 ? 2 : 3;
+                            float a3[2][4] = {};
+                            mm16h(a3, lm_blk(sm, al_off(I, 0)), lm_t16(sm, 0, 0));
+                            mm16h(a3, lm_blk(sm, al_off(I, 1)), sw == 0 ? lm_t16(sm, 1, 0) : lm_blk(sm, SC_T10B));
+                            store16h(sm, sw == 0 ? SC_X20 : SC_X30, a3, 1.f);             // X20 / X30
+                        } else if (sw == 1) {
+                            mm16h(acc, lm_blk(sm, al_off(3, 2)), lm_t16(sm, 2, 2));       // A32 T22
+                            store16h(sm, SC_Y32, acc, 1.f);
+                            __syncwarp();
+                            float a2[2][4] = {};
+                            mm16h(a2, lm_t16(sm, 3, 3), lm_blk(sm, SC_Y32));
+                            acc_to_t16(3, 2, a2, -1.f);                                   // T32
+                            float a3[2][4] = {};
+                            mm16h(a3, lm_blk(sm, al_off(2, 1)), lm_t16(sm, 1, 1));
+                            store16h(sm, SC_X21, a3, 1.f);                                // X21
+                        } else {
+                            mm16h(acc, lm_blk(sm, al_off(3, 1)), lm_t16(sm, 1, 1));
+                            store16h(sm, SC_X31, acc, 1.f);                               // X31
+                        }
+                    }
+                    named_bar_sync(BAR_AUX, 128);
+                    // L2: T_LL = -T_LR X, written straight to the fp16 tile:
+                    //   T20 = -T22 X20, T21 = -T22 X21, T30 = -(T32 X20 + T33 X30), T31 = -(T32 X21 + T33 X31)
+                    {
+                        float acc[2][4] = {};
+                        const int J = sw & 1;
+                        if (sw < 2) {
+                            mm16h(acc, lm_t16(sm, 2, 2), lm_blk(sm, J == 0 ? SC_X20 : SC_X21));
+                            acc_to_t16(2, J, acc, -1.f);
+                        } else {
+                            mm16h(acc, lm_t16(sm, 3, 2), lm_blk(sm, J == 0 ? SC_X20 : SC_X21));
+                            mm16h(acc, lm_t16(sm, 3, 3), lm_blk(sm, J == 0 ? SC_X30 : SC_X31));
+                            acc_to_t16(3, J, acc, -1.f);
+                        }
+                    }
+                    if (tmax >= kRangeHi) range_bad = 1u;
+                    fence_proxy_async();
+                    named_bar_sync(BAR_AUX, 128);
+                    if (at == 0) mbar_arrive(bar_t);
+                    PIPE_MARK(128, 0, 3);
+                }
+                if (!cur.valid) break;
+                const Cursor nxt = next_chunk(p, sOrder, b, G, units, cur);
+                const int L = chunk_len(cur);
+                const uint32_t sl = ci & 1u;
+                // ================ A4: V^T, P diagonal and metadata of chunk ci ================
+                if (ci > 0) bad |= !warp_wait(bar_s, (ci - 1) & 1u);   // the chain is done with the last V^T
+                bad |= !warp_wait(bar_in, ci & 1u);
+                tma_pending = false;
+                PIPE_MARK(128, 0, 4);
+                {
+                    // V^T: thread -> value columns 2 vp and 2 vp + 1, tokens 32 th .. 32 th + 31
+                    const int vp = at & 63, th = at >> 6;
+                    const uint32_t v0 = 2u * (uint32_t)vp, v1 = v0 + 1u;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t w[8];
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) {
+                            const int r = 32 * th + 8 * j + t;
+                            uint32_t voff;
+                            if constexpr (kScalar)   // 64-channel swizzled blocks: element (r, v0) of block v0 / 64
+                                voff = (v0 >> 6) * 8192u + (uint32_t)r * 128u +
+                                       ((((v0 & 63u) >> 3) ^ ((uint32_t)r & 7u)) << 4) + (v0 & 7u) * 2u;
+                            else
+                                voff = (uint32_t)r * 256u + (uint32_t)vp * 4u;
+                            w[t] = r < L ? *reinterpret_cast<const uint32_t*>(sm + IN_V + voff) : 0u;
+                        }
+                        const uint32_t ch = (uint32_t)(4 * th + j);
+                        st_tile4(sm, VT + v0 * 128u + ((ch ^ (v0 & 7u)) << 4), __byte_perm(w[0], w[1], 0x5410),
+                              __byte_perm(w[2], w[3], 0x5410), __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
+                        st_tile4(sm, VT + v1 * 128u + ((ch ^ (v1 & 7u)) << 4), __byte_perm(w[0], w[1], 0x7632),
+                              __byte_perm(w[2], w[3], 0x7632), __byte_perm(w[4], w[5], 0x7632), __byte_perm(w[6], w[7], 0x7632));
+                    }
+                }
+                if constexpr (!kScalar) {
+                    // q_r . k_r in fp32 over one 64-channel half; 16-byte chunks visited in a
+                    // row-dependent order (conflict-free)
+                    const int r = at & 63, hh = at >> 6;
+                    float pd = 0.f;
+                    if (r < L) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const uint32_t off = (uint32_t)r * 256u + (uint32_t)hh * 128u + (((uint32_t)(j + r) & 7u) << 4);
+                            const uint4 qv = *reinterpret_cast<const uint4*>(sm + IN_Q + off);
+                            const uint4 kv = *reinterpret_cast<const uint4*>(sm + IN_K + off);
+                            const uint32_t qa[4] = {qv.x, qv.y, qv.z, qv.w}, ka[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 a2 = bf16x2_to_float2(qa[e]), b2 = bf16x2_to_float2(ka[e]);
+                                pd = fmaf(a2.x, b2.x, pd);
+                                pd = fmaf(a2.y, b2.y, pd);
+                            }
+                        }
+                    }
+                    reinterpret_cast<float*>(sm + S_PD)[hh * 64 + r] = pd;
+                }
                 if (at == 0) {
                     int32_t* meta = sMeta + sl * 8u;
                     meta[0] = 1;
-                    meta[1] = h;
+                    meta[1] = cur.h;
                     meta[2] = cur.n;
-                    meta[3] = (int32_t)t0;
+                    meta[3] = (int32_t)cur.t0;
                     meta[4] = L;
-                    meta[5] = t0 == cur.bos ? 1 : 0;
-                    meta[6] = t0 + kChunk >= cur.eos ? 1 : 0;
+                    meta[5] = cur.t0 == cur.bos ? 1 : 0;
+                    meta[6] = cur.t0 + kChunk >= cur.eos ? 1 : 0;
+                    meta[7] = nxt.valid ? 1 : 0;   // another chunk follows in this CTA
                 }
-            }
-            fence_proxy_async();
-            if (named_bar_or(BAR_FE, kFeThreads, bad || *sAbort != 0u)) {
-                aborted = true;
-                break;
-            }
-            PIPE_MARK(128, 0, 5);
-            // ================ F5: hand the chunk to the chain; load the next one ================
-            // the next chunk's inputs: right away for the channel-wise gate (its A/P MMA reads the
-            // operand tiles); for the scalar gate once the A/P MMA, which reads the input tiles
-            // themselves, is done (in F6)
-            // (issued by an element thread: a TMA issue blocks its thread for several hundred
-            // cycles, which the aux warps' read-out and solve cannot spare)
-            auto load_next = [&]() {
-                if constexpr (kScalar)
-                    issue_chunk_loads_s(sm, bar_in, &tm_q, &tm_k, &tm_v, nxt.h, nxt.t0);
-                else
-                    issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, nxt.h, nxt.t0);
-            };
-            if (issuer) mbar_arrive(bar_formed);
-            if (!kScalar && loader && nxt.valid) load_next();
-            if (!kScalar) {
-                tma_pending = nxt.valid;
-                tma_parity = (ci + 1u) & 1u;
-            }
-            // beta of the next chunk: its latency is hidden behind the read-out and the solve (the
-            // load is unconditional, row clamped, so that nothing consumes it before the next F0)
-            if (is_aux && at < kChunk && nxt.valid) {
-                const int L1 = (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk);
-                beta_reg = p.beta[(nxt.t0 + (at < L1 ? at : L1 - 1)) * H + nxt.h];
-            }
-            // ================ F6: A / P read-out (aux warps, one per TMEM lane quarter) ================
-            // The element warps meanwhile compute the next chunk's gate (it overlaps the read-out and
-            // the solve).
-            if (!is_aux) {
-                if constexpr (kScalar) {
-                    // warp 8: the next chunk's gate input, then (once the A/P MMA has read the input
-                    // tiles) the next chunk's TMA loads
-                    if (warp == kElemWarp0) {
-                        if (nxt.valid) load_g_scalar(nxt);
-                        const bool ap_done = warp_wait(bar_ap, ci & 1u);
-                        if (!ap_done) *sAbort = 1u;
-                        if (ap_done && nxt.valid) {
-                            if (loader) load_next();
-                            tma_pending = true;
-                            tma_parity = (ci + 1u) & 1u;
-                        }
-                    }
-                } else if (nxt.valid) {
-                    const int L1 = (int)(nxt.eos - nxt.t0 < kChunk ? nxt.eos - nxt.t0 : kChunk);
-                    gate_tokens(p, nxt.h, nxt.t0, L1, c0, r0, a);
+                fence_proxy_async();
+                PIPE_MARK(128, 0, 5);
+                if (named_bar_or(BAR_FE, kFeThreads, bad || *sAbort != 0u)) {
+                    aborted = true;
+                    break;
                 }
-            } else {
-                const bool ap_done = warp_wait(bar_ap, ci & 1u);
-                if (!ap_done) *sAbort = 1u;
-                fence_after_sync();
                 PIPE_MARK(128, 0, 6);
-                const bool isA = quarter < 2;
-                const int r = (quarter & 1) * 32 + lane;      // token row of A (k rows) or P (q rows)
-                const int I = r >> 4;
-                const float be = reinterpret_cast<const float*>(sm + S_BETA)[sl * 64u + r];
-                const float pdg = reinterpret_cast<const float*>(sm + S_PD)[r] +
-                                  reinterpret_cast<const float*>(sm + S_PD)[64 + r];
-                float pmax = 0.f;
-#pragma unroll 1
-                for (int J = 0; J < 4; ++J) {
-                    float row[16];
-                    auto pick = [&](uint32_t col_a, uint32_t col_b, int I_a) {
-                        uint32_t ta[16], tb[16];
-                        tmem_ld16(taddr(tbase, quarter, TM_AP + col_a), ta);
-                        tmem_ld16(taddr(tbase, quarter, TM_AP + col_b), tb);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int x = 0; x < 16; ++x) row[x] = __uint_as_float(I == I_a ? ta[x] : tb[x]);
-                    };
-                    if constexpr (kScalar) {
-                        // raw K K^T / Q K^T times the scalar decay 2^(Gamma_r - Gamma_i) (<= 1 on and
-                        // below the diagonal)
-                        uint32_t raw[16];
-                        tmem_ld16(taddr(tbase, quarter, TM_AP + (uint32_t)J * 16u), raw);
-                        tmem_wait_ld();
-                        const float* gam = reinterpret_cast<const float*>(sm + S_GAM);
-                        const float gr = gam[r];
-#pragma unroll
-                        for (int x = 0; x < 16; ++x) {
-                            const int i = J * 16 + x;
-                            const bool keep = isA ? (i < r) : (i <= r);
-                            row[x] = keep ? __uint_as_float(raw[x]) * fast_ex2(gr - gam[i]) : 0.f;
-                        }
-                    } else {
-                    if ((quarter & 1) == 0) {        // I in {0, 1}
-                        if (J == 0) pick(0, 64, 0);            // I=0: diagonal; I=1: C1 of block 0
-                        else if (J == 1) pick(16, 16, 1);      // I=1: diagonal (I=0: masked)
-                        else {
-#pragma unroll
-                            for (int x = 0; x < 16; ++x) row[x] = 0.f;
-                        }
-                    } else {                         // I in {2, 3}
-                        if (J == 0) pick(112, 144, 2);         // I=2: C2 of block 0; I=3: C3 of block 0
-                        else if (J == 1) pick(80, 128, 2);     // I=2: C1 of block 1; I=3: C2 of block 1
-                        else if (J == 2) pick(32, 96, 2);      // I=2: diagonal; I=3: C1 of block 2
-                        else pick(48, 48, 3);                  // I=3: diagonal (I=2: masked)
-                    }
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        const int i = J * 16 + x;
-                        row[x] = i < r ? row[x] : ((i == r && !isA) ? pdg : 0.f);
-                    }
-                    }
-                    if (isA) {
-                        float* a32 = reinterpret_cast<float*>(sm + A32) + r * kF32Pitch + J * 16;
-#pragma unroll
-                        for (int x = 0; x < 16; x += 4)
-                            *reinterpret_cast<float4*>(a32 + x) =
-                                make_float4(be * row[x], be * row[x + 1], be * row[x + 2], be * row[x + 3]);
-                    } else {
-                        // P^T (MN-major, K = token i, N = row r): 16-bit stores, a warp writes 64
-                        // contiguous bytes per i
-#pragma unroll
-                        for (int x = 0; x < 16; ++x) {
-                            const int i = J * 16 + x;
-                            pmax = fmaxf(pmax, fabsf(row[x]));
-                            st_tile_h(sm, PT + sw128_off((uint32_t)i, (uint32_t)r, 64u),
-                                      __half_as_ushort(__float2half_rn(fminf(fmaxf(row[x], -65504.f), 65504.f))));
-                        }
+                // the next chunk's inputs: the current ones are consumed (for the scalar gate the A/P
+                // MMA reads them too, so the loads wait for it at the start of the next read-out)
+                if constexpr (!kScalar) {
+                    if (loader && nxt.valid) {
+                        load_inputs(nxt);
+                        tma_pending = true;
+                        tma_parity = (ci + 1u) & 1u;
                     }
                 }
-                if (pmax >= kRangeHi) range_bad = 1u;
-                fence_proxy_async();
-                tmem_wait_ld();
-                fence_before_sync();
-                named_bar_sync(BAR_AUX, 128);
-                PIPE_MARK(128, 0, 7);
-                const int sw = warp - kAuxWarp0;
-                const float* a32 = reinterpret_cast<const float*>(sm + A32);
-                float* t32 = reinterpret_cast<float*>(sm + T32);
-                float tmax = 0.f;
-                auto Ab = [&](int I, int J) { return a32 + 16 * I * kF32Pitch + 16 * J; };
-                auto Tb = [&](int I, int J) { return t32 + 16 * I * kF32Pitch + 16 * J; };
-                // one warp writes the fp16 copy of finished block (I, J): lane -> (row, 8-col chunk)
-                auto to_t16 = [&](int I, int J) {
-                    const int rr = lane >> 1, ch = lane & 1;
-                    const float* src = Tb(I, J) + rr * kF32Pitch + ch * 8;
-                    const float4 lo4 = *reinterpret_cast<const float4*>(src);
-                    const float4 hi4 = *reinterpret_cast<const float4*>(src + 4);
-                    tmax = fmaxf(tmax, fmaxf(fmaxf(fmaxf(fabsf(lo4.x), fabsf(lo4.y)), fmaxf(fabsf(lo4.z), fabsf(lo4.w))),
-                                             fmaxf(fmaxf(fabsf(hi4.x), fabsf(hi4.y)), fmaxf(fabsf(hi4.z), fabsf(hi4.w)))));
-                    st_v4(sm, T16 + sw128_chunk_off(16 * I + rr, 2 * J + ch, 64), pack_f16s(lo4.x, lo4.y),
-                          pack_f16s(lo4.z, lo4.w), pack_f16s(hi4.x, hi4.y), pack_f16s(hi4.z, hi4.w));
-                };
-                // sign * (a 16 x 16 warp-MMA accumulator) straight into block (I, J) of the fp16 tile
-                auto acc_to_t16 = [&](int I, int J, const float (&acc)[2][4], float sign) {
-                    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-                    for (int nh = 0; nh < 2; ++nh) {
-                        const uint32_t col = (uint32_t)(16 * J + 8 * nh + 2 * t);
-                        tmax = fmaxf(tmax, fmaxf(fmaxf(fabsf(acc[nh][0]), fabsf(acc[nh][1])),
-                                                 fmaxf(fabsf(acc[nh][2]), fabsf(acc[nh][3]))));
-                        *reinterpret_cast<uint32_t*>(sm + T16 + sw128_off((uint32_t)(16 * I + g), col, 64u)) =
-                            pack_f16s(sign * acc[nh][0], sign * acc[nh][1]);
-                        *reinterpret_cast<uint32_t*>(sm + T16 + sw128_off((uint32_t)(16 * I + g + 8), col, 64u)) =
-                            pack_f16s(sign * acc[nh][2], sign * acc[nh][3]);
-                    }
-                };
-                // L0: the four 16 x 16 diagonal blocks by forward substitution in fp32, one column
-                // per thread (threads 0-63), right-looking
-                if (sw < 2) {
-                    const int bI = at >> 4, jc = at & 15, o = bI * 16;
-                    float x[16];
-#pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == jc) ? 1.f : 0.f;
-#pragma unroll
-                    for (int ii = 0; ii < 15; ++ii) {
-                        const float xi = x[ii];
-#pragma unroll
-                        for (int rr = ii + 1; rr < 16; ++rr) x[rr] = fmaf(-a32[(o + rr) * kF32Pitch + o + ii], xi, x[rr]);
-                    }
-#pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) t32[(o + rr) * kF32Pitch + o + jc] = x[rr];
-                }
-                named_bar_sync(BAR_AUX, 128);
-                PIPE_MARK(128, 0, 8);
-                // L1 (16 x 16 warp-MMA products, fp16 operands, fp32 accumulation):
-                //   T10 = -T11 (A10 T00), T32 = -T33 (A32 T22),
-                //   X20 = A20 T00 + A21 T10, X30 = A30 T00 + A31 T10, X21 = A21 T11, X31 = A31 T11.
-                // Aux warps 0 and 2 both form T10 (in their own scratch) so that neither waits for
-                // the other.  Scratch: T's and A's blocks above the diagonal.
-                {
-                    float* const a32w = reinterpret_cast<float*>(sm + A32);
-                    auto Aw = [&](int I, int J) { return a32w + 16 * I * kF32Pitch + 16 * J; };
-                    float acc[2][4] = {};
-                    if (sw == 0 || sw == 2) {
-                        float* ysc = sw == 0 ? Tb(0, 1) : Aw(0, 1);     // A10 T00
-                        float* t10 = sw == 0 ? Tb(1, 0) : Aw(0, 2);     // T10
-                        warpmma::mm16_acc_h(Ab(1, 0), kF32Pitch, Tb(0, 0), kF32Pitch, acc);
-                        warpmma::store16(ysc, kF32Pitch, acc, 1.f);
-                        __syncwarp();
-                        float a2[2][4] = {};
-                        warpmma::mm16_acc_h(Tb(1, 1), kF32Pitch, ysc, kF32Pitch, a2);
-                        warpmma::store16(t10, kF32Pitch, a2, -1.f);
-                        __syncwarp();
-                        if (sw == 0) to_t16(1, 0);
-                        const int I = sw == 0 ? 2 : 3;
-                        float a3[2][4] = {};
-                        warpmma::mm16_acc_h(Ab(I, 0), kF32Pitch, Tb(0, 0), kF32Pitch, a3);
-                        warpmma::mm16_acc_h(Ab(I, 1), kF32Pitch, t10, kF32Pitch, a3);
-                        warpmma::store16(Tb(0, I), kF32Pitch, a3, 1.f);            // X20 / X30
-                    } else if (sw == 1) {
-                        warpmma::mm16_acc_h(Ab(3, 2), kF32Pitch, Tb(2, 2), kF32Pitch, acc);
-                        warpmma::store16(Tb(2, 3), kF32Pitch, acc, 1.f);            // A32 T22
-                        __syncwarp();
-                        float a2[2][4] = {};
-                        warpmma::mm16_acc_h(Tb(3, 3), kF32Pitch, Tb(2, 3), kF32Pitch, a2);
-                        warpmma::store16(Tb(3, 2), kF32Pitch, a2, -1.f);           // T32
-                        __syncwarp();
-                        to_t16(3, 2);
-                        float a3[2][4] = {};
-                        warpmma::mm16_acc_h(Ab(2, 1), kF32Pitch, Tb(1, 1), kF32Pitch, a3);
-                        warpmma::store16(Tb(1, 2), kF32Pitch, a3, 1.f);            // X21
-                    } else {
-                        warpmma::mm16_acc_h(Ab(3, 1), kF32Pitch, Tb(1, 1), kF32Pitch, acc);
-                        warpmma::store16(Tb(1, 3), kF32Pitch, acc, 1.f);            // X31
-#pragma unroll
-                        for (int d = 0; d < 4; ++d) to_t16(d, d);
-                    }
-                }
-                named_bar_sync(BAR_AUX, 128);
-                // L2: T_LL = -T_LR X, written straight to the fp16 tile:
-                //   T20 = -T22 X20, T21 = -T22 X21, T30 = -(T32 X20 + T33 X30), T31 = -(T32 X21 + T33 X31)
-                {
-                    float acc[2][4] = {};
-                    const int J = sw & 1;
-                    if (sw < 2) {
-                        warpmma::mm16_acc_h(Tb(2, 2), kF32Pitch, Tb(J, 2), kF32Pitch, acc);
-                        acc_to_t16(2, J, acc, -1.f);
-                    } else {
-                        warpmma::mm16_acc_h(Tb(3, 2), kF32Pitch, Tb(J, 2), kF32Pitch, acc);
-                        warpmma::mm16_acc_h(Tb(3, 3), kF32Pitch, Tb(J, 3), kF32Pitch, acc);
-                        acc_to_t16(3, J, acc, -1.f);
-                    }
-                }
-                if (tmax >= kRangeHi) range_bad = 1u;
-                fence_proxy_async();
-                named_bar_sync(BAR_AUX, 128);
-                if (at == 0) mbar_arrive(bar_t);
+                next_in = nxt;
+                cur = nxt;
+                ++ci;
             }
-            if (named_bar_or(BAR_FE, kFeThreads, *sAbort != 0u)) {
-                aborted = true;
-                break;
+            if (aborted) {
+                *sAbort = 1u;
+                if (loader && tma_pending) mbar_wait_bounded(bar_in, tma_parity);
             }
-            cur = nxt;
-            ++ci;
         }
         if (range_bad) record_error(KDA_DEVERR_RANGE);
-        if (!aborted) {
-            if (issuer) {
-                sMeta[(ci & 1u) * 8u] = 0;   // end of work for the chain
-                *sEnd = 1u;
-                mbar_arrive(bar_apready);
-                mbar_arrive(bar_formed);
-            }
-        } else {
-            *sAbort = 1u;
-            if ((issuer || loader) && tma_pending) mbar_wait_bounded(bar_in, tma_parity);
-        }
     }
 
     // wind-down: every role has drained its own asynchronous operations

@@ -2,8 +2,8 @@
 
 Builds the instrumented library (``build.py --phase-clocks``: the same kernel with clock64()
 marks between its phases, accumulated per CTA), runs one workload through it and prints the
-average cycles per 64-token chunk of each phase, for the front end (thread 128) and the state
-chain (thread 0).  Run it by path from the repository root (importing the package loads the
+average cycles per 64-token chunk of each phase, for the aux warps (thread 128), the element
+warps (thread 256) and the state chain (thread 0).  Run it by path from the repository root (importing the package loads the
 product library, so this script sets KDA_LIBRARY before it imports the package):
 
     python gated_delta_rule_135_b200/phase_clocks.py [--workload 2] [--gdn]
@@ -24,24 +24,30 @@ _ROOT = os.path.dirname(_HERE)
 # index = slot of the kernel's phase marks; each counts the cycles since the previous mark
 # of the same role
 PHASES = [
-    ("FE", "solve L1 + L2, loop to the next chunk"),
-    ("FE", "F0 block products of a / beta"),
-    ("FE", "F2 A/P operand tiles, P diagonal"),
-    ("FE", "F3 signal A/P operands ready"),
-    ("FE", "F4 wait for the previous state update"),
-    ("FE", "F4 B1, Khat, V^T tiles"),
-    ("FE", "F5/F6 hand-off, next TMA, wait for A/P"),
-    ("FE", "F6 A / P read-out"),
-    ("FE", "solve L0 (diagonal blocks)"),
+    ("aux", "wait for the A/P product of chunk n-1"),
+    ("aux", "A / P read-out of chunk n-1"),
+    ("aux", "solve L0 (diagonal blocks)"),
+    ("aux", "solve L1 + L2, T written"),
+    ("aux", "wait for the last [S|O] MMA and the inputs"),
+    ("aux", "V^T, P diagonal, metadata of chunk n"),
+    ("aux", "meet the element warps"),
+    ("-", "(unused)"),
+    ("-", "(unused)"),
     ("chain", "wait for the previous [S|O] MMA"),
     ("chain", "output of the previous chunk"),
-    ("chain", "wait for A/P operands, issue the A/P MMA"),
+    ("chain", "wait for A/P operands and read-out, issue"),
     ("chain", "(between marks)"),
     ("chain", "wait for the chunk's operands"),
     ("chain", "S^T -> fp16, [O|Y] MMA, S <- S Diag(gamma_C)"),
     ("chain", "wait [O|Y], Y^T += beta V^T -> fp16"),
     ("chain", "wait T, U MMA, wait U"),
     ("chain", "U -> fp16, [S|O] MMA issue"),
+    ("elem", "beta, block products / gate scan"),
+    ("elem", "wait for the inputs and the last A/P MMA"),
+    ("elem", "A/P operand tiles"),
+    ("elem", "wait for the last [S|O] MMA"),
+    ("elem", "B1, Khat tiles, meet the aux warps"),
+    ("elem", "next chunk: TMA, beta, gate"),
 ]
 
 
@@ -89,12 +95,13 @@ def main(argv=None) -> int:
         raise RuntimeError("reading the phase counters failed")
     chunks = sum((s + 63) // 64 for s in w.seq_lens) * w.H
     print(f"instrumented kernel {e0.elapsed_time(e1):.3f} ms, {chunks} chunk-heads")
-    tot = {"FE": 0.0, "chain": 0.0}
+    tot = {"aux": 0.0, "elem": 0.0, "chain": 0.0, "-": 0.0}
     for (role, name), c in zip(PHASES, buf):
         per = c / chunks
         tot[role] += per
-        print(f"{role:5s}  {name:46s} {per:8.0f} cycles/chunk")
-    print(f"front end {tot['FE']:.0f}, chain {tot['chain']:.0f} cycles/chunk")
+        if role != "-":
+            print(f"{role:5s}  {name:46s} {per:8.0f} cycles/chunk")
+    print(f"aux {tot['aux']:.0f}, element {tot['elem']:.0f}, chain {tot['chain']:.0f} cycles/chunk")
     return 0
 
 
