@@ -16,15 +16,16 @@
 //                         U^T        = Y^T T^T                                             K = 64
 //                         U^T -> fp16 (TMEM);  [S | O]^T += U^T [Khat | P^T]              N = 192
 //                         O^T -> bf16 out (times scale 2^sigma_v)
-//   aux warps 4-7       beta, V^T, the exact diagonal q_r . k_r of P, the A/P MMA issue, the
-//                       A / P read-out (with all front-end warps) and T = (I + A)^-1
-//   element warps 8-15  gate and decay factors (thread: 4 channels x 8 tokens) and every
-//                       decayed operand tile
+//   element warps 8-15  chunk n: beta, gate and decay factors (thread: 4 channels x 8 tokens)
+//                       and every decayed operand tile
+//   aux warps 4-7       meanwhile chunk n - 1: the A / P read-out (one warp per TMEM lane
+//                       quarter) and T = (I + A)^-1; then chunk n's V^T, the exact diagonal
+//                       q_r . k_r of P, its metadata, and the TMA loads of chunk n + 1
 //
 // Y = beta V - beta gamma K S and U = T Y is the WY/UT form U = T diag(beta)(V - (gamma K) S)
 // of the chunk (U~ - W S with the product by T taken last), so that the part of the chain that
-// needs the state does not wait for the triangular solve: the front end (aux + element warps)
-// builds chunk j+1 while the chain warps finish chunk j.
+// needs the state does not wait for the triangular solve: the element warps build chunk n + 1
+// while the aux warps solve chunk n and the chain warps finish it.
 //
 // Decay factors (16-token blocks, R_r = e^{Gamma_r - Gamma_(block start)} <= 1 and
 // E_r = e^{Gamma_(block end) - Gamma_r} <= 1, formed as running products of a_t): the A/P MMA
@@ -150,6 +151,10 @@ struct Params {
 
 #ifdef KDA_PHASE_CLOCKS
 __device__ unsigned long long g_pipe_phase_cycles[kPhases];
+constexpr int kMaxCtaRecords = 1024;
+// per CTA: global timer at entry and at exit (ns), chunks run, SM id, then its phase cycles
+constexpr int kCtaRec = 4 + kPhases;
+__device__ unsigned long long g_pipe_cta[kMaxCtaRecords][kCtaRec];
 // thread `who` adds the cycles since its role's previous mark to slot i
 #define PIPE_MARK(who, slot, i)                                            \
     do {                                                                   \
@@ -598,6 +603,10 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+#ifdef KDA_PHASE_CLOCKS
+    const unsigned long long t_entry = global_ns();
+    unsigned long long n_chunks = 0;
+#endif
     const int G = gridDim.x, b = blockIdx.x;
     const int H = p.H;
     const int units = p.N * H;
@@ -1013,6 +1022,9 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             PIPE_MARK(0, 1, 17);
             have_prev = true;
+#ifdef KDA_PHASE_CLOCKS
+            ++n_chunks;
+#endif
             prev_h = m_h;
             prev_n = m_n;
             prev_t0 = m_t0;
@@ -1643,8 +1655,18 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     fence_after_sync();
     if (warp == 0) tmem_dealloc(tbase, TM_COLS);
 #ifdef KDA_PHASE_CLOCKS
-    if (tid == 0)
+    if (tid == 0) {
         for (int i = 0; i < kPhases; ++i) atomicAdd(&g_pipe_phase_cycles[i], (unsigned long long)sPh[i]);
+        if (blockIdx.x < kMaxCtaRecords) {
+            unsigned int smid;
+            asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+            g_pipe_cta[blockIdx.x][0] = t_entry;
+            g_pipe_cta[blockIdx.x][1] = global_ns();
+            g_pipe_cta[blockIdx.x][2] = n_chunks;
+            g_pipe_cta[blockIdx.x][3] = smid;
+            for (int i = 0; i < kPhases; ++i) g_pipe_cta[blockIdx.x][4 + i] = sPh[i];
+        }
+    }
 #endif
 }
 
@@ -1724,13 +1746,25 @@ cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
 
 #ifdef KDA_PHASE_CLOCKS
 // Debug builds only: copies and clears the per-phase cycle totals of the pipelined kernel
-// (slots 0-8: front end, thread 128; slots 9-17: chain, thread 0).
+// (slots 0-6: aux warps, thread 128; slots 9-17: chain, thread 0; slots 18-23: element warps,
+// thread 256).
 extern "C" int kda_debug_pipe_phase_cycles(unsigned long long* out) {
     if (cudaMemcpyFromSymbol(out, pipe::g_pipe_phase_cycles, sizeof(unsigned long long) * pipe::kPhases) !=
         cudaSuccess)
         return -1;
     unsigned long long zero[pipe::kPhases] = {};
     return cudaMemcpyToSymbol(pipe::g_pipe_phase_cycles, zero, sizeof zero) == cudaSuccess ? pipe::kPhases : -1;
+}
+// Debug builds only: per-CTA records of the last launch (entry and exit global time in ns, chunks
+// run, SM id, then the CTA's cycles per phase slot), up to max_ctas of them; returns how many
+// were copied.
+extern "C" int kda_debug_pipe_cta(unsigned long long* out, int max_ctas) {
+    const int n = max_ctas < pipe::kMaxCtaRecords ? max_ctas : pipe::kMaxCtaRecords;
+    if (n <= 0) return 0;
+    return cudaMemcpyFromSymbol(out, pipe::g_pipe_cta, sizeof(unsigned long long) * pipe::kCtaRec * (size_t)n) ==
+                   cudaSuccess
+               ? n
+               : -1;
 }
 #endif
 

@@ -102,6 +102,32 @@ def main(argv=None) -> int:
         if role != "-":
             print(f"{role:5s}  {name:46s} {per:8.0f} cycles/chunk")
     print(f"aux {tot['aux']:.0f}, element {tot['elem']:.0f}, chain {tot['chain']:.0f} cycles/chunk")
+    # per-CTA spans of the same launch: the kernel ends with its slowest CTA
+    lib.kda_debug_pipe_cta.restype = ctypes.c_int
+    nrec = 4 + len(PHASES)
+    rec = (ctypes.c_ulonglong * (nrec * 1024))()
+    n = lib.kda_debug_pipe_cta(rec, 1024)
+    ctas = []
+    for i in range(max(n, 0)):
+        r = rec[nrec * i:nrec * (i + 1)]
+        if r[1] > r[0] and r[2] > 0:
+            ctas.append({"us": (r[1] - r[0]) / 1e3, "chunks": r[2], "sm": r[3], "t0": r[0], "ph": r[4:]})
+    if ctas:
+        ctas.sort(key=lambda c: c["us"])
+        start = min(c["t0"] for c in ctas)
+        per = sorted(c["us"] / c["chunks"] for c in ctas)
+        print(f"CTAs {len(ctas)}: span min {ctas[0]['us']:.1f} median {ctas[len(ctas) // 2]['us']:.1f} "
+              f"max {ctas[-1]['us']:.1f} us; us per chunk min {per[0]:.3f} median {per[len(per) // 2]:.3f} "
+              f"max {per[-1]:.3f}; latest start {max(c['t0'] - start for c in ctas) / 1e3:.1f} us")
+        by_rate = sorted(ctas, key=lambda c: c["us"] / c["chunks"])
+        for label, group in (("fastest", by_rate[:8]), ("slowest", by_rate[-8:])):
+            print(f"{label} 8 CTAs per chunk (us {sum(c['us'] / c['chunks'] for c in group) / 8:.3f}; "
+                  f"SMs {[c['sm'] for c in group]}; chunks {[c['chunks'] for c in group]}):")
+            for k, (role, name) in enumerate(PHASES):
+                if role == "-":
+                    continue
+                v = sum(c["ph"][k] / c["chunks"] for c in group) / len(group)
+                print(f"   {role:5s}  {name:46s} {v:8.0f}")
     return 0
 
 
