@@ -748,71 +748,43 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             return hmax_to_float(m);
         };
 
-        // The front end's A/P MMA of chunk cc (thread 0): its operand tiles are written and the
-        // previous chunk's product has been read out of TMEM.  It does not depend on the state, so it
-        // goes before the previous chunk's output when both barriers are already complete, and after
-        // it otherwise.  block = false only tests the barriers; ap_open stays set until the step is
-        // settled (the MMA issued, the end of the work seen, or a wait run out).
-        bool ap_open = false;   // thread 0: chunk cc's A/P step not settled yet
-        bool ap_seen = false;   // thread 0: chunk cc's A/P operand tiles seen ready
-        auto issue_ap = [&](bool block) {
-            if (!ap_seen) {
-                if (block) {
-                    if (!mbar_wait_bounded(bar_apready, cc & 1u)) {
-                        record_error(KDA_DEVERR_TIMEOUT);
-                        *sAbort = 1u;
-                        ap_open = false;
-                        return;
-                    }
-                } else if (!mbar_test_wait(bar_apready, cc & 1u)) {
-                    return;
-                }
-                ap_seen = true;
+        // The front end's A/P MMA of chunk cc (thread 0), as soon as its operand tiles are written
+        // and the previous chunk's product has been read out of TMEM.  It does not depend on the
+        // state, so it goes before the previous chunk's output: the front end waits for it twice
+        // (its read-out, and the next chunk's operand tiles, which overwrite its inputs).
+        auto issue_ap = [&]() {
+            if (!mbar_wait_bounded(bar_apready, cc & 1u) ||
+                (cc > 0 && !mbar_wait_bounded(bar_ro, (cc - 1) & 1u))) {
+                record_error(KDA_DEVERR_TIMEOUT);
+                *sAbort = 1u;
+                return;
             }
-            {
-                if (cc > 0) {
-                    if (block) {
-                        if (!mbar_wait_bounded(bar_ro, (cc - 1) & 1u)) {
-                            record_error(KDA_DEVERR_TIMEOUT);
-                            *sAbort = 1u;
-                            ap_open = false;
-                            return;
-                        }
-                    } else if (!mbar_test_wait(bar_ro, (cc - 1) & 1u)) {
-                        return;
-                    }
-                }
-                fence_after_sync();
-                if constexpr (kScalar) {
-                    // [K ; Q] K^T straight from the swizzled input blocks (the decay is applied at
-                    // read-out)
-                    const uint32_t a0 = smem_u32(sm + IN_Q);
+            fence_after_sync();
+            if constexpr (kScalar) {
+                // [K ; Q] K^T straight from the swizzled input blocks (the decay is applied at
+                // read-out)
+                const uint32_t a0 = smem_u32(sm + IN_Q);
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(a0, 128, ks), IDESC_AP_S,
-                                ks > 0 ? 1u : 0u);
-                } else {
-                    const uint32_t a0 = smem_u32(sm + AP_A), b0 = smem_u32(sm + AP_B);
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(a0, 128, ks), IDESC_AP_S,
+                            ks > 0 ? 1u : 0u);
+            } else {
+                const uint32_t a0 = smem_u32(sm + AP_A), b0 = smem_u32(sm + AP_B);
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
-                                ks > 0 ? 1u : 0u);
-                }
-                mma_commit(bar_ap);
-                ++issued_ap;
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_f16(tbase + TM_AP, desc_kmajor(a0, 128, ks), desc_kmajor(b0, 160, ks), IDESC_AP,
+                            ks > 0 ? 1u : 0u);
             }
-            ap_open = false;
+            mma_commit(bar_ap);
+            ++issued_ap;
         };
 
         // whether another chunk follows (the front end marks a CTA's last chunk in its metadata)
         bool more = unit_from(p, sOrder, b, G, units, 0).valid;
         while (true) {
             bool bad = false;
-            if (tid == 0 && more) {
-                ap_open = true;
-                ap_seen = false;
-                issue_ap(false);
-            }
+            if (tid == 0 && more) issue_ap();
+            PIPE_MARK(0, 1, 11);
             // the previous chunk's output (and final state), once its [S | O] MMA is done
             if (have_prev) {
                 bad |= !warp_wait(bar_s, (cc - 1) & 1u);
@@ -823,8 +795,6 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             PIPE_MARK(0, 1, 10);
             if (!more) break;
-            if (tid == 0 && ap_open) issue_ap(true);
-            PIPE_MARK(0, 1, 11);
             PIPE_MARK(0, 1, 12);
             bad |= !warp_wait(bar_formed, cc & 1u);
             const int32_t* meta = sMeta + (cc & 1u) * 8u;
