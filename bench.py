@@ -72,7 +72,7 @@ def parse():
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward kda_bwd (all gradients) instead of the forward")
     ap.add_argument("--lower-bound", type=float, default=None,
-                    help="override the workload's gate clamp (below -5.3 kda_fwd takes the staged kernels)")
+                    help="override the workload's gate clamp (below -9.5 kda_fwd takes the staged kernels)")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the workload's head count (small cases for profiling)")
     ap.add_argument("--segments", type=int, default=0,

@@ -21,7 +21,7 @@ LIB_PATH = os.environ.get("KDA_LIBRARY", os.path.join(_HERE, "libkda.so"))
 
 HEAD_DIM = 128
 CHUNK = 64
-FUSED_MIN_LOWER_BOUND = -5.3
+FUSED_MIN_LOWER_BOUND = -9.5
 
 KDA_OK = 0
 STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",

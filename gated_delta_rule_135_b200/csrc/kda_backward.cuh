@@ -992,7 +992,8 @@ cudaError_t launch_bwd(const StagedArgs& a, const BwdArgs& d, char* ws, const Bw
             u, du, dO, cs, dsn, table, count, H, a.scale, dkhat, dqg, dw, dgc);
         bwd::t_side_bwd_kernel<<<g3, bwd::kB3Threads, bwd::kB3aSmem, stream>>>(
             k, v, a.beta, gamma, tm, du, dw, table, count, H, d.dk, d.dv, dG, d.dbeta, da);
-        auto decay = fused_supported(a.lower_bound) ? bwd::decay_bwd_kernel<true> : bwd::decay_bwd_kernel<false>;
+        // the factored pair sums need 16 tokens of decay inside the fp32 range (16 x 5.3 < 87)
+        auto decay = a.lower_bound >= -5.3f ? bwd::decay_bwd_kernel<true> : bwd::decay_bwd_kernel<false>;
         decay<<<g3, bwd::kB3bThreads, bwd::kB3bSmem, stream>>>(
             q, k, a.g, a.beta, a.A_log, a.dt_bias, a.lower_bound, a.scale, gamma, u, dO, da, dqg, dkhat, dgc, dG,
             table, count, H, d.dq, d.dk, d.dg, d.dbeta, dalog_part, ddt_part);

@@ -27,12 +27,13 @@
 // needs the state does not wait for the triangular solve: the element warps build chunk n + 1
 // while the aux warps solve chunk n and the chain warps finish it.
 //
-// Decay factors (16-token blocks, R_r = e^{Gamma_r - Gamma_(block start)} <= 1 and
-// E_r = e^{Gamma_(block end) - Gamma_r} <= 1, formed as running products of a_t): the A/P MMA
-// (bf16, M = 128 x N = 160) multiplies [k R ; q R] by the diagonal-block operand k E / R_block
-// (>= 1, at most e^{16 |lower_bound|}) and the block-distance operands k E, k E F2, k E F3.
-// So the kernel requires lower_bound >= -5.3 (16 x 5.3 = 84.8 < 87); steeper gates take the
-// staged path.  P's main diagonal (no decay, the dominant output term) is taken exactly in fp32.
+// Decay factors (16-token blocks; running products of a_t): the A/P MMA (bf16, M = 128 x N = 160)
+// multiplies [k R' ; q R'] (R'_r = e^{Gamma_r - Gamma_(block middle)}) by the diagonal-block
+// operand k E' (E'_i = e^{Gamma_(block middle) - Gamma_i}) and the block-distance operands
+// k E F_d (E = e^{Gamma_(block end) - Gamma_i} <= 1, F_d <= 1 the decay from block J's end to the
+// middle of block J + d).  Every factor lies within e^{+-8 |lower_bound|}, so with |q|, |k| < 2^15
+// the kernel takes lower_bound >= -9.5 (8 x 9.5 = 76 and 2^15 e^76 < 3.4e38); steeper gates take
+// the staged path.  P's main diagonal (no decay, the dominant output term) is taken exactly in fp32.
 //
 // Operand precision: decay blocks bf16, everything that multiplies T, S, Y, U or P in fp16,
 // accumulation and the carried state in fp32.
@@ -88,7 +89,8 @@ constexpr int kPhases = 24;
 // rewrite for the next chunk while the aux warps solve): A's diagonal 16 x 16 blocks in fp32
 // (row pitch 20 floats), its six blocks below the diagonal and the solve's intermediate blocks
 // in fp16 (row pitch 24 halves; both pitches keep row accesses free of bank conflicts).
-constexpr uint32_t SV = 210432;
+constexpr uint32_t S_PHALF = 210432;                    // fp32 [4][128] product of a over each block's first 8 tokens
+constexpr uint32_t SV = S_PHALF + 2048;
 constexpr int kAdPitch = 20;
 constexpr int kHp = 24;
 constexpr uint32_t kHBlk = 16 * kHp * 2;                // bytes of one fp16 block
@@ -1096,7 +1098,8 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 // ================ E0: beta; block products of a / the scalar gate's scan ================
                 if (et < kChunk) reinterpret_cast<float*>(sm + S_BETA)[sl * 64u + et] = et < L ? beta_reg : 0.f;
-                float po[4];   // channel gate: product of a over the other 8-token half of the block
+                float po[4];    // channel gate: product of a over the other 8-token half of the block
+                float own4[4];  // and over this thread's own 8 tokens
                 if constexpr (kScalar) {
                     // the inputs must have landed: rows past the valid length are zeroed in the tiles,
                     // which are MMA operands themselves
@@ -1114,10 +1117,13 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         float own = a[0][e];
 #pragma unroll
                         for (int i = 1; i < 8; ++i) own *= a[i][e];
+                        own4[e] = own;
                         po[e] = __shfl_xor_sync(0xffffffffu, own, 16);
-                        if ((lane >> 4) == 0) own *= po[e];          // block product (both halves agree)
-                        if ((lane >> 4) == 0)
-                            reinterpret_cast<float*>(sm + S_PTOT)[eI * kHeadDim + c0 + e] = own;
+                        if ((lane >> 4) == 0) {
+                            // block product (both halves agree) and the first half's product
+                            reinterpret_cast<float*>(sm + S_PTOT)[eI * kHeadDim + c0 + e] = own * po[e];
+                            reinterpret_cast<float*>(sm + S_PHALF)[eI * kHeadDim + c0 + e] = own;
+                        }
                     }
                 }
                 named_bar_sync(BAR_ELEM, 256);
@@ -1128,20 +1134,52 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     // the previous chunk's A/P MMA has read the tiles this phase rewrites
                     if (ci > 0) bad |= !warp_wait(bar_ap, (ci - 1) & 1u);
                     PIPE_MARK(256, 2, 19);
+                    // Decays are taken relative to the middle of each 16-token block: the A side k R' and
+                    // q R' with R'_r = (product of a from the block start to r) / M_I (M_I = product over
+                    // the block's first 8 tokens), the diagonal-block B side k E / S2_I (S2_I = product over
+                    // its last 8 tokens), so every factor lies within e^{+-8 |lower_bound|}.  The
+                    // block-distance operands of block J carry M of the row block J + d.
                     const float* ptot = reinterpret_cast<const float*>(sm + S_PTOT);
-                    float4 pt[4];
+                    const float* phalf = reinterpret_cast<const float*>(sm + S_PHALF);
+                    const bool second = (lane >> 4) != 0;
+                    auto ld4 = [&](const float* base, int J) {
+                        const float4 x = *reinterpret_cast<const float4*>(base + (J < 3 ? J : 3) * kHeadDim + c0);
+                        return x;
+                    };
+                    const float4 P1 = ld4(ptot, eI + 1), P2 = ld4(ptot, eI + 2);
+                    const float4 M1 = ld4(phalf, eI + 1), M2 = ld4(phalf, eI + 2), M3 = ld4(phalf, eI + 3);
+                    const float2 F1a_ = make_float2(M1.x, M1.y), F1b_ = make_float2(M1.z, M1.w);
+                    const float2 P1a = make_float2(P1.x, P1.y), P1b = make_float2(P1.z, P1.w);
+                    const float2 F2a_ = __fmul2_rn(P1a, make_float2(M2.x, M2.y)), F2b_ = __fmul2_rn(P1b, make_float2(M2.z, M2.w));
+                    const float2 F3a_ = __fmul2_rn(__fmul2_rn(P1a, make_float2(P2.x, P2.y)), make_float2(M3.x, M3.y));
+                    const float2 F3b_ = __fmul2_rn(__fmul2_rn(P1b, make_float2(P2.z, P2.w)), make_float2(M3.z, M3.w));
+                    // Each thread's factors start from its own 8-token half (so that none underflows
+                    // when the other half decays steeply): E is the suffix product within the half,
+                    // the diagonal-block operand k E (first half) or k E / S2 (second half), the
+                    // block-distance operands k E times the rest of the block (first half: S2) and
+                    // F_d, and R' = (running product) / M (first half) or the running product.
+                    float xs[4], cs[4], r0p[4];
 #pragma unroll
-                    for (int J = 0; J < 4; ++J) pt[J] = *reinterpret_cast<const float4*>(ptot + J * kHeadDim + c0);
-                    auto pick = [&](int J) { return J == 0 ? pt[0] : (J == 1 ? pt[1] : (J == 2 ? pt[2] : pt[3])); };
-                    const float4 pbI = pick(eI);
-                    const float invB[4] = {fast_rcp(pbI.x), fast_rcp(pbI.y), fast_rcp(pbI.z), fast_rcp(pbI.w)};
-                    const float4 p1 = pick(eI < 3 ? eI + 1 : 3), p2 = pick(eI < 2 ? eI + 2 : 3);
-                    const float2 invB01 = make_float2(invB[0], invB[1]), invB23 = make_float2(invB[2], invB[3]);
-                    const float2 F2a = make_float2(p1.x, p1.y), F2b = make_float2(p1.z, p1.w);
-                    const float2 F3a = __fmul2_rn(F2a, make_float2(p2.x, p2.y)), F3b = __fmul2_rn(F2b, make_float2(p2.z, p2.w));
+                    for (int e = 0; e < 4; ++e) {
+                        xs[e] = second ? fast_rcp(own4[e]) : 1.f;
+                        cs[e] = second ? 1.f : po[e];
+                        r0p[e] = second ? 1.f : fast_rcp(own4[e]);
+                    }
+                    const float2 invB01 = make_float2(xs[0], xs[1]), invB23 = make_float2(xs[2], xs[3]);
+                    const float2 F1a = __fmul2_rn(make_float2(cs[0], cs[1]), F1a_),
+                                 F1b = __fmul2_rn(make_float2(cs[2], cs[3]), F1b_);
+                    const float2 F2a = __fmul2_rn(make_float2(cs[0], cs[1]), F2a_),
+                                 F2b = __fmul2_rn(make_float2(cs[2], cs[3]), F2b_);
+                    const float2 F3a = __fmul2_rn(make_float2(cs[0], cs[1]), F3a_),
+                                 F3b = __fmul2_rn(make_float2(cs[2], cs[3]), F3b_);
                     uint32_t mq = 0u, mk = 0u;
                     float2 E[8][2], Rr[2];
-                    decay_suffix(a, po, (lane >> 4) != 0, E, Rr);
+                    {
+                        const float one4[4] = {1.f, 1.f, 1.f, 1.f};
+                        decay_suffix(a, one4, false, E, Rr);
+                    }
+                    Rr[0] = make_float2(r0p[0], r0p[1]);
+                    Rr[1] = make_float2(r0p[2], r0p[3]);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const int r = r0 + i;
@@ -1164,8 +1202,8 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         st_tile2(sm, AP_B + quad_off(160u, (uint32_t)r0, i, (uint32_t)c0),
                                  pack_bf16v(__fmul2_rn(kE01, invB01)), pack_bf16v(__fmul2_rn(kE23, invB23)));
                         if (eI <= 2)
-                            st_tile2(sm, AP_B + quad_off(160u, 64u + (uint32_t)r0, i, (uint32_t)c0), pack_bf16v(kE01),
-                                     pack_bf16v(kE23));
+                            st_tile2(sm, AP_B + quad_off(160u, 64u + (uint32_t)r0, i, (uint32_t)c0),
+                                     pack_bf16v(__fmul2_rn(kE01, F1a)), pack_bf16v(__fmul2_rn(kE23, F1b)));
                         if (eI <= 1)
                             st_tile2(sm, AP_B + quad_off(160u, 112u + (uint32_t)r0, i, (uint32_t)c0),
                                      pack_bf16v(__fmul2_rn(kE01, F2a)), pack_bf16v(__fmul2_rn(kE23, F2b)));

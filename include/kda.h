@@ -118,9 +118,10 @@ kda_status kda_fwd(const void* q, const void* k, const void* v,
                    void* out, float* final_state,
                    kda_dims dims, kda_stream_t stream);
 
-/* Gates at or above this clamp keep every factored intra-chunk decay of the
- * fused kernel inside the fp32/bf16 exponent range (16 tokens x 5.3 = 84.8 < 87). */
-#define KDA_FUSED_MIN_LOWER_BOUND (-5.3f)
+/* Gates at or above this clamp keep every factored intra-chunk decay of the fused kernel inside
+ * the fp32/bf16 exponent range: its factors span at most 8 tokens of decay around the middle of a
+ * 16-token block, e^{8 x 9.5} = e^76, and |k| e^76 < 3.4e38 for |k| < 2^15. */
+#define KDA_FUSED_MIN_LOWER_BOUND (-9.5f)
 
 /*
  * kda_fwd_staged -- the same forward as four separate kernels with intermediates in a

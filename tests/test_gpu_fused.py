@@ -1,5 +1,5 @@
 """GPU parity of the product path kda_fwd (the fused tcgen05 kernel for
-lower_bound >= -5.3) against the fp64 recurrent oracle."""
+lower_bound >= -9.5) against the fp64 recurrent oracle."""
 import numpy as np
 import pytest
 import torch
@@ -35,7 +35,9 @@ SMALL = [
     ("partial_chunk", W.custom([37], H=2, packed=False, init="normal")),
     ("varlen_ragged", W.custom([70, 0, 129, 64, 1, 200, 17], H=3, init="normal")),
     ("many_heads", W.custom([300], H=20, packed=False, init=None)),
-    ("lb_at_limit", W.custom([190], H=2, packed=False, init="normal", lower_bound=-5.3)),
+    ("lb_5_3", W.custom([190], H=2, packed=False, init="normal", lower_bound=-5.3)),
+    ("lb_steep_7", W.custom([190, 70], H=2, init="normal", lower_bound=-7.0)),
+    ("lb_at_limit_9_5", W.custom([190], H=3, packed=False, init="normal", lower_bound=-9.5)),
     ("lb_mild", W.custom([190], H=2, packed=False, init="normal", lower_bound=-1.0)),
 ]
 

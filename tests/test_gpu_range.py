@@ -135,6 +135,24 @@ def test_range_state_grows_then_decays():
     assert e_st <= STATE_REL_L2, f"state rel-L2 {e_st:.3e}"
 
 
+def test_steep_gate_with_large_keys():
+    """The steepest clamp the fused kernel takes (-9.5) with entries of q and k up to ~50 (|q . k|
+    still below 2^15) and most gates at the clamp: every decayed operand stays finite (factors are
+    taken around the middle of each 16-token block), and the result matches the oracle."""
+    kda = _kda()
+    w = W.custom([300, 90], H=2, init="normal", lower_bound=-9.5, wid=49)
+    x = _unnormalised(W.make_inputs(w), 13)
+    x["k"] = (x["k"].float() * 10.0).to(torch.bfloat16)
+    x["q"] = (x["q"].float() * 10.0).to(torch.bfloat16)
+    kn2 = x["k"].float().pow(2).sum(-1)
+    x["beta"] = (torch.rand(kn2.shape, generator=torch.Generator("cpu").manual_seed(17)) * 1.9 / kn2).contiguous()
+    x["g"] = x["g"] + 3.0       # softplus(g + dt_bias) large: log a at the clamp for most tokens
+    out, fin = _run(kda, x)
+    assert kda.kda_check_device_error() == 0
+    ref_o, ref_f = run_oracle(x)
+    _check(out, fin, ref_o, ref_f, "steep gate, large keys")
+
+
 def test_out_of_range_keys_are_flagged_not_inf():
     """Keys far outside the operating range (|k| ~ 1e5): the kernel saturates instead of
     producing inf or NaN, and reports KDA_DEVERR_RANGE."""
