@@ -81,7 +81,7 @@ constexpr uint32_t S_ORDER = MISC + 4096;      // int16 [kSortLimit]
 constexpr int kSortLimit = 512;
 constexpr uint32_t S_META = S_ORDER + 2 * kSortLimit;   // int32 [2][8] chunk metadata
 constexpr uint32_t S_BARS = S_META + 64;                // u64 [16]
-constexpr int kNumBars = 9;
+constexpr int kNumBars = 10;
 constexpr uint32_t S_TMEM = S_BARS + 128;               // u32 tmem base, u32 abort flag
 constexpr uint32_t S_PH = S_TMEM + 16;                  // u64 [kPhases + 3] (phase-clock builds)
 constexpr int kPhases = 24;
@@ -385,7 +385,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 // a[i][e] = a_t for token r0 + i, channel c0 + e: a = max(2^(-e^A_log * log2(1 + 2^x2)), e^lb)
 // with x2 = (g + dt_bias) log2 e, i.e. e^(-e^A_log softplus(g + dt_bias)) clamped at e^lb.
 // Rows past the chunk's valid length get a = 1.
-__device__ __forceinline__ void gate_tokens(const Params& p, int h, int64_t t0, int L, int c0, int r0,
+// gs: the chunk's raw gate input, fp32 [64 tokens][128 channels] in shared memory (a TMA box)
+__device__ __forceinline__ void gate_tokens(const Params& p, int h, const float* gs, int L, int c0, int r0,
                                             float (&a)[8][4]) {
     const float nexpA = -expf(p.A_log[h]);
     const float alb = fast_ex2(p.lower_bound * kLog2e);
@@ -394,12 +395,7 @@ __device__ __forceinline__ void gate_tokens(const Params& p, int h, int64_t t0, 
     const float2 l2e = make_float2(kLog2e, kLog2e);
     float4 gv[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int r = r0 + i;
-        gv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < L)
-            gv[i] = __ldg(reinterpret_cast<const float4*>(p.g + ((t0 + r) * p.H + h) * kHeadDim + c0));
-    }
+    for (int i = 0; i < 8; ++i) gv[i] = *reinterpret_cast<const float4*>(gs + (r0 + i) * kHeadDim + c0);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const float2 x01 = __ffma2_rn(make_float2(gv[i].x, gv[i].y), l2e, db01);
@@ -600,7 +596,7 @@ __device__ __forceinline__ void issue_chunk_loads_s(unsigned char* sm, uint64_t*
 template <bool kScalar>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                 const Params p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -624,6 +620,7 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t* bar_s = bar_in + 6;        // [S | O] MMA done (chunk's shared operands free again)
     uint64_t* bar_apready = bar_in + 7;  // chunk's A/P operand tiles written (the chain issues the MMA)
     uint64_t* bar_ro = bar_in + 8;       // chunk's A/P product read out of TMEM (the accumulator is free)
+    uint64_t* bar_g = bar_in + 9;        // channel gate: chunk's raw gate input landed (TMA, in the A/P tiles)
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + S_TMEM);
     volatile uint32_t* sAbort = sTmem + 1;
 #ifdef KDA_PHASE_CLOCKS
@@ -1042,12 +1039,24 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, c.h, c.t0);
         };
 
+        // channel gate: chunk c's raw gate input into the A/P operand region (free between a chunk's
+        // A/P MMA and the next chunk's operand tiles); the element warps read it for the gate
+        bool g_pending = false;
+        uint32_t g_parity = 0;
+        auto load_gate_input = [&](const Cursor& c, uint32_t parity) {
+            mbar_arrive_expect_tx(bar_g, 32768u);
+            tma_load_2d(sm + AP_A, &tm_g, c.h * kHeadDim, (int)c.t0, bar_g);
+            g_pending = true;
+            g_parity = parity;
+        };
+
         Cursor cur = unit_from(p, sOrder, b, G, units, 0);
         uint32_t ci = 0;
         if (loader && cur.valid) {
             load_inputs(cur);
             tma_pending = true;
             tma_parity = 0;
+            if constexpr (!kScalar) load_gate_input(cur, 0);
         }
         if (!is_aux) {
             // ======================= element warps =======================
@@ -1073,7 +1082,8 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if constexpr (kScalar) {
                     if (warp == kElemWarp0) load_g_scalar(cur);
                 } else {
-                    gate_tokens(p, cur.h, cur.t0, chunk_len(cur), c0, r0, a);
+                    if (!warp_wait(bar_g, 0u)) *sAbort = 1u;
+                    gate_tokens(p, cur.h, reinterpret_cast<const float*>(sm + AP_A), chunk_len(cur), c0, r0, a);
                 }
             }
             while (cur.valid) {
@@ -1082,18 +1092,12 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const int L = chunk_len(cur);
                 const uint32_t sl = ci & 1u;
                 bool bad = false;
-                // the next chunk's gate input into L2
-                if (nxt.valid) {
-                    const int L1 = chunk_len(nxt);
-                    if constexpr (kScalar) {
-                        if (warp == kElemWarp0) {
-                            if (2 * lane < L1) prefetch_l2(p.g + (nxt.t0 + 2 * lane) * H + nxt.h);
-                            if (2 * lane + 1 < L1) prefetch_l2(p.g + (nxt.t0 + 2 * lane + 1) * H + nxt.h);
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            if (r0 + i < L1) prefetch_l2(p.g + ((nxt.t0 + r0 + i) * H + nxt.h) * kHeadDim + c0);
+                // scalar gate: the next chunk's gate input into L2 (the channel gate's comes by TMA)
+                if constexpr (kScalar) {
+                    if (nxt.valid && warp == kElemWarp0) {
+                        const int L1 = chunk_len(nxt);
+                        if (2 * lane < L1) prefetch_l2(p.g + (nxt.t0 + 2 * lane) * H + nxt.h);
+                        if (2 * lane + 1 < L1) prefetch_l2(p.g + (nxt.t0 + 2 * lane + 1) * H + nxt.h);
                     }
                 }
                 // ================ E0: beta; block products of a / the scalar gate's scan ================
@@ -1344,7 +1348,8 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if constexpr (kScalar) {
                         if (warp == kElemWarp0) load_g_scalar(nxt);
                     } else {
-                        gate_tokens(p, nxt.h, nxt.t0, chunk_len(nxt), c0, r0, a);
+                        if (!warp_wait(bar_g, (ci + 1u) & 1u)) *sAbort = 1u;
+                        gate_tokens(p, nxt.h, reinterpret_cast<const float*>(sm + AP_A), chunk_len(nxt), c0, r0, a);
                     }
                 }
                 PIPE_MARK(256, 2, 23);
@@ -1570,6 +1575,18 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (ci > 0) bad |= !warp_wait(bar_s, (ci - 1) & 1u);   // the chain is done with the last V^T
                 bad |= !warp_wait(bar_in, ci & 1u);
                 tma_pending = false;
+                // channel gate: the next chunk's gate input, once this chunk's A/P MMA has read the
+                // operand tiles it lands in
+                if constexpr (!kScalar) {
+                    if (loader && nxt.valid) {
+                        if (mbar_wait_bounded(bar_ap, ci & 1u)) {
+                            load_gate_input(nxt, (ci + 1u) & 1u);
+                        } else {
+                            record_error(KDA_DEVERR_TIMEOUT);
+                            *sAbort = 1u;
+                        }
+                    }
+                }
                 PIPE_MARK(128, 0, 4);
                 {
                     // V^T: thread -> value columns 2 vp and 2 vp + 1, tokens 32 th .. 32 th + 31
@@ -1652,6 +1669,7 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (aborted) {
                 *sAbort = 1u;
                 if (loader && tma_pending) mbar_wait_bounded(bar_in, tma_parity);
+                if (loader && g_pending) mbar_wait_bounded(bar_g, g_parity);
             }
         }
         if (range_bad) record_error(KDA_DEVERR_RANGE);
@@ -1719,7 +1737,7 @@ cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
     if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
     if ((err = cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
     if (sm_count <= 0) return cudaErrorInvalidDevice;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, tg;
     const int64_t rows = a.total_tokens, cols = (int64_t)a.H * kHeadDim;
     // channel-wise gate: 128-channel unswizzled boxes (CUDA cores read them); scalar gate:
     // 64-channel 128-byte-swizzled boxes (the MMA reads them)
@@ -1728,6 +1746,11 @@ cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
         !make_map(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box, kScalar) ||
         !make_map(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box, kScalar))
         return cudaErrorInvalidValue;
+    if (kScalar) {
+        tg = tq;   // unused: the scalar gate input is read with plain loads
+    } else if (!make_map(&tg, a.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols)) {
+        return cudaErrorInvalidValue;
+    }
     Params p;
     p.g = a.g;
     p.beta = a.beta;
@@ -1746,7 +1769,7 @@ cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
     const int64_t units = (int64_t)a.N * a.H;
     const int grid = (int)(units < sm_count ? units : sm_count);
     if (grid <= 0) return cudaSuccess;
-    kda_pipe_kernel<kScalar><<<grid, kThreads, SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+    kda_pipe_kernel<kScalar><<<grid, kThreads, SMEM_ALLOC, stream>>>(tq, tk, tv, tg, p);
     return cudaGetLastError();
 }
 
