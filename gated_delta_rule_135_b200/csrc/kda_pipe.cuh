@@ -16,11 +16,12 @@
 //                         U^T        = Y^T T^T                                             K = 64
 //                         U^T -> fp16 (TMEM);  [S | O]^T += U^T [Khat | P^T]              N = 192
 //                         O^T -> bf16 out (times scale 2^sigma_v)
-//   element warps 8-15  chunk n: beta, gate and decay factors (thread: 4 channels x 8 tokens)
-//                       and every decayed operand tile
+//   element warps 8-15  chunk n: beta, gate and decay factors (thread: 4 channels x 8 tokens),
+//                       every decayed operand tile and the chunk's metadata (scalar gate: V^T)
 //   aux warps 4-7       meanwhile chunk n - 1: the A / P read-out (one warp per TMEM lane
-//                       quarter) and T = (I + A)^-1; then chunk n's V^T, the exact diagonal
-//                       q_r . k_r of P, its metadata, and the TMA loads of chunk n + 1
+//                       quarter) and T = (I + A)^-1; chunk n's V^T and exact P diagonal q_r . k_r
+//                       (channel gate), and the TMA load of chunk n + 1's gate input
+//   (the chain's thread 0 also issues the A/P MMA and the TMA loads of the next chunk's q, k, v)
 //
 // Y = beta V - beta gamma K S and U = T Y is the WY/UT form U = T diag(beta)(V - (gamma K) S)
 // of the chunk (U~ - W S with the product by T taken last), so that the part of the chain that
@@ -53,10 +54,9 @@ namespace pipe {
 using namespace umma;
 
 constexpr int kThreads = 512;
-constexpr int kFeThreads = 384;          // warps 4-15
 constexpr int kAuxWarp0 = 4, kElemWarp0 = 8;
 // named barriers (0 is __syncthreads)
-constexpr uint32_t BAR_FE = 1, BAR_CHAIN = 2, BAR_AUX = 3, BAR_ELEM = 4;
+constexpr uint32_t BAR_CHAIN = 2, BAR_AUX = 3, BAR_ELEM = 4;
 
 // ---- shared memory (bytes from a 1024-aligned base) ----
 constexpr uint32_t IN_Q = 0;           // bf16 [64][128] row-major TMA boxes
@@ -75,14 +75,12 @@ constexpr uint32_t MISC = 204800;
 constexpr uint32_t S_BETA = MISC;              // fp32 [2][64] (by chunk parity)
 constexpr uint32_t S_GC = MISC + 512;          // fp32 [2][128] gamma_C = e^{Gamma_63}
 constexpr uint32_t S_PTOT = MISC + 1536;       // fp32 [4][128] per-block products of a
-constexpr uint32_t S_PD = MISC + 3584;         // fp32 [2][64] halves of q_r . k_r (of the chunk the aux
-                                               // warps formed last)
 constexpr uint32_t S_ORDER = MISC + 4096;      // int16 [kSortLimit]
 constexpr int kSortLimit = 512;
-constexpr uint32_t S_META = S_ORDER + 2 * kSortLimit;   // int32 [2][8] chunk metadata
-constexpr uint32_t S_BARS = S_META + 64;                // u64 [16]
-constexpr int kNumBars = 10;
-constexpr uint32_t S_TMEM = S_BARS + 128;               // u32 tmem base, u32 abort flag
+constexpr uint32_t S_META = S_ORDER + 2 * kSortLimit;   // int32 [2][16] chunk metadata
+constexpr uint32_t S_BARS = S_META + 128;               // u64 [16]
+constexpr int kNumBars = 11;
+constexpr uint32_t S_TMEM = S_BARS + 128;               // u32 tmem base, abort flag, read-out data sequence
 constexpr uint32_t S_PH = S_TMEM + 16;                  // u64 [kPhases + 3] (phase-clock builds)
 constexpr int kPhases = 24;
 // The triangular solve's scratch, apart from the A/P operand tiles (which the element warps
@@ -100,9 +98,10 @@ constexpr uint32_t SV_SC = SV_AL + 6 * kHBlk;           // fp16 [8][16][24] inte
 constexpr uint32_t SC_Y0 = SV_SC, SC_Y2 = SV_SC + kHBlk, SC_T10B = SV_SC + 2 * kHBlk, SC_X20 = SV_SC + 3 * kHBlk,
                    SC_X30 = SV_SC + 4 * kHBlk, SC_X21 = SV_SC + 5 * kHBlk, SC_X31 = SV_SC + 6 * kHBlk,
                    SC_Y32 = SV_SC + 7 * kHBlk;
-constexpr uint32_t SMEM_BYTES = SV_SC + 8 * kHBlk;
+constexpr uint32_t S_PD2 = SV_SC + 8 * kHBlk;          // fp32 [2][2][64] halves of q_r . k_r, by chunk parity
+constexpr uint32_t SMEM_BYTES = S_PD2 + 1024;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
-static_assert(S_PH + 8 * (kPhases + 3) <= SV, "phase slots below the solve scratch");
+static_assert(S_PH + 8 * (kPhases + 3) <= S_PHALF, "phase slots below the half-block products");
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
 // ---- TMEM columns ----
@@ -271,6 +270,25 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
     const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
     if (!ok && (threadIdx.x & 31) == 0) record_error(KDA_DEVERR_TIMEOUT);
     return ok;
+}
+
+// A monotonic sequence number in shared memory (a counter cannot skip a phase the way an mbarrier
+// parity can): the writer publishes with a release store after a barrier over the producing threads,
+// the reader waits for a value with acquire loads, at most limit_ns.
+__device__ __forceinline__ void seq_publish(uint32_t* seq, uint32_t v) {
+    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(seq)), "r"(v) : "memory");
+}
+__device__ __forceinline__ bool seq_wait(const uint32_t* seq, uint32_t target, uint64_t limit_ns = 1000000000ull) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(seq)) : "memory");
+    if (v >= target) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        __nanosleep(100);
+        asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(seq)) : "memory");
+        if (v >= target) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
 }
 
 // ---- 16 x 16 fp16 block products of the triangular solve (mma.sync m16n8k16, fp32 accumulation) ----
@@ -621,8 +639,10 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t* bar_apready = bar_in + 7;  // chunk's A/P operand tiles written (the chain issues the MMA)
     uint64_t* bar_ro = bar_in + 8;       // chunk's A/P product read out of TMEM (the accumulator is free)
     uint64_t* bar_g = bar_in + 9;        // channel gate: chunk's raw gate input landed (TMA, in the A/P tiles)
+    uint64_t* bar_vt = bar_in + 10;      // channel gate: chunk's V^T and P diagonal formed (aux warps)
     uint32_t* sTmem = reinterpret_cast<uint32_t*>(sm + S_TMEM);
     volatile uint32_t* sAbort = sTmem + 1;
+    uint32_t* sRdSeq = sTmem + 2;   // chunks whose beta, P diagonal (and scalar Gamma) the element warps published
 #ifdef KDA_PHASE_CLOCKS
     volatile unsigned long long* sPh = reinterpret_cast<volatile unsigned long long*>(sm + S_PH);
 #endif
@@ -632,6 +652,7 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int i = 0; i < kNumBars; ++i) mbar_init(bar_in + i, 1);
         mbar_init_fence();
         *sAbort = 0u;
+        *sRdSeq = 0u;
     }
     if (warp == 0) {
         tmem_alloc(sTmem, TM_COLS);
@@ -691,6 +712,8 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         int prev_h = 0, prev_n = 0, prev_L = 0, prev_last = 0;
         int64_t prev_t0 = 0;
         uint32_t issued_y = 0, issued_u = 0, issued_s = 0, done_s = 0, issued_ap = 0;   // thread 0's MMA commits
+        bool in_pending = false;   // thread 0: input loads issued (drained on abort)
+        uint32_t in_parity = 0;
         bool aborted = false;
 
         // O^T (TMEM) of the previous chunk -> out, and its final state if it ended a unit.  Lane v
@@ -796,10 +819,28 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!more) break;
             PIPE_MARK(0, 1, 12);
             bad |= !warp_wait(bar_formed, cc & 1u);
-            const int32_t* meta = sMeta + (cc & 1u) * 8u;
+            const int32_t* meta = sMeta + (cc & 1u) * 16u;
             const int m_h = meta[1], m_n = meta[2], m_t0 = meta[3], m_L = meta[4], m_first = meta[5],
                       m_last = meta[6];
             more = meta[7] != 0;
+            // channel gate: the aux warps' V^T (they read this chunk's inputs for it and for P's diagonal)
+            if constexpr (!kScalar) bad |= !warp_wait(bar_vt, cc & 1u);
+            // the next chunk's q, k, v: the element (and aux) warps are done with this chunk's input
+            // tiles (and, for the scalar gate, the A/P MMA that reads them has completed)
+            if (tid == 0 && more && !bad) {
+                const bool ok = !kScalar || mbar_wait_bounded(bar_ap, cc & 1u);
+                if (ok) {
+                    if constexpr (kScalar)
+                        issue_chunk_loads_s(sm, bar_in, &tm_q, &tm_k, &tm_v, meta[8], meta[9]);
+                    else
+                        issue_chunk_loads(sm, bar_in, &tm_q, &tm_k, &tm_v, meta[8], meta[9]);
+                    in_pending = true;
+                    in_parity = (cc + 1u) & 1u;
+                } else {
+                    record_error(KDA_DEVERR_TIMEOUT);
+                    *sAbort = 1u;
+                }
+            }
             if (named_bar_or(BAR_CHAIN, 128, bad || *sAbort != 0u)) {
                 aborted = true;
                 break;
@@ -1007,14 +1048,17 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (issued_u > 0) mbar_wait_bounded(bar_u, (issued_u - 1) & 1u);
             if (issued_s > done_s) mbar_wait_bounded(bar_s, (issued_s - 1) & 1u);
             if (issued_ap > 0) mbar_wait_bounded(bar_ap, (issued_ap - 1) & 1u);
+            if (in_pending) mbar_wait_bounded(bar_in, in_parity);
         }
         if (aborted && tid == 0) *sAbort = 1u;
     } else {
         // =============================== front end ===============================
         // Element warps 8-15 build chunk n (gate, decay factors, the A/P operand tiles, the chain's
         // operand tiles) while aux warps 4-7 read out the A/P product of chunk n - 1 and solve
-        // T = (I + A)^-1 for it, then form chunk n's V^T and P diagonal.  The two groups meet once per
-        // chunk (BAR_FE), after both have written chunk n's chain operands.
+        // T = (I + A)^-1 for it (and, for the channel gate, form V^T and P's exact diagonal).  The
+        // two groups share no barrier: they meet through mbarriers (A/P operands ready, A/P product
+        // done, read-out done, the chain's [S | O] MMA done) and a published sequence number, so the
+        // aux warps take a chunk as soon as its product lands.
         const bool is_aux = warp < kElemWarp0;
         const int at = tid - 128;           // aux thread (warps 4-7)
         const int et = tid - 256;           // element thread (warps 8-15)
@@ -1223,8 +1267,12 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     named_bar_sync(BAR_ELEM, 256);
                 }
                 PIPE_MARK(256, 2, 20);
-                // the A/P operands are ready: the chain issues the MMA
-                if (elead) mbar_arrive(bar_apready);
+                // the A/P operands are ready (the chain issues the MMA), and so are the chunk's beta,
+                // P diagonal and scalar Gamma, which the aux warps read (published after the barrier)
+                if (elead) {
+                    seq_publish(sRdSeq, ci + 1u);
+                    mbar_arrive(bar_apready);
+                }
                 // ================ E4: the chain's operands (once it is done with the last chunk's) ================
                 if (ci > 0) bad |= !warp_wait(bar_s, (ci - 1) & 1u);
                 PIPE_MARK(256, 2, 21);
@@ -1334,13 +1382,55 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             make_float4(gc[0], gc[1], gc[2], gc[3]);
                     }
                 }
+                if constexpr (kScalar) {
+                    // V^T (bf16 [128 v][64 i], 128-byte rows, 16-byte chunk j at j ^ (v & 7)): thread ->
+                    // value columns 2 vp and 2 vp + 1, tokens 16 tq .. 16 tq + 15 (the channel gate's
+                    // aux warps form it, with P's diagonal)
+                    const int vp = et & 63, tq = et >> 6;
+                    const uint32_t v0 = 2u * (uint32_t)vp, v1 = v0 + 1u;
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        uint32_t w[8];
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) {
+                            const int r = 16 * tq + 8 * j + t;
+                            uint32_t voff;
+                            if constexpr (kScalar)   // 64-channel swizzled blocks: element (r, v0) of block v0 / 64
+                                voff = (v0 >> 6) * 8192u + (uint32_t)r * 128u +
+                                       ((((v0 & 63u) >> 3) ^ ((uint32_t)r & 7u)) << 4) + (v0 & 7u) * 2u;
+                            else
+                                voff = (uint32_t)r * 256u + (uint32_t)vp * 4u;
+                            w[t] = r < L ? *reinterpret_cast<const uint32_t*>(sm + IN_V + voff) : 0u;
+                        }
+                        const uint32_t ch = (uint32_t)(2 * tq + j);
+                        st_tile4(sm, VT + v0 * 128u + ((ch ^ (v0 & 7u)) << 4), __byte_perm(w[0], w[1], 0x5410),
+                                 __byte_perm(w[2], w[3], 0x5410), __byte_perm(w[4], w[5], 0x5410),
+                                 __byte_perm(w[6], w[7], 0x5410));
+                        st_tile4(sm, VT + v1 * 128u + ((ch ^ (v1 & 7u)) << 4), __byte_perm(w[0], w[1], 0x7632),
+                                 __byte_perm(w[2], w[3], 0x7632), __byte_perm(w[4], w[5], 0x7632),
+                                 __byte_perm(w[6], w[7], 0x7632));
+                    }
+                }
+                if (elead) {
+                    int32_t* meta = sMeta + sl * 16u;
+                    meta[0] = 1;
+                    meta[1] = cur.h;
+                    meta[2] = cur.n;
+                    meta[3] = (int32_t)cur.t0;
+                    meta[4] = L;
+                    meta[5] = cur.t0 == cur.bos ? 1 : 0;
+                    meta[6] = cur.t0 + kChunk >= cur.eos ? 1 : 0;
+                    meta[7] = nxt.valid ? 1 : 0;   // another chunk follows in this CTA
+                    meta[8] = nxt.h;
+                    meta[9] = (int32_t)nxt.t0;
+                }
                 fence_proxy_async();
-                if (named_bar_or(BAR_FE, kFeThreads, bad || *sAbort != 0u)) {
+                if (named_bar_or(BAR_ELEM, 256, bad || *sAbort != 0u)) {
                     aborted = true;
                     break;
                 }
                 PIPE_MARK(256, 2, 22);
-                // hand the chunk to the chain
+                // hand the chunk to the chain (which then loads the next chunk's inputs over these)
                 if (elead) mbar_arrive(bar_formed);
                 // ================ E6: the next chunk's beta and gate ================
                 if (nxt.valid) {
@@ -1359,12 +1449,11 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (aborted) *sAbort = 1u;
         } else {
             // ======================= aux warps =======================
-            // Iteration k: the read-out and solve of chunk k - 1, then chunk k's V^T, P diagonal and
-            // metadata.  One more iteration after the last chunk solves that chunk.
+            // For each chunk: once its A/P MMA is done, the next chunk's gate input (channel gate);
+            // then the A / P read-out (once the chain is done with the last chunk's P and T) and the
+            // solve.
             const int sw = warp - kAuxWarp0;
             float tmax = 0.f;
-            Cursor next_in;         // the chunk whose inputs the next TMA loads bring (scalar gate)
-            next_in.valid = false;
             // sign * (a 16 x 16 warp-MMA accumulator) into block (I, J) of the fp16 T tile
             auto acc_to_t16 = [&](int I, int J, const float (&acc)[2][4], float sign) {
                 const int g = lane >> 2, t = lane & 3;
@@ -1379,290 +1468,254 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         pack_f16s(sign * acc[nh][2], sign * acc[nh][3]);
                 }
             };
-            while (true) {
-                bool bad = false;
-                if (ci > 0) {
-                    const uint32_t cj = ci - 1, slp = cj & 1u;
-                    // ================ A0: A / P read-out of chunk cj (one warp per TMEM lane quarter) ================
-                    const bool ap_done = warp_wait(bar_ap, cj & 1u);
-                    if (!ap_done) *sAbort = 1u;
-                    if constexpr (kScalar) {
-                        if (loader && ap_done && next_in.valid) {
-                            load_inputs(next_in);
-                            tma_pending = true;
-                            tma_parity = ci & 1u;
-                        }
-                    }
-                    fence_after_sync();
-                    PIPE_MARK(128, 0, 0);
-                    const bool isA = quarter < 2;
-                    const int r = (quarter & 1) * 32 + lane;      // token row of A (k rows) or P (q rows)
-                    const int I = r >> 4;
-                    const float be = reinterpret_cast<const float*>(sm + S_BETA)[slp * 64u + r];
-                    float pdg = 0.f;
-                    if constexpr (!kScalar)
-                        pdg = reinterpret_cast<const float*>(sm + S_PD)[r] + reinterpret_cast<const float*>(sm + S_PD)[64 + r];
-                    float pmax = 0.f;
-#pragma unroll 1
-                    for (int J = 0; J < 4; ++J) {
-                        float row[16];
-                        auto pick = [&](uint32_t col_a, uint32_t col_b, int I_a) {
-                            uint32_t ta[16], tb[16];
-                            tmem_ld16(taddr(tbase, quarter, TM_AP + col_a), ta);
-                            tmem_ld16(taddr(tbase, quarter, TM_AP + col_b), tb);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int x = 0; x < 16; ++x) row[x] = __uint_as_float(I == I_a ? ta[x] : tb[x]);
-                        };
-                        if constexpr (kScalar) {
-                            // raw K K^T / Q K^T times the scalar decay 2^(Gamma_r - Gamma_i) (<= 1 on
-                            // and below the diagonal)
-                            uint32_t raw[16];
-                            tmem_ld16(taddr(tbase, quarter, TM_AP + (uint32_t)J * 16u), raw);
-                            tmem_wait_ld();
-                            const float* gam = reinterpret_cast<const float*>(sm + s_gam(slp));
-                            const float gr = gam[r];
-#pragma unroll
-                            for (int x = 0; x < 16; ++x) {
-                                const int i = J * 16 + x;
-                                const bool keep = isA ? (i < r) : (i <= r);
-                                row[x] = keep ? __uint_as_float(raw[x]) * fast_ex2(gr - gam[i]) : 0.f;
-                            }
-                        } else {
-                            if ((quarter & 1) == 0) {        // I in {0, 1}
-                                if (J == 0) pick(0, 64, 0);            // I=0: diagonal; I=1: C1 of block 0
-                                else if (J == 1) pick(16, 16, 1);      // I=1: diagonal (I=0: masked)
-                                else {
-#pragma unroll
-                                    for (int x = 0; x < 16; ++x) row[x] = 0.f;
-                                }
-                            } else {                         // I in {2, 3}
-                                if (J == 0) pick(112, 144, 2);         // I=2: C2 of block 0; I=3: C3 of block 0
-                                else if (J == 1) pick(80, 128, 2);     // I=2: C1 of block 1; I=3: C2 of block 1
-                                else if (J == 2) pick(32, 96, 2);      // I=2: diagonal; I=3: C1 of block 2
-                                else pick(48, 48, 3);                  // I=3: diagonal (I=2: masked)
-                            }
-#pragma unroll
-                            for (int x = 0; x < 16; ++x) {
-                                const int i = J * 16 + x;
-                                row[x] = i < r ? row[x] : ((i == r && !isA) ? pdg : 0.f);
-                            }
-                        }
-                        if (isA) {
-                            // beta-scaled A: diagonal blocks in fp32 (the forward substitution), the
-                            // blocks below in fp16 (operands of the block products)
-                            if (J == I) {
-                                float* ad = reinterpret_cast<float*>(sm + SV_AD) + (I * 16 + (r & 15)) * kAdPitch;
-#pragma unroll
-                                for (int x = 0; x < 16; x += 4)
-                                    *reinterpret_cast<float4*>(ad + x) =
-                                        make_float4(be * row[x], be * row[x + 1], be * row[x + 2], be * row[x + 3]);
-                            } else if (J < I) {
-                                uint32_t hv[8];
-#pragma unroll
-                                for (int x = 0; x < 8; ++x) hv[x] = warpmma::pack_half2(be * row[2 * x], be * row[2 * x + 1]);
-                                const uint32_t off = al_off(I, J) + (uint32_t)(r & 15) * kHp * 2u;
-                                st_v4(sm, off, hv[0], hv[1], hv[2], hv[3]);
-                                st_v4(sm, off + 16u, hv[4], hv[5], hv[6], hv[7]);
-                            }
-                        } else {
-                            // P^T (MN-major, K = token i, N = row r): 16-bit stores, a warp writes 64
-                            // contiguous bytes per i
-#pragma unroll
-                            for (int x = 0; x < 16; ++x) {
-                                const int i = J * 16 + x;
-                                pmax = fmaxf(pmax, fabsf(row[x]));
-                                st_tile_h(sm, PT + sw128_off((uint32_t)i, (uint32_t)r, 64u),
-                                          __half_as_ushort(__float2half_rn(fminf(fmaxf(row[x], -65504.f), 65504.f))));
-                            }
-                        }
-                    }
-                    if (pmax >= kRangeHi) range_bad = 1u;
-                    fence_proxy_async();
-                    tmem_wait_ld();
-                    fence_before_sync();
-                    named_bar_sync(BAR_AUX, 128);
-                    // the accumulator is free for the next chunk's A/P MMA
-                    if (at == 0) mbar_arrive(bar_ro);
-                    PIPE_MARK(128, 0, 1);
-                    // ================ A1: T = (I + A)^-1 of chunk cj ================
-                    // L0: the four 16 x 16 diagonal blocks by forward substitution in fp32, one column
-                    // per thread (threads 0-63), right-looking; written to the fp16 T tile
-                    if (sw < 2) {
-                        const int bI = at >> 4, jc = at & 15, o = bI * 16;
-                        const float* ad = reinterpret_cast<const float*>(sm + SV_AD) + bI * 16 * kAdPitch;
-                        float x[16];
-#pragma unroll
-                        for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == jc) ? 1.f : 0.f;
-#pragma unroll
-                        for (int ii = 0; ii < 15; ++ii) {
-                            const float xi = x[ii];
-#pragma unroll
-                            for (int rr = ii + 1; rr < 16; ++rr) x[rr] = fmaf(-ad[rr * kAdPitch + ii], xi, x[rr]);
-                        }
-#pragma unroll
-                        for (int rr = 0; rr < 16; ++rr) {
-                            tmax = fmaxf(tmax, fabsf(x[rr]));
-                            st_tile_h(sm, T16 + sw128_off((uint32_t)(o + rr), (uint32_t)(o + jc), 64u),
-                                      __half_as_ushort(__float2half_rn(fminf(fmaxf(x[rr], -65504.f), 65504.f))));
-                        }
-                    }
-                    named_bar_sync(BAR_AUX, 128);
-                    PIPE_MARK(128, 0, 2);
-                    // L1 (16 x 16 warp-MMA products, fp16 operands, fp32 accumulation):
-                    //   T10 = -T11 (A10 T00), T32 = -T33 (A32 T22),
-                    //   X20 = A20 T00 + A21 T10, X30 = A30 T00 + A31 T10, X21 = A21 T11, X31 = A31 T11.
-                    // Aux warps 0 and 2 both form T10 (warp 2 in its own scratch) so that neither waits
-                    // for the other.
-                    {
-                        float acc[2][4] = {};
-                        if (sw == 0 || sw == 2) {
-                            const uint32_t ysc = sw == 0 ? SC_Y0 : SC_Y2;
-                            mm16h(acc, lm_blk(sm, al_off(1, 0)), lm_t16(sm, 0, 0));       // A10 T00
-                            store16h(sm, ysc, acc, 1.f);
-                            __syncwarp();
-                            float a2[2][4] = {};
-                            mm16h(a2, lm_t16(sm, 1, 1), lm_blk(sm, ysc));                 // T10
-                            if (sw == 0) acc_to_t16(1, 0, a2, -1.f);
-                            else store16h(sm, SC_T10B, a2, -1.f);
-                            __syncwarp();
-                            const int I = sw == 0 ? 2 : 3;
-                            float a3[2][4] = {};
-                            mm16h(a3, lm_blk(sm, al_off(I, 0)), lm_t16(sm, 0, 0));
-                            mm16h(a3, lm_blk(sm, al_off(I, 1)), sw == 0 ? lm_t16(sm, 1, 0) : lm_blk(sm, SC_T10B));
-                            store16h(sm, sw == 0 ? SC_X20 : SC_X30, a3, 1.f);             // X20 / X30
-                        } else if (sw == 1) {
-                            mm16h(acc, lm_blk(sm, al_off(3, 2)), lm_t16(sm, 2, 2));       // A32 T22
-                            store16h(sm, SC_Y32, acc, 1.f);
-                            __syncwarp();
-                            float a2[2][4] = {};
-                            mm16h(a2, lm_t16(sm, 3, 3), lm_blk(sm, SC_Y32));
-                            acc_to_t16(3, 2, a2, -1.f);                                   // T32
-                            float a3[2][4] = {};
-                            mm16h(a3, lm_blk(sm, al_off(2, 1)), lm_t16(sm, 1, 1));
-                            store16h(sm, SC_X21, a3, 1.f);                                // X21
-                        } else {
-                            mm16h(acc, lm_blk(sm, al_off(3, 1)), lm_t16(sm, 1, 1));
-                            store16h(sm, SC_X31, acc, 1.f);                               // X31
-                        }
-                    }
-                    named_bar_sync(BAR_AUX, 128);
-                    // L2: T_LL = -T_LR X, written straight to the fp16 tile:
-                    //   T20 = -T22 X20, T21 = -T22 X21, T30 = -(T32 X20 + T33 X30), T31 = -(T32 X21 + T33 X31)
-                    {
-                        float acc[2][4] = {};
-                        const int J = sw & 1;
-                        if (sw < 2) {
-                            mm16h(acc, lm_t16(sm, 2, 2), lm_blk(sm, J == 0 ? SC_X20 : SC_X21));
-                            acc_to_t16(2, J, acc, -1.f);
-                        } else {
-                            mm16h(acc, lm_t16(sm, 3, 2), lm_blk(sm, J == 0 ? SC_X20 : SC_X21));
-                            mm16h(acc, lm_t16(sm, 3, 3), lm_blk(sm, J == 0 ? SC_X30 : SC_X31));
-                            acc_to_t16(3, J, acc, -1.f);
-                        }
-                    }
-                    if (tmax >= kRangeHi) range_bad = 1u;
-                    fence_proxy_async();
-                    named_bar_sync(BAR_AUX, 128);
-                    if (at == 0) mbar_arrive(bar_t);
-                    PIPE_MARK(128, 0, 3);
-                }
-                if (!cur.valid) break;
+            while (cur.valid) {
                 const Cursor nxt = next_chunk(p, sOrder, b, G, units, cur);
-                const int L = chunk_len(cur);
-                const uint32_t sl = ci & 1u;
-                // ================ A4: V^T, P diagonal and metadata of chunk ci ================
-                if (ci > 0) bad |= !warp_wait(bar_s, (ci - 1) & 1u);   // the chain is done with the last V^T
-                bad |= !warp_wait(bar_in, ci & 1u);
-                tma_pending = false;
-                // channel gate: the next chunk's gate input, once this chunk's A/P MMA has read the
-                // operand tiles it lands in
+                const uint32_t cj = ci, slp = cj & 1u;
+                bool bad = false;
+                // the chain is done with the last chunk's V^T, P^T and T (its [S | O] MMA has completed)
+                if (cj > 0) bad |= !warp_wait(bar_s, (cj - 1u) & 1u);
                 if constexpr (!kScalar) {
-                    if (loader && nxt.valid) {
-                        if (mbar_wait_bounded(bar_ap, ci & 1u)) {
-                            load_gate_input(nxt, (ci + 1u) & 1u);
-                        } else {
-                            record_error(KDA_DEVERR_TIMEOUT);
-                            *sAbort = 1u;
+                    // ================ A-1: V^T and P's exact diagonal of chunk cj ================
+                    const int L = chunk_len(cur);
+                    bad |= !warp_wait(bar_in, cj & 1u);
+                    {
+                        // V^T: thread -> value columns 2 vp and 2 vp + 1, tokens 32 th .. 32 th + 31
+                        const int vp = at & 63, th = at >> 6;
+                        const uint32_t v0 = 2u * (uint32_t)vp, v1 = v0 + 1u;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint32_t w[8];
+#pragma unroll
+                            for (int t = 0; t < 8; ++t) {
+                                const int r = 32 * th + 8 * j + t;
+                                w[t] = r < L ? *reinterpret_cast<const uint32_t*>(sm + IN_V + (uint32_t)r * 256u + (uint32_t)vp * 4u)
+                                             : 0u;
+                            }
+                            const uint32_t ch = (uint32_t)(4 * th + j);
+                            st_tile4(sm, VT + v0 * 128u + ((ch ^ (v0 & 7u)) << 4), __byte_perm(w[0], w[1], 0x5410),
+                                     __byte_perm(w[2], w[3], 0x5410), __byte_perm(w[4], w[5], 0x5410),
+                                     __byte_perm(w[6], w[7], 0x5410));
+                            st_tile4(sm, VT + v1 * 128u + ((ch ^ (v1 & 7u)) << 4), __byte_perm(w[0], w[1], 0x7632),
+                                     __byte_perm(w[2], w[3], 0x7632), __byte_perm(w[4], w[5], 0x7632),
+                                     __byte_perm(w[6], w[7], 0x7632));
                         }
                     }
-                }
-                PIPE_MARK(128, 0, 4);
-                {
-                    // V^T: thread -> value columns 2 vp and 2 vp + 1, tokens 32 th .. 32 th + 31
-                    const int vp = at & 63, th = at >> 6;
-                    const uint32_t v0 = 2u * (uint32_t)vp, v1 = v0 + 1u;
+                    {
+                        // q_r . k_r in fp32 over one 64-channel half; 16-byte chunks visited in a
+                        // row-dependent order (conflict-free)
+                        const int r = at & 63, hh = at >> 6;
+                        float pd = 0.f;
+                        if (r < L) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t w[8];
+                            for (int j = 0; j < 8; ++j) {
+                                const uint32_t off = (uint32_t)r * 256u + (uint32_t)hh * 128u + (((uint32_t)(j + r) & 7u) << 4);
+                                const uint4 qv = *reinterpret_cast<const uint4*>(sm + IN_Q + off);
+                                const uint4 kv = *reinterpret_cast<const uint4*>(sm + IN_K + off);
+                                const uint32_t qa[4] = {qv.x, qv.y, qv.z, qv.w}, ka[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-                        for (int t = 0; t < 8; ++t) {
-                            const int r = 32 * th + 8 * j + t;
-                            uint32_t voff;
-                            if constexpr (kScalar)   // 64-channel swizzled blocks: element (r, v0) of block v0 / 64
-                                voff = (v0 >> 6) * 8192u + (uint32_t)r * 128u +
-                                       ((((v0 & 63u) >> 3) ^ ((uint32_t)r & 7u)) << 4) + (v0 & 7u) * 2u;
-                            else
-                                voff = (uint32_t)r * 256u + (uint32_t)vp * 4u;
-                            w[t] = r < L ? *reinterpret_cast<const uint32_t*>(sm + IN_V + voff) : 0u;
-                        }
-                        const uint32_t ch = (uint32_t)(4 * th + j);
-                        st_tile4(sm, VT + v0 * 128u + ((ch ^ (v0 & 7u)) << 4), __byte_perm(w[0], w[1], 0x5410),
-                              __byte_perm(w[2], w[3], 0x5410), __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
-                        st_tile4(sm, VT + v1 * 128u + ((ch ^ (v1 & 7u)) << 4), __byte_perm(w[0], w[1], 0x7632),
-                              __byte_perm(w[2], w[3], 0x7632), __byte_perm(w[4], w[5], 0x7632), __byte_perm(w[6], w[7], 0x7632));
-                    }
-                }
-                if constexpr (!kScalar) {
-                    // q_r . k_r in fp32 over one 64-channel half; 16-byte chunks visited in a
-                    // row-dependent order (conflict-free)
-                    const int r = at & 63, hh = at >> 6;
-                    float pd = 0.f;
-                    if (r < L) {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const uint32_t off = (uint32_t)r * 256u + (uint32_t)hh * 128u + (((uint32_t)(j + r) & 7u) << 4);
-                            const uint4 qv = *reinterpret_cast<const uint4*>(sm + IN_Q + off);
-                            const uint4 kv = *reinterpret_cast<const uint4*>(sm + IN_K + off);
-                            const uint32_t qa[4] = {qv.x, qv.y, qv.z, qv.w}, ka[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 a2 = bf16x2_to_float2(qa[e]), b2 = bf16x2_to_float2(ka[e]);
-                                pd = fmaf(a2.x, b2.x, pd);
-                                pd = fmaf(a2.y, b2.y, pd);
+                                for (int e = 0; e < 4; ++e) {
+                                    const float2 a2 = bf16x2_to_float2(qa[e]), b2 = bf16x2_to_float2(ka[e]);
+                                    pd = fmaf(a2.x, b2.x, pd);
+                                    pd = fmaf(a2.y, b2.y, pd);
+                                }
                             }
                         }
+                        reinterpret_cast<float*>(sm + S_PD2)[(slp * 2u + (uint32_t)hh) * 64u + r] = pd;
                     }
-                    reinterpret_cast<float*>(sm + S_PD)[hh * 64 + r] = pd;
+                    fence_proxy_async();
+                    named_bar_sync(BAR_AUX, 128);
+                    if (at == 0) mbar_arrive(bar_vt);
                 }
-                if (at == 0) {
-                    int32_t* meta = sMeta + sl * 8u;
-                    meta[0] = 1;
-                    meta[1] = cur.h;
-                    meta[2] = cur.n;
-                    meta[3] = (int32_t)cur.t0;
-                    meta[4] = L;
-                    meta[5] = cur.t0 == cur.bos ? 1 : 0;
-                    meta[6] = cur.t0 + kChunk >= cur.eos ? 1 : 0;
-                    meta[7] = nxt.valid ? 1 : 0;   // another chunk follows in this CTA
+                // ================ A0: wait for the chunk's A/P product ================
+                bad |= !warp_wait(bar_ap, cj & 1u);
+                // channel gate: the next chunk's gate input into the operand tiles the MMA has read
+                if constexpr (!kScalar) {
+                    if (loader && nxt.valid && !bad) load_gate_input(nxt, (cj + 1u) & 1u);
                 }
+                // the element warps have published the chunk's beta (and scalar Gamma)
+                bad |= !__all_sync(0xffffffffu, seq_wait(sRdSeq, cj + 1u));
+                if (bad) *sAbort = 1u;
+                fence_after_sync();
+                PIPE_MARK(128, 0, 0);
+                const bool isA = quarter < 2;
+                const int r = (quarter & 1) * 32 + lane;      // token row of A (k rows) or P (q rows)
+                const int I = r >> 4;
+                const float be = reinterpret_cast<const float*>(sm + S_BETA)[slp * 64u + r];
+                float pdg = 0.f;
+                if constexpr (!kScalar) {
+                    const float* pd = reinterpret_cast<const float*>(sm + S_PD2) + slp * 128u;
+                    pdg = pd[r] + pd[64 + r];
+                }
+                float pmax = 0.f;
+#pragma unroll 1
+                for (int J = 0; J < 4; ++J) {
+                    float row[16];
+                    auto pick = [&](uint32_t col_a, uint32_t col_b, int I_a) {
+                        uint32_t ta[16], tb[16];
+                        tmem_ld16(taddr(tbase, quarter, TM_AP + col_a), ta);
+                        tmem_ld16(taddr(tbase, quarter, TM_AP + col_b), tb);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) row[x] = __uint_as_float(I == I_a ? ta[x] : tb[x]);
+                    };
+                    if constexpr (kScalar) {
+                        // raw K K^T / Q K^T times the scalar decay 2^(Gamma_r - Gamma_i) (<= 1 on
+                        // and below the diagonal)
+                        uint32_t raw[16];
+                        tmem_ld16(taddr(tbase, quarter, TM_AP + (uint32_t)J * 16u), raw);
+                        tmem_wait_ld();
+                        const float* gam = reinterpret_cast<const float*>(sm + s_gam(slp));
+                        const float gr = gam[r];
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            const int i = J * 16 + x;
+                            const bool keep = isA ? (i < r) : (i <= r);
+                            row[x] = keep ? __uint_as_float(raw[x]) * fast_ex2(gr - gam[i]) : 0.f;
+                        }
+                    } else {
+                        if ((quarter & 1) == 0) {        // I in {0, 1}
+                            if (J == 0) pick(0, 64, 0);            // I=0: diagonal; I=1: C1 of block 0
+                            else if (J == 1) pick(16, 16, 1);      // I=1: diagonal (I=0: masked)
+                            else {
+#pragma unroll
+                                for (int x = 0; x < 16; ++x) row[x] = 0.f;
+                            }
+                        } else {                         // I in {2, 3}
+                            if (J == 0) pick(112, 144, 2);         // I=2: C2 of block 0; I=3: C3 of block 0
+                            else if (J == 1) pick(80, 128, 2);     // I=2: C1 of block 1; I=3: C2 of block 1
+                            else if (J == 2) pick(32, 96, 2);      // I=2: diagonal; I=3: C1 of block 2
+                            else pick(48, 48, 3);                  // I=3: diagonal (I=2: masked)
+                        }
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            const int i = J * 16 + x;
+                            row[x] = i < r ? row[x] : ((i == r && !isA) ? pdg : 0.f);
+                        }
+                    }
+                    if (isA) {
+                        // beta-scaled A: diagonal blocks in fp32 (the forward substitution), the
+                        // blocks below in fp16 (operands of the block products)
+                        if (J == I) {
+                            float* ad = reinterpret_cast<float*>(sm + SV_AD) + (I * 16 + (r & 15)) * kAdPitch;
+#pragma unroll
+                            for (int x = 0; x < 16; x += 4)
+                                *reinterpret_cast<float4*>(ad + x) =
+                                    make_float4(be * row[x], be * row[x + 1], be * row[x + 2], be * row[x + 3]);
+                        } else if (J < I) {
+                            uint32_t hv[8];
+#pragma unroll
+                            for (int x = 0; x < 8; ++x) hv[x] = warpmma::pack_half2(be * row[2 * x], be * row[2 * x + 1]);
+                            const uint32_t off = al_off(I, J) + (uint32_t)(r & 15) * kHp * 2u;
+                            st_v4(sm, off, hv[0], hv[1], hv[2], hv[3]);
+                            st_v4(sm, off + 16u, hv[4], hv[5], hv[6], hv[7]);
+                        }
+                    } else {
+                        // P^T (MN-major, K = token i, N = row r): 16-bit stores, a warp writes 64
+                        // contiguous bytes per i
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            const int i = J * 16 + x;
+                            pmax = fmaxf(pmax, fabsf(row[x]));
+                            st_tile_h(sm, PT + sw128_off((uint32_t)i, (uint32_t)r, 64u),
+                                      __half_as_ushort(__float2half_rn(fminf(fmaxf(row[x], -65504.f), 65504.f))));
+                        }
+                    }
+                }
+                if (pmax >= kRangeHi) range_bad = 1u;
                 fence_proxy_async();
-                PIPE_MARK(128, 0, 5);
-                if (named_bar_or(BAR_FE, kFeThreads, bad || *sAbort != 0u)) {
+                tmem_wait_ld();
+                fence_before_sync();
+                named_bar_sync(BAR_AUX, 128);
+                // the accumulator is free for the next chunk's A/P MMA
+                if (at == 0) mbar_arrive(bar_ro);
+                PIPE_MARK(128, 0, 1);
+                // ================ A1: T = (I + A)^-1 of chunk cj ================
+                // L0: the four 16 x 16 diagonal blocks by forward substitution in fp32, one column
+                // per thread (threads 0-63), right-looking; written to the fp16 T tile
+                if (sw < 2) {
+                    const int bI = at >> 4, jc = at & 15, o = bI * 16;
+                    const float* ad = reinterpret_cast<const float*>(sm + SV_AD) + bI * 16 * kAdPitch;
+                    float x[16];
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == jc) ? 1.f : 0.f;
+#pragma unroll
+                    for (int ii = 0; ii < 15; ++ii) {
+                        const float xi = x[ii];
+#pragma unroll
+                        for (int rr = ii + 1; rr < 16; ++rr) x[rr] = fmaf(-ad[rr * kAdPitch + ii], xi, x[rr]);
+                    }
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) {
+                        tmax = fmaxf(tmax, fabsf(x[rr]));
+                        st_tile_h(sm, T16 + sw128_off((uint32_t)(o + rr), (uint32_t)(o + jc), 64u),
+                                  __half_as_ushort(__float2half_rn(fminf(fmaxf(x[rr], -65504.f), 65504.f))));
+                    }
+                }
+                named_bar_sync(BAR_AUX, 128);
+                PIPE_MARK(128, 0, 2);
+                // L1 (16 x 16 warp-MMA products, fp16 operands, fp32 accumulation):
+                //   T10 = -T11 (A10 T00), T32 = -T33 (A32 T22),
+                //   X20 = A20 T00 + A21 T10, X30 = A30 T00 + A31 T10, X21 = A21 T11, X31 = A31 T11.
+                // Aux warps 0 and 2 both form T10 (warp 2 in its own scratch) so that neither waits
+                // for the other.
+                {
+                    float acc[2][4] = {};
+                    if (sw == 0 || sw == 2) {
+                        const uint32_t ysc = sw == 0 ? SC_Y0 : SC_Y2;
+                        mm16h(acc, lm_blk(sm, al_off(1, 0)), lm_t16(sm, 0, 0));       // A10 T00
+                        store16h(sm, ysc, acc, 1.f);
+                        __syncwarp();
+                        float a2[2][4] = {};
+                        mm16h(a2, lm_t16(sm, 1, 1), lm_blk(sm, ysc));                 // T10
+                        if (sw == 0) acc_to_t16(1, 0, a2, -1.f);
+                        else store16h(sm, SC_T10B, a2, -1.f);
+                        __syncwarp();
+                        const int I = sw == 0 ? 2 : 3;
+                        float a3[2][4] = {};
+                        mm16h(a3, lm_blk(sm, al_off(I, 0)), lm_t16(sm, 0, 0));
+                        mm16h(a3, lm_blk(sm, al_off(I, 1)), sw == 0 ? lm_t16(sm, 1, 0) : lm_blk(sm, SC_T10B));
+                        store16h(sm, sw == 0 ? SC_X20 : SC_X30, a3, 1.f);             // X20 / X30
+                    } else if (sw == 1) {
+                        mm16h(acc, lm_blk(sm, al_off(3, 2)), lm_t16(sm, 2, 2));       // A32 T22
+                        store16h(sm, SC_Y32, acc, 1.f);
+                        __syncwarp();
+                        float a2[2][4] = {};
+                        mm16h(a2, lm_t16(sm, 3, 3), lm_blk(sm, SC_Y32));
+                        acc_to_t16(3, 2, a2, -1.f);                                   // T32
+                        float a3[2][4] = {};
+                        mm16h(a3, lm_blk(sm, al_off(2, 1)), lm_t16(sm, 1, 1));
+                        store16h(sm, SC_X21, a3, 1.f);                                // X21
+                    } else {
+                        mm16h(acc, lm_blk(sm, al_off(3, 1)), lm_t16(sm, 1, 1));
+                        store16h(sm, SC_X31, acc, 1.f);                               // X31
+                    }
+                }
+                named_bar_sync(BAR_AUX, 128);
+                // L2: T_LL = -T_LR X, written straight to the fp16 tile:
+                //   T20 = -T22 X20, T21 = -T22 X21, T30 = -(T32 X20 + T33 X30), T31 = -(T32 X21 + T33 X31)
+                {
+                    float acc[2][4] = {};
+                    const int J = sw & 1;
+                    if (sw < 2) {
+                        mm16h(acc, lm_t16(sm, 2, 2), lm_blk(sm, J == 0 ? SC_X20 : SC_X21));
+                        acc_to_t16(2, J, acc, -1.f);
+                    } else {
+                        mm16h(acc, lm_t16(sm, 3, 2), lm_blk(sm, J == 0 ? SC_X20 : SC_X21));
+                        mm16h(acc, lm_t16(sm, 3, 3), lm_blk(sm, J == 0 ? SC_X30 : SC_X31));
+                        acc_to_t16(3, J, acc, -1.f);
+                    }
+                }
+                if (tmax >= kRangeHi) range_bad = 1u;
+                fence_proxy_async();
+                named_bar_sync(BAR_AUX, 128);
+                if (at == 0) mbar_arrive(bar_t);
+                PIPE_MARK(128, 0, 3);
+                PIPE_MARK(128, 0, 4);
+                if (named_bar_or(BAR_AUX, 128, *sAbort != 0u)) {
                     aborted = true;
                     break;
                 }
-                PIPE_MARK(128, 0, 6);
-                // the next chunk's inputs: the current ones are consumed (for the scalar gate the A/P
-                // MMA reads them too, so the loads wait for it at the start of the next read-out)
-                if constexpr (!kScalar) {
-                    if (loader && nxt.valid) {
-                        load_inputs(nxt);
-                        tma_pending = true;
-                        tma_parity = (ci + 1u) & 1u;
-                    }
-                }
-                next_in = nxt;
+                PIPE_MARK(128, 0, 5);
                 cur = nxt;
                 ++ci;
             }

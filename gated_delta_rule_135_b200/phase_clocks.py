@@ -24,30 +24,30 @@ _ROOT = os.path.dirname(_HERE)
 # index = slot of the kernel's phase marks; each counts the cycles since the previous mark
 # of the same role
 PHASES = [
-    ("aux", "wait for the A/P product of chunk n-1"),
-    ("aux", "A / P read-out of chunk n-1"),
+    ("aux", "wait for A/P product, last [S|O], chunk data"),
+    ("aux", "A / P read-out"),
     ("aux", "solve L0 (diagonal blocks)"),
     ("aux", "solve L1 + L2, T written"),
-    ("aux", "wait for the last [S|O] MMA and the inputs"),
-    ("aux", "V^T, P diagonal, metadata of chunk n"),
-    ("aux", "meet the element warps"),
+    ("-", "(unused)"),
+    ("aux", "meet the other aux warps"),
+    ("-", "(unused)"),
     ("-", "(unused)"),
     ("-", "(unused)"),
     ("chain", "wait for the previous [S|O] MMA"),
     ("chain", "output of the previous chunk"),
     ("chain", "wait for A/P operands and read-out, issue"),
     ("chain", "(between marks)"),
-    ("chain", "wait for the chunk's operands"),
+    ("chain", "wait for the chunk's operands, next TMA"),
     ("chain", "S^T -> fp16, [O|Y] MMA, S <- S Diag(gamma_C)"),
     ("chain", "wait [O|Y], Y^T += beta V^T -> fp16"),
     ("chain", "wait T, U MMA, wait U"),
     ("chain", "U -> fp16, [S|O] MMA issue"),
     ("elem", "beta, block products / gate scan"),
     ("elem", "wait for the inputs and the last A/P MMA"),
-    ("elem", "A/P operand tiles"),
+    ("elem", "A/P operand tiles, P diagonal"),
     ("elem", "wait for the last [S|O] MMA"),
-    ("elem", "B1, Khat tiles, meet the aux warps"),
-    ("elem", "next chunk: TMA, beta, gate"),
+    ("elem", "B1, Khat, V^T tiles, metadata"),
+    ("elem", "next chunk: beta, gate"),
 ]
 
 
