@@ -63,8 +63,10 @@ constexpr uint32_t IN_Q = 0;           // bf16 [64][128] row-major TMA boxes
 constexpr uint32_t IN_K = 16384;
 constexpr uint32_t IN_V = 32768;
 constexpr uint32_t IN_BYTES = 49152;
-constexpr uint32_t AP_A = 49152;       // bf16 K-major [128 rows][128]: k R rows 0-63, q R rows 64-127
-constexpr uint32_t AP_B = 81920;       // bf16 K-major [160 rows][128]: XD | C1 | C2 | C3
+constexpr uint32_t AP_A = 49152;       // bf16 K-major [128 rows][128]: k R' rows 0-63, q R' rows 64-127
+                                       // (between a chunk's A/P MMA and the next chunk's tiles: the
+                                       // next chunk's raw gate input, fp32 [64][128])
+constexpr uint32_t AP_B = 81920;       // bf16 K-major [160 rows][128]: k E' | C1 | C2 | C3
 constexpr uint32_t B1 = 122880;        // fp16 K-major [128 rows][128]: gamma q rows 0-63, -beta gamma k 64-127
 constexpr uint32_t B2 = 155648;        // fp16 MN-major, K = 64 tokens: Khat (c 0-63 | c 64-127) | P^T
 constexpr uint32_t KH = B2;
@@ -225,9 +227,6 @@ __device__ __forceinline__ uint32_t quad_off(uint32_t rows, uint32_t rowbase, in
            ((c0 & 7u) << 1);
 }
 
-__device__ __forceinline__ void st_v2(unsigned char* base, uint32_t off, uint32_t a, uint32_t b) {
-    *reinterpret_cast<uint2*>(base + off) = make_uint2(a, b);
-}
 // Shared-memory stores the compiler may move later shared loads above: the operand tiles
 // written in one phase are never read back in it (the phase ends with a fence and a barrier,
 // which order them before every later use).
