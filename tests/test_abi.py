@@ -40,6 +40,14 @@ def test_library_exports_every_declared_symbol():
     assert declared <= set(kda.EXPORTED) | declared
 
 
+def test_binding_fused_bound_matches_header():
+    """The binding's fused-kernel clamp bound (used to label bench lines) is the header's."""
+    text = open(os.path.join(ROOT, "include", "kda.h")).read()
+    m = re.search(r"#define\s+KDA_FUSED_MIN_LOWER_BOUND\s+\(?\s*(-?[0-9.]+)f?\s*\)?", text)
+    assert m, "KDA_FUSED_MIN_LOWER_BOUND not found in include/kda.h"
+    assert float(m.group(1)) == kda.FUSED_MIN_LOWER_BOUND
+
+
 def test_strerror_covers_every_status():
     for code, name in kda.STATUS_NAMES.items():
         assert kda.kda_strerror(code).startswith(name)
