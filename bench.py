@@ -617,6 +617,10 @@ def main():
     stream = torch.cuda.current_stream()
     fused = args.gdn or x["lower_bound"] >= kda.FUSED_MIN_LOWER_BOUND
     launches_per_step = 1 if fused else 5
+    # one long sequence in the fixed layout: the library splits it into segments itself
+    lib_segments = (kda.kda_fwd_segments(w.H, w.T) if fused and w.N == 1 and x["cu_seqlens"] is None else 1)
+    if lib_segments > 1:
+        launches_per_step = lib_segments + 3   # segment offsets, two map passes, R - 1 folds, final pass
     fwd = kda.kda_gdn_fwd if args.gdn else kda.kda_fwd
     seg_ws = {}
     if args.segments:
@@ -670,10 +674,13 @@ def main():
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak,
             "traffic": (dram_traffic_from_profile("kda_pipe_kernel<scalar gate>" if args.gdn else "kda_pipe_kernel",
-                                                  w.T * w.H) if fused and not args.segments else None),
+                                                  w.T * w.H)
+                        if fused and not args.segments and lib_segments == 1 else None),
             "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
             else "fallback 6650 GB/s",
             "kernel": (f"segmented prefill ({args.segments} segments: 3 fused launches + folds)" if args.segments
+                       else (f"{fwd.__name__} split into {lib_segments} segments by the library (3 fused launches "
+                             f"+ folds)") if lib_segments > 1
                        else ("kda_pipe_kernel<scalar gate>" if args.gdn else "kda_pipe_kernel") if fused
                        else "staged kernels"),
             "kernel_ms": kernel_ms, "algorithmic_bytes": alg_bytes,

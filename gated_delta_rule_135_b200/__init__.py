@@ -96,6 +96,8 @@ def _load():
     lib.kda_decode.argtypes = [vp] * 7 + [f32, f32, vp, vp, ctypes.c_int32, ctypes.c_int32, vp]
     lib.kda_selftest_wait_timeout.restype = ctypes.c_int
     lib.kda_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp, vp]
+    lib.kda_fwd_segments.restype = ctypes.c_int32
+    lib.kda_fwd_segments.argtypes = [kda_dims, ctypes.c_int32]
     return lib
 
 
@@ -107,7 +109,7 @@ EXPORTED = ("kda_fwd", "kda_fwd_staged", "kda_staged_workspace_size",
             "kda_last_device_error_bits", "kda_version", "kda_fwd_staged_noalloc",
             "kda_noalloc_scratch_bytes", "kda_decode", "kda_gdn_fwd", "kda_gdn_decode",
             "kda_state_affine", "kda_bwd", "kda_bwd_workspace_size", "kda_fwd_workspace_size",
-            "kda_selftest_wait_timeout")
+            "kda_selftest_wait_timeout", "kda_fwd_segments")
 
 
 def lib() -> ctypes.CDLL:
@@ -389,6 +391,14 @@ def kda_bwd_workspace_size(q: torch.Tensor, cu_seqlens: Optional[torch.Tensor] =
         batch = q.shape[0]
     dims = make_dims(H, total_tokens=total, cu_seqlens=cu_seqlens, batch=batch)
     return int(_lib.kda_bwd_workspace_size(dims, int(cu_seqlens is not None)))
+
+
+def kda_fwd_segments(num_heads: int, seqlen: int, batch: int = 1, varlen: bool = False) -> int:
+    """How many segments kda_fwd / kda_gdn_fwd split a call with these dims into on the current
+    device (1: none; only one sequence in the fixed layout is split)."""
+    dims = make_dims(num_heads, total_tokens=seqlen * batch, batch=batch, seqlen=seqlen) if not varlen else \
+        make_dims(num_heads, total_tokens=seqlen, cu_seqlens=torch.zeros(2, dtype=torch.int32))
+    return int(_lib.kda_fwd_segments(dims, 1 if varlen else 0))
 
 
 def kda_selftest_wait_timeout(limit_ns: int, observed: Optional[torch.Tensor] = None, stream=None) -> None:

@@ -207,6 +207,87 @@ kda_status kda_fwd_staged(const void* q, const void* k, const void* v, const flo
                                                                                      : KDA_ERR_CUDA;
 }
 
+namespace {
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+// Segments for a fused-forward call: one sequence in the fixed layout (its boundaries are known
+// on the host) whose heads leave SMs idle.
+int segments_for(const StagedArgs& a, bool varlen) {
+    if (varlen || a.N != 1) return 1;
+    return kda::choose_segments(a.total_tokens, a.H, sm_count());
+}
+
+// One long sequence as R segments run together (the context-parallel decomposition on one GPU):
+// (1) every segment from S = I with v = 0 gives its A map, (2) from S = 0 its B map, (3) the
+// maps fold into each segment's starting state, S_r = A_{r-1} S_{r-1} + B_{r-1}, and (4) every
+// segment runs from its state and writes the output.  Workspace (stream-ordered): the segment
+// offsets and three [R][H][128][128] fp32 state arrays.
+cudaError_t launch_segmented(const StagedArgs& a, int R, bool gdn, cudaStream_t s) {
+    auto fused = [&](const StagedArgs& x) { return gdn ? kda::launch_pipe_gdn(x, s) : kda::launch_pipe(x, s); };
+    const int64_t T = a.total_tokens;
+    const size_t per_seg = (size_t)a.H * kda::kHeadDim * kda::kHeadDim;   // floats
+    const size_t map_bytes = (size_t)R * per_seg * sizeof(float);
+    char* ws = nullptr;
+    cudaError_t err = cudaMallocAsync(reinterpret_cast<void**>(&ws), 256 + 3 * map_bytes, s);
+    if (err != cudaSuccess) return err;
+    int32_t* cu = reinterpret_cast<int32_t*>(ws);
+    float* A = reinterpret_cast<float*>(ws + 256);
+    float* B = A + (size_t)R * per_seg;
+    float* S = B + (size_t)R * per_seg;
+    kda::cp::segment_offsets_kernel<<<1, 64, 0, s>>>(cu, R, kda::cp::segment_step(T, R), T);
+    err = cudaGetLastError();
+    StagedArgs m = a;
+    m.cu_seqlens = cu;
+    m.N = R;
+    m.seqlen = T;
+    m.out = nullptr;
+    m.initial_state = nullptr;
+    if (err == cudaSuccess) {   // A maps
+        m.flags = kda::kFlagVZero | kda::kFlagInitIdentity;
+        m.final_state = A;
+        err = fused(m);
+    }
+    if (err == cudaSuccess) {   // B maps
+        m.flags = 0;
+        m.final_state = B;
+        err = fused(m);
+    }
+    const size_t st_bytes = per_seg * sizeof(float);
+    if (err == cudaSuccess)
+        err = a.initial_state ? cudaMemcpyAsync(S, a.initial_state, st_bytes, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(S, 0, st_bytes, s);
+    for (int r = 1; r < R && err == cudaSuccess; ++r)
+        err = kda::launch_state_affine(A + (size_t)(r - 1) * per_seg, S + (size_t)(r - 1) * per_seg,
+                                       B + (size_t)(r - 1) * per_seg, S + (size_t)r * per_seg, a.H, s);
+    if (err == cudaSuccess) {   // every segment from its state; its final states over the B maps
+        StagedArgs f = a;
+        f.cu_seqlens = cu;
+        f.N = R;
+        f.seqlen = T;
+        f.initial_state = S;
+        f.final_state = B;
+        err = fused(f);
+    }
+    if (err == cudaSuccess && a.final_state)
+        err = cudaMemcpyAsync(a.final_state, B + (size_t)(R - 1) * per_seg, st_bytes, cudaMemcpyDeviceToDevice, s);
+    const cudaError_t err2 = cudaFreeAsync(ws, s);
+    return err != cudaSuccess ? err : err2;
+}
+
+}  // namespace
+
+int32_t kda_fwd_segments(kda_dims dims, int32_t varlen) {
+    if (dims.num_heads < 1 || dims.seqlen < 0) return 1;
+    if (varlen || dims.batch != 1) return 1;
+    return kda::choose_segments(dims.seqlen, dims.num_heads, sm_count());
+}
+
 kda_status kda_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
                    const float* A_log, const float* dt_bias, float lower_bound, float scale,
                    const float* initial_state, const int32_t* cu_seqlens, void* out,
@@ -217,8 +298,11 @@ kda_status kda_fwd(const void* q, const void* k, const void* v, const float* g, 
     if (st != KDA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (a.total_tokens == 0) return copy_states_only(a, s);
-    if (kda::fused_supported(lower_bound))
-        return kda::launch_pipe(a, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    if (kda::fused_supported(lower_bound)) {
+        const int R = segments_for(a, cu_seqlens != nullptr);
+        const cudaError_t err = R > 1 ? launch_segmented(a, R, false, s) : kda::launch_pipe(a, s);
+        return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
     kda::StagedLayout L = kda::staged_layout(a.total_tokens, a.H, a.N);
     void* ws = nullptr;
     if (cudaMallocAsync(&ws, L.total, s) != cudaSuccess) return KDA_ERR_CUDA;
@@ -237,7 +321,9 @@ kda_status kda_gdn_fwd(const void* q, const void* k, const void* v, const float*
     if (st != KDA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (a.total_tokens == 0) return copy_states_only(a, s);
-    return kda::launch_pipe_gdn(a, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    const int R = segments_for(a, cu_seqlens != nullptr);
+    const cudaError_t err = R > 1 ? launch_segmented(a, R, true, s) : kda::launch_pipe_gdn(a, s);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 namespace {

@@ -25,6 +25,10 @@ cudaError_t once_per_device(F setup) {
     return err;
 }
 
+// StagedArgs::flags of the fused forward (the segment maps of one long sequence)
+constexpr uint32_t kFlagVZero = 1u;          // treat v as zero
+constexpr uint32_t kFlagInitIdentity = 2u;   // start every sequence from S = I (initial_state NULL)
+
 struct StagedArgs {
     const void* q;
     const void* k;
@@ -44,6 +48,7 @@ struct StagedArgs {
     int H;
     int N;                 // number of sequences
     float* t_mat;          // optional: T = (I + A)^-1 of every chunk, [max_chunks][H][64][64]
+    uint32_t flags;        // fused forward only: kFlagVZero | kFlagInitIdentity; out may then be NULL
 };
 
 struct StagedLayout {

@@ -150,6 +150,7 @@ struct Params {
     int64_t total_tokens;
     int H;
     int N;
+    uint32_t flags;   // kFlagVZero, kFlagInitIdentity (the segment maps of one long sequence)
 };
 
 #ifdef KDA_PHASE_CLOCKS
@@ -689,9 +690,16 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             decode_unit(p, sOrder, u, &n, &h, &bos, &eos);
             if (eos > bos) continue;
             const int64_t off = ((int64_t)n * H + h) * kHeadDim * kHeadDim;
+            const bool ident = (p.flags & kFlagInitIdentity) != 0;
             for (int e = tid; e < kHeadDim * kHeadDim / 4; e += kThreads) {
-                const float4 s = p.initial_state ? reinterpret_cast<const float4*>(p.initial_state + off)[e]
-                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                const int row = (4 * e) / kHeadDim, col = (4 * e) % kHeadDim;
+                float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (p.initial_state) {
+                    s = reinterpret_cast<const float4*>(p.initial_state + off)[e];
+                } else if (ident) {
+                    s = make_float4(row == col ? 1.f : 0.f, row == col + 1 ? 1.f : 0.f, row == col + 2 ? 1.f : 0.f,
+                                    row == col + 3 ? 1.f : 0.f);
+                }
                 reinterpret_cast<float4*>(p.final_state + off)[e] = s;
             }
         }
@@ -725,7 +733,7 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int64_t row_stride = (int64_t)H * kHeadDim;
             __nv_bfloat16* base = p.out + (prev_t0 * H + prev_h) * kHeadDim + (v & ~1) + (odd ? row_stride : 0);
 #pragma unroll 1
-            for (int cb = 0; cb < 2; ++cb) {
+            for (int cb = 0; cb < (p.out ? 2 : 0); ++cb) {   // no output: a segment-map pass
                 uint32_t o[32];
                 tmem_ld32(lane_base + TM_O + 32u * cb, o);
                 tmem_wait_ld();
@@ -850,11 +858,14 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 sigma = 0;
                 const float* is = p.initial_state
                     ? p.initial_state + ((int64_t)m_n * H + m_h) * kHeadDim * kHeadDim + v : nullptr;
+                const bool ident = (p.flags & kFlagInitIdentity) != 0;
 #pragma unroll 1
                 for (int cb = 0; cb < 4; ++cb) {
                     uint32_t s[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) s[j] = is ? __float_as_uint(is[(32 * cb + j) * kHeadDim]) : 0u;
+                    for (int j = 0; j < 32; ++j)
+                        s[j] = is ? __float_as_uint(is[(32 * cb + j) * kHeadDim])
+                                  : ((ident && 32 * cb + j == v) ? 0x3f800000u : 0u);
                     tmem_st32(lane_base + TM_S + 32u * cb, s);
                 }
                 tmem_wait_st();
@@ -1399,7 +1410,8 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                        ((((v0 & 63u) >> 3) ^ ((uint32_t)r & 7u)) << 4) + (v0 & 7u) * 2u;
                             else
                                 voff = (uint32_t)r * 256u + (uint32_t)vp * 4u;
-                            w[t] = r < L ? *reinterpret_cast<const uint32_t*>(sm + IN_V + voff) : 0u;
+                            w[t] = (r < L && !(p.flags & kFlagVZero)) ? *reinterpret_cast<const uint32_t*>(sm + IN_V + voff)
+                                                                      : 0u;
                         }
                         const uint32_t ch = (uint32_t)(2 * tq + j);
                         st_tile4(sm, VT + v0 * 128u + ((ch ^ (v0 & 7u)) << 4), __byte_perm(w[0], w[1], 0x5410),
@@ -1487,8 +1499,9 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                             for (int t = 0; t < 8; ++t) {
                                 const int r = 32 * th + 8 * j + t;
-                                w[t] = r < L ? *reinterpret_cast<const uint32_t*>(sm + IN_V + (uint32_t)r * 256u + (uint32_t)vp * 4u)
-                                             : 0u;
+                                w[t] = (r < L && !(p.flags & kFlagVZero))
+                                           ? *reinterpret_cast<const uint32_t*>(sm + IN_V + (uint32_t)r * 256u + (uint32_t)vp * 4u)
+                                           : 0u;
                             }
                             const uint32_t ch = (uint32_t)(4 * th + j);
                             st_tile4(sm, VT + v0 * 128u + ((ch ^ (v0 & 7u)) << 4), __byte_perm(w[0], w[1], 0x5410),
@@ -1818,6 +1831,7 @@ cudaError_t launch(const StagedArgs& a, cudaStream_t stream) {
     p.total_tokens = a.total_tokens;
     p.H = a.H;
     p.N = a.N;
+    p.flags = a.flags;
     const int64_t units = (int64_t)a.N * a.H;
     const int grid = (int)(units < sm_count ? units : sm_count);
     if (grid <= 0) return cudaSuccess;

@@ -107,6 +107,14 @@ typedef struct {
  * affected fp16 operands (never inf or NaN), records KDA_DEVERR_RANGE in the device error word
  * and the output is then not guaranteed; kda_fwd_staged computes such inputs in fp32.
  *
+ * One long sequence with few heads (fixed layout, batch 1, when kda_fwd_segments() > 1): the fused
+ * kernel runs one CTA per (sequence, head), so such a call would leave most SMs idle.  kda_fwd then
+ * splits the sequence into R chunk-aligned segments and runs them together: every segment's affine
+ * state map (from S = I with v = 0, and from S = 0), their fold into each segment's starting state
+ * (S_r = A_{r-1} S_{r-1} + B_{r-1}, kda_state_affine), and every segment from its state.  The result
+ * is the same recurrence (up to rounding); the call allocates 3 R H 64 KiB of workspace
+ * stream-ordered and launches R + 3 kernels.
+ *
  * lower_bound: <= 0 (may be -INFINITY: no clamp); NaN or > 0 is rejected.
  * scale: finite.  Returns KDA_OK or an error code; never aborts.
  */
@@ -117,6 +125,12 @@ kda_status kda_fwd(const void* q, const void* k, const void* v,
                    const float* initial_state, const int32_t* cu_seqlens,
                    void* out, float* final_state,
                    kda_dims dims, kda_stream_t stream);
+
+/* The number of segments kda_fwd and kda_gdn_fwd split a call with these dims into on the current
+ * device (1: none).  Only one sequence in the fixed layout (varlen == 0, batch == 1) of at least
+ * 8192 tokens is split; the count minimises an estimate of three passes over R H units against
+ * one pass over H units. */
+int32_t kda_fwd_segments(kda_dims dims, int32_t varlen);
 
 /* Gates at or above this clamp keep every factored intra-chunk decay of the fused kernel inside
  * the fp32/bf16 exponent range: its factors span at most 8 tokens of decay around the middle of a

@@ -105,3 +105,31 @@ def test_segmented_prefill_long_sequence_full_size():
     assert oracle.rel_l2(o, ref_o) <= OUT_REL_L2
     assert oracle.max_abs(o, ref_o) <= OUT_MAX_ABS
     assert oracle.rel_l2(fin.cpu().numpy(), ref_f) <= STATE_REL_L2
+
+
+@pytest.mark.parametrize("gdn", [False, True], ids=["kda", "scalar_gate"])
+def test_library_splits_one_long_sequence(gdn):
+    """kda_fwd / kda_gdn_fwd on one 16384-token sequence with two heads (2 of 148 SMs busy
+    unsplit) take the segmented decomposition inside the library; the output and the final state
+    (written over the initial state, in place) match the fp64 oracle on the unsplit sequence."""
+    kda, _ = _kda()
+    H, T = 2, 16384
+    R = kda.kda_fwd_segments(H, T)
+    assert R > 1, "the library should split this call"
+    assert kda.kda_fwd_segments(H, T, varlen=True) == 1 and kda.kda_fwd_segments(H, T // 2, batch=2) == 1
+    x = W.make_inputs(W.custom([T], H=H, packed=False, init="normal", wid=77))
+    if gdn:
+        x = W.gdn_inputs(x)
+    xd = to_device(x)
+    fin = xd["initial_state"].clone()
+    fwd = kda.kda_gdn_fwd if gdn else kda.kda_fwd
+    out, fin = fwd(xd["q"], xd["k"], xd["v"], xd["g"], xd["beta"], xd["A_log"], xd["dt_bias"], x["lower_bound"],
+                   x["scale"], fin, None, final_state=fin, batch=1)
+    assert kda.kda_check_device_error() == 0
+    f = oracle.gdn_recurrent if gdn else oracle.recurrent
+    ref_o, ref_f = f(x["q"], x["k"], x["v"], x["g"], x["beta"], x["A_log"], x["dt_bias"], x["lower_bound"],
+                     x["scale"], x["initial_state"], None)
+    o = out.float().cpu().numpy().astype(np.float64)
+    assert oracle.rel_l2(o, ref_o) <= OUT_REL_L2, f"R={R}"
+    assert oracle.max_abs(o, ref_o) <= OUT_MAX_ABS, f"R={R}"
+    assert oracle.rel_l2(fin.cpu().numpy(), ref_f) <= STATE_REL_L2, f"R={R}"
