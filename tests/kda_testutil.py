@@ -50,3 +50,41 @@ def check(out, fin, ref_out, ref_fin, label=""):
         assert np.all(np.isfinite(f)), msg + " (non-finite state)"
         assert e_st <= STATE_REL_L2, msg + f" state rel-L2 {e_st:.3e}"
     return e_rel, e_abs, e_st
+
+
+BWD_NAMES = ("dq", "dk", "dv", "dg", "dbeta", "dA_log", "ddt_bias", "d_initial_state")
+
+
+def head_slice(x: dict, dO, dF, heads):
+    """The inputs and cotangents of the given heads only (the recurrence treats heads independently)."""
+    xs = dict(x)
+    for key in ("q", "k", "v", "g", "beta"):
+        xs[key] = x[key][:, heads].contiguous()
+    xs["A_log"], xs["dt_bias"] = x["A_log"][heads].contiguous(), x["dt_bias"][heads].contiguous()
+    if x["initial_state"] is not None:
+        xs["initial_state"] = x["initial_state"][:, heads].contiguous()
+    return xs, dO[:, heads].contiguous(), None if dF is None else dF[:, heads].contiguous()
+
+
+def backward_oracle(args):
+    """Chunked fp64 backward oracle on one set of heads (one task of a spawn pool)."""
+    from oracle import backward as OB
+    x, dO, dF = args
+    torch.set_num_threads(1)
+    cu = x["cu_seqlens"]
+    if cu is None:   # the fixed layout: batch sequences of seqlen tokens each
+        cu = torch.arange(x["batch"] + 1, dtype=torch.int32) * x["seqlen"]
+    r = OB.grads_chunked(x["q"], x["k"], x["v"], x["g"], x["beta"], x["A_log"], x["dt_bias"], x["lower_bound"],
+                         x["scale"], x["initial_state"], cu, dO, dF)
+    return dict(zip(BWD_NAMES, r))
+
+
+def backward_oracle_all_heads(x: dict, dO, dF, H: int, procs: int = 0):
+    """The backward oracle for every head, one head per task on a spawn pool (spawn: the parent
+    has a CUDA context, which a forked child must not inherit)."""
+    import multiprocessing as mp
+    import os
+    procs = procs or min(H, os.cpu_count() or 1)
+    tasks = [head_slice(x, dO, dF, [h]) for h in range(H)]
+    with mp.get_context("spawn").Pool(procs) as pool:
+        return pool.map(backward_oracle, tasks, chunksize=1)
