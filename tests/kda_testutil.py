@@ -81,10 +81,24 @@ def backward_oracle(args):
 
 def backward_oracle_all_heads(x: dict, dO, dF, H: int, procs: int = 0):
     """The backward oracle for every head, one head per task on a spawn pool (spawn: the parent
-    has a CUDA context, which a forked child must not inherit)."""
+    has a CUDA context, which a forked child must not inherit).  Each worker runs single-threaded
+    (its BLAS and OpenMP pools too): one process per core, not one thread pool per process."""
     import multiprocessing as mp
     import os
-    procs = procs or min(H, os.cpu_count() or 1)
+    procs = procs or min(H, len(os.sched_getaffinity(0)))
     tasks = [head_slice(x, dO, dF, [h]) for h in range(H)]
-    with mp.get_context("spawn").Pool(procs) as pool:
-        return pool.map(backward_oracle, tasks, chunksize=1)
+    # read by the children at start-up: one thread each, and glibc malloc keeps the oracle's
+    # many short-lived arrays on its heap instead of mapping and unmapping pages for each
+    env = {"OMP_NUM_THREADS": "1", "OPENBLAS_NUM_THREADS": "1", "MKL_NUM_THREADS": "1",
+           "MALLOC_MMAP_THRESHOLD_": str(1 << 30), "MALLOC_TRIM_THRESHOLD_": str(1 << 32)}
+    saved = {k: os.environ.get(k) for k in env}
+    os.environ.update(env)
+    try:
+        with mp.get_context("spawn").Pool(procs) as pool:
+            return pool.map(backward_oracle, tasks, chunksize=1)
+    finally:
+        for k, v in saved.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
