@@ -168,8 +168,8 @@ typedef struct {
 
 /* Bytes of workspace kda_fwd_staged needs for `dims`, whichever layout the call uses: the
  * larger of the varlen reading (N = num_seqs, Ttot = seqlen) and the fixed one (N = batch,
- * Ttot = batch * seqlen).  kda_fwd itself takes no workspace (its staged fallback allocates
- * stream-ordered).  0 for invalid dims. */
+ * Ttot = batch * seqlen).  kda_fwd itself takes no workspace (its staged fallback and its
+ * split of one long sequence allocate stream-ordered).  0 for invalid dims. */
 size_t kda_fwd_workspace_size(kda_dims dims);
 
 /* varlen != 0: the call passes cu_seqlens (N = num_seqs, Ttot = seqlen);
