@@ -235,3 +235,13 @@ def test_selftest_rejects_bad_limits():
     assert lib.kda_selftest_wait_timeout(0, None, None) == 1                  # KDA_ERR_INVALID_ARG
     assert lib.kda_selftest_wait_timeout(2_000_000_000, None, None) == 1
     assert lib.kda_selftest_wait_timeout(1000, ctypes.c_void_p(FAKE + 2), None) == 3   # KDA_ERR_ALIGNMENT
+
+
+def test_segment_query_leaves_varlen_batched_and_short_calls_unsplit():
+    """kda_fwd_segments: only one fixed-layout sequence of at least 128 chunks is ever split (on
+    a host without a GPU nothing is); varlen calls, batches and invalid dims get 1."""
+    assert kda.kda_fwd_segments(2, 131072, varlen=True) == 1
+    assert kda.kda_fwd_segments(2, 65536, batch=2) == 1
+    assert kda.kda_fwd_segments(2, 128 * 64 - 1) == 1
+    assert kda.kda_fwd_segments(0, 131072) == 1
+    assert kda.kda_fwd_segments(32, 131072) >= 1
